@@ -1,0 +1,216 @@
+"""numpy front end of the fp64 CPU oracle (``kvq_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: imported by the test suite, the package smoke check
+and the CPU-baseline leg of the benchmark; never by the product path.  It
+shares no code with the CUDA library.
+
+Each function states the passage of "Dual-QK: Sharp Queries and Flat Keys for
+Prunable 2-bit KV Caches" it follows; the C file's header has the full list.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "kvq_oracle.c")
+LIB = os.path.join(HERE, "libkvq_oracle.so")
+D = 128
+T = 128
+GROUP = 32
+
+_lock = threading.Lock()
+_lib = None
+
+CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into a shared library next to its source."""
+    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
+        tmp = LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *CFLAGS, SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, LIB)
+    return LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(LIB)
+            P = ctypes.c_void_p
+            L = ctypes.c_long
+            I = ctypes.c_int
+            lib.orc_f16_rne.restype = ctypes.c_uint16
+            lib.orc_f16_rne.argtypes = [ctypes.c_double]
+            lib.orc_bf16_rne.restype = ctypes.c_uint16
+            lib.orc_bf16_rne.argtypes = [ctypes.c_double]
+            lib.orc_f16_to_f64.restype = ctypes.c_double
+            lib.orc_f16_to_f64.argtypes = [ctypes.c_uint16]
+            lib.orc_bf16_to_f64.restype = ctypes.c_double
+            lib.orc_bf16_to_f64.argtypes = [ctypes.c_uint16]
+            lib.orc_f16_rne_array.argtypes = [P, L, P]
+            lib.orc_bf16_rne_array.argtypes = [P, L, P]
+            lib.orc_transform.argtypes = [P, P, L, I, P]
+            lib.orc_quantize_group.argtypes = [P, I, I, P, P, P]
+            lib.orc_page_bytes.restype = L
+            lib.orc_page_bytes.argtypes = [I]
+            lib.orc_append_unit.argtypes = [P, I, L, L, P, P]
+            lib.orc_dequant_unit.argtypes = [P, I, L, P, P]
+            lib.orc_num_selected.restype = I
+            lib.orc_num_selected.argtypes = [ctypes.c_float, I]
+            lib.orc_select.argtypes = [P, I, I, I, P, P]
+            lib.orc_decode_dense.argtypes = [P, P, L, P, I, I, P, I, P]
+            lib.orc_attention.argtypes = [P, P, P, L, I, I, P]
+            _lib = lib
+    return _lib
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+# ------------------------------------------------------------- conversions
+def f16_rne(x) -> np.ndarray:
+    """binary64 -> binary16 bits, one rounding to nearest even."""
+    x = _f64(x)
+    out = np.empty(x.shape, dtype=np.uint16)
+    _load().orc_f16_rne_array(_p(x), x.size, _p(out))
+    return out
+
+
+def bf16_rne(x) -> np.ndarray:
+    """binary64 -> bfloat16 bits, one rounding to nearest even."""
+    x = _f64(x)
+    out = np.empty(x.shape, dtype=np.uint16)
+    _load().orc_bf16_rne_array(_p(x), x.size, _p(out))
+    return out
+
+
+def f16_value(bits: int) -> float:
+    return _load().orc_f16_to_f64(int(bits))
+
+
+def bf16_value(bits: int) -> float:
+    return _load().orc_bf16_to_f64(int(bits))
+
+
+# --------------------------------------------------------------- transform
+def transform(X, M) -> np.ndarray:
+    """Rows of X times M (Dual-QK §3.1): fixed-order fma chain over channels."""
+    X = _f64(X)
+    M = _f64(M)
+    d = M.shape[0]
+    assert M.shape == (d, d) and X.shape[-1] == d
+    Y = np.empty_like(X)
+    _load().orc_transform(_p(X), _p(M), X.size // d, d, _p(Y))
+    return Y
+
+
+# --------------------------------------------------------------- quantizer
+def quantize_group(x, bits: int = 2):
+    """One (token, group) of the asymmetric min/max quantizer (Dual-QK §3.3).
+
+    Returns (scale fp16 bits, zero fp16 bits, codes uint8[len]).
+    """
+    x = _f64(x)
+    s = np.zeros(1, np.uint16)
+    z = np.zeros(1, np.uint16)
+    c = np.zeros(x.size, np.uint8)
+    _load().orc_quantize_group(_p(x), x.size, (1 << bits) - 1, _p(s), _p(z), _p(c))
+    return int(s[0]), int(z[0]), c
+
+
+def page_bytes(bits: int) -> int:
+    return int(_load().orc_page_bytes(bits))
+
+
+def new_unit(capacity: int, bits: int) -> np.ndarray:
+    """Zeroed pages of one (batch, KV head): uint8 [capacity/128][page bytes]."""
+    assert capacity % T == 0
+    return np.zeros((capacity // T, page_bytes(bits)), dtype=np.uint8)
+
+
+def append_unit(unit: np.ndarray, bits: int, pos0: int, Kp, V) -> None:
+    """Quantize and store tokens pos0.. of one unit (K' already transformed)."""
+    Kp = _f64(Kp).reshape(-1, D)
+    V = _f64(V).reshape(-1, D)
+    assert Kp.shape == V.shape
+    assert unit.flags.c_contiguous and unit.dtype == np.uint8
+    assert (pos0 + Kp.shape[0]) <= unit.shape[0] * T
+    _load().orc_append_unit(_p(unit), bits, pos0, Kp.shape[0], _p(Kp), _p(V))
+
+
+def dequant_unit(unit: np.ndarray, bits: int, n: int):
+    """Dequantized K' and V of tokens 0..n-1: float64 [n][128] each."""
+    Kh = np.zeros((max(n, 0), D))
+    Vh = np.zeros((max(n, 0), D))
+    _load().orc_dequant_unit(_p(np.ascontiguousarray(unit)), bits, n, _p(Kh), _p(Vh))
+    return Kh, Vh
+
+
+# --------------------------------------------------------------- selection
+def num_selected(sparsity: float, d: int = D) -> int:
+    return int(_load().orc_num_selected(float(sparsity), d))
+
+
+def select(qp, k: int):
+    """Channel 0 plus the top k-1 channels by pooled energy (Dual-QK Eq. 4).
+
+    qp: [g][d] transformed queries of one GQA group. Returns (idx int32[k]
+    ascending, e2 float64[d]).
+    """
+    qp = _f64(qp)
+    g, d = qp.shape
+    assert 1 <= k <= d
+    e2 = np.zeros(d)
+    idx = np.zeros(k, np.int32)
+    _load().orc_select(_p(qp), g, d, k, _p(e2), _p(idx))
+    return idx, e2
+
+
+# --------------------------------------------------------------- attention
+def decode_dense(Khat, Vhat, qp, idx) -> np.ndarray:
+    """Softmax attention over retained channels idx, 1/sqrt(d) scaling."""
+    Khat = _f64(Khat)
+    Vhat = _f64(Vhat)
+    qp = _f64(qp)
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    g, d = qp.shape
+    n = Khat.shape[0]
+    out = np.zeros((g, d))
+    _load().orc_decode_dense(_p(Khat), _p(Vhat), n, _p(qp), g, d, _p(idx), idx.size, _p(out))
+    return out
+
+
+def attention(q, K, V) -> np.ndarray:
+    """Plain softmax(q K^T / sqrt(d)) V."""
+    q = _f64(q)
+    K = _f64(K)
+    V = _f64(V)
+    g, d = q.shape
+    out = np.zeros((g, d))
+    _load().orc_attention(_p(q), _p(K), _p(V), K.shape[0], g, d, _p(out))
+    return out
+
+
+# ------------------------------------------------------ whole decode step
+def decode_unit(unit: np.ndarray, bits: int, n: int, qp, sparsity: float):
+    """Select channels for one GQA group and attend over n cached tokens.
+
+    Returns (out [g][d] float64, idx int32[k]).
+    """
+    k = num_selected(sparsity)
+    idx, _ = select(qp, k)
+    Kh, Vh = dequant_unit(unit, bits, n)
+    return decode_dense(Kh, Vh, qp, idx), idx
