@@ -1,0 +1,447 @@
+#!/usr/bin/env python3
+"""Decode-step benchmark: KV tokens scanned per second over a prunable INT2
+KV cache on B200, with achieved HBM bandwidth against the measured peak.
+
+One step = one decode step of the whole hot path: append the new token per
+(sequence, KV head) (transform + quantize + pack), transform the query and
+select channels, channel-skipping split-context attention and the merge.
+Inputs are device resident; L2 is flushed between steps (a 256 MiB write,
+outside the timed events).  `e2e` repeats the loop through the Python
+binding with the step's inputs copied from pinned host memory and the output
+copied back inside the timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun every rank runs the same per-GPU workload (weak scaling, no
+data-path collective); the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from long_context_decode_dual_b200 import workloads as W  # noqa: E402
+
+METRIC = "KV tokens scanned/s per decode step (INT2, 40% pruned); % of HBM peak GB/s"
+UNIT = "KV tokens scanned/s"
+DEFAULT_WORKLOAD = "longctx_b1_128k"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+CSRC = os.path.join(ROOT, "long_context_decode_dual_b200", "csrc")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.txt")
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ---------------------------------------------------------------- helpers
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def decode_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(CSRC)):
+        if name.startswith("kvq_decode") or name.endswith(".cuh"):
+            with open(os.path.join(CSRC, name), "rb") as f:
+                h.update(name.encode())
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(workload: str):
+    """DRAM bytes per decode launch from a committed ncu summary, if it was
+    taken on the current decode kernel source for this workload."""
+    try:
+        kv = {}
+        with open(TRAFFIC_FILE) as f:
+            for line in f:
+                if ":" in line and not line.startswith("#"):
+                    a, b = line.split(":", 1)
+                    kv[a.strip()] = b.strip()
+        if kv.get("kernel_source_sha") != decode_source_hash():
+            return None, "stale"
+        if kv.get("workload") != workload:
+            return None, "other workload"
+        return float(kv["dram_bytes_per_launch"]), kv.get("note", "")
+    except Exception:
+        return None, "absent"
+
+
+def algorithmic_decode_bytes(wl: W.Workload, k: int, length: int) -> int:
+    """Bytes one decode launch must read: per (sequence, KV head) and page, the
+    k-1 selected key rows, the value codes, channel 0 and both metadata
+    blocks; plus the selection inputs and the partial outputs are ignored
+    (they are < 0.1%)."""
+    R = 128 * wl.bits // 8
+    per_page = (k - 1) * R + 128 * R + 256 + 2048 + 2048
+    n_pages = (length + 127) // 128
+    return wl.batch * wl.n_kv_heads * n_pages * per_page
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.proc = None
+        self.uuid = uuid
+
+    def __enter__(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+        if self.uuid:
+            cmd.insert(1, f"--id={self.uuid}")
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        rows = [r.split(", ") for r in (self.out or "").strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip() == "Active"})
+        hi = sorted(sm)[len(sm) // 2:] if sm else []
+        return {"sm_mhz": statistics.median(hi) if hi else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------ oracle (CPU)
+def oracle_sample(wl: W.Workload, n_steps: int, budget_s: float = 30.0, skip_first: int = 1):
+    """Time the fp64 CPU oracle on a bounded sample of the workload: one
+    (sequence 0, KV head 0) unit with the full context, n_steps decode steps
+    (append one token, transform the query and select, attend)."""
+    from oracle import oracle as orc
+    A, Ai = W.make_transform(wl.seed, 0)
+    K, V = W.make_kv_unit(wl, 0, 0)
+    unit = orc.new_unit(wl.capacity, wl.bits)
+    orc.append_unit(unit, wl.bits, 0, orc.transform(W.as_float(K, wl.dtype), A), W.as_float(V, wl.dtype))
+    length = wl.n_ctx
+    g = wl.group_size
+    times, tokens = [], []
+    t_start = time.perf_counter()
+    for i in range(n_steps):
+        kn, vn = W.make_step_kv(wl, i)
+        q = W.make_q(wl, i)
+        t0 = time.perf_counter()
+        orc.append_unit(unit, wl.bits, length, orc.transform(W.as_float(kn[0, 0], wl.dtype), A),
+                        W.as_float(vn[0, 0], wl.dtype))
+        length += 1
+        qp = orc.transform(W.as_float(q[0, :g], wl.dtype), Ai)
+        orc.decode_unit(unit, wl.bits, length, qp, wl.sparsity)
+        times.append(time.perf_counter() - t0)
+        tokens.append(length)
+        if time.perf_counter() - t_start > budget_s and i >= 1:
+            break
+    skip = min(skip_first, len(times) - 1)
+    value = sum(tokens[skip:]) / sum(times[skip:])
+    sample = (f"1 of {wl.batch * wl.n_kv_heads} (sequence, KV head) units, full {wl.n_ctx}-token "
+              f"context, {len(times) - skip} timed decode steps (append+select+attend), fp64, "
+              f"single thread")
+    return value, times[skip:], sample
+
+
+# ------------------------------------------------------------ reference arm
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = W.workload(args.workload, **({"sparsity": args.sparsity} if args.sparsity is not None else {}),
+                    bits=args.bits, n_steps=args.warmup + args.steps + 1)
+    from oracle import oracle as orc
+    k = orc.num_selected(wl.sparsity)
+    value, times, sample = oracle_sample(wl, args.warmup + args.steps, budget_s=1e9,
+                                         skip_first=args.warmup)
+    tokens_per_s = value
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tokens_per_s, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.mean(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(wl, k),
+        "cpu_baseline": {"value": tokens_per_s, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": tokens_per_s, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(wl: W.Workload, k: int):
+    return {"workload": wl.name, "batch": wl.batch, "n_q_heads": wl.n_q_heads,
+            "n_kv_heads": wl.n_kv_heads, "context": wl.n_ctx, "head_dim": 128, "bits": wl.bits,
+            "group": 32, "sparsity": wl.sparsity, "k": k,
+            "step": "append 1 token + query transform/select + decode + merge",
+            "l2": "flushed between steps (256 MiB write, outside the timed events)"}
+
+
+# ------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from long_context_decode_dual_b200 import kvq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    kvq.lib()
+
+    n_pool = 8
+    total_steps = args.warmup + args.steps
+    n_appends = total_steps * (2 if args.e2e else 1) + 1
+    over = {"bits": args.bits, "n_steps": n_appends}
+    if args.sparsity is not None:
+        over["sparsity"] = args.sparsity
+    wl = W.workload(args.workload, **over)
+    B, Hq, Hkv = wl.batch, wl.n_q_heads, wl.n_kv_heads
+
+    t0 = time.perf_counter()
+    A_np, Ai_np = W.make_transforms(wl)
+    K_np, V_np = W.make_kv(wl)
+    log(f"[bench] inputs generated in {time.perf_counter() - t0:.1f}s")
+
+    def dev_in(x):
+        if wl.dtype == "f32":
+            return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    A = torch.from_numpy(A_np).to(dev)
+    Ai = torch.from_numpy(Ai_np).to(dev)
+    Kd, Vd = dev_in(K_np), dev_in(V_np)
+    stream = torch.cuda.current_stream(dev)
+
+    cache = kvq.new_cache(B, Hkv, wl.capacity, wl.bits, device=dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    kvq.append(cache, Kd, Vd, A)
+    ev1.record()
+    torch.cuda.synchronize(dev)
+    prefill_ms = ev0.elapsed_time(ev1)
+    assert kvq.read_status(cache) == 0
+
+    q_pool = [dev_in(W.make_q(wl, i)) for i in range(n_pool)]
+    kv_pool = [tuple(dev_in(t) for t in W.make_step_kv(wl, i)) for i in range(n_pool)]
+    k = kvq.num_selected(wl.sparsity)
+    sel = kvq.alloc_selection(cache, Hq, k, dev)
+    out = torch.empty(B, Hq, 128, dtype=torch.float32, device=dev)
+    ws = kvq.alloc_workspace(kvq.decode_workspace_bytes(cache, Hq, k), dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(i, q, kn, vn, d0=None, d1=None):
+        kvq.append(cache, kn, vn, A)
+        kvq.select_channels(cache, q, Ai, wl.sparsity, out=sel)
+        if d0 is not None:
+            d0.record()
+        kvq.decode_attn(cache, sel, out=out, ws=ws)
+        if d1 is not None:
+            d1.record()
+
+    launches_per_step = 5   # append + length advance, select, decode partial, merge
+    length = wl.n_ctx
+    for i in range(args.warmup):
+        step(i, q_pool[i % n_pool], *kv_pool[i % n_pool])
+        length += 1
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    evs = [(E(), E(), E(), E()) for _ in range(args.steps)]
+    tokens = []
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    torch.cuda.synchronize(dev)
+    with ClockSampler(uuid) as clocks:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            a, b_, d0, d1 = evs[i]
+            a.record()
+            j = args.warmup + i
+            step(j, q_pool[j % n_pool], *kv_pool[j % n_pool], d0, d1)
+            b_.record()
+            length += 1
+            tokens.append(B * Hkv * length)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    step_ms = [a.elapsed_time(b_) for a, b_, _, _ in evs]
+    dec_ms = [d0.elapsed_time(d1) for _, _, d0, d1 in evs]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    value = world * sum(tokens) / (total_ms * 1e-3)
+    assert kvq.read_status(cache) == 0
+
+    # roofline of the dominant kernel (decode partial + merge, timed together)
+    hbm_peak, peak_src = measured_peaks()
+    alg_bytes = [algorithmic_decode_bytes(wl, k, tok // (B * Hkv)) for tok in tokens]
+    achieved = statistics.mean(ab / (ms * 1e-3) for ab, ms in zip(alg_bytes, dec_ms)) / 1e9
+    traffic, traffic_note = committed_traffic(wl.name)
+
+    # end to end through the Python binding with host buffers
+    e2e = None
+    if args.e2e:
+        pin = lambda x: torch.from_numpy(np.ascontiguousarray(x).view(  # noqa: E731
+            np.int16 if wl.dtype == "bf16" else np.float32)).pin_memory()
+        qh = [pin(W.make_q(wl, i)) for i in range(n_pool)]
+        kvh = [tuple(pin(t) for t in W.make_step_kv(wl, i)) for i in range(n_pool)]
+        q_dev = torch.empty_like(q_pool[0])
+        kn_dev, vn_dev = torch.empty_like(kv_pool[0][0]), torch.empty_like(kv_pool[0][1])
+        out_h = torch.empty(B, Hq, 128, dtype=torch.float32).pin_memory()
+        as_dev = (lambda t: t.view(torch.bfloat16)) if wl.dtype == "bf16" else (lambda t: t)
+        e_evs = [(E(), E()) for _ in range(args.steps)]
+        e_tok = []
+        torch.cuda.synchronize(dev)
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            a, b_ = e_evs[i]
+            a.record()
+            j = i % n_pool
+            q_dev.view(torch.int16 if wl.dtype == "bf16" else torch.float32).copy_(qh[j], non_blocking=True)
+            kn_dev.view(torch.int16 if wl.dtype == "bf16" else torch.float32).copy_(kvh[j][0], non_blocking=True)
+            vn_dev.view(torch.int16 if wl.dtype == "bf16" else torch.float32).copy_(kvh[j][1], non_blocking=True)
+            step(i, as_dev(q_dev), as_dev(kn_dev), as_dev(vn_dev))
+            out_h.copy_(out, non_blocking=True)
+            b_.record()
+            length += 1
+            e_tok.append(B * Hkv * length)
+        torch.cuda.synchronize(dev)
+        e_ms = sum(a.elapsed_time(b_) for a, b_ in e_evs)
+        if world > 1:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        elem = 2 if wl.dtype == "bf16" else 4
+        h2d = (B * Hq * 128 + 2 * B * Hkv * 128) * elem
+        e2e = {"value": world * sum(e_tok) / (e_ms * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": B * Hq * 128 * 4}
+
+    # the unpruned BF16 comparator on the same keys and values
+    comparator = None
+    if args.comparator and wl.dtype == "bf16":
+        n_tok = wl.n_ctx
+        qc = q_pool[0]
+        cws = kvq.alloc_workspace(kvq.bf16_workspace_bytes(B, Hq, Hkv, n_tok), dev)
+        cout = torch.empty(B, Hq, 128, dtype=torch.float32, device=dev)
+        for _ in range(3):
+            kvq.bf16_decode_attn(qc, Kd, Vd, out=cout, ws=cws)
+        c_ms = []
+        for i in range(max(5, min(args.steps, 20))):
+            flush.fill_(i & 0xFF)
+            a, b_ = E(), E()
+            a.record()
+            kvq.bf16_decode_attn(qc, Kd, Vd, out=cout, ws=cws)
+            b_.record()
+            torch.cuda.synchronize(dev)
+            c_ms.append(a.elapsed_time(b_))
+        cb = B * Hkv * n_tok * 512
+        cm = statistics.mean(c_ms)
+        comparator = {"kernel": "bf16 unpruned decode attention", "ms": cm,
+                      "tokens_per_s": B * Hkv * n_tok / (cm * 1e-3),
+                      "achieved_gbs": cb / (cm * 1e-3) / 1e9, "frac_of_peak": cb / (cm * 1e-3) / 1e9 / hbm_peak,
+                      "speedup_of_int2_decode": cm / statistics.mean(dec_ms)}
+
+    # CPU baseline: the oracle on a bounded sample (rank 0, one GPU only)
+    cpu = None
+    if args.cpu_baseline and world == 1:
+        cv, ct, sample = oracle_sample(wl.with_(n_steps=8), 6, budget_s=25.0)
+        cpu = {"value": cv, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample}
+
+    csum = clocks.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": config_dict(wl, k),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": traffic,
+                     "kernel": "decode partial + merge (kvq_decode_attn)",
+                     "peak_source": f"{peak_src} hbm_gbs", "traffic_note": traffic_note},
+        "decode_ms": statistics.mean(dec_ms),
+        "decode_alg_bytes": statistics.mean(alg_bytes),
+        "prefill_ms": prefill_ms,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": csum,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "comparator": comparator,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(W.WORKLOADS))
+    ap.add_argument("--sparsity", type=float, default=None)
+    ap.add_argument("--bits", type=int, default=2, choices=[2, 4])
+    ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--no-comparator", dest="comparator", action="store_false")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,215 @@
+/*
+ * kvq.h -- C ABI of a B200 (sm_100a) library for decode-step attention over a
+ * prunable 2-bit KV cache, following "Dual-QK: Sharp Queries and Flat Keys for
+ * Prunable 2-bit KV Caches" (§3.1 dual transforms, §3.2 dynamic query-channel
+ * pruning, §3.3 INT2 KV quantization and channel-major page layout, §3.4 one
+ * global softmax across the cache).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor arguments are DEVICE pointers to caller-owned memory.  The
+ *    library allocates nothing and keeps no global state; it is safe to call
+ *    from several host threads on different caches or streams.
+ *  - Every call is asynchronous on the given stream (NULL = legacy default
+ *    stream).  A return of KVQ_OK means the work was validated and enqueued;
+ *    results are ready when the stream reaches that point.
+ *  - Argument errors are found on the host before anything is launched and
+ *    reported as a negative status; nothing is enqueued then.  Conditions
+ *    only the device can see (a sequence that would overflow its capacity)
+ *    set a sticky flag in the cache's device status word and leave the data
+ *    untouched; read it with kvq_read_status().
+ *  - Head dimension d = 128 and quantization group = 32 channels are the
+ *    supported shape; other values return KVQ_ERR_SHAPE.
+ *  - Tensors are dense, row-major, innermost dimension last, with the
+ *    shapes given per argument.  Float inputs are either float32 or bf16
+ *    (bit patterns in uint16), chosen by a KVQ_DTYPE_* argument.
+ *
+ * Cache format (one "page" = 128 tokens of one (sequence, KV head))
+ * ------------------------------------------------------------------
+ *  rowbytes R = 128 * bits / 8   (32 for INT2, 64 for INT4)
+ *  offset 0        key codes, 128 rows x R bytes, row r = transformed key
+ *                  channel r; row 0 is unused and stays zero
+ *  offset 128R     value codes, 128 rows x R bytes, row r = value channel r
+ *  offset 256R     channel 0 of the transformed key, 128 x bf16
+ *  offset 256R+256 key metadata [4 groups][128 tokens] x {fp16 scale, fp16 zero}
+ *  +2048           value metadata, same shape
+ *  page bytes = 256R + 4352 (12544 for INT2, 20736 for INT4)
+ *  Code of token t (0..127) of a page: byte t*bits/8 of its row, bit
+ *  (t mod (8/bits))*bits, least significant first.  Key groups are channels
+ *  {1..31}, {32..63}, {64..95}, {96..127} (channel 0 is kept in bf16 and left
+ *  out of the range); value groups are {0..31} ... {96..127}.
+ *  Pages of one (sequence b, KV head h) are contiguous; unit (b, h) starts at
+ *  byte ((b * n_kv_heads + h) * (capacity / 128)) * page_bytes.
+ *  Dequantized value = scale * code + zero.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *kvq_stream_t;   /* same type as cudaStream_t */
+
+/* return codes */
+enum {
+    KVQ_OK = 0,
+    KVQ_ERR_ARG = -1,        /* null pointer, negative count, unknown dtype    */
+    KVQ_ERR_SHAPE = -2,      /* unsupported head_dim / group / bits / GQA ratio */
+    KVQ_ERR_CAPACITY = -3,   /* request can never fit the cache's capacity      */
+    KVQ_ERR_WORKSPACE = -4,  /* workspace pointer null or too small             */
+    KVQ_ERR_CUDA = -5,       /* a CUDA runtime call or kernel launch failed     */
+    KVQ_ERR_ALIGN = -6       /* a pointer is not aligned as documented          */
+};
+
+/* input element types */
+enum { KVQ_DTYPE_F32 = 0, KVQ_DTYPE_BF16 = 1 };
+
+/* device status flags (sticky; cleared by kvq_cache_init) */
+enum { KVQ_DEV_CAPACITY = 1u };
+
+/* Cache descriptor.  The struct itself is host memory; the pointers in it are
+ * device memory owned by the caller. */
+typedef struct {
+    int32_t batch;        /* sequences B >= 1                                */
+    int32_t n_kv_heads;   /* KV heads per sequence >= 1                      */
+    int32_t head_dim;     /* must be 128                                     */
+    int32_t group;        /* quantization group in channels, must be 32      */
+    int32_t bits;         /* code width: 2 (INT2) or 4 (INT4)                */
+    int32_t capacity;     /* tokens per sequence, a positive multiple of 128 */
+    void *pages;          /* kvq_cache_bytes() bytes, 256-byte aligned        */
+    int32_t *seq_len;     /* [batch] tokens currently stored per sequence    */
+    uint32_t *status;     /* one word of KVQ_DEV_* flags                     */
+} kvq_cache;
+
+/* Bytes of one 128-token page for the given code width (0 if unsupported). */
+size_t kvq_page_bytes(int bits);
+
+/* Bytes of the whole page array of a cache (0 if the descriptor is invalid). */
+size_t kvq_cache_bytes(const kvq_cache *cache);
+
+/* Zero every page, every seq_len entry and the status word (stream-ordered).
+ * Returns KVQ_ERR_ARG / KVQ_ERR_SHAPE / KVQ_ERR_ALIGN on a bad descriptor. */
+int kvq_cache_init(const kvq_cache *cache, kvq_stream_t stream);
+
+/*
+ * kvq_append -- quantize n_new tokens per (sequence, KV head) into the cache
+ * at positions seq_len[b] .. seq_len[b]+n_new-1, then advance seq_len[b].
+ * Dual-QK §3.1 (keys multiplied by the fixed transform, K' = K A), §3.3
+ * (channel 0 of K' kept as bf16 and excluded from the range; the other key
+ * channels and all value channels quantized per token with an asymmetric
+ * min/max grid, round to nearest; channel-major 128-token pages).
+ *
+ *  K, V    [batch][n_kv_heads][n_new][128], dtype KVQ_DTYPE_F32 or _BF16
+ *  A       [n_kv_heads][128][128] float64, row-major: K'[j] = sum_c K[c] A[c][j]
+ *          summed c = 0..127 as a chain of fused multiply-adds from 0.0
+ *  Arithmetic (defines the stored bits): K' in float64; per token and group
+ *  zero = fp16(min), scale = fp16((max-min)/(2^bits-1)) (fp16 rounding to
+ *  nearest even from float64), code = clamp(rint((x - zero)/scale), 0,
+ *  2^bits-1) in float64, or 0 when scale == 0; channel 0 -> bf16 (nearest
+ *  even from float64).  Bits of other tokens sharing a code byte are kept.
+ *  Values must stay within the fp16 range after the transform.
+ *  A sequence whose seq_len + n_new would exceed capacity is left untouched
+ *  and sets KVQ_DEV_CAPACITY.  n_new == 0 is a no-op.
+ *  Errors: KVQ_ERR_ARG (null pointer, n_new < 0, bad dtype), KVQ_ERR_SHAPE,
+ *  KVQ_ERR_CAPACITY (n_new > capacity), KVQ_ERR_CUDA.
+ */
+int kvq_append(const kvq_cache *cache, const void *K, const void *V, int dtype,
+               int n_new, const double *A, kvq_stream_t stream);
+
+/* k = ceil((1 - sparsity) * head_dim) (with a 1e-9 guard), the number of key
+ * channels kept per KV head, channel 0 included.  Returns -1 if sparsity is
+ * outside [0, 1) or head_dim < 1.  Dual-QK §4.1 (x% query-channel sparsity). */
+int kvq_num_selected(float sparsity, int head_dim);
+
+/*
+ * kvq_select_channels -- transform the decode query and choose the key
+ * channels to read.  Dual-QK §3.1 (queries multiplied by the paired inverse
+ * transpose, q' = q A^{-T}, so q'.K' = q.K), §3.2 Eq. 4 (energy pooled over
+ * the g = n_q_heads / n_kv_heads query heads of a KV head, e_j^2 =
+ * sum_h q'_{h,j}^2; one mask per KV head); channel 0 is always kept.
+ *
+ *  q       [batch][n_q_heads][128], dtype F32 or BF16; query head h belongs
+ *          to KV head h / g
+ *  Ainvt   [n_kv_heads][128][128] float64, q'[j] = sum_c q[c] Ainvt[c][j]
+ *          (fma chain over c from 0.0), e^2 by an fma chain over h ascending
+ *  idx     out [batch][n_kv_heads][k] int32: channel 0 and the k-1 channels of
+ *          1..127 with the largest e^2 (ties to the lower index), ascending
+ *  qsel    out [batch][n_q_heads][k] float32: q'[h][idx[i]] rounded to fp32
+ *  qgsum   out [batch][n_q_heads][4] float32: per key group, the float64 sum
+ *          of q'[h][c] over selected c != 0 of that group (ascending c),
+ *          rounded to fp32 (the zero-point term of the dequantized dot)
+ *  k_out   out (HOST int*, may be NULL): k
+ *  Errors: KVQ_ERR_ARG (null, sparsity outside [0,1)), KVQ_ERR_SHAPE
+ *  (n_q_heads not a multiple of n_kv_heads, or g > 32), KVQ_ERR_CUDA.
+ */
+int kvq_select_channels(const kvq_cache *cache, const void *q, int dtype,
+                        int n_q_heads, const double *Ainvt, float sparsity,
+                        int32_t *idx, float *qsel, float *qgsum, int *k_out,
+                        kvq_stream_t stream);
+
+/* Workspace bytes kvq_decode_attn needs for this cache on the CURRENT device
+ * (it sizes the split over the context by the device's SM count).
+ * 0 if the arguments are invalid. */
+size_t kvq_decode_workspace(const kvq_cache *cache, int n_q_heads, int k);
+
+/*
+ * kvq_decode_attn -- attention of one decode query per head over every
+ * cached token, reading only the selected key channels.  Dual-QK §3.2 (scores
+ * use the retained channels, scaled by 1/sqrt(128) with the full dimension),
+ * §3.3 (only the selected 32-byte key rows of each page are fetched; values
+ * and metadata are read in full), §3.4 (one softmax over all tokens, then
+ * value aggregation).  Realised as a split over the context (flash-decoding):
+ * per split a running max, sum and output, then one exact merge.
+ *
+ *  score_h(t) = [qsel_h0 * ch0(t) + sum_g (scale_g(t) * sum_{c in S_g}
+ *               qsel_hc * code_c(t) + zero_g(t) * qgsum_hg)] / sqrt(128)
+ *  out     [batch][n_q_heads][128] float32 = sum_t p_h(t) v_hat(t) / sum_t p_h(t)
+ *          (zeros for a sequence with no tokens)
+ *  idx, qsel, qgsum, k exactly as produced by kvq_select_channels
+ *  ws      device workspace of at least kvq_decode_workspace() bytes,
+ *          16-byte aligned; contents need no initialisation
+ *  Arithmetic: float32 (tensor-core products of exact small integers and
+ *  split float16 operands, float32 accumulation).
+ *  Errors: KVQ_ERR_ARG, KVQ_ERR_SHAPE, KVQ_ERR_WORKSPACE, KVQ_ERR_ALIGN,
+ *  KVQ_ERR_CUDA.
+ */
+int kvq_decode_attn(const kvq_cache *cache, int n_q_heads, const int32_t *idx,
+                    const float *qsel, const float *qgsum, int k, float *out,
+                    void *ws, size_t ws_bytes, kvq_stream_t stream);
+
+/* Workspace bytes for kvq_bf16_decode_attn on the current device. */
+size_t kvq_bf16_decode_workspace(int batch, int n_q_heads, int n_kv_heads, int n_tokens);
+
+/*
+ * kvq_bf16_decode_attn -- the unpruned, unquantized comparator: plain
+ * softmax(q K^T / sqrt(128)) V per query head over n_tokens bf16 keys and
+ * values (what Dual-QK compares against as "unpruned BF16", §4.4).
+ *  q       [batch][n_q_heads][128] bf16
+ *  K, V    [batch][n_kv_heads][n_tokens][128] bf16 (original coordinates),
+ *          16-byte aligned; may be NULL when n_tokens == 0
+ *  out     [batch][n_q_heads][128] float32
+ *  ws      at least kvq_bf16_decode_workspace() bytes, 16-byte aligned
+ * Arithmetic in float32.  Errors as for kvq_decode_attn.
+ */
+int kvq_bf16_decode_attn(const void *q, const void *K, const void *V, int batch,
+                         int n_q_heads, int n_kv_heads, int n_tokens, float *out,
+                         void *ws, size_t ws_bytes, kvq_stream_t stream);
+
+/* Copy the device status word into *flags (synchronises the stream).
+ * KVQ_ERR_ARG on null pointers, KVQ_ERR_CUDA on a failed copy. */
+int kvq_read_status(const kvq_cache *cache, uint32_t *flags, kvq_stream_t stream);
+
+/* Static description of a status code. */
+const char *kvq_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int kvq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KVQ_H */

@@ -1,0 +1,200 @@
+// kvq_append: key transform, channel-0 protection, group min/max quantization
+// and channel-major packing into 128-token pages.
+//
+// "Dual-QK: Sharp Queries and Flat Keys for Prunable 2-bit KV Caches":
+//   §3.1 keys are multiplied by the fixed key transform (K' = K A);
+//   §3.3 key channel 0 is kept in BF16 and excluded from the quantization
+//        range; the remaining channels (and the values) use an asymmetric
+//        min/max grid per token; within each 128-token page the codes are
+//        stored channel-major, one channel of one page per 32-byte row.
+//
+// One CTA = one (sequence, KV head) and a tile of kTile destination positions
+// aligned to kTile, so the code bytes a CTA writes belong to it alone; thread
+// j owns channel j and warp w owns quantization group w.  The arithmetic is
+// float64 with a fixed order (fma chain over the input channel), which makes
+// the stored bytes reproducible bit for bit.
+#include "kvq_internal.cuh"
+
+namespace kvq {
+namespace {
+
+constexpr int kTile = 16;   // destination positions per CTA (multiple of 8)
+
+__device__ __forceinline__ double warp_min(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmin(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ double warp_max(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// Quantize value x of this lane against the group range (lanes of the warp;
+// `in_range` false leaves the lane out of min/max).  Returns the code and,
+// through s_bits / z_bits, the fp16 scale / zero-point bit patterns.
+template <int BITS>
+__device__ __forceinline__ uint32_t quantize_lane(double x, bool in_range, uint16_t &s_bits,
+                                                  uint16_t &z_bits) {
+    constexpr int L = (1 << BITS) - 1;
+    const double lo = warp_min(in_range ? x : __longlong_as_double(0x7ff0000000000000LL));
+    const double hi = warp_max(in_range ? x : __longlong_as_double(0xfff0000000000000LL));
+    const __half zh = __double2half(lo);
+    const __half sh = __double2half((hi - lo) / (double)L);
+    z_bits = __half_as_ushort(zh);
+    s_bits = __half_as_ushort(sh);
+    const double z = (double)__half2float(zh);
+    const double s = (double)__half2float(sh);
+    if (s == 0.0) return 0u;
+    double r = rint((x - z) / s);
+    r = fmin(fmax(r, 0.0), (double)L);
+    return (uint32_t)r;
+}
+
+// Merge the kTile codes of one channel row into its packed bytes.
+// `valid` has bit tt set for tile positions this call writes.
+template <int BITS>
+__device__ __forceinline__ void store_row(uint8_t *row_tile, const uint32_t (&codes)[kTile],
+                                          uint32_t valid) {
+    if constexpr (BITS == 2) {
+        uint32_t word = 0, mask = 0;
+#pragma unroll
+        for (int tt = 0; tt < kTile; tt++) {
+            word |= codes[tt] << (2 * tt);
+            if (valid >> tt & 1u) mask |= 3u << (2 * tt);
+        }
+        uint32_t *p = reinterpret_cast<uint32_t *>(row_tile);
+        *p = (*p & ~mask) | (word & mask);
+    } else {
+        unsigned long long word = 0, mask = 0;
+#pragma unroll
+        for (int tt = 0; tt < kTile; tt++) {
+            word |= (unsigned long long)codes[tt] << (4 * tt);
+            if (valid >> tt & 1u) mask |= 15ull << (4 * tt);
+        }
+        unsigned long long *p = reinterpret_cast<unsigned long long *>(row_tile);
+        *p = (*p & ~mask) | (word & mask);
+    }
+}
+
+template <typename Tin, int BITS>
+__global__ void __launch_bounds__(128)
+append_kernel(uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len,
+              uint32_t *__restrict__ status, const Tin *__restrict__ K,
+              const Tin *__restrict__ V, const double *__restrict__ A, int Hkv, int NB,
+              int n_new, int capacity) {
+    constexpr int R = row_bytes(BITS);
+    __shared__ double ks[kTile][kD];
+    __shared__ double vs[kTile][kD];
+
+    const int b = blockIdx.z, h = blockIdx.y;
+    const int len = seq_len[b];
+    if (len < 0 || len + n_new > capacity) {
+        if (threadIdx.x == 0) atomicOr(status, (uint32_t)KVQ_DEV_CAPACITY);
+        return;
+    }
+    const int first = (len / kTile) * kTile + blockIdx.x * kTile;
+    const int lo = max(first, len), hi = min(first + kTile, len + n_new);
+    if (lo >= hi) return;
+
+    // stage the inputs of the tile as float64 (zeros outside [lo, hi))
+    const size_t in_base = ((size_t)b * Hkv + h) * (size_t)n_new;
+    for (int e = threadIdx.x; e < kTile * kD; e += blockDim.x) {
+        const int tt = e / kD, c = e % kD, pos = first + tt;
+        double kv = 0.0, vv = 0.0;
+        if (pos >= lo && pos < hi) {
+            const size_t src = (in_base + (size_t)(pos - len)) * kD + c;
+            kv = in_to_double(K[src]);
+            vv = in_to_double(V[src]);
+        }
+        ks[tt][c] = kv;
+        vs[tt][c] = vv;
+    }
+    __syncthreads();
+
+    const int j = threadIdx.x;          // channel
+    const int lane = j & 31;
+    const int grp = j >> 5;             // quantization group (= warp)
+
+    // K'[t][j] = sum_c K[t][c] A[c][j], fma chain c = 0..127 from 0.0
+    double acc[kTile];
+#pragma unroll
+    for (int tt = 0; tt < kTile; tt++) acc[tt] = 0.0;
+    const double *Ah = A + (size_t)h * kD * kD + j;
+#pragma unroll 4
+    for (int c = 0; c < kD; c++) {
+        const double a = __ldg(Ah + (size_t)c * kD);
+#pragma unroll
+        for (int tt = 0; tt < kTile; tt++) acc[tt] = fma(ks[tt][c], a, acc[tt]);
+    }
+
+    uint8_t *page = pages + (((size_t)b * Hkv + h) * NB + (size_t)(first / kT)) * page_bytes(BITS);
+    const int t0 = first % kT;
+    uint32_t valid = 0;
+#pragma unroll
+    for (int tt = 0; tt < kTile; tt++)
+        if (first + tt >= lo && first + tt < hi) valid |= 1u << tt;
+
+    uint16_t *ch0 = reinterpret_cast<uint16_t *>(page + off_ch0(BITS));
+    uint32_t *kmeta = reinterpret_cast<uint32_t *>(page + off_kmeta(BITS));
+    uint32_t *vmeta = reinterpret_cast<uint32_t *>(page + off_vmeta(BITS));
+
+    // keys: channel 0 -> bf16; group 0 covers channels 1..31
+    uint32_t codes[kTile];
+#pragma unroll
+    for (int tt = 0; tt < kTile; tt++) {
+        uint16_t sb, zb;
+        codes[tt] = quantize_lane<BITS>(acc[tt], j != 0, sb, zb);
+        if (valid >> tt & 1u) {
+            if (lane == 0) kmeta[grp * kT + t0 + tt] = (uint32_t)sb | ((uint32_t)zb << 16);
+            if (j == 0) ch0[t0 + tt] = __bfloat16_as_ushort(__double2bfloat16(acc[tt]));
+        }
+    }
+    if (j != 0) store_row<BITS>(page + (size_t)j * R + t0 * BITS / 8, codes, valid);
+
+    // values: no transform, group g covers channels 32g..32g+31
+#pragma unroll
+    for (int tt = 0; tt < kTile; tt++) {
+        uint16_t sb, zb;
+        codes[tt] = quantize_lane<BITS>(vs[tt][j], true, sb, zb);
+        if ((valid >> tt & 1u) && lane == 0)
+            vmeta[grp * kT + t0 + tt] = (uint32_t)sb | ((uint32_t)zb << 16);
+    }
+    store_row<BITS>(page + off_vcodes(BITS) + (size_t)j * R + t0 * BITS / 8, codes, valid);
+}
+
+__global__ void advance_kernel(int32_t *seq_len, int B, int n_new, int capacity) {
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b < B) {
+        const int len = seq_len[b];
+        if (len >= 0 && len + n_new <= capacity) seq_len[b] = len + n_new;
+    }
+}
+
+template <typename Tin, int BITS>
+cudaError_t launch_append_t(const kvq_cache &c, const void *K, const void *V, int n_new,
+                            const double *A, cudaStream_t st) {
+    const int NB = c.capacity / kT;
+    dim3 grid((unsigned)((n_new + kTile - 1) / kTile + 1), (unsigned)c.n_kv_heads, (unsigned)c.batch);
+    append_kernel<Tin, BITS><<<grid, 128, 0, st>>>(
+        static_cast<uint8_t *>(c.pages), c.seq_len, c.status, static_cast<const Tin *>(K),
+        static_cast<const Tin *>(V), A, c.n_kv_heads, NB, n_new, c.capacity);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    advance_kernel<<<(c.batch + 127) / 128, 128, 0, st>>>(c.seq_len, c.batch, n_new, c.capacity);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_append(const kvq_cache &c, const void *K, const void *V, int dtype, int n_new,
+                          const double *A, cudaStream_t st) {
+    if (dtype == KVQ_DTYPE_F32)
+        return c.bits == 2 ? launch_append_t<float, 2>(c, K, V, n_new, A, st)
+                           : launch_append_t<float, 4>(c, K, V, n_new, A, st);
+    return c.bits == 2 ? launch_append_t<uint16_t, 2>(c, K, V, n_new, A, st)
+                       : launch_append_t<uint16_t, 4>(c, K, V, n_new, A, st);
+}
+
+}  // namespace kvq

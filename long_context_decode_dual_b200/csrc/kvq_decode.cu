@@ -1,0 +1,39 @@
+// Decode planning (split of the context over CTAs), workspace layout and the
+// choice of partial kernel; the merge is combine_kernel.
+#include "kvq_internal.cuh"
+
+namespace kvq {
+
+cudaError_t launch_decode_simt(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
+                               const float *qgsum, int k, float *part_o, float2 *part_ml, int S,
+                               cudaStream_t st);
+cudaError_t launch_combine(int rows, const float *part_o, const float2 *part_ml, int S, float *out,
+                           cudaStream_t st);
+
+// Splits per (sequence, KV head): enough CTAs for about four per SM, at
+// least two pages per split, at most one split per page of capacity.
+int decode_splits(const kvq_cache &c, int Hq, int k, int num_sms) {
+    (void)Hq;
+    (void)k;
+    const int units = c.batch * c.n_kv_heads;
+    const int nblk = c.capacity / kT;
+    int S = (4 * num_sms + units - 1) / units;
+    const int max_s = (nblk + 1) / 2 > 0 ? (nblk + 1) / 2 : 1;
+    if (S > max_s) S = max_s;
+    return S < 1 ? 1 : S;
+}
+
+size_t decode_ws_bytes(const kvq_cache &c, int Hq, int S) {
+    return (size_t)c.batch * Hq * S * (kD * sizeof(float) + sizeof(float2));
+}
+
+cudaError_t launch_decode(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
+                          const float *qgsum, int k, float *out, void *ws, int S, cudaStream_t st) {
+    float *part_o = static_cast<float *>(ws);
+    float2 *part_ml = reinterpret_cast<float2 *>(part_o + (size_t)c.batch * Hq * S * kD);
+    cudaError_t e = launch_decode_simt(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, st);
+    if (e != cudaSuccess) return e;
+    return launch_combine(c.batch * Hq, part_o, part_ml, S, out, st);
+}
+
+}  // namespace kvq

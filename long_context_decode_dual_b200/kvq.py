@@ -1,0 +1,253 @@
+"""Python binding of the kvq C ABI (include/kvq.h).
+
+Argument marshalling only: every step of the decode path runs in the CUDA
+kernels of ``libkvq.so``.  PyTorch supplies device memory and streams.  There
+is no fallback: if the library is missing, importing it raises.
+
+Names follow the C entry points:
+  kvq_append           -> append(cache, K, V, A)
+  kvq_select_channels  -> select_channels(cache, q, Ainvt, sparsity)
+  kvq_decode_attn      -> decode_attn(cache, sel)
+  kvq_bf16_decode_attn -> bf16_decode_attn(q, K, V)
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkvq.so")
+
+KVQ_OK = 0
+KVQ_DTYPE_F32 = 0
+KVQ_DTYPE_BF16 = 1
+KVQ_DEV_CAPACITY = 1
+HEAD_DIM = 128
+GROUP = 32
+BLOCK_TOKENS = 128
+
+
+class KvqError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn}: {status_string(status)} ({status})")
+        self.status = status
+
+
+class CacheDesc(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+        ("group", ctypes.c_int32), ("bits", ctypes.c_int32), ("capacity", ctypes.c_int32),
+        ("pages", ctypes.c_void_p), ("seq_len", ctypes.c_void_p), ("status", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+EXPORTS = (
+    "kvq_page_bytes", "kvq_cache_bytes", "kvq_cache_init", "kvq_append", "kvq_num_selected",
+    "kvq_select_channels", "kvq_decode_workspace", "kvq_decode_attn",
+    "kvq_bf16_decode_workspace", "kvq_bf16_decode_attn", "kvq_read_status",
+    "kvq_status_string", "kvq_version",
+)
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"kvq CUDA library not built: {LIB_PATH} is missing "
+                               "(run python -m long_context_decode_dual_b200.build)")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        C = ctypes.POINTER(CacheDesc)
+        sig = {
+            "kvq_page_bytes": (S, [I]),
+            "kvq_cache_bytes": (S, [C]),
+            "kvq_cache_init": (I, [C, P]),
+            "kvq_append": (I, [C, P, P, I, I, P, P]),
+            "kvq_num_selected": (I, [ctypes.c_float, I]),
+            "kvq_select_channels": (I, [C, P, I, I, P, ctypes.c_float, P, P, P, ctypes.POINTER(I), P]),
+            "kvq_decode_workspace": (S, [C, I, I]),
+            "kvq_decode_attn": (I, [C, I, P, P, P, I, P, P, S, P]),
+            "kvq_bf16_decode_workspace": (S, [I, I, I, I]),
+            "kvq_bf16_decode_attn": (I, [P, P, P, I, I, I, I, P, P, S, P]),
+            "kvq_read_status": (I, [C, ctypes.POINTER(ctypes.c_uint32), P]),
+            "kvq_status_string": (ctypes.c_char_p, [I]),
+            "kvq_version": (I, []),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().kvq_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != KVQ_OK:
+        raise KvqError(fn, status)
+
+
+def _stream(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return KVQ_DTYPE_F32
+    if t.dtype in (torch.bfloat16, torch.int16, torch.uint16):
+        return KVQ_DTYPE_BF16
+    raise TypeError(f"unsupported input dtype {t.dtype} (float32 or bfloat16)")
+
+
+def num_selected(sparsity: float, head_dim: int = HEAD_DIM) -> int:
+    return int(lib().kvq_num_selected(float(sparsity), head_dim))
+
+
+@dataclasses.dataclass
+class KVCache:
+    """A prunable INT2/INT4 KV cache in device memory (kvq_cache)."""
+    batch: int
+    n_kv_heads: int
+    capacity: int
+    bits: int
+    pages: torch.Tensor
+    seq_len: torch.Tensor
+    status: torch.Tensor
+
+    @property
+    def desc(self) -> CacheDesc:
+        return CacheDesc(self.batch, self.n_kv_heads, HEAD_DIM, GROUP, self.bits, self.capacity,
+                         self.pages.data_ptr(), self.seq_len.data_ptr(), self.status.data_ptr())
+
+    @property
+    def n_blocks(self) -> int:
+        return self.capacity // BLOCK_TOKENS
+
+    def unit_pages(self, b: int, h: int) -> torch.Tensor:
+        """Pages of one (sequence, KV head): uint8 [capacity/128][page bytes]."""
+        pb = page_bytes(self.bits)
+        return self.pages.view(self.batch, self.n_kv_heads, self.n_blocks, pb)[b, h]
+
+
+def page_bytes(bits: int) -> int:
+    return int(lib().kvq_page_bytes(bits))
+
+
+def new_cache(batch: int, n_kv_heads: int, capacity: int, bits: int = 2,
+              device="cuda", stream=None) -> KVCache:
+    desc = CacheDesc(batch, n_kv_heads, HEAD_DIM, GROUP, bits, capacity, 0, 0, 0)
+    nbytes = int(lib().kvq_cache_bytes(ctypes.byref(desc)))
+    if nbytes == 0:
+        raise KvqError("kvq_cache_bytes", -2)
+    pages = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    seq_len = torch.empty(batch, dtype=torch.int32, device=device)
+    status = torch.empty(1, dtype=torch.int32, device=device)
+    c = KVCache(batch, n_kv_heads, capacity, bits, pages, seq_len, status)
+    _check("kvq_cache_init", lib().kvq_cache_init(ctypes.byref(c.desc), _stream(stream)))
+    return c
+
+
+def append(cache: KVCache, K: torch.Tensor, V: torch.Tensor, A: torch.Tensor, stream=None) -> None:
+    """kvq_append: K, V [B][Hkv][n_new][128] (f32 or bf16), A [Hkv][128][128] f64."""
+    assert K.is_contiguous() and V.is_contiguous() and A.is_contiguous()
+    assert K.shape == V.shape and K.dim() == 4 and A.dtype == torch.float64
+    _check("kvq_append", lib().kvq_append(ctypes.byref(cache.desc), _ptr(K), _ptr(V), _dtype_code(K),
+                                          int(K.shape[2]), _ptr(A), _stream(stream)))
+
+
+@dataclasses.dataclass
+class Selection:
+    idx: torch.Tensor     # [B][Hkv][k] int32
+    qsel: torch.Tensor    # [B][Hq][k] f32
+    qgsum: torch.Tensor   # [B][Hq][4] f32
+    k: int
+
+
+def alloc_selection(cache: KVCache, n_q_heads: int, k: int, device="cuda") -> Selection:
+    return Selection(
+        torch.empty(cache.batch, cache.n_kv_heads, k, dtype=torch.int32, device=device),
+        torch.empty(cache.batch, n_q_heads, k, dtype=torch.float32, device=device),
+        torch.empty(cache.batch, n_q_heads, 4, dtype=torch.float32, device=device), k)
+
+
+def select_channels(cache: KVCache, q: torch.Tensor, Ainvt: torch.Tensor, sparsity: float,
+                    out: Optional[Selection] = None, stream=None) -> Selection:
+    """kvq_select_channels: q [B][Hq][128] (f32 or bf16), Ainvt [Hkv][128][128] f64."""
+    assert q.is_contiguous() and Ainvt.is_contiguous() and Ainvt.dtype == torch.float64
+    Hq = int(q.shape[1])
+    k = num_selected(sparsity)
+    if k < 0:
+        raise KvqError("kvq_num_selected", -1)
+    sel = out if out is not None else alloc_selection(cache, Hq, k, q.device)
+    assert sel.k == k
+    kout = ctypes.c_int(0)
+    _check("kvq_select_channels", lib().kvq_select_channels(
+        ctypes.byref(cache.desc), _ptr(q), _dtype_code(q), Hq, _ptr(Ainvt), float(sparsity),
+        _ptr(sel.idx), _ptr(sel.qsel), _ptr(sel.qgsum), ctypes.byref(kout), _stream(stream)))
+    assert kout.value == k
+    return sel
+
+
+def decode_workspace_bytes(cache: KVCache, n_q_heads: int, k: int) -> int:
+    return int(lib().kvq_decode_workspace(ctypes.byref(cache.desc), n_q_heads, k))
+
+
+def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+
+
+def decode_attn(cache: KVCache, sel: Selection, out: Optional[torch.Tensor] = None,
+                ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """kvq_decode_attn: returns out [B][Hq][128] f32."""
+    B, Hq, k = cache.batch, int(sel.qsel.shape[1]), sel.k
+    if out is None:
+        out = torch.empty(B, Hq, HEAD_DIM, dtype=torch.float32, device=sel.qsel.device)
+    if ws is None:
+        ws = alloc_workspace(decode_workspace_bytes(cache, Hq, k), sel.qsel.device)
+    _check("kvq_decode_attn", lib().kvq_decode_attn(
+        ctypes.byref(cache.desc), Hq, _ptr(sel.idx), _ptr(sel.qsel), _ptr(sel.qgsum), k, _ptr(out),
+        _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def bf16_workspace_bytes(B: int, Hq: int, Hkv: int, N: int) -> int:
+    return int(lib().kvq_bf16_decode_workspace(B, Hq, Hkv, N))
+
+
+def bf16_decode_attn(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                     out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """kvq_bf16_decode_attn: q [B][Hq][128], K, V [B][Hkv][N][128], all bf16."""
+    B, Hq = int(q.shape[0]), int(q.shape[1])
+    Hkv, N = int(K.shape[1]), int(K.shape[2])
+    for t in (q, K, V):
+        assert t.is_contiguous() and _dtype_code(t) == KVQ_DTYPE_BF16
+    if out is None:
+        out = torch.empty(B, Hq, HEAD_DIM, dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = alloc_workspace(bf16_workspace_bytes(B, Hq, Hkv, N), q.device)
+    _check("kvq_bf16_decode_attn", lib().kvq_bf16_decode_attn(
+        _ptr(q), _ptr(K), _ptr(V), B, Hq, Hkv, N, _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def read_status(cache: KVCache, stream=None) -> int:
+    flags = ctypes.c_uint32(0)
+    _check("kvq_read_status", lib().kvq_read_status(ctypes.byref(cache.desc), ctypes.byref(flags),
+                                                    _stream(stream)))
+    return int(flags.value)

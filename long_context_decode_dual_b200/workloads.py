@@ -211,6 +211,15 @@ def make_kv(wl: Workload, n_tokens: Optional[int] = None, stream_k: int = _S_K,
     return _store(K, wl.dtype), _store(V, wl.dtype)
 
 
+def make_kv_unit(wl: Workload, b: int, h: int, n_tokens: Optional[int] = None):
+    """Keys and values [n][d] of one (batch, KV head): the same draws as make_kv."""
+    n = wl.n_ctx if n_tokens is None else n_tokens
+    k = _draw(_rng(wl.seed, _S_K, (b << 8) | h), (n, HEAD_DIM), wl.dist)
+    k[:, outlier_channels(wl, h)] *= np.float32(wl.outlier_scale)
+    v = _draw(_rng(wl.seed, _S_V, (b << 8) | h), (n, HEAD_DIM), wl.dist)
+    return _store(k, wl.dtype), _store(v, wl.dtype)
+
+
 def make_q(wl: Workload, step: int = 0):
     """Decode query [B][Hq][d] for one step, in the workload's input dtype."""
     q = _rng(wl.seed, _S_Q, step).standard_normal(

@@ -1,0 +1,101 @@
+"""Shared helpers for the GPU parity tests: seeded inputs from the workload
+generator, the oracle's cache/selection/decode for the same inputs, and the
+CUDA path through the Python binding of the C ABI."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from long_context_decode_dual_b200 import kvq
+from long_context_decode_dual_b200 import workloads as W
+from oracle import oracle as orc
+
+
+def to_dev(x: np.ndarray, dtype: str) -> torch.Tensor:
+    if dtype == "f32":
+        return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).cuda()
+    return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def dev64(x: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float64)).cuda()
+
+
+class Case:
+    """Inputs of one workload (possibly shortened) plus both implementations."""
+
+    def __init__(self, wl: W.Workload, n_ctx: int | None = None, capacity: int | None = None):
+        self.wl = wl if n_ctx is None else wl.with_(n_ctx=n_ctx)
+        self.capacity = capacity or self.wl.capacity
+        self.A, self.Ai = W.make_transforms(self.wl)
+        self.K, self.V = W.make_kv(self.wl)
+        self._oracle_units = {}
+
+    # ---------------------------------------------------------------- GPU
+    def gpu_cache(self, chunks=None) -> kvq.KVCache:
+        wl = self.wl
+        cache = kvq.new_cache(wl.batch, wl.n_kv_heads, self.capacity, wl.bits)
+        A = dev64(self.A)
+        n = self.K.shape[2]
+        chunks = chunks or [n]
+        pos = 0
+        for c in chunks:
+            kvq.append(cache, to_dev(self.K[:, :, pos:pos + c], wl.dtype),
+                       to_dev(self.V[:, :, pos:pos + c], wl.dtype), A)
+            pos += c
+        assert pos == n
+        return cache
+
+    def q(self, step: int = 0) -> np.ndarray:
+        return W.make_q(self.wl, step)
+
+    # ------------------------------------------------------------- oracle
+    def oracle_unit(self, b: int, h: int, n: int | None = None) -> np.ndarray:
+        key = (b, h, n)
+        if key not in self._oracle_units:
+            wl = self.wl
+            n = self.K.shape[2] if n is None else n
+            Kf = W.as_float(self.K[b, h, :n], wl.dtype)
+            Vf = W.as_float(self.V[b, h, :n], wl.dtype)
+            u = orc.new_unit(self.capacity, wl.bits)
+            orc.append_unit(u, wl.bits, 0, orc.transform(Kf, self.A[h]), Vf)
+            self._oracle_units[key] = u
+        return self._oracle_units[key]
+
+    def oracle_qp(self, q: np.ndarray, b: int, h: int) -> np.ndarray:
+        g = self.wl.group_size
+        qf = W.as_float(q[b, h * g:(h + 1) * g], self.wl.dtype)
+        return orc.transform(qf, self.Ai[h])
+
+    def oracle_decode(self, q: np.ndarray, b: int, h: int, sparsity: float, n: int | None = None):
+        n = self.K.shape[2] if n is None else n
+        qp = self.oracle_qp(q, b, h)
+        out, idx = orc.decode_unit(self.oracle_unit(b, h), self.wl.bits, n, qp, sparsity)
+        return out, idx, qp
+
+
+def expected_qsel_qgsum(qp: np.ndarray, idx: np.ndarray):
+    """fp32 rounding of q'[h][idx] and of the float64 ascending sum per key
+    group of the kept channels other than channel 0 (the documented
+    definition of kvq_select_channels' outputs)."""
+    qsel = qp[:, idx].astype(np.float32)
+    g = qp.shape[0]
+    qgsum = np.zeros((g, 4), dtype=np.float32)
+    for hl in range(g):
+        for gr in range(4):
+            s = 0.0
+            for c in idx:
+                if c != 0 and c // 32 == gr:
+                    s += float(qp[hl, c])
+            qgsum[hl, gr] = np.float32(s)
+    return qsel, qgsum
+
+
+def rel_errors(out: np.ndarray, ref: np.ndarray):
+    """Per output vector: max and mean of |out - ref| / ||ref||_inf."""
+    ref = np.asarray(ref, dtype=np.float64)
+    out = np.asarray(out, dtype=np.float64)
+    scale = np.abs(ref).max(axis=-1, keepdims=True)
+    scale = np.where(scale == 0, 1.0, scale)
+    e = np.abs(out - ref) / scale
+    return e.max(), e.mean()

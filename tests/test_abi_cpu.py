@@ -1,0 +1,66 @@
+"""The C ABI library loads on a machine without a GPU and exports every entry
+point declared in include/kvq.h; host-side validation answers without
+touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from long_context_decode_dual_b200 import kvq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kvq.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kvq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared()
+    assert len(names) >= 12
+    L = kvq.lib()
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing, missing
+    assert set(names) == set(kvq.EXPORTS)
+
+
+def test_host_side_queries():
+    L = kvq.lib()
+    assert L.kvq_version() == 100
+    assert L.kvq_page_bytes(2) == 12544 and L.kvq_page_bytes(4) == 20736 and L.kvq_page_bytes(3) == 0
+    for s, k in ((0.0, 128), (0.2, 103), (0.4, 77), (0.6, 52), (0.25, 96)):
+        assert kvq.num_selected(s) == k
+    assert kvq.num_selected(1.0) == -1 and kvq.num_selected(-0.1) == -1
+    d = kvq.CacheDesc(2, 8, 128, 32, 2, 256, 0, 0, 0)
+    assert L.kvq_cache_bytes(ctypes.byref(d)) == 2 * 8 * 2 * 12544
+    bad = kvq.CacheDesc(2, 8, 64, 32, 2, 256, 0, 0, 0)
+    assert L.kvq_cache_bytes(ctypes.byref(bad)) == 0
+    assert kvq.status_string(-3) == "capacity exceeded"
+
+
+def test_validation_rejects_before_launch():
+    L = kvq.lib()
+    nullc = kvq.CacheDesc(1, 1, 128, 32, 2, 128, 0, 0, 0)
+    assert L.kvq_cache_init(ctypes.byref(nullc), None) == -1
+    assert L.kvq_append(None, None, None, 0, 1, None, None) == -1
+    fake = kvq.CacheDesc(1, 1, 128, 32, 3, 128, 256, 256, 256)     # bits 3
+    assert L.kvq_append(ctypes.byref(fake), 8, 8, 0, 1, 8, None) == -2
+    mis = kvq.CacheDesc(1, 1, 128, 32, 2, 128, 0x1010, 256, 256)  # pages not 256-aligned
+    assert L.kvq_append(ctypes.byref(mis), 8, 8, 0, 1, 8, None) == -6
+    ok = kvq.CacheDesc(1, 1, 128, 32, 2, 128, 0x1000, 256, 256)
+    assert L.kvq_append(ctypes.byref(ok), 8, 8, 0, -1, 8, None) == -1
+    assert L.kvq_append(ctypes.byref(ok), 8, 8, 7, 1, 8, None) == -1             # dtype
+    assert L.kvq_append(ctypes.byref(ok), 8, 8, 0, 129, 8, None) == -3          # > capacity
+    assert L.kvq_append(ctypes.byref(ok), 8, 8, 0, 0, 8, None) == 0             # no-op
+    two = kvq.CacheDesc(1, 2, 128, 32, 2, 128, 0x1000, 256, 256)
+    assert L.kvq_select_channels(ctypes.byref(two), 8, 0, 3, 8, ctypes.c_float(0.4), 8, 8, 8,
+                                 None, None) == -2                              # 3 % 2 heads
+    assert L.kvq_select_channels(ctypes.byref(two), 8, 0, 4, 8, ctypes.c_float(1.5), 8, 8, 8,
+                                 None, None) == -1                              # sparsity
+    assert L.kvq_decode_attn(ctypes.byref(two), 6, 8, 8, 8, 77, 8, 8, 1 << 20, None) == -2  # g = 3
+    assert L.kvq_decode_attn(ctypes.byref(two), 4, 8, 8, 8, 0, 8, 8, 1 << 20, None) == -1   # k = 0
+    assert L.kvq_bf16_decode_attn(8, 8, 8, 1, 3, 2, 10, 8, 8, 1 << 20, None) == -2

@@ -1,0 +1,217 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Bars: packed codes, fp16 scale/zero bit patterns, bf16 channel 0 and the
+selected channel indices are bit-exact; qsel / qgsum are the documented fp32
+roundings, bit-exact; the attention output is within 2e-3 max and 1e-3 mean
+relative error (|o - o_ref| / ||o_ref||_inf per output vector) of the oracle
+run on the same codes and the same selected channels.
+"""
+import numpy as np
+import pytest
+import torch
+
+from long_context_decode_dual_b200 import kvq
+from long_context_decode_dual_b200 import workloads as W
+from oracle import oracle as orc
+
+from helpers import Case, dev64, expected_qsel_qgsum, rel_errors, to_dev
+
+pytestmark = pytest.mark.gpu
+
+TOL_MAX = 2e-3
+TOL_MEAN = 1e-3
+
+
+def _check_pages(case: Case, cache: kvq.KVCache, units=None, n=None):
+    pages = cache.pages.cpu().numpy()
+    wl = case.wl
+    pb = kvq.page_bytes(wl.bits)
+    pages = pages.reshape(wl.batch, wl.n_kv_heads, case.capacity // 128, pb)
+    units = units or [(b, h) for b in range(wl.batch) for h in range(wl.n_kv_heads)]
+    for b, h in units:
+        ref = case.oracle_unit(b, h, n)
+        got = pages[b, h]
+        if not np.array_equal(got, ref):
+            bad = np.argwhere(got != ref)
+            raise AssertionError(f"unit {(b, h)}: {len(bad)} bytes differ, first (page, byte) {bad[:4].tolist()}")
+
+
+def _cases_small():
+    return [
+        ("single_head_4k", None),
+        ("llama8b_b8_32k", 300),
+        ("longctx_b1_128k", 257),
+        ("sweep_b32_16k", 130),
+        ("pipeline_128k_t4", 1000),
+    ]
+
+
+@pytest.mark.parametrize("name,n_ctx", _cases_small())
+@pytest.mark.parametrize("bits", [2, 4])
+def test_append_bit_exact(name, n_ctx, bits):
+    case = Case(W.workload(name, bits=bits), n_ctx=n_ctx)
+    cache = case.gpu_cache()
+    assert cache.seq_len.cpu().tolist() == [case.K.shape[2]] * case.wl.batch
+    assert kvq.read_status(cache) == 0
+    _check_pages(case, cache)
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_append_in_chunks_keeps_neighbouring_codes(bits):
+    case = Case(W.workload("llama8b_b8_32k", batch=2, bits=bits), n_ctx=291)
+    cache = case.gpu_cache(chunks=[7, 1, 130, 1, 3, 16, 133])
+    _check_pages(case, cache)
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_append_rounding_edges(bits):
+    """Keys whose transformed values sit on or next to fp16 / bf16 rounding
+    ties, in the fp16 subnormal range, and groups with a zero range."""
+    rng = np.random.default_rng(123)
+    edges = np.array([1 + 2.0 ** -11, 1 + 2.0 ** -11 + 2.0 ** -45, 1 + 2.0 ** -11 - 2.0 ** -45,
+                      1 + 3 * 2.0 ** -11, 1 + 2.0 ** -8 + 2.0 ** -40, 1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8,
+                      2.0 ** -20, 3 * 2.0 ** -25, 1.0, 2.0 ** -14 * (1 + 2.0 ** -11), 1000.5])
+    wl = W.workload("single_head_4k", bits=bits)
+    n = 256
+    case = Case(wl, n_ctx=n)
+    A = np.diag(rng.choice(edges, 128)).reshape(1, 128, 128)
+    K = rng.choice([1.0, -1.0, 1.5, 0.75, 2.0, -0.5], size=(1, 1, n, 128)).astype(np.float32)
+    K[0, 0, :16, 1:32] = 0.5          # zero-range groups
+    V = rng.choice([0.25, -3.0, 1.0 + 2.0 ** -11, 7.5], size=(1, 1, n, 128)).astype(np.float32)
+    case.A, case.K, case.V = A, K, V
+    cache = case.gpu_cache()
+    _check_pages(case, cache)
+
+
+def test_append_capacity_overflow_sets_flag():
+    case = Case(W.workload("llama8b_b8_32k", batch=2), n_ctx=200, capacity=256)
+    cache = case.gpu_cache()
+    before = cache.pages.clone()
+    extra = W.make_kv(case.wl.with_(n_ctx=100))
+    kvq.append(cache, to_dev(extra[0], "bf16"), to_dev(extra[1], "bf16"), dev64(case.A))
+    assert kvq.read_status(cache) & kvq.KVQ_DEV_CAPACITY
+    assert cache.seq_len.cpu().tolist() == [200, 200]
+    assert torch.equal(before, cache.pages)
+    with pytest.raises(kvq.KvqError):
+        kvq.append(cache, to_dev(extra[0][:, :, :1].repeat(300, axis=2), "bf16"),
+                   to_dev(extra[1][:, :, :1].repeat(300, axis=2), "bf16"), dev64(case.A))
+
+
+def _check_selection(case: Case, q: np.ndarray, sel: kvq.Selection, sparsity: float):
+    wl = case.wl
+    g = wl.group_size
+    k = orc.num_selected(sparsity)
+    assert sel.k == k
+    idx = sel.idx.cpu().numpy()
+    qsel = sel.qsel.cpu().numpy()
+    qgsum = sel.qgsum.cpu().numpy()
+    for b in range(wl.batch):
+        for h in range(wl.n_kv_heads):
+            qp = case.oracle_qp(q, b, h)
+            ref_idx, _ = orc.select(qp, k)
+            assert np.array_equal(idx[b, h], ref_idx), (b, h)
+            rq, rg = expected_qsel_qgsum(qp, ref_idx)
+            assert np.array_equal(qsel[b, h * g:(h + 1) * g], rq), (b, h)
+            assert np.array_equal(qgsum[b, h * g:(h + 1) * g], rg), (b, h)
+
+
+@pytest.mark.parametrize("name", list(W.WORKLOADS))
+@pytest.mark.parametrize("sparsity", W.SWEEP_SPARSITIES)
+def test_select_bit_exact(name, sparsity):
+    case = Case(W.workload(name), n_ctx=128)
+    cache = kvq.new_cache(case.wl.batch, case.wl.n_kv_heads, case.capacity, 2)
+    for step in range(2):
+        q = case.q(step)
+        sel = kvq.select_channels(cache, to_dev(q, case.wl.dtype), dev64(case.Ai), sparsity)
+        _check_selection(case, q, sel, sparsity)
+
+
+def test_select_ties_go_to_lower_channel():
+    wl = W.workload("llama8b_b8_32k", batch=2)
+    case = Case(wl, n_ctx=128)
+    case.Ai = np.broadcast_to(np.eye(128), (wl.n_kv_heads, 128, 128)).copy()
+    rng = np.random.default_rng(5)
+    q = W.bf16_bits_from_f32(rng.integers(-2, 3, size=(2, 32, 128)).astype(np.float32))
+    cache = kvq.new_cache(2, 8, 128, 2)
+    for s in (0.2, 0.4, 0.6):
+        sel = kvq.select_channels(cache, to_dev(q, "bf16"), dev64(case.Ai), s)
+        _check_selection(case, q, sel, s)
+
+
+def _decode_and_compare(case: Case, cache, sparsity, steps=(0,), units=None, n=None):
+    wl = case.wl
+    g = wl.group_size
+    errs = []
+    for step in steps:
+        q = case.q(step)
+        sel = kvq.select_channels(cache, to_dev(q, wl.dtype), dev64(case.Ai), sparsity)
+        out = kvq.decode_attn(cache, sel).cpu().numpy()
+        us = units or [(b, h) for b in range(wl.batch) for h in range(wl.n_kv_heads)]
+        for b, h in us:
+            ref, ref_idx, _ = case.oracle_decode(q, b, h, sparsity, n)
+            assert np.array_equal(sel.idx[b, h].cpu().numpy(), ref_idx)
+            got = out[b, h * g:(h + 1) * g]
+            emax, emean = rel_errors(got, ref)
+            errs.append((emax, emean))
+            assert emax <= TOL_MAX and emean <= TOL_MEAN, (step, b, h, emax, emean)
+    return errs
+
+
+@pytest.mark.parametrize("name,n_ctx", _cases_small())
+@pytest.mark.parametrize("bits", [2, 4])
+def test_decode_parity(name, n_ctx, bits):
+    case = Case(W.workload(name, bits=bits), n_ctx=n_ctx)
+    cache = case.gpu_cache()
+    _decode_and_compare(case, cache, case.wl.sparsity, steps=(0, 1))
+
+
+@pytest.mark.parametrize("sparsity", W.SWEEP_SPARSITIES)
+def test_decode_parity_sparsity_sweep(sparsity):
+    case = Case(W.workload("sweep_b32_16k", batch=4), n_ctx=700)
+    cache = case.gpu_cache()
+    _decode_and_compare(case, cache, sparsity)
+
+
+@pytest.mark.parametrize("g", [1, 2, 4, 8])
+def test_decode_parity_group_sizes(g):
+    case = Case(W.workload("llama8b_b8_32k", batch=2, n_q_heads=4 * g, n_kv_heads=4), n_ctx=515)
+    cache = case.gpu_cache()
+    _decode_and_compare(case, cache, 0.4)
+
+
+def test_decode_edge_lengths():
+    case = Case(W.workload("llama8b_b8_32k", batch=4), n_ctx=300)
+    cache = case.gpu_cache()
+    q = case.q(0)
+    g = case.wl.group_size
+    # ragged lengths: the caller owns seq_len; decode must honour it
+    lens = [0, 1, 128, 129]
+    cache.seq_len.copy_(torch.tensor(lens, dtype=torch.int32))
+    sel = kvq.select_channels(cache, to_dev(q, "bf16"), dev64(case.Ai), 0.4)
+    out = kvq.decode_attn(cache, sel).cpu().numpy()
+    assert not out[0].any()                                     # empty sequence -> zeros
+    for b, n in enumerate(lens[1:], start=1):
+        for h in (0, 5):
+            ref, _, _ = case.oracle_decode(q, b, h, 0.4, n)
+            emax, emean = rel_errors(out[b, h * g:(h + 1) * g], ref)
+            assert emax <= TOL_MAX and emean <= TOL_MEAN, (b, h, emax)
+    # a single token: the output is that token's dequantized value row
+    _, Vh = orc.dequant_unit(case.oracle_unit(1, 0), 2, 1)
+    np.testing.assert_allclose(out[1, 0], Vh[0], rtol=1e-6, atol=1e-6)
+
+
+def test_bf16_comparator_matches_plain_attention():
+    wl = W.workload("llama8b_b8_32k", batch=2)
+    case = Case(wl, n_ctx=1000)
+    q = case.q(0)
+    out = kvq.bf16_decode_attn(to_dev(q, "bf16"), to_dev(case.K, "bf16"), to_dev(case.V, "bf16")).cpu().numpy()
+    g = wl.group_size
+    for b in range(2):
+        for h in range(wl.n_kv_heads):
+            ref = orc.attention(W.as_float(q[b, h * g:(h + 1) * g], "bf16"),
+                                W.as_float(case.K[b, h], "bf16"), W.as_float(case.V[b, h], "bf16"))
+            emax, emean = rel_errors(out[b, h * g:(h + 1) * g], ref)
+            assert emax <= TOL_MAX and emean <= TOL_MEAN, (b, h, emax)
+    empty = kvq.bf16_decode_attn(to_dev(q, "bf16"), to_dev(case.K[:, :, :0], "bf16"),
+                                 to_dev(case.V[:, :, :0], "bf16"))
+    assert not empty.any()
