@@ -199,6 +199,34 @@ int kvq_bf16_decode_attn(const void *q, const void *K, const void *V, int batch,
                          int n_q_heads, int n_kv_heads, int n_tokens, float *out,
                          void *ws, size_t ws_bytes, kvq_stream_t stream);
 
+/*
+ * kvq_decode_attn_static -- kvq_decode_attn for callers that cannot allocate
+ * device memory at call time (for example a plugin inside an inference engine
+ * that owns all device memory and offers no scratch buffer, or a decode loop
+ * that must not call cudaMalloc, which may synchronise the device).  The
+ * paper has no counterpart; this is a deployment convenience.
+ *
+ * Same arguments, arithmetic and result as kvq_decode_attn, without ws /
+ * ws_bytes: the split partials live in one static device array of
+ * kvq_decode_static_scratch_bytes() bytes (4 MiB) that every GPU loading this
+ * library holds until the process exits.  The library allocates nothing.
+ *  - The first call on a device, with that device current, looks up the
+ *    array's device address (cudaGetSymbolAddress) and caches it; make that
+ *    first call before any stream capture.
+ *  - All calls share the one array, and it keeps the last call's contents.
+ *    Nothing in it needs to start at zero.  Calls whose kernels can overlap
+ *    on the GPU (different streams, or different host threads) race on it:
+ *    serialise them.
+ *  - A request needing more than the maximum (kvq_decode_workspace() >
+ *    kvq_decode_static_scratch_bytes()) returns KVQ_ERR_WORKSPACE and
+ *    launches nothing.
+ * Errors: as kvq_decode_attn, plus KVQ_ERR_CUDA if the address lookup fails.
+ */
+size_t kvq_decode_static_scratch_bytes(void);
+int kvq_decode_attn_static(const kvq_cache *cache, int n_q_heads, const int32_t *idx,
+                           const float *qsel, const float *qgsum, int k, float *out,
+                           kvq_stream_t stream);
+
 /* Copy the device status word into *flags (synchronises the stream).
  * KVQ_ERR_ARG on null pointers, KVQ_ERR_CUDA on a failed copy. */
 int kvq_read_status(const kvq_cache *cache, uint32_t *flags, kvq_stream_t stream);

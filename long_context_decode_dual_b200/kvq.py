@@ -51,7 +51,8 @@ EXPORTS = (
     "kvq_page_bytes", "kvq_cache_bytes", "kvq_cache_init", "kvq_append", "kvq_num_selected",
     "kvq_select_channels", "kvq_decode_workspace", "kvq_decode_attn",
     "kvq_bf16_decode_workspace", "kvq_bf16_decode_attn", "kvq_read_status",
-    "kvq_status_string", "kvq_version",
+    "kvq_status_string", "kvq_version", "kvq_decode_static_scratch_bytes",
+    "kvq_decode_attn_static",
 )
 
 
@@ -79,6 +80,8 @@ def lib() -> ctypes.CDLL:
             "kvq_read_status": (I, [C, ctypes.POINTER(ctypes.c_uint32), P]),
             "kvq_status_string": (ctypes.c_char_p, [I]),
             "kvq_version": (I, []),
+            "kvq_decode_static_scratch_bytes": (S, []),
+            "kvq_decode_attn_static": (I, [C, I, P, P, P, I, P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -223,6 +226,27 @@ def decode_attn(cache: KVCache, sel: Selection, out: Optional[torch.Tensor] = No
         ctypes.byref(cache.desc), Hq, _ptr(sel.idx), _ptr(sel.qsel), _ptr(sel.qgsum), k, _ptr(out),
         _ptr(ws), ws.numel(), _stream(stream)))
     return out
+
+
+def decode_attn_static(cache: KVCache, sel: Selection, out: Optional[torch.Tensor] = None,
+                       stream=None) -> torch.Tensor:
+    """kvq_decode_attn_static: decode without a caller workspace.
+
+    For callers that cannot allocate device memory when they decode; the
+    split partials use the library's one static device array, shared by all
+    calls (serialise calls that could overlap on the GPU).
+    """
+    B, Hq, k = cache.batch, int(sel.qsel.shape[1]), sel.k
+    if out is None:
+        out = torch.empty(B, Hq, HEAD_DIM, dtype=torch.float32, device=sel.qsel.device)
+    _check("kvq_decode_attn_static", lib().kvq_decode_attn_static(
+        ctypes.byref(cache.desc), Hq, _ptr(sel.idx), _ptr(sel.qsel), _ptr(sel.qgsum), k, _ptr(out),
+        _stream(stream)))
+    return out
+
+
+def decode_static_scratch_bytes() -> int:
+    return int(lib().kvq_decode_static_scratch_bytes())
 
 
 def bf16_workspace_bytes(B: int, Hq: int, Hkv: int, N: int) -> int:
