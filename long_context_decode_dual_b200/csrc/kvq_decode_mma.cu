@@ -1,0 +1,471 @@
+// Channel-skipping decode attention on the tensor cores: INT2 codes, four
+// query heads per KV head (the GQA 4:1 shape of the Dual-QK workloads).
+//
+// "Dual-QK: Sharp Queries and Flat Keys for Prunable 2-bit KV Caches":
+//   §3.2 scores over the retained channels only, 1/sqrt(d) with the full d;
+//   §3.3 only the 32-byte key rows selected by the shared mask are copied
+//        from each 128-token page; values and metadata are read in full;
+//   §3.4 one softmax over every token (online per warp, merged per CTA and
+//        then across CTAs), followed by value aggregation.
+//
+// Both contractions of a page are small dense GEMMs once the codes are
+// unpacked, and they run as mma.sync m16n8k16 (f16 in, f32 accumulate):
+//   scores^T[token][head] = codes^T[token][channel] . q'[channel][head]
+//   out^T[channel][head]  = codes[channel][token]   . w[token][head]
+// Codes stay exact: a 2-bit field masked in place inside a 16-bit half is an
+// fp16 subnormal equal to code * 2^(pos-24), so unpacking is one AND per two
+// codes; the power of two is compensated exactly on the other operand or in
+// fp32 afterwards.  Query and weights are split into fp16 hi + lo parts that
+// occupy the two columns of each head (n = 8 = 4 heads x {hi, lo}), giving
+// near-fp32 operands.  Per-token, per-group scale and zero-point are applied
+// in fp32 after the score MMAs, folded into the weights before the value
+// MMAs, and the value zero-point term sum_t p(t) z(t) is one more MMA.
+//
+// One CTA = one (sequence, KV head, split of the context), four warps; each
+// warp owns whole pages (its own online softmax) with a two-stage cp.async
+// ring in shared memory.  Selected key rows land in fixed slots: group g owns
+// slots 32g..32g+31, filled in ascending channel order, so every MMA k-step
+// (16 slots) lies inside one group and its scale applies to the whole step.
+#include "kvq_internal.cuh"
+
+namespace kvq {
+namespace {
+
+constexpr int kWarps = 4;
+constexpr int kSlotBytes = 128 * 32;              // 4 groups x 32 slots x 32 B
+constexpr int kFixBytes = fixed_bytes(2);         // value codes, ch0, metadata
+constexpr int kStageBytes = kSlotBytes + kFixBytes;
+constexpr int kMaxTasks = 2 * 127;                // 16-byte copies of key rows
+constexpr int kPexStride = 164;                   // floats per head in the p exchange
+
+struct __align__(16) MmaShared {
+    uint8_t stage[kWarps][2][kStageBytes];
+    uint32_t task[kMaxTasks];          // src offset | dst offset << 16 (bytes)
+    float q[4][kD];                    // qsel of the 4 heads, by selected position
+    float qg[4][kNG];
+    int slot_pos[kD];                  // slot -> position in the selected list, -1 = pad
+    int nks[kNG];                      // MMA k-steps per key group (0, 1 or 2)
+    int n_tasks;
+};
+
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
+__device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2 *>(&u); }
+__device__ __forceinline__ float lo_f16(uint32_t w) { return __half2float(__ushort_as_half((uint16_t)(w & 0xffffu))); }
+__device__ __forceinline__ float hi_f16(uint32_t w) { return __half2float(__ushort_as_half((uint16_t)(w >> 16))); }
+
+// fp16 hi/lo split of a float: hi = fp16(x), lo = fp16(x - hi)
+__device__ __forceinline__ uint16_t f16_part(float x, int part) {
+    const __half hi = __float2half_rn(x);
+    if (part == 0) return __half_as_ushort(hi);
+    return __half_as_ushort(__float2half_rn(x - __half2float(hi)));
+}
+
+__global__ void __launch_bounds__(128, 2)
+decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len, int Hkv,
+                  int NB, int Hq, const int32_t *__restrict__ idx, const float *__restrict__ qsel,
+                  const float *__restrict__ qgsum, int k, float *__restrict__ part_o,
+                  float2 *__restrict__ part_ml, int S) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    MmaShared &sh = *reinterpret_cast<MmaShared *>(smem_raw);
+
+    const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int gid = lane >> 2, tig = lane & 3;
+    const size_t unit = (size_t)b * Hkv + h;
+    const size_t qrow0 = (size_t)b * Hq + (size_t)h * 4;
+
+    // ------------------------------------------------------------ prologue
+    // The selected list is ascending, so each group's channels sit in one
+    // contiguous run of positions; a channel's slot is 32g + (its position -
+    // the first position of its group).
+    for (int e = tid; e < 4 * k; e += 128) {
+        const int hl = e / k, i = e % k;
+        sh.q[hl][i] = qsel[(qrow0 + hl) * k + i];
+    }
+    if (tid < 4 * kNG) sh.qg[tid / kNG][tid % kNG] = qgsum[qrow0 * kNG + tid];
+    for (int i = tid; i < kD; i += 128) sh.slot_pos[i] = -1;
+    if (tid < kNG) sh.nks[tid] = 0;
+    __syncthreads();
+    const int32_t *sel = idx + unit * k;
+    const int my_c = (tid >= 1 && tid < k) ? sel[tid] : -1;
+    if (my_c >= 0) atomicAdd(&sh.nks[my_c >> 5], 1);          // counts for now
+    __syncthreads();
+    if (my_c >= 0) {
+        const int g = my_c >> 5;
+        int start = 1;
+        for (int gg = 0; gg < g; gg++) start += sh.nks[gg];
+        const int slot = 32 * g + (tid - start);
+        sh.slot_pos[slot] = tid;
+        sh.task[2 * (tid - 1)] = (uint32_t)(my_c * 32) | ((uint32_t)(slot * 32) << 16);
+        sh.task[2 * (tid - 1) + 1] = (uint32_t)(my_c * 32 + 16) | ((uint32_t)(slot * 32 + 16) << 16);
+    }
+    if (tid == 0) sh.n_tasks = 2 * (k - 1);
+    __syncthreads();
+    if (tid < kNG) sh.nks[tid] = (sh.nks[tid] + 15) >> 4;       // counts -> k-steps
+    __syncthreads();
+
+    // score-MMA B fragments: column gid = (head gid>>1, part gid&1); k-slots
+    // 2tig, 2tig+1, 2tig+8, 2tig+9 of a step = slots +tig, +tig+4, +tig+8, +tig+12
+    // (this slot order makes the code loads bank-conflict free)
+    const int hh = gid >> 1, part = gid & 1;
+    uint32_t bq[8][2];
+#pragma unroll
+    for (int ks = 0; ks < 8; ks++) {
+        const int base = 32 * (ks >> 1) + 16 * (ks & 1);
+#pragma unroll
+        for (int r = 0; r < 2; r++) {
+            const int s0 = base + tig + 8 * r, s1 = s0 + 4;
+            const int p0 = sh.slot_pos[s0], p1 = sh.slot_pos[s1];
+            const float q0 = p0 >= 0 ? sh.q[hh][p0] : 0.f;
+            const float q1 = p1 >= 0 ? sh.q[hh][p1] : 0.f;
+            bq[ks][r] = (uint32_t)f16_part(q0, part) | ((uint32_t)f16_part(q1, part) << 16);
+        }
+    }
+    int nks[kNG];
+#pragma unroll
+    for (int g = 0; g < kNG; g++) nks[g] = sh.nks[g];
+    float qg_t[kNG];
+#pragma unroll
+    for (int g = 0; g < kNG; g++) qg_t[g] = sh.qg[tig][g];
+    const float q0_t = sh.q[tig][0];                 // channel-0 coefficient of head tig
+    const int n_tasks = sh.n_tasks;
+
+    // ------------------------------------------------------------ pages
+    const int len = min(max(seq_len[b], 0), NB * kT);
+    const int nblk = (len + kT - 1) / kT;
+    const int bps = (nblk + S - 1) / S;
+    const int blk0 = s * bps;
+    const int blk1 = min(nblk, blk0 + bps);
+
+    auto issue = [&](uint8_t *dst, int blk) {
+        const uint8_t *src = pages + (unit * NB + (size_t)blk) * page_bytes(2);
+        for (int e = lane; e < n_tasks; e += 32) {
+            const uint32_t t = sh.task[e];
+            cp_async16(dst + (t >> 16), src + (t & 0xffffu));
+        }
+#pragma unroll 4
+        for (int e = lane; e < kFixBytes / 16; e += 32)
+            cp_async16(dst + kSlotBytes + 16 * e, src + off_vcodes(2) + 16 * e);
+        cp_async_commit();
+    };
+
+    float m_run = -INFINITY;      // running max of head tig (base-2 domain)
+    float l_thr = 0.f;            // this thread's share of the running sum of head tig
+    float co[8][4];               // out^T: rows 16mt+gid / +8, columns head tig {hi, lo}
+    float cz[4];                  // value zero-point term: row gid = group gid
+#pragma unroll
+    for (int mt = 0; mt < 8; mt++)
+#pragma unroll
+        for (int r = 0; r < 4; r++) co[mt][r] = 0.f;
+#pragma unroll
+    for (int r = 0; r < 4; r++) cz[r] = 0.f;
+
+    const uint32_t lane_row_off = 4u * gid;          // word gid of a 32-byte code row
+    const float zmask = gid < 4 ? 1.f : 0.f;
+
+    int it = 0;
+    const int first = blk0 + warp;
+    if (first < blk1) issue(sh.stage[warp][0], first);
+    for (int pg = first; pg < blk1; pg += kWarps, it++) {
+        uint8_t *cur = sh.stage[warp][it & 1];
+        if (pg + kWarps < blk1) {
+            issue(sh.stage[warp][(it + 1) & 1], pg + kWarps);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncwarp();
+
+        const uint8_t *vcodes = cur + kSlotBytes;
+        const uint32_t *ch0w = reinterpret_cast<const uint32_t *>(vcodes + 128 * 32);
+        const uint32_t *kmeta = reinterpret_cast<const uint32_t *>(vcodes + 128 * 32 + 256);
+        const uint32_t *vmeta = kmeta + kNG * kT;
+
+        // ---------------- scores: thread holds tokens 16gid + 2i (+1), head tig
+        float sc[8][2], zt[8][2];
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            sc[i][0] = sc[i][1] = 0.f;
+            zt[i][0] = zt[i][1] = 0.f;
+        }
+#pragma unroll
+        for (int g = 0; g < kNG; g++) {
+            if (nks[g] == 0) continue;
+            float C[8][4];
+#pragma unroll
+            for (int i = 0; i < 8; i++) C[i][0] = C[i][1] = C[i][2] = C[i][3] = 0.f;
+#pragma unroll
+            for (int j = 0; j < 2; j++) {
+                if (j >= nks[g]) break;
+                const uint8_t *sb = cur + (32 * g + 16 * j + tig) * 32 + lane_row_off;
+                const uint32_t Wa = *reinterpret_cast<const uint32_t *>(sb);
+                const uint32_t Wb = *reinterpret_cast<const uint32_t *>(sb + 4 * 32);
+                const uint32_t Wc = *reinterpret_cast<const uint32_t *>(sb + 8 * 32);
+                const uint32_t Wd = *reinterpret_cast<const uint32_t *>(sb + 12 * 32);
+                const uint32_t Xab[2] = {__byte_perm(Wa, Wb, 0x5410), __byte_perm(Wa, Wb, 0x7632)};
+                const uint32_t Xcd[2] = {__byte_perm(Wc, Wd, 0x5410), __byte_perm(Wc, Wd, 0x7632)};
+                const uint32_t Yab[2] = {Xab[0] >> 8, Xab[1] >> 8};
+                const uint32_t Ycd[2] = {Xcd[0] >> 8, Xcd[1] >> 8};
+                const uint32_t b0 = bq[2 * g + j][0], b1 = bq[2 * g + j][1];
+#pragma unroll
+                for (int i = 0; i < 8; i++) {
+                    const int hf = i >> 2;
+                    const uint32_t x1 = (i & 2) ? Yab[hf] : Xab[hf];
+                    const uint32_t x2 = (i & 2) ? Ycd[hf] : Xcd[hf];
+                    const uint32_t m0 = 0x00030003u << (4 * (i & 1));
+                    const uint32_t m1 = m0 << 2;
+                    mma16816(C[i], x1 & m0, x1 & m1, x2 & m0, x2 & m1, b0, b1);
+                }
+            }
+            // scale and zero-point of group g for the thread's 16 tokens
+            const uint4 *kw4 = reinterpret_cast<const uint4 *>(kmeta + g * kT + 16 * gid);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; q4++) {
+                const uint4 w = kw4[q4];
+                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                    const int tt = 4 * q4 + e, i = tt >> 1, r = tt & 1;
+                    sc[i][r] = fmaf(lo_f16(ws[e]), C[i][2 * r] + C[i][2 * r + 1], sc[i][r]);
+                    zt[i][r] = fmaf(hi_f16(ws[e]), qg_t[g], zt[i][r]);
+                }
+            }
+        }
+        // full scores (base-2 domain), masked beyond the sequence
+        const uint4 *c04 = reinterpret_cast<const uint4 *>(ch0w + 8 * gid);
+        float mx = -INFINITY;
+        const int tok0 = pg * kT + 16 * gid;
+#pragma unroll
+        for (int q2 = 0; q2 < 2; q2++) {
+            const uint4 w = c04[q2];
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; e++) {
+                const int i = 4 * q2 + e;      // tokens 2i, 2i+1 of the 16
+#pragma unroll
+                for (int r = 0; r < 2; r++) {
+                    const float c0v = __uint_as_float(r ? (ws[e] & 0xffff0000u) : (ws[e] << 16));
+                    const float comp = __int_as_float((127 + 24 - 4 * (i & 1) - 2 * r) << 23);
+                    float v = fmaf(sc[i][r], comp, fmaf(q0_t, c0v, zt[i][r])) * kScoreScaleLog2;
+                    v = (tok0 + 2 * i + r < len) ? v : -INFINITY;
+                    sc[i][r] = v;
+                    mx = fmaxf(mx, v);
+                }
+            }
+        }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        const float m_new = fmaxf(m_run, mx);
+        const float alpha = exp2f(m_run - m_new);
+        m_run = m_new;
+        float psum = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; i++)
+#pragma unroll
+            for (int r = 0; r < 2; r++) {
+                sc[i][r] = exp2f(sc[i][r] - m_new);
+                psum += sc[i][r];
+            }
+        l_thr = fmaf(l_thr, alpha, psum);
+#pragma unroll
+        for (int mt = 0; mt < 8; mt++)
+#pragma unroll
+            for (int r = 0; r < 4; r++) co[mt][r] *= alpha;
+#pragma unroll
+        for (int r = 0; r < 4; r++) cz[r] *= alpha;
+
+        // ---------------- p exchange through the (now free) slot area
+        __syncwarp();
+        float *pex = reinterpret_cast<float *>(cur);
+        {
+            float *dst = pex + tig * kPexStride + 16 * gid + 4 * (gid >> 1);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; q4++)
+                *reinterpret_cast<float4 *>(dst + 4 * q4) =
+                    make_float4(sc[2 * q4][0], sc[2 * q4][1], sc[2 * q4 + 1][0], sc[2 * q4 + 1][1]);
+        }
+        __syncwarp();
+        float pv[32];                          // head hh, tokens 32tig .. 32tig+31
+        {
+            const float *src = pex + hh * kPexStride + 32 * tig + 4 * tig;
+#pragma unroll
+            for (int q4 = 0; q4 < 8; q4++) {
+                const float4 v = *reinterpret_cast<const float4 *>(src + 4 * q4);
+                pv[4 * q4] = v.x;
+                pv[4 * q4 + 1] = v.y;
+                pv[4 * q4 + 2] = v.z;
+                pv[4 * q4 + 3] = v.w;
+            }
+        }
+        // weights of value k-step j = 4u + f: tokens 16u+f, +8 (pair a) and
+        // 16u+f+4, +12 (pair b), scaled by 4^(3-f) to offset the code scaling
+        uint32_t ph[8][2], pl[8][2];
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            const int u = j >> 2, f = j & 3;
+            const float F = (float)(1 << (2 * (3 - f)));
+#pragma unroll
+            for (int r = 0; r < 2; r++) {
+                const float xa = pv[16 * u + f + 4 * r] * F, xb = pv[16 * u + f + 8 + 4 * r] * F;
+                const __half2 hi = __floats2half2_rn(xa, xb);
+                const float2 hf = __half22float2(hi);
+                ph[j][r] = h2u(hi);
+                pl[j][r] = h2u(__floats2half2_rn(xa - hf.x, xb - hf.y));
+            }
+        }
+
+        // ---------------- values, group by group
+#pragma unroll
+        for (int g = 0; g < kNG; g++) {
+            uint32_t bw[8][2];
+            {
+                const uint4 *vw4 = reinterpret_cast<const uint4 *>(vmeta + g * kT + 32 * tig);
+                uint32_t vw[32];
+#pragma unroll
+                for (int q4 = 0; q4 < 8; q4++) {
+                    const uint4 w = vw4[q4];
+                    vw[4 * q4] = w.x;
+                    vw[4 * q4 + 1] = w.y;
+                    vw[4 * q4 + 2] = w.z;
+                    vw[4 * q4 + 3] = w.w;
+                }
+#pragma unroll
+                for (int j = 0; j < 8; j++) {
+                    const int u = j >> 2, f = j & 3;
+#pragma unroll
+                    for (int r = 0; r < 2; r++) {
+                        const __half2 sp = u2h(__byte_perm(vw[16 * u + f + 4 * r], vw[16 * u + f + 8 + 4 * r], 0x5410));
+                        const __half2 P = u2h(ph[j][r]);
+                        const __half2 wh = __hmul2(P, sp);
+                        const __half2 res = __hfma2(P, sp, __hneg2(wh));
+                        const __half2 wl = __hfma2(u2h(pl[j][r]), sp, res);
+                        bw[j][r] = part ? h2u(wl) : h2u(wh);
+                    }
+                }
+            }
+#pragma unroll
+            for (int m2 = 0; m2 < 2; m2++) {
+                const int mt = 2 * g + m2;
+                const uint2 r0 = *reinterpret_cast<const uint2 *>(vcodes + (16 * mt + gid) * 32 + 8 * tig);
+                const uint2 r1 = *reinterpret_cast<const uint2 *>(vcodes + (16 * mt + gid + 8) * 32 + 8 * tig);
+                const uint32_t W0[2] = {r0.x, r0.y}, W1[2] = {r1.x, r1.y};
+                const uint32_t Y0[2] = {r0.x >> 8, r0.y >> 8}, Y1[2] = {r1.x >> 8, r1.y >> 8};
+#pragma unroll
+                for (int j = 0; j < 8; j++) {
+                    const int u = j >> 2, f = j & 3;
+                    const uint32_t m = 0x00030003u << (2 * f);
+                    mma16816(co[mt], W0[u] & m, W1[u] & m, Y0[u] & m, Y1[u] & m, bw[j][0], bw[j][1]);
+                }
+            }
+        }
+        // zero-point term: rows = groups (row gid holds group gid), times p
+        {
+            const uint4 *zw4 = reinterpret_cast<const uint4 *>(vmeta + (gid & 3) * kT + 32 * tig);
+            uint32_t zw[32];
+#pragma unroll
+            for (int q4 = 0; q4 < 8; q4++) {
+                const uint4 w = zw4[q4];
+                zw[4 * q4] = w.x;
+                zw[4 * q4 + 1] = w.y;
+                zw[4 * q4 + 2] = w.z;
+                zw[4 * q4 + 3] = w.w;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                const int u = j >> 2, f = j & 3;
+                const __half2 sc2 = __float2half2_rn(zmask / (float)(1 << (2 * (3 - f))));
+                uint32_t a[2];
+#pragma unroll
+                for (int r = 0; r < 2; r++)
+                    a[r] = h2u(__hmul2(u2h(__byte_perm(zw[16 * u + f + 4 * r], zw[16 * u + f + 8 + 4 * r], 0x7632)), sc2));
+                mma16816(cz, a[0], 0u, a[1], 0u, part ? pl[j][0] : ph[j][0], part ? pl[j][1] : ph[j][1]);
+            }
+        }
+        __syncwarp();
+    }
+
+    // ------------------------------------------------------------ merge
+    // per warp: head tig's max, sum and output; then across the 4 warps
+    float l_head = l_thr;
+    l_head += __shfl_xor_sync(0xffffffffu, l_head, 4);
+    l_head += __shfl_xor_sync(0xffffffffu, l_head, 8);
+    l_head += __shfl_xor_sync(0xffffffffu, l_head, 16);
+    float zsum[kNG];
+#pragma unroll
+    for (int g = 0; g < kNG; g++) {
+        const float v = cz[0] + cz[1];                   // valid in lanes with gid == group
+        zsum[g] = __shfl_sync(0xffffffffu, v, 4 * g + tig);
+    }
+    __syncthreads();                                     // stages are free now
+    float *mo = reinterpret_cast<float *>(sh.stage[0][0]);       // [warp][head][128]
+    float *mml = mo + kWarps * 4 * kD;                           // [warp][head][2]
+    constexpr float kCodeScale = 262144.f;                       // 2^18
+#pragma unroll
+    for (int mt = 0; mt < 8; mt++) {
+        const float z = zsum[mt >> 1];
+        mo[(warp * 4 + tig) * kD + 16 * mt + gid] = fmaf(co[mt][0] + co[mt][1], kCodeScale, z);
+        mo[(warp * 4 + tig) * kD + 16 * mt + gid + 8] = fmaf(co[mt][2] + co[mt][3], kCodeScale, z);
+    }
+    if (gid == 0) {
+        mml[(warp * 4 + tig) * 2] = m_run;
+        mml[(warp * 4 + tig) * 2 + 1] = l_head;
+    }
+    __syncthreads();
+    {
+        const int c = tid;
+#pragma unroll
+        for (int hl = 0; hl < 4; hl++) {
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < kWarps; w++) M = fmaxf(M, mml[(w * 4 + hl) * 2]);
+            float o = 0.f, L = 0.f;
+            if (M != -INFINITY) {
+#pragma unroll
+                for (int w = 0; w < kWarps; w++) {
+                    const float wt = exp2f(mml[(w * 4 + hl) * 2] - M);
+                    L = fmaf(wt, mml[(w * 4 + hl) * 2 + 1], L);
+                    o = fmaf(wt, mo[(w * 4 + hl) * kD + c], o);
+                }
+            }
+            const size_t row = (qrow0 + hl) * S + s;
+            part_o[row * kD + c] = o;
+            if (c == 0) part_ml[row] = make_float2(M, L);
+        }
+    }
+}
+
+}  // namespace
+
+int decode_mma_splits(int units, int nblk, int num_sms) {
+    int S = (2 * num_sms + units - 1) / units;
+    const int max_s = nblk / 4 > 0 ? nblk / 4 : 1;   // at least one page per warp
+    if (S > max_s) S = max_s;
+    return S < 1 ? 1 : S;
+}
+
+cudaError_t launch_decode_mma(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
+                              const float *qgsum, int k, float *part_o, float2 *part_ml, int S,
+                              cudaStream_t st) {
+    const size_t smem = sizeof(MmaShared);
+    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)S, (unsigned)c.n_kv_heads, (unsigned)c.batch);
+    decode_mma_kernel<<<grid, 128, smem, st>>>(static_cast<const uint8_t *>(c.pages), c.seq_len,
+                                               c.n_kv_heads, c.capacity / kT, Hq, idx, qsel, qgsum, k,
+                                               part_o, part_ml, S);
+    return cudaGetLastError();
+}
+
+size_t decode_mma_smem_bytes() { return sizeof(MmaShared); }
+
+}  // namespace kvq

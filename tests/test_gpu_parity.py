@@ -215,3 +215,35 @@ def test_bf16_comparator_matches_plain_attention():
     empty = kvq.bf16_decode_attn(to_dev(q, "bf16"), to_dev(case.K[:, :, :0], "bf16"),
                                  to_dev(case.V[:, :, :0], "bf16"))
     assert not empty.any()
+
+
+def test_decode_parity_sharp_attention():
+    """Queries scaled x8: most softmax weights are tiny, a few dominate."""
+    case = Case(W.workload("llama8b_b8_32k", batch=2), n_ctx=1500)
+    cache = case.gpu_cache()
+    q = (W.f32_from_bf16_bits(case.q(3)) * 8.0).astype(np.float32)
+    qb = W.bf16_bits_from_f32(q)
+    sel = kvq.select_channels(cache, to_dev(qb, "bf16"), dev64(case.Ai), 0.4)
+    out = kvq.decode_attn(cache, sel).cpu().numpy()
+    for b in range(2):
+        for h in range(8):
+            ref, _, _ = case.oracle_decode(qb, b, h, 0.4)
+            emax, emean = rel_errors(out[b, h * 4:(h + 1) * 4], ref)
+            assert emax <= TOL_MAX and emean <= TOL_MEAN, (b, h, emax)
+
+
+@pytest.mark.parametrize("name,units,sparsities", [
+    ("longctx_b1_128k", [(0, 0), (0, 5)], (0.4,)),
+    ("sweep_b32_16k", [(0, 0), (31, 7)], (0.0, 0.4, 0.6)),
+    ("llama8b_b8_32k", [(7, 3)], (0.4,)),
+])
+def test_full_size_sampled(name, units, sparsities):
+    """Full workload sizes in the benchmark's launch configuration: every
+    sequence and head runs on the GPU; sampled (sequence, KV head) units are
+    checked against the oracle (pages bit-exact, channels bit-exact, output
+    within tolerance)."""
+    case = Case(W.workload(name))
+    cache = case.gpu_cache()
+    _check_pages(case, cache, units=units)
+    for s in sparsities:
+        _decode_and_compare(case, cache, s, steps=(0,), units=units)
