@@ -266,32 +266,32 @@ def run_ours(args):
     q_pool = [dev_in(W.make_q(wl, i)) for i in range(n_pool)]
     kv_pool = [tuple(dev_in(t) for t in W.make_step_kv(wl, i)) for i in range(n_pool)]
     k = kvq.num_selected(wl.sparsity)
-    sel = kvq.alloc_selection(cache, Hq, k, dev)
-    out = torch.empty(B, Hq, 128, dtype=torch.float32, device=dev)
-    ws = kvq.alloc_workspace(kvq.decode_workspace_bytes(cache, Hq, k), dev)
+    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    step = kvq.DecodeStep(cache, A, Ai, wl.sparsity, Hq, tdt)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
-    def step(i, q, kn, vn, d0=None, d1=None):
-        kvq.append(cache, kn, vn, A)
-        kvq.select_channels(cache, q, Ai, wl.sparsity, out=sel)
-        if d0 is not None:
-            d0.record()
-        kvq.decode_attn(cache, sel, out=out, ws=ws)
-        if d1 is not None:
-            d1.record()
+    def stage(i):
+        step.q.copy_(q_pool[i % n_pool])
+        step.k_new.copy_(kv_pool[i % n_pool][0])
+        step.v_new.copy_(kv_pool[i % n_pool][1])
 
     launches_per_step = 5   # append + length advance, select, decode partial, merge
+    step.time_decode()
     length = wl.n_ctx
     for i in range(args.warmup):
-        step(i, q_pool[i % n_pool], *kv_pool[i % n_pool])
+        stage(i)
+        step.run()
         length += 1
+        if i == 0 and args.graph:
+            torch.cuda.synchronize(dev)
+            step.capture()
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
 
     E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    evs = [(E(), E(), E(), E()) for _ in range(args.steps)]
-    tokens = []
+    a, b_ = E(), E()
+    step_ms, dec_ms, alg_bytes, tokens = [], [], [], []
     uuid = None
     try:
         uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
@@ -300,19 +300,20 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     with ClockSampler(uuid) as clocks:
         for i in range(args.steps):
-            flush.fill_(i & 0xFF)
-            a, b_, d0, d1 = evs[i]
-            a.record()
             j = args.warmup + i
-            step(j, q_pool[j % n_pool], *kv_pool[j % n_pool], d0, d1)
+            stage(j)
+            flush.fill_(i & 0xFF)
+            a.record()
+            step.run()
             b_.record()
+            torch.cuda.synchronize(dev)          # untimed: lets each step's events be read
             length += 1
+            step_ms.append(a.elapsed_time(b_))
+            dec_ms.append(step.decode_events[0].elapsed_time(step.decode_events[1]))
+            alg_bytes.append(algorithmic_decode_bytes(wl, k, length))
             tokens.append(B * Hkv * length)
-        torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    step_ms = [a.elapsed_time(b_) for a, b_, _, _ in evs]
-    dec_ms = [d0.elapsed_time(d1) for _, _, d0, d1 in evs]
     total_ms = sum(step_ms)
     if world > 1:
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
@@ -330,32 +331,24 @@ def run_ours(args):
     # end to end through the Python binding with host buffers
     e2e = None
     if args.e2e:
-        pin = lambda x: torch.from_numpy(np.ascontiguousarray(x).view(  # noqa: E731
-            np.int16 if wl.dtype == "bf16" else np.float32)).pin_memory()
-        qh = [pin(W.make_q(wl, i)) for i in range(n_pool)]
-        kvh = [tuple(pin(t) for t in W.make_step_kv(wl, i)) for i in range(n_pool)]
-        q_dev = torch.empty_like(q_pool[0])
-        kn_dev, vn_dev = torch.empty_like(kv_pool[0][0]), torch.empty_like(kv_pool[0][1])
+        npdt = np.int16 if wl.dtype == "bf16" else np.float32
+        pin = lambda x: torch.from_numpy(np.ascontiguousarray(x).view(npdt)).pin_memory()  # noqa: E731
+        as_t = (lambda t: t.view(torch.bfloat16)) if wl.dtype == "bf16" else (lambda t: t)
+        qh = [as_t(pin(W.make_q(wl, i))) for i in range(n_pool)]
+        kvh = [tuple(as_t(pin(t)) for t in W.make_step_kv(wl, i)) for i in range(n_pool)]
         out_h = torch.empty(B, Hq, 128, dtype=torch.float32).pin_memory()
-        as_dev = (lambda t: t.view(torch.bfloat16)) if wl.dtype == "bf16" else (lambda t: t)
-        e_evs = [(E(), E()) for _ in range(args.steps)]
-        e_tok = []
+        e_tok, e_ms = [], 0.0
         torch.cuda.synchronize(dev)
         for i in range(args.steps):
             flush.fill_(i & 0xFF)
-            a, b_ = e_evs[i]
             a.record()
             j = i % n_pool
-            q_dev.view(torch.int16 if wl.dtype == "bf16" else torch.float32).copy_(qh[j], non_blocking=True)
-            kn_dev.view(torch.int16 if wl.dtype == "bf16" else torch.float32).copy_(kvh[j][0], non_blocking=True)
-            vn_dev.view(torch.int16 if wl.dtype == "bf16" else torch.float32).copy_(kvh[j][1], non_blocking=True)
-            step(i, as_dev(q_dev), as_dev(kn_dev), as_dev(vn_dev))
-            out_h.copy_(out, non_blocking=True)
+            step.run_host(qh[j], kvh[j][0], kvh[j][1], out_h)
             b_.record()
+            torch.cuda.synchronize(dev)
+            e_ms += a.elapsed_time(b_)
             length += 1
             e_tok.append(B * Hkv * length)
-        torch.cuda.synchronize(dev)
-        e_ms = sum(a.elapsed_time(b_) for a, b_ in e_evs)
         if world > 1:
             t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -407,6 +400,7 @@ def run_ours(args):
                      "kernel": "decode partial + merge (kvq_decode_attn)",
                      "peak_source": f"{peak_src} hbm_gbs", "traffic_note": traffic_note},
         "decode_ms": statistics.mean(dec_ms),
+        "step_launch": "cuda graph" if args.graph else "eager",
         "decode_alg_bytes": statistics.mean(alg_bytes),
         "prefill_ms": prefill_ms,
         "gpu_launches": launches_per_step * args.steps,
@@ -435,6 +429,8 @@ def main():
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-comparator", dest="comparator", action="store_false")
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="launch the step's kernels eagerly instead of replaying a CUDA graph")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -13,6 +13,8 @@
  *  - Every call is asynchronous on the given stream (NULL = legacy default
  *    stream).  A return of KVQ_OK means the work was validated and enqueued;
  *    results are ready when the stream reaches that point.
+ *  - Calls that use the same cache must be ordered on one stream (or by
+ *    events): they share its pages, lengths and status counters.
  *  - Argument errors are found on the host before anything is launched and
  *    reported as a negative status; nothing is enqueued then.  Conditions
  *    only the device can see (a sequence that would overflow its capacity)
@@ -82,8 +84,16 @@ typedef struct {
     int32_t capacity;     /* tokens per sequence, a positive multiple of 128 */
     void *pages;          /* kvq_cache_bytes() bytes, 256-byte aligned        */
     int32_t *seq_len;     /* [batch] tokens currently stored per sequence    */
-    uint32_t *status;     /* one word of KVQ_DEV_* flags                     */
+    uint32_t *status;     /* kvq_status_words() words, 4-byte aligned: word 0
+                             holds the KVQ_DEV_* flags, the rest are
+                             completion counters the calls use to finish a
+                             step in the same kernel; every call leaves them
+                             at zero (kvq_cache_init zeroes them)           */
 } kvq_cache;
+
+/* Words of the cache's status array: 1 + batch + batch * n_kv_heads
+ * (0 if an argument is below 1). */
+size_t kvq_status_words(int batch, int n_kv_heads);
 
 /* Bytes of one 128-token page for the given code width (0 if unsupported). */
 size_t kvq_page_bytes(int bits);
@@ -91,7 +101,7 @@ size_t kvq_page_bytes(int bits);
 /* Bytes of the whole page array of a cache (0 if the descriptor is invalid). */
 size_t kvq_cache_bytes(const kvq_cache *cache);
 
-/* Zero every page, every seq_len entry and the status word (stream-ordered).
+/* Zero every page, every seq_len entry and the status array (stream-ordered).
  * Returns KVQ_ERR_ARG / KVQ_ERR_SHAPE / KVQ_ERR_ALIGN on a bad descriptor. */
 int kvq_cache_init(const kvq_cache *cache, kvq_stream_t stream);
 
@@ -227,7 +237,7 @@ int kvq_decode_attn_static(const kvq_cache *cache, int n_q_heads, const int32_t 
                            const float *qsel, const float *qgsum, int k, float *out,
                            kvq_stream_t stream);
 
-/* Copy the device status word into *flags (synchronises the stream).
+/* Copy the device status flags (word 0) into *flags (synchronises the stream).
  * KVQ_ERR_ARG on null pointers, KVQ_ERR_CUDA on a failed copy. */
 int kvq_read_status(const kvq_cache *cache, uint32_t *flags, kvq_stream_t stream);
 

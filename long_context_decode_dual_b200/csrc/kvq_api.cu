@@ -58,6 +58,11 @@ const char *kvq_status_string(int s) {
     }
 }
 
+size_t kvq_status_words(int batch, int n_kv_heads) {
+    if (batch < 1 || n_kv_heads < 1) return 0;
+    return 1 + (size_t)batch + (size_t)batch * n_kv_heads;
+}
+
 size_t kvq_page_bytes(int bits) { return (bits == 2 || bits == 4) ? (size_t)page_bytes(bits) : 0; }
 
 size_t kvq_cache_bytes(const kvq_cache *c) {
@@ -72,7 +77,8 @@ int kvq_cache_init(const kvq_cache *c, kvq_stream_t stream) {
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e = cudaMemsetAsync(c->pages, 0, kvq_cache_bytes(c), s);
     if (e == cudaSuccess) e = cudaMemsetAsync(c->seq_len, 0, sizeof(int32_t) * c->batch, s);
-    if (e == cudaSuccess) e = cudaMemsetAsync(c->status, 0, sizeof(uint32_t), s);
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(c->status, 0, sizeof(uint32_t) * kvq_status_words(c->batch, c->n_kv_heads), s);
     return cuda_status(e);
 }
 

@@ -117,16 +117,34 @@ append_kernel(uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len,
     const int lane = j & 31;
     const int grp = j >> 5;             // quantization group (= warp)
 
-    // K'[t][j] = sum_c K[t][c] A[c][j], fma chain c = 0..127 from 0.0
+    // K'[t][j] = sum_c K[t][c] A[c][j], fma chain c = 0..127 from 0.0.  A full
+    // tile interleaves its kTile chains (A read once per c); a partial tile (a
+    // decode step appends one token) runs only the chains of its tokens.
     double acc[kTile];
 #pragma unroll
     for (int tt = 0; tt < kTile; tt++) acc[tt] = 0.0;
     const double *Ah = A + (size_t)h * kD * kD + j;
+    if (hi - lo == kTile) {
 #pragma unroll 4
-    for (int c = 0; c < kD; c++) {
-        const double a = __ldg(Ah + (size_t)c * kD);
+        for (int c = 0; c < kD; c++) {
+            const double a = __ldg(Ah + (size_t)c * kD);
 #pragma unroll
-        for (int tt = 0; tt < kTile; tt++) acc[tt] = fma(ks[tt][c], a, acc[tt]);
+            for (int tt = 0; tt < kTile; tt++) acc[tt] = fma(ks[tt][c], a, acc[tt]);
+        }
+    } else {
+#pragma unroll
+        for (int tt = 0; tt < kTile; tt++) {
+            if (first + tt < lo || first + tt >= hi) continue;     // uniform over the CTA
+            double a_reg[8];
+            double x = 0.0;
+            for (int c0 = 0; c0 < kD; c0 += 8) {
+#pragma unroll
+                for (int u = 0; u < 8; u++) a_reg[u] = __ldg(Ah + (size_t)(c0 + u) * kD);
+#pragma unroll
+                for (int u = 0; u < 8; u++) x = fma(ks[tt][c0 + u], a_reg[u], x);
+            }
+            acc[tt] = x;
+        }
     }
 
     uint8_t *page = pages + (((size_t)b * Hkv + h) * NB + (size_t)(first / kT)) * page_bytes(BITS);
@@ -145,6 +163,8 @@ append_kernel(uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len,
 #pragma unroll
     for (int tt = 0; tt < kTile; tt++) {
         uint16_t sb, zb;
+        codes[tt] = 0;
+        if (!(valid >> tt & 1u)) continue;                        // uniform over the CTA
         codes[tt] = quantize_lane<BITS>(acc[tt], j != 0, sb, zb);
         if (valid >> tt & 1u) {
             if (lane == 0) kmeta[grp * kT + t0 + tt] = (uint32_t)sb | ((uint32_t)zb << 16);
@@ -157,11 +177,91 @@ append_kernel(uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len,
 #pragma unroll
     for (int tt = 0; tt < kTile; tt++) {
         uint16_t sb, zb;
+        codes[tt] = 0;
+        if (!(valid >> tt & 1u)) continue;
         codes[tt] = quantize_lane<BITS>(vs[tt][j], true, sb, zb);
         if ((valid >> tt & 1u) && lane == 0)
             vmeta[grp * kT + t0 + tt] = (uint32_t)sb | ((uint32_t)zb << 16);
     }
     store_row<BITS>(page + off_vcodes(BITS) + (size_t)j * R + t0 * BITS / 8, codes, valid);
+}
+
+// Appends of a few tokens (a decode step adds one): one CTA per (sequence,
+// KV head) walks the new tokens in order, so code bytes shared by
+// neighbouring tokens are updated by one thread each.  A of the head is staged
+// in shared memory first (one cp.async burst instead of a DRAM round trip per
+// row of the fma chain).  The last CTA of a sequence to finish advances its
+// length, using the sequence's completion counter in the status array.
+constexpr int kSmallMax = 4;
+
+template <typename Tin, int BITS>
+__global__ void __launch_bounds__(128)
+append_small_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len,
+                    uint32_t *__restrict__ status, const Tin *__restrict__ K,
+                    const Tin *__restrict__ V, const double *__restrict__ A, int Hkv, int NB,
+                    int n_new, int capacity) {
+    constexpr int R = row_bytes(BITS);
+    constexpr int PER = 8 / BITS;
+    extern __shared__ __align__(16) double As[];          // [128][128]
+    __shared__ double ks[kSmallMax][kD];
+    __shared__ double vs[kSmallMax][kD];
+    __shared__ int s_len;
+
+    const int h = blockIdx.x, b = blockIdx.y, j = threadIdx.x;
+    const int lane = j & 31, grp = j >> 5;
+    const double *Ah = A + (size_t)h * kD * kD;
+    for (int e = j; e < kD * kD / 2; e += blockDim.x) cp_async16(As + 2 * e, Ah + 2 * e);
+    cp_async_commit();
+    const size_t in_base = ((size_t)b * Hkv + h) * (size_t)n_new;
+    for (int e = j; e < n_new * kD; e += blockDim.x) {
+        ks[e / kD][e % kD] = in_to_double(K[in_base * kD + e]);
+        vs[e / kD][e % kD] = in_to_double(V[in_base * kD + e]);
+    }
+    if (j == 0) s_len = seq_len[b];
+    cp_async_wait<0>();
+    __syncthreads();
+    const int len = s_len;
+    const bool ok = len >= 0 && len + n_new <= capacity;
+
+    if (ok) {
+        uint8_t *unit = pages + ((size_t)b * Hkv + h) * NB * (size_t)page_bytes(BITS);
+        for (int i = 0; i < n_new; i++) {
+            const int pos = len + i, t = pos % kT;
+            uint8_t *page = unit + (size_t)(pos / kT) * page_bytes(BITS);
+            double x = 0.0;
+#pragma unroll 8
+            for (int c = 0; c < kD; c++) x = fma(ks[i][c], As[c * kD + j], x);
+            const int byte = t / PER, sh = (t % PER) * BITS;
+            const uint8_t clear = (uint8_t)~(((1u << BITS) - 1u) << sh);
+            uint16_t sb, zb;
+            const uint32_t kc = quantize_lane<BITS>(x, j != 0, sb, zb);
+            if (lane == 0)
+                reinterpret_cast<uint32_t *>(page + off_kmeta(BITS))[grp * kT + t] = (uint32_t)sb | ((uint32_t)zb << 16);
+            if (j == 0) {
+                reinterpret_cast<uint16_t *>(page + off_ch0(BITS))[t] = __bfloat16_as_ushort(__double2bfloat16(x));
+            } else {
+                uint8_t *p = page + (size_t)j * R + byte;
+                *p = (uint8_t)((*p & clear) | (kc << sh));
+            }
+            const uint32_t vc = quantize_lane<BITS>(vs[i][j], true, sb, zb);
+            if (lane == 0)
+                reinterpret_cast<uint32_t *>(page + off_vmeta(BITS))[grp * kT + t] = (uint32_t)sb | ((uint32_t)zb << 16);
+            uint8_t *p = page + off_vcodes(BITS) + (size_t)j * R + byte;
+            *p = (uint8_t)((*p & clear) | (vc << sh));
+        }
+    } else if (j == 0) {
+        atomicOr(status, (uint32_t)KVQ_DEV_CAPACITY);
+    }
+
+    __syncthreads();
+    if (j == 0) {
+        __threadfence();
+        const unsigned prev = atomicAdd(status + 1 + b, 1u);
+        if (prev == (unsigned)Hkv - 1u) {          // every head of sequence b has read its length
+            if (ok) seq_len[b] = len + n_new;
+            atomicExch(status + 1 + b, 0u);
+        }
+    }
 }
 
 __global__ void advance_kernel(int32_t *seq_len, int B, int n_new, int capacity) {
@@ -176,6 +276,17 @@ template <typename Tin, int BITS>
 cudaError_t launch_append_t(const kvq_cache &c, const void *K, const void *V, int n_new,
                             const double *A, cudaStream_t st) {
     const int NB = c.capacity / kT;
+    if (n_new <= kSmallMax) {
+        constexpr int smem = kD * kD * (int)sizeof(double);
+        static std::atomic<uint64_t> done{0};
+        cudaError_t e = set_smem_once(append_small_kernel<Tin, BITS>, smem, done);
+        if (e != cudaSuccess) return e;
+        dim3 grid((unsigned)c.n_kv_heads, (unsigned)c.batch);
+        append_small_kernel<Tin, BITS><<<grid, 128, smem, st>>>(
+            static_cast<uint8_t *>(c.pages), c.seq_len, c.status, static_cast<const Tin *>(K),
+            static_cast<const Tin *>(V), A, c.n_kv_heads, NB, n_new, c.capacity);
+        return cudaGetLastError();
+    }
     dim3 grid((unsigned)((n_new + kTile - 1) / kTile + 1), (unsigned)c.n_kv_heads, (unsigned)c.batch);
     append_kernel<Tin, BITS><<<grid, 128, 0, st>>>(
         static_cast<uint8_t *>(c.pages), c.seq_len, c.status, static_cast<const Tin *>(K),

@@ -184,7 +184,8 @@ cudaError_t launch_bf16_t(const void *q, const void *K, const void *V, int B, in
                           float *part_o, float2 *part_ml, int S, cudaStream_t st) {
     const size_t smem = 4 * (size_t)kTileBytes + sizeof(float) * (G * kD + 2 * kTT * G + kTT * G + 2 * G + G * kD + G);
     auto fn = bf16_decode_kernel<G>;
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static std::atomic<uint64_t> done{0};
+    cudaError_t e = set_smem_once(fn, (int)smem, done);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)S, (unsigned)Hkv, (unsigned)B);
     fn<<<grid, 128, smem, st>>>(static_cast<const uint16_t *>(q), static_cast<const uint16_t *>(K),

@@ -6,28 +6,34 @@ namespace kvq {
 
 cudaError_t launch_decode_simt(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
                                const float *qgsum, int k, float *part_o, float2 *part_ml, int S,
-                               cudaStream_t st);
-cudaError_t launch_combine(int rows, const float *part_o, const float2 *part_ml, int S, float *out,
-                           cudaStream_t st);
+                               float *out, cudaStream_t st);
 cudaError_t launch_decode_mma(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
                               const float *qgsum, int k, float *part_o, float2 *part_ml, int S,
-                              cudaStream_t st);
+                              float *out, cudaStream_t st);
 int decode_mma_splits(int units, int nblk, int num_sms);
 
 // The tensor-core kernel covers INT2 codes with 4 query heads per KV head;
 // other shapes use the CUDA-core kernel.
 static bool use_mma(const kvq_cache &c, int Hq) { return c.bits == 2 && Hq == 4 * c.n_kv_heads; }
 
-// Splits per (sequence, KV head): enough CTAs for about four per SM, at
-// least two pages per split, at most one split per page of capacity.
+// Splits per (sequence, KV head): enough CTAs to fill the SMs, at least two
+// pages per split, and at most kMaxSplits (the merge keeps two floats per
+// split and head in the kernels' staging memory).
+constexpr int kMaxSplits = 256;
+
 int decode_splits(const kvq_cache &c, int Hq, int k, int num_sms) {
     (void)k;
     const int units = c.batch * c.n_kv_heads;
     const int nblk = c.capacity / kT;
-    if (use_mma(c, Hq)) return decode_mma_splits(units, nblk, num_sms);
-    int S = (4 * num_sms + units - 1) / units;
-    const int max_s = (nblk + 1) / 2 > 0 ? (nblk + 1) / 2 : 1;
-    if (S > max_s) S = max_s;
+    int S;
+    if (use_mma(c, Hq)) {
+        S = decode_mma_splits(units, nblk, num_sms);
+    } else {
+        S = (4 * num_sms + units - 1) / units;
+        const int max_s = (nblk + 1) / 2 > 0 ? (nblk + 1) / 2 : 1;
+        if (S > max_s) S = max_s;
+    }
+    if (S > kMaxSplits) S = kMaxSplits;
     return S < 1 ? 1 : S;
 }
 
@@ -39,10 +45,9 @@ cudaError_t launch_decode(const kvq_cache &c, int Hq, const int32_t *idx, const 
                           const float *qgsum, int k, float *out, void *ws, int S, cudaStream_t st) {
     float *part_o = static_cast<float *>(ws);
     float2 *part_ml = reinterpret_cast<float2 *>(part_o + (size_t)c.batch * Hq * S * kD);
-    cudaError_t e = use_mma(c, Hq) ? launch_decode_mma(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, st)
-                                   : launch_decode_simt(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, st);
-    if (e != cudaSuccess) return e;
-    return launch_combine(c.batch * Hq, part_o, part_ml, S, out, st);
+    // one launch: the last CTA of each (sequence, KV head) merges the splits
+    return use_mma(c, Hq) ? launch_decode_mma(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, st)
+                          : launch_decode_simt(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, st);
 }
 
 }  // namespace kvq

@@ -73,7 +73,8 @@ __global__ void __launch_bounds__(128, 2)
 decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len, int Hkv,
                   int NB, int Hq, const int32_t *__restrict__ idx, const float *__restrict__ qsel,
                   const float *__restrict__ qgsum, int k, float *__restrict__ part_o,
-                  float2 *__restrict__ part_ml, int S) {
+                  float2 *__restrict__ part_ml, int S, float *__restrict__ out,
+                  uint32_t *__restrict__ counters) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     MmaShared &sh = *reinterpret_cast<MmaShared *>(smem_raw);
 
@@ -442,6 +443,8 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
             if (c == 0) part_ml[row] = make_float2(M, L);
         }
     }
+    merge_unit_if_last<4>(part_o, part_ml, S, qrow0, out, counters + unit,
+                          reinterpret_cast<float *>(sh.stage[1][0]));
 }
 
 }  // namespace
@@ -455,14 +458,15 @@ int decode_mma_splits(int units, int nblk, int num_sms) {
 
 cudaError_t launch_decode_mma(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
                               const float *qgsum, int k, float *part_o, float2 *part_ml, int S,
-                              cudaStream_t st) {
+                              float *out, cudaStream_t st) {
     const size_t smem = sizeof(MmaShared);
-    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static std::atomic<uint64_t> done{0};
+    cudaError_t e = set_smem_once(decode_mma_kernel, (int)smem, done);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)S, (unsigned)c.n_kv_heads, (unsigned)c.batch);
     decode_mma_kernel<<<grid, 128, smem, st>>>(static_cast<const uint8_t *>(c.pages), c.seq_len,
                                                c.n_kv_heads, c.capacity / kT, Hq, idx, qsel, qgsum, k,
-                                               part_o, part_ml, S);
+                                               part_o, part_ml, S, out, unit_counter(c, 0, 0));
     return cudaGetLastError();
 }
 

@@ -49,7 +49,8 @@ __global__ void __launch_bounds__(128)
 decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len, int Hkv,
                    int NB, int Hq, const int32_t *__restrict__ idx, const float *__restrict__ qsel,
                    const float *__restrict__ qgsum, int k, float *__restrict__ part_o,
-                   float2 *__restrict__ part_ml, int S) {
+                   float2 *__restrict__ part_ml, int S, float *__restrict__ out,
+                   uint32_t *__restrict__ counters) {
     constexpr int R = row_bytes(BITS);
     constexpr int FIX = fixed_bytes(BITS);
     constexpr int PER = 8 / BITS;
@@ -211,20 +212,25 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
         part_o[row * kD + tid] = o_acc[hl];
         if (tid == 0) part_ml[row] = make_float2(m_run[hl], l_run[hl]);
     }
+    merge_unit_if_last<G>(part_o, part_ml, S, (size_t)b * Hq + (size_t)h * G, out, counters + unit,
+                          reinterpret_cast<float *>(smem));
 }
 
 template <int BITS, int G>
 cudaError_t launch_simt_t(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
-                          const float *qgsum, int k, float *part_o, float2 *part_ml, int S,
+                          const float *qgsum, int k, float *part_o, float2 *part_ml, int S, float *out,
                           cudaStream_t st) {
     const int stage_bytes = (k - 1) * row_bytes(BITS) + fixed_bytes(BITS);
     const size_t smem = (size_t)2 * stage_bytes + SimtSmem<G>::extra;
+    constexpr int kMaxSmem = 2 * (127 * row_bytes(BITS) + fixed_bytes(BITS)) + SimtSmem<G>::extra;
+    static std::atomic<uint64_t> done{0};
     auto fn = decode_simt_kernel<BITS, G>;
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_smem_once(fn, kMaxSmem, done);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)S, (unsigned)c.n_kv_heads, (unsigned)c.batch);
     fn<<<grid, 128, smem, st>>>(static_cast<const uint8_t *>(c.pages), c.seq_len, c.n_kv_heads,
-                                c.capacity / kT, Hq, idx, qsel, qgsum, k, part_o, part_ml, S);
+                                c.capacity / kT, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out,
+                                unit_counter(c, 0, 0));
     return cudaGetLastError();
 }
 
@@ -253,10 +259,10 @@ combine_kernel(const float *__restrict__ part_o, const float2 *__restrict__ part
 
 cudaError_t launch_decode_simt(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
                                const float *qgsum, int k, float *part_o, float2 *part_ml, int S,
-                               cudaStream_t st) {
+                               float *out, cudaStream_t st) {
     const int g = Hq / c.n_kv_heads;
 #define KVQ_SIMT_CASE(BITS, G) \
-    if (c.bits == BITS && g == G) return launch_simt_t<BITS, G>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, st);
+    if (c.bits == BITS && g == G) return launch_simt_t<BITS, G>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, st);
     KVQ_SIMT_CASE(2, 1) KVQ_SIMT_CASE(2, 2) KVQ_SIMT_CASE(2, 4) KVQ_SIMT_CASE(2, 8)
     KVQ_SIMT_CASE(4, 1) KVQ_SIMT_CASE(4, 2) KVQ_SIMT_CASE(4, 4) KVQ_SIMT_CASE(4, 8)
 #undef KVQ_SIMT_CASE

@@ -7,6 +7,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "kvq.h"
 
 namespace kvq {
@@ -48,10 +50,101 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
 
-// ------------------------------------------------------------ split plan
-struct SplitPlan {
-    int n_splits;
-};
+// ------------------------------------------------------------ launch set-up
+// Raise a kernel's dynamic shared memory limit to `bytes` once per device and
+// kernel instance, so that later launches (including those recorded into a
+// CUDA graph) make no attribute calls.  `bytes` must be the instance's maximum.
+template <typename Kernel>
+cudaError_t set_smem_once(Kernel *fn, int bytes, std::atomic<uint64_t> &done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_release);
+    return e;
+}
+
+// ------------------------------------------------------------ split merge
+// Each CTA of a (sequence, KV head) unit writes one partial (running max m,
+// sum l and output o per query head) for its split of the context.  The last
+// CTA to arrive -- found with the unit's completion counter, which it resets
+// -- merges them: out = sum_s e^{m_s - M} o_s / sum_s e^{m_s - M} l_s, the one
+// softmax over the whole context (Dual-QK §3.4).  Nothing waits: the other
+// CTAs simply exit.  Called by every thread of a 128-thread CTA; `scratch` is
+// shared memory for 2 * G * S + G floats.  The (m, l) pairs are read in one
+// parallel pass and turned into per-split weights, then each thread sums G
+// consecutive outputs over the splits with independent vector loads.
+template <int G>
+__device__ __forceinline__ void merge_unit_if_last(const float *part_o, const float2 *part_ml, int S,
+                                                   size_t qrow0, float *out, uint32_t *counter,
+                                                   float *scratch) {
+    __shared__ int s_last;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const unsigned prev = atomicAdd(counter, 1u);
+        s_last = prev == (unsigned)S - 1u;
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    float *wm = scratch;             // [G][S] max, then weight
+    float *wl = scratch + G * S;     // [G][S] sum
+    float *inv = wl + G * S;         // [G] 1 / total sum
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    for (int e = t; e < G * S; e += blockDim.x) {
+        const float2 v = __ldcg(part_ml + qrow0 * S + e);     // rows qrow0.. are contiguous
+        wm[e] = v.x;
+        wl[e] = v.y;
+    }
+    __syncthreads();
+    for (int hl = warp; hl < G; hl += blockDim.x / 32) {
+        float M = -INFINITY;
+        for (int s = lane; s < S; s += 32) M = fmaxf(M, wm[hl * S + s]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float L = 0.f;
+        for (int s = lane; s < S; s += 32) {
+            const float w = (M == -INFINITY) ? 0.f : exp2f(wm[hl * S + s] - M);
+            wm[hl * S + s] = w;
+            L = fmaf(w, wl[hl * S + s], L);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        if (lane == 0) inv[hl] = L > 0.f ? 1.f / L : 0.f;
+    }
+    __syncthreads();
+    // thread t owns outputs [t*G, t*G + G) of the unit's [G][128] block
+    const int hl = (t * G) / kD, c0 = (t * G) % kD;
+    float acc[G];
+#pragma unroll
+    for (int u = 0; u < G; u++) acc[u] = 0.f;
+    const float *po = part_o + ((qrow0 + hl) * S) * kD + c0;
+#pragma unroll 8
+    for (int s = 0; s < S; s++) {
+        const float w = wm[hl * S + s];
+        if constexpr (G % 4 == 0) {
+#pragma unroll
+            for (int u = 0; u < G; u += 4) {
+                const float4 v = __ldcg(reinterpret_cast<const float4 *>(po + (size_t)s * kD + u));
+                acc[u] = fmaf(w, v.x, acc[u]);
+                acc[u + 1] = fmaf(w, v.y, acc[u + 1]);
+                acc[u + 2] = fmaf(w, v.z, acc[u + 2]);
+                acc[u + 3] = fmaf(w, v.w, acc[u + 3]);
+            }
+        } else {
+#pragma unroll
+            for (int u = 0; u < G; u++) acc[u] = fmaf(w, __ldcg(po + (size_t)s * kD + u), acc[u]);
+        }
+    }
+    const float r = inv[hl];
+#pragma unroll
+    for (int u = 0; u < G; u++) out[(qrow0 + hl) * kD + c0 + u] = acc[u] * r;
+    __syncthreads();
+    if (t == 0) atomicExch(counter, 0u);
+}
 
 }  // namespace kvq
 
@@ -66,6 +159,10 @@ size_t decode_ws_bytes(const kvq_cache &c, int Hq, int n_splits);
 cudaError_t launch_decode(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
                           const float *qgsum, int k, float *out, void *ws, int n_splits,
                           cudaStream_t st);
+// completion counter of unit (b, h) in the cache's status array
+inline uint32_t *unit_counter(const kvq_cache &c, int b, int h) {
+    return c.status + 1 + c.batch + (size_t)b * c.n_kv_heads + h;
+}
 int bf16_splits(int B, int Hkv, int N, int num_sms);
 size_t bf16_ws_bytes(int B, int Hq, int n_splits);
 cudaError_t launch_bf16_decode(const void *q, const void *K, const void *V, int B, int Hq, int Hkv,

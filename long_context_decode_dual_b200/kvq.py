@@ -48,7 +48,7 @@ class CacheDesc(ctypes.Structure):
 _lib = None
 
 EXPORTS = (
-    "kvq_page_bytes", "kvq_cache_bytes", "kvq_cache_init", "kvq_append", "kvq_num_selected",
+    "kvq_status_words", "kvq_page_bytes", "kvq_cache_bytes", "kvq_cache_init", "kvq_append", "kvq_num_selected",
     "kvq_select_channels", "kvq_decode_workspace", "kvq_decode_attn",
     "kvq_bf16_decode_workspace", "kvq_bf16_decode_attn", "kvq_read_status",
     "kvq_status_string", "kvq_version", "kvq_decode_static_scratch_bytes",
@@ -67,6 +67,7 @@ def lib() -> ctypes.CDLL:
         P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
         C = ctypes.POINTER(CacheDesc)
         sig = {
+            "kvq_status_words": (S, [I, I]),
             "kvq_page_bytes": (S, [I]),
             "kvq_cache_bytes": (S, [C]),
             "kvq_cache_init": (I, [C, P]),
@@ -159,7 +160,8 @@ def new_cache(batch: int, n_kv_heads: int, capacity: int, bits: int = 2,
         raise KvqError("kvq_cache_bytes", -2)
     pages = torch.empty(nbytes, dtype=torch.uint8, device=device)
     seq_len = torch.empty(batch, dtype=torch.int32, device=device)
-    status = torch.empty(1, dtype=torch.int32, device=device)
+    status = torch.empty(int(lib().kvq_status_words(batch, n_kv_heads)), dtype=torch.int32,
+                         device=device)
     c = KVCache(batch, n_kv_heads, capacity, bits, pages, seq_len, status)
     _check("kvq_cache_init", lib().kvq_cache_init(ctypes.byref(c.desc), _stream(stream)))
     return c
@@ -275,3 +277,77 @@ def read_status(cache: KVCache, stream=None) -> int:
     _check("kvq_read_status", lib().kvq_read_status(ctypes.byref(cache.desc), ctypes.byref(flags),
                                                     _stream(stream)))
     return int(flags.value)
+
+
+class DecodeStep:
+    """One decode step of the path -- append the new token, select channels,
+    decode -- on static device buffers, replayable as a CUDA graph.
+
+    Fill ``q`` [B][Hq][128] and ``k_new`` / ``v_new`` [B][Hkv][1][128] (f32 or
+    bf16, the dtype given), call :meth:`run`; the result is in ``out``
+    [B][Hq][128] f32.  :meth:`capture` records the three calls once (after at
+    least one eager :meth:`run`, so every kernel is loaded); later runs replay
+    the graph.  :meth:`run_host` copies the inputs from (pinned) host tensors
+    and the output back, around the same step.
+    """
+
+    def __init__(self, cache: KVCache, A: torch.Tensor, Ainvt: torch.Tensor, sparsity: float,
+                 n_q_heads: int, dtype: torch.dtype = torch.bfloat16):
+        dev = cache.pages.device
+        B, Hkv = cache.batch, cache.n_kv_heads
+        self.cache, self.A, self.Ainvt, self.sparsity = cache, A, Ainvt, float(sparsity)
+        self.q = torch.zeros(B, n_q_heads, HEAD_DIM, dtype=dtype, device=dev)
+        self.k_new = torch.zeros(B, Hkv, 1, HEAD_DIM, dtype=dtype, device=dev)
+        self.v_new = torch.zeros(B, Hkv, 1, HEAD_DIM, dtype=dtype, device=dev)
+        self.k = num_selected(sparsity)
+        self.sel = alloc_selection(cache, n_q_heads, self.k, dev)
+        self.out = torch.empty(B, n_q_heads, HEAD_DIM, dtype=torch.float32, device=dev)
+        self.ws = alloc_workspace(decode_workspace_bytes(cache, n_q_heads, self.k), dev)
+        self.graph = None
+        self.decode_events = None      # optional (start, end) events around the decode call
+
+    def _pre(self):
+        append(self.cache, self.k_new, self.v_new, self.A)
+        select_channels(self.cache, self.q, self.Ainvt, self.sparsity, out=self.sel)
+
+    def _decode(self):
+        decode_attn(self.cache, self.sel, out=self.out, ws=self.ws)
+
+    def time_decode(self) -> None:
+        """Record timing events around the decode call of every later run."""
+        self.decode_events = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+
+    def capture(self) -> None:
+        """Record the step as two CUDA graphs (append + select, decode); the
+        decode timing events, if any, are recorded between the two replays."""
+        pre, dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(pre):
+            self._pre()
+        with torch.cuda.graph(dec):
+            self._decode()
+        self.graph = (pre, dec)
+
+    def run(self) -> torch.Tensor:
+        ev = self.decode_events
+        if self.graph is not None:
+            self.graph[0].replay()
+        else:
+            self._pre()
+        if ev is not None:
+            ev[0].record()
+        if self.graph is not None:
+            self.graph[1].replay()
+        else:
+            self._decode()
+        if ev is not None:
+            ev[1].record()
+        return self.out
+
+    def run_host(self, q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tensor,
+                 out_host: torch.Tensor) -> torch.Tensor:
+        self.q.copy_(q_host, non_blocking=True)
+        self.k_new.copy_(k_host, non_blocking=True)
+        self.v_new.copy_(v_host, non_blocking=True)
+        self.run()
+        out_host.copy_(self.out, non_blocking=True)
+        return out_host

@@ -247,3 +247,49 @@ def test_full_size_sampled(name, units, sparsities):
     _check_pages(case, cache, units=units)
     for s in sparsities:
         _decode_and_compare(case, cache, s, steps=(0,), units=units)
+
+
+def test_decode_step_graph_replay_matches_eager():
+    """The captured step (append -> select -> decode as one CUDA graph) gives
+    the same bytes and outputs as the same calls launched one by one."""
+    wl = W.workload("llama8b_b8_32k", batch=2)
+    case = Case(wl, n_ctx=400)
+    A, Ai = dev64(case.A), dev64(case.Ai)
+    steps = [kvq.DecodeStep(case.gpu_cache(), A, Ai, 0.4, wl.n_q_heads) for _ in range(2)]
+    outs = [[], []]
+    for i in range(4):
+        kn, vn = W.make_step_kv(wl, i)
+        q = case.q(i)
+        for m, st in enumerate(steps):
+            st.q.copy_(to_dev(q, "bf16"))
+            st.k_new.copy_(to_dev(kn, "bf16"))
+            st.v_new.copy_(to_dev(vn, "bf16"))
+            outs[m].append(st.run().clone())
+            if m == 1 and i == 0:
+                torch.cuda.synchronize()
+                st.capture()
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+    assert torch.equal(steps[0].cache.pages, steps[1].cache.pages)
+    assert steps[1].cache.seq_len.tolist() == [404, 404]
+
+
+def test_small_append_capacity_and_lengths():
+    """Decode-sized appends (one token) advance every sequence's length once
+    per call, and stop at capacity with the flag set and the pages intact."""
+    wl = W.workload("llama8b_b8_32k", batch=3)
+    case = Case(wl, n_ctx=254, capacity=256)
+    cache = case.gpu_cache()
+    A = dev64(case.A)
+    for i in range(2):
+        kn, vn = W.make_step_kv(wl, i)
+        kvq.append(cache, to_dev(kn, "bf16"), to_dev(vn, "bf16"), A)
+    assert cache.seq_len.tolist() == [256, 256, 256] and kvq.read_status(cache) == 0
+    before = cache.pages.clone()
+    kn, vn = W.make_step_kv(wl, 5)
+    kvq.append(cache, to_dev(kn, "bf16"), to_dev(vn, "bf16"), A)
+    assert kvq.read_status(cache) & kvq.KVQ_DEV_CAPACITY
+    assert cache.seq_len.tolist() == [256, 256, 256]
+    assert torch.equal(before, cache.pages)
+    # the counters the calls use are back at zero
+    assert not cache.status[1:].any()
