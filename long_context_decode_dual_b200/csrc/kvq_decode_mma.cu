@@ -21,25 +21,30 @@
 // in fp32 after the score MMAs, folded into the weights before the value
 // MMAs, and the value zero-point term sum_t p(t) z(t) is one more MMA.
 //
-// One CTA = one (sequence, KV head, split of the context), four warps; each
-// warp owns whole pages (its own online softmax) with a two-stage cp.async
-// ring in shared memory.  Selected key rows land in fixed slots: group g owns
-// slots 32g..32g+31, filled in ascending channel order, so every MMA k-step
-// (16 slots) lies inside one group and its scale applies to the whole step.
+// Work split: one CTA = one (sequence, KV head, split of the context), eight
+// warps in four pairs.  A pair processes one 128-token page at a time from a
+// two-stage cp.async ring; warp w of the pair takes half w of every 16-token
+// word of the page (64 tokens) and keeps its own online softmax.  Selected key
+// rows land in fixed slots: group g owns slots 32g..32g+31, filled in
+// ascending channel order, so every MMA k-step (16 slots) lies inside one
+// group and its scale applies to the whole step.
 #include "kvq_internal.cuh"
 
 namespace kvq {
 namespace {
 
-constexpr int kWarps = 4;
+constexpr int kPairs = 4;
+constexpr int kThreads = 64 * kPairs;
 constexpr int kSlotBytes = 128 * 32;              // 4 groups x 32 slots x 32 B
 constexpr int kFixBytes = fixed_bytes(2);         // value codes, ch0, metadata
 constexpr int kStageBytes = kSlotBytes + kFixBytes;
 constexpr int kMaxTasks = 2 * 127;                // 16-byte copies of key rows
-constexpr int kPexStride = 164;                   // floats per head in the p exchange
+// chunk (16 B) offsets inside the fixed part of a staged page
+constexpr int kVmetaChunk = (4096 + 256 + 2048) / 16;   // 400
+constexpr int kFixChunks = kFixBytes / 16;              // 528
 
 struct __align__(16) MmaShared {
-    uint8_t stage[kWarps][2][kStageBytes];
+    uint8_t stage[kPairs][2][kStageBytes];
     uint32_t task[kMaxTasks];          // src offset | dst offset << 16 (bytes)
     float q[4][kD];                    // qsel of the 4 heads, by selected position
     float qg[4][kNG];
@@ -57,6 +62,10 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ void pair_sync(int pair) {
+    asm volatile("bar.sync %0, 64;\n" ::"r"(pair + 1) : "memory");
+}
+
 __device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
 __device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2 *>(&u); }
 __device__ __forceinline__ float lo_f16(uint32_t w) { return __half2float(__ushort_as_half((uint16_t)(w & 0xffffu))); }
@@ -69,7 +78,18 @@ __device__ __forceinline__ uint16_t f16_part(float x, int part) {
     return __half_as_ushort(__float2half_rn(x - __half2float(hi)));
 }
 
-__global__ void __launch_bounds__(128, 2)
+// Value metadata chunks (4 tokens each) are stored swizzled within each
+// group's 32 chunks so that the four thread columns of a warp, which read
+// chunks 8 apart, hit different banks.
+__device__ __forceinline__ int vmeta_chunk(int c) { return c ^ ((c >> 3) & 7); }
+
+// position of local token l (0..63) in a warp's softmax-weight exchange
+// buffer, and the start of head h's block (skews keep both access patterns
+// free of bank conflicts)
+__device__ __forceinline__ int pex_pos(int l) { return l + 4 * (l >> 4); }
+__device__ __forceinline__ int pex_head(int h) { return 96 * h + ((h & 1) ? 4 : 0) + ((h & 2) ? 16 : 0); }
+
+__global__ void __launch_bounds__(kThreads, 2)
 decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len, int Hkv,
                   int NB, int Hq, const int32_t *__restrict__ idx, const float *__restrict__ qsel,
                   const float *__restrict__ qgsum, int k, float *__restrict__ part_o,
@@ -80,6 +100,7 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
 
     const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int pair = warp >> 1, half = warp & 1, pt = tid & 63;   // pt: thread within the pair
     const int gid = lane >> 2, tig = lane & 3;
     const size_t unit = (size_t)b * Hkv + h;
     const size_t qrow0 = (size_t)b * Hq + (size_t)h * 4;
@@ -88,12 +109,12 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
     // The selected list is ascending, so each group's channels sit in one
     // contiguous run of positions; a channel's slot is 32g + (its position -
     // the first position of its group).
-    for (int e = tid; e < 4 * k; e += 128) {
+    for (int e = tid; e < 4 * k; e += kThreads) {
         const int hl = e / k, i = e % k;
         sh.q[hl][i] = qsel[(qrow0 + hl) * k + i];
     }
     if (tid < 4 * kNG) sh.qg[tid / kNG][tid % kNG] = qgsum[qrow0 * kNG + tid];
-    for (int i = tid; i < kD; i += 128) sh.slot_pos[i] = -1;
+    if (tid < kD) sh.slot_pos[tid] = -1;
     if (tid < kNG) sh.nks[tid] = 0;
     __syncthreads();
     const int32_t *sel = idx + unit * k;
@@ -147,15 +168,22 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
     const int blk0 = s * bps;
     const int blk1 = min(nblk, blk0 + bps);
 
+    // the pair's 64 threads copy one page into a stage
     auto issue = [&](uint8_t *dst, int blk) {
         const uint8_t *src = pages + (unit * NB + (size_t)blk) * page_bytes(2);
-        for (int e = lane; e < n_tasks; e += 32) {
+        for (int e = pt; e < n_tasks; e += 64) {
             const uint32_t t = sh.task[e];
             cp_async16(dst + (t >> 16), src + (t & 0xffffu));
         }
-#pragma unroll 4
-        for (int e = lane; e < kFixBytes / 16; e += 32)
-            cp_async16(dst + kSlotBytes + 16 * e, src + off_vcodes(2) + 16 * e);
+#pragma unroll 3
+        for (int e = pt; e < kFixChunks; e += 64) {
+            int d = e;
+            if (e >= kVmetaChunk) {
+                const int c = e - kVmetaChunk;
+                d = kVmetaChunk + (c & ~31) + vmeta_chunk(c & 31);
+            }
+            cp_async16(dst + kSlotBytes + 16 * d, src + off_vcodes(2) + 16 * e);
+        }
         cp_async_commit();
     };
 
@@ -170,40 +198,38 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
 #pragma unroll
     for (int r = 0; r < 4; r++) cz[r] = 0.f;
 
-    const uint32_t lane_row_off = 4u * gid;          // word gid of a 32-byte code row
+    const uint32_t lane_row_off = 4u * gid;                  // word gid of a 32-byte code row
+    const uint32_t half_sel = half ? 0x7632u : 0x5410u;      // this warp's 16-bit half of a word
+    const uint32_t vx_sel = half ? 0x4332u : 0x4110u;        // {half, high byte of half}
     const float zmask = gid < 4 ? 1.f : 0.f;
 
     int it = 0;
-    const int first = blk0 + warp;
-    if (first < blk1) issue(sh.stage[warp][0], first);
-    for (int pg = first; pg < blk1; pg += kWarps, it++) {
-        uint8_t *cur = sh.stage[warp][it & 1];
-        if (pg + kWarps < blk1) {
-            issue(sh.stage[warp][(it + 1) & 1], pg + kWarps);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
-        }
-        __syncwarp();
+    const int first = blk0 + pair;
+    if (first < blk1) issue(sh.stage[pair][0], first);
+    for (int pg = first; pg < blk1; pg += kPairs, it++) {
+        uint8_t *cur = sh.stage[pair][it & 1];
+        cp_async_wait<0>();
+        pair_sync(pair);                                     // page pg staged; other stage free
+        if (pg + kPairs < blk1) issue(sh.stage[pair][(it + 1) & 1], pg + kPairs);
 
         const uint8_t *vcodes = cur + kSlotBytes;
         const uint32_t *ch0w = reinterpret_cast<const uint32_t *>(vcodes + 128 * 32);
         const uint32_t *kmeta = reinterpret_cast<const uint32_t *>(vcodes + 128 * 32 + 256);
         const uint32_t *vmeta = kmeta + kNG * kT;
 
-        // ---------------- scores: thread holds tokens 16gid + 2i (+1), head tig
-        float sc[8][2], zt[8][2];
+        // ---------------- scores: tokens 16gid + 8half + 2i + r, head tig
+        float sc[4][2], zt[4][2];
 #pragma unroll
-        for (int i = 0; i < 8; i++) {
+        for (int i = 0; i < 4; i++) {
             sc[i][0] = sc[i][1] = 0.f;
             zt[i][0] = zt[i][1] = 0.f;
         }
 #pragma unroll
         for (int g = 0; g < kNG; g++) {
             if (nks[g] == 0) continue;
-            float C[8][4];
+            float C[4][4];
 #pragma unroll
-            for (int i = 0; i < 8; i++) C[i][0] = C[i][1] = C[i][2] = C[i][3] = 0.f;
+            for (int i = 0; i < 4; i++) C[i][0] = C[i][1] = C[i][2] = C[i][3] = 0.f;
 #pragma unroll
             for (int j = 0; j < 2; j++) {
                 if (j >= nks[g]) break;
@@ -212,25 +238,22 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
                 const uint32_t Wb = *reinterpret_cast<const uint32_t *>(sb + 4 * 32);
                 const uint32_t Wc = *reinterpret_cast<const uint32_t *>(sb + 8 * 32);
                 const uint32_t Wd = *reinterpret_cast<const uint32_t *>(sb + 12 * 32);
-                const uint32_t Xab[2] = {__byte_perm(Wa, Wb, 0x5410), __byte_perm(Wa, Wb, 0x7632)};
-                const uint32_t Xcd[2] = {__byte_perm(Wc, Wd, 0x5410), __byte_perm(Wc, Wd, 0x7632)};
-                const uint32_t Yab[2] = {Xab[0] >> 8, Xab[1] >> 8};
-                const uint32_t Ycd[2] = {Xcd[0] >> 8, Xcd[1] >> 8};
+                const uint32_t Xab = __byte_perm(Wa, Wb, half_sel), Xcd = __byte_perm(Wc, Wd, half_sel);
+                const uint32_t Yab = Xab >> 8, Ycd = Xcd >> 8;
                 const uint32_t b0 = bq[2 * g + j][0], b1 = bq[2 * g + j][1];
 #pragma unroll
-                for (int i = 0; i < 8; i++) {
-                    const int hf = i >> 2;
-                    const uint32_t x1 = (i & 2) ? Yab[hf] : Xab[hf];
-                    const uint32_t x2 = (i & 2) ? Ycd[hf] : Xcd[hf];
+                for (int i = 0; i < 4; i++) {
+                    const uint32_t x1 = (i & 2) ? Yab : Xab;
+                    const uint32_t x2 = (i & 2) ? Ycd : Xcd;
                     const uint32_t m0 = 0x00030003u << (4 * (i & 1));
                     const uint32_t m1 = m0 << 2;
                     mma16816(C[i], x1 & m0, x1 & m1, x2 & m0, x2 & m1, b0, b1);
                 }
             }
-            // scale and zero-point of group g for the thread's 16 tokens
-            const uint4 *kw4 = reinterpret_cast<const uint4 *>(kmeta + g * kT + 16 * gid);
+            // scale and zero-point of group g for the thread's 8 tokens
+            const uint4 *kw4 = reinterpret_cast<const uint4 *>(kmeta + g * kT + 16 * gid + 8 * half);
 #pragma unroll
-            for (int q4 = 0; q4 < 4; q4++) {
+            for (int q4 = 0; q4 < 2; q4++) {
                 const uint4 w = kw4[q4];
                 const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -242,19 +265,16 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
             }
         }
         // full scores (base-2 domain), masked beyond the sequence
-        const uint4 *c04 = reinterpret_cast<const uint4 *>(ch0w + 8 * gid);
         float mx = -INFINITY;
-        const int tok0 = pg * kT + 16 * gid;
-#pragma unroll
-        for (int q2 = 0; q2 < 2; q2++) {
-            const uint4 w = c04[q2];
+        const int tok0 = pg * kT + 16 * gid + 8 * half;
+        {
+            const uint4 w = *reinterpret_cast<const uint4 *>(ch0w + 8 * gid + 4 * half);
             const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-            for (int e = 0; e < 4; e++) {
-                const int i = 4 * q2 + e;      // tokens 2i, 2i+1 of the 16
+            for (int i = 0; i < 4; i++) {
 #pragma unroll
                 for (int r = 0; r < 2; r++) {
-                    const float c0v = __uint_as_float(r ? (ws[e] & 0xffff0000u) : (ws[e] << 16));
+                    const float c0v = __uint_as_float(r ? (ws[i] & 0xffff0000u) : (ws[i] << 16));
                     const float comp = __int_as_float((127 + 24 - 4 * (i & 1) - 2 * r) << 23);
                     float v = fmaf(sc[i][r], comp, fmaf(q0_t, c0v, zt[i][r])) * kScoreScaleLog2;
                     v = (tok0 + 2 * i + r < len) ? v : -INFINITY;
@@ -267,16 +287,17 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
         const float m_new = fmaxf(m_run, mx);
-        const float alpha = exp2f(m_run - m_new);
-        m_run = m_new;
+        // a half-page with no valid token leaves this warp's state unchanged
+        const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m_run - m_new);
         float psum = 0.f;
 #pragma unroll
-        for (int i = 0; i < 8; i++)
+        for (int i = 0; i < 4; i++)
 #pragma unroll
             for (int r = 0; r < 2; r++) {
-                sc[i][r] = exp2f(sc[i][r] - m_new);
+                sc[i][r] = (m_new == -INFINITY) ? 0.f : exp2f(sc[i][r] - m_new);
                 psum += sc[i][r];
             }
+        m_run = m_new;
         l_thr = fmaf(l_thr, alpha, psum);
 #pragma unroll
         for (int mt = 0; mt < 8; mt++)
@@ -285,39 +306,37 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
 #pragma unroll
         for (int r = 0; r < 4; r++) cz[r] *= alpha;
 
-        // ---------------- p exchange through the (now free) slot area
-        __syncwarp();
-        float *pex = reinterpret_cast<float *>(cur);
+        // ---------------- softmax weights: score layout -> value layout,
+        // through this warp's half of the (now free) slot area
+        pair_sync(pair);                                     // both warps are done with the slots
+        float *pex = reinterpret_cast<float *>(cur) + 512 * half;
         {
-            float *dst = pex + tig * kPexStride + 16 * gid + 4 * (gid >> 1);
-#pragma unroll
-            for (int q4 = 0; q4 < 4; q4++)
-                *reinterpret_cast<float4 *>(dst + 4 * q4) =
-                    make_float4(sc[2 * q4][0], sc[2 * q4][1], sc[2 * q4 + 1][0], sc[2 * q4 + 1][1]);
+            float *dst = pex + pex_head(tig) + pex_pos(8 * gid);
+            *reinterpret_cast<float4 *>(dst) = make_float4(sc[0][0], sc[0][1], sc[1][0], sc[1][1]);
+            *reinterpret_cast<float4 *>(dst + 4) = make_float4(sc[2][0], sc[2][1], sc[3][0], sc[3][1]);
         }
         __syncwarp();
-        float pv[32];                          // head hh, tokens 32tig .. 32tig+31
-        {
-            const float *src = pex + hh * kPexStride + 32 * tig + 4 * tig;
+        float pv[2][8];                        // head hh, local tokens 8(2tig+u) + j
 #pragma unroll
-            for (int q4 = 0; q4 < 8; q4++) {
-                const float4 v = *reinterpret_cast<const float4 *>(src + 4 * q4);
-                pv[4 * q4] = v.x;
-                pv[4 * q4 + 1] = v.y;
-                pv[4 * q4 + 2] = v.z;
-                pv[4 * q4 + 3] = v.w;
-            }
+        for (int u = 0; u < 2; u++) {
+            const float *src = pex + pex_head(hh) + pex_pos(8 * (2 * tig + u));
+            const float4 v0 = *reinterpret_cast<const float4 *>(src);
+            const float4 v1 = *reinterpret_cast<const float4 *>(src + 4);
+            pv[u][0] = v0.x; pv[u][1] = v0.y; pv[u][2] = v0.z; pv[u][3] = v0.w;
+            pv[u][4] = v1.x; pv[u][5] = v1.y; pv[u][6] = v1.z; pv[u][7] = v1.w;
         }
-        // weights of value k-step j = 4u + f: tokens 16u+f, +8 (pair a) and
-        // 16u+f+4, +12 (pair b), scaled by 4^(3-f) to offset the code scaling
-        uint32_t ph[8][2], pl[8][2];
+        // value k-step j = 2u + v uses fields f0 = 2v (k-slots 2tig, 2tig+1) and
+        // f1 = 2v+1 (k-slots 2tig+8, 2tig+9) of word 2tig+u's half, i.e. local
+        // tokens (f, f+4); weights are scaled by 4^(3-f) to offset the code scale
+        uint32_t ph[4][2], pl[4][2];
 #pragma unroll
-        for (int j = 0; j < 8; j++) {
-            const int u = j >> 2, f = j & 3;
-            const float F = (float)(1 << (2 * (3 - f)));
+        for (int j = 0; j < 4; j++) {
+            const int u = j >> 1;
 #pragma unroll
             for (int r = 0; r < 2; r++) {
-                const float xa = pv[16 * u + f + 4 * r] * F, xb = pv[16 * u + f + 8 + 4 * r] * F;
+                const int f = 2 * (j & 1) + r;
+                const float F = (float)(1 << (2 * (3 - f)));
+                const float xa = pv[u][f] * F, xb = pv[u][f + 4] * F;
                 const __half2 hi = __floats2half2_rn(xa, xb);
                 const float2 hf = __half22float2(hi);
                 ph[j][r] = h2u(hi);
@@ -328,24 +347,24 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
         // ---------------- values, group by group
 #pragma unroll
         for (int g = 0; g < kNG; g++) {
-            uint32_t bw[8][2];
+            uint32_t bw[4][2];
             {
-                const uint4 *vw4 = reinterpret_cast<const uint4 *>(vmeta + g * kT + 32 * tig);
-                uint32_t vw[32];
+                uint32_t vw[2][8];         // {s, z} of local tokens 8(2tig+u) + j
 #pragma unroll
-                for (int q4 = 0; q4 < 8; q4++) {
-                    const uint4 w = vw4[q4];
-                    vw[4 * q4] = w.x;
-                    vw[4 * q4 + 1] = w.y;
-                    vw[4 * q4 + 2] = w.z;
-                    vw[4 * q4 + 3] = w.w;
-                }
+                for (int u = 0; u < 2; u++)
 #pragma unroll
-                for (int j = 0; j < 8; j++) {
-                    const int u = j >> 2, f = j & 3;
+                    for (int c = 0; c < 2; c++) {
+                        const int chunk = 4 * (2 * tig + u) + 2 * half + c;
+                        const uint4 w = *reinterpret_cast<const uint4 *>(vmeta + g * kT + 4 * vmeta_chunk(chunk));
+                        vw[u][4 * c] = w.x; vw[u][4 * c + 1] = w.y; vw[u][4 * c + 2] = w.z; vw[u][4 * c + 3] = w.w;
+                    }
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    const int u = j >> 1;
 #pragma unroll
                     for (int r = 0; r < 2; r++) {
-                        const __half2 sp = u2h(__byte_perm(vw[16 * u + f + 4 * r], vw[16 * u + f + 8 + 4 * r], 0x5410));
+                        const int f = 2 * (j & 1) + r;
+                        const __half2 sp = u2h(__byte_perm(vw[u][f], vw[u][f + 4], 0x5410));
                         const __half2 P = u2h(ph[j][r]);
                         const __half2 wh = __hmul2(P, sp);
                         const __half2 res = __hfma2(P, sp, __hneg2(wh));
@@ -359,44 +378,46 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
                 const int mt = 2 * g + m2;
                 const uint2 r0 = *reinterpret_cast<const uint2 *>(vcodes + (16 * mt + gid) * 32 + 8 * tig);
                 const uint2 r1 = *reinterpret_cast<const uint2 *>(vcodes + (16 * mt + gid + 8) * 32 + 8 * tig);
-                const uint32_t W0[2] = {r0.x, r0.y}, W1[2] = {r1.x, r1.y};
-                const uint32_t Y0[2] = {r0.x >> 8, r0.y >> 8}, Y1[2] = {r1.x >> 8, r1.y >> 8};
+                const uint32_t x0[2] = {__byte_perm(r0.x, 0u, vx_sel), __byte_perm(r0.y, 0u, vx_sel)};
+                const uint32_t x1[2] = {__byte_perm(r1.x, 0u, vx_sel), __byte_perm(r1.y, 0u, vx_sel)};
 #pragma unroll
-                for (int j = 0; j < 8; j++) {
-                    const int u = j >> 2, f = j & 3;
-                    const uint32_t m = 0x00030003u << (2 * f);
-                    mma16816(co[mt], W0[u] & m, W1[u] & m, Y0[u] & m, Y1[u] & m, bw[j][0], bw[j][1]);
+                for (int j = 0; j < 4; j++) {
+                    const int u = j >> 1;
+                    const uint32_t mA = 0x00030003u << (4 * (j & 1));
+                    const uint32_t mB = mA << 2;
+                    mma16816(co[mt], x0[u] & mA, x1[u] & mA, x0[u] & mB, x1[u] & mB, bw[j][0], bw[j][1]);
                 }
             }
         }
         // zero-point term: rows = groups (row gid holds group gid), times p
         {
-            const uint4 *zw4 = reinterpret_cast<const uint4 *>(vmeta + (gid & 3) * kT + 32 * tig);
-            uint32_t zw[32];
+            uint32_t zw[2][8];
+            const int zg = gid & 3;
 #pragma unroll
-            for (int q4 = 0; q4 < 8; q4++) {
-                const uint4 w = zw4[q4];
-                zw[4 * q4] = w.x;
-                zw[4 * q4 + 1] = w.y;
-                zw[4 * q4 + 2] = w.z;
-                zw[4 * q4 + 3] = w.w;
-            }
+            for (int u = 0; u < 2; u++)
 #pragma unroll
-            for (int j = 0; j < 8; j++) {
-                const int u = j >> 2, f = j & 3;
-                const __half2 sc2 = __float2half2_rn(zmask / (float)(1 << (2 * (3 - f))));
+                for (int c = 0; c < 2; c++) {
+                    const int chunk = 4 * (2 * tig + u) + 2 * half + c;
+                    const uint4 w = *reinterpret_cast<const uint4 *>(vmeta + zg * kT + 4 * vmeta_chunk(chunk));
+                    zw[u][4 * c] = w.x; zw[u][4 * c + 1] = w.y; zw[u][4 * c + 2] = w.z; zw[u][4 * c + 3] = w.w;
+                }
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const int u = j >> 1;
                 uint32_t a[2];
 #pragma unroll
-                for (int r = 0; r < 2; r++)
-                    a[r] = h2u(__hmul2(u2h(__byte_perm(zw[16 * u + f + 4 * r], zw[16 * u + f + 8 + 4 * r], 0x7632)), sc2));
+                for (int r = 0; r < 2; r++) {
+                    const int f = 2 * (j & 1) + r;
+                    const __half2 sc2 = __float2half2_rn(zmask / (float)(1 << (2 * (3 - f))));
+                    a[r] = h2u(__hmul2(u2h(__byte_perm(zw[u][f], zw[u][f + 4], 0x7632)), sc2));
+                }
                 mma16816(cz, a[0], 0u, a[1], 0u, part ? pl[j][0] : ph[j][0], part ? pl[j][1] : ph[j][1]);
             }
         }
-        __syncwarp();
     }
 
     // ------------------------------------------------------------ merge
-    // per warp: head tig's max, sum and output; then across the 4 warps
+    // per warp: head tig's max, sum and output; then across the 8 warps
     float l_head = l_thr;
     l_head += __shfl_xor_sync(0xffffffffu, l_head, 4);
     l_head += __shfl_xor_sync(0xffffffffu, l_head, 8);
@@ -408,6 +429,7 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
         zsum[g] = __shfl_sync(0xffffffffu, v, 4 * g + tig);
     }
     __syncthreads();                                     // stages are free now
+    constexpr int kWarps = kThreads / 32;
     float *mo = reinterpret_cast<float *>(sh.stage[0][0]);       // [warp][head][128]
     float *mml = mo + kWarps * 4 * kD;                           // [warp][head][2]
     constexpr float kCodeScale = 262144.f;                       // 2^18
@@ -422,36 +444,33 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
         mml[(warp * 4 + tig) * 2 + 1] = l_head;
     }
     __syncthreads();
-    {
-        const int c = tid;
+    for (int e = tid; e < 4 * kD; e += kThreads) {
+        const int hl = e / kD, c = e % kD;
+        float M = -INFINITY;
 #pragma unroll
-        for (int hl = 0; hl < 4; hl++) {
-            float M = -INFINITY;
+        for (int w = 0; w < kWarps; w++) M = fmaxf(M, mml[(w * 4 + hl) * 2]);
+        float o = 0.f, L = 0.f;
+        if (M != -INFINITY) {
 #pragma unroll
-            for (int w = 0; w < kWarps; w++) M = fmaxf(M, mml[(w * 4 + hl) * 2]);
-            float o = 0.f, L = 0.f;
-            if (M != -INFINITY) {
-#pragma unroll
-                for (int w = 0; w < kWarps; w++) {
-                    const float wt = exp2f(mml[(w * 4 + hl) * 2] - M);
-                    L = fmaf(wt, mml[(w * 4 + hl) * 2 + 1], L);
-                    o = fmaf(wt, mo[(w * 4 + hl) * kD + c], o);
-                }
+            for (int w = 0; w < kWarps; w++) {
+                const float wt = exp2f(mml[(w * 4 + hl) * 2] - M);
+                L = fmaf(wt, mml[(w * 4 + hl) * 2 + 1], L);
+                o = fmaf(wt, mo[(w * 4 + hl) * kD + c], o);
             }
-            const size_t row = (qrow0 + hl) * S + s;
-            part_o[row * kD + c] = o;
-            if (c == 0) part_ml[row] = make_float2(M, L);
         }
+        const size_t row = (qrow0 + hl) * S + s;
+        part_o[row * kD + c] = o;
+        if (c == 0) part_ml[row] = make_float2(M, L);
     }
-    merge_unit_if_last<4>(part_o, part_ml, S, qrow0, out, counters + unit,
-                          reinterpret_cast<float *>(sh.stage[1][0]));
+    merge_unit_if_last<4, kThreads>(part_o, part_ml, S, qrow0, out, counters + unit,
+                          reinterpret_cast<float *>(sh.stage[2][0]));
 }
 
 }  // namespace
 
 int decode_mma_splits(int units, int nblk, int num_sms) {
     int S = (2 * num_sms + units - 1) / units;
-    const int max_s = nblk / 4 > 0 ? nblk / 4 : 1;   // at least one page per warp
+    const int max_s = nblk / kPairs > 0 ? nblk / kPairs : 1;   // at least one page per pair
     if (S > max_s) S = max_s;
     return S < 1 ? 1 : S;
 }
@@ -464,9 +483,9 @@ cudaError_t launch_decode_mma(const kvq_cache &c, int Hq, const int32_t *idx, co
     cudaError_t e = set_smem_once(decode_mma_kernel, (int)smem, done);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)S, (unsigned)c.n_kv_heads, (unsigned)c.batch);
-    decode_mma_kernel<<<grid, 128, smem, st>>>(static_cast<const uint8_t *>(c.pages), c.seq_len,
-                                               c.n_kv_heads, c.capacity / kT, Hq, idx, qsel, qgsum, k,
-                                               part_o, part_ml, S, out, unit_counter(c, 0, 0));
+    decode_mma_kernel<<<grid, kThreads, smem, st>>>(static_cast<const uint8_t *>(c.pages), c.seq_len,
+                                                    c.n_kv_heads, c.capacity / kT, Hq, idx, qsel, qgsum, k,
+                                                    part_o, part_ml, S, out, unit_counter(c, 0, 0));
     return cudaGetLastError();
 }
 

@@ -72,14 +72,16 @@ cudaError_t set_smem_once(Kernel *fn, int bytes, std::atomic<uint64_t> &done) {
 // CTA to arrive -- found with the unit's completion counter, which it resets
 // -- merges them: out = sum_s e^{m_s - M} o_s / sum_s e^{m_s - M} l_s, the one
 // softmax over the whole context (Dual-QK §3.4).  Nothing waits: the other
-// CTAs simply exit.  Called by every thread of a 128-thread CTA; `scratch` is
+// CTAs simply exit.  Called by every thread of an NT-thread CTA; `scratch` is
 // shared memory for 2 * G * S + G floats.  The (m, l) pairs are read in one
-// parallel pass and turned into per-split weights, then each thread sums G
-// consecutive outputs over the splits with independent vector loads.
-template <int G>
+// parallel pass and turned into per-split weights, then each thread sums
+// G * 128 / NT consecutive outputs over the splits with independent loads.
+template <int G, int NT>
 __device__ __forceinline__ void merge_unit_if_last(const float *part_o, const float2 *part_ml, int S,
                                                    size_t qrow0, float *out, uint32_t *counter,
                                                    float *scratch) {
+    constexpr int OPT = G * kD / NT;                 // outputs per thread
+    static_assert(OPT >= 1 && G * kD == OPT * NT, "merge: G * 128 must be a multiple of the CTA size");
     __shared__ int s_last;
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -94,13 +96,13 @@ __device__ __forceinline__ void merge_unit_if_last(const float *part_o, const fl
     float *wl = scratch + G * S;     // [G][S] sum
     float *inv = wl + G * S;         // [G] 1 / total sum
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    for (int e = t; e < G * S; e += blockDim.x) {
+    for (int e = t; e < G * S; e += NT) {
         const float2 v = __ldcg(part_ml + qrow0 * S + e);     // rows qrow0.. are contiguous
         wm[e] = v.x;
         wl[e] = v.y;
     }
     __syncthreads();
-    for (int hl = warp; hl < G; hl += blockDim.x / 32) {
+    for (int hl = warp; hl < G; hl += NT / 32) {
         float M = -INFINITY;
         for (int s = lane; s < S; s += 32) M = fmaxf(M, wm[hl * S + s]);
 #pragma unroll
@@ -116,32 +118,36 @@ __device__ __forceinline__ void merge_unit_if_last(const float *part_o, const fl
         if (lane == 0) inv[hl] = L > 0.f ? 1.f / L : 0.f;
     }
     __syncthreads();
-    // thread t owns outputs [t*G, t*G + G) of the unit's [G][128] block
-    const int hl = (t * G) / kD, c0 = (t * G) % kD;
-    float acc[G];
+    // thread t owns outputs [t*OPT, t*OPT + OPT) of the unit's [G][128] block
+    const int hl = (t * OPT) / kD, c0 = (t * OPT) % kD;
+    float acc[OPT];
 #pragma unroll
-    for (int u = 0; u < G; u++) acc[u] = 0.f;
+    for (int u = 0; u < OPT; u++) acc[u] = 0.f;
     const float *po = part_o + ((qrow0 + hl) * S) * kD + c0;
 #pragma unroll 8
     for (int s = 0; s < S; s++) {
         const float w = wm[hl * S + s];
-        if constexpr (G % 4 == 0) {
+        if constexpr (OPT % 4 == 0) {
 #pragma unroll
-            for (int u = 0; u < G; u += 4) {
+            for (int u = 0; u < OPT; u += 4) {
                 const float4 v = __ldcg(reinterpret_cast<const float4 *>(po + (size_t)s * kD + u));
                 acc[u] = fmaf(w, v.x, acc[u]);
                 acc[u + 1] = fmaf(w, v.y, acc[u + 1]);
                 acc[u + 2] = fmaf(w, v.z, acc[u + 2]);
                 acc[u + 3] = fmaf(w, v.w, acc[u + 3]);
             }
+        } else if constexpr (OPT == 2) {
+            const float2 v = __ldcg(reinterpret_cast<const float2 *>(po + (size_t)s * kD));
+            acc[0] = fmaf(w, v.x, acc[0]);
+            acc[1] = fmaf(w, v.y, acc[1]);
         } else {
 #pragma unroll
-            for (int u = 0; u < G; u++) acc[u] = fmaf(w, __ldcg(po + (size_t)s * kD + u), acc[u]);
+            for (int u = 0; u < OPT; u++) acc[u] = fmaf(w, __ldcg(po + (size_t)s * kD + u), acc[u]);
         }
     }
     const float r = inv[hl];
 #pragma unroll
-    for (int u = 0; u < G; u++) out[(qrow0 + hl) * kD + c0 + u] = acc[u] * r;
+    for (int u = 0; u < OPT; u++) out[(qrow0 + hl) * kD + c0 + u] = acc[u] * r;
     __syncthreads();
     if (t == 0) atomicExch(counter, 0u);
 }

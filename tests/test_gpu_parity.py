@@ -293,3 +293,29 @@ def test_small_append_capacity_and_lengths():
     assert torch.equal(before, cache.pages)
     # the counters the calls use are back at zero
     assert not cache.status[1:].any()
+
+
+@pytest.mark.parametrize("name,n_ctx,bits,g", [("llama8b_b8_32k", 300, 2, 4), ("longctx_b1_128k", 5000, 2, 4),
+                                              ("llama8b_b8_32k", 300, 4, 4), ("llama8b_b8_32k", 300, 2, 8)])
+def test_decode_writes_stay_in_bounds(name, n_ctx, bits, g):
+    """Sentinel words after the output and after the workspace survive."""
+    wl = W.workload(name, bits=bits, n_q_heads=8 * g)
+    case = Case(wl, n_ctx=n_ctx)
+    cache = case.gpu_cache()
+    q = case.q(0)
+    sel = kvq.select_channels(cache, to_dev(q, "bf16"), dev64(case.Ai), 0.4)
+    n_out = wl.batch * wl.n_q_heads * 128
+    guard = 4096
+    out_buf = torch.full((n_out + guard,), float("nan"), dtype=torch.float32, device="cuda")
+    wsb = kvq.decode_workspace_bytes(cache, wl.n_q_heads, sel.k)
+    ws_buf = torch.full((wsb + 4 * guard,), 0xA5, dtype=torch.uint8, device="cuda")
+    out = out_buf[:n_out].view(wl.batch, wl.n_q_heads, 128)
+    for _ in range(2):
+        kvq.decode_attn(cache, sel, out=out, ws=ws_buf)
+    torch.cuda.synchronize()
+    assert torch.isnan(out_buf[n_out:]).all()
+    assert (ws_buf[wsb:] == 0xA5).all()
+    assert torch.isfinite(out).all()
+    ref, _, _ = case.oracle_decode(q, wl.batch - 1, wl.n_kv_heads - 1, 0.4)
+    emax, _ = rel_errors(out[-1, -g:].cpu().numpy(), ref)
+    assert emax <= TOL_MAX
