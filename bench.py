@@ -275,7 +275,7 @@ def run_ours(args):
         step.k_new.copy_(kv_pool[i % n_pool][0])
         step.v_new.copy_(kv_pool[i % n_pool][1])
 
-    launches_per_step = 5   # append + length advance, select, decode partial, merge
+    launches_per_step = 3   # one-token append (fused length advance), select, decode (fused merge)
     step.time_decode()
     length = wl.n_ctx
     for i in range(args.warmup):

@@ -33,8 +33,13 @@
  *                  channel r; row 0 is unused and stays zero
  *  offset 128R     value codes, 128 rows x R bytes, row r = value channel r
  *  offset 256R     channel 0 of the transformed key, 128 x bf16
- *  offset 256R+256 key metadata [4 groups][128 tokens] x {fp16 scale, fp16 zero}
+ *  offset 256R+256 key metadata: 512 words {fp16 scale (low half), fp16 zero}
  *  +2048           value metadata, same shape
+ *  Metadata word of token t (0..127), group g (0..3):
+ *      128 g + 4 sw(g, t / 4) + t % 4,   sw(g, c) = c XOR ((c / 8) XOR 4 (g % 2))
+ *  i.e. each group's 32 chunks of 4 tokens are stored XOR-permuted within
+ *  blocks of 8 chunks (a layout that lets the decode kernels read metadata
+ *  without shared-memory bank conflicts after a contiguous copy).
  *  page bytes = 256R + 4352 (12544 for INT2, 20736 for INT4)
  *  Code of token t (0..127) of a page: byte t*bits/8 of its row, bit
  *  (t mod (8/bits))*bits, least significant first.  Key groups are channels
@@ -71,7 +76,15 @@ enum {
 enum { KVQ_DTYPE_F32 = 0, KVQ_DTYPE_BF16 = 1 };
 
 /* device status flags (sticky; cleared by kvq_cache_init) */
-enum { KVQ_DEV_CAPACITY = 1u };
+enum {
+    KVQ_DEV_CAPACITY = 1u,   /* an append would have overflowed a sequence           */
+    KVQ_DEV_TIMEOUT = 2u,    /* a bounded wait for an asynchronous copy gave up; the
+                                result of that call is not valid                    */
+    KVQ_DEV_INDEX = 4u       /* a decode got a channel list that is not channel 0
+                                followed by ascending channels in 1..127; it read
+                                no key rows outside the page and its result is not
+                                valid                                               */
+};
 
 /* Cache descriptor.  The struct itself is host memory; the pointers in it are
  * device memory owned by the caller. */

@@ -167,7 +167,7 @@ append_kernel(uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len,
         if (!(valid >> tt & 1u)) continue;                        // uniform over the CTA
         codes[tt] = quantize_lane<BITS>(acc[tt], j != 0, sb, zb);
         if (valid >> tt & 1u) {
-            if (lane == 0) kmeta[grp * kT + t0 + tt] = (uint32_t)sb | ((uint32_t)zb << 16);
+            if (lane == 0) kmeta[meta_word(grp, t0 + tt)] = (uint32_t)sb | ((uint32_t)zb << 16);
             if (j == 0) ch0[t0 + tt] = __bfloat16_as_ushort(__double2bfloat16(acc[tt]));
         }
     }
@@ -181,7 +181,7 @@ append_kernel(uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len,
         if (!(valid >> tt & 1u)) continue;
         codes[tt] = quantize_lane<BITS>(vs[tt][j], true, sb, zb);
         if ((valid >> tt & 1u) && lane == 0)
-            vmeta[grp * kT + t0 + tt] = (uint32_t)sb | ((uint32_t)zb << 16);
+            vmeta[meta_word(grp, t0 + tt)] = (uint32_t)sb | ((uint32_t)zb << 16);
     }
     store_row<BITS>(page + off_vcodes(BITS) + (size_t)j * R + t0 * BITS / 8, codes, valid);
 }
@@ -236,7 +236,7 @@ append_small_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len,
             uint16_t sb, zb;
             const uint32_t kc = quantize_lane<BITS>(x, j != 0, sb, zb);
             if (lane == 0)
-                reinterpret_cast<uint32_t *>(page + off_kmeta(BITS))[grp * kT + t] = (uint32_t)sb | ((uint32_t)zb << 16);
+                reinterpret_cast<uint32_t *>(page + off_kmeta(BITS))[meta_word(grp, t)] = (uint32_t)sb | ((uint32_t)zb << 16);
             if (j == 0) {
                 reinterpret_cast<uint16_t *>(page + off_ch0(BITS))[t] = __bfloat16_as_ushort(__double2bfloat16(x));
             } else {
@@ -245,7 +245,7 @@ append_small_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len,
             }
             const uint32_t vc = quantize_lane<BITS>(vs[i][j], true, sb, zb);
             if (lane == 0)
-                reinterpret_cast<uint32_t *>(page + off_vmeta(BITS))[grp * kT + t] = (uint32_t)sb | ((uint32_t)zb << 16);
+                reinterpret_cast<uint32_t *>(page + off_vmeta(BITS))[meta_word(grp, t)] = (uint32_t)sb | ((uint32_t)zb << 16);
             uint8_t *p = page + off_vcodes(BITS) + (size_t)j * R + byte;
             *p = (uint8_t)((*p & clear) | (vc << sh));
         }

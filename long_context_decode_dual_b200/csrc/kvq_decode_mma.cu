@@ -15,19 +15,23 @@
 // Codes stay exact: a 2-bit field masked in place inside a 16-bit half is an
 // fp16 subnormal equal to code * 2^(pos-24), so unpacking is one AND per two
 // codes; the power of two is compensated exactly on the other operand or in
-// fp32 afterwards.  Query and weights are split into fp16 hi + lo parts that
-// occupy the two columns of each head (n = 8 = 4 heads x {hi, lo}), giving
-// near-fp32 operands.  Per-token, per-group scale and zero-point are applied
-// in fp32 after the score MMAs, folded into the weights before the value
-// MMAs, and the value zero-point term sum_t p(t) z(t) is one more MMA.
+// fp32 afterwards.  Query and softmax weights are split into fp16 hi + lo
+// parts, giving near-fp32 operands.  Score MMAs put the parts in the two
+// columns of each head (n = 8 = 4 heads x {hi, lo}) and apply each key
+// group's per-token scale in fp32 afterwards; value MMAs take a group pair
+// per tile (rows: 8 channels of each group, columns: 4 heads x 2 groups) and
+// run hi and lo as two MMAs, so the per-token value scale is folded into the
+// weights once per group.  The value zero-point term sum_t p(t) z(t) is one
+// more MMA pair.
 //
 // Work split: one CTA = one (sequence, KV head, split of the context), eight
 // warps in four pairs.  A pair processes one 128-token page at a time from a
-// two-stage cp.async ring; warp w of the pair takes half w of every 16-token
-// word of the page (64 tokens) and keeps its own online softmax.  Selected key
-// rows land in fixed slots: group g owns slots 32g..32g+31, filled in
-// ascending channel order, so every MMA k-step (16 slots) lies inside one
-// group and its scale applies to the whole step.
+// two-stage ring filled by bulk asynchronous copies (one for the contiguous
+// tail of the page, one per run of consecutive selected key rows) completing
+// on an mbarrier; warp w of the pair takes half w of every 16-token word of
+// the page (64 tokens) and keeps its own online softmax.  Selected key rows
+// land in fixed slots: group g owns slots 32g..32g+31, filled in ascending
+// channel order, so every score k-step (16 slots) lies inside one group.
 #include "kvq_internal.cuh"
 
 namespace kvq {
@@ -35,22 +39,25 @@ namespace {
 
 constexpr int kPairs = 4;
 constexpr int kThreads = 64 * kPairs;
+static_assert(kThreads == 8 * 32, "one warp per score k-step in the prologue");
 constexpr int kSlotBytes = 128 * 32;              // 4 groups x 32 slots x 32 B
 constexpr int kFixBytes = fixed_bytes(2);         // value codes, ch0, metadata
 constexpr int kStageBytes = kSlotBytes + kFixBytes;
-constexpr int kMaxTasks = 2 * 127;                // 16-byte copies of key rows
-// chunk (16 B) offsets inside the fixed part of a staged page
-constexpr int kVmetaChunk = (4096 + 256 + 2048) / 16;   // 400
-constexpr int kFixChunks = kFixBytes / 16;              // 528
+constexpr int kMaxRuns = 127;
+constexpr uint32_t kWaitPolls = 1u << 20;         // bound on mbarrier polls per stage
 
 struct __align__(16) MmaShared {
     uint8_t stage[kPairs][2][kStageBytes];
-    uint32_t task[kMaxTasks];          // src offset | dst offset << 16 (bytes)
+    uint64_t mbar[kPairs][2];
+    uint32_t run[kMaxRuns];            // src row | dst slot << 7 | rows << 14
+    int run_pos[kD];                   // first selected position of each run
+    uint2 bq[8][32];                   // score-MMA B fragments per k-step and lane
     float q[4][kD];                    // qsel of the 4 heads, by selected position
     float qg[4][kNG];
     int slot_pos[kD];                  // slot -> position in the selected list, -1 = pad
-    int nks[kNG];                      // MMA k-steps per key group (0, 1 or 2)
-    int n_tasks;
+    int nks[kNG];                      // score k-steps per key group (0, 1 or 2)
+    int run_warp[4];
+    int n_runs;
 };
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -66,6 +73,42 @@ __device__ __forceinline__ void pair_sync(int pair) {
     asm volatile("bar.sync %0, 64;\n" ::"r"(pair + 1) : "memory");
 }
 
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+// Wait for a stage's copies.  The wait is bounded: after kWaitPolls polls the
+// device status word gets KVQ_DEV_TIMEOUT and the caller goes on (that call's
+// output is then reported invalid) instead of waiting forever; both warps of
+// a pair keep the same control flow either way.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint32_t *status) {
+    for (uint32_t i = 0; i < kWaitPolls; i++)
+        if (mbar_try_wait(bar, parity)) return true;
+    atomicOr(status, (uint32_t)KVQ_DEV_TIMEOUT);
+    return false;
+}
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
 __device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2 *>(&u); }
 __device__ __forceinline__ float lo_f16(uint32_t w) { return __half2float(__ushort_as_half((uint16_t)(w & 0xffffu))); }
@@ -78,10 +121,8 @@ __device__ __forceinline__ uint16_t f16_part(float x, int part) {
     return __half_as_ushort(__float2half_rn(x - __half2float(hi)));
 }
 
-// Value metadata chunks (4 tokens each) are stored swizzled within each
-// group's 32 chunks so that the four thread columns of a warp, which read
-// chunks 8 apart, hit different banks.
-__device__ __forceinline__ int vmeta_chunk(int c) { return c ^ ((c >> 3) & 7); }
+// 4-token metadata chunk c of group g (the page format's XOR permutation)
+__device__ __forceinline__ int meta_chunk(int g, int c) { return c ^ (((c >> 3) & 3) ^ ((g & 1) << 2)); }
 
 // position of local token l (0..63) in a warp's softmax-weight exchange
 // buffer, and the start of head h's block (skews keep both access patterns
@@ -94,7 +135,7 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
                   int NB, int Hq, const int32_t *__restrict__ idx, const float *__restrict__ qsel,
                   const float *__restrict__ qgsum, int k, float *__restrict__ part_o,
                   float2 *__restrict__ part_ml, int S, float *__restrict__ out,
-                  uint32_t *__restrict__ counters) {
+                  uint32_t *__restrict__ counters, uint32_t *__restrict__ status) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     MmaShared &sh = *reinterpret_cast<MmaShared *>(smem_raw);
 
@@ -106,9 +147,10 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
     const size_t qrow0 = (size_t)b * Hq + (size_t)h * 4;
 
     // ------------------------------------------------------------ prologue
-    // The selected list is ascending, so each group's channels sit in one
-    // contiguous run of positions; a channel's slot is 32g + (its position -
-    // the first position of its group).
+    // Selected positions 1..k-1 hold channels >= 1 ascending, so each group is
+    // one contiguous run of positions: a channel's slot is 32g + (its position
+    // - the first position of its group).  Runs of consecutive channels inside
+    // a group become one bulk copy each.
     for (int e = tid; e < 4 * k; e += kThreads) {
         const int hl = e / k, i = e % k;
         sh.q[hl][i] = qsel[(qrow0 + hl) * k + i];
@@ -116,50 +158,88 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
     if (tid < 4 * kNG) sh.qg[tid / kNG][tid % kNG] = qgsum[qrow0 * kNG + tid];
     if (tid < kD) sh.slot_pos[tid] = -1;
     if (tid < kNG) sh.nks[tid] = 0;
-    __syncthreads();
+    if (tid < 2 * kPairs) mbar_init(smem_u32(&sh.mbar[tid >> 1][tid & 1]), 1);
+    // the list must be channel 0 followed by ascending channels in 1..127;
+    // any other list copies no key rows and raises KVQ_DEV_INDEX
     const int32_t *sel = idx + unit * k;
-    const int my_c = (tid >= 1 && tid < k) ? sel[tid] : -1;
+    int my_c = -1, prev_c = -2;
+    bool bad = false;
+    if (tid < k) {
+        const int c = sel[tid];
+        if (tid == 0) {
+            bad = c != 0;
+        } else {
+            prev_c = sel[tid - 1];
+            bad = c <= prev_c || c > kD - 1;
+            my_c = c;
+        }
+    }
+    const bool any_bad = __syncthreads_or(bad);
+    if (any_bad) my_c = -1;
+    if (any_bad && tid == 0) atomicOr(status, (uint32_t)KVQ_DEV_INDEX);
+    const int k_rows = any_bad ? 0 : k - 1;
+    const bool run_start = my_c >= 0 && (tid == 1 || prev_c != my_c - 1 || (my_c & 31) == 0);
     if (my_c >= 0) atomicAdd(&sh.nks[my_c >> 5], 1);          // counts for now
+    unsigned start_mask = 0;
+    if (tid < kD) {
+        start_mask = __ballot_sync(0xffffffffu, run_start);
+        if (lane == 0) sh.run_warp[warp] = __popc(start_mask);
+    }
     __syncthreads();
+    int my_slot = -1, my_run = -1;
     if (my_c >= 0) {
         const int g = my_c >> 5;
         int start = 1;
         for (int gg = 0; gg < g; gg++) start += sh.nks[gg];
-        const int slot = 32 * g + (tid - start);
-        sh.slot_pos[slot] = tid;
-        sh.task[2 * (tid - 1)] = (uint32_t)(my_c * 32) | ((uint32_t)(slot * 32) << 16);
-        sh.task[2 * (tid - 1) + 1] = (uint32_t)(my_c * 32 + 16) | ((uint32_t)(slot * 32 + 16) << 16);
+        my_slot = 32 * g + (tid - start);
+        sh.slot_pos[my_slot] = tid;
+        if (run_start) {
+            my_run = __popc(start_mask & ((1u << lane) - 1u));
+            for (int w = 0; w < warp; w++) my_run += sh.run_warp[w];
+            sh.run_pos[my_run] = tid;
+        }
     }
-    if (tid == 0) sh.n_tasks = 2 * (k - 1);
+    if (tid == 0) sh.n_runs = sh.run_warp[0] + sh.run_warp[1] + sh.run_warp[2] + sh.run_warp[3];
     __syncthreads();
+    if (my_run >= 0) {
+        const int next = (my_run + 1 < sh.n_runs) ? sh.run_pos[my_run + 1] : k_rows + 1;
+        sh.run[my_run] = (uint32_t)my_c | ((uint32_t)my_slot << 7) | ((uint32_t)(next - tid) << 14);
+    }
     if (tid < kNG) sh.nks[tid] = (sh.nks[tid] + 15) >> 4;       // counts -> k-steps
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     __syncthreads();
 
     // score-MMA B fragments: column gid = (head gid>>1, part gid&1); k-slots
     // 2tig, 2tig+1, 2tig+8, 2tig+9 of a step = slots +tig, +tig+4, +tig+8, +tig+12
-    // (this slot order makes the code loads bank-conflict free)
+    // (this slot order makes the code loads bank-conflict free); kept in
+    // shared memory as one 8-byte word per k-step and lane
     const int hh = gid >> 1, part = gid & 1;
-    uint32_t bq[8][2];
-#pragma unroll
-    for (int ks = 0; ks < 8; ks++) {
+    {
+        const int ks = tid >> 5;                     // 8 warps: one k-step each
         const int base = 32 * (ks >> 1) + 16 * (ks & 1);
+        uint32_t w[2];
 #pragma unroll
         for (int r = 0; r < 2; r++) {
             const int s0 = base + tig + 8 * r, s1 = s0 + 4;
             const int p0 = sh.slot_pos[s0], p1 = sh.slot_pos[s1];
             const float q0 = p0 >= 0 ? sh.q[hh][p0] : 0.f;
             const float q1 = p1 >= 0 ? sh.q[hh][p1] : 0.f;
-            bq[ks][r] = (uint32_t)f16_part(q0, part) | ((uint32_t)f16_part(q1, part) << 16);
+            w[r] = (uint32_t)f16_part(q0, part) | ((uint32_t)f16_part(q1, part) << 16);
         }
+        sh.bq[ks][lane] = make_uint2(w[0], w[1]);
     }
+    __syncthreads();
     int nks[kNG];
 #pragma unroll
     for (int g = 0; g < kNG; g++) nks[g] = sh.nks[g];
+    // zero-point and channel-0 coefficients of head tig, pre-scaled to the
+    // base-2 score domain
     float qg_t[kNG];
 #pragma unroll
-    for (int g = 0; g < kNG; g++) qg_t[g] = sh.qg[tig][g];
-    const float q0_t = sh.q[tig][0];                 // channel-0 coefficient of head tig
-    const int n_tasks = sh.n_tasks;
+    for (int g = 0; g < kNG; g++) qg_t[g] = sh.qg[tig][g] * kScoreScaleLog2;
+    const float q0_t = sh.q[tig][0] * kScoreScaleLog2;
+    const int n_runs = sh.n_runs;
+    const uint32_t tx_bytes = 32u * (uint32_t)k_rows + (uint32_t)kFixBytes;
 
     // ------------------------------------------------------------ pages
     const int len = min(max(seq_len[b], 0), NB * kT);
@@ -168,29 +248,28 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
     const int blk0 = s * bps;
     const int blk1 = min(nblk, blk0 + bps);
 
-    // the pair's 64 threads copy one page into a stage
-    auto issue = [&](uint8_t *dst, int blk) {
+    // the pair's first warp stages a page: lane 0 arms the stage's barrier and
+    // copies the contiguous tail, the lanes then copy one run of selected key
+    // rows each
+    auto issue = [&](int st, int blk) {
         const uint8_t *src = pages + (unit * NB + (size_t)blk) * page_bytes(2);
-        for (int e = pt; e < n_tasks; e += 64) {
-            const uint32_t t = sh.task[e];
-            cp_async16(dst + (t >> 16), src + (t & 0xffffu));
+        const uint32_t dst = smem_u32(sh.stage[pair][st]);
+        const uint32_t bar = smem_u32(&sh.mbar[pair][st]);
+        if (lane == 0) {
+            mbar_expect_tx(bar, tx_bytes);
+            bulk_g2s(dst + kSlotBytes, src + off_vcodes(2), (uint32_t)kFixBytes, bar);
         }
-#pragma unroll 3
-        for (int e = pt; e < kFixChunks; e += 64) {
-            int d = e;
-            if (e >= kVmetaChunk) {
-                const int c = e - kVmetaChunk;
-                d = kVmetaChunk + (c & ~31) + vmeta_chunk(c & 31);
-            }
-            cp_async16(dst + kSlotBytes + 16 * d, src + off_vcodes(2) + 16 * e);
+        __syncwarp();
+        for (int r = lane; r < n_runs; r += 32) {
+            const uint32_t w = sh.run[r];
+            bulk_g2s(dst + ((w >> 7) & 127u) * 32u, src + (w & 127u) * 32u, (w >> 14) * 32u, bar);
         }
-        cp_async_commit();
     };
 
     float m_run = -INFINITY;      // running max of head tig (base-2 domain)
     float l_thr = 0.f;            // this thread's share of the running sum of head tig
-    float co[8][4];               // out^T: rows 16mt+gid / +8, columns head tig {hi, lo}
-    float cz[4];                  // value zero-point term: row gid = group gid
+    float co[8][4];               // out^T tiles; [0]: channel a, head tig; [3]: channel b, head tig
+    float cz[4];                  // value zero-point term: [0] = group gid, head tig
 #pragma unroll
     for (int mt = 0; mt < 8; mt++)
 #pragma unroll
@@ -204,13 +283,17 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
     const float zmask = gid < 4 ? 1.f : 0.f;
 
     int it = 0;
+    uint32_t late = 0;            // stages whose last wait gave up, with the parity waited for
     const int first = blk0 + pair;
-    if (first < blk1) issue(sh.stage[pair][0], first);
+    if (half == 0 && first < blk1) issue(0, first);
     for (int pg = first; pg < blk1; pg += kPairs, it++) {
-        uint8_t *cur = sh.stage[pair][it & 1];
-        cp_async_wait<0>();
-        pair_sync(pair);                                     // page pg staged; other stage free
-        if (pg + kPairs < blk1) issue(sh.stage[pair][(it + 1) & 1], pg + kPairs);
+        const int st = it & 1;
+        uint8_t *cur = sh.stage[pair][st];
+        const uint32_t par = (uint32_t)(it >> 1) & 1u;
+        late = mbar_wait_bounded(smem_u32(&sh.mbar[pair][st]), par, status)
+                   ? late & ~(3u << (2 * st)) : (late & ~(3u << (2 * st))) | ((2u | par) << (2 * st));
+        pair_sync(pair);                                     // both warps left the other stage
+        if (half == 0 && pg + kPairs < blk1) issue(st ^ 1, pg + kPairs);
 
         const uint8_t *vcodes = cur + kSlotBytes;
         const uint32_t *ch0w = reinterpret_cast<const uint32_t *>(vcodes + 128 * 32);
@@ -240,7 +323,8 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
                 const uint32_t Wd = *reinterpret_cast<const uint32_t *>(sb + 12 * 32);
                 const uint32_t Xab = __byte_perm(Wa, Wb, half_sel), Xcd = __byte_perm(Wc, Wd, half_sel);
                 const uint32_t Yab = Xab >> 8, Ycd = Xcd >> 8;
-                const uint32_t b0 = bq[2 * g + j][0], b1 = bq[2 * g + j][1];
+                const uint2 bb = sh.bq[2 * g + j][lane];
+                const uint32_t b0 = bb.x, b1 = bb.y;
 #pragma unroll
                 for (int i = 0; i < 4; i++) {
                     const uint32_t x1 = (i & 2) ? Yab : Xab;
@@ -251,10 +335,10 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
                 }
             }
             // scale and zero-point of group g for the thread's 8 tokens
-            const uint4 *kw4 = reinterpret_cast<const uint4 *>(kmeta + g * kT + 16 * gid + 8 * half);
 #pragma unroll
             for (int q4 = 0; q4 < 2; q4++) {
-                const uint4 w = kw4[q4];
+                const uint4 w = *reinterpret_cast<const uint4 *>(
+                    kmeta + 128 * g + 4 * meta_chunk(g, 4 * gid + 2 * half + q4));
                 const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                 for (int e = 0; e < 4; e++) {
@@ -264,9 +348,8 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
                 }
             }
         }
-        // full scores (base-2 domain), masked beyond the sequence
+        // full scores (base-2 domain), masked beyond the sequence on the last page
         float mx = -INFINITY;
-        const int tok0 = pg * kT + 16 * gid + 8 * half;
         {
             const uint4 w = *reinterpret_cast<const uint4 *>(ch0w + 8 * gid + 4 * half);
             const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
@@ -275,36 +358,47 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
 #pragma unroll
                 for (int r = 0; r < 2; r++) {
                     const float c0v = __uint_as_float(r ? (ws[i] & 0xffff0000u) : (ws[i] << 16));
-                    const float comp = __int_as_float((127 + 24 - 4 * (i & 1) - 2 * r) << 23);
-                    float v = fmaf(sc[i][r], comp, fmaf(q0_t, c0v, zt[i][r])) * kScoreScaleLog2;
-                    v = (tok0 + 2 * i + r < len) ? v : -INFINITY;
-                    sc[i][r] = v;
-                    mx = fmaxf(mx, v);
+                    // 2^(24 - field position) undoes the code scaling; times log2(e)/sqrt(d)
+                    const float comp = __int_as_float((127 + 24 - 4 * (i & 1) - 2 * r) << 23) * kScoreScaleLog2;
+                    sc[i][r] = fmaf(sc[i][r], comp, fmaf(q0_t, c0v, zt[i][r]));
                 }
             }
+            if ((pg + 1) * kT > len) {                       // partial page
+                const int tok0 = pg * kT + 16 * gid + 8 * half;
+#pragma unroll
+                for (int i = 0; i < 4; i++)
+#pragma unroll
+                    for (int r = 0; r < 2; r++)
+                        if (tok0 + 2 * i + r >= len) sc[i][r] = -INFINITY;
+            }
+#pragma unroll
+            for (int i = 0; i < 4; i++) mx = fmaxf(mx, fmaxf(sc[i][0], sc[i][1]));
         }
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
         const float m_new = fmaxf(m_run, mx);
         // a half-page with no valid token leaves this warp's state unchanged
-        const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m_run - m_new);
+        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+        const float alpha = ex2(m_run - m_use);
         float psum = 0.f;
 #pragma unroll
         for (int i = 0; i < 4; i++)
 #pragma unroll
             for (int r = 0; r < 2; r++) {
-                sc[i][r] = (m_new == -INFINITY) ? 0.f : exp2f(sc[i][r] - m_new);
+                sc[i][r] = ex2(sc[i][r] - m_use);
                 psum += sc[i][r];
             }
         m_run = m_new;
         l_thr = fmaf(l_thr, alpha, psum);
+        if (!__all_sync(0xffffffffu, alpha == 1.f)) {
 #pragma unroll
-        for (int mt = 0; mt < 8; mt++)
-#pragma unroll
-            for (int r = 0; r < 4; r++) co[mt][r] *= alpha;
-#pragma unroll
-        for (int r = 0; r < 4; r++) cz[r] *= alpha;
+            for (int mt = 0; mt < 8; mt++) {
+                co[mt][0] *= alpha;
+                co[mt][3] *= alpha;
+            }
+            cz[0] *= alpha;
+        }
 
         // ---------------- softmax weights: score layout -> value layout,
         // through this warp's half of the (now free) slot area
@@ -316,46 +410,50 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
             *reinterpret_cast<float4 *>(dst + 4) = make_float4(sc[2][0], sc[2][1], sc[3][0], sc[3][1]);
         }
         __syncwarp();
-        float pv[2][8];                        // head hh, local tokens 8(2tig+u) + j
-#pragma unroll
-        for (int u = 0; u < 2; u++) {
-            const float *src = pex + pex_head(hh) + pex_pos(8 * (2 * tig + u));
-            const float4 v0 = *reinterpret_cast<const float4 *>(src);
-            const float4 v1 = *reinterpret_cast<const float4 *>(src + 4);
-            pv[u][0] = v0.x; pv[u][1] = v0.y; pv[u][2] = v0.z; pv[u][3] = v0.w;
-            pv[u][4] = v1.x; pv[u][5] = v1.y; pv[u][6] = v1.z; pv[u][7] = v1.w;
-        }
         // value k-step j = 2u + v uses fields f0 = 2v (k-slots 2tig, 2tig+1) and
         // f1 = 2v+1 (k-slots 2tig+8, 2tig+9) of word 2tig+u's half, i.e. local
         // tokens (f, f+4); weights are scaled by 4^(3-f) to offset the code scale
         uint32_t ph[4][2], pl[4][2];
+        {
+            float pv[2][8];                    // head hh, local tokens 8(2tig+u) + j
 #pragma unroll
-        for (int j = 0; j < 4; j++) {
-            const int u = j >> 1;
+            for (int u = 0; u < 2; u++) {
+                const float *src = pex + pex_head(hh) + pex_pos(8 * (2 * tig + u));
+                const float4 v0 = *reinterpret_cast<const float4 *>(src);
+                const float4 v1 = *reinterpret_cast<const float4 *>(src + 4);
+                pv[u][0] = v0.x; pv[u][1] = v0.y; pv[u][2] = v0.z; pv[u][3] = v0.w;
+                pv[u][4] = v1.x; pv[u][5] = v1.y; pv[u][6] = v1.z; pv[u][7] = v1.w;
+            }
 #pragma unroll
-            for (int r = 0; r < 2; r++) {
-                const int f = 2 * (j & 1) + r;
-                const float F = (float)(1 << (2 * (3 - f)));
-                const float xa = pv[u][f] * F, xb = pv[u][f + 4] * F;
-                const __half2 hi = __floats2half2_rn(xa, xb);
-                const float2 hf = __half22float2(hi);
-                ph[j][r] = h2u(hi);
-                pl[j][r] = h2u(__floats2half2_rn(xa - hf.x, xb - hf.y));
+            for (int j = 0; j < 4; j++) {
+                const int u = j >> 1;
+#pragma unroll
+                for (int r = 0; r < 2; r++) {
+                    const int f = 2 * (j & 1) + r;
+                    const float F = (float)(1 << (2 * (3 - f)));
+                    const float xa = pv[u][f] * F, xb = pv[u][f + 4] * F;
+                    const __half2 hi = __floats2half2_rn(xa, xb);
+                    const float2 hf = __half22float2(hi);
+                    ph[j][r] = h2u(hi);
+                    pl[j][r] = h2u(__floats2half2_rn(xa - hf.x, xb - hf.y));
+                }
             }
         }
 
-        // ---------------- values, group by group
+        // ---------------- values: tile mt = group pair pp, rows 8 channels of
+        // each group; this thread's weight column belongs to group 2pp + part
 #pragma unroll
-        for (int g = 0; g < kNG; g++) {
-            uint32_t bw[4][2];
+        for (int pp = 0; pp < 2; pp++) {
+            const int gv = 2 * pp + part;
+            uint32_t bh[4][2], bl[4][2];
             {
-                uint32_t vw[2][8];         // {s, z} of local tokens 8(2tig+u) + j
+                uint32_t vw[2][8];             // {s, z} of local tokens 8(2tig+u) + j, group gv
 #pragma unroll
                 for (int u = 0; u < 2; u++)
 #pragma unroll
                     for (int c = 0; c < 2; c++) {
-                        const int chunk = 4 * (2 * tig + u) + 2 * half + c;
-                        const uint4 w = *reinterpret_cast<const uint4 *>(vmeta + g * kT + 4 * vmeta_chunk(chunk));
+                        const uint4 w = *reinterpret_cast<const uint4 *>(
+                            vmeta + 128 * gv + 4 * meta_chunk(gv, 4 * (2 * tig + u) + 2 * half + c));
                         vw[u][4 * c] = w.x; vw[u][4 * c + 1] = w.y; vw[u][4 * c + 2] = w.z; vw[u][4 * c + 3] = w.w;
                     }
 #pragma unroll
@@ -367,17 +465,17 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
                         const __half2 sp = u2h(__byte_perm(vw[u][f], vw[u][f + 4], 0x5410));
                         const __half2 P = u2h(ph[j][r]);
                         const __half2 wh = __hmul2(P, sp);
-                        const __half2 res = __hfma2(P, sp, __hneg2(wh));
-                        const __half2 wl = __hfma2(u2h(pl[j][r]), sp, res);
-                        bw[j][r] = part ? h2u(wl) : h2u(wh);
+                        bh[j][r] = h2u(wh);
+                        bl[j][r] = h2u(__hfma2(u2h(pl[j][r]), sp, __hfma2(P, sp, __hneg2(wh))));
                     }
                 }
             }
 #pragma unroll
-            for (int m2 = 0; m2 < 2; m2++) {
-                const int mt = 2 * g + m2;
-                const uint2 r0 = *reinterpret_cast<const uint2 *>(vcodes + (16 * mt + gid) * 32 + 8 * tig);
-                const uint2 r1 = *reinterpret_cast<const uint2 *>(vcodes + (16 * mt + gid + 8) * 32 + 8 * tig);
+            for (int sub = 0; sub < 4; sub++) {
+                const int mt = 4 * pp + sub;
+                const int ca = 64 * pp + 8 * sub + gid;
+                const uint2 r0 = *reinterpret_cast<const uint2 *>(vcodes + ca * 32 + 8 * tig);
+                const uint2 r1 = *reinterpret_cast<const uint2 *>(vcodes + (ca + 32) * 32 + 8 * tig);
                 const uint32_t x0[2] = {__byte_perm(r0.x, 0u, vx_sel), __byte_perm(r0.y, 0u, vx_sel)};
                 const uint32_t x1[2] = {__byte_perm(r1.x, 0u, vx_sel), __byte_perm(r1.y, 0u, vx_sel)};
 #pragma unroll
@@ -385,7 +483,9 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
                     const int u = j >> 1;
                     const uint32_t mA = 0x00030003u << (4 * (j & 1));
                     const uint32_t mB = mA << 2;
-                    mma16816(co[mt], x0[u] & mA, x1[u] & mA, x0[u] & mB, x1[u] & mB, bw[j][0], bw[j][1]);
+                    const uint32_t a0 = x0[u] & mA, a1 = x1[u] & mA, a2 = x0[u] & mB, a3 = x1[u] & mB;
+                    mma16816(co[mt], a0, a1, a2, a3, bh[j][0], bh[j][1]);
+                    mma16816(co[mt], a0, a1, a2, a3, bl[j][0], bl[j][1]);
                 }
             }
         }
@@ -397,8 +497,8 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
             for (int u = 0; u < 2; u++)
 #pragma unroll
                 for (int c = 0; c < 2; c++) {
-                    const int chunk = 4 * (2 * tig + u) + 2 * half + c;
-                    const uint4 w = *reinterpret_cast<const uint4 *>(vmeta + zg * kT + 4 * vmeta_chunk(chunk));
+                    const uint4 w = *reinterpret_cast<const uint4 *>(
+                        vmeta + 128 * zg + 4 * meta_chunk(zg, 4 * (2 * tig + u) + 2 * half + c));
                     zw[u][4 * c] = w.x; zw[u][4 * c + 1] = w.y; zw[u][4 * c + 2] = w.z; zw[u][4 * c + 3] = w.w;
                 }
 #pragma unroll
@@ -411,10 +511,20 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
                     const __half2 sc2 = __float2half2_rn(zmask / (float)(1 << (2 * (3 - f))));
                     a[r] = h2u(__hmul2(u2h(__byte_perm(zw[u][f], zw[u][f + 4], 0x7632)), sc2));
                 }
-                mma16816(cz, a[0], 0u, a[1], 0u, part ? pl[j][0] : ph[j][0], part ? pl[j][1] : ph[j][1]);
+                mma16816(cz, a[0], 0u, a[1], 0u, ph[j][0], ph[j][1]);
+                mma16816(cz, a[0], 0u, a[1], 0u, pl[j][0], pl[j][1]);
             }
         }
+        // order this thread's generic accesses to the stage before the bulk
+        // copies that refill it
+        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
     }
+    // a stage whose wait gave up may still receive bytes: wait once more
+    // (bounded) before the staging memory is reused below
+#pragma unroll
+    for (int st = 0; st < 2; st++)
+        if (late & (2u << (2 * st)))
+            mbar_wait_bounded(smem_u32(&sh.mbar[pair][st]), (late >> (2 * st)) & 1u, status);
 
     // ------------------------------------------------------------ merge
     // per warp: head tig's max, sum and output; then across the 8 warps
@@ -424,10 +534,7 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
     l_head += __shfl_xor_sync(0xffffffffu, l_head, 16);
     float zsum[kNG];
 #pragma unroll
-    for (int g = 0; g < kNG; g++) {
-        const float v = cz[0] + cz[1];                   // valid in lanes with gid == group
-        zsum[g] = __shfl_sync(0xffffffffu, v, 4 * g + tig);
-    }
+    for (int g = 0; g < kNG; g++) zsum[g] = __shfl_sync(0xffffffffu, cz[0], 4 * g + tig);
     __syncthreads();                                     // stages are free now
     constexpr int kWarps = kThreads / 32;
     float *mo = reinterpret_cast<float *>(sh.stage[0][0]);       // [warp][head][128]
@@ -435,9 +542,9 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
     constexpr float kCodeScale = 262144.f;                       // 2^18
 #pragma unroll
     for (int mt = 0; mt < 8; mt++) {
-        const float z = zsum[mt >> 1];
-        mo[(warp * 4 + tig) * kD + 16 * mt + gid] = fmaf(co[mt][0] + co[mt][1], kCodeScale, z);
-        mo[(warp * 4 + tig) * kD + 16 * mt + gid + 8] = fmaf(co[mt][2] + co[mt][3], kCodeScale, z);
+        const int pp = mt >> 2, ca = 64 * pp + 8 * (mt & 3) + gid;
+        mo[(warp * 4 + tig) * kD + ca] = fmaf(co[mt][0], kCodeScale, zsum[2 * pp]);
+        mo[(warp * 4 + tig) * kD + ca + 32] = fmaf(co[mt][3], kCodeScale, zsum[2 * pp + 1]);
     }
     if (gid == 0) {
         mml[(warp * 4 + tig) * 2] = m_run;
@@ -463,7 +570,7 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
         if (c == 0) part_ml[row] = make_float2(M, L);
     }
     merge_unit_if_last<4, kThreads>(part_o, part_ml, S, qrow0, out, counters + unit,
-                          reinterpret_cast<float *>(sh.stage[2][0]));
+                                    reinterpret_cast<float *>(sh.stage[2][0]));
 }
 
 }  // namespace
@@ -485,7 +592,7 @@ cudaError_t launch_decode_mma(const kvq_cache &c, int Hq, const int32_t *idx, co
     dim3 grid((unsigned)S, (unsigned)c.n_kv_heads, (unsigned)c.batch);
     decode_mma_kernel<<<grid, kThreads, smem, st>>>(static_cast<const uint8_t *>(c.pages), c.seq_len,
                                                     c.n_kv_heads, c.capacity / kT, Hq, idx, qsel, qgsum, k,
-                                                    part_o, part_ml, S, out, unit_counter(c, 0, 0));
+                                                    part_o, part_ml, S, out, unit_counter(c, 0, 0), c.status);
     return cudaGetLastError();
 }
 

@@ -50,7 +50,7 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
                    int NB, int Hq, const int32_t *__restrict__ idx, const float *__restrict__ qsel,
                    const float *__restrict__ qgsum, int k, float *__restrict__ part_o,
                    float2 *__restrict__ part_ml, int S, float *__restrict__ out,
-                   uint32_t *__restrict__ counters) {
+                   uint32_t *__restrict__ counters, uint32_t *__restrict__ status) {
     constexpr int R = row_bytes(BITS);
     constexpr int FIX = fixed_bytes(BITS);
     constexpr int PER = 8 / BITS;
@@ -71,7 +71,14 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
     int *sgs = reinterpret_cast<int *>(sred + 4 * G);
 
     const size_t unit = (size_t)b * Hkv + h;
-    for (int i = tid; i < k; i += 128) sidx[i] = idx[unit * k + i];
+    // the list must be channel 0 followed by ascending channels in 1..127;
+    // another list is clamped into the page and raises KVQ_DEV_INDEX
+    bool bad = false;
+    for (int i = tid; i < k; i += 128) {
+        const int c = idx[unit * k + i];
+        bad |= (i == 0) ? c != 0 : (c <= idx[unit * k + i - 1] || c > kD - 1);
+        sidx[i] = min(max(c, 0), kD - 1);
+    }
     for (int e = tid; e < G * k; e += 128) {
         const int hl = e / k, i = e % k;
         sq[i * G + hl] = qsel[((size_t)b * Hq + (size_t)h * G + hl) * k + i];
@@ -80,7 +87,7 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
         const int hl = tid / kNG, gr = tid % kNG;
         sqg[gr * G + hl] = qgsum[((size_t)b * Hq + (size_t)h * G + hl) * kNG + gr];
     }
-    __syncthreads();
+    if (__syncthreads_or(bad) && tid == 0) atomicOr(status, (uint32_t)KVQ_DEV_INDEX);
     if (tid == 0) {
         // selected list positions 1..k-1 hold channels >= 1 ascending; group
         // gr spans positions [sgs[gr], sgs[gr+1])
@@ -156,7 +163,7 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
 #pragma unroll
                     for (int hl = 0; hl < G; hl++) d[hl] = fmaf(sq[i * G + hl], cf, d[hl]);
                 }
-                const uint32_t sz = kmeta[gr * kT + t];
+                const uint32_t sz = kmeta[meta_word(gr, t)];
                 const float sg = h2f_lo(sz), zg = h2f_hi(sz);
 #pragma unroll
                 for (int hl = 0; hl < G; hl++) sc[hl] = fmaf(sg, d[hl], fmaf(zg, sqg[gr * G + hl], sc[hl]));
@@ -191,7 +198,7 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
 #pragma unroll
                 for (int e = 0; e < 32 / BITS; e++) {
                     const int t = tb * PER + e;
-                    const uint32_t sz = vmeta[vg * kT + t];
+                    const uint32_t sz = vmeta[meta_word(vg, t)];
                     const float v = fmaf(h2f_lo(sz), (float)((w >> (e * BITS)) & CMASK), h2f_hi(sz));
 #pragma unroll
                     for (int hl = 0; hl < G; hl++) {
@@ -230,7 +237,7 @@ cudaError_t launch_simt_t(const kvq_cache &c, int Hq, const int32_t *idx, const 
     dim3 grid((unsigned)S, (unsigned)c.n_kv_heads, (unsigned)c.batch);
     fn<<<grid, 128, smem, st>>>(static_cast<const uint8_t *>(c.pages), c.seq_len, c.n_kv_heads,
                                 c.capacity / kT, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out,
-                                unit_counter(c, 0, 0));
+                                unit_counter(c, 0, 0), c.status);
     return cudaGetLastError();
 }
 

@@ -24,6 +24,12 @@ __host__ __device__ constexpr int off_ch0(int bits) { return 256 * row_bytes(bit
 __host__ __device__ constexpr int off_kmeta(int bits) { return off_ch0(bits) + 256; }
 __host__ __device__ constexpr int off_vmeta(int bits) { return off_kmeta(bits) + 2048; }
 __host__ __device__ constexpr int page_bytes(int bits) { return off_vmeta(bits) + 2048; }
+// word index of the {scale, zero} pair of token t (0..127), group g (0..3)
+// inside a page's key or value metadata block (chunks of 4 tokens are stored
+// XOR-permuted within blocks of 8 chunks, see include/kvq.h)
+__host__ __device__ constexpr int meta_word(int g, int t) {
+    return 128 * g + 4 * ((t >> 2) ^ (((t >> 5) & 3) ^ ((g & 1) << 2))) + (t & 3);
+}
 // bytes from the value codes to the end of the page: what every decode step
 // reads in full (value codes, channel 0, key and value metadata)
 __host__ __device__ constexpr int fixed_bytes(int bits) { return page_bytes(bits) - off_vcodes(bits); }

@@ -26,6 +26,8 @@ KVQ_OK = 0
 KVQ_DTYPE_F32 = 0
 KVQ_DTYPE_BF16 = 1
 KVQ_DEV_CAPACITY = 1
+KVQ_DEV_TIMEOUT = 2
+KVQ_DEV_INDEX = 4
 HEAD_DIM = 128
 GROUP = 32
 BLOCK_TOKENS = 128

@@ -175,8 +175,11 @@ void orc_quantize_group(const double *x, int len, int levels,
 /*   [0, 128R)            key codes, row r = channel r (row 0 unused, zero)  */
 /*   [128R, 256R)         value codes, row r = channel r                     */
 /*   [256R, 256R+256)     channel 0 of K' as bf16, one per token             */
-/*   next 2048 bytes      key metadata  [group][token] {fp16 scale, fp16 zero}*/
+/*   next 2048 bytes      key metadata: 512 words {fp16 scale, fp16 zero}      */
 /*   next 2048 bytes      value metadata, same shape                         */
+/*   metadata word of token t, group g: 128g + 4*sw(g, t/4) + t%4 with       */
+/*   sw(g, c) = c XOR ((c/8) XOR 4*(g%2)) (chunks of 4 tokens XOR-permuted    */
+/*   within blocks of 8 chunks).                                             */
 /*   codes: token t of the page sits in byte t*bits/8 of its row, at bit     */
 /*   (t mod (8/bits))*bits (least significant first).                        */
 /* ------------------------------------------------------------------------ */
@@ -197,6 +200,13 @@ static int get_code(const uint8_t *row, int bits, int t)
 {
     int per = 8 / bits;
     return (row[t / per] >> ((t % per) * bits)) & ((1 << bits) - 1);
+}
+
+static int meta_word_index(int g, int t)
+{
+    int chunk = t / 4;
+    int perm = chunk ^ ((chunk / 8) ^ (4 * (g % 2)));
+    return 128 * g + 4 * perm + t % 4;
 }
 
 static void put_u16(uint8_t *p, uint16_t v) { p[0] = (uint8_t)(v & 0xFF); p[1] = (uint8_t)(v >> 8); }
@@ -229,14 +239,14 @@ void orc_append_unit(uint8_t *unit, int bits, long pos0, long n,
             orc_quantize_group(k + c0, len, levels, &s16, &z16, codes);
             for (int c = 0; c < len; c++)
                 put_code(kcodes + (long)(c0 + c) * R, bits, t, codes[c]);
-            put_u16(kmeta + 4 * (g * ORC_T + t), s16);
-            put_u16(kmeta + 4 * (g * ORC_T + t) + 2, z16);
+            put_u16(kmeta + 4 * meta_word_index(g, t), s16);
+            put_u16(kmeta + 4 * meta_word_index(g, t) + 2, z16);
             /* values: group g covers channels 32g .. 32g+31 */
             orc_quantize_group(v + g * ORC_G, ORC_G, levels, &s16, &z16, codes);
             for (int c = 0; c < ORC_G; c++)
                 put_code(vcodes + (long)(g * ORC_G + c) * R, bits, t, codes[c]);
-            put_u16(vmeta + 4 * (g * ORC_T + t), s16);
-            put_u16(vmeta + 4 * (g * ORC_T + t) + 2, z16);
+            put_u16(vmeta + 4 * meta_word_index(g, t), s16);
+            put_u16(vmeta + 4 * meta_word_index(g, t) + 2, z16);
         }
     }
 }
@@ -254,14 +264,14 @@ void orc_dequant_unit(const uint8_t *unit, int bits, long n, double *Khat, doubl
         kh[0] = orc_bf16_to_f64(get_u16(ch0 + 2 * t));
         for (int c = 1; c < ORC_D; c++) {
             int g = c / ORC_G;
-            double s = orc_f16_to_f64(get_u16(kmeta + 4 * (g * ORC_T + t)));
-            double z = orc_f16_to_f64(get_u16(kmeta + 4 * (g * ORC_T + t) + 2));
+            double s = orc_f16_to_f64(get_u16(kmeta + 4 * meta_word_index(g, t)));
+            double z = orc_f16_to_f64(get_u16(kmeta + 4 * meta_word_index(g, t) + 2));
             kh[c] = s * get_code(kcodes + (long)c * R, bits, t) + z;
         }
         for (int c = 0; c < ORC_D; c++) {
             int g = c / ORC_G;
-            double s = orc_f16_to_f64(get_u16(vmeta + 4 * (g * ORC_T + t)));
-            double z = orc_f16_to_f64(get_u16(vmeta + 4 * (g * ORC_T + t) + 2));
+            double s = orc_f16_to_f64(get_u16(vmeta + 4 * meta_word_index(g, t)));
+            double z = orc_f16_to_f64(get_u16(vmeta + 4 * meta_word_index(g, t) + 2));
             vh[c] = s * get_code(vcodes + (long)c * R, bits, t) + z;
         }
     }

@@ -319,3 +319,40 @@ def test_decode_writes_stay_in_bounds(name, n_ctx, bits, g):
     ref, _, _ = case.oracle_decode(q, wl.batch - 1, wl.n_kv_heads - 1, 0.4)
     emax, _ = rel_errors(out[-1, -g:].cpu().numpy(), ref)
     assert emax <= TOL_MAX
+
+
+@pytest.mark.parametrize("bits,g", [(2, 4), (4, 4), (2, 2)])
+def test_decode_rejects_malformed_channel_list(bits, g):
+    """A channel list that is not 0 followed by ascending channels in 1..127
+    raises KVQ_DEV_INDEX; a valid list afterwards still decodes correctly and
+    raises no flag."""
+    wl = W.workload("llama8b_b8_32k", batch=1, bits=bits, n_q_heads=8 * g)
+    case = Case(wl, n_ctx=260)
+    cache = case.gpu_cache()
+    q = case.q(0)
+    sel = kvq.select_channels(cache, to_dev(q, "bf16"), dev64(case.Ai), 0.5)
+    assert kvq.read_status(cache) == 0
+    good = sel.idx.clone()
+    for bad in ("duplicate", "descending", "out_of_range", "first_not_zero"):
+        idx = good.clone()
+        if bad == "duplicate":
+            idx[0, 3, 5] = idx[0, 3, 4]
+        elif bad == "descending":
+            idx[0, 0, 1:] = idx[0, 0, 1:].flip(0)
+        elif bad == "out_of_range":
+            idx[0, 7, -1] = 128
+        else:
+            idx[0, 2, 0] = 1
+        sel.idx.copy_(idx)
+        out = kvq.decode_attn(cache, sel)
+        torch.cuda.synchronize()
+        assert kvq.read_status(cache) & kvq.KVQ_DEV_INDEX, bad
+        assert not cache.status[1:].any()
+        cache.status.zero_()
+    sel.idx.copy_(good)
+    out = kvq.decode_attn(cache, sel).cpu().numpy()
+    assert kvq.read_status(cache) == 0
+    for h in range(wl.n_kv_heads):
+        ref, _, _ = case.oracle_decode(q, 0, h, 0.5)
+        emax, emean = rel_errors(out[0, h * g:(h + 1) * g], ref)
+        assert emax <= TOL_MAX and emean <= TOL_MEAN

@@ -96,10 +96,17 @@ def test_page_layout_hand_computed(bits):
     levels = (1 << bits) - 1
     s_exp = orc.f16_rne(np.array([3.0 / levels]))[0]
     for g in range(4):
-        off = 4 * (g * 128 + t)
+        # token 2 is in chunk 0 of block 0: permuted chunk 0 ^ (0 ^ 4 (g % 2))
+        chunk = 0 ^ (4 if g % 2 else 0)
+        off = 4 * (128 * g + 4 * chunk + t % 4)
         assert _u16(pg, kmeta + off) == s_exp
         assert _u16(pg, kmeta + off + 2) == 0
         assert _u16(pg, vmeta + off) == s_exp
+    # a token in block 3 of the chunks (t = 101: chunk 25, 25 ^ (3 ^ 4) = 30 in odd groups)
+    unit2 = orc.new_unit(128, bits)
+    orc.append_unit(unit2, bits, 101, k[None], v[None])
+    assert _u16(unit2[0], kmeta + 4 * (128 * 1 + 4 * 30 + 1)) == s_exp
+    assert _u16(unit2[0], kmeta + 4 * (128 * 2 + 4 * (25 ^ 3) + 1)) == s_exp
     # everything else stays zero; the other page untouched
     assert not unit[0].any()
     # row 0 of the key codes is never written
