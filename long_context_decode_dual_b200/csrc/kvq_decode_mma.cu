@@ -3,8 +3,8 @@
 //
 // "Dual-QK: Sharp Queries and Flat Keys for Prunable 2-bit KV Caches":
 //   §3.2 scores over the retained channels only, 1/sqrt(d) with the full d;
-//   §3.3 only the 32-byte key rows selected by the shared mask are copied
-//        from each 128-token page; values and metadata are read in full;
+//   §3.3 only the key rows selected by the shared mask are read from each
+//        128-token page; values and metadata are read in full;
 //   §3.4 one softmax over every token (online per warp, merged per CTA and
 //        then across CTAs), followed by value aggregation.
 //
@@ -15,23 +15,28 @@
 // Codes stay exact: a 2-bit field masked in place inside a 16-bit half is an
 // fp16 subnormal equal to code * 2^(pos-24), so unpacking is one AND per two
 // codes; the power of two is compensated exactly on the other operand or in
-// fp32 afterwards.  Query and softmax weights are split into fp16 hi + lo
-// parts, giving near-fp32 operands.  Score MMAs put the parts in the two
-// columns of each head (n = 8 = 4 heads x {hi, lo}) and apply each key
-// group's per-token scale in fp32 afterwards; value MMAs take a group pair
-// per tile (rows: 8 channels of each group, columns: 4 heads x 2 groups) and
-// run hi and lo as two MMAs, so the per-token value scale is folded into the
-// weights once per group.  The value zero-point term sum_t p(t) z(t) is one
-// more MMA pair.
+// fp32 afterwards.  The query is split into fp16 hi + lo parts, which occupy
+// the two columns of each head in the score MMAs (n = 8 = 4 heads x {hi,lo}):
+// scores need near-fp32 operands because the softmax exponentiates them.  The
+// score k-steps run over all 128 channel rows of a page with q' = 0 on the
+// channels that are not selected, so every k-step lies inside one key group
+// and its per-token scale is applied in fp32 afterwards.  Softmax weights
+// enter the value MMAs as fp16 (the usual flash-attention rounding of P; the
+// error it adds is below 6e-4 of the output's largest entry); value MMAs take
+// a group pair per tile (rows: 8 channels of each group, columns: 4 heads x 2
+// groups) so the per-token value scale is folded into the weights once per
+// group.  The value zero-point term sum_t p(t) z(t) is one more MMA.
 //
 // Work split: one CTA = one (sequence, KV head, split of the context), eight
 // warps in four pairs.  A pair processes one 128-token page at a time from a
-// two-stage ring filled by bulk asynchronous copies (one for the contiguous
-// tail of the page, one per run of consecutive selected key rows) completing
-// on an mbarrier; warp w of the pair takes half w of every 16-token word of
-// the page (64 tokens) and keeps its own online softmax.  Selected key rows
-// land in fixed slots: group g owns slots 32g..32g+31, filled in ascending
-// channel order, so every score k-step (16 slots) lies inside one group.
+// two-stage ring filled by bulk asynchronous copies completing on an
+// mbarrier: key rows are copied in 64-byte chunks (two rows, the unit in which
+// the memory system fetches anyway) as a few runs of chunks that hold a
+// selected row, into their own place in the stage, and the tail of the page
+// (value codes, channel 0, metadata) in one copy.  Warp w of the pair takes
+// half w of every 16-token word of the page (64 tokens) and keeps its own
+// online softmax; its softmax weights pass from the score layout to the value
+// layout through a small buffer of its own.
 #include "kvq_internal.cuh"
 
 namespace kvq {
@@ -39,25 +44,28 @@ namespace {
 
 constexpr int kPairs = 4;
 constexpr int kThreads = 64 * kPairs;
-static_assert(kThreads == 8 * 32, "one warp per score k-step in the prologue");
-constexpr int kSlotBytes = 128 * 32;              // 4 groups x 32 slots x 32 B
+constexpr int kWarps = kThreads / 32;
+static_assert(kWarps == 8, "one warp per score k-step in the prologue");
+constexpr int kKeyBytes = 128 * 32;               // key code rows of a page
 constexpr int kFixBytes = fixed_bytes(2);         // value codes, ch0, metadata
-constexpr int kStageBytes = kSlotBytes + kFixBytes;
-constexpr int kMaxRuns = 127;
+constexpr int kStageBytes = kKeyBytes + kFixBytes;
+static_assert(kStageBytes == page_bytes(2), "a stage holds one page image");
+constexpr int kChunks = kKeyBytes / 64;           // 64-byte chunks of key rows
+constexpr int kMaxCopies = kChunks / 2 + 2;       // runs after gap filling, plus the tail
 constexpr uint32_t kWaitPolls = 1u << 20;         // bound on mbarrier polls per stage
 
 struct __align__(16) MmaShared {
     uint8_t stage[kPairs][2][kStageBytes];
     uint64_t mbar[kPairs][2];
-    uint32_t run[kMaxRuns];            // src row | dst slot << 7 | rows << 14
-    int run_pos[kD];                   // first selected position of each run
+    uint4 pex[kWarps][4][8];           // per warp: fp16 softmax weights [head][8-token block]
+    uint2 copy[kMaxCopies];            // {byte offset in the page, bytes}
     uint2 bq[8][32];                   // score-MMA B fragments per k-step and lane
     float q[4][kD];                    // qsel of the 4 heads, by selected position
     float qg[4][kNG];
-    int slot_pos[kD];                  // slot -> position in the selected list, -1 = pad
-    int nks[kNG];                      // score k-steps per key group (0, 1 or 2)
-    int run_warp[4];
-    int n_runs;
+    int chan_pos[kD];                  // channel -> position in the selected list, -1 = not selected
+    uint32_t touched[2];               // chunk bitmask halves
+    uint32_t tx_bytes;
+    int n_copies;
 };
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -67,6 +75,16 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
         "{%0,%1,%2,%3};\n"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// the same with a zero accumulator in
+__device__ __forceinline__ void mma16816_z(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                           uint32_t a3, uint32_t b0, uint32_t b1) {
+    const float z = 0.f;
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};\n"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(z));
 }
 
 __device__ __forceinline__ void pair_sync(int pair) {
@@ -124,12 +142,6 @@ __device__ __forceinline__ uint16_t f16_part(float x, int part) {
 // 4-token metadata chunk c of group g (the page format's XOR permutation)
 __device__ __forceinline__ int meta_chunk(int g, int c) { return c ^ (((c >> 3) & 3) ^ ((g & 1) << 2)); }
 
-// position of local token l (0..63) in a warp's softmax-weight exchange
-// buffer, and the start of head h's block (skews keep both access patterns
-// free of bank conflicts)
-__device__ __forceinline__ int pex_pos(int l) { return l + 4 * (l >> 4); }
-__device__ __forceinline__ int pex_head(int h) { return 96 * h + ((h & 1) ? 4 : 0) + ((h & 2) ? 16 : 0); }
-
 __global__ void __launch_bounds__(kThreads, 2)
 decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len, int Hkv,
                   int NB, int Hq, const int32_t *__restrict__ idx, const float *__restrict__ qsel,
@@ -141,105 +153,93 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
 
     const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int pair = warp >> 1, half = warp & 1, pt = tid & 63;   // pt: thread within the pair
+    const int pair = warp >> 1, half = warp & 1;
     const int gid = lane >> 2, tig = lane & 3;
     const size_t unit = (size_t)b * Hkv + h;
     const size_t qrow0 = (size_t)b * Hq + (size_t)h * 4;
 
     // ------------------------------------------------------------ prologue
-    // Selected positions 1..k-1 hold channels >= 1 ascending, so each group is
-    // one contiguous run of positions: a channel's slot is 32g + (its position
-    // - the first position of its group).  Runs of consecutive channels inside
-    // a group become one bulk copy each.
     for (int e = tid; e < 4 * k; e += kThreads) {
         const int hl = e / k, i = e % k;
         sh.q[hl][i] = qsel[(qrow0 + hl) * k + i];
     }
     if (tid < 4 * kNG) sh.qg[tid / kNG][tid % kNG] = qgsum[qrow0 * kNG + tid];
-    if (tid < kD) sh.slot_pos[tid] = -1;
-    if (tid < kNG) sh.nks[tid] = 0;
+    if (tid < kD) sh.chan_pos[tid] = -1;
     if (tid < 2 * kPairs) mbar_init(smem_u32(&sh.mbar[tid >> 1][tid & 1]), 1);
     // the list must be channel 0 followed by ascending channels in 1..127;
-    // any other list copies no key rows and raises KVQ_DEV_INDEX
+    // any other list reads no key rows and raises KVQ_DEV_INDEX
     const int32_t *sel = idx + unit * k;
-    int my_c = -1, prev_c = -2;
+    int my_c = -1;
     bool bad = false;
     if (tid < k) {
-        const int c = sel[tid];
-        if (tid == 0) {
-            bad = c != 0;
-        } else {
-            prev_c = sel[tid - 1];
-            bad = c <= prev_c || c > kD - 1;
-            my_c = c;
-        }
+        my_c = sel[tid];
+        bad = (tid == 0) ? my_c != 0 : (my_c <= sel[tid - 1] || my_c > kD - 1);
     }
     const bool any_bad = __syncthreads_or(bad);
-    if (any_bad) my_c = -1;
     if (any_bad && tid == 0) atomicOr(status, (uint32_t)KVQ_DEV_INDEX);
-    const int k_rows = any_bad ? 0 : k - 1;
-    const bool run_start = my_c >= 0 && (tid == 1 || prev_c != my_c - 1 || (my_c & 31) == 0);
-    if (my_c >= 0) atomicAdd(&sh.nks[my_c >> 5], 1);          // counts for now
-    unsigned start_mask = 0;
-    if (tid < kD) {
-        start_mask = __ballot_sync(0xffffffffu, run_start);
-        if (lane == 0) sh.run_warp[warp] = __popc(start_mask);
-    }
-    __syncthreads();
-    int my_slot = -1, my_run = -1;
-    if (my_c >= 0) {
-        const int g = my_c >> 5;
-        int start = 1;
-        for (int gg = 0; gg < g; gg++) start += sh.nks[gg];
-        my_slot = 32 * g + (tid - start);
-        sh.slot_pos[my_slot] = tid;
-        if (run_start) {
-            my_run = __popc(start_mask & ((1u << lane) - 1u));
-            for (int w = 0; w < warp; w++) my_run += sh.run_warp[w];
-            sh.run_pos[my_run] = tid;
-        }
-    }
-    if (tid == 0) sh.n_runs = sh.run_warp[0] + sh.run_warp[1] + sh.run_warp[2] + sh.run_warp[3];
-    __syncthreads();
-    if (my_run >= 0) {
-        const int next = (my_run + 1 < sh.n_runs) ? sh.run_pos[my_run + 1] : k_rows + 1;
-        sh.run[my_run] = (uint32_t)my_c | ((uint32_t)my_slot << 7) | ((uint32_t)(next - tid) << 14);
-    }
-    if (tid < kNG) sh.nks[tid] = (sh.nks[tid] + 15) >> 4;       // counts -> k-steps
-    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    if (!any_bad && tid < k) sh.chan_pos[my_c] = tid;
     __syncthreads();
 
-    // score-MMA B fragments: column gid = (head gid>>1, part gid&1); k-slots
-    // 2tig, 2tig+1, 2tig+8, 2tig+9 of a step = slots +tig, +tig+4, +tig+8, +tig+12
-    // (this slot order makes the code loads bank-conflict free); kept in
-    // shared memory as one 8-byte word per k-step and lane
+    // score-MMA B fragments of k-step ks (channels 16ks..16ks+15): column gid =
+    // (head gid>>1, part gid&1); k-slots 2tig, 2tig+1, 2tig+8, 2tig+9 are
+    // channels +tig, +tig+4, +tig+8, +tig+12 (this order makes the code loads
+    // bank-conflict free).  Channel 0 and unselected channels get q' = 0.
     const int hh = gid >> 1, part = gid & 1;
     {
-        const int ks = tid >> 5;                     // 8 warps: one k-step each
-        const int base = 32 * (ks >> 1) + 16 * (ks & 1);
+        const int ks = warp;
         uint32_t w[2];
 #pragma unroll
         for (int r = 0; r < 2; r++) {
-            const int s0 = base + tig + 8 * r, s1 = s0 + 4;
-            const int p0 = sh.slot_pos[s0], p1 = sh.slot_pos[s1];
-            const float q0 = p0 >= 0 ? sh.q[hh][p0] : 0.f;
-            const float q1 = p1 >= 0 ? sh.q[hh][p1] : 0.f;
+            const int c0 = 16 * ks + tig + 8 * r, c1 = c0 + 4;
+            const int p0 = sh.chan_pos[c0], p1 = sh.chan_pos[c1];
+            const float q0 = p0 >= 1 ? sh.q[hh][p0] : 0.f;
+            const float q1 = p1 >= 1 ? sh.q[hh][p1] : 0.f;
             w[r] = (uint32_t)f16_part(q0, part) | ((uint32_t)f16_part(q1, part) << 16);
         }
         sh.bq[ks][lane] = make_uint2(w[0], w[1]);
     }
+    // 64-byte chunks of key rows that hold a selected row
+    if (tid < kChunks) {
+        const bool t = sh.chan_pos[2 * tid] >= 1 || sh.chan_pos[2 * tid + 1] >= 1;
+        const unsigned m = __ballot_sync(0xffffffffu, t);
+        if (lane == 0) sh.touched[warp] = m;
+    }
     __syncthreads();
-    int nks[kNG];
-#pragma unroll
-    for (int g = 0; g < kNG; g++) nks[g] = sh.nks[g];
+    if (tid == 0) {
+        // copy list: runs of touched chunks, single untouched chunks between
+        // two touched ones filled in (one copy instead of two); a run that
+        // reaches the last chunk continues through the page tail
+        const uint64_t T = (uint64_t)sh.touched[0] | ((uint64_t)sh.touched[1] << 32);
+        uint64_t M = T | ((T << 1) & (T >> 1));
+        const bool tail_joined = (M >> 63) & 1u;
+        int n = 0;
+        uint32_t bytes = 0;
+        while (M) {
+            const int st = __ffsll((long long)M) - 1;
+            const uint64_t inv = ~(M >> st);
+            const int len = inv ? __ffsll((long long)inv) - 1 : kChunks - st;
+            uint32_t sz = 64u * (uint32_t)len;
+            if (st + len == kChunks) sz += (uint32_t)kFixBytes;
+            sh.copy[n++] = make_uint2(64u * (uint32_t)st, sz);
+            bytes += sz;
+            M = (len == kChunks) ? 0ull : (M & ~(((1ull << len) - 1ull) << st));
+        }
+        if (!tail_joined) {
+            sh.copy[n++] = make_uint2((uint32_t)kKeyBytes, (uint32_t)kFixBytes);
+            bytes += (uint32_t)kFixBytes;
+        }
+        sh.n_copies = n;
+        sh.tx_bytes = bytes;
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    __syncthreads();
+
     // zero-point and channel-0 coefficients of head tig, pre-scaled to the
     // base-2 score domain
     float qg_t[kNG];
 #pragma unroll
     for (int g = 0; g < kNG; g++) qg_t[g] = sh.qg[tig][g] * kScoreScaleLog2;
     const float q0_t = sh.q[tig][0] * kScoreScaleLog2;
-    const int n_runs = sh.n_runs;
-    const uint32_t tx_bytes = 32u * (uint32_t)k_rows + (uint32_t)kFixBytes;
 
     // ------------------------------------------------------------ pages
     const int len = min(max(seq_len[b], 0), NB * kT);
@@ -248,21 +248,16 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
     const int blk0 = s * bps;
     const int blk1 = min(nblk, blk0 + bps);
 
-    // the pair's first warp stages a page: lane 0 arms the stage's barrier and
-    // copies the contiguous tail, the lanes then copy one run of selected key
-    // rows each
+    // one thread of the pair arms the stage's barrier and issues its copies
     auto issue = [&](int st, int blk) {
         const uint8_t *src = pages + (unit * NB + (size_t)blk) * page_bytes(2);
         const uint32_t dst = smem_u32(sh.stage[pair][st]);
         const uint32_t bar = smem_u32(&sh.mbar[pair][st]);
-        if (lane == 0) {
-            mbar_expect_tx(bar, tx_bytes);
-            bulk_g2s(dst + kSlotBytes, src + off_vcodes(2), (uint32_t)kFixBytes, bar);
-        }
-        __syncwarp();
-        for (int r = lane; r < n_runs; r += 32) {
-            const uint32_t w = sh.run[r];
-            bulk_g2s(dst + ((w >> 7) & 127u) * 32u, src + (w & 127u) * 32u, (w >> 14) * 32u, bar);
+        mbar_expect_tx(bar, sh.tx_bytes);
+        const int n = sh.n_copies;
+        for (int r = 0; r < n; r++) {
+            const uint2 c = sh.copy[r];
+            bulk_g2s(dst + c.x, src + c.x, c.y, bar);
         }
     };
 
@@ -277,25 +272,26 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
 #pragma unroll
     for (int r = 0; r < 4; r++) cz[r] = 0.f;
 
-    const uint32_t lane_row_off = 4u * gid;                  // word gid of a 32-byte code row
     const uint32_t half_sel = half ? 0x7632u : 0x5410u;      // this warp's 16-bit half of a word
     const uint32_t vx_sel = half ? 0x4332u : 0x4110u;        // {half, high byte of half}
     const float zmask = gid < 4 ? 1.f : 0.f;
+    uint4 *pexw = &sh.pex[warp][0][0];
 
     int it = 0;
     uint32_t late = 0;            // stages whose last wait gave up, with the parity waited for
+    const bool issuer = (tid & 63) == 0;
     const int first = blk0 + pair;
-    if (half == 0 && first < blk1) issue(0, first);
+    if (issuer && first < blk1) issue(0, first);
     for (int pg = first; pg < blk1; pg += kPairs, it++) {
         const int st = it & 1;
-        uint8_t *cur = sh.stage[pair][st];
+        const uint8_t *cur = sh.stage[pair][st];
         const uint32_t par = (uint32_t)(it >> 1) & 1u;
         late = mbar_wait_bounded(smem_u32(&sh.mbar[pair][st]), par, status)
                    ? late & ~(3u << (2 * st)) : (late & ~(3u << (2 * st))) | ((2u | par) << (2 * st));
         pair_sync(pair);                                     // both warps left the other stage
-        if (half == 0 && pg + kPairs < blk1) issue(st ^ 1, pg + kPairs);
+        if (issuer && pg + kPairs < blk1) issue(st ^ 1, pg + kPairs);
 
-        const uint8_t *vcodes = cur + kSlotBytes;
+        const uint8_t *vcodes = cur + kKeyBytes;
         const uint32_t *ch0w = reinterpret_cast<const uint32_t *>(vcodes + 128 * 32);
         const uint32_t *kmeta = reinterpret_cast<const uint32_t *>(vcodes + 128 * 32 + 256);
         const uint32_t *vmeta = kmeta + kNG * kT;
@@ -307,31 +303,31 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
             sc[i][0] = sc[i][1] = 0.f;
             zt[i][0] = zt[i][1] = 0.f;
         }
+        const uint8_t *kb = cur + tig * 32 + 4 * gid;
 #pragma unroll
         for (int g = 0; g < kNG; g++) {
-            if (nks[g] == 0) continue;
             float C[4][4];
 #pragma unroll
-            for (int i = 0; i < 4; i++) C[i][0] = C[i][1] = C[i][2] = C[i][3] = 0.f;
-#pragma unroll
             for (int j = 0; j < 2; j++) {
-                if (j >= nks[g]) break;
-                const uint8_t *sb = cur + (32 * g + 16 * j + tig) * 32 + lane_row_off;
+                const int ks = 2 * g + j;
+                const uint8_t *sb = kb + ks * 512;
                 const uint32_t Wa = *reinterpret_cast<const uint32_t *>(sb);
                 const uint32_t Wb = *reinterpret_cast<const uint32_t *>(sb + 4 * 32);
                 const uint32_t Wc = *reinterpret_cast<const uint32_t *>(sb + 8 * 32);
                 const uint32_t Wd = *reinterpret_cast<const uint32_t *>(sb + 12 * 32);
                 const uint32_t Xab = __byte_perm(Wa, Wb, half_sel), Xcd = __byte_perm(Wc, Wd, half_sel);
                 const uint32_t Yab = Xab >> 8, Ycd = Xcd >> 8;
-                const uint2 bb = sh.bq[2 * g + j][lane];
-                const uint32_t b0 = bb.x, b1 = bb.y;
+                const uint2 bb = sh.bq[ks][lane];
 #pragma unroll
                 for (int i = 0; i < 4; i++) {
                     const uint32_t x1 = (i & 2) ? Yab : Xab;
                     const uint32_t x2 = (i & 2) ? Ycd : Xcd;
                     const uint32_t m0 = 0x00030003u << (4 * (i & 1));
                     const uint32_t m1 = m0 << 2;
-                    mma16816(C[i], x1 & m0, x1 & m1, x2 & m0, x2 & m1, b0, b1);
+                    if (j == 0)
+                        mma16816_z(C[i], x1 & m0, x1 & m1, x2 & m0, x2 & m1, bb.x, bb.y);
+                    else
+                        mma16816(C[i], x1 & m0, x1 & m1, x2 & m0, x2 & m1, bb.x, bb.y);
                 }
             }
             // scale and zero-point of group g for the thread's 8 tokens
@@ -400,44 +396,32 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
             cz[0] *= alpha;
         }
 
-        // ---------------- softmax weights: score layout -> value layout,
-        // through this warp's half of the (now free) slot area
-        pair_sync(pair);                                     // both warps are done with the slots
-        float *pex = reinterpret_cast<float *>(cur) + 512 * half;
+        // ---------------- softmax weights: score layout -> value layout.
+        // Local token l = 8 * block + e; the value MMAs take tokens (f, f+4)
+        // of a block as one fp16 pair, scaled by 4^(3-f) to offset the code
+        // scale of field f; word f of (head, block) holds that pair.
         {
-            float *dst = pex + pex_head(tig) + pex_pos(8 * gid);
-            *reinterpret_cast<float4 *>(dst) = make_float4(sc[0][0], sc[0][1], sc[1][0], sc[1][1]);
-            *reinterpret_cast<float4 *>(dst + 4) = make_float4(sc[2][0], sc[2][1], sc[3][0], sc[3][1]);
+            uint32_t wv[4];
+#pragma unroll
+            for (int f = 0; f < 4; f++) {
+                const float F = (float)(1 << (2 * (3 - f)));
+                const int i0 = f >> 1, r0 = f & 1;           // token f = 2 i0 + r0, token f+4 = 2(i0+2) + r0
+                wv[f] = h2u(__floats2half2_rn(sc[i0][r0] * F, sc[i0 + 2][r0] * F));
+            }
+            pexw[tig * 8 + gid] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
         }
         __syncwarp();
         // value k-step j = 2u + v uses fields f0 = 2v (k-slots 2tig, 2tig+1) and
         // f1 = 2v+1 (k-slots 2tig+8, 2tig+9) of word 2tig+u's half, i.e. local
-        // tokens (f, f+4); weights are scaled by 4^(3-f) to offset the code scale
-        uint32_t ph[4][2], pl[4][2];
-        {
-            float pv[2][8];                    // head hh, local tokens 8(2tig+u) + j
+        // tokens (f, f+4) of block 2tig+u
+        uint32_t ph[4][2];
 #pragma unroll
-            for (int u = 0; u < 2; u++) {
-                const float *src = pex + pex_head(hh) + pex_pos(8 * (2 * tig + u));
-                const float4 v0 = *reinterpret_cast<const float4 *>(src);
-                const float4 v1 = *reinterpret_cast<const float4 *>(src + 4);
-                pv[u][0] = v0.x; pv[u][1] = v0.y; pv[u][2] = v0.z; pv[u][3] = v0.w;
-                pv[u][4] = v1.x; pv[u][5] = v1.y; pv[u][6] = v1.z; pv[u][7] = v1.w;
-            }
-#pragma unroll
-            for (int j = 0; j < 4; j++) {
-                const int u = j >> 1;
-#pragma unroll
-                for (int r = 0; r < 2; r++) {
-                    const int f = 2 * (j & 1) + r;
-                    const float F = (float)(1 << (2 * (3 - f)));
-                    const float xa = pv[u][f] * F, xb = pv[u][f + 4] * F;
-                    const __half2 hi = __floats2half2_rn(xa, xb);
-                    const float2 hf = __half22float2(hi);
-                    ph[j][r] = h2u(hi);
-                    pl[j][r] = h2u(__floats2half2_rn(xa - hf.x, xb - hf.y));
-                }
-            }
+        for (int u = 0; u < 2; u++) {
+            const uint4 w = pexw[hh * 8 + 2 * tig + u];
+            ph[2 * u][0] = w.x;
+            ph[2 * u][1] = w.y;
+            ph[2 * u + 1][0] = w.z;
+            ph[2 * u + 1][1] = w.w;
         }
 
         // ---------------- values: tile mt = group pair pp, rows 8 channels of
@@ -445,9 +429,9 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
 #pragma unroll
         for (int pp = 0; pp < 2; pp++) {
             const int gv = 2 * pp + part;
-            uint32_t bh[4][2], bl[4][2];
+            uint32_t bw[4][2];
             {
-                uint32_t vw[2][8];             // {s, z} of local tokens 8(2tig+u) + j, group gv
+                uint32_t vw[2][8];             // {s, z} of local tokens 8(2tig+u) + e, group gv
 #pragma unroll
                 for (int u = 0; u < 2; u++)
 #pragma unroll
@@ -463,10 +447,7 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
                     for (int r = 0; r < 2; r++) {
                         const int f = 2 * (j & 1) + r;
                         const __half2 sp = u2h(__byte_perm(vw[u][f], vw[u][f + 4], 0x5410));
-                        const __half2 P = u2h(ph[j][r]);
-                        const __half2 wh = __hmul2(P, sp);
-                        bh[j][r] = h2u(wh);
-                        bl[j][r] = h2u(__hfma2(u2h(pl[j][r]), sp, __hfma2(P, sp, __hneg2(wh))));
+                        bw[j][r] = h2u(__hmul2(u2h(ph[j][r]), sp));
                     }
                 }
             }
@@ -483,9 +464,7 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
                     const int u = j >> 1;
                     const uint32_t mA = 0x00030003u << (4 * (j & 1));
                     const uint32_t mB = mA << 2;
-                    const uint32_t a0 = x0[u] & mA, a1 = x1[u] & mA, a2 = x0[u] & mB, a3 = x1[u] & mB;
-                    mma16816(co[mt], a0, a1, a2, a3, bh[j][0], bh[j][1]);
-                    mma16816(co[mt], a0, a1, a2, a3, bl[j][0], bl[j][1]);
+                    mma16816(co[mt], x0[u] & mA, x1[u] & mA, x0[u] & mB, x1[u] & mB, bw[j][0], bw[j][1]);
                 }
             }
         }
@@ -512,12 +491,8 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
                     a[r] = h2u(__hmul2(u2h(__byte_perm(zw[u][f], zw[u][f + 4], 0x7632)), sc2));
                 }
                 mma16816(cz, a[0], 0u, a[1], 0u, ph[j][0], ph[j][1]);
-                mma16816(cz, a[0], 0u, a[1], 0u, pl[j][0], pl[j][1]);
             }
         }
-        // order this thread's generic accesses to the stage before the bulk
-        // copies that refill it
-        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
     }
     // a stage whose wait gave up may still receive bytes: wait once more
     // (bounded) before the staging memory is reused below
@@ -536,7 +511,6 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
 #pragma unroll
     for (int g = 0; g < kNG; g++) zsum[g] = __shfl_sync(0xffffffffu, cz[0], 4 * g + tig);
     __syncthreads();                                     // stages are free now
-    constexpr int kWarps = kThreads / 32;
     float *mo = reinterpret_cast<float *>(sh.stage[0][0]);       // [warp][head][128]
     float *mml = mo + kWarps * 4 * kD;                           // [warp][head][2]
     constexpr float kCodeScale = 262144.f;                       // 2^18
