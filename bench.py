@@ -267,7 +267,7 @@ def run_ours(args):
     kv_pool = [tuple(dev_in(t) for t in W.make_step_kv(wl, i)) for i in range(n_pool)]
     k = kvq.num_selected(wl.sparsity)
     tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
-    step = kvq.DecodeStep(cache, A, Ai, wl.sparsity, Hq, tdt)
+    step = kvq.DecodeStep(cache, A, Ai, wl.sparsity, Hq, tdt, fused=args.fused)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def stage(i):
@@ -429,6 +429,8 @@ def main():
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-comparator", dest="comparator", action="store_false")
+    ap.add_argument("--unfused", dest="fused", action="store_false",
+                    help="run the step as three launches (append, select, decode) instead of one")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="launch the step's kernels eagerly instead of replaying a CUDA graph")
     args = ap.parse_args()

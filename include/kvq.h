@@ -127,7 +127,8 @@ int kvq_cache_init(const kvq_cache *cache, kvq_stream_t stream);
  * min/max grid, round to nearest; channel-major 128-token pages).
  *
  *  K, V    [batch][n_kv_heads][n_new][128], dtype KVQ_DTYPE_F32 or _BF16
- *  A       [n_kv_heads][128][128] float64, row-major: K'[j] = sum_c K[c] A[c][j]
+ *  A       [n_kv_heads][128][128] float64, row-major, 16-byte aligned:
+ *          K'[j] = sum_c K[c] A[c][j]
  *          summed c = 0..127 as a chain of fused multiply-adds from 0.0
  *  Arithmetic (defines the stored bits): K' in float64; per token and group
  *  zero = fp16(min), scale = fp16((max-min)/(2^bits-1)) (fp16 rounding to
@@ -157,7 +158,8 @@ int kvq_num_selected(float sparsity, int head_dim);
  *
  *  q       [batch][n_q_heads][128], dtype F32 or BF16; query head h belongs
  *          to KV head h / g
- *  Ainvt   [n_kv_heads][128][128] float64, q'[j] = sum_c q[c] Ainvt[c][j]
+ *  Ainvt   [n_kv_heads][128][128] float64, row-major, 16-byte aligned:
+ *          q'[j] = sum_c q[c] Ainvt[c][j]
  *          (fma chain over c from 0.0), e^2 by an fma chain over h ascending
  *  idx     out [batch][n_kv_heads][k] int32: channel 0 and the k-1 channels of
  *          1..127 with the largest e^2 (ties to the lower index), ascending
@@ -183,10 +185,11 @@ size_t kvq_decode_workspace(const kvq_cache *cache, int n_q_heads, int k);
  * kvq_decode_attn -- attention of one decode query per head over every
  * cached token, reading only the selected key channels.  Dual-QK §3.2 (scores
  * use the retained channels, scaled by 1/sqrt(128) with the full dimension),
- * §3.3 (only the selected 32-byte key rows of each page are fetched; values
- * and metadata are read in full), §3.4 (one softmax over all tokens, then
- * value aggregation).  Realised as a split over the context (flash-decoding):
- * per split a running max, sum and output, then one exact merge.
+ * §3.3 (only key rows holding selected channels are fetched -- in 64-byte
+ * chunks of two rows, the unit the memory system fetches; values and
+ * metadata are read in full), §3.4 (one softmax over all tokens, then value
+ * aggregation).  Realised as a split over the context (flash-decoding): per
+ * split a running max, sum and output, then one exact merge.
  *
  *  score_h(t) = [qsel_h0 * ch0(t) + sum_g (scale_g(t) * sum_{c in S_g}
  *               qsel_hc * code_c(t) + zero_g(t) * qgsum_hg)] / sqrt(128)
@@ -195,13 +198,39 @@ size_t kvq_decode_workspace(const kvq_cache *cache, int n_q_heads, int k);
  *  idx, qsel, qgsum, k exactly as produced by kvq_select_channels
  *  ws      device workspace of at least kvq_decode_workspace() bytes,
  *          16-byte aligned; contents need no initialisation
- *  Arithmetic: float32 (tensor-core products of exact small integers and
- *  split float16 operands, float32 accumulation).
+ *  Arithmetic: float32 accumulation of tensor-core products of exact small
+ *  integers with the query as a float16 hi + lo pair and the softmax weights
+ *  as float16 (INT2, 4 query heads per KV head), or of CUDA-core float32
+ *  products (other shapes).
  *  Errors: KVQ_ERR_ARG, KVQ_ERR_SHAPE, KVQ_ERR_WORKSPACE, KVQ_ERR_ALIGN,
  *  KVQ_ERR_CUDA.
  */
 int kvq_decode_attn(const kvq_cache *cache, int n_q_heads, const int32_t *idx,
                     const float *qsel, const float *qgsum, int k, float *out,
+                    void *ws, size_t ws_bytes, kvq_stream_t stream);
+
+/*
+ * kvq_decode_step -- one whole decode step: kvq_append of the n_new new
+ * tokens, kvq_select_channels of the query, then kvq_decode_attn over every
+ * token including the new ones.  Same arguments, results and errors as those
+ * three calls made in that order on `stream` (idx / qsel / qgsum are written
+ * too), and the same stored bits.  With INT2 codes, 4 query heads per KV head
+ * and n_new <= 4 the step is one kernel launch: each CTA repeats the channel
+ * choice of its (sequence, KV head) with the same float64 arithmetic, and the
+ * CTA holding the last page appends the new tokens before reading it.
+ *
+ *  q       [batch][n_q_heads][128]; k_new, v_new [batch][n_kv_heads][n_new][128];
+ *          all of dtype KVQ_DTYPE_F32 or _BF16
+ *  A, Ainvt  as for kvq_append / kvq_select_channels (16-byte aligned)
+ *  idx, qsel, qgsum  outputs as for kvq_select_channels
+ *  out, ws, ws_bytes  as for kvq_decode_attn (kvq_decode_workspace() with the
+ *          k of `sparsity`)
+ *  Errors: the union of the three calls' errors.
+ */
+int kvq_decode_step(const kvq_cache *cache, const void *q, const void *k_new,
+                    const void *v_new, int dtype, int n_q_heads, int n_new,
+                    const double *A, const double *Ainvt, float sparsity,
+                    int32_t *idx, float *qsel, float *qgsum, float *out,
                     void *ws, size_t ws_bytes, kvq_stream_t stream);
 
 /* Workspace bytes for kvq_bf16_decode_attn on the current device. */

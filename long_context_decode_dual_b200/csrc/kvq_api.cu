@@ -88,7 +88,7 @@ int kvq_append(const kvq_cache *c, const void *K, const void *V, int dtype, int 
     if (st) return st;
     if (!K || !V || !A || n_new < 0) return KVQ_ERR_ARG;
     if (dtype != KVQ_DTYPE_F32 && dtype != KVQ_DTYPE_BF16) return KVQ_ERR_ARG;
-    if (!aligned(K, dtype_align(dtype)) || !aligned(V, dtype_align(dtype)) || !aligned(A, 8))
+    if (!aligned(K, dtype_align(dtype)) || !aligned(V, dtype_align(dtype)) || !aligned(A, 16))
         return KVQ_ERR_ALIGN;
     if (n_new > c->capacity) return KVQ_ERR_CAPACITY;
     if (n_new == 0) return KVQ_OK;
@@ -112,7 +112,7 @@ int kvq_select_channels(const kvq_cache *c, const void *q, int dtype, int n_q_he
     const int k = kvq_num_selected(sparsity, kD);
     if (k < 0) return KVQ_ERR_ARG;
     if (n_q_heads < 1 || n_q_heads % c->n_kv_heads || n_q_heads / c->n_kv_heads > 32) return KVQ_ERR_SHAPE;
-    if (!aligned(q, dtype_align(dtype)) || !aligned(Ainvt, 8) || !aligned(idx, 4) || !aligned(qsel, 4) ||
+    if (!aligned(q, dtype_align(dtype)) || !aligned(Ainvt, 16) || !aligned(idx, 4) || !aligned(qsel, 4) ||
         !aligned(qgsum, 4))
         return KVQ_ERR_ALIGN;
     if (k_out) *k_out = k;
@@ -138,6 +138,33 @@ int kvq_decode_attn(const kvq_cache *c, int n_q_heads, const int32_t *idx, const
     if (!ws || ws_bytes < decode_ws_bytes(*c, n_q_heads, S)) return KVQ_ERR_WORKSPACE;
     if (!aligned(ws, 16)) return KVQ_ERR_ALIGN;
     return cuda_status(launch_decode(*c, n_q_heads, idx, qsel, qgsum, k, out, ws, S, (cudaStream_t)stream));
+}
+
+int kvq_decode_step(const kvq_cache *c, const void *q, const void *k_new, const void *v_new, int dtype,
+                    int n_q_heads, int n_new, const double *A, const double *Ainvt, float sparsity,
+                    int32_t *idx, float *qsel, float *qgsum, float *out, void *ws, size_t ws_bytes,
+                    kvq_stream_t stream) {
+    int st = check_cache(c);
+    if (st) return st;
+    if (!q || !A || !Ainvt || !idx || !qsel || !qgsum || !out || n_new < 0) return KVQ_ERR_ARG;
+    if (n_new > 0 && (!k_new || !v_new)) return KVQ_ERR_ARG;
+    if (dtype != KVQ_DTYPE_F32 && dtype != KVQ_DTYPE_BF16) return KVQ_ERR_ARG;
+    const int k = kvq_num_selected(sparsity, kD);
+    if (k < 0) return KVQ_ERR_ARG;
+    st = check_decode_args(c, n_q_heads, k);
+    if (st) return st;
+    const size_t al = dtype_align(dtype);
+    if (!aligned(q, al) || (n_new > 0 && (!aligned(k_new, al) || !aligned(v_new, al))) || !aligned(A, 16) ||
+        !aligned(Ainvt, 16) || !aligned(idx, 4) || !aligned(qsel, 4) || !aligned(qgsum, 4) || !aligned(out, 4))
+        return KVQ_ERR_ALIGN;
+    if (n_new > c->capacity) return KVQ_ERR_CAPACITY;
+    const int sms = num_sms();
+    if (sms <= 0) return KVQ_ERR_CUDA;
+    const int S = decode_splits(*c, n_q_heads, k, sms);
+    if (!ws || ws_bytes < decode_ws_bytes(*c, n_q_heads, S)) return KVQ_ERR_WORKSPACE;
+    if (!aligned(ws, 16)) return KVQ_ERR_ALIGN;
+    return cuda_status(launch_decode_step(*c, n_q_heads, q, k_new, v_new, dtype, n_new, A, Ainvt, k, idx, qsel,
+                                          qgsum, out, ws, S, (cudaStream_t)stream));
 }
 
 size_t kvq_bf16_decode_workspace(int B, int Hq, int Hkv, int N) {

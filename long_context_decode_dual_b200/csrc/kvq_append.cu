@@ -20,38 +20,6 @@ namespace {
 
 constexpr int kTile = 16;   // destination positions per CTA (multiple of 8)
 
-__device__ __forceinline__ double warp_min(double v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmin(v, __shfl_xor_sync(0xffffffffu, v, o));
-    return v;
-}
-__device__ __forceinline__ double warp_max(double v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
-    return v;
-}
-
-// Quantize value x of this lane against the group range (lanes of the warp;
-// `in_range` false leaves the lane out of min/max).  Returns the code and,
-// through s_bits / z_bits, the fp16 scale / zero-point bit patterns.
-template <int BITS>
-__device__ __forceinline__ uint32_t quantize_lane(double x, bool in_range, uint16_t &s_bits,
-                                                  uint16_t &z_bits) {
-    constexpr int L = (1 << BITS) - 1;
-    const double lo = warp_min(in_range ? x : __longlong_as_double(0x7ff0000000000000LL));
-    const double hi = warp_max(in_range ? x : __longlong_as_double(0xfff0000000000000LL));
-    const __half zh = __double2half(lo);
-    const __half sh = __double2half((hi - lo) / (double)L);
-    z_bits = __half_as_ushort(zh);
-    s_bits = __half_as_ushort(sh);
-    const double z = (double)__half2float(zh);
-    const double s = (double)__half2float(sh);
-    if (s == 0.0) return 0u;
-    double r = rint((x - z) / s);
-    r = fmin(fmax(r, 0.0), (double)L);
-    return (uint32_t)r;
-}
-
 // Merge the kTile codes of one channel row into its packed bytes.
 // `valid` has bit tt set for tile positions this call writes.
 template <int BITS>
@@ -187,11 +155,14 @@ append_kernel(uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len,
 }
 
 // Appends of a few tokens (a decode step adds one): one CTA per (sequence,
-// KV head) walks the new tokens in order, so code bytes shared by
-// neighbouring tokens are updated by one thread each.  A of the head is staged
-// in shared memory first (one cp.async burst instead of a DRAM round trip per
-// row of the fma chain).  The last CTA of a sequence to finish advances its
-// length, using the sequence's completion counter in the status array.
+// KV head, quantization group), so the key transform's columns -- and the
+// reads of A they need, 32 KB per CTA, staged with one cp.async burst -- are
+// spread over 4 * n_kv_heads * batch SMs.  Warp w transforms and quantizes new
+// token w (lane = channel of the group); the codes then go through shared
+// memory to one thread per channel row, which merges the new tokens into the
+// packed bytes in order (neighbouring tokens share bytes).  The last CTA of a
+// sequence to finish advances its length, using the sequence's completion
+// counter in the status array.
 constexpr int kSmallMax = 4;
 
 template <typename Tin, int BITS>
@@ -202,62 +173,72 @@ append_small_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len,
                     int n_new, int capacity) {
     constexpr int R = row_bytes(BITS);
     constexpr int PER = 8 / BITS;
-    extern __shared__ __align__(16) double As[];          // [128][128]
+    static_assert(kSmallMax * 32 == 128, "one warp per new token");
+    __shared__ __align__(16) double As[kD][kGroup];        // A[:, 32 grp .. 32 grp + 31]
     __shared__ double ks[kSmallMax][kD];
-    __shared__ double vs[kSmallMax][kD];
+    __shared__ uint8_t kcode[kSmallMax][kGroup];
+    __shared__ uint8_t vcode[kSmallMax][kGroup];
     __shared__ int s_len;
 
-    const int h = blockIdx.x, b = blockIdx.y, j = threadIdx.x;
-    const int lane = j & 31, grp = j >> 5;
-    const double *Ah = A + (size_t)h * kD * kD;
-    for (int e = j; e < kD * kD / 2; e += blockDim.x) cp_async16(As + 2 * e, Ah + 2 * e);
+    const int grp = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    const int j = grp * kGroup + lane;                     // this lane's channel
+    const double *Ah = A + (size_t)h * kD * kD + grp * kGroup;
+    for (int e = t; e < kD * kGroup / 2; e += 128) {
+        const int c = e >> 4, part = e & 15;
+        cp_async16(&As[c][2 * part], Ah + (size_t)c * kD + 2 * part);
+    }
     cp_async_commit();
     const size_t in_base = ((size_t)b * Hkv + h) * (size_t)n_new;
-    for (int e = j; e < n_new * kD; e += blockDim.x) {
-        ks[e / kD][e % kD] = in_to_double(K[in_base * kD + e]);
-        vs[e / kD][e % kD] = in_to_double(V[in_base * kD + e]);
-    }
-    if (j == 0) s_len = seq_len[b];
+    for (int e = t; e < n_new * kD; e += 128) ks[e / kD][e % kD] = in_to_double(K[in_base * kD + e]);
+    const double v = (w < n_new) ? in_to_double(V[(in_base + w) * kD + j]) : 0.0;
+    if (t == 0) s_len = seq_len[b];
     cp_async_wait<0>();
     __syncthreads();
     const int len = s_len;
     const bool ok = len >= 0 && len + n_new <= capacity;
+    uint8_t *unit = pages + ((size_t)b * Hkv + h) * NB * (size_t)page_bytes(BITS);
 
-    if (ok) {
-        uint8_t *unit = pages + ((size_t)b * Hkv + h) * NB * (size_t)page_bytes(BITS);
-        for (int i = 0; i < n_new; i++) {
-            const int pos = len + i, t = pos % kT;
-            uint8_t *page = unit + (size_t)(pos / kT) * page_bytes(BITS);
-            double x = 0.0;
-#pragma unroll 8
-            for (int c = 0; c < kD; c++) x = fma(ks[i][c], As[c * kD + j], x);
-            const int byte = t / PER, sh = (t % PER) * BITS;
-            const uint8_t clear = (uint8_t)~(((1u << BITS) - 1u) << sh);
-            uint16_t sb, zb;
-            const uint32_t kc = quantize_lane<BITS>(x, j != 0, sb, zb);
-            if (lane == 0)
-                reinterpret_cast<uint32_t *>(page + off_kmeta(BITS))[meta_word(grp, t)] = (uint32_t)sb | ((uint32_t)zb << 16);
-            if (j == 0) {
-                reinterpret_cast<uint16_t *>(page + off_ch0(BITS))[t] = __bfloat16_as_ushort(__double2bfloat16(x));
-            } else {
-                uint8_t *p = page + (size_t)j * R + byte;
-                *p = (uint8_t)((*p & clear) | (kc << sh));
+    if (ok && w < n_new) {                                 // uniform over the warp
+        const int pos = len + w, tt = pos % kT;
+        uint8_t *page = unit + (size_t)(pos / kT) * page_bytes(BITS);
+        // K'[t][j] = sum_c K[t][c] A[c][j], fma chain c = 0..127 from 0.0
+        double x = 0.0;
+#pragma unroll 16
+        for (int c = 0; c < kD; c++) x = fma(ks[w][c], As[c][lane], x);
+        uint16_t sb, zb;
+        kcode[w][lane] = (uint8_t)quantize_lane<BITS>(x, j != 0, sb, zb);
+        if (lane == 0)
+            reinterpret_cast<uint32_t *>(page + off_kmeta(BITS))[meta_word(grp, tt)] = (uint32_t)sb | ((uint32_t)zb << 16);
+        if (j == 0) reinterpret_cast<uint16_t *>(page + off_ch0(BITS))[tt] = __bfloat16_as_ushort(__double2bfloat16(x));
+        vcode[w][lane] = (uint8_t)quantize_lane<BITS>(v, true, sb, zb);
+        if (lane == 0)
+            reinterpret_cast<uint32_t *>(page + off_vmeta(BITS))[meta_word(grp, tt)] = (uint32_t)sb | ((uint32_t)zb << 16);
+    }
+    __syncthreads();
+    if (ok && t < 2 * kGroup) {
+        // thread t < 32: key row of channel j; 32 <= t < 64: value row
+        const bool val = t >= kGroup;
+        if (val || j != 0) {
+            for (int i = 0; i < n_new; i++) {
+                const int pos = len + i, tt = pos % kT;
+                const int byte = tt / PER, sh = (tt % PER) * BITS;
+                uint8_t *p = unit + (size_t)(pos / kT) * page_bytes(BITS) + (val ? off_vcodes(BITS) : 0) +
+                             (size_t)j * R + byte;
+                const uint8_t clear = (uint8_t)~(((1u << BITS) - 1u) << sh);
+                const uint32_t code = val ? vcode[i][lane] : kcode[i][lane];
+                *p = (uint8_t)((*p & clear) | (code << sh));
             }
-            const uint32_t vc = quantize_lane<BITS>(vs[i][j], true, sb, zb);
-            if (lane == 0)
-                reinterpret_cast<uint32_t *>(page + off_vmeta(BITS))[meta_word(grp, t)] = (uint32_t)sb | ((uint32_t)zb << 16);
-            uint8_t *p = page + off_vcodes(BITS) + (size_t)j * R + byte;
-            *p = (uint8_t)((*p & clear) | (vc << sh));
         }
-    } else if (j == 0) {
+    } else if (!ok && t == 0) {
         atomicOr(status, (uint32_t)KVQ_DEV_CAPACITY);
     }
 
     __syncthreads();
-    if (j == 0) {
+    if (t == 0) {
         __threadfence();
         const unsigned prev = atomicAdd(status + 1 + b, 1u);
-        if (prev == (unsigned)Hkv - 1u) {          // every head of sequence b has read its length
+        if (prev == (unsigned)(Hkv * kNG) - 1u) {   // every CTA of sequence b has read its length
             if (ok) seq_len[b] = len + n_new;
             atomicExch(status + 1 + b, 0u);
         }
@@ -277,12 +258,8 @@ cudaError_t launch_append_t(const kvq_cache &c, const void *K, const void *V, in
                             const double *A, cudaStream_t st) {
     const int NB = c.capacity / kT;
     if (n_new <= kSmallMax) {
-        constexpr int smem = kD * kD * (int)sizeof(double);
-        static std::atomic<uint64_t> done{0};
-        cudaError_t e = set_smem_once(append_small_kernel<Tin, BITS>, smem, done);
-        if (e != cudaSuccess) return e;
-        dim3 grid((unsigned)c.n_kv_heads, (unsigned)c.batch);
-        append_small_kernel<Tin, BITS><<<grid, 128, smem, st>>>(
+        dim3 grid((unsigned)kNG, (unsigned)c.n_kv_heads, (unsigned)c.batch);
+        append_small_kernel<Tin, BITS><<<grid, 128, 0, st>>>(
             static_cast<uint8_t *>(c.pages), c.seq_len, c.status, static_cast<const Tin *>(K),
             static_cast<const Tin *>(V), A, c.n_kv_heads, NB, n_new, c.capacity);
         return cudaGetLastError();

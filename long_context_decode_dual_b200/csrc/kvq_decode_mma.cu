@@ -1,10 +1,15 @@
 // Channel-skipping decode attention on the tensor cores: INT2 codes, four
-// query heads per KV head (the GQA 4:1 shape of the Dual-QK workloads).
+// query heads per KV head (the GQA 4:1 shape of the Dual-QK workloads), and
+// the whole decode step -- append, channel choice, attention -- fused into one
+// launch on the same page machinery.
 //
 // "Dual-QK: Sharp Queries and Flat Keys for Prunable 2-bit KV Caches":
-//   §3.2 scores over the retained channels only, 1/sqrt(d) with the full d;
-//   §3.3 only the key rows selected by the shared mask are read from each
-//        128-token page; values and metadata are read in full;
+//   §3.1 keys enter the cache transformed (K' = K A), queries are transformed
+//        by A^{-T}, so transformed scores equal the original ones;
+//   §3.2 Eq. 4: one channel mask per KV head from the pooled query energy;
+//        scores over the retained channels only, 1/sqrt(d) with the full d;
+//   §3.3 only the key rows selected by the mask are read from each 128-token
+//        page; values and metadata are read in full;
 //   §3.4 one softmax over every token (online per warp, merged per CTA and
 //        then across CTAs), followed by value aggregation.
 //
@@ -37,7 +42,22 @@
 // half w of every 16-token word of the page (64 tokens) and keeps its own
 // online softmax; its softmax weights pass from the score layout to the value
 // layout through a small buffer of its own.
+//
+// The fused step kernel runs as clusters of two CTAs, the two taking
+// consecutive splits of one (sequence, KV head).  CTA r of a cluster computes
+// q' for channels 64r..64r+63 (64 columns of A^{-T}, staged in shared memory;
+// the same fixed-order float64 arithmetic as kvq_select_channels) and their
+// pooled energies; after a cluster barrier both CTAs read the 128 energies and
+// all of q' through distributed shared memory and make the same channel
+// choice.  In the cluster whose splits receive the new tokens, CTA r also
+// transforms, quantizes and writes key groups 2r and 2r+1 of them (the
+// arithmetic of kvq_append; code bits are OR-ed into positions that are still
+// zero) before the same barrier, so the page owner stages those pages after
+// it.  (Pairs of CTAs pack the SMs' two CTA slots exactly; clusters of four
+// leave slots of some GPCs unused.)
 #include "kvq_internal.cuh"
+
+#include <cooperative_groups.h>
 
 namespace kvq {
 namespace {
@@ -45,7 +65,7 @@ namespace {
 constexpr int kPairs = 4;
 constexpr int kThreads = 64 * kPairs;
 constexpr int kWarps = kThreads / 32;
-static_assert(kWarps == 8, "one warp per score k-step in the prologue");
+static_assert(kWarps == 8, "one warp per score k-step in the plan");
 constexpr int kKeyBytes = 128 * 32;               // key code rows of a page
 constexpr int kFixBytes = fixed_bytes(2);         // value codes, ch0, metadata
 constexpr int kStageBytes = kKeyBytes + kFixBytes;
@@ -53,20 +73,51 @@ static_assert(kStageBytes == page_bytes(2), "a stage holds one page image");
 constexpr int kChunks = kKeyBytes / 64;           // 64-byte chunks of key rows
 constexpr int kMaxCopies = kChunks / 2 + 2;       // runs after gap filling, plus the tail
 constexpr uint32_t kWaitPolls = 1u << 20;         // bound on mbarrier polls per stage
+constexpr int kStepMaxNew = 4;                    // new tokens per fused step
+constexpr int kCluster = 2;                       // CTAs per cluster of the fused step
+constexpr int kCols = kD / kCluster;              // channels whose q' one CTA of a cluster computes
 
 struct __align__(16) MmaShared {
     uint8_t stage[kPairs][2][kStageBytes];
     uint64_t mbar[kPairs][2];
     uint4 pex[kWarps][4][8];           // per warp: fp16 softmax weights [head][8-token block]
-    uint2 copy[kMaxCopies];            // {byte offset in the page, bytes}
+    uint2 copy[kMaxCopies];            // {byte offset in the page, bytes}; the last one is the tail
     uint2 bq[8][32];                   // score-MMA B fragments per k-step and lane
     float q[4][kD];                    // qsel of the 4 heads, by selected position
     float qg[4][kNG];
     int chan_pos[kD];                  // channel -> position in the selected list, -1 = not selected
     uint32_t touched[2];               // chunk bitmask halves
-    uint32_t tx_bytes;
+    uint32_t tx_keys;                  // bytes of the key-chunk copies of one page
     int n_copies;
+    int warp_cnt[4];
+    int s_len;
+    double qp_own[4][kCols];           // fused step: q' of this CTA's channels (read by the cluster)
+    double e2_own[kCols];              // and their pooled energies
 };
+
+// Prologue scratch of the fused step.  No page copy has been issued yet, so
+// the staging memory P is free: P[0, 64K) holds A^{-T}[:, 64r..64r+63] and
+// later rows 64..127 of A[:, 64r..64r+63]; P[64K, 96K) rows 0..63 of the latter;
+// then energies and ranks.  Smaller arrays use the softmax exchange buffers
+// and the B-fragment table, which the page loop fills later.
+constexpr int kBlkRowBytes = kCols * (int)sizeof(double);        // 512
+constexpr int kOffAHi = 0;                                        // A rows 64..127
+constexpr int kOffALo = kD * kBlkRowBytes;                        // A rows 0..63
+constexpr int kOffE2 = kOffALo + 64 * kBlkRowBytes;               // double[128]
+constexpr int kOffRank = kOffE2 + kD * (int)sizeof(double);       // int[2][128]
+constexpr int kOffQp = 0;                                         // double[4][128], after the append
+static_assert(kOffRank + 2 * kD * (int)sizeof(int) <= kPairs * 2 * kStageBytes, "scratch fits the stages");
+static_assert(kOffQp + 4 * kD * (int)sizeof(double) <= kOffALo, "q' copy below the low rows of A");
+struct PexScratch {                    // in MmaShared::pex
+    float qin[4][kD];                  // query rows (bf16 / f32 inputs are exact in f32)
+    float ks[kStepMaxNew][kD];         // new key rows
+};
+struct BqScratch {                     // in MmaShared::bq
+    float vs[kStepMaxNew][kCols];      // new value rows, this CTA's channels
+    int sel[kD];
+};
+static_assert(sizeof(PexScratch) <= sizeof(((MmaShared *)0)->pex), "query and key rows fit the exchange buffers");
+static_assert(sizeof(BqScratch) <= sizeof(((MmaShared *)0)->bq), "value rows and flags fit the fragment table");
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -96,7 +147,11 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)_
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
 }
+// expect bytes without arriving (the arrival comes with the key copies)
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
 }
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
@@ -142,49 +197,57 @@ __device__ __forceinline__ uint16_t f16_part(float x, int part) {
 // 4-token metadata chunk c of group g (the page format's XOR permutation)
 __device__ __forceinline__ int meta_chunk(int g, int c) { return c ^ (((c >> 3) & 3) ^ ((g & 1) << 2)); }
 
-__global__ void __launch_bounds__(kThreads, 2)
-decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len, int Hkv,
-                  int NB, int Hq, const int32_t *__restrict__ idx, const float *__restrict__ qsel,
-                  const float *__restrict__ qgsum, int k, float *__restrict__ part_o,
-                  float2 *__restrict__ part_ml, int S, float *__restrict__ out,
-                  uint32_t *__restrict__ counters, uint32_t *__restrict__ status) {
-    extern __shared__ __align__(16) uint8_t smem_raw[];
-    MmaShared &sh = *reinterpret_cast<MmaShared *>(smem_raw);
+// context split of this CTA: pages [blk0, blk1) of the first `len` tokens
+struct Split {
+    int blk0, blk1;
+};
+__device__ __forceinline__ Split split_of(int len, int S, int s) {
+    const int nblk = (len + kT - 1) / kT;
+    const int bps = (nblk + S - 1) / S;
+    const int blk0 = s * bps;
+    return {blk0, min(nblk, blk0 + bps)};
+}
 
-    const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int pair = warp >> 1, half = warp & 1;
+// The fused step's split: the last cluster also appends the new tokens, which
+// costs about kAppendPages pages of work per CTA, so it takes that many fewer
+// pages; the other splits take equal shares of the rest.  owner_of() is the
+// inverse (the split holding page pg).
+constexpr int kAppendPages = 8;
+struct StepPlan {
+    int S, nblk, bps, head, tail_bps;   // head = pages of the first S - kCluster splits
+};
+__device__ __forceinline__ StepPlan step_plan(int len, int S) {
+    StepPlan p;
+    p.S = S;
+    p.nblk = (len + kT - 1) / kT;
+    p.bps = (p.nblk + kCluster * kAppendPages + S - 1) / S;
+    p.head = min(p.nblk, (S - kCluster) * p.bps);
+    p.tail_bps = (p.nblk - p.head + kCluster - 1) / kCluster;
+    return p;
+}
+__device__ __forceinline__ Split step_split(const StepPlan &p, int s) {
+    if (s < p.S - kCluster) {
+        const int blk0 = min(p.nblk, s * p.bps);
+        return {blk0, min(p.nblk, blk0 + p.bps)};
+    }
+    const int blk0 = min(p.nblk, p.head + (s - (p.S - kCluster)) * p.tail_bps);
+    return {blk0, min(p.nblk, blk0 + p.tail_bps)};
+}
+__device__ __forceinline__ int owner_of(const StepPlan &p, int pg) {
+    if (pg < p.head) return pg / p.bps;
+    return p.S - kCluster + (pg - p.head) / max(p.tail_bps, 1);
+}
+
+// The page plan from the channel choice (sh.chan_pos, sh.q): score-MMA B
+// fragments, and the copy list of a page.  Called by every thread after a
+// barrier that follows the last write of chan_pos / q; ends with a barrier.
+__device__ __forceinline__ void build_plan(MmaShared &sh, int tid, int warp, int lane) {
     const int gid = lane >> 2, tig = lane & 3;
-    const size_t unit = (size_t)b * Hkv + h;
-    const size_t qrow0 = (size_t)b * Hq + (size_t)h * 4;
-
-    // ------------------------------------------------------------ prologue
-    for (int e = tid; e < 4 * k; e += kThreads) {
-        const int hl = e / k, i = e % k;
-        sh.q[hl][i] = qsel[(qrow0 + hl) * k + i];
-    }
-    if (tid < 4 * kNG) sh.qg[tid / kNG][tid % kNG] = qgsum[qrow0 * kNG + tid];
-    if (tid < kD) sh.chan_pos[tid] = -1;
-    if (tid < 2 * kPairs) mbar_init(smem_u32(&sh.mbar[tid >> 1][tid & 1]), 1);
-    // the list must be channel 0 followed by ascending channels in 1..127;
-    // any other list reads no key rows and raises KVQ_DEV_INDEX
-    const int32_t *sel = idx + unit * k;
-    int my_c = -1;
-    bool bad = false;
-    if (tid < k) {
-        my_c = sel[tid];
-        bad = (tid == 0) ? my_c != 0 : (my_c <= sel[tid - 1] || my_c > kD - 1);
-    }
-    const bool any_bad = __syncthreads_or(bad);
-    if (any_bad && tid == 0) atomicOr(status, (uint32_t)KVQ_DEV_INDEX);
-    if (!any_bad && tid < k) sh.chan_pos[my_c] = tid;
-    __syncthreads();
-
-    // score-MMA B fragments of k-step ks (channels 16ks..16ks+15): column gid =
-    // (head gid>>1, part gid&1); k-slots 2tig, 2tig+1, 2tig+8, 2tig+9 are
-    // channels +tig, +tig+4, +tig+8, +tig+12 (this order makes the code loads
-    // bank-conflict free).  Channel 0 and unselected channels get q' = 0.
     const int hh = gid >> 1, part = gid & 1;
+    // B fragments of k-step ks (channels 16ks..16ks+15): column gid = (head
+    // gid>>1, part gid&1); k-slots 2tig, 2tig+1, 2tig+8, 2tig+9 are channels
+    // +tig, +tig+4, +tig+8, +tig+12 (this order makes the code loads
+    // bank-conflict free).  Channel 0 and unselected channels get q' = 0.
     {
         const int ks = warp;
         uint32_t w[2];
@@ -206,33 +269,59 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
     }
     __syncthreads();
     if (tid == 0) {
-        // copy list: runs of touched chunks, single untouched chunks between
-        // two touched ones filled in (one copy instead of two); a run that
-        // reaches the last chunk continues through the page tail
+        // runs of touched chunks, single untouched chunks between two touched
+        // ones filled in (one copy instead of two); then the page tail
         const uint64_t T = (uint64_t)sh.touched[0] | ((uint64_t)sh.touched[1] << 32);
         uint64_t M = T | ((T << 1) & (T >> 1));
-        const bool tail_joined = (M >> 63) & 1u;
         int n = 0;
         uint32_t bytes = 0;
         while (M) {
             const int st = __ffsll((long long)M) - 1;
             const uint64_t inv = ~(M >> st);
             const int len = inv ? __ffsll((long long)inv) - 1 : kChunks - st;
-            uint32_t sz = 64u * (uint32_t)len;
-            if (st + len == kChunks) sz += (uint32_t)kFixBytes;
-            sh.copy[n++] = make_uint2(64u * (uint32_t)st, sz);
-            bytes += sz;
+            sh.copy[n++] = make_uint2(64u * (uint32_t)st, 64u * (uint32_t)len);
+            bytes += 64u * (uint32_t)len;
             M = (len == kChunks) ? 0ull : (M & ~(((1ull << len) - 1ull) << st));
         }
-        if (!tail_joined) {
-            sh.copy[n++] = make_uint2((uint32_t)kKeyBytes, (uint32_t)kFixBytes);
-            bytes += (uint32_t)kFixBytes;
-        }
+        sh.copy[n++] = make_uint2((uint32_t)kKeyBytes, (uint32_t)kFixBytes);
         sh.n_copies = n;
-        sh.tx_bytes = bytes;
+        sh.tx_keys = bytes;
     }
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     __syncthreads();
+}
+
+// Copies of one page into stage st of a pair, issued by one thread: the tail
+// (value codes, channel 0, metadata) expects its bytes without arriving; the
+// key chunks arrive on the barrier, so the stage's phase completes once both
+// parts have landed.
+__device__ __forceinline__ void issue_tail(MmaShared &sh, int pair, int st, const uint8_t *src) {
+    const uint32_t bar = smem_u32(&sh.mbar[pair][st]);
+    mbar_expect_tx(bar, (uint32_t)kFixBytes);
+    bulk_g2s(smem_u32(sh.stage[pair][st]) + kKeyBytes, src + kKeyBytes, (uint32_t)kFixBytes, bar);
+}
+__device__ __forceinline__ void issue_keys(MmaShared &sh, int pair, int st, const uint8_t *src) {
+    const uint32_t bar = smem_u32(&sh.mbar[pair][st]);
+    const uint32_t dst = smem_u32(sh.stage[pair][st]);
+    mbar_arrive_expect_tx(bar, sh.tx_keys);
+    const int n = sh.n_copies - 1;
+    for (int r = 0; r < n; r++) {
+        const uint2 c = sh.copy[r];
+        bulk_g2s(dst + c.x, src + c.x, c.y, bar);
+    }
+}
+
+// The page loop and the merges: pages [sp.blk0, sp.blk1) of the unit, pair
+// `pair` taking every kPairs-th.  `first_tail_issued`: the tail of the pair's
+// first page is already in flight into stage 0.
+__device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restrict__ unit_pages, int len,
+                                          Split sp, int S, int s, size_t qrow0, float *__restrict__ part_o,
+                                          float2 *__restrict__ part_ml, float *__restrict__ out,
+                                          uint32_t *counter, uint32_t *status, bool first_tail_issued) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int pair = warp >> 1, half = warp & 1;
+    const int gid = lane >> 2, tig = lane & 3;
+    const int hh = gid >> 1, part = gid & 1;
 
     // zero-point and channel-0 coefficients of head tig, pre-scaled to the
     // base-2 score domain
@@ -240,26 +329,6 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
 #pragma unroll
     for (int g = 0; g < kNG; g++) qg_t[g] = sh.qg[tig][g] * kScoreScaleLog2;
     const float q0_t = sh.q[tig][0] * kScoreScaleLog2;
-
-    // ------------------------------------------------------------ pages
-    const int len = min(max(seq_len[b], 0), NB * kT);
-    const int nblk = (len + kT - 1) / kT;
-    const int bps = (nblk + S - 1) / S;
-    const int blk0 = s * bps;
-    const int blk1 = min(nblk, blk0 + bps);
-
-    // one thread of the pair arms the stage's barrier and issues its copies
-    auto issue = [&](int st, int blk) {
-        const uint8_t *src = pages + (unit * NB + (size_t)blk) * page_bytes(2);
-        const uint32_t dst = smem_u32(sh.stage[pair][st]);
-        const uint32_t bar = smem_u32(&sh.mbar[pair][st]);
-        mbar_expect_tx(bar, sh.tx_bytes);
-        const int n = sh.n_copies;
-        for (int r = 0; r < n; r++) {
-            const uint2 c = sh.copy[r];
-            bulk_g2s(dst + c.x, src + c.x, c.y, bar);
-        }
-    };
 
     float m_run = -INFINITY;      // running max of head tig (base-2 domain)
     float l_thr = 0.f;            // this thread's share of the running sum of head tig
@@ -280,16 +349,24 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
     int it = 0;
     uint32_t late = 0;            // stages whose last wait gave up, with the parity waited for
     const bool issuer = (tid & 63) == 0;
-    const int first = blk0 + pair;
-    if (issuer && first < blk1) issue(0, first);
-    for (int pg = first; pg < blk1; pg += kPairs, it++) {
+    const int first = sp.blk0 + pair;
+    if (issuer && first < sp.blk1) {
+        const uint8_t *src = unit_pages + (size_t)first * page_bytes(2);
+        if (!first_tail_issued) issue_tail(sh, pair, 0, src);
+        issue_keys(sh, pair, 0, src);
+    }
+    for (int pg = first; pg < sp.blk1; pg += kPairs, it++) {
         const int st = it & 1;
         const uint8_t *cur = sh.stage[pair][st];
         const uint32_t par = (uint32_t)(it >> 1) & 1u;
         late = mbar_wait_bounded(smem_u32(&sh.mbar[pair][st]), par, status)
                    ? late & ~(3u << (2 * st)) : (late & ~(3u << (2 * st))) | ((2u | par) << (2 * st));
         pair_sync(pair);                                     // both warps left the other stage
-        if (issuer && pg + kPairs < blk1) issue(st ^ 1, pg + kPairs);
+        if (issuer && pg + kPairs < sp.blk1) {
+            const uint8_t *src = unit_pages + (size_t)(pg + kPairs) * page_bytes(2);
+            issue_tail(sh, pair, st ^ 1, src);
+            issue_keys(sh, pair, st ^ 1, src);
+        }
 
         const uint8_t *vcodes = cur + kKeyBytes;
         const uint32_t *ch0w = reinterpret_cast<const uint32_t *>(vcodes + 128 * 32);
@@ -446,8 +523,8 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
 #pragma unroll
                     for (int r = 0; r < 2; r++) {
                         const int f = 2 * (j & 1) + r;
-                        const __half2 sp = u2h(__byte_perm(vw[u][f], vw[u][f + 4], 0x5410));
-                        bw[j][r] = h2u(__hmul2(u2h(ph[j][r]), sp));
+                        const __half2 sp2 = u2h(__byte_perm(vw[u][f], vw[u][f + 4], 0x5410));
+                        bw[j][r] = h2u(__hmul2(u2h(ph[j][r]), sp2));
                     }
                 }
             }
@@ -543,18 +620,283 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
         part_o[row * kD + c] = o;
         if (c == 0) part_ml[row] = make_float2(M, L);
     }
-    merge_unit_if_last<4, kThreads>(part_o, part_ml, S, qrow0, out, counters + unit,
+    static_assert(merge_scratch_floats(4, kThreads, 256) * 4 <= 2 * 2 * kStageBytes, "merge scratch fits stages 2-3");
+    merge_unit_if_last<4, kThreads>(part_o, part_ml, S, qrow0, out, counter,
                                     reinterpret_cast<float *>(sh.stage[2][0]));
+}
+
+// ---------------------------------------------------------------- decode
+__global__ void __launch_bounds__(kThreads, 2)
+decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len, int Hkv,
+                  int NB, int Hq, const int32_t *__restrict__ idx, const float *__restrict__ qsel,
+                  const float *__restrict__ qgsum, int k, float *__restrict__ part_o,
+                  float2 *__restrict__ part_ml, int S, float *__restrict__ out,
+                  uint32_t *__restrict__ counters, uint32_t *__restrict__ status) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    MmaShared &sh = *reinterpret_cast<MmaShared *>(smem_raw);
+
+    const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const size_t unit = (size_t)b * Hkv + h;
+    const size_t qrow0 = (size_t)b * Hq + (size_t)h * 4;
+
+    for (int e = tid; e < 4 * k; e += kThreads) {
+        const int hl = e / k, i = e % k;
+        sh.q[hl][i] = qsel[(qrow0 + hl) * k + i];
+    }
+    if (tid < 4 * kNG) sh.qg[tid / kNG][tid % kNG] = qgsum[qrow0 * kNG + tid];
+    if (tid < kD) sh.chan_pos[tid] = -1;
+    if (tid < 2 * kPairs) mbar_init(smem_u32(&sh.mbar[tid >> 1][tid & 1]), 1);
+    // the list must be channel 0 followed by ascending channels in 1..127;
+    // any other list reads no key rows and raises KVQ_DEV_INDEX
+    const int32_t *sel = idx + unit * k;
+    int my_c = -1;
+    bool bad = false;
+    if (tid < k) {
+        my_c = sel[tid];
+        bad = (tid == 0) ? my_c != 0 : (my_c <= sel[tid - 1] || my_c > kD - 1);
+    }
+    const bool any_bad = __syncthreads_or(bad);
+    if (any_bad && tid == 0) atomicOr(status, (uint32_t)KVQ_DEV_INDEX);
+    if (!any_bad && tid < k) sh.chan_pos[my_c] = tid;
+    __syncthreads();
+    build_plan(sh, tid, warp, lane);
+
+    const int len = min(max(seq_len[b], 0), NB * kT);
+    run_pages(sh, pages + unit * NB * (size_t)page_bytes(2), len, split_of(len, S, s), S, s, qrow0, part_o,
+              part_ml, out, counters + unit, status, false);
+}
+
+// ---------------------------------------------------------------- fused step
+__device__ __forceinline__ void cluster_arrive() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+
+template <typename Tin>
+__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 2)
+step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint32_t *__restrict__ status,
+                int Hkv, int NB, int Hq, const Tin *__restrict__ q, const Tin *__restrict__ k_new,
+                const Tin *__restrict__ v_new, int n_new, const double *__restrict__ A,
+                const double *__restrict__ Ainvt, int k, int32_t *__restrict__ idx, float *__restrict__ qsel,
+                float *__restrict__ qgsum, float *__restrict__ part_o, float2 *__restrict__ part_ml, int S,
+                float *__restrict__ out) {
+    namespace cg = cooperative_groups;
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    MmaShared &sh = *reinterpret_cast<MmaShared *>(smem_raw);
+    uint8_t *P = &sh.stage[0][0][0];
+    double (*aiT)[kCols] = reinterpret_cast<double (*)[kCols]>(P);              // A^{-T}[:, 64r + .]
+    double (*a_hi)[kCols] = reinterpret_cast<double (*)[kCols]>(P + kOffAHi);   // A[64 + ., 64r + .]
+    double (*a_lo)[kCols] = reinterpret_cast<double (*)[kCols]>(P + kOffALo);   // A[., 64r + .]
+    double *e2 = reinterpret_cast<double *>(P + kOffE2);
+    int (*rank_part)[kD] = reinterpret_cast<int (*)[kD]>(P + kOffRank);
+    double (*qp)[kD] = reinterpret_cast<double (*)[kD]>(P + kOffQp);
+    PexScratch &px = *reinterpret_cast<PexScratch *>(&sh.pex[0][0][0]);
+    BqScratch &bx = *reinterpret_cast<BqScratch *>(&sh.bq[0][0]);
+
+    cg::cluster_group cluster = cg::this_cluster();
+    const int r = (int)cluster.block_rank();        // channels 64r..64r+63
+    const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int B = gridDim.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const size_t unit = (size_t)b * Hkv + h;
+    const size_t qrow0 = (size_t)b * Hq + (size_t)h * 4;
+    uint8_t *unit_pages = pages + unit * NB * (size_t)page_bytes(2);
+    const int capacity = NB * kT;
+    // 64-column block of a 128 x 128 float64 matrix: 128 rows of 512 bytes
+    auto stage_block = [&](double (*dst)[kCols], const double *src, int row0, int rows) {
+        for (int e = tid; e < rows * (kBlkRowBytes / 16); e += kThreads) {
+            const int c = e >> 5, part = e & 31;
+            cp_async16(&dst[c][2 * part], src + (size_t)(row0 + c) * kD + 2 * part);
+        }
+    };
+
+    if (tid == 0) sh.s_len = seq_len[b];
+    if (tid < kD) sh.chan_pos[tid] = -1;
+    if (tid < 2 * kPairs) mbar_init(smem_u32(&sh.mbar[tid >> 1][tid & 1]), 1);
+    const double *Ai_blk = Ainvt + (size_t)h * kD * kD + r * kCols;
+    const double *A_blk = A + (size_t)h * kD * kD + r * kCols;
+    stage_block(aiT, Ai_blk, 0, kD);
+    for (int e = tid; e < 4 * kD; e += kThreads) px.qin[e / kD][e % kD] = in_to_float(q[qrow0 * kD + e]);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    __syncthreads();
+
+    // new length (a step that would overflow the capacity appends nothing and
+    // raises KVQ_DEV_CAPACITY, like kvq_append) and this CTA's pages
+    const int L0 = sh.s_len;
+    const bool ok = L0 >= 0 && L0 + n_new <= capacity;
+    const int len = min(max(ok ? L0 + n_new : L0, 0), capacity);
+    const StepPlan plan = step_plan(len, S);
+    const Split sp = step_split(plan, s);
+    // new tokens w in [w0, w1) land in the pages of this cluster's splits
+    int w0 = 0, w1 = 0;
+    if (ok && n_new > 0) {
+        const int s_first = s - r;
+        w0 = n_new;
+        for (int w = n_new - 1; w >= 0; w--) {
+            const int owner = owner_of(plan, (L0 + w) / kT);
+            if (owner >= s_first && owner < s_first + kCluster) {
+                w1 = max(w1, w + 1);
+                w0 = w;
+            }
+        }
+        if (w1 == 0) w0 = 0;
+    }
+    const int nw = w1 - w0;
+    const size_t in_base = unit * (size_t)n_new + w0;
+    if (nw > 0) {
+        stage_block(a_lo, A_blk, 0, 64);
+        for (int e = tid; e < nw * kD; e += kThreads) px.ks[e / kD][e % kD] = in_to_float(k_new[in_base * kD + e]);
+        for (int e = tid; e < nw * kCols; e += kThreads)
+            bx.vs[e / kCols][e % kCols] = in_to_float(v_new[(in_base + e / kCols) * kD + r * kCols + e % kCols]);
+    }
+    cp_async_commit();
+    // every CTA of sequence b has read its length once the counter reaches
+    // S * Hkv; the last one stores the new length
+    if (tid == 0) {
+        if (!ok && s == 0 && h == 0) atomicOr(status, (uint32_t)KVQ_DEV_CAPACITY);
+        const unsigned prev = atomicAdd(status + 1 + b, 1u);
+        if (prev == (unsigned)(S * Hkv) - 1u) {
+            if (ok) seq_len[b] = L0 + n_new;
+            atomicExch(status + 1 + b, 0u);
+        }
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+
+    // q'[hl][64r + jj] = sum_c q[hl][c] Ainvt[c][64r + jj], fma chain c =
+    // 0..127 from 0.0; hl = warp / 2, jj = 32 (warp % 2) + lane
+    {
+        const int hl = warp >> 1, jj = (warp & 1) * 32 + lane;
+        double acc = 0.0;
+#pragma unroll 16
+        for (int c = 0; c < kD; c++) acc = fma((double)px.qin[hl][c], aiT[c][jj], acc);
+        sh.qp_own[hl][jj] = acc;
+    }
+    __syncthreads();                                // A^{-T} block no longer needed
+    if (nw > 0) {
+        // K'[t][j] = sum_c K[t][c] A[c][j], fma chain c = 0..127 from 0.0, for
+        // token w0 + warp / 2 and channel j = 64r + jj: rows 0..63 of A while
+        // rows 64..127 are staged
+        stage_block(a_hi, A_blk, 64, 64);
+        cp_async_commit();
+        const int w = warp >> 1, jj = (warp & 1) * 32 + lane, j = r * kCols + jj;
+        double x = 0.0;
+        if (w < nw) {
+#pragma unroll 16
+            for (int c = 0; c < 64; c++) x = fma((double)px.ks[w][c], a_lo[c][jj], x);
+        }
+        cp_async_wait<0>();
+        __syncthreads();
+        if (w < nw) {                               // uniform over the warp
+#pragma unroll 16
+            for (int c = 64; c < kD; c++) x = fma((double)px.ks[w][c], a_hi[c - 64][jj], x);
+            const int g = 2 * r + (warp & 1);       // this warp's key group
+            const int pos = L0 + w0 + w, tt = pos % kT;
+            uint8_t *page = unit_pages + (size_t)(pos / kT) * page_bytes(2);
+            uint16_t sb, zb;
+            const uint32_t kc = quantize_lane<2>(x, j != 0, sb, zb);
+            if (lane == 0)
+                reinterpret_cast<uint32_t *>(page + off_kmeta(2))[meta_word(g, tt)] = (uint32_t)sb | ((uint32_t)zb << 16);
+            if (j == 0) reinterpret_cast<uint16_t *>(page + off_ch0(2))[tt] = __bfloat16_as_ushort(__double2bfloat16(x));
+            const uint32_t vc = quantize_lane<2>((double)bx.vs[w][jj], true, sb, zb);
+            if (lane == 0)
+                reinterpret_cast<uint32_t *>(page + off_vmeta(2))[meta_word(g, tt)] = (uint32_t)sb | ((uint32_t)zb << 16);
+            // positions at or beyond the stored length hold zero bits, so the
+            // codes are OR-ed in (the other new tokens share the words)
+            const int word = tt / 16, shf = 2 * (tt % 16);
+            if (j != 0) atomicOr(reinterpret_cast<uint32_t *>(page + (size_t)j * row_bytes(2)) + word, kc << shf);
+            atomicOr(reinterpret_cast<uint32_t *>(page + off_vcodes(2) + (size_t)j * row_bytes(2)) + word, vc << shf);
+            // the page is read next through the async proxy (bulk copies)
+            asm volatile("fence.proxy.async.global;\n" ::: "memory");
+        }
+    }
+    __syncthreads();
+    if (tid < kCols) {
+        double e = 0.0;
+#pragma unroll
+        for (int hl = 0; hl < 4; hl++) e = fma(sh.qp_own[hl][tid], sh.qp_own[hl][tid], e);
+        sh.e2_own[tid] = e;
+    }
+    cluster.sync();            // the cluster's q', energies and new tokens are in place
+    if (tid < kD) {
+        const MmaShared *peer = cluster.map_shared_rank(&sh, tid / kCols);
+        const int l = tid % kCols;
+        e2[tid] = peer->e2_own[l];
+#pragma unroll
+        for (int hl = 0; hl < 4; hl++) qp[hl][tid] = peer->qp_own[hl][l];
+    }
+    __syncthreads();
+    cluster_arrive();          // done reading the other CTA's shared memory (waited for at exit)
+
+    // ---- channel choice (the arithmetic of kvq_select_channels)
+    {
+        const int j = tid & (kD - 1), part = tid >> 7;
+        const double e = e2[j];
+        int rk = 0;
+        const int i0 = part == 0 ? 1 : 64, i1 = part == 0 ? 64 : kD;
+        for (int i = i0; i < i1; i++) {
+            const double ei = e2[i];
+            rk += (ei > e) || (ei == e && i < j);
+        }
+        rank_part[part][j] = rk;
+    }
+    __syncthreads();
+    int pos = -1;
+    if (tid < kD) {
+        const bool sel = (tid == 0) || (rank_part[0][tid] + rank_part[1][tid] < k - 1);
+        bx.sel[tid] = sel;
+        const unsigned ballot = __ballot_sync(0xffffffffu, sel);
+        if (lane == 0) sh.warp_cnt[warp] = __popc(ballot);
+        if (sel) pos = (int)__popc(ballot & ((1u << lane) - 1u));
+    }
+    __syncthreads();
+    if (pos >= 0) {
+        for (int w = 0; w < warp; w++) pos += sh.warp_cnt[w];
+        sh.chan_pos[tid] = pos;
+#pragma unroll
+        for (int hl = 0; hl < 4; hl++) {
+            const float qf = (float)qp[hl][tid];
+            sh.q[hl][pos] = qf;
+            if (s == 0) qsel[(qrow0 + hl) * k + pos] = qf;
+        }
+        if (s == 0) idx[unit * k + pos] = tid;
+    }
+    if (tid < 4 * kNG) {
+        // zero-point sum of key group gr (channel 0 is bf16, not in group 0),
+        // channels ascending from 0.0
+        const int hl = tid / kNG, gr = tid % kNG;
+        double sm = 0.0;
+        for (int c = (gr == 0 ? 1 : gr * kGroup); c < (gr + 1) * kGroup; c++)
+            if (bx.sel[c]) sm += qp[hl][c];
+        const float gf = (float)sm;
+        sh.qg[hl][gr] = gf;
+        if (s == 0) qgsum[(qrow0 + hl) * kNG + gr] = gf;
+    }
+    __syncthreads();
+    build_plan(sh, tid, warp, lane);
+
+    run_pages(sh, unit_pages, len, sp, S, s, qrow0, part_o, part_ml, out,
+              status + 1 + B + unit, status, false);
+    cluster_wait();            // the other CTA no longer reads this CTA's shared memory
 }
 
 }  // namespace
 
+// Splits per (sequence, KV head): about two CTAs per SM in all, a multiple of
+// the fused step's cluster size (at least one cluster), at most one split per
+// kPairs pages unless that is below one cluster.
 int decode_mma_splits(int units, int nblk, int num_sms) {
-    int S = (2 * num_sms + units - 1) / units;
-    const int max_s = nblk / kPairs > 0 ? nblk / kPairs : 1;   // at least one page per pair
+    int S = (2 * num_sms) / units;
+    const int max_s = nblk / kPairs;
     if (S > max_s) S = max_s;
-    return S < 1 ? 1 : S;
+    S -= S % kCluster;
+    return S < kCluster ? kCluster : S;
 }
+
+int step_mma_max_new() { return kStepMaxNew; }
 
 cudaError_t launch_decode_mma(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
                               const float *qgsum, int k, float *part_o, float2 *part_ml, int S,
@@ -567,6 +909,33 @@ cudaError_t launch_decode_mma(const kvq_cache &c, int Hq, const int32_t *idx, co
     decode_mma_kernel<<<grid, kThreads, smem, st>>>(static_cast<const uint8_t *>(c.pages), c.seq_len,
                                                     c.n_kv_heads, c.capacity / kT, Hq, idx, qsel, qgsum, k,
                                                     part_o, part_ml, S, out, unit_counter(c, 0, 0), c.status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_step_mma(const kvq_cache &c, int Hq, const void *q, const void *k_new, const void *v_new,
+                            int dtype, int n_new, const double *A, const double *Ainvt, int k, int32_t *idx,
+                            float *qsel, float *qgsum, float *part_o, float2 *part_ml, int S, float *out,
+                            cudaStream_t st) {
+    const size_t smem = sizeof(MmaShared);
+    dim3 grid((unsigned)S, (unsigned)c.n_kv_heads, (unsigned)c.batch);
+    cudaError_t e;
+    if (dtype == KVQ_DTYPE_F32) {
+        static std::atomic<uint64_t> done{0};
+        e = set_smem_once(step_mma_kernel<float>, (int)smem, done);
+        if (e != cudaSuccess) return e;
+        step_mma_kernel<float><<<grid, kThreads, smem, st>>>(
+            static_cast<uint8_t *>(c.pages), c.seq_len, c.status, c.n_kv_heads, c.capacity / kT, Hq,
+            static_cast<const float *>(q), static_cast<const float *>(k_new), static_cast<const float *>(v_new),
+            n_new, A, Ainvt, k, idx, qsel, qgsum, part_o, part_ml, S, out);
+    } else {
+        static std::atomic<uint64_t> done{0};
+        e = set_smem_once(step_mma_kernel<uint16_t>, (int)smem, done);
+        if (e != cudaSuccess) return e;
+        step_mma_kernel<uint16_t><<<grid, kThreads, smem, st>>>(
+            static_cast<uint8_t *>(c.pages), c.seq_len, c.status, c.n_kv_heads, c.capacity / kT, Hq,
+            static_cast<const uint16_t *>(q), static_cast<const uint16_t *>(k_new),
+            static_cast<const uint16_t *>(v_new), n_new, A, Ainvt, k, idx, qsel, qgsum, part_o, part_ml, S, out);
+    }
     return cudaGetLastError();
 }
 

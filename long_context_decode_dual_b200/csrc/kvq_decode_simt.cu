@@ -219,6 +219,7 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
         part_o[row * kD + tid] = o_acc[hl];
         if (tid == 0) part_ml[row] = make_float2(m_run[hl], l_run[hl]);
     }
+    static_assert(merge_scratch_floats(G, 128, 256) * 4 <= 2 * fixed_bytes(BITS), "merge scratch fits the stages");
     merge_unit_if_last<G, 128>(part_o, part_ml, S, (size_t)b * Hq + (size_t)h * G, out, counters + unit,
                           reinterpret_cast<float *>(smem));
 }

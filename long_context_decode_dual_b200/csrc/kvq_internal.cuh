@@ -47,6 +47,39 @@ __device__ __forceinline__ float in_to_float(uint16_t bf) {
     return __uint_as_float(((uint32_t)bf) << 16);
 }
 
+// ------------------------------------------------------------ quantization
+__device__ __forceinline__ double warp_min(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmin(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ double warp_max(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// Quantize value x of this lane against the group range (lanes of the warp;
+// `in_range` false leaves the lane out of min/max).  Returns the code and,
+// through s_bits / z_bits, the fp16 scale / zero-point bit patterns.
+template <int BITS>
+__device__ __forceinline__ uint32_t quantize_lane(double x, bool in_range, uint16_t &s_bits,
+                                                  uint16_t &z_bits) {
+    constexpr int L = (1 << BITS) - 1;
+    const double lo = warp_min(in_range ? x : __longlong_as_double(0x7ff0000000000000LL));
+    const double hi = warp_max(in_range ? x : __longlong_as_double(0xfff0000000000000LL));
+    const __half zh = __double2half(lo);
+    const __half sh = __double2half((hi - lo) / (double)L);
+    z_bits = __half_as_ushort(zh);
+    s_bits = __half_as_ushort(sh);
+    const double z = (double)__half2float(zh);
+    const double s = (double)__half2float(sh);
+    if (s == 0.0) return 0u;
+    double r = rint((x - z) / s);
+    r = fmin(fmax(r, 0.0), (double)L);
+    return (uint32_t)r;
+}
+
 // ------------------------------------------------------------ cp.async
 __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src) {
     uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
@@ -79,15 +112,27 @@ cudaError_t set_smem_once(Kernel *fn, int bytes, std::atomic<uint64_t> &done) {
 // -- merges them: out = sum_s e^{m_s - M} o_s / sum_s e^{m_s - M} l_s, the one
 // softmax over the whole context (Dual-QK §3.4).  Nothing waits: the other
 // CTAs simply exit.  Called by every thread of an NT-thread CTA; `scratch` is
-// shared memory for 2 * G * S + G floats.  The (m, l) pairs are read in one
-// parallel pass and turned into per-split weights, then each thread sums
-// G * 128 / NT consecutive outputs over the splits with independent loads.
+// 16-byte aligned shared memory for merge_scratch_floats(G, NT, S) floats.
+// The (m, l) pairs are read in one parallel pass and turned into per-split
+// weights; then the G * 128 outputs, as float4 columns, are summed over the
+// splits with R = NT / columns threads per column (each a strided subset of
+// the splits, many independent loads in flight), and the R partial sums are
+// added in a fixed order.
+template <int G, int NT>
+struct MergeShape {
+    static constexpr int F = G * kD / 4;                 // float4 columns
+    static constexpr int R = NT >= F ? NT / F : 1;       // threads per column
+    static constexpr int CPT = NT >= F ? 1 : F / NT;     // columns per thread
+    static_assert(NT >= F ? NT % F == 0 : F % NT == 0, "merge: columns and threads must divide");
+};
+__host__ __device__ constexpr int merge_scratch_floats(int G, int NT, int S) {
+    return 2 * G * S + G + 4 + (NT > G * kD / 4 ? NT / (G * kD / 4) * G * kD : 0);
+}
 template <int G, int NT>
 __device__ __forceinline__ void merge_unit_if_last(const float *part_o, const float2 *part_ml, int S,
                                                    size_t qrow0, float *out, uint32_t *counter,
                                                    float *scratch) {
-    constexpr int OPT = G * kD / NT;                 // outputs per thread
-    static_assert(OPT >= 1 && G * kD == OPT * NT, "merge: G * 128 must be a multiple of the CTA size");
+    using MS = MergeShape<G, NT>;
     __shared__ int s_last;
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -101,6 +146,7 @@ __device__ __forceinline__ void merge_unit_if_last(const float *part_o, const fl
     float *wm = scratch;             // [G][S] max, then weight
     float *wl = scratch + G * S;     // [G][S] sum
     float *inv = wl + G * S;         // [G] 1 / total sum
+    float4 *part = reinterpret_cast<float4 *>(scratch + ((2 * G * S + G + 3) & ~3));   // [R][F]
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     for (int e = t; e < G * S; e += NT) {
         const float2 v = __ldcg(part_ml + qrow0 * S + e);     // rows qrow0.. are contiguous
@@ -124,36 +170,50 @@ __device__ __forceinline__ void merge_unit_if_last(const float *part_o, const fl
         if (lane == 0) inv[hl] = L > 0.f ? 1.f / L : 0.f;
     }
     __syncthreads();
-    // thread t owns outputs [t*OPT, t*OPT + OPT) of the unit's [G][128] block
-    const int hl = (t * OPT) / kD, c0 = (t * OPT) % kD;
-    float acc[OPT];
+    const int sub = t / (NT / MS::R >= 1 ? NT / MS::R : 1);   // split subset of this thread
+    const int col0 = (t % (NT / MS::R)) * MS::CPT;
 #pragma unroll
-    for (int u = 0; u < OPT; u++) acc[u] = 0.f;
-    const float *po = part_o + ((qrow0 + hl) * S) * kD + c0;
+    for (int cc = 0; cc < MS::CPT; cc++) {
+        const int col = col0 + cc, hl = (4 * col) / kD, c0 = (4 * col) % kD;
+        const float4 *po = reinterpret_cast<const float4 *>(part_o + ((qrow0 + hl) * S) * kD + c0);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 8
-    for (int s = 0; s < S; s++) {
-        const float w = wm[hl * S + s];
-        if constexpr (OPT % 4 == 0) {
-#pragma unroll
-            for (int u = 0; u < OPT; u += 4) {
-                const float4 v = __ldcg(reinterpret_cast<const float4 *>(po + (size_t)s * kD + u));
-                acc[u] = fmaf(w, v.x, acc[u]);
-                acc[u + 1] = fmaf(w, v.y, acc[u + 1]);
-                acc[u + 2] = fmaf(w, v.z, acc[u + 2]);
-                acc[u + 3] = fmaf(w, v.w, acc[u + 3]);
-            }
-        } else if constexpr (OPT == 2) {
-            const float2 v = __ldcg(reinterpret_cast<const float2 *>(po + (size_t)s * kD));
-            acc[0] = fmaf(w, v.x, acc[0]);
-            acc[1] = fmaf(w, v.y, acc[1]);
+        for (int s = sub; s < S; s += MS::R) {
+            const float w = wm[hl * S + s];
+            const float4 v = __ldcg(po + (size_t)s * (kD / 4));
+            acc.x = fmaf(w, v.x, acc.x);
+            acc.y = fmaf(w, v.y, acc.y);
+            acc.z = fmaf(w, v.z, acc.z);
+            acc.w = fmaf(w, v.w, acc.w);
+        }
+        if constexpr (MS::R == 1) {
+            const float r = inv[hl];
+            float *o = out + (qrow0 + hl) * kD + c0;          // out is only 4-byte aligned
+            o[0] = acc.x * r;
+            o[1] = acc.y * r;
+            o[2] = acc.z * r;
+            o[3] = acc.w * r;
         } else {
-#pragma unroll
-            for (int u = 0; u < OPT; u++) acc[u] = fmaf(w, __ldcg(po + (size_t)s * kD + u), acc[u]);
+            part[sub * MS::F + col] = acc;
         }
     }
-    const float r = inv[hl];
-#pragma unroll
-    for (int u = 0; u < OPT; u++) out[(qrow0 + hl) * kD + c0 + u] = acc[u] * r;
+    if constexpr (MS::R > 1) {
+        __syncthreads();
+        for (int col = t; col < MS::F; col += NT) {
+            const int hl = (4 * col) / kD, c0 = (4 * col) % kD;
+            float4 a = part[col];
+            for (int q = 1; q < MS::R; q++) {
+                const float4 v = part[q * MS::F + col];
+                a.x += v.x; a.y += v.y; a.z += v.z; a.w += v.w;
+            }
+            const float r = inv[hl];
+            float *o = out + (qrow0 + hl) * kD + c0;
+            o[0] = a.x * r;
+            o[1] = a.y * r;
+            o[2] = a.z * r;
+            o[3] = a.w * r;
+        }
+    }
     __syncthreads();
     if (t == 0) atomicExch(counter, 0u);
 }
@@ -171,6 +231,10 @@ size_t decode_ws_bytes(const kvq_cache &c, int Hq, int n_splits);
 cudaError_t launch_decode(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
                           const float *qgsum, int k, float *out, void *ws, int n_splits,
                           cudaStream_t st);
+cudaError_t launch_decode_step(const kvq_cache &c, int Hq, const void *q, const void *k_new,
+                               const void *v_new, int dtype, int n_new, const double *A,
+                               const double *Ainvt, int k, int32_t *idx, float *qsel, float *qgsum,
+                               float *out, void *ws, int n_splits, cudaStream_t st);
 // completion counter of unit (b, h) in the cache's status array
 inline uint32_t *unit_counter(const kvq_cache &c, int b, int h) {
     return c.status + 1 + c.batch + (size_t)b * c.n_kv_heads + h;

@@ -7,100 +7,116 @@
 //        e_j^2 = sum_h q'_{h,j}^2, one mask per KV head, chosen per query.
 // Channel 0 is always kept; ties go to the lower channel index.
 //
-// One CTA = one (sequence, KV head), 512 threads.  A^{-T} of the head is
-// staged in shared memory with one cp.async burst, then thread (slot, j) runs
-// the fixed-order fp64 fma chains q'[h][j] for heads h = slot, slot+4, ....  The selection is
-// exact and order-free: each candidate counts the channels that beat it
-// (rank, split four ways), then a ballot prefix sum writes the kept channels
-// in ascending order.
+// One thread-block cluster of four CTAs = one (sequence, KV head); CTA r owns
+// channels 32r..32r+31 (key group r).  It stages its 32 columns of A^{-T}
+// (32 KB) with one cp.async burst and runs the fixed-order fp64 fma chains
+// q'[h][j] of its channels, then their pooled energies.  After a cluster
+// barrier every CTA reads the four energy blocks through distributed shared
+// memory and makes the same exact, order-free choice (each candidate counts
+// the channels that beat it), so no CTA waits for another's decision; each
+// writes the outputs of its own channels: their list positions (a ballot
+// prefix sum over the 128 flags), q' in fp32 and its group's zero-point sum.
 #include "kvq_internal.cuh"
+
+#include <cooperative_groups.h>
 
 namespace kvq {
 namespace {
 
-constexpr int kThreads = 512;
+namespace cg = cooperative_groups;
+
+constexpr int kThreads = 256;
+constexpr int kCtas = kNG;                 // CTAs per cluster, one per key group
 
 template <typename Tin>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __cluster_dims__(kCtas, 1, 1) __launch_bounds__(kThreads)
 select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, int Hq, int Hkv, int g,
               int k, int32_t *__restrict__ idx, float *__restrict__ qsel,
               float *__restrict__ qgsum) {
-    extern __shared__ __align__(16) double sm[];   // Ainvt[128][128], qin[g][128], qp[g][128]
+    extern __shared__ __align__(16) double sm[];   // As[128][32], qin[g][128], qp[g][32]
     double *As = sm;
-    double *qin = sm + kD * kD;
+    double *qin = sm + kD * kGroup;
     double *qp = qin + (size_t)g * kD;
+    __shared__ double e2own[kGroup];
     __shared__ double e2s[kD];
-    __shared__ int rank_part[4][kD];
+    __shared__ int rank_part[2][kD];
     __shared__ int sel_s[kD];
     __shared__ int warp_cnt[4];
 
-    const int h = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
-    const int j = t & (kD - 1), slot = t >> 7;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int r = (int)cluster.block_rank();       // = blockIdx.x
+    const int h = blockIdx.y, b = blockIdx.z, t = threadIdx.x;
+    const int lane = t & 31, warp = t >> 5;
     const size_t qrow0 = (size_t)b * Hq + (size_t)h * g;
 
-    // A^{-T} of this KV head in one cp.async burst
-    const double *Ai = Ainvt + (size_t)h * kD * kD;
-    for (int e = t; e < kD * kD / 2; e += kThreads) cp_async16(As + 2 * e, Ai + 2 * e);
+    // columns 32r..32r+31 of A^{-T} for this KV head: 128 rows of 256 bytes
+    const double *Ai = Ainvt + (size_t)h * kD * kD + r * kGroup;
+    for (int e = t; e < kD * kGroup / 2; e += kThreads) {
+        const int c = e >> 4, part = e & 15;
+        cp_async16(As + c * kGroup + 2 * part, Ai + (size_t)c * kD + 2 * part);
+    }
     cp_async_commit();
     for (int e = t; e < g * kD; e += kThreads) qin[e] = in_to_double(q[qrow0 * kD + e]);
     cp_async_wait<0>();
     __syncthreads();
 
     // q'[hl][j] = sum_c q[hl][c] Ainvt[c][j], fma chain c = 0..127 from 0.0
-    for (int hl = slot; hl < g; hl += 4) {
+    for (int hl = warp; hl < g; hl += kThreads / 32) {
         double acc = 0.0;
 #pragma unroll 16
-        for (int c = 0; c < kD; c++) acc = fma(qin[hl * kD + c], As[c * kD + j], acc);
-        qp[hl * kD + j] = acc;
+        for (int c = 0; c < kD; c++) acc = fma(qin[hl * kD + c], As[c * kGroup + lane], acc);
+        qp[hl * kGroup + lane] = acc;
     }
     __syncthreads();
     // e_j^2, fma chain over heads ascending from 0.0
-    if (t < kD) {
+    if (t < kGroup) {
         double e = 0.0;
-        for (int hl = 0; hl < g; hl++) e = fma(qp[hl * kD + j], qp[hl * kD + j], e);
-        e2s[j] = e;
+        for (int hl = 0; hl < g; hl++) e = fma(qp[hl * kGroup + t], qp[hl * kGroup + t], e);
+        e2own[t] = e;
+    }
+    cluster.sync();                                // every CTA's energies are ready
+    if (t < kD) {
+        const double *src = cluster.map_shared_rank(e2own, t / kGroup);
+        e2s[t] = src[t % kGroup];
     }
     __syncthreads();
-    // rank of candidate j >= 1 among channels 1..127, counted in four parts
+    // rank of candidate j >= 1 among channels 1..127, counted in two halves
     {
+        const int j = t & (kD - 1), part = t >> 7;
         const double e = e2s[j];
-        int r = 0;
-        const int i0 = 1 + 32 * slot, i1 = min(kD, i0 + 32);
+        int rk = 0;
+        const int i0 = part == 0 ? 1 : 64, i1 = part == 0 ? 64 : kD;
         for (int i = i0; i < i1; i++) {
             const double ei = e2s[i];
-            r += (ei > e) || (ei == e && i < j);
+            rk += (ei > e) || (ei == e && i < j);
         }
-        rank_part[slot][j] = r;
+        rank_part[part][j] = rk;
     }
     __syncthreads();
+    int pos = -1;
     if (t < kD) {
-        const int lane = t & 31, warp = t >> 5;
-        const bool sel = (j == 0) ||
-                         (rank_part[0][j] + rank_part[1][j] + rank_part[2][j] + rank_part[3][j] < k - 1);
-        sel_s[j] = sel;
+        const bool sel = (t == 0) || (rank_part[0][t] + rank_part[1][t] < k - 1);
+        sel_s[t] = sel;
         const unsigned ballot = __ballot_sync(0xffffffffu, sel);
         if (lane == 0) warp_cnt[warp] = __popc(ballot);
-        __syncwarp();
-        // (warp_cnt of the other warps is read after the barrier below)
-        rank_part[0][j] = sel ? (int)__popc(ballot & ((1u << lane) - 1u)) : -1;
+        if (sel) pos = (int)__popc(ballot & ((1u << lane) - 1u));
     }
     __syncthreads();
-    if (t < kD) {
-        int pos = rank_part[0][j];
-        if (pos >= 0) {
-            for (int w = 0; w < (t >> 5); w++) pos += warp_cnt[w];
-            idx[((size_t)b * Hkv + h) * k + pos] = j;
-            for (int hl = 0; hl < g; hl++) qsel[(qrow0 + hl) * k + pos] = (float)qp[hl * kD + j];
-        }
+    // this CTA's channels are t = 32r..32r+31 (warp r)
+    if (warp == r && pos >= 0) {
+        for (int w = 0; w < r; w++) pos += warp_cnt[w];
+        idx[((size_t)b * Hkv + h) * k + pos] = t;
+        for (int hl = 0; hl < g; hl++) qsel[(qrow0 + hl) * k + pos] = (float)qp[hl * kGroup + lane];
     }
-    // zero-point sums per key group (channel 0 is bf16, not in group 0)
-    for (int u = t; u < g * kNG; u += kThreads) {
-        const int hl = u / kNG, gr = u % kNG;
+    // zero-point sum of key group r (channel 0 is bf16, not in group 0),
+    // channels ascending from 0.0
+    for (int hl = t; hl < g; hl += kThreads) {
         double s = 0.0;
-        for (int c = (gr == 0 ? 1 : gr * kGroup); c < (gr + 1) * kGroup; c++)
-            if (sel_s[c]) s += qp[hl * kD + c];
-        qgsum[(qrow0 + hl) * kNG + gr] = (float)s;
+        for (int c = (r == 0 ? 1 : 0); c < kGroup; c++)
+            if (sel_s[r * kGroup + c]) s += qp[hl * kGroup + c];
+        qgsum[(qrow0 + hl) * kNG + r] = (float)s;
     }
+    cluster.sync();                                // keep e2own alive until all have read it
 }
 
 }  // namespace
@@ -108,10 +124,10 @@ select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, int H
 cudaError_t launch_select(const kvq_cache &c, const void *q, int dtype, int Hq, const double *Ainvt,
                           int k, int32_t *idx, float *qsel, float *qgsum, cudaStream_t st) {
     const int g = Hq / c.n_kv_heads;
-    const size_t smem = (size_t)(kD * kD + 2 * g * kD) * sizeof(double);
-    constexpr int kMaxSmem = (kD * kD + 2 * 32 * kD) * (int)sizeof(double);      // g <= 32
+    const size_t smem = (size_t)(kD * kGroup + g * kD + g * kGroup) * sizeof(double);
+    constexpr int kMaxSmem = (kD * kGroup + 32 * kD + 32 * kGroup) * (int)sizeof(double);   // g <= 32
     static std::atomic<uint64_t> done_f32{0}, done_bf16{0};
-    dim3 grid((unsigned)c.n_kv_heads, (unsigned)c.batch);
+    dim3 grid((unsigned)kCtas, (unsigned)c.n_kv_heads, (unsigned)c.batch);
     cudaError_t e;
     if (dtype == KVQ_DTYPE_F32) {
         e = set_smem_once(select_kernel<float>, kMaxSmem, done_f32);

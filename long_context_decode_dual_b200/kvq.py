@@ -8,6 +8,7 @@ Names follow the C entry points:
   kvq_append           -> append(cache, K, V, A)
   kvq_select_channels  -> select_channels(cache, q, Ainvt, sparsity)
   kvq_decode_attn      -> decode_attn(cache, sel)
+  kvq_decode_step      -> decode_step(cache, q, k_new, v_new, A, Ainvt, sparsity)
   kvq_bf16_decode_attn -> bf16_decode_attn(q, K, V)
 """
 from __future__ import annotations
@@ -54,7 +55,7 @@ EXPORTS = (
     "kvq_select_channels", "kvq_decode_workspace", "kvq_decode_attn",
     "kvq_bf16_decode_workspace", "kvq_bf16_decode_attn", "kvq_read_status",
     "kvq_status_string", "kvq_version", "kvq_decode_static_scratch_bytes",
-    "kvq_decode_attn_static",
+    "kvq_decode_attn_static", "kvq_decode_step",
 )
 
 
@@ -85,6 +86,7 @@ def lib() -> ctypes.CDLL:
             "kvq_version": (I, []),
             "kvq_decode_static_scratch_bytes": (S, []),
             "kvq_decode_attn_static": (I, [C, I, P, P, P, I, P, P]),
+            "kvq_decode_step": (I, [C, P, P, P, I, I, I, P, P, ctypes.c_float, P, P, P, P, P, S, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -232,6 +234,35 @@ def decode_attn(cache: KVCache, sel: Selection, out: Optional[torch.Tensor] = No
     return out
 
 
+def decode_step(cache: KVCache, q: torch.Tensor, k_new: Optional[torch.Tensor], v_new: Optional[torch.Tensor],
+                A: torch.Tensor, Ainvt: torch.Tensor, sparsity: float, sel: Optional[Selection] = None,
+                out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                stream=None) -> tuple[torch.Tensor, Selection]:
+    """kvq_decode_step: append k_new / v_new [B][Hkv][n_new][128], select the
+    channels of q [B][Hq][128], decode; returns (out [B][Hq][128] f32, sel)."""
+    assert q.is_contiguous() and A.is_contiguous() and Ainvt.is_contiguous()
+    assert A.dtype == torch.float64 and Ainvt.dtype == torch.float64
+    B, Hq = cache.batch, int(q.shape[1])
+    n_new = 0 if k_new is None else int(k_new.shape[2])
+    if n_new:
+        assert k_new.is_contiguous() and v_new.is_contiguous() and k_new.dtype == q.dtype == v_new.dtype
+    k = num_selected(sparsity)
+    if k < 0:
+        raise KvqError("kvq_num_selected", -1)
+    if sel is None:
+        sel = alloc_selection(cache, Hq, k, q.device)
+    assert sel.k == k
+    if out is None:
+        out = torch.empty(B, Hq, HEAD_DIM, dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = alloc_workspace(decode_workspace_bytes(cache, Hq, k), q.device)
+    _check("kvq_decode_step", lib().kvq_decode_step(
+        ctypes.byref(cache.desc), _ptr(q), _ptr(k_new if n_new else None), _ptr(v_new if n_new else None),
+        _dtype_code(q), Hq, n_new, _ptr(A), _ptr(Ainvt), float(sparsity), _ptr(sel.idx), _ptr(sel.qsel),
+        _ptr(sel.qgsum), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+    return out, sel
+
+
 def decode_attn_static(cache: KVCache, sel: Selection, out: Optional[torch.Tensor] = None,
                        stream=None) -> torch.Tensor:
     """kvq_decode_attn_static: decode without a caller workspace.
@@ -287,17 +318,20 @@ class DecodeStep:
 
     Fill ``q`` [B][Hq][128] and ``k_new`` / ``v_new`` [B][Hkv][1][128] (f32 or
     bf16, the dtype given), call :meth:`run`; the result is in ``out``
-    [B][Hq][128] f32.  :meth:`capture` records the three calls once (after at
-    least one eager :meth:`run`, so every kernel is loaded); later runs replay
-    the graph.  :meth:`run_host` copies the inputs from (pinned) host tensors
-    and the output back, around the same step.
+    [B][Hq][128] f32.  ``fused`` (default) makes the step one kvq_decode_step
+    call; otherwise it is kvq_append, kvq_select_channels and kvq_decode_attn.
+    :meth:`capture` records the step once (after at least one eager
+    :meth:`run`, so every kernel is loaded); later runs replay the graph.
+    :meth:`run_host` copies the inputs from (pinned) host tensors and the
+    output back, around the same step.
     """
 
     def __init__(self, cache: KVCache, A: torch.Tensor, Ainvt: torch.Tensor, sparsity: float,
-                 n_q_heads: int, dtype: torch.dtype = torch.bfloat16):
+                 n_q_heads: int, dtype: torch.dtype = torch.bfloat16, fused: bool = True):
         dev = cache.pages.device
         B, Hkv = cache.batch, cache.n_kv_heads
         self.cache, self.A, self.Ainvt, self.sparsity = cache, A, Ainvt, float(sparsity)
+        self.fused = fused
         self.q = torch.zeros(B, n_q_heads, HEAD_DIM, dtype=dtype, device=dev)
         self.k_new = torch.zeros(B, Hkv, 1, HEAD_DIM, dtype=dtype, device=dev)
         self.v_new = torch.zeros(B, Hkv, 1, HEAD_DIM, dtype=dtype, device=dev)
@@ -309,22 +343,32 @@ class DecodeStep:
         self.decode_events = None      # optional (start, end) events around the decode call
 
     def _pre(self):
-        append(self.cache, self.k_new, self.v_new, self.A)
-        select_channels(self.cache, self.q, self.Ainvt, self.sparsity, out=self.sel)
+        if not self.fused:
+            append(self.cache, self.k_new, self.v_new, self.A)
+            select_channels(self.cache, self.q, self.Ainvt, self.sparsity, out=self.sel)
 
     def _decode(self):
-        decode_attn(self.cache, self.sel, out=self.out, ws=self.ws)
+        if self.fused:
+            decode_step(self.cache, self.q, self.k_new, self.v_new, self.A, self.Ainvt, self.sparsity,
+                        sel=self.sel, out=self.out, ws=self.ws)
+        else:
+            decode_attn(self.cache, self.sel, out=self.out, ws=self.ws)
 
     def time_decode(self) -> None:
-        """Record timing events around the decode call of every later run."""
+        """Record timing events around the decode call (the whole fused step)
+        of every later run."""
         self.decode_events = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
 
     def capture(self) -> None:
-        """Record the step as two CUDA graphs (append + select, decode); the
-        decode timing events, if any, are recorded between the two replays."""
-        pre, dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        with torch.cuda.graph(pre):
-            self._pre()
+        """Record the step as CUDA graphs: append + select (unfused only) and
+        the decode call; the decode timing events, if any, are recorded
+        between the replays."""
+        pre = None
+        if not self.fused:
+            pre = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(pre):
+                self._pre()
+        dec = torch.cuda.CUDAGraph()
         with torch.cuda.graph(dec):
             self._decode()
         self.graph = (pre, dec)
@@ -332,7 +376,8 @@ class DecodeStep:
     def run(self) -> torch.Tensor:
         ev = self.decode_events
         if self.graph is not None:
-            self.graph[0].replay()
+            if self.graph[0] is not None:
+                self.graph[0].replay()
         else:
             self._pre()
         if ev is not None:

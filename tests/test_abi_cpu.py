@@ -52,15 +52,18 @@ def test_validation_rejects_before_launch():
     mis = kvq.CacheDesc(1, 1, 128, 32, 2, 128, 0x1010, 256, 256)  # pages not 256-aligned
     assert L.kvq_append(ctypes.byref(mis), 8, 8, 0, 1, 8, None) == -6
     ok = kvq.CacheDesc(1, 1, 128, 32, 2, 128, 0x1000, 256, 256)
-    assert L.kvq_append(ctypes.byref(ok), 8, 8, 0, -1, 8, None) == -1
-    assert L.kvq_append(ctypes.byref(ok), 8, 8, 7, 1, 8, None) == -1             # dtype
-    assert L.kvq_append(ctypes.byref(ok), 8, 8, 0, 129, 8, None) == -3          # > capacity
-    assert L.kvq_append(ctypes.byref(ok), 8, 8, 0, 0, 8, None) == 0             # no-op
+    assert L.kvq_append(ctypes.byref(ok), 8, 8, 0, -1, 16, None) == -1
+    assert L.kvq_append(ctypes.byref(ok), 8, 8, 7, 1, 16, None) == -1            # dtype
+    assert L.kvq_append(ctypes.byref(ok), 8, 8, 0, 1, 8, None) == -6             # A not 16-aligned
+    assert L.kvq_append(ctypes.byref(ok), 8, 8, 0, 129, 16, None) == -3         # > capacity
+    assert L.kvq_append(ctypes.byref(ok), 8, 8, 0, 0, 16, None) == 0            # no-op
     two = kvq.CacheDesc(1, 2, 128, 32, 2, 128, 0x1000, 256, 256)
     assert L.kvq_select_channels(ctypes.byref(two), 8, 0, 3, 8, ctypes.c_float(0.4), 8, 8, 8,
                                  None, None) == -2                              # 3 % 2 heads
     assert L.kvq_select_channels(ctypes.byref(two), 8, 0, 4, 8, ctypes.c_float(1.5), 8, 8, 8,
                                  None, None) == -1                              # sparsity
+    assert L.kvq_select_channels(ctypes.byref(two), 8, 0, 4, 8, ctypes.c_float(0.4), 8, 8, 8,
+                                 None, None) == -6                              # Ainvt not 16-aligned
     assert L.kvq_decode_attn(ctypes.byref(two), 6, 8, 8, 8, 77, 8, 8, 1 << 20, None) == -2  # g = 3
     assert L.kvq_decode_attn(ctypes.byref(two), 4, 8, 8, 8, 0, 8, 8, 1 << 20, None) == -1   # k = 0
     assert L.kvq_bf16_decode_attn(8, 8, 8, 1, 3, 2, 10, 8, 8, 1 << 20, None) == -2

@@ -14,7 +14,7 @@ from long_context_decode_dual_b200 import kvq
 from long_context_decode_dual_b200 import workloads as W
 from oracle import oracle as orc
 
-from helpers import Case, dev64, expected_qsel_qgsum, rel_errors, to_dev
+from helpers import Case, check_pages, dev64, expected_qsel_qgsum, rel_errors, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -22,18 +22,7 @@ TOL_MAX = 2e-3
 TOL_MEAN = 1e-3
 
 
-def _check_pages(case: Case, cache: kvq.KVCache, units=None, n=None):
-    pages = cache.pages.cpu().numpy()
-    wl = case.wl
-    pb = kvq.page_bytes(wl.bits)
-    pages = pages.reshape(wl.batch, wl.n_kv_heads, case.capacity // 128, pb)
-    units = units or [(b, h) for b in range(wl.batch) for h in range(wl.n_kv_heads)]
-    for b, h in units:
-        ref = case.oracle_unit(b, h, n)
-        got = pages[b, h]
-        if not np.array_equal(got, ref):
-            bad = np.argwhere(got != ref)
-            raise AssertionError(f"unit {(b, h)}: {len(bad)} bytes differ, first (page, byte) {bad[:4].tolist()}")
+_check_pages = check_pages
 
 
 def _cases_small():
@@ -249,13 +238,14 @@ def test_full_size_sampled(name, units, sparsities):
         _decode_and_compare(case, cache, s, steps=(0,), units=units)
 
 
-def test_decode_step_graph_replay_matches_eager():
-    """The captured step (append -> select -> decode as one CUDA graph) gives
-    the same bytes and outputs as the same calls launched one by one."""
+@pytest.mark.parametrize("fused", [True, False])
+def test_decode_step_graph_replay_matches_eager(fused):
+    """The captured step (one fused launch, or append -> select -> decode)
+    gives the same bytes and outputs as the same calls launched one by one."""
     wl = W.workload("llama8b_b8_32k", batch=2)
     case = Case(wl, n_ctx=400)
     A, Ai = dev64(case.A), dev64(case.Ai)
-    steps = [kvq.DecodeStep(case.gpu_cache(), A, Ai, 0.4, wl.n_q_heads) for _ in range(2)]
+    steps = [kvq.DecodeStep(case.gpu_cache(), A, Ai, 0.4, wl.n_q_heads, fused=fused) for _ in range(2)]
     outs = [[], []]
     for i in range(4):
         kn, vn = W.make_step_kv(wl, i)
