@@ -40,7 +40,7 @@ DEFAULT_WORKLOAD = "longctx_b1_128k"
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 CSRC = os.path.join(ROOT, "long_context_decode_dual_b200", "csrc")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.txt")
+PROFILES = os.path.join(ROOT, "profiles")
 
 
 def log(*a):
@@ -59,6 +59,8 @@ def measured_peaks():
 
 
 def decode_source_hash() -> str:
+    """Hash of the sources of the timed kernel (the fused step and the decode
+    kernels share kvq_decode_mma.cu and the internal header)."""
     h = hashlib.sha256()
     for name in sorted(os.listdir(CSRC)):
         if name.startswith("kvq_decode") or name.endswith(".cuh"):
@@ -68,23 +70,33 @@ def decode_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def committed_traffic(workload: str):
-    """DRAM bytes per decode launch from a committed ncu summary, if it was
-    taken on the current decode kernel source for this workload."""
+def committed_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` from a committed ncu summary
+    (profiles/traffic_<kernel>_<workload>.txt), if it was taken on the
+    current kernel source."""
     try:
         kv = {}
-        with open(TRAFFIC_FILE) as f:
+        with open(os.path.join(PROFILES, f"traffic_{kernel}_{workload}.txt")) as f:
             for line in f:
                 if ":" in line and not line.startswith("#"):
                     a, b = line.split(":", 1)
                     kv[a.strip()] = b.strip()
         if kv.get("kernel_source_sha") != decode_source_hash():
             return None, "stale"
-        if kv.get("workload") != workload:
-            return None, "other workload"
         return float(kv["dram_bytes_per_launch"]), kv.get("note", "")
     except Exception:
         return None, "absent"
+
+
+def algorithmic_step_bytes(wl: W.Workload, k: int, length: int) -> int:
+    """Bytes one fused step launch must move: the decode bytes over `length`
+    tokens, A^{-T} of every KV head and the A columns the appending CTAs read
+    (float64, 128 x 128 each), the query rows and the new token's key and
+    value (bf16 or f32)."""
+    elem = 2 if wl.dtype == "bf16" else 4
+    transforms = 2 * wl.n_kv_heads * 128 * 128 * 8
+    inputs = wl.batch * (wl.n_q_heads + 2 * wl.n_kv_heads) * 128 * elem
+    return algorithmic_decode_bytes(wl, k, length) + transforms + inputs
 
 
 def algorithmic_decode_bytes(wl: W.Workload, k: int, length: int) -> int:
@@ -275,7 +287,10 @@ def run_ours(args):
         step.k_new.copy_(kv_pool[i % n_pool][0])
         step.v_new.copy_(kv_pool[i % n_pool][1])
 
-    launches_per_step = 3   # one-token append (fused length advance), select, decode (fused merge)
+    # fused: one kvq_decode_step launch; unfused: one-token append (with its
+    # length advance), select, decode (with its merge)
+    launches_per_step = 1 if args.fused else 3
+    alg_fn = algorithmic_step_bytes if args.fused else algorithmic_decode_bytes
     step.time_decode()
     length = wl.n_ctx
     for i in range(args.warmup):
@@ -310,7 +325,7 @@ def run_ours(args):
             length += 1
             step_ms.append(a.elapsed_time(b_))
             dec_ms.append(step.decode_events[0].elapsed_time(step.decode_events[1]))
-            alg_bytes.append(algorithmic_decode_bytes(wl, k, length))
+            alg_bytes.append(alg_fn(wl, k, length))
             tokens.append(B * Hkv * length)
     if world > 1:
         dist.barrier()
@@ -324,9 +339,9 @@ def run_ours(args):
 
     # roofline of the dominant kernel (decode partial + merge, timed together)
     hbm_peak, peak_src = measured_peaks()
-    alg_bytes = [algorithmic_decode_bytes(wl, k, tok // (B * Hkv)) for tok in tokens]
+    alg_bytes = [alg_fn(wl, k, tok // (B * Hkv)) for tok in tokens]
     achieved = statistics.mean(ab / (ms * 1e-3) for ab, ms in zip(alg_bytes, dec_ms)) / 1e9
-    traffic, traffic_note = committed_traffic(wl.name)
+    traffic, traffic_note = committed_traffic("step_mma" if args.fused else "decode_mma", wl.name)
 
     # end to end through the Python binding with host buffers
     e2e = None
@@ -397,7 +412,8 @@ def run_ours(args):
         "config": config_dict(wl, k),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "traffic": traffic,
-                     "kernel": "decode partial + merge (kvq_decode_attn)",
+                     "kernel": ("fused step (kvq_decode_step: append + select + decode + merge)" if args.fused
+                                else "decode partial + merge (kvq_decode_attn)"),
                      "peak_source": f"{peak_src} hbm_gbs", "traffic_note": traffic_note},
         "decode_ms": statistics.mean(dec_ms),
         "step_launch": "cuda graph" if args.graph else "eager",

@@ -21,9 +21,9 @@ cudaError_t launch_step_mma(const kvq_cache &c, int Hq, const void *q, const voi
 // other shapes use the CUDA-core kernel.
 static bool use_mma(const kvq_cache &c, int Hq) { return c.bits == 2 && Hq == 4 * c.n_kv_heads; }
 
-// Splits per (sequence, KV head): enough CTAs to fill the SMs, at least two
-// pages per split, and at most kMaxSplits (the merge keeps two floats per
-// split and head in the kernels' staging memory).
+// Splits per (sequence, KV head): enough CTAs to fill the SMs (the
+// tensor-core plan: decode_mma_splits), at least two pages per split for the
+// CUDA-core kernel, and at most kMaxSplits (which bounds the workspace).
 constexpr int kMaxSplits = 256;
 
 int decode_splits(const kvq_cache &c, int Hq, int k, int num_sms) {

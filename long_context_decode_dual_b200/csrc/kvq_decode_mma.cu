@@ -105,9 +105,9 @@ constexpr int kOffAHi = 0;                                        // A rows 64..
 constexpr int kOffALo = kD * kBlkRowBytes;                        // A rows 0..63
 constexpr int kOffE2 = kOffALo + 64 * kBlkRowBytes;               // double[128]
 constexpr int kOffRank = kOffE2 + kD * (int)sizeof(double);       // int[2][128]
-constexpr int kOffQp = 0;                                         // double[4][128], after the append
+constexpr int kOffQp = kStageBytes;                               // double[4][128] in stage[0][1], after the append
 static_assert(kOffRank + 2 * kD * (int)sizeof(int) <= kPairs * 2 * kStageBytes, "scratch fits the stages");
-static_assert(kOffQp + 4 * kD * (int)sizeof(double) <= kOffALo, "q' copy below the low rows of A");
+static_assert(kOffQp + 4 * kD * (int)sizeof(double) <= 2 * kStageBytes, "q' copy inside stage[0][1]");
 struct PexScratch {                    // in MmaShared::pex
     float qin[4][kD];                  // query rows (bf16 / f32 inputs are exact in f32)
     float ks[kStepMaxNew][kD];         // new key rows
@@ -311,13 +311,23 @@ __device__ __forceinline__ void issue_keys(MmaShared &sh, int pair, int st, cons
     }
 }
 
+// A whole page into stage st of a pair in one copy (before the copy list is
+// known; at most one more 64-byte chunk per unselected pair of rows than the
+// list would fetch, and the memory system fetches those chunks anyway).
+__device__ __forceinline__ void issue_page(MmaShared &sh, int pair, int st, const uint8_t *src) {
+    const uint32_t bar = smem_u32(&sh.mbar[pair][st]);
+    mbar_arrive_expect_tx(bar, (uint32_t)kStageBytes);
+    bulk_g2s(smem_u32(sh.stage[pair][st]), src, (uint32_t)kStageBytes, bar);
+}
+
 // The page loop and the merges: pages [sp.blk0, sp.blk1) of the unit, pair
-// `pair` taking every kPairs-th.  `first_tail_issued`: the tail of the pair's
-// first page is already in flight into stage 0.
+// `pair` taking every kPairs-th.  `first_issued`: the pair's first page is
+// already in flight, whole, into stage 0 (one copy that arrives on the
+// barrier).
 __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restrict__ unit_pages, int len,
                                           Split sp, int S, int s, size_t qrow0, float *__restrict__ part_o,
                                           float2 *__restrict__ part_ml, float *__restrict__ out,
-                                          uint32_t *counter, uint32_t *status, bool first_tail_issued) {
+                                          uint32_t *counter, uint32_t *status, bool first_issued) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int pair = warp >> 1, half = warp & 1;
     const int gid = lane >> 2, tig = lane & 3;
@@ -350,9 +360,9 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
     uint32_t late = 0;            // stages whose last wait gave up, with the parity waited for
     const bool issuer = (tid & 63) == 0;
     const int first = sp.blk0 + pair;
-    if (issuer && first < sp.blk1) {
+    if (issuer && first < sp.blk1 && !first_issued) {
         const uint8_t *src = unit_pages + (size_t)first * page_bytes(2);
-        if (!first_tail_issued) issue_tail(sh, pair, 0, src);
+        issue_tail(sh, pair, 0, src);
         issue_keys(sh, pair, 0, src);
     }
     for (int pg = first; pg < sp.blk1; pg += kPairs, it++) {
@@ -775,7 +785,14 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
         for (int c = 0; c < kD; c++) acc = fma((double)px.qin[hl][c], aiT[c][jj], acc);
         sh.qp_own[hl][jj] = acc;
     }
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");   // staging memory goes to bulk copies next
     __syncthreads();                                // A^{-T} block no longer needed
+    // A cluster that appends nothing requests its pairs' first pages now,
+    // whole, so their DRAM latency overlaps the channel choice (stage[p][0]
+    // is clear of the scratch still in use: energies, ranks, q' copy).
+    const bool early = nw == 0;
+    if (early && (tid & 63) == 0 && sp.blk0 + (tid >> 6) < sp.blk1)
+        issue_page(sh, tid >> 6, 0, unit_pages + (size_t)(sp.blk0 + (tid >> 6)) * page_bytes(2));
     if (nw > 0) {
         // K'[t][j] = sum_c K[t][c] A[c][j], fma chain c = 0..127 from 0.0, for
         // token w0 + warp / 2 and channel j = 64r + jj: rows 0..63 of A while
@@ -879,7 +896,7 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
     build_plan(sh, tid, warp, lane);
 
     run_pages(sh, unit_pages, len, sp, S, s, qrow0, part_o, part_ml, out,
-              status + 1 + B + unit, status, false);
+              status + 1 + B + unit, status, early);
     cluster_wait();            // the other CTA no longer reads this CTA's shared memory
 }
 
