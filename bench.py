@@ -223,6 +223,30 @@ def config_dict(wl: W.Workload, k: int):
             "l2": "flushed between steps (256 MiB write, outside the timed events)"}
 
 
+# ------------------------------------------------------------- ranks
+# More than one GPU runs independent replicas (weak scaling): rank r decodes
+# its own sequences (the workload's seed offset by r), no data crosses GPUs,
+# and the job's time is the slowest rank's.
+def rank_workload(wl: W.Workload, rank: int) -> W.Workload:
+    return wl if rank == 0 else wl.with_(seed=wl.seed + 7919 * rank)
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest x over all ranks (every rank calls this, in the same order)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: float, max_ms: float, world: int) -> float:
+    """Units all ranks processed per second, over the slowest rank's time."""
+    return world * tokens_per_rank / (max_ms * 1e-3)
+
+
 # ------------------------------------------------------------- our arm
 def run_ours(args):
     import torch
@@ -248,7 +272,7 @@ def run_ours(args):
     over = {"bits": args.bits, "n_steps": n_appends}
     if args.sparsity is not None:
         over["sparsity"] = args.sparsity
-    wl = W.workload(args.workload, **over)
+    wl = rank_workload(W.workload(args.workload, **over), rank)
     B, Hq, Hkv = wl.batch, wl.n_q_heads, wl.n_kv_heads
 
     t0 = time.perf_counter()
@@ -329,12 +353,8 @@ def run_ours(args):
             tokens.append(B * Hkv * length)
     if world > 1:
         dist.barrier()
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-    value = world * sum(tokens) / (total_ms * 1e-3)
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
+    value = job_throughput(sum(tokens), total_ms, world)
     assert kvq.read_status(cache) == 0
 
     # roofline of the dominant kernel (decode partial + merge, timed together)
@@ -364,13 +384,10 @@ def run_ours(args):
             e_ms += a.elapsed_time(b_)
             length += 1
             e_tok.append(B * Hkv * length)
-        if world > 1:
-            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(e_ms, world, dev)
         elem = 2 if wl.dtype == "bf16" else 4
         h2d = (B * Hq * 128 + 2 * B * Hkv * 128) * elem
-        e2e = {"value": world * sum(e_tok) / (e_ms * 1e-3), "unit": UNIT,
+        e2e = {"value": job_throughput(sum(e_tok), e_ms, world), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": B * Hq * 128 * 4}
 
     # the unpruned BF16 comparator on the same keys and values
