@@ -34,6 +34,15 @@
  *                               1/sqrt(d) normalisation) and §3.4 (one softmax
  *                               over all scores, then value aggregation).
  *   orc_attention               textbook softmax(q K^T / sqrt(d)) V.
+ *   orc_protected_slot, orc_protect_store, orc_protect_dequant
+ *                               Dual-QK §3.3 (the first 64 and the most
+ *                               recent 256 tokens kept in BF16 for keys and
+ *                               values, same query-channel mask) and §3.4
+ *                               (all precision tiers share one softmax):
+ *                               a sink slot per early position, a ring of
+ *                               slots for the recent window, and the
+ *                               dequantized cache with the protected
+ *                               positions replaced by their BF16 values.
  *
  * Parity pins: every function here is checked by the CPU test suite against
  * closed forms, library routines or brute force (see tests/test_oracle_*.py).
@@ -369,4 +378,66 @@ void orc_attention(const double *q, const double *K, const double *V, long n,
     for (int j = 0; j < d; j++) all[j] = j;
     orc_decode_dense(K, V, n, q, g, d, all, d, out);
     free(all);
+}
+
+/* ------------------------------------------------------------------------ */
+/* protected BF16 tier                                                       */
+/* ------------------------------------------------------------------------ */
+/* Positions below n_sink keep slot pos; later positions use a ring of
+ * n_recent slots after them.  -1: the position has no slot.                 */
+long orc_protected_slot(long pos, int n_sink, int n_recent)
+{
+    if (pos < n_sink) return pos;
+    if (n_recent <= 0) return -1;
+    return n_sink + pos % n_recent;
+}
+
+/* Protected set of a sequence of length len: [0, sink_end) and
+ * [recent_start, len).                                                      */
+static void protected_bounds(long len, int n_sink, int n_recent, long *sink_end, long *recent_start)
+{
+    long se = len < n_sink ? len : n_sink;
+    long rs = len - n_recent;
+    if (rs < se) rs = se;
+    *sink_end = se;
+    *recent_start = rs;
+}
+
+int orc_is_protected(long pos, long len, int n_sink, int n_recent)
+{
+    long se, rs;
+    protected_bounds(len, n_sink, n_recent, &se, &rs);
+    return pos < se || (pos >= rs && pos < len);
+}
+
+/* Store tokens pos0 .. pos0+n-1 (K' transformed, V as given; [n][128]) of a
+ * sequence whose length becomes len_after: a token gets its slot when it is
+ * a sink token or one of the last n_recent tokens; each slot holds 128 BF16
+ * key values then 128 BF16 value values.                                    */
+void orc_protect_store(uint16_t *slots, int n_sink, int n_recent, long pos0, long n,
+                       long len_after, const double *Kp, const double *V)
+{
+    for (long i = 0; i < n; i++) {
+        long pos = pos0 + i;
+        if (!(pos < n_sink || (n_recent > 0 && pos >= len_after - n_recent))) continue;
+        long slot = orc_protected_slot(pos, n_sink, n_recent);
+        uint16_t *dst = slots + slot * 2 * ORC_D;
+        for (int c = 0; c < ORC_D; c++) dst[c] = orc_bf16_rne(Kp[i * ORC_D + c]);
+        for (int c = 0; c < ORC_D; c++) dst[ORC_D + c] = orc_bf16_rne(V[i * ORC_D + c]);
+    }
+}
+
+/* Replace the rows of protected positions of a dequantized cache (Khat,
+ * Vhat: [len][128]) by their BF16 values from the slots.                    */
+void orc_protect_dequant(const uint16_t *slots, int n_sink, int n_recent, long len,
+                         double *Khat, double *Vhat)
+{
+    for (long pos = 0; pos < len; pos++) {
+        if (!orc_is_protected(pos, len, n_sink, n_recent)) continue;
+        const uint16_t *src = slots + orc_protected_slot(pos, n_sink, n_recent) * 2 * ORC_D;
+        for (int c = 0; c < ORC_D; c++) {
+            Khat[pos * ORC_D + c] = orc_bf16_to_f64(src[c]);
+            Vhat[pos * ORC_D + c] = orc_bf16_to_f64(src[ORC_D + c]);
+        }
+    }
 }

@@ -68,6 +68,12 @@ def _load():
             lib.orc_select.argtypes = [P, I, I, I, P, P]
             lib.orc_decode_dense.argtypes = [P, P, L, P, I, I, P, I, P]
             lib.orc_attention.argtypes = [P, P, P, L, I, I, P]
+            lib.orc_protected_slot.restype = L
+            lib.orc_protected_slot.argtypes = [L, I, I]
+            lib.orc_is_protected.restype = I
+            lib.orc_is_protected.argtypes = [L, L, I, I]
+            lib.orc_protect_store.argtypes = [P, I, I, L, L, L, P, P]
+            lib.orc_protect_dequant.argtypes = [P, I, I, L, P, P]
             _lib = lib
     return _lib
 
@@ -213,4 +219,42 @@ def decode_unit(unit: np.ndarray, bits: int, n: int, qp, sparsity: float):
     k = num_selected(sparsity)
     idx, _ = select(qp, k)
     Kh, Vh = dequant_unit(unit, bits, n)
+    return decode_dense(Kh, Vh, qp, idx), idx
+
+
+# ------------------------------------------------------ protected BF16 tier
+def protected_slot(pos: int, n_sink: int, n_recent: int) -> int:
+    """Slot of a position in the protected tier (Dual-QK §3.3), -1 if none."""
+    return int(_load().orc_protected_slot(pos, n_sink, n_recent))
+
+
+def is_protected(pos: int, length: int, n_sink: int, n_recent: int) -> bool:
+    return bool(_load().orc_is_protected(pos, length, n_sink, n_recent))
+
+
+def new_slots(n_sink: int, n_recent: int) -> np.ndarray:
+    """Zeroed protected slots of one unit: uint16 [n_sink + n_recent][256]
+    (128 BF16 key values, then 128 BF16 value values)."""
+    return np.zeros((n_sink + n_recent, 2 * D), dtype=np.uint16)
+
+
+def protect_store(slots: np.ndarray, n_sink: int, n_recent: int, pos0: int, Kp, V, len_after: int) -> None:
+    """Store the BF16 copies of tokens pos0.. that belong to the protected
+    tier of a sequence of length len_after."""
+    Kp = _f64(Kp).reshape(-1, D)
+    V = _f64(V).reshape(-1, D)
+    assert slots.flags.c_contiguous and slots.dtype == np.uint16
+    assert slots.shape == (n_sink + n_recent, 2 * D)
+    _load().orc_protect_store(_p(slots), n_sink, n_recent, pos0, Kp.shape[0], len_after, _p(Kp), _p(V))
+
+
+def decode_unit_protected(unit: np.ndarray, slots: np.ndarray, bits: int, n: int, qp, sparsity: float,
+                          n_sink: int, n_recent: int):
+    """decode_unit with the protected tier: the first n_sink and the last
+    n_recent tokens are read from their BF16 slots, the rest from the INT2
+    codes; one softmax over all of them (Dual-QK §3.3, §3.4)."""
+    k = num_selected(sparsity)
+    idx, _ = select(qp, k)
+    Kh, Vh = dequant_unit(unit, bits, n)
+    _load().orc_protect_dequant(_p(np.ascontiguousarray(slots)), n_sink, n_recent, n, _p(Kh), _p(Vh))
     return decode_dense(Kh, Vh, qp, idx), idx
