@@ -88,7 +88,7 @@ def committed_traffic(kernel: str, workload: str):
         return None, "absent"
 
 
-def algorithmic_step_bytes(wl: W.Workload, k: int, length: int) -> int:
+def algorithmic_step_bytes(wl: W.Workload, k: int, length: int, protect=(0, 0)) -> int:
     """Bytes one fused step launch must move: the decode bytes over `length`
     tokens, A^{-T} of every KV head and the A columns the appending CTAs read
     (float64, 128 x 128 each), the query rows and the new token's key and
@@ -96,18 +96,24 @@ def algorithmic_step_bytes(wl: W.Workload, k: int, length: int) -> int:
     elem = 2 if wl.dtype == "bf16" else 4
     transforms = 2 * wl.n_kv_heads * 128 * 128 * 8
     inputs = wl.batch * (wl.n_q_heads + 2 * wl.n_kv_heads) * 128 * elem
-    return algorithmic_decode_bytes(wl, k, length) + transforms + inputs
+    return algorithmic_decode_bytes(wl, k, length, protect) + transforms + inputs
 
 
-def algorithmic_decode_bytes(wl: W.Workload, k: int, length: int) -> int:
-    """Bytes one decode launch must read: per (sequence, KV head) and page, the
-    k-1 selected key rows, the value codes, channel 0 and both metadata
-    blocks; plus the selection inputs and the partial outputs are ignored
-    (they are < 0.1%)."""
+def algorithmic_decode_bytes(wl: W.Workload, k: int, length: int, protect=(0, 0)) -> int:
+    """Bytes one decode launch must read: per (sequence, KV head) and page of
+    coded tokens, the k-1 selected key rows, the value codes, channel 0 and
+    both metadata blocks; with a protected tier (n_sink, n_recent), the pages
+    cover only the coded tokens and each protected token adds its k selected
+    BF16 key channels and its 128 BF16 values.  The selection inputs and the
+    partial outputs are ignored (< 0.1%)."""
+    n_sink, n_recent = protect
     R = 128 * wl.bits // 8
     per_page = (k - 1) * R + 128 * R + 256 + 2048 + 2048
-    n_pages = (length + 127) // 128
-    return wl.batch * wl.n_kv_heads * n_pages * per_page
+    sink_end = min(n_sink, length)
+    recent_start = max(sink_end, length - n_recent)
+    n_pages = (recent_start + 127) // 128
+    n_prot = sink_end + (length - recent_start)
+    return wl.batch * wl.n_kv_heads * (n_pages * per_page + n_prot * (2 * k + 256))
 
 
 class ClockSampler:
@@ -215,12 +221,15 @@ def run_reference(args):
     return 0
 
 
-def config_dict(wl: W.Workload, k: int):
-    return {"workload": wl.name, "batch": wl.batch, "n_q_heads": wl.n_q_heads,
-            "n_kv_heads": wl.n_kv_heads, "context": wl.n_ctx, "head_dim": 128, "bits": wl.bits,
-            "group": 32, "sparsity": wl.sparsity, "k": k,
-            "step": "append 1 token + query transform/select + decode + merge",
-            "l2": "flushed between steps (256 MiB write, outside the timed events)"}
+def config_dict(wl: W.Workload, k: int, protect=(0, 0)):
+    d = {"workload": wl.name, "batch": wl.batch, "n_q_heads": wl.n_q_heads,
+         "n_kv_heads": wl.n_kv_heads, "context": wl.n_ctx, "head_dim": 128, "bits": wl.bits,
+         "group": 32, "sparsity": wl.sparsity, "k": k,
+         "step": "append 1 token + query transform/select + decode + merge",
+         "l2": "flushed between steps (256 MiB write, outside the timed events)"}
+    if protect != (0, 0):
+        d["protected_bf16"] = {"sink": protect[0], "recent": protect[1]}
+    return d
 
 
 # ------------------------------------------------------------- ranks
@@ -290,7 +299,8 @@ def run_ours(args):
     Kd, Vd = dev_in(K_np), dev_in(V_np)
     stream = torch.cuda.current_stream(dev)
 
-    cache = kvq.new_cache(B, Hkv, wl.capacity, wl.bits, device=dev)
+    protect = (64, 256) if args.protect else (0, 0)
+    cache = kvq.new_cache(B, Hkv, wl.capacity, wl.bits, device=dev, n_sink=protect[0], n_recent=protect[1])
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record()
     kvq.append(cache, Kd, Vd, A)
@@ -349,7 +359,7 @@ def run_ours(args):
             length += 1
             step_ms.append(a.elapsed_time(b_))
             dec_ms.append(step.decode_events[0].elapsed_time(step.decode_events[1]))
-            alg_bytes.append(alg_fn(wl, k, length))
+            alg_bytes.append(alg_fn(wl, k, length, protect))
             tokens.append(B * Hkv * length)
     if world > 1:
         dist.barrier()
@@ -359,7 +369,7 @@ def run_ours(args):
 
     # roofline of the dominant kernel (decode partial + merge, timed together)
     hbm_peak, peak_src = measured_peaks()
-    alg_bytes = [alg_fn(wl, k, tok // (B * Hkv)) for tok in tokens]
+    alg_bytes = [alg_fn(wl, k, tok // (B * Hkv), protect) for tok in tokens]
     achieved = statistics.mean(ab / (ms * 1e-3) for ab, ms in zip(alg_bytes, dec_ms)) / 1e9
     traffic, traffic_note = committed_traffic("step_mma" if args.fused else "decode_mma", wl.name)
 
@@ -426,7 +436,7 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": config_dict(wl, k),
+        "config": config_dict(wl, k, protect),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "traffic": traffic,
                      "kernel": ("fused step (kvq_decode_step: append + select + decode + merge)" if args.fused
@@ -462,6 +472,8 @@ def main():
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-comparator", dest="comparator", action="store_false")
+    ap.add_argument("--protect", action="store_true",
+                    help="keep the first 64 and the last 256 tokens in BF16 (the pages' protected tier)")
     ap.add_argument("--unfused", dest="fused", action="store_false",
                     help="run the step as three launches (append, select, decode) instead of one")
     ap.add_argument("--no-graph", dest="graph", action="store_false",

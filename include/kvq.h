@@ -48,6 +48,23 @@
  *  Pages of one (sequence b, KV head h) are contiguous; unit (b, h) starts at
  *  byte ((b * n_kv_heads + h) * (capacity / 128)) * page_bytes.
  *  Dequantized value = scale * code + zero.
+ *
+ * Protected BF16 tier (optional; Dual-QK §3.3 keeps the first 64 and the most
+ * recent 256 tokens in BF16 for keys and values, with the same query-channel
+ * mask, §3.4 one softmax over all tiers)
+ * ---------------------------------------------------------------------------
+ *  With n_sink + n_recent > 0 the page array is followed, per unit (b, h) in
+ *  the same order, by n_sink + n_recent slots of 512 bytes: 128 bf16 values of
+ *  the transformed key, then 128 bf16 values of the value (round to nearest
+ *  even).  Position p owns slot p if p < n_sink, else slot n_sink + p mod
+ *  n_recent (a ring over the recent window).  Every appended token is coded in
+ *  the pages as usual; a token is also written to its slot if p < n_sink or
+ *  if it is among the last n_recent tokens once the append completes.  For a
+ *  sequence of length L, positions [0, min(n_sink, L)) and
+ *  [max(min(n_sink, L), L - n_recent), L) are read from their slots and all
+ *  others from the codes.
+ *  Bytes of token positions at or beyond seq_len are zero in the pages (as
+ *  kvq_cache_init leaves them; appends write each position once).
  */
 #ifndef KVQ_H
 #define KVQ_H
@@ -102,7 +119,13 @@ typedef struct {
                              completion counters the calls use to finish a
                              step in the same kernel; every call leaves them
                              at zero (kvq_cache_init zeroes them)           */
+    int32_t n_sink;       /* protected BF16 tier: first tokens kept, >= 0     */
+    int32_t n_recent;     /* and most recent tokens kept, >= 0; together at
+                             most KVQ_MAX_PROTECTED (0 and 0: no tier)       */
 } kvq_cache;
+
+/* Largest n_sink + n_recent. */
+#define KVQ_MAX_PROTECTED 1024
 
 /* Words of the cache's status array: 1 + batch + batch * n_kv_heads
  * (0 if an argument is below 1). */
@@ -111,7 +134,8 @@ size_t kvq_status_words(int batch, int n_kv_heads);
 /* Bytes of one 128-token page for the given code width (0 if unsupported). */
 size_t kvq_page_bytes(int bits);
 
-/* Bytes of the whole page array of a cache (0 if the descriptor is invalid). */
+/* Bytes of the whole page array of a cache, protected slots included (0 if
+ * the descriptor is invalid). */
 size_t kvq_cache_bytes(const kvq_cache *cache);
 
 /* Zero every page, every seq_len entry and the status array (stream-ordered).

@@ -51,7 +51,7 @@ __global__ void __launch_bounds__(128)
 append_kernel(uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len,
               uint32_t *__restrict__ status, const Tin *__restrict__ K,
               const Tin *__restrict__ V, const double *__restrict__ A, int Hkv, int NB,
-              int n_new, int capacity) {
+              int n_new, int capacity, int n_sink, int n_recent) {
     constexpr int R = row_bytes(BITS);
     __shared__ double ks[kTile][kD];
     __shared__ double vs[kTile][kD];
@@ -152,6 +152,21 @@ append_kernel(uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len,
             vmeta[meta_word(grp, t0 + tt)] = (uint32_t)sb | ((uint32_t)zb << 16);
     }
     store_row<BITS>(page + off_vcodes(BITS) + (size_t)j * R + t0 * BITS / 8, codes, valid);
+
+    // protected tier: BF16 copies of sink tokens and of the last n_recent
+    // tokens of the sequence once this append completes
+    if (n_sink + n_recent > 0) {
+        uint16_t *slots = reinterpret_cast<uint16_t *>(
+            unit_slots(pages, gridDim.z, Hkv, NB, BITS, (size_t)b * Hkv + h, n_sink + n_recent));
+#pragma unroll
+        for (int tt = 0; tt < kTile; tt++) {
+            const int pos = first + tt;
+            if (!(valid >> tt & 1u) || !stores_slot(pos, len + n_new, n_sink, n_recent)) continue;
+            uint16_t *dst = slots + (size_t)slot_of(pos, n_sink, n_recent) * (kSlotBytes / 2);
+            dst[j] = __bfloat16_as_ushort(__double2bfloat16(acc[tt]));
+            dst[kD + j] = __bfloat16_as_ushort(__double2bfloat16(vs[tt][j]));
+        }
+    }
 }
 
 // Appends of a few tokens (a decode step adds one): one CTA per (sequence,
@@ -170,7 +185,7 @@ __global__ void __launch_bounds__(128)
 append_small_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len,
                     uint32_t *__restrict__ status, const Tin *__restrict__ K,
                     const Tin *__restrict__ V, const double *__restrict__ A, int Hkv, int NB,
-                    int n_new, int capacity) {
+                    int n_new, int capacity, int n_sink, int n_recent) {
     constexpr int R = row_bytes(BITS);
     constexpr int PER = 8 / BITS;
     static_assert(kSmallMax * 32 == 128, "one warp per new token");
@@ -214,6 +229,14 @@ append_small_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len,
         vcode[w][lane] = (uint8_t)quantize_lane<BITS>(v, true, sb, zb);
         if (lane == 0)
             reinterpret_cast<uint32_t *>(page + off_vmeta(BITS))[meta_word(grp, tt)] = (uint32_t)sb | ((uint32_t)zb << 16);
+        // protected tier: BF16 copies (sink tokens, the last n_recent tokens)
+        if (n_sink + n_recent > 0 && stores_slot(pos, len + n_new, n_sink, n_recent)) {
+            uint16_t *dst = reinterpret_cast<uint16_t *>(
+                unit_slots(pages, gridDim.z, Hkv, NB, BITS, (size_t)b * Hkv + h, n_sink + n_recent) +
+                (size_t)slot_of(pos, n_sink, n_recent) * kSlotBytes);
+            dst[j] = __bfloat16_as_ushort(__double2bfloat16(x));
+            dst[kD + j] = __bfloat16_as_ushort(__double2bfloat16(v));
+        }
     }
     __syncthreads();
     if (ok && t < 2 * kGroup) {
@@ -261,13 +284,13 @@ cudaError_t launch_append_t(const kvq_cache &c, const void *K, const void *V, in
         dim3 grid((unsigned)kNG, (unsigned)c.n_kv_heads, (unsigned)c.batch);
         append_small_kernel<Tin, BITS><<<grid, 128, 0, st>>>(
             static_cast<uint8_t *>(c.pages), c.seq_len, c.status, static_cast<const Tin *>(K),
-            static_cast<const Tin *>(V), A, c.n_kv_heads, NB, n_new, c.capacity);
+            static_cast<const Tin *>(V), A, c.n_kv_heads, NB, n_new, c.capacity, c.n_sink, c.n_recent);
         return cudaGetLastError();
     }
     dim3 grid((unsigned)((n_new + kTile - 1) / kTile + 1), (unsigned)c.n_kv_heads, (unsigned)c.batch);
     append_kernel<Tin, BITS><<<grid, 128, 0, st>>>(
         static_cast<uint8_t *>(c.pages), c.seq_len, c.status, static_cast<const Tin *>(K),
-        static_cast<const Tin *>(V), A, c.n_kv_heads, NB, n_new, c.capacity);
+        static_cast<const Tin *>(V), A, c.n_kv_heads, NB, n_new, c.capacity, c.n_sink, c.n_recent);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     advance_kernel<<<(c.batch + 127) / 128, 128, 0, st>>>(c.seq_len, c.batch, n_new, c.capacity);

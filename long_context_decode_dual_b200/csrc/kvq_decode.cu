@@ -10,7 +10,7 @@ cudaError_t launch_decode_simt(const kvq_cache &c, int Hq, const int32_t *idx, c
 cudaError_t launch_decode_mma(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
                               const float *qgsum, int k, float *part_o, float2 *part_ml, int S,
                               float *out, cudaStream_t st);
-int decode_mma_splits(int units, int nblk, int num_sms);
+int decode_mma_splits(int units, int nblk, int num_sms, int tier);
 int step_mma_max_new();
 cudaError_t launch_step_mma(const kvq_cache &c, int Hq, const void *q, const void *k_new, const void *v_new,
                             int dtype, int n_new, const double *A, const double *Ainvt, int k, int32_t *idx,
@@ -30,16 +30,19 @@ int decode_splits(const kvq_cache &c, int Hq, int k, int num_sms) {
     (void)k;
     const int units = c.batch * c.n_kv_heads;
     const int nblk = c.capacity / kT;
+    const int tier = tier_ctas(c);                 // extra splits that read the protected tier
     int S;
     if (use_mma(c, Hq)) {
-        S = decode_mma_splits(units, nblk, num_sms);
+        S = decode_mma_splits(units, nblk, num_sms, tier);
     } else {
         S = (4 * num_sms + units - 1) / units;
         const int max_s = (nblk + 1) / 2 > 0 ? (nblk + 1) / 2 : 1;
         if (S > max_s) S = max_s;
+        if (S < 1) S = 1;
+        S += tier;
     }
     if (S > kMaxSplits) S = kMaxSplits;
-    return S < 1 ? 1 : S;
+    return S;
 }
 
 size_t decode_ws_bytes(const kvq_cache &c, int Hq, int S) {

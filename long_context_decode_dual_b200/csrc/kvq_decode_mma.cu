@@ -321,10 +321,11 @@ __device__ __forceinline__ void issue_page(MmaShared &sh, int pair, int st, cons
 }
 
 // The page loop and the merges: pages [sp.blk0, sp.blk1) of the unit, pair
-// `pair` taking every kPairs-th.  `first_issued`: the pair's first page is
+// `pair` taking every kPairs-th; tokens outside [lo, hi) (beyond the length,
+// or in the protected tier) are left out of the softmax.  `first_issued`: the pair's first page is
 // already in flight, whole, into stage 0 (one copy that arrives on the
 // barrier).
-__device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restrict__ unit_pages, int len,
+__device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restrict__ unit_pages, int lo, int hi,
                                           Split sp, int S, int s, size_t qrow0, float *__restrict__ part_o,
                                           float2 *__restrict__ part_ml, float *__restrict__ out,
                                           uint32_t *counter, uint32_t *status, bool first_issued) {
@@ -446,13 +447,15 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
                     sc[i][r] = fmaf(sc[i][r], comp, fmaf(q0_t, c0v, zt[i][r]));
                 }
             }
-            if ((pg + 1) * kT > len) {                       // partial page
+            if (pg * kT < lo || (pg + 1) * kT > hi) {       // page with tokens outside [lo, hi)
                 const int tok0 = pg * kT + 16 * gid + 8 * half;
 #pragma unroll
                 for (int i = 0; i < 4; i++)
 #pragma unroll
-                    for (int r = 0; r < 2; r++)
-                        if (tok0 + 2 * i + r >= len) sc[i][r] = -INFINITY;
+                    for (int r = 0; r < 2; r++) {
+                        const int tok = tok0 + 2 * i + r;
+                        if (tok < lo || tok >= hi) sc[i][r] = -INFINITY;
+                    }
             }
 #pragma unroll
             for (int i = 0; i < 4; i++) mx = fmaxf(mx, fmaxf(sc[i][0], sc[i][1]));
@@ -635,13 +638,35 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
                                     reinterpret_cast<float *>(sh.stage[2][0]));
 }
 
+// A CTA that handles the protected tier instead of pages: half `half_idx` of
+// the unit's slots, then the split merge.  Needs the channel choice in
+// sh.chan_pos / sh.q (a barrier after their last write).
+__device__ __forceinline__ void tier_cta(MmaShared &sh, const uint8_t *slots, int len, int n_sink, int n_recent,
+                                         int half_idx, int k, float *part_o, float2 *part_ml, size_t qrow0, int S,
+                                         int s, float *out, uint32_t *counter) {
+    int *list = reinterpret_cast<int *>(sh.stage[0][0]);                    // position -> channel
+    float *scratch = reinterpret_cast<float *>(sh.stage[0][0] + kD * sizeof(int));
+    static_assert(kD * sizeof(int) + tier_scratch_floats(4) * 4 <= 2 * (size_t)kStageBytes * 2,
+                  "tier scratch ends before the merge scratch in stages 2-3");
+    const int tid = threadIdx.x;
+    if (tid < kD) list[tid] = 0;
+    __syncthreads();
+    if (tid < kD && sh.chan_pos[tid] >= 0) list[sh.chan_pos[tid]] = tid;
+    __syncthreads();
+    const int NP = n_sink + n_recent, per = (NP + 1) / 2;
+    const int slot0 = min(NP, half_idx * per), slot1 = min(NP, slot0 + per);
+    tier_partial<4, kThreads>(slots, len, n_sink, n_recent, slot0, slot1, &sh.q[0][0], kD, 1, list, k, part_o,
+                              part_ml, qrow0, S, s, scratch);
+    merge_unit_if_last<4, kThreads>(part_o, part_ml, S, qrow0, out, counter, reinterpret_cast<float *>(sh.stage[2][0]));
+}
+
 // ---------------------------------------------------------------- decode
 __global__ void __launch_bounds__(kThreads, 2)
 decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len, int Hkv,
                   int NB, int Hq, const int32_t *__restrict__ idx, const float *__restrict__ qsel,
                   const float *__restrict__ qgsum, int k, float *__restrict__ part_o,
                   float2 *__restrict__ part_ml, int S, float *__restrict__ out,
-                  uint32_t *__restrict__ counters, uint32_t *__restrict__ status) {
+                  uint32_t *__restrict__ counters, uint32_t *__restrict__ status, int n_sink, int n_recent) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     MmaShared &sh = *reinterpret_cast<MmaShared *>(smem_raw);
 
@@ -673,8 +698,15 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
     build_plan(sh, tid, warp, lane);
 
     const int len = min(max(seq_len[b], 0), NB * kT);
-    run_pages(sh, pages + unit * NB * (size_t)page_bytes(2), len, split_of(len, S, s), S, s, qrow0, part_o,
-              part_ml, out, counters + unit, status, false);
+    const int S_pages = S - ((n_sink + n_recent > 0) ? 2 : 0);   // the last two splits take the tier
+    if (s >= S_pages) {
+        tier_cta(sh, unit_slots(const_cast<uint8_t *>(pages), gridDim.z, Hkv, NB, 2, unit, n_sink + n_recent), len,
+                 n_sink, n_recent, s - S_pages, k, part_o, part_ml, qrow0, S, s, out, counters + unit);
+        return;
+    }
+    const Tier tr = tier_of(len, n_sink, n_recent);
+    run_pages(sh, pages + unit * NB * (size_t)page_bytes(2), tr.sink_end, tr.recent_start,
+              split_of(tr.recent_start, S_pages, s), S, s, qrow0, part_o, part_ml, out, counters + unit, status, false);
 }
 
 // ---------------------------------------------------------------- fused step
@@ -692,7 +724,7 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
                 const Tin *__restrict__ v_new, int n_new, const double *__restrict__ A,
                 const double *__restrict__ Ainvt, int k, int32_t *__restrict__ idx, float *__restrict__ qsel,
                 float *__restrict__ qgsum, float *__restrict__ part_o, float2 *__restrict__ part_ml, int S,
-                float *__restrict__ out) {
+                float *__restrict__ out, int n_sink, int n_recent) {
     namespace cg = cooperative_groups;
     extern __shared__ __align__(16) uint8_t smem_raw[];
     MmaShared &sh = *reinterpret_cast<MmaShared *>(smem_raw);
@@ -738,21 +770,35 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
     const int L0 = sh.s_len;
     const bool ok = L0 >= 0 && L0 + n_new <= capacity;
     const int len = min(max(ok ? L0 + n_new : L0, 0), capacity);
-    const StepPlan plan = step_plan(len, S);
-    const Split sp = step_split(plan, s);
-    // new tokens w in [w0, w1) land in the pages of this cluster's splits
+    // with a protected tier the last cluster reads the BF16 slots instead of
+    // pages; the pages cover the coded tokens [sink_end, recent_start)
+    const int NPt = n_sink + n_recent;
+    const int S_pages = S - (NPt > 0 ? kCluster : 0);
+    const bool is_tier = s >= S_pages;
+    const Tier tr = tier_of(len, n_sink, n_recent);
+    const StepPlan plan = step_plan(tr.recent_start, S_pages);
+    const Split sp = is_tier ? Split{0, 0} : step_split(plan, s);
+    // New tokens w in [w0, w1) are transformed here: in the cluster whose
+    // splits hold their pages (it writes their codes before it stages those
+    // pages), or -- all of them -- in the tier cluster, which writes their
+    // BF16 slots and the codes of pages no split reads in this step.
     int w0 = 0, w1 = 0;
     if (ok && n_new > 0) {
-        const int s_first = s - r;
-        w0 = n_new;
-        for (int w = n_new - 1; w >= 0; w--) {
-            const int owner = owner_of(plan, (L0 + w) / kT);
-            if (owner >= s_first && owner < s_first + kCluster) {
-                w1 = max(w1, w + 1);
-                w0 = w;
+        if (is_tier) {
+            w1 = n_new;
+        } else {
+            const int s_first = s - r;
+            w0 = n_new;
+            for (int w = n_new - 1; w >= 0; w--) {
+                const int pg = (L0 + w) / kT;
+                const int owner = pg < plan.nblk ? owner_of(plan, pg) : -1;
+                if (owner >= s_first && owner < s_first + kCluster) {
+                    w1 = max(w1, w + 1);
+                    w0 = w;
+                }
             }
+            if (w1 == 0) w0 = 0;
         }
-        if (w1 == 0) w0 = 0;
     }
     const int nw = w1 - w0;
     const size_t in_base = unit * (size_t)n_new + w0;
@@ -790,7 +836,7 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
     // A cluster that appends nothing requests its pairs' first pages now,
     // whole, so their DRAM latency overlaps the channel choice (stage[p][0]
     // is clear of the scratch still in use: energies, ranks, q' copy).
-    const bool early = nw == 0;
+    const bool early = nw == 0 && !is_tier;
     if (early && (tid & 63) == 0 && sp.blk0 + (tid >> 6) < sp.blk1)
         issue_page(sh, tid >> 6, 0, unit_pages + (size_t)(sp.blk0 + (tid >> 6)) * page_bytes(2));
     if (nw > 0) {
@@ -810,6 +856,17 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
         if (w < nw) {                               // uniform over the warp
 #pragma unroll 16
             for (int c = 64; c < kD; c++) x = fma((double)px.ks[w][c], a_hi[c - 64][jj], x);
+            const int pos = L0 + w0 + w;
+            if (is_tier && stores_slot(pos, L0 + n_new, n_sink, n_recent)) {
+                uint16_t *dst = reinterpret_cast<uint16_t *>(unit_slots(pages, B, Hkv, NB, 2, unit, NPt) +
+                                                             (size_t)slot_of(pos, n_sink, n_recent) * kSlotBytes);
+                dst[j] = __bfloat16_as_ushort(__double2bfloat16(x));
+                dst[kD + j] = __bfloat16_as_ushort(__double2bfloat16((double)bx.vs[w][jj]));
+            }
+        }
+        // codes: by the cluster of the page, or by the tier cluster when no
+        // split reads the page in this step (uniform over the warp)
+        if (w < nw && (!is_tier || (L0 + w0 + w) / kT >= plan.nblk)) {
             const int g = 2 * r + (warp & 1);       // this warp's key group
             const int pos = L0 + w0 + w, tt = pos % kT;
             uint8_t *page = unit_pages + (size_t)(pos / kT) * page_bytes(2);
@@ -895,22 +952,28 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
     __syncthreads();
     build_plan(sh, tid, warp, lane);
 
-    run_pages(sh, unit_pages, len, sp, S, s, qrow0, part_o, part_ml, out,
-              status + 1 + B + unit, status, early);
+    if (is_tier)
+        tier_cta(sh, unit_slots(pages, B, Hkv, NB, 2, unit, NPt), len, n_sink, n_recent, s - S_pages, k, part_o,
+                 part_ml, qrow0, S, s, out, status + 1 + B + unit);
+    else
+        run_pages(sh, unit_pages, tr.sink_end, tr.recent_start, sp, S, s, qrow0, part_o, part_ml, out,
+                  status + 1 + B + unit, status, early);
     cluster_wait();            // the other CTA no longer reads this CTA's shared memory
 }
 
 }  // namespace
 
-// Splits per (sequence, KV head): about two CTAs per SM in all, a multiple of
-// the fused step's cluster size (at least one cluster), at most one split per
-// kPairs pages unless that is below one cluster.
-int decode_mma_splits(int units, int nblk, int num_sms) {
-    int S = (2 * num_sms) / units;
+// Splits per (sequence, KV head): about two CTAs per SM in all (counting the
+// `tier` CTAs that handle the protected tier), the page splits a multiple of
+// the fused step's cluster size (at least one cluster), at most one page
+// split per kPairs pages unless that is below one cluster.  Returns page
+// splits + tier.
+int decode_mma_splits(int units, int nblk, int num_sms, int tier) {
+    int S = (2 * num_sms) / units - tier;
     const int max_s = nblk / kPairs;
     if (S > max_s) S = max_s;
     S -= S % kCluster;
-    return S < kCluster ? kCluster : S;
+    return (S < kCluster ? kCluster : S) + tier;
 }
 
 int step_mma_max_new() { return kStepMaxNew; }
@@ -925,7 +988,8 @@ cudaError_t launch_decode_mma(const kvq_cache &c, int Hq, const int32_t *idx, co
     dim3 grid((unsigned)S, (unsigned)c.n_kv_heads, (unsigned)c.batch);
     decode_mma_kernel<<<grid, kThreads, smem, st>>>(static_cast<const uint8_t *>(c.pages), c.seq_len,
                                                     c.n_kv_heads, c.capacity / kT, Hq, idx, qsel, qgsum, k,
-                                                    part_o, part_ml, S, out, unit_counter(c, 0, 0), c.status);
+                                                    part_o, part_ml, S, out, unit_counter(c, 0, 0), c.status,
+                                                    c.n_sink, c.n_recent);
     return cudaGetLastError();
 }
 
@@ -943,7 +1007,7 @@ cudaError_t launch_step_mma(const kvq_cache &c, int Hq, const void *q, const voi
         step_mma_kernel<float><<<grid, kThreads, smem, st>>>(
             static_cast<uint8_t *>(c.pages), c.seq_len, c.status, c.n_kv_heads, c.capacity / kT, Hq,
             static_cast<const float *>(q), static_cast<const float *>(k_new), static_cast<const float *>(v_new),
-            n_new, A, Ainvt, k, idx, qsel, qgsum, part_o, part_ml, S, out);
+            n_new, A, Ainvt, k, idx, qsel, qgsum, part_o, part_ml, S, out, c.n_sink, c.n_recent);
     } else {
         static std::atomic<uint64_t> done{0};
         e = set_smem_once(step_mma_kernel<uint16_t>, (int)smem, done);
@@ -951,7 +1015,8 @@ cudaError_t launch_step_mma(const kvq_cache &c, int Hq, const void *q, const voi
         step_mma_kernel<uint16_t><<<grid, kThreads, smem, st>>>(
             static_cast<uint8_t *>(c.pages), c.seq_len, c.status, c.n_kv_heads, c.capacity / kT, Hq,
             static_cast<const uint16_t *>(q), static_cast<const uint16_t *>(k_new),
-            static_cast<const uint16_t *>(v_new), n_new, A, Ainvt, k, idx, qsel, qgsum, part_o, part_ml, S, out);
+            static_cast<const uint16_t *>(v_new), n_new, A, Ainvt, k, idx, qsel, qgsum, part_o, part_ml, S, out,
+            c.n_sink, c.n_recent);
     }
     return cudaGetLastError();
 }

@@ -50,7 +50,8 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
                    int NB, int Hq, const int32_t *__restrict__ idx, const float *__restrict__ qsel,
                    const float *__restrict__ qgsum, int k, float *__restrict__ part_o,
                    float2 *__restrict__ part_ml, int S, float *__restrict__ out,
-                   uint32_t *__restrict__ counters, uint32_t *__restrict__ status) {
+                   uint32_t *__restrict__ counters, uint32_t *__restrict__ status, int n_sink, int n_recent,
+                   int stage_area) {
     constexpr int R = row_bytes(BITS);
     constexpr int FIX = fixed_bytes(BITS);
     constexpr int PER = 8 / BITS;
@@ -63,7 +64,7 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
     const int ksel = k - 1;
     const int stage_bytes = ksel * R + FIX;
     uint8_t *stage[2] = {smem, smem + stage_bytes};
-    float *sq = reinterpret_cast<float *>(smem + 2 * stage_bytes);
+    float *sq = reinterpret_cast<float *>(smem + stage_area);     // stage_area >= 2 * stage_bytes
     float *sqg = sq + kD * G;
     int *sidx = reinterpret_cast<int *>(sqg + kNG * G);
     float *sp = reinterpret_cast<float *>(sidx + kD);
@@ -102,8 +103,24 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
 
     // a caller-owned length outside [0, capacity] is clamped, never followed
     const int len = min(max(seq_len[b], 0), NB * kT);
-    const int nblk = (len + kT - 1) / kT;
-    const int bps = (nblk + S - 1) / S;
+    // with a protected tier the last two splits read its BF16 slots; the
+    // pages cover the coded tokens [lo, hi)
+    const int NPt = n_sink + n_recent;
+    const int S_pages = S - (NPt > 0 ? 2 : 0);
+    const size_t qrow0 = (size_t)b * Hq + (size_t)h * G;
+    if (s >= S_pages) {
+        const int per = (NPt + 1) / 2;
+        const int slot0 = min(NPt, (s - S_pages) * per), slot1 = min(NPt, slot0 + per);
+        tier_partial<G, 128>(unit_slots(const_cast<uint8_t *>(pages), gridDim.z, Hkv, NB, BITS, unit, NPt), len,
+                             n_sink, n_recent, slot0, slot1, sq, 1, G, sidx, k, part_o, part_ml, qrow0, S, s,
+                             reinterpret_cast<float *>(smem));
+        merge_unit_if_last<G, 128>(part_o, part_ml, S, qrow0, out, counters + unit, reinterpret_cast<float *>(smem));
+        return;
+    }
+    const Tier tr = tier_of(len, n_sink, n_recent);
+    const int lo = tr.sink_end, hi = tr.recent_start;
+    const int nblk = (hi + kT - 1) / kT;
+    const int bps = (nblk + S_pages - 1) / S_pages;
     const int blk0 = s * bps;
     const int blk1 = min(nblk, blk0 + bps);
 
@@ -147,7 +164,7 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
         // ---- scores: thread t = token t of the page
         {
             const int t = tid;
-            const bool valid = blk * kT + t < len;
+            const bool valid = blk * kT + t >= lo && blk * kT + t < hi;
             float sc[G];
             const float c0 = __uint_as_float(((uint32_t)ch0[t]) << 16);
 #pragma unroll
@@ -179,11 +196,12 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
             for (int hl = 0; hl < G; hl++) {
                 const float bm = fmaxf(fmaxf(sred[hl], sred[G + hl]), fmaxf(sred[2 * G + hl], sred[3 * G + hl]));
                 const float mn = fmaxf(m_run[hl], bm);
-                const float alpha = exp2f(m_run[hl] - mn);   // 0 on the first page
+                const float mu = (mn == -INFINITY) ? 0.f : mn;   // a page with no valid token
+                const float alpha = exp2f(m_run[hl] - mu);       // 0 on the first page
                 m_run[hl] = mn;
                 o_acc[hl] *= alpha;
                 l_run[hl] *= alpha;
-                sp[t * G + hl] = exp2f(sc[hl] - mn);
+                sp[t * G + hl] = exp2f(sc[hl] - mu);
             }
             __syncthreads();
         }
@@ -229,8 +247,12 @@ cudaError_t launch_simt_t(const kvq_cache &c, int Hq, const int32_t *idx, const 
                           const float *qgsum, int k, float *part_o, float2 *part_ml, int S, float *out,
                           cudaStream_t st) {
     const int stage_bytes = (k - 1) * row_bytes(BITS) + fixed_bytes(BITS);
-    const size_t smem = (size_t)2 * stage_bytes + SimtSmem<G>::extra;
-    constexpr int kMaxSmem = 2 * (127 * row_bytes(BITS) + fixed_bytes(BITS)) + SimtSmem<G>::extra;
+    // the stage area doubles as the scratch of the protected-tier splits
+    constexpr int kTierBytes = (tier_scratch_floats(G) * 4 + 15) / 16 * 16;
+    const int stage_area = tier_ctas(c) ? max(2 * stage_bytes, kTierBytes) : 2 * stage_bytes;
+    const size_t smem = (size_t)stage_area + SimtSmem<G>::extra;
+    constexpr int kMaxStages = 2 * (127 * row_bytes(BITS) + fixed_bytes(BITS));
+    constexpr int kMaxSmem = (kMaxStages > kTierBytes ? kMaxStages : kTierBytes) + SimtSmem<G>::extra;
     static std::atomic<uint64_t> done{0};
     auto fn = decode_simt_kernel<BITS, G>;
     cudaError_t e = set_smem_once(fn, kMaxSmem, done);
@@ -238,7 +260,7 @@ cudaError_t launch_simt_t(const kvq_cache &c, int Hq, const int32_t *idx, const 
     dim3 grid((unsigned)S, (unsigned)c.n_kv_heads, (unsigned)c.batch);
     fn<<<grid, 128, smem, st>>>(static_cast<const uint8_t *>(c.pages), c.seq_len, c.n_kv_heads,
                                 c.capacity / kT, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out,
-                                unit_counter(c, 0, 0), c.status);
+                                unit_counter(c, 0, 0), c.status, c.n_sink, c.n_recent, stage_area);
     return cudaGetLastError();
 }
 

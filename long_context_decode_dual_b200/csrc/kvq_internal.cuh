@@ -34,6 +34,35 @@ __host__ __device__ constexpr int meta_word(int g, int t) {
 // reads in full (value codes, channel 0, key and value metadata)
 __host__ __device__ constexpr int fixed_bytes(int bits) { return page_bytes(bits) - off_vcodes(bits); }
 
+// ------------------------------------------------------------ protected tier
+// slot of the protected BF16 tier: 128 bf16 of K' then 128 bf16 of V
+constexpr int kSlotBytes = 2 * kD * 2;
+// protected set of a sequence of length len: [0, sink_end) and [recent_start, len);
+// the codes are read for [sink_end, recent_start)
+struct Tier {
+    int sink_end, recent_start;
+};
+__host__ __device__ inline Tier tier_of(int len, int n_sink, int n_recent) {
+    const int se = len < n_sink ? len : n_sink;
+    int rs = len - n_recent;
+    if (rs < se) rs = se;
+    return {se, rs};
+}
+__host__ __device__ inline int slot_of(int pos, int n_sink, int n_recent) {
+    return pos < n_sink ? pos : n_sink + pos % n_recent;
+}
+// a new token gets its slot when it is a sink token or among the last n_recent
+// of the sequence once the append completes (length len_after)
+__host__ __device__ inline bool stores_slot(int pos, int len_after, int n_sink, int n_recent) {
+    return pos < n_sink || (n_recent > 0 && pos >= len_after - n_recent);
+}
+// the unit's slots: after every page of the cache
+__host__ __device__ inline uint8_t *unit_slots(void *pages, int B, int Hkv, int NB, int bits, size_t unit, int NP) {
+    return static_cast<uint8_t *>(pages) + (size_t)B * Hkv * NB * page_bytes(bits) + unit * (size_t)NP * kSlotBytes;
+}
+// extra CTAs per (sequence, KV head) of a decode that handle the tier
+inline int tier_ctas(const kvq_cache &c) { return c.n_sink + c.n_recent > 0 ? 2 : 0; }
+
 // log2(e) / sqrt(128): scores are kept in the base-2 exponent domain
 constexpr float kScoreScaleLog2 = 0.12751743074460787f;
 
@@ -216,6 +245,117 @@ __device__ __forceinline__ void merge_unit_if_last(const float *part_o, const fl
     }
     __syncthreads();
     if (t == 0) atomicExch(counter, 0u);
+}
+
+// ------------------------------------------------------------ protected tier partial
+// The protected tier's share of one unit's softmax (Dual-QK §3.3: BF16 keys
+// and values, the same query-channel mask; §3.4: one softmax over all tiers),
+// for the unit's slots [slot0, slot1): scores of the G query heads over the
+// selected channels (1/sqrt(128), base-2 exponent domain like the codes'
+// scores), an online softmax over chunks of kTierChunk slots, value
+// aggregation, written as split s of the unit's partials (m, l, o).  Slots
+// that hold no protected position of a sequence of length len count as empty.
+// Called by every thread of an NT-thread CTA; q'[head hl] of list position i
+// is q[hl * hs + i * ps], `chan` the channel list, both in shared memory;
+// `scratch` is shared memory of tier_scratch_floats(G) floats.
+constexpr int kTierChunk = 32;
+__host__ __device__ constexpr int tier_scratch_floats(int G) {
+    return kD * (kTierChunk + 1) + kTierChunk * kD + G * kTierChunk + 4 * G;
+}
+template <int G, int NT>
+__device__ void tier_partial(const uint8_t *__restrict__ slots, int len, int n_sink, int n_recent, int slot0,
+                             int slot1, const float *q, int hs, int ps, const int *chan, int k,
+                             float *__restrict__ part_o, float2 *__restrict__ part_ml, size_t qrow0, int S, int s,
+                             float *scratch) {
+    constexpr int C = kTierChunk;
+    constexpr int OPT = G * kD / NT;                   // outputs per thread, all of one head
+    static_assert(OPT >= 1 && OPT * NT == G * kD && kD % OPT == 0, "tier: outputs must divide the threads");
+    float *kT = scratch;                               // [128][C + 1] keys, channel-major
+    float *vv = kT + kD * (C + 1);                     // [C][128] values
+    float *sc = vv + C * kD;                           // [G][C] scores, then weights
+    float *m_run = sc + G * C;                         // [G]
+    float *m_use = m_run + G;                          // [G]
+    float *alpha = m_use + G;                          // [G]
+    float *l_run = alpha + G;                          // [G]
+    const Tier tr = tier_of(len, n_sink, n_recent);
+    const int t = threadIdx.x;
+    const int oh = (t * OPT) / kD, oc = (t * OPT) % kD;
+    float o[OPT];
+#pragma unroll
+    for (int u = 0; u < OPT; u++) o[u] = 0.f;
+    if (t < G) {
+        m_run[t] = -INFINITY;
+        l_run[t] = 0.f;
+    }
+    for (int c0 = slot0; c0 < slot1; c0 += C) {
+        const int n = min(C, slot1 - c0);
+        __syncthreads();                               // the previous chunk is consumed
+        for (int e = t; e < C * (kD / 2); e += NT) {
+            const int tt = e / (kD / 2), cp = e % (kD / 2);
+            uint32_t kw = 0, vw = 0;
+            if (tt < n) {
+                const uint32_t *row = reinterpret_cast<const uint32_t *>(slots + (size_t)(c0 + tt) * kSlotBytes);
+                kw = __ldg(row + cp);
+                vw = __ldg(row + kD / 2 + cp);
+            }
+            kT[(2 * cp) * (C + 1) + tt] = __uint_as_float(kw << 16);
+            kT[(2 * cp + 1) * (C + 1) + tt] = __uint_as_float(kw & 0xffff0000u);
+            vv[tt * kD + 2 * cp] = __uint_as_float(vw << 16);
+            vv[tt * kD + 2 * cp + 1] = __uint_as_float(vw & 0xffff0000u);
+        }
+        __syncthreads();
+        for (int e = t; e < G * C; e += NT) {
+            const int hl = e / C, tt = e % C, slot = c0 + tt;
+            bool valid = false;
+            if (tt < n) {
+                if (slot < n_sink) {
+                    valid = slot < tr.sink_end;
+                } else if (n_recent > 0) {
+                    // the one position of the recent window that owns this ring slot
+                    const int j = slot - n_sink;
+                    const int p = tr.recent_start + ((j - tr.recent_start % n_recent) % n_recent + n_recent) % n_recent;
+                    valid = p < len;
+                }
+            }
+            float v = -INFINITY;
+            if (valid) {
+                float a = 0.f;
+                for (int i = 0; i < k; i++) a = fmaf(q[hl * hs + i * ps], kT[chan[i] * (C + 1) + tt], a);
+                v = a * kScoreScaleLog2;
+            }
+            sc[e] = v;
+        }
+        __syncthreads();
+        if (t < G) {
+            float m = m_run[t];
+            for (int tt = 0; tt < C; tt++) m = fmaxf(m, sc[t * C + tt]);
+            const float mu = (m == -INFINITY) ? 0.f : m;
+            alpha[t] = exp2f(m_run[t] - mu);
+            m_use[t] = mu;
+            m_run[t] = m;
+        }
+        __syncthreads();
+        for (int e = t; e < G * C; e += NT) sc[e] = exp2f(sc[e] - m_use[e / C]);
+        __syncthreads();
+        if (t < G) {
+            float ls = 0.f;
+            for (int tt = 0; tt < C; tt++) ls += sc[t * C + tt];
+            l_run[t] = fmaf(l_run[t], alpha[t], ls);
+        }
+        const float a = alpha[oh];
+#pragma unroll
+        for (int u = 0; u < OPT; u++) o[u] *= a;
+        for (int tt = 0; tt < n; tt++) {
+            const float p = sc[oh * C + tt];
+#pragma unroll
+            for (int u = 0; u < OPT; u++) o[u] = fmaf(p, vv[tt * kD + oc + u], o[u]);
+        }
+    }
+    __syncthreads();
+    const size_t row = (qrow0 + oh) * S + s;
+#pragma unroll
+    for (int u = 0; u < OPT; u++) part_o[row * kD + oc + u] = o[u];
+    if (oc == 0) part_ml[row] = make_float2(m_run[oh], l_run[oh]);
 }
 
 }  // namespace kvq

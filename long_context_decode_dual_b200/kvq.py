@@ -45,6 +45,7 @@ class CacheDesc(ctypes.Structure):
         ("batch", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
         ("group", ctypes.c_int32), ("bits", ctypes.c_int32), ("capacity", ctypes.c_int32),
         ("pages", ctypes.c_void_p), ("seq_len", ctypes.c_void_p), ("status", ctypes.c_void_p),
+        ("n_sink", ctypes.c_int32), ("n_recent", ctypes.c_int32),
     ]
 
 
@@ -136,20 +137,37 @@ class KVCache:
     pages: torch.Tensor
     seq_len: torch.Tensor
     status: torch.Tensor
+    n_sink: int = 0           # protected BF16 tier: first tokens kept
+    n_recent: int = 0         # and most recent tokens kept
 
     @property
     def desc(self) -> CacheDesc:
         return CacheDesc(self.batch, self.n_kv_heads, HEAD_DIM, GROUP, self.bits, self.capacity,
-                         self.pages.data_ptr(), self.seq_len.data_ptr(), self.status.data_ptr())
+                         self.pages.data_ptr(), self.seq_len.data_ptr(), self.status.data_ptr(),
+                         self.n_sink, self.n_recent)
 
     @property
     def n_blocks(self) -> int:
         return self.capacity // BLOCK_TOKENS
 
+    @property
+    def page_array_bytes(self) -> int:
+        return self.batch * self.n_kv_heads * self.n_blocks * page_bytes(self.bits)
+
+    def all_pages(self) -> torch.Tensor:
+        """The page array without the protected slots: uint8 [B][Hkv][blocks][page bytes]."""
+        return self.pages[:self.page_array_bytes].view(self.batch, self.n_kv_heads, self.n_blocks,
+                                                       page_bytes(self.bits))
+
     def unit_pages(self, b: int, h: int) -> torch.Tensor:
         """Pages of one (sequence, KV head): uint8 [capacity/128][page bytes]."""
-        pb = page_bytes(self.bits)
-        return self.pages.view(self.batch, self.n_kv_heads, self.n_blocks, pb)[b, h]
+        return self.all_pages()[b, h]
+
+    def slots(self) -> torch.Tensor:
+        """Protected BF16 slots: int16 bit patterns [B][Hkv][n_sink + n_recent][256]
+        (128 of the transformed key, then 128 of the value)."""
+        n = self.n_sink + self.n_recent
+        return self.pages[self.page_array_bytes:].view(torch.int16).view(self.batch, self.n_kv_heads, n, 256)
 
 
 def page_bytes(bits: int) -> int:
@@ -157,8 +175,8 @@ def page_bytes(bits: int) -> int:
 
 
 def new_cache(batch: int, n_kv_heads: int, capacity: int, bits: int = 2,
-              device="cuda", stream=None) -> KVCache:
-    desc = CacheDesc(batch, n_kv_heads, HEAD_DIM, GROUP, bits, capacity, 0, 0, 0)
+              device="cuda", stream=None, n_sink: int = 0, n_recent: int = 0) -> KVCache:
+    desc = CacheDesc(batch, n_kv_heads, HEAD_DIM, GROUP, bits, capacity, 0, 0, 0, n_sink, n_recent)
     nbytes = int(lib().kvq_cache_bytes(ctypes.byref(desc)))
     if nbytes == 0:
         raise KvqError("kvq_cache_bytes", -2)
@@ -166,7 +184,7 @@ def new_cache(batch: int, n_kv_heads: int, capacity: int, bits: int = 2,
     seq_len = torch.empty(batch, dtype=torch.int32, device=device)
     status = torch.empty(int(lib().kvq_status_words(batch, n_kv_heads)), dtype=torch.int32,
                          device=device)
-    c = KVCache(batch, n_kv_heads, capacity, bits, pages, seq_len, status)
+    c = KVCache(batch, n_kv_heads, capacity, bits, pages, seq_len, status, n_sink, n_recent)
     _check("kvq_cache_init", lib().kvq_cache_init(ctypes.byref(c.desc), _stream(stream)))
     return c
 

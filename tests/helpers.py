@@ -103,10 +103,8 @@ def rel_errors(out: np.ndarray, ref: np.ndarray):
 
 def check_pages(case: Case, cache: kvq.KVCache, units=None, n=None):
     """The cache's pages of the given units equal the oracle's, byte for byte."""
-    pages = cache.pages.cpu().numpy()
+    pages = cache.all_pages().cpu().numpy()
     wl = case.wl
-    pb = kvq.page_bytes(wl.bits)
-    pages = pages.reshape(wl.batch, wl.n_kv_heads, case.capacity // 128, pb)
     units = units or [(b, h) for b in range(wl.batch) for h in range(wl.n_kv_heads)]
     for b, h in units:
         ref = case.oracle_unit(b, h, n)
