@@ -109,9 +109,12 @@ constexpr int kOffQp = kStageBytes;                               // double[4][1
 static_assert(kOffRank + 2 * kD * (int)sizeof(int) <= kPairs * 2 * kStageBytes, "scratch fits the stages");
 static_assert(kOffQp + 4 * kD * (int)sizeof(double) <= 2 * kStageBytes, "q' copy inside stage[0][1]");
 struct PexScratch {                    // in MmaShared::pex
-    float qin[4][kD];                  // query rows (bf16 / f32 inputs are exact in f32)
-    float ks[kStepMaxNew][kD];         // new key rows
+    double qin[4][kD];                 // query rows, float64 (exact for bf16 / f32 inputs)
 };
+// new key rows: float (exact) in MmaShared::q until the channel choice, then
+// float64 in the staging memory freed by the A^{-T} block
+constexpr int kOffKs = kBlkRowBytes * 64;                         // past the high rows of A
+static_assert(kOffKs + kStepMaxNew * kD * (int)sizeof(double) <= kOffALo, "new key rows below the low rows of A");
 struct BqScratch {                     // in MmaShared::bq
     float vs[kStepMaxNew][kCols];      // new value rows, this CTA's channels
     int sel[kD];
@@ -309,15 +312,6 @@ __device__ __forceinline__ void issue_keys(MmaShared &sh, int pair, int st, cons
         const uint2 c = sh.copy[r];
         bulk_g2s(dst + c.x, src + c.x, c.y, bar);
     }
-}
-
-// A whole page into stage st of a pair in one copy (before the copy list is
-// known; at most one more 64-byte chunk per unselected pair of rows than the
-// list would fetch, and the memory system fetches those chunks anyway).
-__device__ __forceinline__ void issue_page(MmaShared &sh, int pair, int st, const uint8_t *src) {
-    const uint32_t bar = smem_u32(&sh.mbar[pair][st]);
-    mbar_arrive_expect_tx(bar, (uint32_t)kStageBytes);
-    bulk_g2s(smem_u32(sh.stage[pair][st]), src, (uint32_t)kStageBytes, bar);
 }
 
 // The page loop and the merges: pages [sp.blk0, sp.blk1) of the unit, pair
@@ -736,6 +730,8 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
     int (*rank_part)[kD] = reinterpret_cast<int (*)[kD]>(P + kOffRank);
     double (*qp)[kD] = reinterpret_cast<double (*)[kD]>(P + kOffQp);
     PexScratch &px = *reinterpret_cast<PexScratch *>(&sh.pex[0][0][0]);
+    float *ks_f = &sh.q[0][0];                                                   // [nw][128]
+    double (*ks)[kD] = reinterpret_cast<double (*)[kD]>(P + kOffKs);             // [nw][128], later
     BqScratch &bx = *reinterpret_cast<BqScratch *>(&sh.bq[0][0]);
 
     cg::cluster_group cluster = cg::this_cluster();
@@ -761,7 +757,7 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
     const double *Ai_blk = Ainvt + (size_t)h * kD * kD + r * kCols;
     const double *A_blk = A + (size_t)h * kD * kD + r * kCols;
     stage_block(aiT, Ai_blk, 0, kD);
-    for (int e = tid; e < 4 * kD; e += kThreads) px.qin[e / kD][e % kD] = in_to_float(q[qrow0 * kD + e]);
+    for (int e = tid; e < 4 * kD; e += kThreads) px.qin[e / kD][e % kD] = in_to_double(q[qrow0 * kD + e]);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     __syncthreads();
 
@@ -804,7 +800,7 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
     const size_t in_base = unit * (size_t)n_new + w0;
     if (nw > 0) {
         stage_block(a_lo, A_blk, 0, 64);
-        for (int e = tid; e < nw * kD; e += kThreads) px.ks[e / kD][e % kD] = in_to_float(k_new[in_base * kD + e]);
+        for (int e = tid; e < nw * kD; e += kThreads) ks_f[e] = in_to_float(k_new[in_base * kD + e]);
         for (int e = tid; e < nw * kCols; e += kThreads)
             bx.vs[e / kCols][e % kCols] = in_to_float(v_new[(in_base + e / kCols) * kD + r * kCols + e % kCols]);
     }
@@ -828,34 +824,29 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
         const int hl = warp >> 1, jj = (warp & 1) * 32 + lane;
         double acc = 0.0;
 #pragma unroll 16
-        for (int c = 0; c < kD; c++) acc = fma((double)px.qin[hl][c], aiT[c][jj], acc);
+        for (int c = 0; c < kD; c++) acc = fma(px.qin[hl][c], aiT[c][jj], acc);
         sh.qp_own[hl][jj] = acc;
     }
-    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");   // staging memory goes to bulk copies next
     __syncthreads();                                // A^{-T} block no longer needed
-    // A cluster that appends nothing requests its pairs' first pages now,
-    // whole, so their DRAM latency overlaps the channel choice (stage[p][0]
-    // is clear of the scratch still in use: energies, ranks, q' copy).
-    const bool early = nw == 0 && !is_tier;
-    if (early && (tid & 63) == 0 && sp.blk0 + (tid >> 6) < sp.blk1)
-        issue_page(sh, tid >> 6, 0, unit_pages + (size_t)(sp.blk0 + (tid >> 6)) * page_bytes(2));
     if (nw > 0) {
         // K'[t][j] = sum_c K[t][c] A[c][j], fma chain c = 0..127 from 0.0, for
         // token w0 + warp / 2 and channel j = 64r + jj: rows 0..63 of A while
         // rows 64..127 are staged
         stage_block(a_hi, A_blk, 64, 64);
         cp_async_commit();
+        for (int e = tid; e < nw * kD; e += kThreads) ks[e / kD][e % kD] = (double)ks_f[e];
+        __syncthreads();
         const int w = warp >> 1, jj = (warp & 1) * 32 + lane, j = r * kCols + jj;
         double x = 0.0;
         if (w < nw) {
 #pragma unroll 16
-            for (int c = 0; c < 64; c++) x = fma((double)px.ks[w][c], a_lo[c][jj], x);
+            for (int c = 0; c < 64; c++) x = fma(ks[w][c], a_lo[c][jj], x);
         }
         cp_async_wait<0>();
         __syncthreads();
         if (w < nw) {                               // uniform over the warp
 #pragma unroll 16
-            for (int c = 64; c < kD; c++) x = fma((double)px.ks[w][c], a_hi[c - 64][jj], x);
+            for (int c = 64; c < kD; c++) x = fma(ks[w][c], a_hi[c - 64][jj], x);
             const int pos = L0 + w0 + w;
             if (is_tier && stores_slot(pos, L0 + n_new, n_sink, n_recent)) {
                 uint16_t *dst = reinterpret_cast<uint16_t *>(unit_slots(pages, B, Hkv, NB, 2, unit, NPt) +
@@ -907,12 +898,15 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
 
     // ---- channel choice (the arithmetic of kvq_select_channels)
     {
+        // energies are >= 0, so their bit patterns order like their values
+        // (integer compares keep the float64 pipe free)
         const int j = tid & (kD - 1), part = tid >> 7;
-        const double e = e2[j];
+        const unsigned long long e = __double_as_longlong(e2[j]);
         int rk = 0;
         const int i0 = part == 0 ? 1 : 64, i1 = part == 0 ? 64 : kD;
+#pragma unroll 4
         for (int i = i0; i < i1; i++) {
-            const double ei = e2[i];
+            const unsigned long long ei = __double_as_longlong(e2[i]);
             rk += (ei > e) || (ei == e && i < j);
         }
         rank_part[part][j] = rk;
@@ -957,7 +951,7 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
                  part_ml, qrow0, S, s, out, status + 1 + B + unit);
     else
         run_pages(sh, unit_pages, tr.sink_end, tr.recent_start, sp, S, s, qrow0, part_o, part_ml, out,
-                  status + 1 + B + unit, status, early);
+                  status + 1 + B + unit, status, false);
     cluster_wait();            // the other CTA no longer reads this CTA's shared memory
 }
 

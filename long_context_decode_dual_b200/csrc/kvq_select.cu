@@ -83,11 +83,13 @@ select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, int H
     // rank of candidate j >= 1 among channels 1..127, counted in two halves
     {
         const int j = t & (kD - 1), part = t >> 7;
-        const double e = e2s[j];
+        // energies are >= 0, so their bit patterns order like their values
+        const unsigned long long e = __double_as_longlong(e2s[j]);
         int rk = 0;
         const int i0 = part == 0 ? 1 : 64, i1 = part == 0 ? 64 : kD;
+#pragma unroll 4
         for (int i = i0; i < i1; i++) {
-            const double ei = e2s[i];
+            const unsigned long long ei = __double_as_longlong(e2s[i]);
             rk += (ei > e) || (ei == e && i < j);
         }
         rank_part[part][j] = rk;

@@ -22,9 +22,11 @@
  *   orc_quantize_group          Dual-QK §3.3 (asymmetric INT2 grid per token,
  *                               min/max range); group of channels, fp16 scale
  *                               and zero-point, codes = clamp(rint((x-z)/s)).
- *   orc_append_unit             Dual-QK §3.3 (channel 0 of K kept in BF16 and
+ *   orc_append_unit(_g)         Dual-QK §3.3 (channel 0 of K kept in BF16 and
  *                               excluded from the range; channel-major rows,
- *                               one 32-byte row per channel of a 128-token page).
+ *                               one 32-byte row per channel of a 128-token page);
+ *                               groups of 32 channels, or of 128 -- the pages'
+ *                               one INT2 grid per token and KV head.
  *   orc_num_selected, orc_select
  *                               Dual-QK §3.2, Eq. 4 (pooled query energy
  *                               e_j^2 = sum_h q'_{h,j}^2 over the GQA group);
@@ -180,22 +182,29 @@ void orc_quantize_group(const double *x, int len, int levels,
 /* ------------------------------------------------------------------------ */
 /* page layout (one page = 128 tokens of one (batch, KV head))               */
 /*                                                                           */
-/*   rowbytes R = 128 * bits / 8                                             */
+/*   rowbytes R = 128 * bits / 8; quantization groups of `group` channels    */
+/*   (32: four groups; 128: the pages' one grid per token), ng = 128/group   */
 /*   [0, 128R)            key codes, row r = channel r (row 0 unused, zero)  */
 /*   [128R, 256R)         value codes, row r = channel r                     */
 /*   [256R, 256R+256)     channel 0 of K' as bf16, one per token             */
-/*   next 2048 bytes      key metadata: 512 words {fp16 scale, fp16 zero}      */
-/*   next 2048 bytes      value metadata, same shape                         */
+/*   next 512*ng bytes    key metadata: 128*ng words {fp16 scale, fp16 zero}  */
+/*   next 512*ng bytes    value metadata, same shape                         */
 /*   metadata word of token t, group g: 128g + 4*sw(g, t/4) + t%4 with       */
 /*   sw(g, c) = c XOR ((c/8) XOR 4*(g%2)) (chunks of 4 tokens XOR-permuted    */
 /*   within blocks of 8 chunks).                                             */
+/*   key group g covers channels max(1, g*group) .. (g+1)*group - 1 (channel */
+/*   0 is kept in bf16); value group g covers g*group .. (g+1)*group - 1.    */
 /*   codes: token t of the page sits in byte t*bits/8 of its row, at bit     */
 /*   (t mod (8/bits))*bits (least significant first).                        */
 /* ------------------------------------------------------------------------ */
-long orc_page_bytes(int bits) { return 256L * (ORC_T * bits / 8) + 256 + 2 * 2048; }
+long orc_page_bytes_g(int bits, int group)
+{
+    return 256L * (ORC_T * bits / 8) + 256 + 2L * 512 * (ORC_D / group);
+}
+long orc_page_bytes(int bits) { return orc_page_bytes_g(bits, ORC_G); }
 
-static uint8_t *page_ptr(uint8_t *unit, int bits, long page)
-{ return unit + page * orc_page_bytes(bits); }
+static uint8_t *page_ptr(uint8_t *unit, int bits, int group, long page)
+{ return unit + page * orc_page_bytes_g(bits, group); }
 
 static void put_code(uint8_t *row, int bits, int t, int code)
 {
@@ -223,67 +232,78 @@ static uint16_t get_u16(const uint8_t *p) { return (uint16_t)(p[0] | (p[1] << 8)
 
 /* Quantize n tokens (K' already transformed, V as given; both [n][128]) and
  * write them at token positions pos0 .. pos0+n-1 of one (batch, KV head)
- * unit of pages.  Other tokens' bits are left as they are.                  */
-void orc_append_unit(uint8_t *unit, int bits, long pos0, long n,
-                     const double *Kp, const double *V)
+ * unit of pages with groups of `group` channels.  Other tokens' bits are left
+ * as they are.                                                              */
+void orc_append_unit_g(uint8_t *unit, int bits, int group, long pos0, long n,
+                       const double *Kp, const double *V)
 {
     const int R = ORC_T * bits / 8;
     const int levels = (1 << bits) - 1;
-    uint8_t codes[ORC_G];
+    const int ng = ORC_D / group;
+    uint8_t codes[ORC_D];
     for (long i = 0; i < n; i++) {
         long pos = pos0 + i;
-        uint8_t *pg = page_ptr(unit, bits, pos / ORC_T);
+        uint8_t *pg = page_ptr(unit, bits, group, pos / ORC_T);
         int t = (int)(pos % ORC_T);
         const double *k = Kp + i * ORC_D;
         const double *v = V + i * ORC_D;
         uint8_t *kcodes = pg, *vcodes = pg + 128 * R;
-        uint8_t *ch0 = pg + 256 * R, *kmeta = ch0 + 256, *vmeta = kmeta + 2048;
+        uint8_t *ch0 = pg + 256 * R, *kmeta = ch0 + 256, *vmeta = kmeta + 512 * ng;
         /* channel 0 of the key: bf16, not in any range */
         put_u16(ch0 + 2 * t, orc_bf16_rne(k[0]));
-        for (int g = 0; g < ORC_NG; g++) {
+        for (int g = 0; g < ng; g++) {
             uint16_t s16, z16;
-            /* keys: group 0 covers channels 1..31, the others 32 channels */
-            int c0 = (g == 0) ? 1 : g * ORC_G;
-            int len = (g + 1) * ORC_G - c0;
+            /* keys: group 0 starts at channel 1 */
+            int c0 = (g == 0) ? 1 : g * group;
+            int len = (g + 1) * group - c0;
             orc_quantize_group(k + c0, len, levels, &s16, &z16, codes);
             for (int c = 0; c < len; c++)
                 put_code(kcodes + (long)(c0 + c) * R, bits, t, codes[c]);
             put_u16(kmeta + 4 * meta_word_index(g, t), s16);
             put_u16(kmeta + 4 * meta_word_index(g, t) + 2, z16);
-            /* values: group g covers channels 32g .. 32g+31 */
-            orc_quantize_group(v + g * ORC_G, ORC_G, levels, &s16, &z16, codes);
-            for (int c = 0; c < ORC_G; c++)
-                put_code(vcodes + (long)(g * ORC_G + c) * R, bits, t, codes[c]);
+            /* values: group g covers channels g*group .. (g+1)*group-1 */
+            orc_quantize_group(v + g * group, group, levels, &s16, &z16, codes);
+            for (int c = 0; c < group; c++)
+                put_code(vcodes + (long)(g * group + c) * R, bits, t, codes[c]);
             put_u16(vmeta + 4 * meta_word_index(g, t), s16);
             put_u16(vmeta + 4 * meta_word_index(g, t) + 2, z16);
         }
     }
 }
+void orc_append_unit(uint8_t *unit, int bits, long pos0, long n, const double *Kp, const double *V)
+{
+    orc_append_unit_g(unit, bits, ORC_G, pos0, n, Kp, V);
+}
 
 /* Dequantize tokens 0 .. n-1 of one unit: Khat[n][128], Vhat[n][128].       */
-void orc_dequant_unit(const uint8_t *unit, int bits, long n, double *Khat, double *Vhat)
+void orc_dequant_unit_g(const uint8_t *unit, int bits, int group, long n, double *Khat, double *Vhat)
 {
     const int R = ORC_T * bits / 8;
+    const int ng = ORC_D / group;
     for (long pos = 0; pos < n; pos++) {
-        const uint8_t *pg = page_ptr((uint8_t *)unit, bits, pos / ORC_T);
+        const uint8_t *pg = page_ptr((uint8_t *)unit, bits, group, pos / ORC_T);
         int t = (int)(pos % ORC_T);
         const uint8_t *kcodes = pg, *vcodes = pg + 128 * R;
-        const uint8_t *ch0 = pg + 256 * R, *kmeta = ch0 + 256, *vmeta = kmeta + 2048;
+        const uint8_t *ch0 = pg + 256 * R, *kmeta = ch0 + 256, *vmeta = kmeta + 512 * ng;
         double *kh = Khat + pos * ORC_D, *vh = Vhat + pos * ORC_D;
         kh[0] = orc_bf16_to_f64(get_u16(ch0 + 2 * t));
         for (int c = 1; c < ORC_D; c++) {
-            int g = c / ORC_G;
+            int g = c / group;
             double s = orc_f16_to_f64(get_u16(kmeta + 4 * meta_word_index(g, t)));
             double z = orc_f16_to_f64(get_u16(kmeta + 4 * meta_word_index(g, t) + 2));
             kh[c] = s * get_code(kcodes + (long)c * R, bits, t) + z;
         }
         for (int c = 0; c < ORC_D; c++) {
-            int g = c / ORC_G;
+            int g = c / group;
             double s = orc_f16_to_f64(get_u16(vmeta + 4 * meta_word_index(g, t)));
             double z = orc_f16_to_f64(get_u16(vmeta + 4 * meta_word_index(g, t) + 2));
             vh[c] = s * get_code(vcodes + (long)c * R, bits, t) + z;
         }
     }
+}
+void orc_dequant_unit(const uint8_t *unit, int bits, long n, double *Khat, double *Vhat)
+{
+    orc_dequant_unit_g(unit, bits, ORC_G, n, Khat, Vhat);
 }
 
 /* ------------------------------------------------------------------------ */

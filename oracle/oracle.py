@@ -63,6 +63,10 @@ def _load():
             lib.orc_page_bytes.argtypes = [I]
             lib.orc_append_unit.argtypes = [P, I, L, L, P, P]
             lib.orc_dequant_unit.argtypes = [P, I, L, P, P]
+            lib.orc_page_bytes_g.restype = L
+            lib.orc_page_bytes_g.argtypes = [I, I]
+            lib.orc_append_unit_g.argtypes = [P, I, I, L, L, P, P]
+            lib.orc_dequant_unit_g.argtypes = [P, I, I, L, P, P]
             lib.orc_num_selected.restype = I
             lib.orc_num_selected.argtypes = [ctypes.c_float, I]
             lib.orc_select.argtypes = [P, I, I, I, P, P]
@@ -137,31 +141,33 @@ def quantize_group(x, bits: int = 2):
     return int(s[0]), int(z[0]), c
 
 
-def page_bytes(bits: int) -> int:
-    return int(_load().orc_page_bytes(bits))
+def page_bytes(bits: int, group: int = GROUP) -> int:
+    return int(_load().orc_page_bytes_g(bits, group))
 
 
-def new_unit(capacity: int, bits: int) -> np.ndarray:
+def new_unit(capacity: int, bits: int, group: int = GROUP) -> np.ndarray:
     """Zeroed pages of one (batch, KV head): uint8 [capacity/128][page bytes]."""
     assert capacity % T == 0
-    return np.zeros((capacity // T, page_bytes(bits)), dtype=np.uint8)
+    return np.zeros((capacity // T, page_bytes(bits, group)), dtype=np.uint8)
 
 
-def append_unit(unit: np.ndarray, bits: int, pos0: int, Kp, V) -> None:
-    """Quantize and store tokens pos0.. of one unit (K' already transformed)."""
+def append_unit(unit: np.ndarray, bits: int, pos0: int, Kp, V, group: int = GROUP) -> None:
+    """Quantize and store tokens pos0.. of one unit (K' already transformed);
+    groups of `group` channels (32, or 128: one grid per token)."""
     Kp = _f64(Kp).reshape(-1, D)
     V = _f64(V).reshape(-1, D)
     assert Kp.shape == V.shape
     assert unit.flags.c_contiguous and unit.dtype == np.uint8
     assert (pos0 + Kp.shape[0]) <= unit.shape[0] * T
-    _load().orc_append_unit(_p(unit), bits, pos0, Kp.shape[0], _p(Kp), _p(V))
+    assert unit.shape[1] == page_bytes(bits, group)
+    _load().orc_append_unit_g(_p(unit), bits, group, pos0, Kp.shape[0], _p(Kp), _p(V))
 
 
-def dequant_unit(unit: np.ndarray, bits: int, n: int):
+def dequant_unit(unit: np.ndarray, bits: int, n: int, group: int = GROUP):
     """Dequantized K' and V of tokens 0..n-1: float64 [n][128] each."""
     Kh = np.zeros((max(n, 0), D))
     Vh = np.zeros((max(n, 0), D))
-    _load().orc_dequant_unit(_p(np.ascontiguousarray(unit)), bits, n, _p(Kh), _p(Vh))
+    _load().orc_dequant_unit_g(_p(np.ascontiguousarray(unit)), bits, group, n, _p(Kh), _p(Vh))
     return Kh, Vh
 
 
@@ -211,14 +217,14 @@ def attention(q, K, V) -> np.ndarray:
 
 
 # ------------------------------------------------------ whole decode step
-def decode_unit(unit: np.ndarray, bits: int, n: int, qp, sparsity: float):
+def decode_unit(unit: np.ndarray, bits: int, n: int, qp, sparsity: float, group: int = GROUP):
     """Select channels for one GQA group and attend over n cached tokens.
 
     Returns (out [g][d] float64, idx int32[k]).
     """
     k = num_selected(sparsity)
     idx, _ = select(qp, k)
-    Kh, Vh = dequant_unit(unit, bits, n)
+    Kh, Vh = dequant_unit(unit, bits, n, group)
     return decode_dense(Kh, Vh, qp, idx), idx
 
 
@@ -249,12 +255,12 @@ def protect_store(slots: np.ndarray, n_sink: int, n_recent: int, pos0: int, Kp, 
 
 
 def decode_unit_protected(unit: np.ndarray, slots: np.ndarray, bits: int, n: int, qp, sparsity: float,
-                          n_sink: int, n_recent: int):
+                          n_sink: int, n_recent: int, group: int = GROUP):
     """decode_unit with the protected tier: the first n_sink and the last
     n_recent tokens are read from their BF16 slots, the rest from the INT2
     codes; one softmax over all of them (Dual-QK §3.3, §3.4)."""
     k = num_selected(sparsity)
     idx, _ = select(qp, k)
-    Kh, Vh = dequant_unit(unit, bits, n)
+    Kh, Vh = dequant_unit(unit, bits, n, group)
     _load().orc_protect_dequant(_p(np.ascontiguousarray(slots)), n_sink, n_recent, n, _p(Kh), _p(Vh))
     return decode_dense(Kh, Vh, qp, idx), idx

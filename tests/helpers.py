@@ -74,18 +74,19 @@ class Case:
         return out, idx, qp
 
 
-def expected_qsel_qgsum(qp: np.ndarray, idx: np.ndarray):
+def expected_qsel_qgsum(qp: np.ndarray, idx: np.ndarray, group: int = 32):
     """fp32 rounding of q'[h][idx] and of the float64 ascending sum per key
     group of the kept channels other than channel 0 (the documented
-    definition of kvq_select_channels' outputs)."""
+    definition of kvq_select_channels' outputs; with one grid per token the
+    single sum is entry 0 and the other entries are 0)."""
     qsel = qp[:, idx].astype(np.float32)
     g = qp.shape[0]
     qgsum = np.zeros((g, 4), dtype=np.float32)
     for hl in range(g):
-        for gr in range(4):
+        for gr in range(128 // group):
             s = 0.0
             for c in idx:
-                if c != 0 and c // 32 == gr:
+                if c != 0 and c // group == gr:
                     s += float(qp[hl, c])
             qgsum[hl, gr] = np.float32(s)
     return qsel, qgsum

@@ -134,3 +134,62 @@ def test_append_dequant_consistent(bits):
         s, z, c = orc.quantize_group(V[t, 96:128], bits)
         np.testing.assert_array_equal(Vh[t, 96:128], orc.f16_value(s) * c + orc.f16_value(z))
         assert Kh[t, 0] == orc.bf16_value(orc.bf16_rne(np.array([K[t, 0]]))[0])
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_one_grid_per_token_layout_hand_computed(bits):
+    """The pages' own format (§3.3: one asymmetric grid per token and KV head
+    over key channels 1..127; values over channels 0..127): one metadata word
+    per token, at the permuted chunk of group 0."""
+    R = 128 * bits // 8
+    pb = orc.page_bytes(bits, 128)
+    assert pb == 256 * R + 256 + 1024
+    unit = orc.new_unit(256, bits, 128)
+    # keys: channel c (1..127) holds c % 4 -> range [0, 3] over the whole row
+    k, v = _token(0)
+    k[127] = 6.0                               # one outlier widens the single grid
+    pos = 128 + 77                             # page 1, token 77 (chunk 19 -> 19 ^ 2 = 17)
+    orc.append_unit(unit, bits, pos, k[None], v[None], group=128)
+    pg = unit[1]
+    t = 77
+    per = 8 // bits
+    levels = (1 << bits) - 1
+    kmeta = 256 * R + 256
+    vmeta = kmeta + 512
+    off = 4 * (4 * 17 + t % 4)
+    s_k = orc.f16_rne(np.array([6.0 / levels]))[0]
+    assert _u16(pg, kmeta + off) == s_k and _u16(pg, kmeta + off + 2) == 0
+    s_v = orc.f16_rne(np.array([3.0 / levels]))[0]
+    assert _u16(pg, vmeta + off) == s_v and _u16(pg, vmeta + off + 2) == 0
+    # key codes on the 6/levels grid: value x -> rint(x * levels / 6)
+    sk = orc.f16_value(s_k)
+    for c in range(1, 128):
+        byte = pg[c * R + t // per]
+        code = (byte >> ((t % per) * bits)) & levels
+        assert code == min(levels, int(np.rint(k[c] / sk))), c
+    for c in range(128):
+        byte = pg[128 * R + c * R + t // per]
+        assert (byte >> ((t % per) * bits)) & levels == (1 if bits == 2 else 5) * (3 - c % 4), c
+    assert pg[256 * R + 2 * t] == 0xC0 and pg[256 * R + 2 * t + 1] == 0x3F
+    assert not unit[0].any() and not pg[:R].any()
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_one_grid_per_token_dequant(bits):
+    rng = np.random.default_rng(9)
+    n = 260
+    K = rng.standard_normal((n, 128))
+    V = rng.standard_normal((n, 128))
+    u = orc.new_unit(384, bits, 128)
+    orc.append_unit(u, bits, 0, K, V, group=128)
+    u2 = orc.new_unit(384, bits, 128)
+    for i in range(0, n, 9):
+        orc.append_unit(u2, bits, i, K[i:i + 9], V[i:i + 9], group=128)
+    assert np.array_equal(u, u2)
+    Kh, Vh = orc.dequant_unit(u, bits, n, group=128)
+    for t in (0, 5, 128, 259):
+        s, z, c = orc.quantize_group(K[t, 1:], bits)
+        np.testing.assert_array_equal(Kh[t, 1:], orc.f16_value(s) * c + orc.f16_value(z))
+        s, z, c = orc.quantize_group(V[t], bits)
+        np.testing.assert_array_equal(Vh[t], orc.f16_value(s) * c + orc.f16_value(z))
+    np.testing.assert_array_equal(Kh[:, 0], [orc.bf16_value(int(b)) for b in orc.bf16_rne(K[:, 0])])
