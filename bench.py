@@ -108,7 +108,8 @@ def algorithmic_decode_bytes(wl: W.Workload, k: int, length: int, protect=(0, 0)
     partial outputs are ignored (< 0.1%)."""
     n_sink, n_recent = protect
     R = 128 * wl.bits // 8
-    per_page = (k - 1) * R + 128 * R + 256 + 2048 + 2048
+    meta = 4 * 128 * (128 // wl.quant_group)            # bytes of one metadata block
+    per_page = (k - 1) * R + 128 * R + 256 + 2 * meta
     sink_end = min(n_sink, length)
     recent_start = max(sink_end, length - n_recent)
     n_pages = (recent_start + 127) // 128
@@ -168,8 +169,9 @@ def oracle_sample(wl: W.Workload, n_steps: int, budget_s: float = 30.0, skip_fir
     from oracle import oracle as orc
     A, Ai = W.make_transform(wl.seed, 0)
     K, V = W.make_kv_unit(wl, 0, 0)
-    unit = orc.new_unit(wl.capacity, wl.bits)
-    orc.append_unit(unit, wl.bits, 0, orc.transform(W.as_float(K, wl.dtype), A), W.as_float(V, wl.dtype))
+    gq = wl.quant_group
+    unit = orc.new_unit(wl.capacity, wl.bits, gq)
+    orc.append_unit(unit, wl.bits, 0, orc.transform(W.as_float(K, wl.dtype), A), W.as_float(V, wl.dtype), group=gq)
     length = wl.n_ctx
     g = wl.group_size
     times, tokens = [], []
@@ -179,10 +181,10 @@ def oracle_sample(wl: W.Workload, n_steps: int, budget_s: float = 30.0, skip_fir
         q = W.make_q(wl, i)
         t0 = time.perf_counter()
         orc.append_unit(unit, wl.bits, length, orc.transform(W.as_float(kn[0, 0], wl.dtype), A),
-                        W.as_float(vn[0, 0], wl.dtype))
+                        W.as_float(vn[0, 0], wl.dtype), group=gq)
         length += 1
         qp = orc.transform(W.as_float(q[0, :g], wl.dtype), Ai)
-        orc.decode_unit(unit, wl.bits, length, qp, wl.sparsity)
+        orc.decode_unit(unit, wl.bits, length, qp, wl.sparsity, gq)
         times.append(time.perf_counter() - t0)
         tokens.append(length)
         if time.perf_counter() - t_start > budget_s and i >= 1:
@@ -201,7 +203,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     wl = W.workload(args.workload, **({"sparsity": args.sparsity} if args.sparsity is not None else {}),
-                    bits=args.bits, n_steps=args.warmup + args.steps + 1)
+                    bits=args.bits, n_steps=args.warmup + args.steps + 1, quant_group=args.group)
     from oracle import oracle as orc
     k = orc.num_selected(wl.sparsity)
     value, times, sample = oracle_sample(wl, args.warmup + args.steps, budget_s=1e9,
@@ -224,7 +226,7 @@ def run_reference(args):
 def config_dict(wl: W.Workload, k: int, protect=(0, 0)):
     d = {"workload": wl.name, "batch": wl.batch, "n_q_heads": wl.n_q_heads,
          "n_kv_heads": wl.n_kv_heads, "context": wl.n_ctx, "head_dim": 128, "bits": wl.bits,
-         "group": 32, "sparsity": wl.sparsity, "k": k,
+         "group": wl.quant_group, "sparsity": wl.sparsity, "k": k,
          "step": "append 1 token + query transform/select + decode + merge",
          "l2": "flushed between steps (256 MiB write, outside the timed events)"}
     if protect != (0, 0):
@@ -278,7 +280,7 @@ def run_ours(args):
     n_pool = 8
     total_steps = args.warmup + args.steps
     n_appends = total_steps * (2 if args.e2e else 1) + 1
-    over = {"bits": args.bits, "n_steps": n_appends}
+    over = {"bits": args.bits, "n_steps": n_appends, "quant_group": args.group}
     if args.sparsity is not None:
         over["sparsity"] = args.sparsity
     wl = rank_workload(W.workload(args.workload, **over), rank)
@@ -300,7 +302,8 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
 
     protect = (64, 256) if args.protect else (0, 0)
-    cache = kvq.new_cache(B, Hkv, wl.capacity, wl.bits, device=dev, n_sink=protect[0], n_recent=protect[1])
+    cache = kvq.new_cache(B, Hkv, wl.capacity, wl.bits, device=dev, n_sink=protect[0], n_recent=protect[1],
+                          group=wl.quant_group)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record()
     kvq.append(cache, Kd, Vd, A)
@@ -472,6 +475,8 @@ def main():
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-comparator", dest="comparator", action="store_false")
+    ap.add_argument("--group", type=int, default=32, choices=[32, 128],
+                    help="channels per quantization group (128: the pages' one grid per token)")
     ap.add_argument("--protect", action="store_true",
                     help="keep the first 64 and the last 256 tokens in BF16 (the pages' protected tier)")
     ap.add_argument("--unfused", dest="fused", action="store_false",

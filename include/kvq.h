@@ -20,8 +20,8 @@
  *    only the device can see (a sequence that would overflow its capacity)
  *    set a sticky flag in the cache's device status word and leave the data
  *    untouched; read it with kvq_read_status().
- *  - Head dimension d = 128 and quantization group = 32 channels are the
- *    supported shape; other values return KVQ_ERR_SHAPE.
+ *  - Head dimension d = 128 and quantization groups of 32 or 128 channels
+ *    are the supported shapes; other values return KVQ_ERR_SHAPE.
  *  - Tensors are dense, row-major, innermost dimension last, with the
  *    shapes given per argument.  Float inputs are either float32 or bf16
  *    (bit patterns in uint16), chosen by a KVQ_DTYPE_* argument.
@@ -29,22 +29,25 @@
  * Cache format (one "page" = 128 tokens of one (sequence, KV head))
  * ------------------------------------------------------------------
  *  rowbytes R = 128 * bits / 8   (32 for INT2, 64 for INT4)
+ *  groups per token ng = 128 / group: 4 (groups of 32 channels) or 1 (the
+ *  pages' own format, Dual-QK §3.3: one grid per token and KV head)
  *  offset 0        key codes, 128 rows x R bytes, row r = transformed key
  *                  channel r; row 0 is unused and stays zero
  *  offset 128R     value codes, 128 rows x R bytes, row r = value channel r
  *  offset 256R     channel 0 of the transformed key, 128 x bf16
- *  offset 256R+256 key metadata: 512 words {fp16 scale (low half), fp16 zero}
- *  +2048           value metadata, same shape
- *  Metadata word of token t (0..127), group g (0..3):
+ *  offset 256R+256 key metadata: 128 ng words {fp16 scale (low half), fp16 zero}
+ *  +512 ng         value metadata, same shape
+ *  Metadata word of token t (0..127), group g (0..ng-1):
  *      128 g + 4 sw(g, t / 4) + t % 4,   sw(g, c) = c XOR ((c / 8) XOR 4 (g % 2))
  *  i.e. each group's 32 chunks of 4 tokens are stored XOR-permuted within
  *  blocks of 8 chunks (a layout that lets the decode kernels read metadata
  *  without shared-memory bank conflicts after a contiguous copy).
- *  page bytes = 256R + 4352 (12544 for INT2, 20736 for INT4)
+ *  page bytes = 256R + 256 + 1024 ng (12544 / 20736 for INT2 / INT4 with
+ *  groups of 32; 9472 / 17664 with one grid per token)
  *  Code of token t (0..127) of a page: byte t*bits/8 of its row, bit
- *  (t mod (8/bits))*bits, least significant first.  Key groups are channels
- *  {1..31}, {32..63}, {64..95}, {96..127} (channel 0 is kept in bf16 and left
- *  out of the range); value groups are {0..31} ... {96..127}.
+ *  (t mod (8/bits))*bits, least significant first.  Key group g is channels
+ *  max(1, g group) .. (g+1) group - 1 (channel 0 is kept in bf16 and left out
+ *  of the range); value group g is channels g group .. (g+1) group - 1.
  *  Pages of one (sequence b, KV head h) are contiguous; unit (b, h) starts at
  *  byte ((b * n_kv_heads + h) * (capacity / 128)) * page_bytes.
  *  Dequantized value = scale * code + zero.
@@ -109,7 +112,8 @@ typedef struct {
     int32_t batch;        /* sequences B >= 1                                */
     int32_t n_kv_heads;   /* KV heads per sequence >= 1                      */
     int32_t head_dim;     /* must be 128                                     */
-    int32_t group;        /* quantization group in channels, must be 32      */
+    int32_t group;        /* quantization group in channels: 32, or 128 (one
+                             grid per token, the pages' format)              */
     int32_t bits;         /* code width: 2 (INT2) or 4 (INT4)                */
     int32_t capacity;     /* tokens per sequence, a positive multiple of 128 */
     void *pages;          /* kvq_cache_bytes() bytes, 256-byte aligned        */
@@ -131,8 +135,9 @@ typedef struct {
  * (0 if an argument is below 1). */
 size_t kvq_status_words(int batch, int n_kv_heads);
 
-/* Bytes of one 128-token page for the given code width (0 if unsupported). */
-size_t kvq_page_bytes(int bits);
+/* Bytes of one 128-token page for the given code width and group size (0 if
+ * unsupported). */
+size_t kvq_page_bytes(int bits, int group);
 
 /* Bytes of the whole page array of a cache, protected slots included (0 if
  * the descriptor is invalid). */
@@ -190,7 +195,8 @@ int kvq_num_selected(float sparsity, int head_dim);
  *  qsel    out [batch][n_q_heads][k] float32: q'[h][idx[i]] rounded to fp32
  *  qgsum   out [batch][n_q_heads][4] float32: per key group, the float64 sum
  *          of q'[h][c] over selected c != 0 of that group (ascending c),
- *          rounded to fp32 (the zero-point term of the dequantized dot)
+ *          rounded to fp32 (the zero-point term of the dequantized dot); with
+ *          one grid per token entry 0 holds the one sum and entries 1..3 are 0
  *  k_out   out (HOST int*, may be NULL): k
  *  Errors: KVQ_ERR_ARG (null, sparsity outside [0,1)), KVQ_ERR_SHAPE
  *  (n_q_heads not a multiple of n_kv_heads, or g > 32), KVQ_ERR_CUDA.

@@ -12,7 +12,8 @@ bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
 int check_cache(const kvq_cache *c) {
     if (!c || !c->pages || !c->seq_len || !c->status) return KVQ_ERR_ARG;
     if (c->batch < 1 || c->n_kv_heads < 1 || c->capacity < 1) return KVQ_ERR_ARG;
-    if (c->head_dim != kD || c->group != kGroup || (c->bits != 2 && c->bits != 4)) return KVQ_ERR_SHAPE;
+    if (c->head_dim != kD || (c->group != kGroup && c->group != kD) || (c->bits != 2 && c->bits != 4))
+        return KVQ_ERR_SHAPE;
     if (c->capacity % kT) return KVQ_ERR_SHAPE;
     if (c->n_sink < 0 || c->n_recent < 0 || c->n_sink + c->n_recent > KVQ_MAX_PROTECTED) return KVQ_ERR_ARG;
     if (!aligned(c->pages, 256) || !aligned(c->seq_len, 4) || !aligned(c->status, 4)) return KVQ_ERR_ALIGN;
@@ -64,14 +65,18 @@ size_t kvq_status_words(int batch, int n_kv_heads) {
     return 1 + (size_t)batch + (size_t)batch * n_kv_heads;
 }
 
-size_t kvq_page_bytes(int bits) { return (bits == 2 || bits == 4) ? (size_t)page_bytes(bits) : 0; }
+size_t kvq_page_bytes(int bits, int group) {
+    if ((bits != 2 && bits != 4) || (group != kGroup && group != kD)) return 0;
+    return (size_t)page_bytes(bits, kD / group);
+}
 
 size_t kvq_cache_bytes(const kvq_cache *c) {
     if (!c || c->batch < 1 || c->n_kv_heads < 1 || c->capacity < 1 || c->capacity % kT) return 0;
-    if (c->head_dim != kD || c->group != kGroup || (c->bits != 2 && c->bits != 4)) return 0;
+    if (c->head_dim != kD || (c->group != kGroup && c->group != kD) || (c->bits != 2 && c->bits != 4)) return 0;
     if (c->n_sink < 0 || c->n_recent < 0 || c->n_sink + c->n_recent > KVQ_MAX_PROTECTED) return 0;
     return (size_t)c->batch * c->n_kv_heads *
-           ((size_t)(c->capacity / kT) * kvq_page_bytes(c->bits) + (size_t)(c->n_sink + c->n_recent) * kSlotBytes);
+           ((size_t)(c->capacity / kT) * kvq_page_bytes(c->bits, c->group) +
+            (size_t)(c->n_sink + c->n_recent) * kSlotBytes);
 }
 
 int kvq_cache_init(const kvq_cache *c, kvq_stream_t stream) {

@@ -46,7 +46,7 @@ __device__ __forceinline__ void store_row(uint8_t *row_tile, const uint32_t (&co
     }
 }
 
-template <typename Tin, int BITS>
+template <typename Tin, int BITS, int NG>
 __global__ void __launch_bounds__(128)
 append_kernel(uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len,
               uint32_t *__restrict__ status, const Tin *__restrict__ K,
@@ -55,6 +55,7 @@ append_kernel(uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len,
     constexpr int R = row_bytes(BITS);
     __shared__ double ks[kTile][kD];
     __shared__ double vs[kTile][kD];
+    __shared__ double red[8];                 // block range of one grid per token (NG == 1)
 
     const int b = blockIdx.z, h = blockIdx.y;
     const int len = seq_len[b];
@@ -115,7 +116,7 @@ append_kernel(uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len,
         }
     }
 
-    uint8_t *page = pages + (((size_t)b * Hkv + h) * NB + (size_t)(first / kT)) * page_bytes(BITS);
+    uint8_t *page = pages + (((size_t)b * Hkv + h) * NB + (size_t)(first / kT)) * page_bytes(BITS, NG);
     const int t0 = first % kT;
     uint32_t valid = 0;
 #pragma unroll
@@ -124,32 +125,36 @@ append_kernel(uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len,
 
     uint16_t *ch0 = reinterpret_cast<uint16_t *>(page + off_ch0(BITS));
     uint32_t *kmeta = reinterpret_cast<uint32_t *>(page + off_kmeta(BITS));
-    uint32_t *vmeta = reinterpret_cast<uint32_t *>(page + off_vmeta(BITS));
+    uint32_t *vmeta = reinterpret_cast<uint32_t *>(page + off_vmeta(BITS, NG));
+    // groups of 32 (NG = 4): warp = group; one grid per token (NG = 1): the CTA
+    const int mg = NG == 1 ? 0 : grp;                   // metadata group of this thread
+    const bool writes_meta = NG == 1 ? j == 0 : lane == 0;
+    auto quantize = [&](double x, bool in_range, uint16_t &sb, uint16_t &zb) -> uint32_t {
+        if constexpr (NG == 1) return quantize_block128<BITS>(x, in_range, red, sb, zb);
+        else return quantize_lane<BITS>(x, in_range, sb, zb);
+    };
 
-    // keys: channel 0 -> bf16; group 0 covers channels 1..31
+    // keys: channel 0 -> bf16; group 0 starts at channel 1
     uint32_t codes[kTile];
 #pragma unroll
     for (int tt = 0; tt < kTile; tt++) {
         uint16_t sb, zb;
         codes[tt] = 0;
         if (!(valid >> tt & 1u)) continue;                        // uniform over the CTA
-        codes[tt] = quantize_lane<BITS>(acc[tt], j != 0, sb, zb);
-        if (valid >> tt & 1u) {
-            if (lane == 0) kmeta[meta_word(grp, t0 + tt)] = (uint32_t)sb | ((uint32_t)zb << 16);
-            if (j == 0) ch0[t0 + tt] = __bfloat16_as_ushort(__double2bfloat16(acc[tt]));
-        }
+        codes[tt] = quantize(acc[tt], j != 0, sb, zb);
+        if (writes_meta) kmeta[meta_word(mg, t0 + tt)] = (uint32_t)sb | ((uint32_t)zb << 16);
+        if (j == 0) ch0[t0 + tt] = __bfloat16_as_ushort(__double2bfloat16(acc[tt]));
     }
     if (j != 0) store_row<BITS>(page + (size_t)j * R + t0 * BITS / 8, codes, valid);
 
-    // values: no transform, group g covers channels 32g..32g+31
+    // values: no transform
 #pragma unroll
     for (int tt = 0; tt < kTile; tt++) {
         uint16_t sb, zb;
         codes[tt] = 0;
         if (!(valid >> tt & 1u)) continue;
-        codes[tt] = quantize_lane<BITS>(vs[tt][j], true, sb, zb);
-        if ((valid >> tt & 1u) && lane == 0)
-            vmeta[meta_word(grp, t0 + tt)] = (uint32_t)sb | ((uint32_t)zb << 16);
+        codes[tt] = quantize(vs[tt][j], true, sb, zb);
+        if (writes_meta) vmeta[meta_word(mg, t0 + tt)] = (uint32_t)sb | ((uint32_t)zb << 16);
     }
     store_row<BITS>(page + off_vcodes(BITS) + (size_t)j * R + t0 * BITS / 8, codes, valid);
 
@@ -157,7 +162,7 @@ append_kernel(uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len,
     // tokens of the sequence once this append completes
     if (n_sink + n_recent > 0) {
         uint16_t *slots = reinterpret_cast<uint16_t *>(
-            unit_slots(pages, gridDim.z, Hkv, NB, BITS, (size_t)b * Hkv + h, n_sink + n_recent));
+            unit_slots(pages, gridDim.z, Hkv, NB, BITS, (size_t)b * Hkv + h, n_sink + n_recent, NG));
 #pragma unroll
         for (int tt = 0; tt < kTile; tt++) {
             const int pos = first + tt;
@@ -276,11 +281,13 @@ __global__ void advance_kernel(int32_t *seq_len, int B, int n_new, int capacity)
     }
 }
 
-template <typename Tin, int BITS>
+template <typename Tin, int BITS, int NG>
 cudaError_t launch_append_t(const kvq_cache &c, const void *K, const void *V, int n_new,
                             const double *A, cudaStream_t st) {
     const int NB = c.capacity / kT;
-    if (n_new <= kSmallMax) {
+    // a few tokens with groups of 32: one CTA per group; otherwise (prefill,
+    // or one grid per token) the tile kernel and the length advance
+    if (NG == kNG && n_new <= kSmallMax) {
         dim3 grid((unsigned)kNG, (unsigned)c.n_kv_heads, (unsigned)c.batch);
         append_small_kernel<Tin, BITS><<<grid, 128, 0, st>>>(
             static_cast<uint8_t *>(c.pages), c.seq_len, c.status, static_cast<const Tin *>(K),
@@ -288,7 +295,7 @@ cudaError_t launch_append_t(const kvq_cache &c, const void *K, const void *V, in
         return cudaGetLastError();
     }
     dim3 grid((unsigned)((n_new + kTile - 1) / kTile + 1), (unsigned)c.n_kv_heads, (unsigned)c.batch);
-    append_kernel<Tin, BITS><<<grid, 128, 0, st>>>(
+    append_kernel<Tin, BITS, NG><<<grid, 128, 0, st>>>(
         static_cast<uint8_t *>(c.pages), c.seq_len, c.status, static_cast<const Tin *>(K),
         static_cast<const Tin *>(V), A, c.n_kv_heads, NB, n_new, c.capacity, c.n_sink, c.n_recent);
     cudaError_t e = cudaGetLastError();
@@ -301,11 +308,20 @@ cudaError_t launch_append_t(const kvq_cache &c, const void *K, const void *V, in
 
 cudaError_t launch_append(const kvq_cache &c, const void *K, const void *V, int dtype, int n_new,
                           const double *A, cudaStream_t st) {
-    if (dtype == KVQ_DTYPE_F32)
-        return c.bits == 2 ? launch_append_t<float, 2>(c, K, V, n_new, A, st)
-                           : launch_append_t<float, 4>(c, K, V, n_new, A, st);
-    return c.bits == 2 ? launch_append_t<uint16_t, 2>(c, K, V, n_new, A, st)
-                       : launch_append_t<uint16_t, 4>(c, K, V, n_new, A, st);
+    const bool one = groups_of(c) == 1;
+#define KVQ_APPEND_CASE(TIN, BITS)                                                              \
+    if (c.bits == BITS)                                                                        \
+        return one ? launch_append_t<TIN, BITS, 1>(c, K, V, n_new, A, st)                      \
+                   : launch_append_t<TIN, BITS, kNG>(c, K, V, n_new, A, st);
+    if (dtype == KVQ_DTYPE_F32) {
+        KVQ_APPEND_CASE(float, 2)
+        KVQ_APPEND_CASE(float, 4)
+    } else {
+        KVQ_APPEND_CASE(uint16_t, 2)
+        KVQ_APPEND_CASE(uint16_t, 4)
+    }
+#undef KVQ_APPEND_CASE
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace kvq

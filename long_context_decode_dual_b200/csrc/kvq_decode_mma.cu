@@ -67,9 +67,9 @@ constexpr int kThreads = 64 * kPairs;
 constexpr int kWarps = kThreads / 32;
 static_assert(kWarps == 8, "one warp per score k-step in the plan");
 constexpr int kKeyBytes = 128 * 32;               // key code rows of a page
-constexpr int kFixBytes = fixed_bytes(2);         // value codes, ch0, metadata
+constexpr int kFixBytes = fixed_bytes(2);         // value codes, ch0, metadata (groups of 32)
 constexpr int kStageBytes = kKeyBytes + kFixBytes;
-static_assert(kStageBytes == page_bytes(2), "a stage holds one page image");
+static_assert(kStageBytes == page_bytes(2) && page_bytes(2, 1) <= kStageBytes, "a stage holds one page image");
 constexpr int kChunks = kKeyBytes / 64;           // 64-byte chunks of key rows
 constexpr int kMaxCopies = kChunks / 2 + 2;       // runs after gap filling, plus the tail
 constexpr uint32_t kWaitPolls = 1u << 20;         // bound on mbarrier polls per stage
@@ -93,6 +93,7 @@ struct __align__(16) MmaShared {
     int s_len;
     double qp_own[4][kCols];           // fused step: q' of this CTA's channels (read by the cluster)
     double e2_own[kCols];              // and their pooled energies
+    double trange[kWarps][4];          // fused step, one grid per token: per-warp key / value ranges
 };
 
 // Prologue scratch of the fused step.  No page copy has been issued yet, so
@@ -244,6 +245,7 @@ __device__ __forceinline__ int owner_of(const StepPlan &p, int pg) {
 // The page plan from the channel choice (sh.chan_pos, sh.q): score-MMA B
 // fragments, and the copy list of a page.  Called by every thread after a
 // barrier that follows the last write of chan_pos / q; ends with a barrier.
+template <int NG>
 __device__ __forceinline__ void build_plan(MmaShared &sh, int tid, int warp, int lane) {
     const int gid = lane >> 2, tig = lane & 3;
     const int hh = gid >> 1, part = gid & 1;
@@ -286,7 +288,7 @@ __device__ __forceinline__ void build_plan(MmaShared &sh, int tid, int warp, int
             bytes += 64u * (uint32_t)len;
             M = (len == kChunks) ? 0ull : (M & ~(((1ull << len) - 1ull) << st));
         }
-        sh.copy[n++] = make_uint2((uint32_t)kKeyBytes, (uint32_t)kFixBytes);
+        sh.copy[n++] = make_uint2((uint32_t)kKeyBytes, (uint32_t)fixed_bytes(2, NG));
         sh.n_copies = n;
         sh.tx_keys = bytes;
     }
@@ -298,10 +300,12 @@ __device__ __forceinline__ void build_plan(MmaShared &sh, int tid, int warp, int
 // (value codes, channel 0, metadata) expects its bytes without arriving; the
 // key chunks arrive on the barrier, so the stage's phase completes once both
 // parts have landed.
+template <int NG>
 __device__ __forceinline__ void issue_tail(MmaShared &sh, int pair, int st, const uint8_t *src) {
+    constexpr uint32_t kFix = (uint32_t)fixed_bytes(2, NG);
     const uint32_t bar = smem_u32(&sh.mbar[pair][st]);
-    mbar_expect_tx(bar, (uint32_t)kFixBytes);
-    bulk_g2s(smem_u32(sh.stage[pair][st]) + kKeyBytes, src + kKeyBytes, (uint32_t)kFixBytes, bar);
+    mbar_expect_tx(bar, kFix);
+    bulk_g2s(smem_u32(sh.stage[pair][st]) + kKeyBytes, src + kKeyBytes, kFix, bar);
 }
 __device__ __forceinline__ void issue_keys(MmaShared &sh, int pair, int st, const uint8_t *src) {
     const uint32_t bar = smem_u32(&sh.mbar[pair][st]);
@@ -319,6 +323,7 @@ __device__ __forceinline__ void issue_keys(MmaShared &sh, int pair, int st, cons
 // or in the protected tier) are left out of the softmax.  `first_issued`: the pair's first page is
 // already in flight, whole, into stage 0 (one copy that arrives on the
 // barrier).
+template <int NG>
 __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restrict__ unit_pages, int lo, int hi,
                                           Split sp, int S, int s, size_t qrow0, float *__restrict__ part_o,
                                           float2 *__restrict__ part_ml, float *__restrict__ out,
@@ -330,9 +335,9 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
 
     // zero-point and channel-0 coefficients of head tig, pre-scaled to the
     // base-2 score domain
-    float qg_t[kNG];
+    float qg_t[NG];
 #pragma unroll
-    for (int g = 0; g < kNG; g++) qg_t[g] = sh.qg[tig][g] * kScoreScaleLog2;
+    for (int g = 0; g < NG; g++) qg_t[g] = sh.qg[tig][g] * kScoreScaleLog2;
     const float q0_t = sh.q[tig][0] * kScoreScaleLog2;
 
     float m_run = -INFINITY;      // running max of head tig (base-2 domain)
@@ -348,7 +353,7 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
 
     const uint32_t half_sel = half ? 0x7632u : 0x5410u;      // this warp's 16-bit half of a word
     const uint32_t vx_sel = half ? 0x4332u : 0x4110u;        // {half, high byte of half}
-    const float zmask = gid < 4 ? 1.f : 0.f;
+    const float zmask = gid < NG ? 1.f : 0.f;                // z-term rows: one per group
     uint4 *pexw = &sh.pex[warp][0][0];
 
     int it = 0;
@@ -356,8 +361,8 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
     const bool issuer = (tid & 63) == 0;
     const int first = sp.blk0 + pair;
     if (issuer && first < sp.blk1 && !first_issued) {
-        const uint8_t *src = unit_pages + (size_t)first * page_bytes(2);
-        issue_tail(sh, pair, 0, src);
+        const uint8_t *src = unit_pages + (size_t)first * page_bytes(2, NG);
+        issue_tail<NG>(sh, pair, 0, src);
         issue_keys(sh, pair, 0, src);
     }
     for (int pg = first; pg < sp.blk1; pg += kPairs, it++) {
@@ -368,15 +373,15 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
                    ? late & ~(3u << (2 * st)) : (late & ~(3u << (2 * st))) | ((2u | par) << (2 * st));
         pair_sync(pair);                                     // both warps left the other stage
         if (issuer && pg + kPairs < sp.blk1) {
-            const uint8_t *src = unit_pages + (size_t)(pg + kPairs) * page_bytes(2);
-            issue_tail(sh, pair, st ^ 1, src);
+            const uint8_t *src = unit_pages + (size_t)(pg + kPairs) * page_bytes(2, NG);
+            issue_tail<NG>(sh, pair, st ^ 1, src);
             issue_keys(sh, pair, st ^ 1, src);
         }
 
         const uint8_t *vcodes = cur + kKeyBytes;
         const uint32_t *ch0w = reinterpret_cast<const uint32_t *>(vcodes + 128 * 32);
         const uint32_t *kmeta = reinterpret_cast<const uint32_t *>(vcodes + 128 * 32 + 256);
-        const uint32_t *vmeta = kmeta + kNG * kT;
+        const uint32_t *vmeta = kmeta + NG * kT;
 
         // ---------------- scores: tokens 16gid + 8half + 2i + r, head tig
         float sc[4][2], zt[4][2];
@@ -387,11 +392,12 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
         }
         const uint8_t *kb = cur + tig * 32 + 4 * gid;
 #pragma unroll
-        for (int g = 0; g < kNG; g++) {
+        for (int g = 0; g < NG; g++) {
+            constexpr int KS = 8 / NG;                  // k-steps (16 channels each) per key group
             float C[4][4];
 #pragma unroll
-            for (int j = 0; j < 2; j++) {
-                const int ks = 2 * g + j;
+            for (int j = 0; j < KS; j++) {
+                const int ks = KS * g + j;
                 const uint8_t *sb = kb + ks * 512;
                 const uint32_t Wa = *reinterpret_cast<const uint32_t *>(sb);
                 const uint32_t Wb = *reinterpret_cast<const uint32_t *>(sb + 4 * 32);
@@ -512,7 +518,7 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
         // each group; this thread's weight column belongs to group 2pp + part
 #pragma unroll
         for (int pp = 0; pp < 2; pp++) {
-            const int gv = 2 * pp + part;
+            const int gv = NG == 1 ? 0 : 2 * pp + part;
             uint32_t bw[4][2];
             {
                 uint32_t vw[2][8];             // {s, z} of local tokens 8(2tig+u) + e, group gv
@@ -555,7 +561,7 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
         // zero-point term: rows = groups (row gid holds group gid), times p
         {
             uint32_t zw[2][8];
-            const int zg = gid & 3;
+            const int zg = NG == 1 ? 0 : (gid & 3);
 #pragma unroll
             for (int u = 0; u < 2; u++)
 #pragma unroll
@@ -591,9 +597,9 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
     l_head += __shfl_xor_sync(0xffffffffu, l_head, 4);
     l_head += __shfl_xor_sync(0xffffffffu, l_head, 8);
     l_head += __shfl_xor_sync(0xffffffffu, l_head, 16);
-    float zsum[kNG];
+    float zsum[NG];
 #pragma unroll
-    for (int g = 0; g < kNG; g++) zsum[g] = __shfl_sync(0xffffffffu, cz[0], 4 * g + tig);
+    for (int g = 0; g < NG; g++) zsum[g] = __shfl_sync(0xffffffffu, cz[0], 4 * g + tig);
     __syncthreads();                                     // stages are free now
     float *mo = reinterpret_cast<float *>(sh.stage[0][0]);       // [warp][head][128]
     float *mml = mo + kWarps * 4 * kD;                           // [warp][head][2]
@@ -601,8 +607,8 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
 #pragma unroll
     for (int mt = 0; mt < 8; mt++) {
         const int pp = mt >> 2, ca = 64 * pp + 8 * (mt & 3) + gid;
-        mo[(warp * 4 + tig) * kD + ca] = fmaf(co[mt][0], kCodeScale, zsum[2 * pp]);
-        mo[(warp * 4 + tig) * kD + ca + 32] = fmaf(co[mt][3], kCodeScale, zsum[2 * pp + 1]);
+        mo[(warp * 4 + tig) * kD + ca] = fmaf(co[mt][0], kCodeScale, zsum[NG == 1 ? 0 : 2 * pp]);
+        mo[(warp * 4 + tig) * kD + ca + 32] = fmaf(co[mt][3], kCodeScale, zsum[NG == 1 ? 0 : 2 * pp + 1]);
     }
     if (gid == 0) {
         mml[(warp * 4 + tig) * 2] = m_run;
@@ -655,6 +661,7 @@ __device__ __forceinline__ void tier_cta(MmaShared &sh, const uint8_t *slots, in
 }
 
 // ---------------------------------------------------------------- decode
+template <int NG>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len, int Hkv,
                   int NB, int Hq, const int32_t *__restrict__ idx, const float *__restrict__ qsel,
@@ -689,17 +696,17 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
     if (any_bad && tid == 0) atomicOr(status, (uint32_t)KVQ_DEV_INDEX);
     if (!any_bad && tid < k) sh.chan_pos[my_c] = tid;
     __syncthreads();
-    build_plan(sh, tid, warp, lane);
+    build_plan<NG>(sh, tid, warp, lane);
 
     const int len = min(max(seq_len[b], 0), NB * kT);
     const int S_pages = S - ((n_sink + n_recent > 0) ? 2 : 0);   // the last two splits take the tier
     if (s >= S_pages) {
-        tier_cta(sh, unit_slots(const_cast<uint8_t *>(pages), gridDim.z, Hkv, NB, 2, unit, n_sink + n_recent), len,
-                 n_sink, n_recent, s - S_pages, k, part_o, part_ml, qrow0, S, s, out, counters + unit);
+        tier_cta(sh, unit_slots(const_cast<uint8_t *>(pages), gridDim.z, Hkv, NB, 2, unit, n_sink + n_recent, NG),
+                 len, n_sink, n_recent, s - S_pages, k, part_o, part_ml, qrow0, S, s, out, counters + unit);
         return;
     }
     const Tier tr = tier_of(len, n_sink, n_recent);
-    run_pages(sh, pages + unit * NB * (size_t)page_bytes(2), tr.sink_end, tr.recent_start,
+    run_pages<NG>(sh, pages + unit * NB * (size_t)page_bytes(2, NG), tr.sink_end, tr.recent_start,
               split_of(tr.recent_start, S_pages, s), S, s, qrow0, part_o, part_ml, out, counters + unit, status, false);
 }
 
@@ -711,7 +718,7 @@ __device__ __forceinline__ void cluster_wait() {
     asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
 }
 
-template <typename Tin>
+template <typename Tin, int NG>
 __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 2)
 step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint32_t *__restrict__ status,
                 int Hkv, int NB, int Hq, const Tin *__restrict__ q, const Tin *__restrict__ k_new,
@@ -741,7 +748,7 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const size_t unit = (size_t)b * Hkv + h;
     const size_t qrow0 = (size_t)b * Hq + (size_t)h * 4;
-    uint8_t *unit_pages = pages + unit * NB * (size_t)page_bytes(2);
+    uint8_t *unit_pages = pages + unit * NB * (size_t)page_bytes(2, NG);
     const int capacity = NB * kT;
     // 64-column block of a 128 x 128 float64 matrix: 128 rows of 512 bytes
     auto stage_block = [&](double (*dst)[kCols], const double *src, int row0, int rows) {
@@ -849,26 +856,52 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
             for (int c = 64; c < kD; c++) x = fma(ks[w][c], a_hi[c - 64][jj], x);
             const int pos = L0 + w0 + w;
             if (is_tier && stores_slot(pos, L0 + n_new, n_sink, n_recent)) {
-                uint16_t *dst = reinterpret_cast<uint16_t *>(unit_slots(pages, B, Hkv, NB, 2, unit, NPt) +
+                uint16_t *dst = reinterpret_cast<uint16_t *>(unit_slots(pages, B, Hkv, NB, 2, unit, NPt, NG) +
                                                              (size_t)slot_of(pos, n_sink, n_recent) * kSlotBytes);
                 dst[j] = __bfloat16_as_ushort(__double2bfloat16(x));
                 dst[kD + j] = __bfloat16_as_ushort(__double2bfloat16((double)bx.vs[w][jj]));
             }
         }
         // codes: by the cluster of the page, or by the tier cluster when no
-        // split reads the page in this step (uniform over the warp)
+        // split reads the page in this step (uniform over the warp).  Groups
+        // of 32: warp = group; one grid per token: the range of token w is
+        // met over warps 2w, 2w+1 of both CTAs (distributed shared memory).
+        const double v = (double)bx.vs[w < nw ? w : 0][jj];
+        double klo = 0.0, khi = 0.0, vlo = 0.0, vhi = 0.0;
+        if constexpr (NG == 1) {
+            if (w < nw) {
+                const double a = warp_min(j != 0 ? x : pos_inf()), bk = warp_max(j != 0 ? x : neg_inf());
+                const double c = warp_min(v), d = warp_max(v);
+                if (lane == 0) {
+                    sh.trange[warp][0] = a;
+                    sh.trange[warp][1] = bk;
+                    sh.trange[warp][2] = c;
+                    sh.trange[warp][3] = d;
+                }
+            }
+            cluster.sync();
+            if (w < nw) {
+                const MmaShared *peer = cluster.map_shared_rank(&sh, r ^ 1);
+                const int w2 = warp & ~1;
+                klo = fmin(fmin(sh.trange[w2][0], sh.trange[w2 + 1][0]), fmin(peer->trange[w2][0], peer->trange[w2 + 1][0]));
+                khi = fmax(fmax(sh.trange[w2][1], sh.trange[w2 + 1][1]), fmax(peer->trange[w2][1], peer->trange[w2 + 1][1]));
+                vlo = fmin(fmin(sh.trange[w2][2], sh.trange[w2 + 1][2]), fmin(peer->trange[w2][2], peer->trange[w2 + 1][2]));
+                vhi = fmax(fmax(sh.trange[w2][3], sh.trange[w2 + 1][3]), fmax(peer->trange[w2][3], peer->trange[w2 + 1][3]));
+            }
+        }
         if (w < nw && (!is_tier || (L0 + w0 + w) / kT >= plan.nblk)) {
-            const int g = 2 * r + (warp & 1);       // this warp's key group
+            const int g = NG == 1 ? 0 : 2 * r + (warp & 1);                  // metadata group
+            const bool meta_writer = NG == 1 ? (r == 0 && (warp & 1) == 0 && lane == 0) : lane == 0;
             const int pos = L0 + w0 + w, tt = pos % kT;
-            uint8_t *page = unit_pages + (size_t)(pos / kT) * page_bytes(2);
+            uint8_t *page = unit_pages + (size_t)(pos / kT) * page_bytes(2, NG);
             uint16_t sb, zb;
-            const uint32_t kc = quantize_lane<2>(x, j != 0, sb, zb);
-            if (lane == 0)
+            const uint32_t kc = NG == 1 ? code_in_range<2>(x, klo, khi, sb, zb) : quantize_lane<2>(x, j != 0, sb, zb);
+            if (meta_writer)
                 reinterpret_cast<uint32_t *>(page + off_kmeta(2))[meta_word(g, tt)] = (uint32_t)sb | ((uint32_t)zb << 16);
             if (j == 0) reinterpret_cast<uint16_t *>(page + off_ch0(2))[tt] = __bfloat16_as_ushort(__double2bfloat16(x));
-            const uint32_t vc = quantize_lane<2>((double)bx.vs[w][jj], true, sb, zb);
-            if (lane == 0)
-                reinterpret_cast<uint32_t *>(page + off_vmeta(2))[meta_word(g, tt)] = (uint32_t)sb | ((uint32_t)zb << 16);
+            const uint32_t vc = NG == 1 ? code_in_range<2>(v, vlo, vhi, sb, zb) : quantize_lane<2>(v, true, sb, zb);
+            if (meta_writer)
+                reinterpret_cast<uint32_t *>(page + off_vmeta(2, NG))[meta_word(g, tt)] = (uint32_t)sb | ((uint32_t)zb << 16);
             // positions at or beyond the stored length hold zero bits, so the
             // codes are OR-ed in (the other new tokens share the words)
             const int word = tt / 16, shf = 2 * (tt % 16);
@@ -934,23 +967,26 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
     }
     if (tid < 4 * kNG) {
         // zero-point sum of key group gr (channel 0 is bf16, not in group 0),
-        // channels ascending from 0.0
+        // kept channels ascending from 0.0; one grid per token: entry 0 sums
+        // every channel, the others are 0
         const int hl = tid / kNG, gr = tid % kNG;
+        constexpr int GS = kD / NG;                 // channels per key group
         double sm = 0.0;
-        for (int c = (gr == 0 ? 1 : gr * kGroup); c < (gr + 1) * kGroup; c++)
-            if (bx.sel[c]) sm += qp[hl][c];
+        if (gr < NG)
+            for (int c = (gr == 0 ? 1 : gr * GS); c < (gr + 1) * GS; c++)
+                if (bx.sel[c]) sm += qp[hl][c];
         const float gf = (float)sm;
         sh.qg[hl][gr] = gf;
         if (s == 0) qgsum[(qrow0 + hl) * kNG + gr] = gf;
     }
     __syncthreads();
-    build_plan(sh, tid, warp, lane);
+    build_plan<NG>(sh, tid, warp, lane);
 
     if (is_tier)
-        tier_cta(sh, unit_slots(pages, B, Hkv, NB, 2, unit, NPt), len, n_sink, n_recent, s - S_pages, k, part_o,
+        tier_cta(sh, unit_slots(pages, B, Hkv, NB, 2, unit, NPt, NG), len, n_sink, n_recent, s - S_pages, k, part_o,
                  part_ml, qrow0, S, s, out, status + 1 + B + unit);
     else
-        run_pages(sh, unit_pages, tr.sink_end, tr.recent_start, sp, S, s, qrow0, part_o, part_ml, out,
+        run_pages<NG>(sh, unit_pages, tr.sink_end, tr.recent_start, sp, S, s, qrow0, part_o, part_ml, out,
                   status + 1 + B + unit, status, false);
     cluster_wait();            // the other CTA no longer reads this CTA's shared memory
 }
@@ -972,18 +1008,42 @@ int decode_mma_splits(int units, int nblk, int num_sms, int tier) {
 
 int step_mma_max_new() { return kStepMaxNew; }
 
+template <int NG>
+cudaError_t launch_decode_mma_t(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
+                                const float *qgsum, int k, float *part_o, float2 *part_ml, int S,
+                                float *out, cudaStream_t st) {
+    const size_t smem = sizeof(MmaShared);
+    static std::atomic<uint64_t> done{0};
+    cudaError_t e = set_smem_once(decode_mma_kernel<NG>, (int)smem, done);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)S, (unsigned)c.n_kv_heads, (unsigned)c.batch);
+    decode_mma_kernel<NG><<<grid, kThreads, smem, st>>>(static_cast<const uint8_t *>(c.pages), c.seq_len,
+                                                        c.n_kv_heads, c.capacity / kT, Hq, idx, qsel, qgsum, k,
+                                                        part_o, part_ml, S, out, unit_counter(c, 0, 0), c.status,
+                                                        c.n_sink, c.n_recent);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_decode_mma(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
                               const float *qgsum, int k, float *part_o, float2 *part_ml, int S,
                               float *out, cudaStream_t st) {
+    return groups_of(c) == 1 ? launch_decode_mma_t<1>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, st)
+                             : launch_decode_mma_t<kNG>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, st);
+}
+
+template <typename Tin, int NG>
+cudaError_t launch_step_mma_t(const kvq_cache &c, int Hq, const void *q, const void *k_new, const void *v_new,
+                              int n_new, const double *A, const double *Ainvt, int k, int32_t *idx, float *qsel,
+                              float *qgsum, float *part_o, float2 *part_ml, int S, float *out, cudaStream_t st) {
     const size_t smem = sizeof(MmaShared);
     static std::atomic<uint64_t> done{0};
-    cudaError_t e = set_smem_once(decode_mma_kernel, (int)smem, done);
+    cudaError_t e = set_smem_once(step_mma_kernel<Tin, NG>, (int)smem, done);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)S, (unsigned)c.n_kv_heads, (unsigned)c.batch);
-    decode_mma_kernel<<<grid, kThreads, smem, st>>>(static_cast<const uint8_t *>(c.pages), c.seq_len,
-                                                    c.n_kv_heads, c.capacity / kT, Hq, idx, qsel, qgsum, k,
-                                                    part_o, part_ml, S, out, unit_counter(c, 0, 0), c.status,
-                                                    c.n_sink, c.n_recent);
+    step_mma_kernel<Tin, NG><<<grid, kThreads, smem, st>>>(
+        static_cast<uint8_t *>(c.pages), c.seq_len, c.status, c.n_kv_heads, c.capacity / kT, Hq,
+        static_cast<const Tin *>(q), static_cast<const Tin *>(k_new), static_cast<const Tin *>(v_new), n_new, A,
+        Ainvt, k, idx, qsel, qgsum, part_o, part_ml, S, out, c.n_sink, c.n_recent);
     return cudaGetLastError();
 }
 
@@ -991,28 +1051,16 @@ cudaError_t launch_step_mma(const kvq_cache &c, int Hq, const void *q, const voi
                             int dtype, int n_new, const double *A, const double *Ainvt, int k, int32_t *idx,
                             float *qsel, float *qgsum, float *part_o, float2 *part_ml, int S, float *out,
                             cudaStream_t st) {
-    const size_t smem = sizeof(MmaShared);
-    dim3 grid((unsigned)S, (unsigned)c.n_kv_heads, (unsigned)c.batch);
-    cudaError_t e;
-    if (dtype == KVQ_DTYPE_F32) {
-        static std::atomic<uint64_t> done{0};
-        e = set_smem_once(step_mma_kernel<float>, (int)smem, done);
-        if (e != cudaSuccess) return e;
-        step_mma_kernel<float><<<grid, kThreads, smem, st>>>(
-            static_cast<uint8_t *>(c.pages), c.seq_len, c.status, c.n_kv_heads, c.capacity / kT, Hq,
-            static_cast<const float *>(q), static_cast<const float *>(k_new), static_cast<const float *>(v_new),
-            n_new, A, Ainvt, k, idx, qsel, qgsum, part_o, part_ml, S, out, c.n_sink, c.n_recent);
-    } else {
-        static std::atomic<uint64_t> done{0};
-        e = set_smem_once(step_mma_kernel<uint16_t>, (int)smem, done);
-        if (e != cudaSuccess) return e;
-        step_mma_kernel<uint16_t><<<grid, kThreads, smem, st>>>(
-            static_cast<uint8_t *>(c.pages), c.seq_len, c.status, c.n_kv_heads, c.capacity / kT, Hq,
-            static_cast<const uint16_t *>(q), static_cast<const uint16_t *>(k_new),
-            static_cast<const uint16_t *>(v_new), n_new, A, Ainvt, k, idx, qsel, qgsum, part_o, part_ml, S, out,
-            c.n_sink, c.n_recent);
-    }
-    return cudaGetLastError();
+    const bool one = groups_of(c) == 1;
+    if (dtype == KVQ_DTYPE_F32)
+        return one ? launch_step_mma_t<float, 1>(c, Hq, q, k_new, v_new, n_new, A, Ainvt, k, idx, qsel, qgsum,
+                                                 part_o, part_ml, S, out, st)
+                   : launch_step_mma_t<float, kNG>(c, Hq, q, k_new, v_new, n_new, A, Ainvt, k, idx, qsel, qgsum,
+                                                   part_o, part_ml, S, out, st);
+    return one ? launch_step_mma_t<uint16_t, 1>(c, Hq, q, k_new, v_new, n_new, A, Ainvt, k, idx, qsel, qgsum,
+                                                part_o, part_ml, S, out, st)
+               : launch_step_mma_t<uint16_t, kNG>(c, Hq, q, k_new, v_new, n_new, A, Ainvt, k, idx, qsel, qgsum,
+                                                  part_o, part_ml, S, out, st);
 }
 
 size_t decode_mma_smem_bytes() { return sizeof(MmaShared); }

@@ -44,7 +44,7 @@ __device__ __forceinline__ float warp_max_f(float v) {
 __device__ __forceinline__ float h2f_lo(uint32_t w) { return __half2float(__ushort_as_half((uint16_t)(w & 0xffffu))); }
 __device__ __forceinline__ float h2f_hi(uint32_t w) { return __half2float(__ushort_as_half((uint16_t)(w >> 16))); }
 
-template <int BITS, int G>
+template <int BITS, int G, int NG>
 __global__ void __launch_bounds__(128)
 decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len, int Hkv,
                    int NB, int Hq, const int32_t *__restrict__ idx, const float *__restrict__ qsel,
@@ -53,7 +53,8 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
                    uint32_t *__restrict__ counters, uint32_t *__restrict__ status, int n_sink, int n_recent,
                    int stage_area) {
     constexpr int R = row_bytes(BITS);
-    constexpr int FIX = fixed_bytes(BITS);
+    constexpr int FIX = fixed_bytes(BITS, NG);
+    constexpr int GS = kD / NG;                       // channels per quantization group
     constexpr int PER = 8 / BITS;
     constexpr uint32_t CMASK = (1u << BITS) - 1u;
     using SM = SimtSmem<G>;
@@ -93,11 +94,11 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
         // selected list positions 1..k-1 hold channels >= 1 ascending; group
         // gr spans positions [sgs[gr], sgs[gr+1])
         int i = 1;
-        for (int gr = 0; gr < kNG; gr++) {
+        for (int gr = 0; gr < NG; gr++) {
             sgs[gr] = i;
-            while (i < k && sidx[i] < (gr + 1) * kGroup) i++;
+            while (i < k && sidx[i] < (gr + 1) * GS) i++;
         }
-        sgs[kNG] = k;
+        sgs[NG] = k;
     }
     __syncthreads();
 
@@ -111,7 +112,7 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
     if (s >= S_pages) {
         const int per = (NPt + 1) / 2;
         const int slot0 = min(NPt, (s - S_pages) * per), slot1 = min(NPt, slot0 + per);
-        tier_partial<G, 128>(unit_slots(const_cast<uint8_t *>(pages), gridDim.z, Hkv, NB, BITS, unit, NPt), len,
+        tier_partial<G, 128>(unit_slots(const_cast<uint8_t *>(pages), gridDim.z, Hkv, NB, BITS, unit, NPt, NG), len,
                              n_sink, n_recent, slot0, slot1, sq, 1, G, sidx, k, part_o, part_ml, qrow0, S, s,
                              reinterpret_cast<float *>(smem));
         merge_unit_if_last<G, 128>(part_o, part_ml, S, qrow0, out, counters + unit, reinterpret_cast<float *>(smem));
@@ -125,7 +126,7 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
     const int blk1 = min(nblk, blk0 + bps);
 
     auto load = [&](uint8_t *dst, int blk) {
-        const uint8_t *pg = pages + (unit * NB + (size_t)blk) * page_bytes(BITS);
+        const uint8_t *pg = pages + (unit * NB + (size_t)blk) * page_bytes(BITS, NG);
         constexpr int CPR = R / 16;
         for (int e = tid; e < ksel * CPR; e += 128) {
             const int i = e / CPR, part = e % CPR;
@@ -159,7 +160,7 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
         const uint8_t *vcodes = cur + ksel * R;
         const uint16_t *ch0 = reinterpret_cast<const uint16_t *>(vcodes + 128 * R);
         const uint32_t *kmeta = reinterpret_cast<const uint32_t *>(vcodes + 128 * R + 256);
-        const uint32_t *vmeta = kmeta + kNG * kT;
+        const uint32_t *vmeta = kmeta + NG * kT;
 
         // ---- scores: thread t = token t of the page
         {
@@ -171,7 +172,7 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
             for (int hl = 0; hl < G; hl++) sc[hl] = sq[hl] * c0;
             const int boff = t / PER, sh = (t % PER) * BITS;
 #pragma unroll
-            for (int gr = 0; gr < kNG; gr++) {
+            for (int gr = 0; gr < NG; gr++) {
                 float d[G];
 #pragma unroll
                 for (int hl = 0; hl < G; hl++) d[hl] = 0.f;
@@ -208,7 +209,7 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
 
         // ---- values: thread c = value channel c
         {
-            const int c = tid, vg = c >> 5;
+            const int c = tid, vg = c / GS;
             const uint8_t *vrow = vcodes + c * R;
 #pragma unroll 1
             for (int tb = 0; tb < R; tb += 4) {
@@ -237,24 +238,28 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
         part_o[row * kD + tid] = o_acc[hl];
         if (tid == 0) part_ml[row] = make_float2(m_run[hl], l_run[hl]);
     }
-    static_assert(merge_scratch_floats(G, 128, 256) * 4 <= 2 * fixed_bytes(BITS), "merge scratch fits the stages");
     merge_unit_if_last<G, 128>(part_o, part_ml, S, (size_t)b * Hq + (size_t)h * G, out, counters + unit,
                           reinterpret_cast<float *>(smem));
 }
 
-template <int BITS, int G>
+template <int BITS, int G, int NG>
 cudaError_t launch_simt_t(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
                           const float *qgsum, int k, float *part_o, float2 *part_ml, int S, float *out,
                           cudaStream_t st) {
-    const int stage_bytes = (k - 1) * row_bytes(BITS) + fixed_bytes(BITS);
-    // the stage area doubles as the scratch of the protected-tier splits
+    const int stage_bytes = (k - 1) * row_bytes(BITS) + fixed_bytes(BITS, NG);
+    // the stage area doubles as the scratch of the protected-tier splits and
+    // of the split merge
     constexpr int kTierBytes = (tier_scratch_floats(G) * 4 + 15) / 16 * 16;
-    const int stage_area = tier_ctas(c) ? max(2 * stage_bytes, kTierBytes) : 2 * stage_bytes;
+    constexpr int kMergeBytes = (merge_scratch_floats(G, 128, 256) * 4 + 15) / 16 * 16;
+    int stage_area = max(2 * stage_bytes, kMergeBytes);
+    if (tier_ctas(c)) stage_area = max(stage_area, kTierBytes);
     const size_t smem = (size_t)stage_area + SimtSmem<G>::extra;
-    constexpr int kMaxStages = 2 * (127 * row_bytes(BITS) + fixed_bytes(BITS));
-    constexpr int kMaxSmem = (kMaxStages > kTierBytes ? kMaxStages : kTierBytes) + SimtSmem<G>::extra;
+    constexpr int kMaxStages = 2 * (127 * row_bytes(BITS) + fixed_bytes(BITS, NG));
+    constexpr int kMaxArea = kMaxStages > kTierBytes ? (kMaxStages > kMergeBytes ? kMaxStages : kMergeBytes)
+                                                     : (kTierBytes > kMergeBytes ? kTierBytes : kMergeBytes);
+    constexpr int kMaxSmem = kMaxArea + SimtSmem<G>::extra;
     static std::atomic<uint64_t> done{0};
-    auto fn = decode_simt_kernel<BITS, G>;
+    auto fn = decode_simt_kernel<BITS, G, NG>;
     cudaError_t e = set_smem_once(fn, kMaxSmem, done);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)S, (unsigned)c.n_kv_heads, (unsigned)c.batch);
@@ -291,8 +296,11 @@ cudaError_t launch_decode_simt(const kvq_cache &c, int Hq, const int32_t *idx, c
                                const float *qgsum, int k, float *part_o, float2 *part_ml, int S,
                                float *out, cudaStream_t st) {
     const int g = Hq / c.n_kv_heads;
-#define KVQ_SIMT_CASE(BITS, G) \
-    if (c.bits == BITS && g == G) return launch_simt_t<BITS, G>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, st);
+    const int ng = groups_of(c);
+#define KVQ_SIMT_CASE(BITS, G)                                                                          \
+    if (c.bits == BITS && g == G)                                                                       \
+        return ng == 1 ? launch_simt_t<BITS, G, 1>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, st) \
+                       : launch_simt_t<BITS, G, kNG>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, st);
     KVQ_SIMT_CASE(2, 1) KVQ_SIMT_CASE(2, 2) KVQ_SIMT_CASE(2, 4) KVQ_SIMT_CASE(2, 8)
     KVQ_SIMT_CASE(4, 1) KVQ_SIMT_CASE(4, 2) KVQ_SIMT_CASE(4, 4) KVQ_SIMT_CASE(4, 8)
 #undef KVQ_SIMT_CASE

@@ -18,12 +18,15 @@ constexpr int kT = 128;        // tokens per page
 constexpr int kGroup = 32;     // channels per quantization group
 constexpr int kNG = kD / kGroup;
 
+// Page layout for `bits`-wide codes and `ng` quantization groups per head
+// (4: groups of 32 channels; 1: the pages' one grid per token).
 __host__ __device__ constexpr int row_bytes(int bits) { return kT * bits / 8; }
 __host__ __device__ constexpr int off_vcodes(int bits) { return 128 * row_bytes(bits); }
 __host__ __device__ constexpr int off_ch0(int bits) { return 256 * row_bytes(bits); }
+__host__ __device__ constexpr int meta_bytes(int ng) { return 4 * kT * ng; }
 __host__ __device__ constexpr int off_kmeta(int bits) { return off_ch0(bits) + 256; }
-__host__ __device__ constexpr int off_vmeta(int bits) { return off_kmeta(bits) + 2048; }
-__host__ __device__ constexpr int page_bytes(int bits) { return off_vmeta(bits) + 2048; }
+__host__ __device__ constexpr int off_vmeta(int bits, int ng = kNG) { return off_kmeta(bits) + meta_bytes(ng); }
+__host__ __device__ constexpr int page_bytes(int bits, int ng = kNG) { return off_vmeta(bits, ng) + meta_bytes(ng); }
 // word index of the {scale, zero} pair of token t (0..127), group g (0..3)
 // inside a page's key or value metadata block (chunks of 4 tokens are stored
 // XOR-permuted within blocks of 8 chunks, see include/kvq.h)
@@ -32,7 +35,9 @@ __host__ __device__ constexpr int meta_word(int g, int t) {
 }
 // bytes from the value codes to the end of the page: what every decode step
 // reads in full (value codes, channel 0, key and value metadata)
-__host__ __device__ constexpr int fixed_bytes(int bits) { return page_bytes(bits) - off_vcodes(bits); }
+__host__ __device__ constexpr int fixed_bytes(int bits, int ng = kNG) { return page_bytes(bits, ng) - off_vcodes(bits); }
+// groups per head of a cache (group = 32 or 128 channels)
+inline int groups_of(const kvq_cache &c) { return kD / c.group; }
 
 // ------------------------------------------------------------ protected tier
 // slot of the protected BF16 tier: 128 bf16 of K' then 128 bf16 of V
@@ -57,8 +62,9 @@ __host__ __device__ inline bool stores_slot(int pos, int len_after, int n_sink, 
     return pos < n_sink || (n_recent > 0 && pos >= len_after - n_recent);
 }
 // the unit's slots: after every page of the cache
-__host__ __device__ inline uint8_t *unit_slots(void *pages, int B, int Hkv, int NB, int bits, size_t unit, int NP) {
-    return static_cast<uint8_t *>(pages) + (size_t)B * Hkv * NB * page_bytes(bits) + unit * (size_t)NP * kSlotBytes;
+__host__ __device__ inline uint8_t *unit_slots(void *pages, int B, int Hkv, int NB, int bits, size_t unit, int NP,
+                                               int ng = kNG) {
+    return static_cast<uint8_t *>(pages) + (size_t)B * Hkv * NB * page_bytes(bits, ng) + unit * (size_t)NP * kSlotBytes;
 }
 // extra CTAs per (sequence, KV head) of a decode that handle the tier
 inline int tier_ctas(const kvq_cache &c) { return c.n_sink + c.n_recent > 0 ? 2 : 0; }
@@ -91,12 +97,12 @@ __device__ __forceinline__ double warp_max(double v) {
 // Quantize value x of this lane against the group range (lanes of the warp;
 // `in_range` false leaves the lane out of min/max).  Returns the code and,
 // through s_bits / z_bits, the fp16 scale / zero-point bit patterns.
+// Code of x on the grid of a group with range [lo, hi]: zero = fp16(lo),
+// scale = fp16((hi - lo) / (2^BITS - 1)), code = clamp(rint((x - zero) / scale)).
 template <int BITS>
-__device__ __forceinline__ uint32_t quantize_lane(double x, bool in_range, uint16_t &s_bits,
+__device__ __forceinline__ uint32_t code_in_range(double x, double lo, double hi, uint16_t &s_bits,
                                                   uint16_t &z_bits) {
     constexpr int L = (1 << BITS) - 1;
-    const double lo = warp_min(in_range ? x : __longlong_as_double(0x7ff0000000000000LL));
-    const double hi = warp_max(in_range ? x : __longlong_as_double(0xfff0000000000000LL));
     const __half zh = __double2half(lo);
     const __half sh = __double2half((hi - lo) / (double)L);
     z_bits = __half_as_ushort(zh);
@@ -107,6 +113,35 @@ __device__ __forceinline__ uint32_t quantize_lane(double x, bool in_range, uint1
     double r = rint((x - z) / s);
     r = fmin(fmax(r, 0.0), (double)L);
     return (uint32_t)r;
+}
+__device__ __forceinline__ double pos_inf() { return __longlong_as_double(0x7ff0000000000000LL); }
+__device__ __forceinline__ double neg_inf() { return __longlong_as_double(0xfff0000000000000LL); }
+
+template <int BITS>
+__device__ __forceinline__ uint32_t quantize_lane(double x, bool in_range, uint16_t &s_bits,
+                                                  uint16_t &z_bits) {
+    const double lo = warp_min(in_range ? x : pos_inf());
+    const double hi = warp_max(in_range ? x : neg_inf());
+    return code_in_range<BITS>(x, lo, hi, s_bits, z_bits);
+}
+// The same over all 128 threads of a CTA (thread = channel; one grid per
+// token).  Called by every thread; `red` is shared memory of 8 doubles that
+// no other code uses between the barriers of two calls.
+template <int BITS>
+__device__ __forceinline__ uint32_t quantize_block128(double x, bool in_range, double *red, uint16_t &s_bits,
+                                                      uint16_t &z_bits) {
+    const int w = threadIdx.x >> 5;
+    const double lo_w = warp_min(in_range ? x : pos_inf());
+    const double hi_w = warp_max(in_range ? x : neg_inf());
+    __syncthreads();                                     // the previous call's reads of red are done
+    if ((threadIdx.x & 31) == 0) {
+        red[w] = lo_w;
+        red[4 + w] = hi_w;
+    }
+    __syncthreads();
+    const double lo = fmin(fmin(red[0], red[1]), fmin(red[2], red[3]));
+    const double hi = fmax(fmax(red[4], red[5]), fmax(red[6], red[7]));
+    return code_in_range<BITS>(x, lo, hi, s_bits, z_bits);
 }
 
 // ------------------------------------------------------------ cp.async

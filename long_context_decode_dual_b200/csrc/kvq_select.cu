@@ -32,7 +32,7 @@ template <typename Tin>
 __global__ void __cluster_dims__(kCtas, 1, 1) __launch_bounds__(kThreads)
 select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, int Hq, int Hkv, int g,
               int k, int32_t *__restrict__ idx, float *__restrict__ qsel,
-              float *__restrict__ qgsum) {
+              float *__restrict__ qgsum, int ng) {
     extern __shared__ __align__(16) double sm[];   // As[128][32], qin[g][128], qp[g][32]
     double *As = sm;
     double *qin = sm + kD * kGroup;
@@ -110,13 +110,29 @@ select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, int H
         idx[((size_t)b * Hkv + h) * k + pos] = t;
         for (int hl = 0; hl < g; hl++) qsel[(qrow0 + hl) * k + pos] = (float)qp[hl * kGroup + lane];
     }
-    // zero-point sum of key group r (channel 0 is bf16, not in group 0),
-    // channels ascending from 0.0
-    for (int hl = t; hl < g; hl += kThreads) {
-        double s = 0.0;
-        for (int c = (r == 0 ? 1 : 0); c < kGroup; c++)
-            if (sel_s[r * kGroup + c]) s += qp[hl * kGroup + c];
-        qgsum[(qrow0 + hl) * kNG + r] = (float)s;
+    // zero-point sum of each key group (channel 0 is bf16, not in group 0),
+    // kept channels ascending from 0.0: groups of 32 -- CTA r sums group r;
+    // one grid per token -- CTA 0 sums all channels (reading the others' q'
+    // through distributed shared memory) into entry 0, the rest are 0
+    if (ng == kNG) {
+        for (int hl = t; hl < g; hl += kThreads) {
+            double s = 0.0;
+            for (int c = (r == 0 ? 1 : 0); c < kGroup; c++)
+                if (sel_s[r * kGroup + c]) s += qp[hl * kGroup + c];
+            qgsum[(qrow0 + hl) * kNG + r] = (float)s;
+        }
+    } else if (r == 0) {
+        const double *pq[kCtas];
+#pragma unroll
+        for (int rr = 0; rr < kCtas; rr++) pq[rr] = cluster.map_shared_rank(qp, rr);
+        for (int hl = t; hl < g; hl += kThreads) {
+            double s = 0.0;
+            for (int c = 1; c < kD; c++)
+                if (sel_s[c]) s += pq[c / kGroup][hl * kGroup + c % kGroup];
+            qgsum[(qrow0 + hl) * kNG] = (float)s;
+#pragma unroll
+            for (int gr = 1; gr < kNG; gr++) qgsum[(qrow0 + hl) * kNG + gr] = 0.f;
+        }
     }
     cluster.sync();                                // keep e2own alive until all have read it
 }
@@ -135,12 +151,12 @@ cudaError_t launch_select(const kvq_cache &c, const void *q, int dtype, int Hq, 
         e = set_smem_once(select_kernel<float>, kMaxSmem, done_f32);
         if (e != cudaSuccess) return e;
         select_kernel<float><<<grid, kThreads, smem, st>>>(static_cast<const float *>(q), Ainvt, Hq,
-                                                           c.n_kv_heads, g, k, idx, qsel, qgsum);
+                                                           c.n_kv_heads, g, k, idx, qsel, qgsum, groups_of(c));
     } else {
         e = set_smem_once(select_kernel<uint16_t>, kMaxSmem, done_bf16);
         if (e != cudaSuccess) return e;
         select_kernel<uint16_t><<<grid, kThreads, smem, st>>>(static_cast<const uint16_t *>(q), Ainvt, Hq,
-                                                              c.n_kv_heads, g, k, idx, qsel, qgsum);
+                                                              c.n_kv_heads, g, k, idx, qsel, qgsum, groups_of(c));
     }
     return cudaGetLastError();
 }

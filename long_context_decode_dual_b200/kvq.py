@@ -72,7 +72,7 @@ def lib() -> ctypes.CDLL:
         C = ctypes.POINTER(CacheDesc)
         sig = {
             "kvq_status_words": (S, [I, I]),
-            "kvq_page_bytes": (S, [I]),
+            "kvq_page_bytes": (S, [I, I]),
             "kvq_cache_bytes": (S, [C]),
             "kvq_cache_init": (I, [C, P]),
             "kvq_append": (I, [C, P, P, I, I, P, P]),
@@ -139,10 +139,11 @@ class KVCache:
     status: torch.Tensor
     n_sink: int = 0           # protected BF16 tier: first tokens kept
     n_recent: int = 0         # and most recent tokens kept
+    group: int = GROUP        # channels per quantization group: 32, or 128 (one grid per token)
 
     @property
     def desc(self) -> CacheDesc:
-        return CacheDesc(self.batch, self.n_kv_heads, HEAD_DIM, GROUP, self.bits, self.capacity,
+        return CacheDesc(self.batch, self.n_kv_heads, HEAD_DIM, self.group, self.bits, self.capacity,
                          self.pages.data_ptr(), self.seq_len.data_ptr(), self.status.data_ptr(),
                          self.n_sink, self.n_recent)
 
@@ -152,12 +153,12 @@ class KVCache:
 
     @property
     def page_array_bytes(self) -> int:
-        return self.batch * self.n_kv_heads * self.n_blocks * page_bytes(self.bits)
+        return self.batch * self.n_kv_heads * self.n_blocks * page_bytes(self.bits, self.group)
 
     def all_pages(self) -> torch.Tensor:
         """The page array without the protected slots: uint8 [B][Hkv][blocks][page bytes]."""
         return self.pages[:self.page_array_bytes].view(self.batch, self.n_kv_heads, self.n_blocks,
-                                                       page_bytes(self.bits))
+                                                       page_bytes(self.bits, self.group))
 
     def unit_pages(self, b: int, h: int) -> torch.Tensor:
         """Pages of one (sequence, KV head): uint8 [capacity/128][page bytes]."""
@@ -170,13 +171,13 @@ class KVCache:
         return self.pages[self.page_array_bytes:].view(torch.int16).view(self.batch, self.n_kv_heads, n, 256)
 
 
-def page_bytes(bits: int) -> int:
-    return int(lib().kvq_page_bytes(bits))
+def page_bytes(bits: int, group: int = GROUP) -> int:
+    return int(lib().kvq_page_bytes(bits, group))
 
 
 def new_cache(batch: int, n_kv_heads: int, capacity: int, bits: int = 2,
-              device="cuda", stream=None, n_sink: int = 0, n_recent: int = 0) -> KVCache:
-    desc = CacheDesc(batch, n_kv_heads, HEAD_DIM, GROUP, bits, capacity, 0, 0, 0, n_sink, n_recent)
+              device="cuda", stream=None, n_sink: int = 0, n_recent: int = 0, group: int = GROUP) -> KVCache:
+    desc = CacheDesc(batch, n_kv_heads, HEAD_DIM, group, bits, capacity, 0, 0, 0, n_sink, n_recent)
     nbytes = int(lib().kvq_cache_bytes(ctypes.byref(desc)))
     if nbytes == 0:
         raise KvqError("kvq_cache_bytes", -2)
@@ -184,7 +185,7 @@ def new_cache(batch: int, n_kv_heads: int, capacity: int, bits: int = 2,
     seq_len = torch.empty(batch, dtype=torch.int32, device=device)
     status = torch.empty(int(lib().kvq_status_words(batch, n_kv_heads)), dtype=torch.int32,
                          device=device)
-    c = KVCache(batch, n_kv_heads, capacity, bits, pages, seq_len, status, n_sink, n_recent)
+    c = KVCache(batch, n_kv_heads, capacity, bits, pages, seq_len, status, n_sink, n_recent, group)
     _check("kvq_cache_init", lib().kvq_cache_init(ctypes.byref(c.desc), _stream(stream)))
     return c
 

@@ -57,6 +57,7 @@ class Workload:
     outlier_scale: float
     sparsity: float
     bits: int = 2
+    quant_group: int = 32   # channels per quantization group: 32, or 128 (one grid per token)
     per_head_transform: bool = True
     n_steps: int = 0
     seed: int = 0

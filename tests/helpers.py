@@ -34,7 +34,7 @@ class Case:
     # ---------------------------------------------------------------- GPU
     def gpu_cache(self, chunks=None) -> kvq.KVCache:
         wl = self.wl
-        cache = kvq.new_cache(wl.batch, wl.n_kv_heads, self.capacity, wl.bits)
+        cache = kvq.new_cache(wl.batch, wl.n_kv_heads, self.capacity, wl.bits, group=wl.quant_group)
         A = dev64(self.A)
         n = self.K.shape[2]
         chunks = chunks or [n]
@@ -57,8 +57,8 @@ class Case:
             n = self.K.shape[2] if n is None else n
             Kf = W.as_float(self.K[b, h, :n], wl.dtype)
             Vf = W.as_float(self.V[b, h, :n], wl.dtype)
-            u = orc.new_unit(self.capacity, wl.bits)
-            orc.append_unit(u, wl.bits, 0, orc.transform(Kf, self.A[h]), Vf)
+            u = orc.new_unit(self.capacity, wl.bits, wl.quant_group)
+            orc.append_unit(u, wl.bits, 0, orc.transform(Kf, self.A[h]), Vf, group=wl.quant_group)
             self._oracle_units[key] = u
         return self._oracle_units[key]
 
@@ -70,7 +70,7 @@ class Case:
     def oracle_decode(self, q: np.ndarray, b: int, h: int, sparsity: float, n: int | None = None):
         n = self.K.shape[2] if n is None else n
         qp = self.oracle_qp(q, b, h)
-        out, idx = orc.decode_unit(self.oracle_unit(b, h), self.wl.bits, n, qp, sparsity)
+        out, idx = orc.decode_unit(self.oracle_unit(b, h), self.wl.bits, n, qp, sparsity, self.wl.quant_group)
         return out, idx, qp
 
 

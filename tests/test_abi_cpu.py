@@ -31,7 +31,8 @@ def test_every_declared_symbol_is_exported():
 def test_host_side_queries():
     L = kvq.lib()
     assert L.kvq_version() == 100
-    assert L.kvq_page_bytes(2) == 12544 and L.kvq_page_bytes(4) == 20736 and L.kvq_page_bytes(3) == 0
+    assert L.kvq_page_bytes(2, 32) == 12544 and L.kvq_page_bytes(4, 32) == 20736 and L.kvq_page_bytes(3, 32) == 0
+    assert L.kvq_page_bytes(2, 128) == 9472 and L.kvq_page_bytes(4, 128) == 17664 and L.kvq_page_bytes(2, 64) == 0
     for s, k in ((0.0, 128), (0.2, 103), (0.4, 77), (0.6, 52), (0.25, 96)):
         assert kvq.num_selected(s) == k
     assert kvq.num_selected(1.0) == -1 and kvq.num_selected(-0.1) == -1
@@ -39,6 +40,12 @@ def test_host_side_queries():
     assert L.kvq_cache_bytes(ctypes.byref(d)) == 2 * 8 * 2 * 12544
     bad = kvq.CacheDesc(2, 8, 64, 32, 2, 256, 0, 0, 0)
     assert L.kvq_cache_bytes(ctypes.byref(bad)) == 0
+    one = kvq.CacheDesc(2, 8, 128, 128, 2, 256, 0, 0, 0)            # one grid per token
+    assert L.kvq_cache_bytes(ctypes.byref(one)) == 2 * 8 * 2 * 9472
+    tier = kvq.CacheDesc(2, 8, 128, 128, 2, 256, 0, 0, 0, 64, 256)  # plus the BF16 slots
+    assert L.kvq_cache_bytes(ctypes.byref(tier)) == 2 * 8 * (2 * 9472 + 320 * 512)
+    assert L.kvq_cache_bytes(ctypes.byref(kvq.CacheDesc(2, 8, 128, 64, 2, 256, 0, 0, 0))) == 0
+    assert L.kvq_cache_bytes(ctypes.byref(kvq.CacheDesc(2, 8, 128, 32, 2, 256, 0, 0, 0, 1000, 25))) == 0
     assert kvq.status_string(-3) == "capacity exceeded"
 
 

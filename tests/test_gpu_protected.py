@@ -38,7 +38,8 @@ def _run(case: Case, n0: int, n_new: int, n_steps: int, n_sink: int, n_recent: i
     wl = case.wl
     g = wl.group_size
     A, Ai = dev64(case.A), dev64(case.Ai)
-    cache = kvq.new_cache(wl.batch, wl.n_kv_heads, case.capacity, wl.bits, n_sink=n_sink, n_recent=n_recent)
+    cache = kvq.new_cache(wl.batch, wl.n_kv_heads, case.capacity, wl.bits, n_sink=n_sink, n_recent=n_recent,
+                          group=wl.quant_group)
     if n0:
         kvq.append(cache, to_dev(case.K[:, :, :n0], wl.dtype), to_dev(case.V[:, :, :n0], wl.dtype), A)
     pos = n0
@@ -61,7 +62,8 @@ def _run(case: Case, n0: int, n_new: int, n_steps: int, n_sink: int, n_recent: i
             unit = case.oracle_unit(b, h, pos)
             slots = _oracle_slots(case, b, h, pos, n_sink, n_recent)
             qp = case.oracle_qp(q, b, h)
-            want, ref_idx = orc.decode_unit_protected(unit, slots, wl.bits, pos, qp, sparsity, n_sink, n_recent)
+            want, ref_idx = orc.decode_unit_protected(unit, slots, wl.bits, pos, qp, sparsity, n_sink, n_recent,
+                                                      wl.quant_group)
             assert np.array_equal(sel.idx[b, h].cpu().numpy(), ref_idx)
             emax, emean = rel_errors(out[b, h * g:(h + 1) * g], want)
             assert emax <= TOL_MAX and emean <= TOL_MEAN, (i, b, h, emax, emean)
