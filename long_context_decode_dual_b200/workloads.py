@@ -22,6 +22,14 @@ Recipe (every array comes from its own numpy PCG64 stream keyed by
   factor in the original (untransformed) space.
 * queries: N(0,1).
 * bf16 inputs are the round-to-nearest-even bf16 of float32 draws.
+* diagonal refinement (optional): ``delta_0 = 1``, ``delta_j = exp(N(0, 0.3^2))``
+  for j >= 1, the free scales divided by their geometric mean (the pages fit
+  D offline, keep its channel-0 entry at one and normalise the free scales to
+  unit geometric mean).  It is folded into the transforms as the pages do:
+  key transform ``A D^{-1}``, query transform ``A^{-T} D``.
+* value rotation (optional): ``Rv = Q H / sqrt(128)``, ``Q`` a seeded Haar
+  orthogonal matrix standing in for the calibrated rotation and ``H`` the
+  Sylvester Hadamard matrix of order 128; ``Rv`` is orthogonal.
 """
 from __future__ import annotations
 
@@ -35,7 +43,7 @@ HEAD_DIM = 128
 BLOCK_TOKENS = 128
 
 # stream ids, one per drawn tensor kind
-_S_A_U, _S_A_W, _S_A_G, _S_OUTLIER, _S_K, _S_V, _S_Q, _S_KNEW, _S_VNEW = range(9)
+_S_A_U, _S_A_W, _S_A_G, _S_OUTLIER, _S_K, _S_V, _S_Q, _S_KNEW, _S_VNEW, _S_DELTA, _S_RV = range(11)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -61,6 +69,9 @@ class Workload:
     per_head_transform: bool = True
     n_steps: int = 0
     seed: int = 0
+    refine: bool = False    # diagonal refinement D folded into the transforms
+    rotate_values: bool = False
+    v_clip: float = 1.0     # value clipping ratio (the pages use 0.92 with rotated values)
 
     @property
     def group_size(self) -> int:
@@ -161,14 +172,59 @@ def make_transform(seed: int, head: int, d: int = HEAD_DIM, sigma: float = 0.3):
     return np.ascontiguousarray(A), np.ascontiguousarray(Ainvt)
 
 
+def make_refinement(seed: int, head: int, d: int = HEAD_DIM, sigma: float = 0.3) -> np.ndarray:
+    """Positive diagonal scales delta [d], delta[0] = 1, free scales with unit
+    geometric mean."""
+    g = _rng(seed, _S_DELTA, head).normal(0.0, sigma, size=d - 1)
+    g -= g.mean()
+    return np.concatenate([[1.0], np.exp(g)])
+
+
+def sylvester_hadamard(n: int) -> np.ndarray:
+    """Hadamard matrix of order n (a power of two), entries +-1."""
+    H = np.ones((1, 1))
+    while H.shape[0] < n:
+        H = np.block([[H, H], [H, -H]])
+    assert H.shape[0] == n
+    return H
+
+
+def make_value_rotation(seed: int, head: int, d: int = HEAD_DIM) -> np.ndarray:
+    """Orthogonal value rotation Q H / sqrt(d), float64 [d][d]."""
+    Q = _haar_q(_rng(seed, _S_RV, head), d)
+    return np.ascontiguousarray(Q @ (sylvester_hadamard(d) / math.sqrt(d)))
+
+
 def make_transforms(wl: Workload):
-    """A and A^{-T} for every KV head: float64 [Hkv][d][d] each."""
+    """A and A^{-T} for every KV head: float64 [Hkv][d][d] each (with the
+    workload's diagonal refinement folded in, when it has one)."""
     As, Ais = [], []
     for h in range(wl.n_kv_heads):
-        A, Ai = make_transform(wl.seed, h if wl.per_head_transform else 0)
+        hh = h if wl.per_head_transform else 0
+        A, Ai = make_transform(wl.seed, hh)
+        if wl.refine:
+            delta = make_refinement(wl.seed, hh)
+            A = A / delta[None, :]
+            Ai = Ai * delta[None, :]
         As.append(A)
         Ais.append(Ai)
     return np.ascontiguousarray(np.stack(As)), np.ascontiguousarray(np.stack(Ais))
+
+
+def make_deltas(wl: Workload) -> Optional[np.ndarray]:
+    """The diagonal refinement of every KV head, float64 [Hkv][d], or None."""
+    if not wl.refine:
+        return None
+    return np.ascontiguousarray(np.stack([make_refinement(wl.seed, h if wl.per_head_transform else 0)
+                                          for h in range(wl.n_kv_heads)]))
+
+
+def make_value_rotations(wl: Workload) -> Optional[np.ndarray]:
+    """The value rotation of every KV head, float64 [Hkv][d][d], or None."""
+    if not wl.rotate_values:
+        return None
+    return np.ascontiguousarray(np.stack([make_value_rotation(wl.seed, h if wl.per_head_transform else 0)
+                                          for h in range(wl.n_kv_heads)]))
 
 
 # ---------------------------------------------------------- keys and values

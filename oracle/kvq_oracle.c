@@ -27,10 +27,21 @@
  *                               one 32-byte row per channel of a 128-token page);
  *                               groups of 32 channels, or of 128 -- the pages'
  *                               one INT2 grid per token and KV head.
+ *   orc_quantize_group_clip     the same grid over [clip*min, clip*max]:
+ *                               Dual-QK App. B.2 (values: per-token asymmetric
+ *                               INT2 with a clipping ratio of 0.92; keys are
+ *                               not clipped); orc_append_unit_c clips values.
  *   orc_num_selected, orc_select
  *                               Dual-QK §3.2, Eq. 4 (pooled query energy
  *                               e_j^2 = sum_h q'_{h,j}^2 over the GQA group);
  *                               channel 0 always kept; ties to the lower index.
+ *   orc_select_scaled           §3.3 diagonal refinement and App. C.2: with
+ *                               A = A0 D, selection uses the base queries
+ *                               q A0 = (q A) D^{-1}, scores the final ones.
+ *   value rotation              §3.3 / App. B.2: values are multiplied by an
+ *                               orthogonal rotation before quantization
+ *                               (orc_transform) and the aggregated output by
+ *                               its transpose (orc_transform with R^T).
  *   orc_dequant_unit            inverse of the quantizer: x = s*code + z.
  *   orc_decode_dense            Dual-QK §3.2 (retained channels, original
  *                               1/sqrt(d) normalisation) and §3.4 (one softmax
@@ -154,14 +165,19 @@ void orc_transform(const double *X, const double *M, long n, int d, double *Y)
 /* ------------------------------------------------------------------------ */
 /* levels = 2^bits - 1.  Writes the fp16 bit patterns of scale and zero and
  * one code per value.                                                       */
-void orc_quantize_group(const double *x, int len, int levels,
-                        uint16_t *s16, uint16_t *z16, uint8_t *codes)
+/* With a clipping ratio `clip` (0 < clip <= 1) the grid spans
+ * [clip*min, clip*max] instead of [min, max]; values outside it take the end
+ * codes.  clip = 1 is the plain min/max grid (the products are exact).       */
+void orc_quantize_group_clip(const double *x, int len, int levels, double clip,
+                             uint16_t *s16, uint16_t *z16, uint8_t *codes)
 {
     double lo = x[0], hi = x[0];
     for (int i = 1; i < len; i++) {
         if (x[i] < lo) lo = x[i];
         if (x[i] > hi) hi = x[i];
     }
+    lo = clip * lo;
+    hi = clip * hi;
     uint16_t zb = orc_f16_rne(lo);
     uint16_t sb = orc_f16_rne((hi - lo) / (double)levels);
     double z = orc_f16_to_f64(zb), s = orc_f16_to_f64(sb);
@@ -177,6 +193,11 @@ void orc_quantize_group(const double *x, int len, int levels,
     }
     *s16 = sb;
     *z16 = zb;
+}
+void orc_quantize_group(const double *x, int len, int levels,
+                        uint16_t *s16, uint16_t *z16, uint8_t *codes)
+{
+    orc_quantize_group_clip(x, len, levels, 1.0, s16, z16, codes);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -230,11 +251,12 @@ static int meta_word_index(int g, int t)
 static void put_u16(uint8_t *p, uint16_t v) { p[0] = (uint8_t)(v & 0xFF); p[1] = (uint8_t)(v >> 8); }
 static uint16_t get_u16(const uint8_t *p) { return (uint16_t)(p[0] | (p[1] << 8)); }
 
-/* Quantize n tokens (K' already transformed, V as given; both [n][128]) and
- * write them at token positions pos0 .. pos0+n-1 of one (batch, KV head)
- * unit of pages with groups of `group` channels.  Other tokens' bits are left
- * as they are.                                                              */
-void orc_append_unit_g(uint8_t *unit, int bits, int group, long pos0, long n,
+/* Quantize n tokens (K' already transformed, V as given -- rotated or not;
+ * both [n][128]) and write them at token positions pos0 .. pos0+n-1 of one
+ * (batch, KV head) unit of pages with groups of `group` channels; the value
+ * grids use the clipping ratio vclip, the key grids none.  Other tokens' bits
+ * are left as they are.                                                     */
+void orc_append_unit_c(uint8_t *unit, int bits, int group, double vclip, long pos0, long n,
                        const double *Kp, const double *V)
 {
     const int R = ORC_T * bits / 8;
@@ -262,13 +284,18 @@ void orc_append_unit_g(uint8_t *unit, int bits, int group, long pos0, long n,
             put_u16(kmeta + 4 * meta_word_index(g, t), s16);
             put_u16(kmeta + 4 * meta_word_index(g, t) + 2, z16);
             /* values: group g covers channels g*group .. (g+1)*group-1 */
-            orc_quantize_group(v + g * group, group, levels, &s16, &z16, codes);
+            orc_quantize_group_clip(v + g * group, group, levels, vclip, &s16, &z16, codes);
             for (int c = 0; c < group; c++)
                 put_code(vcodes + (long)(g * group + c) * R, bits, t, codes[c]);
             put_u16(vmeta + 4 * meta_word_index(g, t), s16);
             put_u16(vmeta + 4 * meta_word_index(g, t) + 2, z16);
         }
     }
+}
+void orc_append_unit_g(uint8_t *unit, int bits, int group, long pos0, long n,
+                       const double *Kp, const double *V)
+{
+    orc_append_unit_c(unit, bits, group, 1.0, pos0, n, Kp, V);
 }
 void orc_append_unit(uint8_t *unit, int bits, long pos0, long n, const double *Kp, const double *V)
 {
@@ -334,13 +361,20 @@ static int cmp_int_asc(const void *a, const void *b)
  * e2 (out, [d]): pooled energy, sum over h ascending as an fma chain.
  * idx (out, [k]): channel 0, then the k-1 channels of 1..d-1 with the
  * largest e2 (ties to the lower index), all sorted ascending.              */
-void orc_select(const double *qp, int g, int d, int k, double *e2, int32_t *idx)
+/* With a diagonal refinement (delta != NULL: delta[j] > 0), qp holds the
+ * final queries q A0 D and the energies are those of the base queries
+ * q A0 = qp D^{-1}: u = qp[h][j] / delta[j] (one rounded division), e2[j] the
+ * fma chain of u*u over h.  delta == NULL: u = qp[h][j].                    */
+void orc_select_scaled(const double *qp, int g, int d, int k, const double *delta,
+                       double *e2, int32_t *idx)
 {
     int *order = (int *)malloc(sizeof(int) * d);
     for (int j = 0; j < d; j++) {
         double e = 0.0;
-        for (int h = 0; h < g; h++)
-            e = fma(qp[h * d + j], qp[h * d + j], e);
+        for (int h = 0; h < g; h++) {
+            double u = delta ? qp[h * d + j] / delta[j] : qp[h * d + j];
+            e = fma(u, u, e);
+        }
         e2[j] = e;
     }
     for (int j = 1; j < d; j++) order[j - 1] = j;
@@ -353,6 +387,10 @@ void orc_select(const double *qp, int g, int d, int k, double *e2, int32_t *idx)
     for (int i = 0; i < k; i++) idx[i] = sel[i];
     free(sel);
     free(order);
+}
+void orc_select(const double *qp, int g, int d, int k, double *e2, int32_t *idx)
+{
+    orc_select_scaled(qp, g, d, k, NULL, e2, idx);
 }
 
 /* ------------------------------------------------------------------------ */

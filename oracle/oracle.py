@@ -59,6 +59,7 @@ def _load():
             lib.orc_bf16_rne_array.argtypes = [P, L, P]
             lib.orc_transform.argtypes = [P, P, L, I, P]
             lib.orc_quantize_group.argtypes = [P, I, I, P, P, P]
+            lib.orc_quantize_group_clip.argtypes = [P, I, I, ctypes.c_double, P, P, P]
             lib.orc_page_bytes.restype = L
             lib.orc_page_bytes.argtypes = [I]
             lib.orc_append_unit.argtypes = [P, I, L, L, P, P]
@@ -66,10 +67,12 @@ def _load():
             lib.orc_page_bytes_g.restype = L
             lib.orc_page_bytes_g.argtypes = [I, I]
             lib.orc_append_unit_g.argtypes = [P, I, I, L, L, P, P]
+            lib.orc_append_unit_c.argtypes = [P, I, I, ctypes.c_double, L, L, P, P]
             lib.orc_dequant_unit_g.argtypes = [P, I, I, L, P, P]
             lib.orc_num_selected.restype = I
             lib.orc_num_selected.argtypes = [ctypes.c_float, I]
             lib.orc_select.argtypes = [P, I, I, I, P, P]
+            lib.orc_select_scaled.argtypes = [P, I, I, I, P, P, P]
             lib.orc_decode_dense.argtypes = [P, P, L, P, I, I, P, I, P]
             lib.orc_attention.argtypes = [P, P, P, L, I, I, P]
             lib.orc_protected_slot.restype = L
@@ -128,8 +131,10 @@ def transform(X, M) -> np.ndarray:
 
 
 # --------------------------------------------------------------- quantizer
-def quantize_group(x, bits: int = 2):
-    """One (token, group) of the asymmetric min/max quantizer (Dual-QK §3.3).
+def quantize_group(x, bits: int = 2, clip: float = 1.0):
+    """One (token, group) of the asymmetric min/max quantizer (Dual-QK §3.3);
+    with clip < 1 the grid spans [clip*min, clip*max] (App. B.2: values use a
+    clipping ratio of 0.92).
 
     Returns (scale fp16 bits, zero fp16 bits, codes uint8[len]).
     """
@@ -137,7 +142,7 @@ def quantize_group(x, bits: int = 2):
     s = np.zeros(1, np.uint16)
     z = np.zeros(1, np.uint16)
     c = np.zeros(x.size, np.uint8)
-    _load().orc_quantize_group(_p(x), x.size, (1 << bits) - 1, _p(s), _p(z), _p(c))
+    _load().orc_quantize_group_clip(_p(x), x.size, (1 << bits) - 1, float(clip), _p(s), _p(z), _p(c))
     return int(s[0]), int(z[0]), c
 
 
@@ -151,16 +156,17 @@ def new_unit(capacity: int, bits: int, group: int = GROUP) -> np.ndarray:
     return np.zeros((capacity // T, page_bytes(bits, group)), dtype=np.uint8)
 
 
-def append_unit(unit: np.ndarray, bits: int, pos0: int, Kp, V, group: int = GROUP) -> None:
-    """Quantize and store tokens pos0.. of one unit (K' already transformed);
-    groups of `group` channels (32, or 128: one grid per token)."""
+def append_unit(unit: np.ndarray, bits: int, pos0: int, Kp, V, group: int = GROUP, vclip: float = 1.0) -> None:
+    """Quantize and store tokens pos0.. of one unit (K' already transformed, V
+    already rotated where the values are rotated); groups of `group` channels
+    (32, or 128: one grid per token); value grids clipped by vclip."""
     Kp = _f64(Kp).reshape(-1, D)
     V = _f64(V).reshape(-1, D)
     assert Kp.shape == V.shape
     assert unit.flags.c_contiguous and unit.dtype == np.uint8
     assert (pos0 + Kp.shape[0]) <= unit.shape[0] * T
     assert unit.shape[1] == page_bytes(bits, group)
-    _load().orc_append_unit_g(_p(unit), bits, group, pos0, Kp.shape[0], _p(Kp), _p(V))
+    _load().orc_append_unit_c(_p(unit), bits, group, float(vclip), pos0, Kp.shape[0], _p(Kp), _p(V))
 
 
 def dequant_unit(unit: np.ndarray, bits: int, n: int, group: int = GROUP):
@@ -176,10 +182,12 @@ def num_selected(sparsity: float, d: int = D) -> int:
     return int(_load().orc_num_selected(float(sparsity), d))
 
 
-def select(qp, k: int):
+def select(qp, k: int, delta=None):
     """Channel 0 plus the top k-1 channels by pooled energy (Dual-QK Eq. 4).
 
-    qp: [g][d] transformed queries of one GQA group. Returns (idx int32[k]
+    qp: [g][d] transformed queries of one GQA group.  delta: the diagonal
+    refinement D folded into the query transform (§3.3), or None; selection
+    then uses the base queries qp / delta (App. C.2).  Returns (idx int32[k]
     ascending, e2 float64[d]).
     """
     qp = _f64(qp)
@@ -187,7 +195,12 @@ def select(qp, k: int):
     assert 1 <= k <= d
     e2 = np.zeros(d)
     idx = np.zeros(k, np.int32)
-    _load().orc_select(_p(qp), g, d, k, _p(e2), _p(idx))
+    if delta is None:
+        _load().orc_select(_p(qp), g, d, k, _p(e2), _p(idx))
+    else:
+        delta = _f64(delta)
+        assert delta.shape == (d,) and np.all(delta > 0)
+        _load().orc_select_scaled(_p(qp), g, d, k, _p(delta), _p(e2), _p(idx))
     return idx, e2
 
 
@@ -216,16 +229,33 @@ def attention(q, K, V) -> np.ndarray:
     return out
 
 
+# ----------------------------------------------------------- value rotation
+def value_rotate(V, Rv) -> np.ndarray:
+    """Values in the rotated basis, V Rv (Dual-QK §3.3, App. B.2: the value
+    rotation precedes quantization); the fma chain of ``transform``."""
+    return transform(V, Rv)
+
+
+def value_unrotate(o, Rv) -> np.ndarray:
+    """Aggregated output back in the original basis, o Rv^T (§3.3: the value
+    rotation is reversed after aggregation; Rv is orthogonal)."""
+    return transform(o, np.ascontiguousarray(_f64(Rv).T))
+
+
 # ------------------------------------------------------ whole decode step
-def decode_unit(unit: np.ndarray, bits: int, n: int, qp, sparsity: float, group: int = GROUP):
-    """Select channels for one GQA group and attend over n cached tokens.
+def decode_unit(unit: np.ndarray, bits: int, n: int, qp, sparsity: float, group: int = GROUP,
+                delta=None, Rv=None):
+    """Select channels for one GQA group and attend over n cached tokens;
+    with delta, selection on the base queries; with Rv, the output is rotated
+    back (the cache then holds rotated values).
 
     Returns (out [g][d] float64, idx int32[k]).
     """
     k = num_selected(sparsity)
-    idx, _ = select(qp, k)
+    idx, _ = select(qp, k, delta)
     Kh, Vh = dequant_unit(unit, bits, n, group)
-    return decode_dense(Kh, Vh, qp, idx), idx
+    out = decode_dense(Kh, Vh, qp, idx)
+    return (out if Rv is None else value_unrotate(out, Rv)), idx
 
 
 # ------------------------------------------------------ protected BF16 tier
@@ -255,12 +285,14 @@ def protect_store(slots: np.ndarray, n_sink: int, n_recent: int, pos0: int, Kp, 
 
 
 def decode_unit_protected(unit: np.ndarray, slots: np.ndarray, bits: int, n: int, qp, sparsity: float,
-                          n_sink: int, n_recent: int, group: int = GROUP):
+                          n_sink: int, n_recent: int, group: int = GROUP, delta=None, Rv=None):
     """decode_unit with the protected tier: the first n_sink and the last
     n_recent tokens are read from their BF16 slots, the rest from the INT2
-    codes; one softmax over all of them (Dual-QK §3.3, §3.4)."""
+    codes; one softmax over all of them, then (with Rv) the inverse value
+    rotation (Dual-QK §3.3, §3.4)."""
     k = num_selected(sparsity)
-    idx, _ = select(qp, k)
+    idx, _ = select(qp, k, delta)
     Kh, Vh = dequant_unit(unit, bits, n, group)
     _load().orc_protect_dequant(_p(np.ascontiguousarray(slots)), n_sink, n_recent, n, _p(Kh), _p(Vh))
-    return decode_dense(Kh, Vh, qp, idx), idx
+    out = decode_dense(Kh, Vh, qp, idx)
+    return (out if Rv is None else value_unrotate(out, Rv)), idx
