@@ -126,6 +126,15 @@ typedef struct {
     int32_t n_sink;       /* protected BF16 tier: first tokens kept, >= 0     */
     int32_t n_recent;     /* and most recent tokens kept, >= 0; together at
                              most KVQ_MAX_PROTECTED (0 and 0: no tier)       */
+    const double *v_rot;  /* value rotation (Dual-QK §3.3, App. B.2), or NULL
+                             for none: [n_kv_heads][128][128] float64,
+                             row-major, 16-byte aligned, orthogonal, device
+                             memory.  Appends store V Rv (coded and in the
+                             protected slots); decodes aggregate in that basis
+                             and return out = o Rv^T                        */
+    double v_clip;        /* clipping ratio of the value grids, in (0, 1]
+                             (the pages use 0.92 with rotated values); 0 means
+                             1, no clipping.  Keys are never clipped.        */
 } kvq_cache;
 
 /* Largest n_sink + n_recent. */
@@ -153,7 +162,8 @@ int kvq_cache_init(const kvq_cache *cache, kvq_stream_t stream);
  * Dual-QK §3.1 (keys multiplied by the fixed transform, K' = K A), §3.3
  * (channel 0 of K' kept as bf16 and excluded from the range; the other key
  * channels and all value channels quantized per token with an asymmetric
- * min/max grid, round to nearest; channel-major 128-token pages).
+ * min/max grid, round to nearest; channel-major 128-token pages), App. B.2
+ * (values rotated by cache->v_rot and their grids clipped by cache->v_clip).
  *
  *  K, V    [batch][n_kv_heads][n_new][128], dtype KVQ_DTYPE_F32 or _BF16
  *  A       [n_kv_heads][128][128] float64, row-major, 16-byte aligned:
@@ -163,7 +173,10 @@ int kvq_cache_init(const kvq_cache *cache, kvq_stream_t stream);
  *  zero = fp16(min), scale = fp16((max-min)/(2^bits-1)) (fp16 rounding to
  *  nearest even from float64), code = clamp(rint((x - zero)/scale), 0,
  *  2^bits-1) in float64, or 0 when scale == 0; channel 0 -> bf16 (nearest
- *  even from float64).  Bits of other tokens sharing a code byte are kept.
+ *  even from float64).  Values: with v_rot, x = (V v_rot)[j] by the same
+ *  fma chain as K'; with a clip ratio r the value grids use min' = r*min and
+ *  max' = r*max (each product rounded to float64) in place of min and max.
+ *  Bits of other tokens sharing a code byte are kept.
  *  Values must stay within the fp16 range after the transform.
  *  A sequence whose seq_len + n_new would exceed capacity is left untouched
  *  and sets KVQ_DEV_CAPACITY.  n_new == 0 is a no-op.
@@ -184,12 +197,19 @@ int kvq_num_selected(float sparsity, int head_dim);
  * transpose, q' = q A^{-T}, so q'.K' = q.K), §3.2 Eq. 4 (energy pooled over
  * the g = n_q_heads / n_kv_heads query heads of a KV head, e_j^2 =
  * sum_h q'_{h,j}^2; one mask per KV head); channel 0 is always kept.
+ * §3.3 / App. C.2 (diagonal refinement): when Ainvt is a base transform times
+ * a positive diagonal D (and A the base key transform times D^{-1}), pass D
+ * as delta; the energies are then those of the base queries,
+ * u_{h,j} = q'_{h,j} / delta_j (one float64 division), e_j^2 = sum_h u_{h,j}^2,
+ * while qsel / qgsum keep q'.
  *
  *  q       [batch][n_q_heads][128], dtype F32 or BF16; query head h belongs
  *          to KV head h / g
  *  Ainvt   [n_kv_heads][128][128] float64, row-major, 16-byte aligned:
  *          q'[j] = sum_c q[c] Ainvt[c][j]
  *          (fma chain over c from 0.0), e^2 by an fma chain over h ascending
+ *  delta   [n_kv_heads][128] float64 positive finite (NULL: no refinement);
+ *          other values give an unspecified but valid channel list
  *  idx     out [batch][n_kv_heads][k] int32: channel 0 and the k-1 channels of
  *          1..127 with the largest e^2 (ties to the lower index), ascending
  *  qsel    out [batch][n_q_heads][k] float32: q'[h][idx[i]] rounded to fp32
@@ -202,7 +222,7 @@ int kvq_num_selected(float sparsity, int head_dim);
  *  (n_q_heads not a multiple of n_kv_heads, or g > 32), KVQ_ERR_CUDA.
  */
 int kvq_select_channels(const kvq_cache *cache, const void *q, int dtype,
-                        int n_q_heads, const double *Ainvt, float sparsity,
+                        int n_q_heads, const double *Ainvt, const double *delta, float sparsity,
                         int32_t *idx, float *qsel, float *qgsum, int *k_out,
                         kvq_stream_t stream);
 
@@ -224,7 +244,9 @@ size_t kvq_decode_workspace(const kvq_cache *cache, int n_q_heads, int k);
  *  score_h(t) = [qsel_h0 * ch0(t) + sum_g (scale_g(t) * sum_{c in S_g}
  *               qsel_hc * code_c(t) + zero_g(t) * qgsum_hg)] / sqrt(128)
  *  out     [batch][n_q_heads][128] float32 = sum_t p_h(t) v_hat(t) / sum_t p_h(t)
- *          (zeros for a sequence with no tokens)
+ *          (zeros for a sequence with no tokens); with cache->v_rot set the
+ *          aggregate is rotated back (Dual-QK §3.3), out = o v_rot^T, in
+ *          float64 over the 128 channels from the float32 merged sums
  *  idx, qsel, qgsum, k exactly as produced by kvq_select_channels
  *  ws      device workspace of at least kvq_decode_workspace() bytes,
  *          16-byte aligned; contents need no initialisation
@@ -251,7 +273,7 @@ int kvq_decode_attn(const kvq_cache *cache, int n_q_heads, const int32_t *idx,
  *
  *  q       [batch][n_q_heads][128]; k_new, v_new [batch][n_kv_heads][n_new][128];
  *          all of dtype KVQ_DTYPE_F32 or _BF16
- *  A, Ainvt  as for kvq_append / kvq_select_channels (16-byte aligned)
+ *  A, Ainvt, delta  as for kvq_append / kvq_select_channels (16-byte aligned)
  *  idx, qsel, qgsum  outputs as for kvq_select_channels
  *  out, ws, ws_bytes  as for kvq_decode_attn (kvq_decode_workspace() with the
  *          k of `sparsity`)
@@ -259,7 +281,7 @@ int kvq_decode_attn(const kvq_cache *cache, int n_q_heads, const int32_t *idx,
  */
 int kvq_decode_step(const kvq_cache *cache, const void *q, const void *k_new,
                     const void *v_new, int dtype, int n_q_heads, int n_new,
-                    const double *A, const double *Ainvt, float sparsity,
+                    const double *A, const double *Ainvt, const double *delta, float sparsity,
                     int32_t *idx, float *qsel, float *qgsum, float *out,
                     void *ws, size_t ws_bytes, kvq_stream_t stream);
 

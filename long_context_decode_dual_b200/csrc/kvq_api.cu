@@ -16,7 +16,9 @@ int check_cache(const kvq_cache *c) {
         return KVQ_ERR_SHAPE;
     if (c->capacity % kT) return KVQ_ERR_SHAPE;
     if (c->n_sink < 0 || c->n_recent < 0 || c->n_sink + c->n_recent > KVQ_MAX_PROTECTED) return KVQ_ERR_ARG;
-    if (!aligned(c->pages, 256) || !aligned(c->seq_len, 4) || !aligned(c->status, 4)) return KVQ_ERR_ALIGN;
+    if (!(c->v_clip == 0.0 || (c->v_clip > 0.0 && c->v_clip <= 1.0))) return KVQ_ERR_ARG;
+    if (!aligned(c->pages, 256) || !aligned(c->seq_len, 4) || !aligned(c->status, 4) || !aligned(c->v_rot, 16))
+        return KVQ_ERR_ALIGN;
     return KVQ_OK;
 }
 
@@ -45,7 +47,7 @@ int check_decode_args(const kvq_cache *c, int Hq, int k) {
 
 extern "C" {
 
-int kvq_version(void) { return 100; }
+int kvq_version(void) { return 101; }
 
 const char *kvq_status_string(int s) {
     switch (s) {
@@ -111,8 +113,8 @@ int kvq_num_selected(float sparsity, int head_dim) {
 }
 
 int kvq_select_channels(const kvq_cache *c, const void *q, int dtype, int n_q_heads,
-                        const double *Ainvt, float sparsity, int32_t *idx, float *qsel,
-                        float *qgsum, int *k_out, kvq_stream_t stream) {
+                        const double *Ainvt, const double *delta, float sparsity, int32_t *idx,
+                        float *qsel, float *qgsum, int *k_out, kvq_stream_t stream) {
     int st = check_cache(c);
     if (st) return st;
     if (!q || !Ainvt || !idx || !qsel || !qgsum) return KVQ_ERR_ARG;
@@ -120,11 +122,12 @@ int kvq_select_channels(const kvq_cache *c, const void *q, int dtype, int n_q_he
     const int k = kvq_num_selected(sparsity, kD);
     if (k < 0) return KVQ_ERR_ARG;
     if (n_q_heads < 1 || n_q_heads % c->n_kv_heads || n_q_heads / c->n_kv_heads > 32) return KVQ_ERR_SHAPE;
-    if (!aligned(q, dtype_align(dtype)) || !aligned(Ainvt, 16) || !aligned(idx, 4) || !aligned(qsel, 4) ||
-        !aligned(qgsum, 4))
+    if (!aligned(q, dtype_align(dtype)) || !aligned(Ainvt, 16) || !aligned(delta, 8) || !aligned(idx, 4) ||
+        !aligned(qsel, 4) || !aligned(qgsum, 4))
         return KVQ_ERR_ALIGN;
     if (k_out) *k_out = k;
-    return cuda_status(launch_select(*c, q, dtype, n_q_heads, Ainvt, k, idx, qsel, qgsum, (cudaStream_t)stream));
+    return cuda_status(
+        launch_select(*c, q, dtype, n_q_heads, Ainvt, delta, k, idx, qsel, qgsum, (cudaStream_t)stream));
 }
 
 size_t kvq_decode_workspace(const kvq_cache *c, int n_q_heads, int k) {
@@ -149,9 +152,9 @@ int kvq_decode_attn(const kvq_cache *c, int n_q_heads, const int32_t *idx, const
 }
 
 int kvq_decode_step(const kvq_cache *c, const void *q, const void *k_new, const void *v_new, int dtype,
-                    int n_q_heads, int n_new, const double *A, const double *Ainvt, float sparsity,
-                    int32_t *idx, float *qsel, float *qgsum, float *out, void *ws, size_t ws_bytes,
-                    kvq_stream_t stream) {
+                    int n_q_heads, int n_new, const double *A, const double *Ainvt, const double *delta,
+                    float sparsity, int32_t *idx, float *qsel, float *qgsum, float *out, void *ws,
+                    size_t ws_bytes, kvq_stream_t stream) {
     int st = check_cache(c);
     if (st) return st;
     if (!q || !A || !Ainvt || !idx || !qsel || !qgsum || !out || n_new < 0) return KVQ_ERR_ARG;
@@ -163,7 +166,8 @@ int kvq_decode_step(const kvq_cache *c, const void *q, const void *k_new, const 
     if (st) return st;
     const size_t al = dtype_align(dtype);
     if (!aligned(q, al) || (n_new > 0 && (!aligned(k_new, al) || !aligned(v_new, al))) || !aligned(A, 16) ||
-        !aligned(Ainvt, 16) || !aligned(idx, 4) || !aligned(qsel, 4) || !aligned(qgsum, 4) || !aligned(out, 4))
+        !aligned(Ainvt, 16) || !aligned(delta, 8) || !aligned(idx, 4) || !aligned(qsel, 4) ||
+        !aligned(qgsum, 4) || !aligned(out, 4))
         return KVQ_ERR_ALIGN;
     if (n_new > c->capacity) return KVQ_ERR_CAPACITY;
     const int sms = num_sms();
@@ -171,8 +175,8 @@ int kvq_decode_step(const kvq_cache *c, const void *q, const void *k_new, const 
     const int S = decode_splits(*c, n_q_heads, k, sms);
     if (!ws || ws_bytes < decode_ws_bytes(*c, n_q_heads, S)) return KVQ_ERR_WORKSPACE;
     if (!aligned(ws, 16)) return KVQ_ERR_ALIGN;
-    return cuda_status(launch_decode_step(*c, n_q_heads, q, k_new, v_new, dtype, n_new, A, Ainvt, k, idx, qsel,
-                                          qgsum, out, ws, S, (cudaStream_t)stream));
+    return cuda_status(launch_decode_step(*c, n_q_heads, q, k_new, v_new, dtype, n_new, A, Ainvt, delta, k, idx,
+                                          qsel, qgsum, out, ws, S, (cudaStream_t)stream));
 }
 
 size_t kvq_bf16_decode_workspace(int B, int Hq, int Hkv, int N) {

@@ -8,6 +8,12 @@
 //        min/max grid per token; within each 128-token page the codes are
 //        stored channel-major, one channel of one page per 32-byte row.
 //
+// With a value rotation (§3.3, App. B.2: values are rotated before they are
+// quantized, with the grid clipped to [clip*min, clip*max]; keys are not
+// clipped) the values go through the same fixed-order transform as the keys,
+// with the rotation in place of A; the protected BF16 copies hold the rotated
+// values too.
+//
 // One CTA = one (sequence, KV head) and a tile of kTile destination positions
 // aligned to kTile, so the code bytes a CTA writes belong to it alone; thread
 // j owns channel j and warp w owns quantization group w.  The arithmetic is
@@ -50,8 +56,8 @@ template <typename Tin, int BITS, int NG>
 __global__ void __launch_bounds__(128)
 append_kernel(uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len,
               uint32_t *__restrict__ status, const Tin *__restrict__ K,
-              const Tin *__restrict__ V, const double *__restrict__ A, int Hkv, int NB,
-              int n_new, int capacity, int n_sink, int n_recent) {
+              const Tin *__restrict__ V, const double *__restrict__ A, const double *__restrict__ Rv,
+              double vclip, int Hkv, int NB, int n_new, int capacity, int n_sink, int n_recent) {
     constexpr int R = row_bytes(BITS);
     __shared__ double ks[kTile][kD];
     __shared__ double vs[kTile][kD];
@@ -86,34 +92,45 @@ append_kernel(uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len,
     const int lane = j & 31;
     const int grp = j >> 5;             // quantization group (= warp)
 
-    // K'[t][j] = sum_c K[t][c] A[c][j], fma chain c = 0..127 from 0.0.  A full
-    // tile interleaves its kTile chains (A read once per c); a partial tile (a
+    // Y[t][j] = sum_c X[t][c] M[c][j], fma chain c = 0..127 from 0.0.  A full
+    // tile interleaves its kTile chains (M read once per c); a partial tile (a
     // decode step appends one token) runs only the chains of its tokens.
-    double acc[kTile];
+    auto transform = [&](const double (*xs)[kD], const double *M, double (&acc)[kTile]) {
 #pragma unroll
-    for (int tt = 0; tt < kTile; tt++) acc[tt] = 0.0;
-    const double *Ah = A + (size_t)h * kD * kD + j;
-    if (hi - lo == kTile) {
+        for (int tt = 0; tt < kTile; tt++) acc[tt] = 0.0;
+        const double *Mh = M + (size_t)h * kD * kD + j;
+        if (hi - lo == kTile) {
 #pragma unroll 4
-        for (int c = 0; c < kD; c++) {
-            const double a = __ldg(Ah + (size_t)c * kD);
+            for (int c = 0; c < kD; c++) {
+                const double a = __ldg(Mh + (size_t)c * kD);
 #pragma unroll
-            for (int tt = 0; tt < kTile; tt++) acc[tt] = fma(ks[tt][c], a, acc[tt]);
-        }
-    } else {
-#pragma unroll
-        for (int tt = 0; tt < kTile; tt++) {
-            if (first + tt < lo || first + tt >= hi) continue;     // uniform over the CTA
-            double a_reg[8];
-            double x = 0.0;
-            for (int c0 = 0; c0 < kD; c0 += 8) {
-#pragma unroll
-                for (int u = 0; u < 8; u++) a_reg[u] = __ldg(Ah + (size_t)(c0 + u) * kD);
-#pragma unroll
-                for (int u = 0; u < 8; u++) x = fma(ks[tt][c0 + u], a_reg[u], x);
+                for (int tt = 0; tt < kTile; tt++) acc[tt] = fma(xs[tt][c], a, acc[tt]);
             }
-            acc[tt] = x;
+        } else {
+#pragma unroll
+            for (int tt = 0; tt < kTile; tt++) {
+                if (first + tt < lo || first + tt >= hi) continue;     // uniform over the CTA
+                double a_reg[8];
+                double x = 0.0;
+                for (int c0 = 0; c0 < kD; c0 += 8) {
+#pragma unroll
+                    for (int u = 0; u < 8; u++) a_reg[u] = __ldg(Mh + (size_t)(c0 + u) * kD);
+#pragma unroll
+                    for (int u = 0; u < 8; u++) x = fma(xs[tt][c0 + u], a_reg[u], x);
+                }
+                acc[tt] = x;
+            }
         }
+    };
+    double acc[kTile];
+    transform(ks, A, acc);                  // K' = K A
+    if (Rv) {
+        // V Rv, written back over the tile's values once every chain has read them
+        double vacc[kTile];
+        transform(vs, Rv, vacc);
+        __syncthreads();
+#pragma unroll
+        for (int tt = 0; tt < kTile; tt++) vs[tt][j] = vacc[tt];
     }
 
     uint8_t *page = pages + (((size_t)b * Hkv + h) * NB + (size_t)(first / kT)) * page_bytes(BITS, NG);
@@ -133,6 +150,10 @@ append_kernel(uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len,
         if constexpr (NG == 1) return quantize_block128<BITS>(x, in_range, red, sb, zb);
         else return quantize_lane<BITS>(x, in_range, sb, zb);
     };
+    auto quantize_v = [&](double x, uint16_t &sb, uint16_t &zb) -> uint32_t {
+        if constexpr (NG == 1) return quantize_block128<BITS>(x, true, red, sb, zb, vclip);
+        else return quantize_lane<BITS>(x, true, sb, zb, vclip);
+    };
 
     // keys: channel 0 -> bf16; group 0 starts at channel 1
     uint32_t codes[kTile];
@@ -147,13 +168,14 @@ append_kernel(uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len,
     }
     if (j != 0) store_row<BITS>(page + (size_t)j * R + t0 * BITS / 8, codes, valid);
 
-    // values: no transform
+    // values (rotated when Rv is given; thread j reads only its own channel
+    // from here on), grids clipped by vclip
 #pragma unroll
     for (int tt = 0; tt < kTile; tt++) {
         uint16_t sb, zb;
         codes[tt] = 0;
         if (!(valid >> tt & 1u)) continue;
-        codes[tt] = quantize(vs[tt][j], true, sb, zb);
+        codes[tt] = quantize_v(vs[tt][j], sb, zb);
         if (writes_meta) vmeta[meta_word(mg, t0 + tt)] = (uint32_t)sb | ((uint32_t)zb << 16);
     }
     store_row<BITS>(page + off_vcodes(BITS) + (size_t)j * R + t0 * BITS / 8, codes, valid);
@@ -180,22 +202,25 @@ append_kernel(uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len,
 // spread over 4 * n_kv_heads * batch SMs.  Warp w transforms and quantizes new
 // token w (lane = channel of the group); the codes then go through shared
 // memory to one thread per channel row, which merges the new tokens into the
-// packed bytes in order (neighbouring tokens share bytes).  The last CTA of a
-// sequence to finish advances its length, using the sequence's completion
-// counter in the status array.
+// packed bytes in order (neighbouring tokens share bytes).  With a value
+// rotation the same staging memory then takes the group's 32 columns of the
+// rotation for the values' chains.  The last CTA of a sequence to finish
+// advances its length, using the sequence's completion counter in the status
+// array.
 constexpr int kSmallMax = 4;
 
 template <typename Tin, int BITS>
 __global__ void __launch_bounds__(128)
 append_small_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len,
                     uint32_t *__restrict__ status, const Tin *__restrict__ K,
-                    const Tin *__restrict__ V, const double *__restrict__ A, int Hkv, int NB,
-                    int n_new, int capacity, int n_sink, int n_recent) {
+                    const Tin *__restrict__ V, const double *__restrict__ A, const double *__restrict__ Rv,
+                    double vclip, int Hkv, int NB, int n_new, int capacity, int n_sink, int n_recent) {
     constexpr int R = row_bytes(BITS);
     constexpr int PER = 8 / BITS;
     static_assert(kSmallMax * 32 == 128, "one warp per new token");
-    __shared__ __align__(16) double As[kD][kGroup];        // A[:, 32 grp .. 32 grp + 31]
+    __shared__ __align__(16) double As[kD][kGroup];        // A[:, 32 grp .. 32 grp + 31], then Rv[...]
     __shared__ double ks[kSmallMax][kD];
+    __shared__ double vsd[kSmallMax][kD];                  // full value rows (value rotation only)
     __shared__ uint8_t kcode[kSmallMax][kGroup];
     __shared__ uint8_t vcode[kSmallMax][kGroup];
     __shared__ int s_len;
@@ -211,7 +236,9 @@ append_small_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len,
     cp_async_commit();
     const size_t in_base = ((size_t)b * Hkv + h) * (size_t)n_new;
     for (int e = t; e < n_new * kD; e += 128) ks[e / kD][e % kD] = in_to_double(K[in_base * kD + e]);
-    const double v = (w < n_new) ? in_to_double(V[(in_base + w) * kD + j]) : 0.0;
+    if (Rv)
+        for (int e = t; e < n_new * kD; e += 128) vsd[e / kD][e % kD] = in_to_double(V[in_base * kD + e]);
+    double v = (w < n_new) ? in_to_double(V[(in_base + w) * kD + j]) : 0.0;
     if (t == 0) s_len = seq_len[b];
     cp_async_wait<0>();
     __syncthreads();
@@ -219,19 +246,41 @@ append_small_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len,
     const bool ok = len >= 0 && len + n_new <= capacity;
     uint8_t *unit = pages + ((size_t)b * Hkv + h) * NB * (size_t)page_bytes(BITS);
 
+    // K'[t][j] = sum_c K[t][c] A[c][j], fma chain c = 0..127 from 0.0
+    double x = 0.0;
+    if (ok && w < n_new) {
+#pragma unroll 16
+        for (int c = 0; c < kD; c++) x = fma(ks[w][c], As[c][lane], x);
+    }
+    if (Rv) {
+        // the same chain for the rotated value, (V Rv)[t][j], with the
+        // group's columns of Rv staged over those of A
+        __syncthreads();
+        const double *Rh = Rv + (size_t)h * kD * kD + grp * kGroup;
+        for (int e = t; e < kD * kGroup / 2; e += 128) {
+            const int c = e >> 4, part = e & 15;
+            cp_async16(&As[c][2 * part], Rh + (size_t)c * kD + 2 * part);
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+        __syncthreads();
+        if (ok && w < n_new) {
+            double y = 0.0;
+#pragma unroll 16
+            for (int c = 0; c < kD; c++) y = fma(vsd[w][c], As[c][lane], y);
+            v = y;
+        }
+    }
+
     if (ok && w < n_new) {                                 // uniform over the warp
         const int pos = len + w, tt = pos % kT;
         uint8_t *page = unit + (size_t)(pos / kT) * page_bytes(BITS);
-        // K'[t][j] = sum_c K[t][c] A[c][j], fma chain c = 0..127 from 0.0
-        double x = 0.0;
-#pragma unroll 16
-        for (int c = 0; c < kD; c++) x = fma(ks[w][c], As[c][lane], x);
         uint16_t sb, zb;
         kcode[w][lane] = (uint8_t)quantize_lane<BITS>(x, j != 0, sb, zb);
         if (lane == 0)
             reinterpret_cast<uint32_t *>(page + off_kmeta(BITS))[meta_word(grp, tt)] = (uint32_t)sb | ((uint32_t)zb << 16);
         if (j == 0) reinterpret_cast<uint16_t *>(page + off_ch0(BITS))[tt] = __bfloat16_as_ushort(__double2bfloat16(x));
-        vcode[w][lane] = (uint8_t)quantize_lane<BITS>(v, true, sb, zb);
+        vcode[w][lane] = (uint8_t)quantize_lane<BITS>(v, true, sb, zb, vclip);
         if (lane == 0)
             reinterpret_cast<uint32_t *>(page + off_vmeta(BITS))[meta_word(grp, tt)] = (uint32_t)sb | ((uint32_t)zb << 16);
         // protected tier: BF16 copies (sink tokens, the last n_recent tokens)
@@ -284,6 +333,8 @@ __global__ void advance_kernel(int32_t *seq_len, int B, int n_new, int capacity)
 template <typename Tin, int BITS, int NG>
 cudaError_t launch_append_t(const kvq_cache &c, const void *K, const void *V, int n_new,
                             const double *A, cudaStream_t st) {
+    const double *Rv = c.v_rot;
+    const double vclip = value_clip(c);
     const int NB = c.capacity / kT;
     // a few tokens with groups of 32: one CTA per group; otherwise (prefill,
     // or one grid per token) the tile kernel and the length advance
@@ -291,13 +342,13 @@ cudaError_t launch_append_t(const kvq_cache &c, const void *K, const void *V, in
         dim3 grid((unsigned)kNG, (unsigned)c.n_kv_heads, (unsigned)c.batch);
         append_small_kernel<Tin, BITS><<<grid, 128, 0, st>>>(
             static_cast<uint8_t *>(c.pages), c.seq_len, c.status, static_cast<const Tin *>(K),
-            static_cast<const Tin *>(V), A, c.n_kv_heads, NB, n_new, c.capacity, c.n_sink, c.n_recent);
+            static_cast<const Tin *>(V), A, Rv, vclip, c.n_kv_heads, NB, n_new, c.capacity, c.n_sink, c.n_recent);
         return cudaGetLastError();
     }
     dim3 grid((unsigned)((n_new + kTile - 1) / kTile + 1), (unsigned)c.n_kv_heads, (unsigned)c.batch);
     append_kernel<Tin, BITS, NG><<<grid, 128, 0, st>>>(
         static_cast<uint8_t *>(c.pages), c.seq_len, c.status, static_cast<const Tin *>(K),
-        static_cast<const Tin *>(V), A, c.n_kv_heads, NB, n_new, c.capacity, c.n_sink, c.n_recent);
+        static_cast<const Tin *>(V), A, Rv, vclip, c.n_kv_heads, NB, n_new, c.capacity, c.n_sink, c.n_recent);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     advance_kernel<<<(c.batch + 127) / 128, 128, 0, st>>>(c.seq_len, c.batch, n_new, c.capacity);

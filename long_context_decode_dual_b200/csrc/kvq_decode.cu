@@ -13,9 +13,9 @@ cudaError_t launch_decode_mma(const kvq_cache &c, int Hq, const int32_t *idx, co
 int decode_mma_splits(int units, int nblk, int num_sms, int tier);
 int step_mma_max_new();
 cudaError_t launch_step_mma(const kvq_cache &c, int Hq, const void *q, const void *k_new, const void *v_new,
-                            int dtype, int n_new, const double *A, const double *Ainvt, int k, int32_t *idx,
-                            float *qsel, float *qgsum, float *part_o, float2 *part_ml, int S, float *out,
-                            cudaStream_t st);
+                            int dtype, int n_new, const double *A, const double *Ainvt, const double *delta,
+                            int k, int32_t *idx, float *qsel, float *qgsum, float *part_o, float2 *part_ml,
+                            int S, float *out, cudaStream_t st);
 
 // The tensor-core kernel covers INT2 codes with 4 query heads per KV head;
 // other shapes use the CUDA-core kernel.
@@ -62,17 +62,17 @@ cudaError_t launch_decode(const kvq_cache &c, int Hq, const int32_t *idx, const 
 // tokens runs as one fused launch; any other shape as the three calls.
 cudaError_t launch_decode_step(const kvq_cache &c, int Hq, const void *q, const void *k_new,
                                const void *v_new, int dtype, int n_new, const double *A,
-                               const double *Ainvt, int k, int32_t *idx, float *qsel, float *qgsum,
-                               float *out, void *ws, int S, cudaStream_t st) {
+                               const double *Ainvt, const double *delta, int k, int32_t *idx, float *qsel,
+                               float *qgsum, float *out, void *ws, int S, cudaStream_t st) {
     if (use_mma(c, Hq) && n_new <= step_mma_max_new()) {
         float *part_o = static_cast<float *>(ws);
         float2 *part_ml = reinterpret_cast<float2 *>(part_o + (size_t)c.batch * Hq * S * kD);
-        return launch_step_mma(c, Hq, q, k_new, v_new, dtype, n_new, A, Ainvt, k, idx, qsel, qgsum, part_o,
-                               part_ml, S, out, st);
+        return launch_step_mma(c, Hq, q, k_new, v_new, dtype, n_new, A, Ainvt, delta, k, idx, qsel, qgsum,
+                               part_o, part_ml, S, out, st);
     }
     cudaError_t e = cudaSuccess;
     if (n_new > 0) e = launch_append(c, k_new, v_new, dtype, n_new, A, st);
-    if (e == cudaSuccess) e = launch_select(c, q, dtype, Hq, Ainvt, k, idx, qsel, qgsum, st);
+    if (e == cudaSuccess) e = launch_select(c, q, dtype, Hq, Ainvt, delta, k, idx, qsel, qgsum, st);
     if (e == cudaSuccess) e = launch_decode(c, Hq, idx, qsel, qgsum, k, out, ws, S, st);
     return e;
 }

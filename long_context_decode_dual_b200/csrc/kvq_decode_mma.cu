@@ -113,11 +113,16 @@ struct PexScratch {                    // in MmaShared::pex
     double qin[4][kD];                 // query rows, float64 (exact for bf16 / f32 inputs)
 };
 // new key rows: float (exact) in MmaShared::q until the channel choice, then
-// float64 in the staging memory freed by the A^{-T} block
+// float64 in the staging memory freed by the A^{-T} block; new value rows in
+// registers, then float64 after the key rows.  With a value rotation its
+// 64-column block follows A's through the same two halves of the staging
+// memory (rows 0..63 where A's were, then rows 64..127).
 constexpr int kOffKs = kBlkRowBytes * 64;                         // past the high rows of A
-static_assert(kOffKs + kStepMaxNew * kD * (int)sizeof(double) <= kOffALo, "new key rows below the low rows of A");
+constexpr int kOffVs = kOffKs + kStepMaxNew * kD * (int)sizeof(double);
+static_assert(kOffVs + kStepMaxNew * kD * (int)sizeof(double) <= kOffALo, "new rows below the low rows of A");
+constexpr int kVPre = kStepMaxNew * kD / kThreads;                 // value elements per thread
+static_assert(kVPre * kThreads == kStepMaxNew * kD, "value rows split evenly over the threads");
 struct BqScratch {                     // in MmaShared::bq
-    float vs[kStepMaxNew][kCols];      // new value rows, this CTA's channels
     int sel[kD];
 };
 static_assert(sizeof(PexScratch) <= sizeof(((MmaShared *)0)->pex), "query and key rows fit the exchange buffers");
@@ -327,7 +332,8 @@ template <int NG>
 __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restrict__ unit_pages, int lo, int hi,
                                           Split sp, int S, int s, size_t qrow0, float *__restrict__ part_o,
                                           float2 *__restrict__ part_ml, float *__restrict__ out,
-                                          uint32_t *counter, uint32_t *status, bool first_issued) {
+                                          uint32_t *counter, uint32_t *status, bool first_issued,
+                                          const double *rot) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int pair = warp >> 1, half = warp & 1;
     const int gid = lane >> 2, tig = lane & 3;
@@ -635,7 +641,7 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
     }
     static_assert(merge_scratch_floats(4, kThreads, 256) * 4 <= 2 * 2 * kStageBytes, "merge scratch fits stages 2-3");
     merge_unit_if_last<4, kThreads>(part_o, part_ml, S, qrow0, out, counter,
-                                    reinterpret_cast<float *>(sh.stage[2][0]));
+                                    reinterpret_cast<float *>(sh.stage[2][0]), rot);
 }
 
 // A CTA that handles the protected tier instead of pages: half `half_idx` of
@@ -643,7 +649,7 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
 // sh.chan_pos / sh.q (a barrier after their last write).
 __device__ __forceinline__ void tier_cta(MmaShared &sh, const uint8_t *slots, int len, int n_sink, int n_recent,
                                          int half_idx, int k, float *part_o, float2 *part_ml, size_t qrow0, int S,
-                                         int s, float *out, uint32_t *counter) {
+                                         int s, float *out, uint32_t *counter, const double *rot) {
     int *list = reinterpret_cast<int *>(sh.stage[0][0]);                    // position -> channel
     float *scratch = reinterpret_cast<float *>(sh.stage[0][0] + kD * sizeof(int));
     static_assert(kD * sizeof(int) + tier_scratch_floats(4) * 4 <= 2 * (size_t)kStageBytes * 2,
@@ -657,7 +663,8 @@ __device__ __forceinline__ void tier_cta(MmaShared &sh, const uint8_t *slots, in
     const int slot0 = min(NP, half_idx * per), slot1 = min(NP, slot0 + per);
     tier_partial<4, kThreads>(slots, len, n_sink, n_recent, slot0, slot1, &sh.q[0][0], kD, 1, list, k, part_o,
                               part_ml, qrow0, S, s, scratch);
-    merge_unit_if_last<4, kThreads>(part_o, part_ml, S, qrow0, out, counter, reinterpret_cast<float *>(sh.stage[2][0]));
+    merge_unit_if_last<4, kThreads>(part_o, part_ml, S, qrow0, out, counter, reinterpret_cast<float *>(sh.stage[2][0]),
+                                    rot);
 }
 
 // ---------------------------------------------------------------- decode
@@ -667,11 +674,13 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
                   int NB, int Hq, const int32_t *__restrict__ idx, const float *__restrict__ qsel,
                   const float *__restrict__ qgsum, int k, float *__restrict__ part_o,
                   float2 *__restrict__ part_ml, int S, float *__restrict__ out,
-                  uint32_t *__restrict__ counters, uint32_t *__restrict__ status, int n_sink, int n_recent) {
+                  uint32_t *__restrict__ counters, uint32_t *__restrict__ status, int n_sink, int n_recent,
+                  const double *__restrict__ v_rot) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     MmaShared &sh = *reinterpret_cast<MmaShared *>(smem_raw);
 
     const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const double *rot = v_rot ? v_rot + (size_t)h * kD * kD : nullptr;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const size_t unit = (size_t)b * Hkv + h;
     const size_t qrow0 = (size_t)b * Hq + (size_t)h * 4;
@@ -702,12 +711,13 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
     const int S_pages = S - ((n_sink + n_recent > 0) ? 2 : 0);   // the last two splits take the tier
     if (s >= S_pages) {
         tier_cta(sh, unit_slots(const_cast<uint8_t *>(pages), gridDim.z, Hkv, NB, 2, unit, n_sink + n_recent, NG),
-                 len, n_sink, n_recent, s - S_pages, k, part_o, part_ml, qrow0, S, s, out, counters + unit);
+                 len, n_sink, n_recent, s - S_pages, k, part_o, part_ml, qrow0, S, s, out, counters + unit, rot);
         return;
     }
     const Tier tr = tier_of(len, n_sink, n_recent);
     run_pages<NG>(sh, pages + unit * NB * (size_t)page_bytes(2, NG), tr.sink_end, tr.recent_start,
-              split_of(tr.recent_start, S_pages, s), S, s, qrow0, part_o, part_ml, out, counters + unit, status, false);
+                  split_of(tr.recent_start, S_pages, s), S, s, qrow0, part_o, part_ml, out, counters + unit, status,
+                  false, rot);
 }
 
 // ---------------------------------------------------------------- fused step
@@ -723,7 +733,8 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 2)
 step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint32_t *__restrict__ status,
                 int Hkv, int NB, int Hq, const Tin *__restrict__ q, const Tin *__restrict__ k_new,
                 const Tin *__restrict__ v_new, int n_new, const double *__restrict__ A,
-                const double *__restrict__ Ainvt, int k, int32_t *__restrict__ idx, float *__restrict__ qsel,
+                const double *__restrict__ Ainvt, const double *__restrict__ delta,
+                const double *__restrict__ v_rot, double vclip, int k, int32_t *__restrict__ idx, float *__restrict__ qsel,
                 float *__restrict__ qgsum, float *__restrict__ part_o, float2 *__restrict__ part_ml, int S,
                 float *__restrict__ out, int n_sink, int n_recent) {
     namespace cg = cooperative_groups;
@@ -739,6 +750,7 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
     PexScratch &px = *reinterpret_cast<PexScratch *>(&sh.pex[0][0][0]);
     float *ks_f = &sh.q[0][0];                                                   // [nw][128]
     double (*ks)[kD] = reinterpret_cast<double (*)[kD]>(P + kOffKs);             // [nw][128], later
+    double (*vsd)[kD] = reinterpret_cast<double (*)[kD]>(P + kOffVs);            // [nw][128], later
     BqScratch &bx = *reinterpret_cast<BqScratch *>(&sh.bq[0][0]);
 
     cg::cluster_group cluster = cg::this_cluster();
@@ -805,11 +817,15 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
     }
     const int nw = w1 - w0;
     const size_t in_base = unit * (size_t)n_new + w0;
+    float vpre[kVPre];
     if (nw > 0) {
         stage_block(a_lo, A_blk, 0, 64);
         for (int e = tid; e < nw * kD; e += kThreads) ks_f[e] = in_to_float(k_new[in_base * kD + e]);
-        for (int e = tid; e < nw * kCols; e += kThreads)
-            bx.vs[e / kCols][e % kCols] = in_to_float(v_new[(in_base + e / kCols) * kD + r * kCols + e % kCols]);
+#pragma unroll
+        for (int i = 0; i < kVPre; i++) {
+            const int e = tid + i * kThreads;
+            vpre[i] = e < nw * kD ? in_to_float(v_new[in_base * kD + e]) : 0.f;
+        }
     }
     cp_async_commit();
     // every CTA of sequence b has read its length once the counter reaches
@@ -842,8 +858,14 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
         stage_block(a_hi, A_blk, 64, 64);
         cp_async_commit();
         for (int e = tid; e < nw * kD; e += kThreads) ks[e / kD][e % kD] = (double)ks_f[e];
+#pragma unroll
+        for (int i = 0; i < kVPre; i++) {
+            const int e = tid + i * kThreads;
+            if (e < nw * kD) vsd[e / kD][e % kD] = (double)vpre[i];
+        }
         __syncthreads();
         const int w = warp >> 1, jj = (warp & 1) * 32 + lane, j = r * kCols + jj;
+        const double *R_blk = v_rot ? v_rot + (size_t)h * kD * kD + r * kCols : nullptr;
         double x = 0.0;
         if (w < nw) {
 #pragma unroll 16
@@ -851,22 +873,49 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
         }
         cp_async_wait<0>();
         __syncthreads();
+        if (R_blk) {                                // rows 0..63 of the rotation over A's
+            stage_block(a_lo, R_blk, 0, 64);
+            cp_async_commit();
+        }
         if (w < nw) {                               // uniform over the warp
 #pragma unroll 16
             for (int c = 64; c < kD; c++) x = fma(ks[w][c], a_hi[c - 64][jj], x);
+        }
+        // value of channel j: (V Rv)[j] by the same chain with the rotation in
+        // place of A, or V[j]
+        double v = w < nw ? vsd[w][j] : 0.0;
+        if (R_blk) {
+            __syncthreads();                        // every read of A's high rows is done
+            stage_block(a_hi, R_blk, 64, 64);
+            cp_async_commit();
+            cp_async_wait<1>();
+            __syncthreads();
+            double y = 0.0;
+            if (w < nw) {
+#pragma unroll 16
+                for (int c = 0; c < 64; c++) y = fma(vsd[w][c], a_lo[c][jj], y);
+            }
+            cp_async_wait<0>();
+            __syncthreads();
+            if (w < nw) {
+#pragma unroll 16
+                for (int c = 64; c < kD; c++) y = fma(vsd[w][c], a_hi[c - 64][jj], y);
+            }
+            v = y;
+        }
+        if (w < nw) {                               // uniform over the warp
             const int pos = L0 + w0 + w;
             if (is_tier && stores_slot(pos, L0 + n_new, n_sink, n_recent)) {
                 uint16_t *dst = reinterpret_cast<uint16_t *>(unit_slots(pages, B, Hkv, NB, 2, unit, NPt, NG) +
                                                              (size_t)slot_of(pos, n_sink, n_recent) * kSlotBytes);
                 dst[j] = __bfloat16_as_ushort(__double2bfloat16(x));
-                dst[kD + j] = __bfloat16_as_ushort(__double2bfloat16((double)bx.vs[w][jj]));
+                dst[kD + j] = __bfloat16_as_ushort(__double2bfloat16(v));
             }
         }
         // codes: by the cluster of the page, or by the tier cluster when no
         // split reads the page in this step (uniform over the warp).  Groups
         // of 32: warp = group; one grid per token: the range of token w is
         // met over warps 2w, 2w+1 of both CTAs (distributed shared memory).
-        const double v = (double)bx.vs[w < nw ? w : 0][jj];
         double klo = 0.0, khi = 0.0, vlo = 0.0, vhi = 0.0;
         if constexpr (NG == 1) {
             if (w < nw) {
@@ -899,7 +948,8 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
             if (meta_writer)
                 reinterpret_cast<uint32_t *>(page + off_kmeta(2))[meta_word(g, tt)] = (uint32_t)sb | ((uint32_t)zb << 16);
             if (j == 0) reinterpret_cast<uint16_t *>(page + off_ch0(2))[tt] = __bfloat16_as_ushort(__double2bfloat16(x));
-            const uint32_t vc = NG == 1 ? code_in_range<2>(v, vlo, vhi, sb, zb) : quantize_lane<2>(v, true, sb, zb);
+            const uint32_t vc = NG == 1 ? code_in_range<2>(v, __dmul_rn(vclip, vlo), __dmul_rn(vclip, vhi), sb, zb)
+                                        : quantize_lane<2>(v, true, sb, zb, vclip);
             if (meta_writer)
                 reinterpret_cast<uint32_t *>(page + off_vmeta(2, NG))[meta_word(g, tt)] = (uint32_t)sb | ((uint32_t)zb << 16);
             // positions at or beyond the stored length hold zero bits, so the
@@ -913,9 +963,15 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
     }
     __syncthreads();
     if (tid < kCols) {
+        // pooled energy; with a diagonal refinement, of the base queries
+        // q'_{h,j} / delta_j (the arithmetic of kvq_select_channels)
+        const double dj = delta ? delta[(size_t)h * kD + r * kCols + tid] : 1.0;
         double e = 0.0;
 #pragma unroll
-        for (int hl = 0; hl < 4; hl++) e = fma(sh.qp_own[hl][tid], sh.qp_own[hl][tid], e);
+        for (int hl = 0; hl < 4; hl++) {
+            const double u = delta ? sh.qp_own[hl][tid] / dj : sh.qp_own[hl][tid];
+            e = fma(u, u, e);
+        }
         sh.e2_own[tid] = e;
     }
     cluster.sync();            // the cluster's q', energies and new tokens are in place
@@ -982,12 +1038,13 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
     __syncthreads();
     build_plan<NG>(sh, tid, warp, lane);
 
+    const double *rot = v_rot ? v_rot + (size_t)h * kD * kD : nullptr;
     if (is_tier)
         tier_cta(sh, unit_slots(pages, B, Hkv, NB, 2, unit, NPt, NG), len, n_sink, n_recent, s - S_pages, k, part_o,
-                 part_ml, qrow0, S, s, out, status + 1 + B + unit);
+                 part_ml, qrow0, S, s, out, status + 1 + B + unit, rot);
     else
         run_pages<NG>(sh, unit_pages, tr.sink_end, tr.recent_start, sp, S, s, qrow0, part_o, part_ml, out,
-                  status + 1 + B + unit, status, false);
+                      status + 1 + B + unit, status, false, rot);
     cluster_wait();            // the other CTA no longer reads this CTA's shared memory
 }
 
@@ -1020,7 +1077,7 @@ cudaError_t launch_decode_mma_t(const kvq_cache &c, int Hq, const int32_t *idx, 
     decode_mma_kernel<NG><<<grid, kThreads, smem, st>>>(static_cast<const uint8_t *>(c.pages), c.seq_len,
                                                         c.n_kv_heads, c.capacity / kT, Hq, idx, qsel, qgsum, k,
                                                         part_o, part_ml, S, out, unit_counter(c, 0, 0), c.status,
-                                                        c.n_sink, c.n_recent);
+                                                        c.n_sink, c.n_recent, c.v_rot);
     return cudaGetLastError();
 }
 
@@ -1033,8 +1090,9 @@ cudaError_t launch_decode_mma(const kvq_cache &c, int Hq, const int32_t *idx, co
 
 template <typename Tin, int NG>
 cudaError_t launch_step_mma_t(const kvq_cache &c, int Hq, const void *q, const void *k_new, const void *v_new,
-                              int n_new, const double *A, const double *Ainvt, int k, int32_t *idx, float *qsel,
-                              float *qgsum, float *part_o, float2 *part_ml, int S, float *out, cudaStream_t st) {
+                              int n_new, const double *A, const double *Ainvt, const double *delta, int k,
+                              int32_t *idx, float *qsel, float *qgsum, float *part_o, float2 *part_ml, int S,
+                              float *out, cudaStream_t st) {
     const size_t smem = sizeof(MmaShared);
     static std::atomic<uint64_t> done{0};
     cudaError_t e = set_smem_once(step_mma_kernel<Tin, NG>, (int)smem, done);
@@ -1043,24 +1101,24 @@ cudaError_t launch_step_mma_t(const kvq_cache &c, int Hq, const void *q, const v
     step_mma_kernel<Tin, NG><<<grid, kThreads, smem, st>>>(
         static_cast<uint8_t *>(c.pages), c.seq_len, c.status, c.n_kv_heads, c.capacity / kT, Hq,
         static_cast<const Tin *>(q), static_cast<const Tin *>(k_new), static_cast<const Tin *>(v_new), n_new, A,
-        Ainvt, k, idx, qsel, qgsum, part_o, part_ml, S, out, c.n_sink, c.n_recent);
+        Ainvt, delta, c.v_rot, value_clip(c), k, idx, qsel, qgsum, part_o, part_ml, S, out, c.n_sink, c.n_recent);
     return cudaGetLastError();
 }
 
 cudaError_t launch_step_mma(const kvq_cache &c, int Hq, const void *q, const void *k_new, const void *v_new,
-                            int dtype, int n_new, const double *A, const double *Ainvt, int k, int32_t *idx,
-                            float *qsel, float *qgsum, float *part_o, float2 *part_ml, int S, float *out,
-                            cudaStream_t st) {
+                            int dtype, int n_new, const double *A, const double *Ainvt, const double *delta,
+                            int k, int32_t *idx, float *qsel, float *qgsum, float *part_o, float2 *part_ml,
+                            int S, float *out, cudaStream_t st) {
     const bool one = groups_of(c) == 1;
     if (dtype == KVQ_DTYPE_F32)
-        return one ? launch_step_mma_t<float, 1>(c, Hq, q, k_new, v_new, n_new, A, Ainvt, k, idx, qsel, qgsum,
-                                                 part_o, part_ml, S, out, st)
-                   : launch_step_mma_t<float, kNG>(c, Hq, q, k_new, v_new, n_new, A, Ainvt, k, idx, qsel, qgsum,
-                                                   part_o, part_ml, S, out, st);
-    return one ? launch_step_mma_t<uint16_t, 1>(c, Hq, q, k_new, v_new, n_new, A, Ainvt, k, idx, qsel, qgsum,
-                                                part_o, part_ml, S, out, st)
-               : launch_step_mma_t<uint16_t, kNG>(c, Hq, q, k_new, v_new, n_new, A, Ainvt, k, idx, qsel, qgsum,
-                                                  part_o, part_ml, S, out, st);
+        return one ? launch_step_mma_t<float, 1>(c, Hq, q, k_new, v_new, n_new, A, Ainvt, delta, k, idx, qsel,
+                                                 qgsum, part_o, part_ml, S, out, st)
+                   : launch_step_mma_t<float, kNG>(c, Hq, q, k_new, v_new, n_new, A, Ainvt, delta, k, idx, qsel,
+                                                   qgsum, part_o, part_ml, S, out, st);
+    return one ? launch_step_mma_t<uint16_t, 1>(c, Hq, q, k_new, v_new, n_new, A, Ainvt, delta, k, idx, qsel,
+                                                qgsum, part_o, part_ml, S, out, st)
+               : launch_step_mma_t<uint16_t, kNG>(c, Hq, q, k_new, v_new, n_new, A, Ainvt, delta, k, idx, qsel,
+                                                  qgsum, part_o, part_ml, S, out, st);
 }
 
 size_t decode_mma_smem_bytes() { return sizeof(MmaShared); }

@@ -51,7 +51,7 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
                    const float *__restrict__ qgsum, int k, float *__restrict__ part_o,
                    float2 *__restrict__ part_ml, int S, float *__restrict__ out,
                    uint32_t *__restrict__ counters, uint32_t *__restrict__ status, int n_sink, int n_recent,
-                   int stage_area) {
+                   int stage_area, const double *__restrict__ v_rot) {
     constexpr int R = row_bytes(BITS);
     constexpr int FIX = fixed_bytes(BITS, NG);
     constexpr int GS = kD / NG;                       // channels per quantization group
@@ -115,7 +115,8 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
         tier_partial<G, 128>(unit_slots(const_cast<uint8_t *>(pages), gridDim.z, Hkv, NB, BITS, unit, NPt, NG), len,
                              n_sink, n_recent, slot0, slot1, sq, 1, G, sidx, k, part_o, part_ml, qrow0, S, s,
                              reinterpret_cast<float *>(smem));
-        merge_unit_if_last<G, 128>(part_o, part_ml, S, qrow0, out, counters + unit, reinterpret_cast<float *>(smem));
+        merge_unit_if_last<G, 128>(part_o, part_ml, S, qrow0, out, counters + unit, reinterpret_cast<float *>(smem),
+                                   v_rot ? v_rot + (size_t)h * kD * kD : nullptr);
         return;
     }
     const Tier tr = tier_of(len, n_sink, n_recent);
@@ -239,7 +240,7 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
         if (tid == 0) part_ml[row] = make_float2(m_run[hl], l_run[hl]);
     }
     merge_unit_if_last<G, 128>(part_o, part_ml, S, (size_t)b * Hq + (size_t)h * G, out, counters + unit,
-                          reinterpret_cast<float *>(smem));
+                               reinterpret_cast<float *>(smem), v_rot ? v_rot + (size_t)h * kD * kD : nullptr);
 }
 
 template <int BITS, int G, int NG>
@@ -265,7 +266,7 @@ cudaError_t launch_simt_t(const kvq_cache &c, int Hq, const int32_t *idx, const 
     dim3 grid((unsigned)S, (unsigned)c.n_kv_heads, (unsigned)c.batch);
     fn<<<grid, 128, smem, st>>>(static_cast<const uint8_t *>(c.pages), c.seq_len, c.n_kv_heads,
                                 c.capacity / kT, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out,
-                                unit_counter(c, 0, 0), c.status, c.n_sink, c.n_recent, stage_area);
+                                unit_counter(c, 0, 0), c.status, c.n_sink, c.n_recent, stage_area, c.v_rot);
     return cudaGetLastError();
 }
 

@@ -38,6 +38,8 @@ __host__ __device__ constexpr int meta_word(int g, int t) {
 __host__ __device__ constexpr int fixed_bytes(int bits, int ng = kNG) { return page_bytes(bits, ng) - off_vcodes(bits); }
 // groups per head of a cache (group = 32 or 128 channels)
 inline int groups_of(const kvq_cache &c) { return kD / c.group; }
+// clipping ratio of the value grids (0 in the descriptor: none)
+inline double value_clip(const kvq_cache &c) { return c.v_clip == 0.0 ? 1.0 : c.v_clip; }
 
 // ------------------------------------------------------------ protected tier
 // slot of the protected BF16 tier: 128 bf16 of K' then 128 bf16 of V
@@ -117,11 +119,15 @@ __device__ __forceinline__ uint32_t code_in_range(double x, double lo, double hi
 __device__ __forceinline__ double pos_inf() { return __longlong_as_double(0x7ff0000000000000LL); }
 __device__ __forceinline__ double neg_inf() { return __longlong_as_double(0xfff0000000000000LL); }
 
+// The grid of a warp's 32 values (lane = channel).  With a clipping ratio
+// `clip` (values, Dual-QK App. B.2) the grid spans [clip*min, clip*max]; the
+// products are rounded on their own (no contraction into the subtraction),
+// and clip = 1 leaves the range as it is.
 template <int BITS>
 __device__ __forceinline__ uint32_t quantize_lane(double x, bool in_range, uint16_t &s_bits,
-                                                  uint16_t &z_bits) {
-    const double lo = warp_min(in_range ? x : pos_inf());
-    const double hi = warp_max(in_range ? x : neg_inf());
+                                                  uint16_t &z_bits, double clip = 1.0) {
+    const double lo = __dmul_rn(clip, warp_min(in_range ? x : pos_inf()));
+    const double hi = __dmul_rn(clip, warp_max(in_range ? x : neg_inf()));
     return code_in_range<BITS>(x, lo, hi, s_bits, z_bits);
 }
 // The same over all 128 threads of a CTA (thread = channel; one grid per
@@ -129,7 +135,7 @@ __device__ __forceinline__ uint32_t quantize_lane(double x, bool in_range, uint1
 // no other code uses between the barriers of two calls.
 template <int BITS>
 __device__ __forceinline__ uint32_t quantize_block128(double x, bool in_range, double *red, uint16_t &s_bits,
-                                                      uint16_t &z_bits) {
+                                                      uint16_t &z_bits, double clip = 1.0) {
     const int w = threadIdx.x >> 5;
     const double lo_w = warp_min(in_range ? x : pos_inf());
     const double hi_w = warp_max(in_range ? x : neg_inf());
@@ -139,8 +145,8 @@ __device__ __forceinline__ uint32_t quantize_block128(double x, bool in_range, d
         red[4 + w] = hi_w;
     }
     __syncthreads();
-    const double lo = fmin(fmin(red[0], red[1]), fmin(red[2], red[3]));
-    const double hi = fmax(fmax(red[4], red[5]), fmax(red[6], red[7]));
+    const double lo = __dmul_rn(clip, fmin(fmin(red[0], red[1]), fmin(red[2], red[3])));
+    const double hi = __dmul_rn(clip, fmax(fmax(red[4], red[5]), fmax(red[6], red[7])));
     return code_in_range<BITS>(x, lo, hi, s_bits, z_bits);
 }
 
@@ -182,6 +188,11 @@ cudaError_t set_smem_once(Kernel *fn, int bytes, std::atomic<uint64_t> &done) {
 // splits with R = NT / columns threads per column (each a strided subset of
 // the splits, many independent loads in flight), and the R partial sums are
 // added in a fixed order.
+// With a value rotation `rot` (the unit's KV head's 128 x 128 float64 matrix,
+// row-major, 16-byte aligned; values were stored as V rot) the merged output
+// is rotated back, out[c] = sum_j o[j] rot[c][j] (rot is orthogonal; §3.3
+// reverses the value rotation after aggregation), in float64 over j
+// ascending, in two halves added at the end when NT = 256.
 template <int G, int NT>
 struct MergeShape {
     static constexpr int F = G * kD / 4;                 // float4 columns
@@ -190,13 +201,14 @@ struct MergeShape {
     static_assert(NT >= F ? NT % F == 0 : F % NT == 0, "merge: columns and threads must divide");
 };
 __host__ __device__ constexpr int merge_scratch_floats(int G, int NT, int S) {
-    return 2 * G * S + G + 4 + (NT > G * kD / 4 ? NT / (G * kD / 4) * G * kD : 0);
+    return ((2 * G * S + G + 3) & ~3) + (NT > G * kD / 4 ? NT / (G * kD / 4) * G * kD : 0) + G * kD;
 }
 template <int G, int NT>
 __device__ __forceinline__ void merge_unit_if_last(const float *part_o, const float2 *part_ml, int S,
                                                    size_t qrow0, float *out, uint32_t *counter,
-                                                   float *scratch) {
+                                                   float *scratch, const double *rot = nullptr) {
     using MS = MergeShape<G, NT>;
+    static_assert(NT % kD == 0 && NT / kD <= 2, "rotation: one or two threads per output channel");
     __shared__ int s_last;
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -211,7 +223,17 @@ __device__ __forceinline__ void merge_unit_if_last(const float *part_o, const fl
     float *wl = scratch + G * S;     // [G][S] sum
     float *inv = wl + G * S;         // [G] 1 / total sum
     float4 *part = reinterpret_cast<float4 *>(scratch + ((2 * G * S + G + 3) & ~3));   // [R][F]
+    float *orot = reinterpret_cast<float *>(part) + (MS::R > 1 ? MS::R * MS::F * 4 : 0);   // [G][128]
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    // merged output of head hl, channels c0..c0+3: to `out`, or to shared
+    // memory when it is still to be rotated back
+    auto emit = [&](int hl, int c0, float4 a) {
+        float *o = rot ? orot + hl * kD + c0 : out + (qrow0 + hl) * kD + c0;   // out is only 4-byte aligned
+        o[0] = a.x;
+        o[1] = a.y;
+        o[2] = a.z;
+        o[3] = a.w;
+    };
     for (int e = t; e < G * S; e += NT) {
         const float2 v = __ldcg(part_ml + qrow0 * S + e);     // rows qrow0.. are contiguous
         wm[e] = v.x;
@@ -252,11 +274,7 @@ __device__ __forceinline__ void merge_unit_if_last(const float *part_o, const fl
         }
         if constexpr (MS::R == 1) {
             const float r = inv[hl];
-            float *o = out + (qrow0 + hl) * kD + c0;          // out is only 4-byte aligned
-            o[0] = acc.x * r;
-            o[1] = acc.y * r;
-            o[2] = acc.z * r;
-            o[3] = acc.w * r;
+            emit(hl, c0, make_float4(acc.x * r, acc.y * r, acc.z * r, acc.w * r));
         } else {
             part[sub * MS::F + col] = acc;
         }
@@ -271,11 +289,31 @@ __device__ __forceinline__ void merge_unit_if_last(const float *part_o, const fl
                 a.x += v.x; a.y += v.y; a.z += v.z; a.w += v.w;
             }
             const float r = inv[hl];
-            float *o = out + (qrow0 + hl) * kD + c0;
-            o[0] = a.x * r;
-            o[1] = a.y * r;
-            o[2] = a.z * r;
-            o[3] = a.w * r;
+            emit(hl, c0, make_float4(a.x * r, a.y * r, a.z * r, a.w * r));
+        }
+    }
+    if (rot) {
+        __syncthreads();
+        constexpr int P = NT / kD;                       // threads per output channel
+        constexpr int J = kD / P;                        // terms per thread
+        const int c = t / P, j0 = (t % P) * J;
+        const double2 *row = reinterpret_cast<const double2 *>(rot + (size_t)c * kD + j0);
+        double acc[G];
+#pragma unroll
+        for (int hl = 0; hl < G; hl++) acc[hl] = 0.0;
+#pragma unroll 8
+        for (int jj = 0; jj < J / 2; jj++) {
+            const double2 r2 = __ldg(row + jj);
+#pragma unroll
+            for (int hl = 0; hl < G; hl++) {
+                acc[hl] = fma((double)orot[hl * kD + j0 + 2 * jj], r2.x, acc[hl]);
+                acc[hl] = fma((double)orot[hl * kD + j0 + 2 * jj + 1], r2.y, acc[hl]);
+            }
+        }
+#pragma unroll
+        for (int hl = 0; hl < G; hl++) {
+            if constexpr (P == 2) acc[hl] += __shfl_xor_sync(0xffffffffu, acc[hl], 1);
+            if (t % P == 0) out[(qrow0 + hl) * kD + c] = (float)acc[hl];
         }
     }
     __syncthreads();
@@ -400,7 +438,7 @@ namespace kvq {
 cudaError_t launch_append(const kvq_cache &c, const void *K, const void *V, int dtype, int n_new,
                           const double *A, cudaStream_t st);
 cudaError_t launch_select(const kvq_cache &c, const void *q, int dtype, int Hq, const double *Ainvt,
-                          int k, int32_t *idx, float *qsel, float *qgsum, cudaStream_t st);
+                          const double *delta, int k, int32_t *idx, float *qsel, float *qgsum, cudaStream_t st);
 int decode_splits(const kvq_cache &c, int Hq, int k, int num_sms);
 size_t decode_ws_bytes(const kvq_cache &c, int Hq, int n_splits);
 cudaError_t launch_decode(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
@@ -408,8 +446,8 @@ cudaError_t launch_decode(const kvq_cache &c, int Hq, const int32_t *idx, const 
                           cudaStream_t st);
 cudaError_t launch_decode_step(const kvq_cache &c, int Hq, const void *q, const void *k_new,
                                const void *v_new, int dtype, int n_new, const double *A,
-                               const double *Ainvt, int k, int32_t *idx, float *qsel, float *qgsum,
-                               float *out, void *ws, int n_splits, cudaStream_t st);
+                               const double *Ainvt, const double *delta, int k, int32_t *idx, float *qsel,
+                               float *qgsum, float *out, void *ws, int n_splits, cudaStream_t st);
 // completion counter of unit (b, h) in the cache's status array
 inline uint32_t *unit_counter(const kvq_cache &c, int b, int h) {
     return c.status + 1 + c.batch + (size_t)b * c.n_kv_heads + h;

@@ -4,7 +4,9 @@
 //   §3.1 the query is multiplied by the inverse transpose of the key
 //        transform, so transformed scores equal the original ones;
 //   §3.2 Eq. 4: channel energy pooled over the query heads sharing a KV head,
-//        e_j^2 = sum_h q'_{h,j}^2, one mask per KV head, chosen per query.
+//        e_j^2 = sum_h q'_{h,j}^2, one mask per KV head, chosen per query;
+//   §3.3, App. C.2: with a diagonal refinement D folded into the transforms
+//        the energies are those of the base queries, q'_{h,j} / delta_j.
 // Channel 0 is always kept; ties go to the lower channel index.
 //
 // One thread-block cluster of four CTAs = one (sequence, KV head); CTA r owns
@@ -30,8 +32,8 @@ constexpr int kCtas = kNG;                 // CTAs per cluster, one per key grou
 
 template <typename Tin>
 __global__ void __cluster_dims__(kCtas, 1, 1) __launch_bounds__(kThreads)
-select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, int Hq, int Hkv, int g,
-              int k, int32_t *__restrict__ idx, float *__restrict__ qsel,
+select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, const double *__restrict__ delta,
+              int Hq, int Hkv, int g, int k, int32_t *__restrict__ idx, float *__restrict__ qsel,
               float *__restrict__ qgsum, int ng) {
     extern __shared__ __align__(16) double sm[];   // As[128][32], qin[g][128], qp[g][32]
     double *As = sm;
@@ -68,10 +70,15 @@ select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, int H
         qp[hl * kGroup + lane] = acc;
     }
     __syncthreads();
-    // e_j^2, fma chain over heads ascending from 0.0
+    // e_j^2, fma chain over heads ascending from 0.0; with a diagonal
+    // refinement D, of the base queries q'_{h,j} / delta_j
     if (t < kGroup) {
+        const double dj = delta ? delta[(size_t)h * kD + r * kGroup + t] : 1.0;
         double e = 0.0;
-        for (int hl = 0; hl < g; hl++) e = fma(qp[hl * kGroup + t], qp[hl * kGroup + t], e);
+        for (int hl = 0; hl < g; hl++) {
+            const double u = delta ? qp[hl * kGroup + t] / dj : qp[hl * kGroup + t];
+            e = fma(u, u, e);
+        }
         e2own[t] = e;
     }
     cluster.sync();                                // every CTA's energies are ready
@@ -140,7 +147,7 @@ select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, int H
 }  // namespace
 
 cudaError_t launch_select(const kvq_cache &c, const void *q, int dtype, int Hq, const double *Ainvt,
-                          int k, int32_t *idx, float *qsel, float *qgsum, cudaStream_t st) {
+                          const double *delta, int k, int32_t *idx, float *qsel, float *qgsum, cudaStream_t st) {
     const int g = Hq / c.n_kv_heads;
     const size_t smem = (size_t)(kD * kGroup + g * kD + g * kGroup) * sizeof(double);
     constexpr int kMaxSmem = (kD * kGroup + 32 * kD + 32 * kGroup) * (int)sizeof(double);   // g <= 32
@@ -150,12 +157,12 @@ cudaError_t launch_select(const kvq_cache &c, const void *q, int dtype, int Hq, 
     if (dtype == KVQ_DTYPE_F32) {
         e = set_smem_once(select_kernel<float>, kMaxSmem, done_f32);
         if (e != cudaSuccess) return e;
-        select_kernel<float><<<grid, kThreads, smem, st>>>(static_cast<const float *>(q), Ainvt, Hq,
+        select_kernel<float><<<grid, kThreads, smem, st>>>(static_cast<const float *>(q), Ainvt, delta, Hq,
                                                            c.n_kv_heads, g, k, idx, qsel, qgsum, groups_of(c));
     } else {
         e = set_smem_once(select_kernel<uint16_t>, kMaxSmem, done_bf16);
         if (e != cudaSuccess) return e;
-        select_kernel<uint16_t><<<grid, kThreads, smem, st>>>(static_cast<const uint16_t *>(q), Ainvt, Hq,
+        select_kernel<uint16_t><<<grid, kThreads, smem, st>>>(static_cast<const uint16_t *>(q), Ainvt, delta, Hq,
                                                               c.n_kv_heads, g, k, idx, qsel, qgsum, groups_of(c));
     }
     return cudaGetLastError();

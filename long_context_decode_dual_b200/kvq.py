@@ -6,9 +6,9 @@ is no fallback: if the library is missing, importing it raises.
 
 Names follow the C entry points:
   kvq_append           -> append(cache, K, V, A)
-  kvq_select_channels  -> select_channels(cache, q, Ainvt, sparsity)
+  kvq_select_channels  -> select_channels(cache, q, Ainvt, sparsity, delta=None)
   kvq_decode_attn      -> decode_attn(cache, sel)
-  kvq_decode_step      -> decode_step(cache, q, k_new, v_new, A, Ainvt, sparsity)
+  kvq_decode_step      -> decode_step(cache, q, k_new, v_new, A, Ainvt, sparsity, delta=None)
   kvq_bf16_decode_attn -> bf16_decode_attn(q, K, V)
 """
 from __future__ import annotations
@@ -46,6 +46,7 @@ class CacheDesc(ctypes.Structure):
         ("group", ctypes.c_int32), ("bits", ctypes.c_int32), ("capacity", ctypes.c_int32),
         ("pages", ctypes.c_void_p), ("seq_len", ctypes.c_void_p), ("status", ctypes.c_void_p),
         ("n_sink", ctypes.c_int32), ("n_recent", ctypes.c_int32),
+        ("v_rot", ctypes.c_void_p), ("v_clip", ctypes.c_double),
     ]
 
 
@@ -77,7 +78,7 @@ def lib() -> ctypes.CDLL:
             "kvq_cache_init": (I, [C, P]),
             "kvq_append": (I, [C, P, P, I, I, P, P]),
             "kvq_num_selected": (I, [ctypes.c_float, I]),
-            "kvq_select_channels": (I, [C, P, I, I, P, ctypes.c_float, P, P, P, ctypes.POINTER(I), P]),
+            "kvq_select_channels": (I, [C, P, I, I, P, P, ctypes.c_float, P, P, P, ctypes.POINTER(I), P]),
             "kvq_decode_workspace": (S, [C, I, I]),
             "kvq_decode_attn": (I, [C, I, P, P, P, I, P, P, S, P]),
             "kvq_bf16_decode_workspace": (S, [I, I, I, I]),
@@ -87,7 +88,7 @@ def lib() -> ctypes.CDLL:
             "kvq_version": (I, []),
             "kvq_decode_static_scratch_bytes": (S, []),
             "kvq_decode_attn_static": (I, [C, I, P, P, P, I, P, P]),
-            "kvq_decode_step": (I, [C, P, P, P, I, I, I, P, P, ctypes.c_float, P, P, P, P, P, S, P]),
+            "kvq_decode_step": (I, [C, P, P, P, I, I, I, P, P, P, ctypes.c_float, P, P, P, P, P, S, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -140,12 +141,15 @@ class KVCache:
     n_sink: int = 0           # protected BF16 tier: first tokens kept
     n_recent: int = 0         # and most recent tokens kept
     group: int = GROUP        # channels per quantization group: 32, or 128 (one grid per token)
+    v_rot: Optional[torch.Tensor] = None   # value rotation [Hkv][128][128] f64 (orthogonal), or None
+    v_clip: float = 1.0       # clipping ratio of the value grids
 
     @property
     def desc(self) -> CacheDesc:
         return CacheDesc(self.batch, self.n_kv_heads, HEAD_DIM, self.group, self.bits, self.capacity,
                          self.pages.data_ptr(), self.seq_len.data_ptr(), self.status.data_ptr(),
-                         self.n_sink, self.n_recent)
+                         self.n_sink, self.n_recent, 0 if self.v_rot is None else self.v_rot.data_ptr(),
+                         float(self.v_clip))
 
     @property
     def n_blocks(self) -> int:
@@ -176,8 +180,16 @@ def page_bytes(bits: int, group: int = GROUP) -> int:
 
 
 def new_cache(batch: int, n_kv_heads: int, capacity: int, bits: int = 2,
-              device="cuda", stream=None, n_sink: int = 0, n_recent: int = 0, group: int = GROUP) -> KVCache:
-    desc = CacheDesc(batch, n_kv_heads, HEAD_DIM, group, bits, capacity, 0, 0, 0, n_sink, n_recent)
+              device="cuda", stream=None, n_sink: int = 0, n_recent: int = 0, group: int = GROUP,
+              v_rot: Optional[torch.Tensor] = None, v_clip: float = 1.0) -> KVCache:
+    """A zeroed cache.  ``v_rot`` (device f64 [Hkv][128][128], orthogonal) makes
+    appends store rotated values and decodes rotate their output back;
+    ``v_clip`` clips the value grids (Dual-QK App. B.2 uses 0.92)."""
+    if v_rot is not None:
+        assert v_rot.dtype == torch.float64 and v_rot.is_contiguous()
+        assert tuple(v_rot.shape) == (n_kv_heads, HEAD_DIM, HEAD_DIM)
+    desc = CacheDesc(batch, n_kv_heads, HEAD_DIM, group, bits, capacity, 0, 0, 0, n_sink, n_recent,
+                     None, float(v_clip))
     nbytes = int(lib().kvq_cache_bytes(ctypes.byref(desc)))
     if nbytes == 0:
         raise KvqError("kvq_cache_bytes", -2)
@@ -185,7 +197,8 @@ def new_cache(batch: int, n_kv_heads: int, capacity: int, bits: int = 2,
     seq_len = torch.empty(batch, dtype=torch.int32, device=device)
     status = torch.empty(int(lib().kvq_status_words(batch, n_kv_heads)), dtype=torch.int32,
                          device=device)
-    c = KVCache(batch, n_kv_heads, capacity, bits, pages, seq_len, status, n_sink, n_recent, group)
+    c = KVCache(batch, n_kv_heads, capacity, bits, pages, seq_len, status, n_sink, n_recent, group, v_rot,
+                float(v_clip))
     _check("kvq_cache_init", lib().kvq_cache_init(ctypes.byref(c.desc), _stream(stream)))
     return c
 
@@ -214,9 +227,11 @@ def alloc_selection(cache: KVCache, n_q_heads: int, k: int, device="cuda") -> Se
 
 
 def select_channels(cache: KVCache, q: torch.Tensor, Ainvt: torch.Tensor, sparsity: float,
-                    out: Optional[Selection] = None, stream=None) -> Selection:
-    """kvq_select_channels: q [B][Hq][128] (f32 or bf16), Ainvt [Hkv][128][128] f64."""
+                    out: Optional[Selection] = None, stream=None, delta: Optional[torch.Tensor] = None) -> Selection:
+    """kvq_select_channels: q [B][Hq][128] (f32 or bf16), Ainvt [Hkv][128][128] f64,
+    delta (diagonal refinement folded into Ainvt) [Hkv][128] f64 or None."""
     assert q.is_contiguous() and Ainvt.is_contiguous() and Ainvt.dtype == torch.float64
+    _check_delta(delta)
     Hq = int(q.shape[1])
     k = num_selected(sparsity)
     if k < 0:
@@ -225,10 +240,15 @@ def select_channels(cache: KVCache, q: torch.Tensor, Ainvt: torch.Tensor, sparsi
     assert sel.k == k
     kout = ctypes.c_int(0)
     _check("kvq_select_channels", lib().kvq_select_channels(
-        ctypes.byref(cache.desc), _ptr(q), _dtype_code(q), Hq, _ptr(Ainvt), float(sparsity),
+        ctypes.byref(cache.desc), _ptr(q), _dtype_code(q), Hq, _ptr(Ainvt), _ptr(delta), float(sparsity),
         _ptr(sel.idx), _ptr(sel.qsel), _ptr(sel.qgsum), ctypes.byref(kout), _stream(stream)))
     assert kout.value == k
     return sel
+
+
+def _check_delta(delta: Optional[torch.Tensor]) -> None:
+    if delta is not None:
+        assert delta.dtype == torch.float64 and delta.is_contiguous() and delta.shape[-1] == HEAD_DIM
 
 
 def decode_workspace_bytes(cache: KVCache, n_q_heads: int, k: int) -> int:
@@ -256,11 +276,12 @@ def decode_attn(cache: KVCache, sel: Selection, out: Optional[torch.Tensor] = No
 def decode_step(cache: KVCache, q: torch.Tensor, k_new: Optional[torch.Tensor], v_new: Optional[torch.Tensor],
                 A: torch.Tensor, Ainvt: torch.Tensor, sparsity: float, sel: Optional[Selection] = None,
                 out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
-                stream=None) -> tuple[torch.Tensor, Selection]:
+                stream=None, delta: Optional[torch.Tensor] = None) -> tuple[torch.Tensor, Selection]:
     """kvq_decode_step: append k_new / v_new [B][Hkv][n_new][128], select the
     channels of q [B][Hq][128], decode; returns (out [B][Hq][128] f32, sel)."""
     assert q.is_contiguous() and A.is_contiguous() and Ainvt.is_contiguous()
     assert A.dtype == torch.float64 and Ainvt.dtype == torch.float64
+    _check_delta(delta)
     B, Hq = cache.batch, int(q.shape[1])
     n_new = 0 if k_new is None else int(k_new.shape[2])
     if n_new:
@@ -277,7 +298,7 @@ def decode_step(cache: KVCache, q: torch.Tensor, k_new: Optional[torch.Tensor], 
         ws = alloc_workspace(decode_workspace_bytes(cache, Hq, k), q.device)
     _check("kvq_decode_step", lib().kvq_decode_step(
         ctypes.byref(cache.desc), _ptr(q), _ptr(k_new if n_new else None), _ptr(v_new if n_new else None),
-        _dtype_code(q), Hq, n_new, _ptr(A), _ptr(Ainvt), float(sparsity), _ptr(sel.idx), _ptr(sel.qsel),
+        _dtype_code(q), Hq, n_new, _ptr(A), _ptr(Ainvt), _ptr(delta), float(sparsity), _ptr(sel.idx), _ptr(sel.qsel),
         _ptr(sel.qgsum), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
     return out, sel
 
@@ -346,10 +367,12 @@ class DecodeStep:
     """
 
     def __init__(self, cache: KVCache, A: torch.Tensor, Ainvt: torch.Tensor, sparsity: float,
-                 n_q_heads: int, dtype: torch.dtype = torch.bfloat16, fused: bool = True):
+                 n_q_heads: int, dtype: torch.dtype = torch.bfloat16, fused: bool = True,
+                 delta: Optional[torch.Tensor] = None):
         dev = cache.pages.device
         B, Hkv = cache.batch, cache.n_kv_heads
         self.cache, self.A, self.Ainvt, self.sparsity = cache, A, Ainvt, float(sparsity)
+        self.delta = delta
         self.fused = fused
         self.q = torch.zeros(B, n_q_heads, HEAD_DIM, dtype=dtype, device=dev)
         self.k_new = torch.zeros(B, Hkv, 1, HEAD_DIM, dtype=dtype, device=dev)
@@ -364,12 +387,12 @@ class DecodeStep:
     def _pre(self):
         if not self.fused:
             append(self.cache, self.k_new, self.v_new, self.A)
-            select_channels(self.cache, self.q, self.Ainvt, self.sparsity, out=self.sel)
+            select_channels(self.cache, self.q, self.Ainvt, self.sparsity, out=self.sel, delta=self.delta)
 
     def _decode(self):
         if self.fused:
             decode_step(self.cache, self.q, self.k_new, self.v_new, self.A, self.Ainvt, self.sparsity,
-                        sel=self.sel, out=self.out, ws=self.ws)
+                        sel=self.sel, out=self.out, ws=self.ws, delta=self.delta)
         else:
             decode_attn(self.cache, self.sel, out=self.out, ws=self.ws)
 

@@ -27,14 +27,34 @@ class Case:
     def __init__(self, wl: W.Workload, n_ctx: int | None = None, capacity: int | None = None):
         self.wl = wl if n_ctx is None else wl.with_(n_ctx=n_ctx)
         self.capacity = capacity or self.wl.capacity
-        self.A, self.Ai = W.make_transforms(self.wl)
+        self.A, self.Ai = W.make_transforms(self.wl)      # refinement folded in when the workload has one
+        self.delta = W.make_deltas(self.wl)                # [Hkv][128] or None
+        self.Rv = W.make_value_rotations(self.wl)          # [Hkv][128][128] or None
         self.K, self.V = W.make_kv(self.wl)
         self._oracle_units = {}
+
+    def cache_kw(self) -> dict:
+        """new_cache keywords of the workload's format (group, value rotation, clip)."""
+        return dict(group=self.wl.quant_group, v_rot=None if self.Rv is None else dev64(self.Rv),
+                    v_clip=self.wl.v_clip)
+
+    def dev_delta(self):
+        return None if self.delta is None else dev64(self.delta)
+
+    def delta_of(self, h: int):
+        return None if self.delta is None else self.delta[h]
+
+    def rv_of(self, h: int):
+        return None if self.Rv is None else self.Rv[h]
+
+    def oracle_values(self, Vf: np.ndarray, h: int) -> np.ndarray:
+        """Values as the cache stores them: rotated when the workload rotates them."""
+        return Vf if self.Rv is None else orc.value_rotate(Vf, self.Rv[h])
 
     # ---------------------------------------------------------------- GPU
     def gpu_cache(self, chunks=None) -> kvq.KVCache:
         wl = self.wl
-        cache = kvq.new_cache(wl.batch, wl.n_kv_heads, self.capacity, wl.bits, group=wl.quant_group)
+        cache = kvq.new_cache(wl.batch, wl.n_kv_heads, self.capacity, wl.bits, **self.cache_kw())
         A = dev64(self.A)
         n = self.K.shape[2]
         chunks = chunks or [n]
@@ -58,7 +78,8 @@ class Case:
             Kf = W.as_float(self.K[b, h, :n], wl.dtype)
             Vf = W.as_float(self.V[b, h, :n], wl.dtype)
             u = orc.new_unit(self.capacity, wl.bits, wl.quant_group)
-            orc.append_unit(u, wl.bits, 0, orc.transform(Kf, self.A[h]), Vf, group=wl.quant_group)
+            orc.append_unit(u, wl.bits, 0, orc.transform(Kf, self.A[h]), self.oracle_values(Vf, h),
+                            group=wl.quant_group, vclip=wl.v_clip)
             self._oracle_units[key] = u
         return self._oracle_units[key]
 
@@ -70,7 +91,8 @@ class Case:
     def oracle_decode(self, q: np.ndarray, b: int, h: int, sparsity: float, n: int | None = None):
         n = self.K.shape[2] if n is None else n
         qp = self.oracle_qp(q, b, h)
-        out, idx = orc.decode_unit(self.oracle_unit(b, h), self.wl.bits, n, qp, sparsity, self.wl.quant_group)
+        out, idx = orc.decode_unit(self.oracle_unit(b, h), self.wl.bits, n, qp, sparsity, self.wl.quant_group,
+                                   delta=self.delta_of(h), Rv=self.rv_of(h))
         return out, idx, qp
 
 

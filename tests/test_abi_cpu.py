@@ -30,7 +30,7 @@ def test_every_declared_symbol_is_exported():
 
 def test_host_side_queries():
     L = kvq.lib()
-    assert L.kvq_version() == 100
+    assert L.kvq_version() == 101
     assert L.kvq_page_bytes(2, 32) == 12544 and L.kvq_page_bytes(4, 32) == 20736 and L.kvq_page_bytes(3, 32) == 0
     assert L.kvq_page_bytes(2, 128) == 9472 and L.kvq_page_bytes(4, 128) == 17664 and L.kvq_page_bytes(2, 64) == 0
     for s, k in ((0.0, 128), (0.2, 103), (0.4, 77), (0.6, 52), (0.25, 96)):
@@ -65,12 +65,22 @@ def test_validation_rejects_before_launch():
     assert L.kvq_append(ctypes.byref(ok), 8, 8, 0, 129, 16, None) == -3         # > capacity
     assert L.kvq_append(ctypes.byref(ok), 8, 8, 0, 0, 16, None) == 0            # no-op
     two = kvq.CacheDesc(1, 2, 128, 32, 2, 128, 0x1000, 256, 256)
-    assert L.kvq_select_channels(ctypes.byref(two), 8, 0, 3, 8, ctypes.c_float(0.4), 8, 8, 8,
+    assert L.kvq_select_channels(ctypes.byref(two), 8, 0, 3, 8, None, ctypes.c_float(0.4), 8, 8, 8,
                                  None, None) == -2                              # 3 % 2 heads
-    assert L.kvq_select_channels(ctypes.byref(two), 8, 0, 4, 8, ctypes.c_float(1.5), 8, 8, 8,
+    assert L.kvq_select_channels(ctypes.byref(two), 8, 0, 4, 8, None, ctypes.c_float(1.5), 8, 8, 8,
                                  None, None) == -1                              # sparsity
-    assert L.kvq_select_channels(ctypes.byref(two), 8, 0, 4, 8, ctypes.c_float(0.4), 8, 8, 8,
+    assert L.kvq_select_channels(ctypes.byref(two), 8, 0, 4, 8, None, ctypes.c_float(0.4), 8, 8, 8,
                                  None, None) == -6                              # Ainvt not 16-aligned
+    assert L.kvq_select_channels(ctypes.byref(two), 8, 0, 4, 16, 12, ctypes.c_float(0.4), 8, 8, 8,
+                                 None, None) == -6                              # delta not 8-aligned
+    # value rotation / clip fields of the descriptor
+    rot_mis = kvq.CacheDesc(1, 1, 128, 32, 2, 128, 0x1000, 256, 256, 0, 0, 0x1008, 0.92)
+    assert L.kvq_append(ctypes.byref(rot_mis), 8, 8, 0, 1, 16, None) == -6      # v_rot not 16-aligned
+    for clip in (-0.5, 1.5, float("nan")):
+        bad_clip = kvq.CacheDesc(1, 1, 128, 32, 2, 128, 0x1000, 256, 256, 0, 0, 0x1000, clip)
+        assert L.kvq_append(ctypes.byref(bad_clip), 8, 8, 0, 1, 16, None) == -1
+    ok_rot = kvq.CacheDesc(1, 1, 128, 32, 2, 128, 0x1000, 256, 256, 0, 0, 0x1000, 0.92)
+    assert L.kvq_append(ctypes.byref(ok_rot), 8, 8, 0, 0, 16, None) == 0        # valid, no-op
     assert L.kvq_decode_attn(ctypes.byref(two), 6, 8, 8, 8, 77, 8, 8, 1 << 20, None) == -2  # g = 3
     assert L.kvq_decode_attn(ctypes.byref(two), 4, 8, 8, 8, 0, 8, 8, 1 << 20, None) == -1   # k = 0
     assert L.kvq_bf16_decode_attn(8, 8, 8, 1, 3, 2, 10, 8, 8, 1 << 20, None) == -2

@@ -29,7 +29,7 @@ def _oracle_slots(case: Case, b: int, h: int, n: int, n_sink: int, n_recent: int
     Kf = W.as_float(case.K[b, h, :n], wl.dtype)
     Vf = W.as_float(case.V[b, h, :n], wl.dtype)
     slots = orc.new_slots(n_sink, n_recent)
-    orc.protect_store(slots, n_sink, n_recent, 0, orc.transform(Kf, case.A[h]), Vf, n)
+    orc.protect_store(slots, n_sink, n_recent, 0, orc.transform(Kf, case.A[h]), case.oracle_values(Vf, h), n)
     return slots
 
 
@@ -37,9 +37,9 @@ def _run(case: Case, n0: int, n_new: int, n_steps: int, n_sink: int, n_recent: i
          sparsity: float = 0.4, units=None):
     wl = case.wl
     g = wl.group_size
-    A, Ai = dev64(case.A), dev64(case.Ai)
+    A, Ai, dl = dev64(case.A), dev64(case.Ai), case.dev_delta()
     cache = kvq.new_cache(wl.batch, wl.n_kv_heads, case.capacity, wl.bits, n_sink=n_sink, n_recent=n_recent,
-                          group=wl.quant_group)
+                          **case.cache_kw())
     if n0:
         kvq.append(cache, to_dev(case.K[:, :, :n0], wl.dtype), to_dev(case.V[:, :, :n0], wl.dtype), A)
     pos = n0
@@ -50,10 +50,10 @@ def _run(case: Case, n0: int, n_new: int, n_steps: int, n_sink: int, n_recent: i
         kn = to_dev(case.K[:, :, pos:pos + n_new], wl.dtype)
         vn = to_dev(case.V[:, :, pos:pos + n_new], wl.dtype)
         if fused:
-            out, sel = kvq.decode_step(cache, qd, kn, vn, A, Ai, sparsity)
+            out, sel = kvq.decode_step(cache, qd, kn, vn, A, Ai, sparsity, delta=dl)
         else:
             kvq.append(cache, kn, vn, A)
-            sel = kvq.select_channels(cache, qd, Ai, sparsity)
+            sel = kvq.select_channels(cache, qd, Ai, sparsity, delta=dl)
             out = kvq.decode_attn(cache, sel)
         torch.cuda.synchronize()
         pos += n_new
@@ -63,7 +63,7 @@ def _run(case: Case, n0: int, n_new: int, n_steps: int, n_sink: int, n_recent: i
             slots = _oracle_slots(case, b, h, pos, n_sink, n_recent)
             qp = case.oracle_qp(q, b, h)
             want, ref_idx = orc.decode_unit_protected(unit, slots, wl.bits, pos, qp, sparsity, n_sink, n_recent,
-                                                      wl.quant_group)
+                                                      wl.quant_group, delta=case.delta_of(h), Rv=case.rv_of(h))
             assert np.array_equal(sel.idx[b, h].cpu().numpy(), ref_idx)
             emax, emean = rel_errors(out[b, h * g:(h + 1) * g], want)
             assert emax <= TOL_MAX and emean <= TOL_MEAN, (i, b, h, emax, emean)
