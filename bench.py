@@ -72,8 +72,8 @@ def decode_source_hash() -> str:
 
 def committed_traffic(kernel: str, workload: str):
     """DRAM bytes per launch of `kernel` from a committed ncu summary
-    (profiles/traffic_<kernel>_<workload>.txt), if it was taken on the
-    current kernel source."""
+    (profiles/traffic_<kernel>_<workload>.txt, the workload name carrying its
+    cache format), if it was taken on the current kernel source."""
     try:
         kv = {}
         with open(os.path.join(PROFILES, f"traffic_{kernel}_{workload}.txt")) as f:
@@ -92,9 +92,15 @@ def algorithmic_step_bytes(wl: W.Workload, k: int, length: int, protect=(0, 0)) 
     """Bytes one fused step launch must move: the decode bytes over `length`
     tokens, A^{-T} of every KV head and the A columns the appending CTAs read
     (float64, 128 x 128 each), the query rows and the new token's key and
-    value (bf16 or f32)."""
+    value (bf16 or f32); with a value rotation, its matrix once for the
+    appending CTAs and once per (sequence, KV head) for the merge; with a
+    refinement, its 128 scales per KV head."""
     elem = 2 if wl.dtype == "bf16" else 4
     transforms = 2 * wl.n_kv_heads * 128 * 128 * 8
+    if wl.rotate_values:
+        transforms += (wl.n_kv_heads + wl.batch * wl.n_kv_heads) * 128 * 128 * 8
+    if wl.refine:
+        transforms += wl.n_kv_heads * 128 * 8
     inputs = wl.batch * (wl.n_q_heads + 2 * wl.n_kv_heads) * 128 * elem
     return algorithmic_decode_bytes(wl, k, length, protect) + transforms + inputs
 
@@ -105,7 +111,8 @@ def algorithmic_decode_bytes(wl: W.Workload, k: int, length: int, protect=(0, 0)
     both metadata blocks; with a protected tier (n_sink, n_recent), the pages
     cover only the coded tokens and each protected token adds its k selected
     BF16 key channels and its 128 BF16 values.  The selection inputs and the
-    partial outputs are ignored (< 0.1%)."""
+    partial outputs are ignored (< 0.1%); so is the value rotation's matrix
+    that the merge reads (128 KB per sequence and KV head)."""
     n_sink, n_recent = protect
     R = 128 * wl.bits // 8
     meta = 4 * 128 * (128 // wl.quant_group)            # bytes of one metadata block
@@ -162,17 +169,29 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------ oracle (CPU)
-def oracle_sample(wl: W.Workload, n_steps: int, budget_s: float = 30.0, skip_first: int = 1):
+def oracle_sample(wl: W.Workload, n_steps: int, budget_s: float = 30.0, skip_first: int = 1, protect=(0, 0)):
     """Time the fp64 CPU oracle on a bounded sample of the workload: one
     (sequence 0, KV head 0) unit with the full context, n_steps decode steps
-    (append one token, transform the query and select, attend)."""
+    (append one token, transform the query and select, attend), with the
+    workload's format (group, value rotation and clip, refinement, protected
+    tier)."""
     from oracle import oracle as orc
-    A, Ai = W.make_transform(wl.seed, 0)
+    A, Ai = (x[0] for x in W.make_transforms(wl.with_(n_kv_heads=1)))
+    delta = W.make_deltas(wl.with_(n_kv_heads=1))
+    delta = None if delta is None else delta[0]
+    Rv = W.make_value_rotations(wl.with_(n_kv_heads=1))
+    Rv = None if Rv is None else Rv[0]
+    vals = (lambda v: v) if Rv is None else (lambda v: orc.value_rotate(v, Rv))
+    n_sink, n_recent = protect
     K, V = W.make_kv_unit(wl, 0, 0)
     gq = wl.quant_group
     unit = orc.new_unit(wl.capacity, wl.bits, gq)
-    orc.append_unit(unit, wl.bits, 0, orc.transform(W.as_float(K, wl.dtype), A), W.as_float(V, wl.dtype), group=gq)
+    slots = orc.new_slots(n_sink, n_recent)
+    Kp, Vr = orc.transform(W.as_float(K, wl.dtype), A), vals(W.as_float(V, wl.dtype))
+    orc.append_unit(unit, wl.bits, 0, Kp, Vr, group=gq, vclip=wl.v_clip)
     length = wl.n_ctx
+    if n_sink + n_recent:
+        orc.protect_store(slots, n_sink, n_recent, 0, Kp, Vr, length)
     g = wl.group_size
     times, tokens = [], []
     t_start = time.perf_counter()
@@ -180,11 +199,16 @@ def oracle_sample(wl: W.Workload, n_steps: int, budget_s: float = 30.0, skip_fir
         kn, vn = W.make_step_kv(wl, i)
         q = W.make_q(wl, i)
         t0 = time.perf_counter()
-        orc.append_unit(unit, wl.bits, length, orc.transform(W.as_float(kn[0, 0], wl.dtype), A),
-                        W.as_float(vn[0, 0], wl.dtype), group=gq)
+        kp, vr = orc.transform(W.as_float(kn[0, 0], wl.dtype), A), vals(W.as_float(vn[0, 0], wl.dtype))
+        orc.append_unit(unit, wl.bits, length, kp, vr, group=gq, vclip=wl.v_clip)
         length += 1
         qp = orc.transform(W.as_float(q[0, :g], wl.dtype), Ai)
-        orc.decode_unit(unit, wl.bits, length, qp, wl.sparsity, gq)
+        if n_sink + n_recent:
+            orc.protect_store(slots, n_sink, n_recent, length - 1, kp, vr, length)
+            orc.decode_unit_protected(unit, slots, wl.bits, length, qp, wl.sparsity, n_sink, n_recent, gq,
+                                      delta=delta, Rv=Rv)
+        else:
+            orc.decode_unit(unit, wl.bits, length, qp, wl.sparsity, gq, delta=delta, Rv=Rv)
         times.append(time.perf_counter() - t0)
         tokens.append(length)
         if time.perf_counter() - t_start > budget_s and i >= 1:
@@ -203,18 +227,19 @@ def run_reference(args):
     if rank != 0:
         return 0
     wl = W.workload(args.workload, **({"sparsity": args.sparsity} if args.sparsity is not None else {}),
-                    bits=args.bits, n_steps=args.warmup + args.steps + 1, quant_group=args.group)
+                    bits=args.bits, n_steps=args.warmup + args.steps + 1, **format_overrides(args))
     from oracle import oracle as orc
     k = orc.num_selected(wl.sparsity)
+    protect = protect_of(args)
     value, times, sample = oracle_sample(wl, args.warmup + args.steps, budget_s=1e9,
-                                         skip_first=args.warmup)
+                                         skip_first=args.warmup, protect=protect)
     tokens_per_s = value
     line = {
         "impl": "reference", "metric": METRIC, "value": tokens_per_s, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * statistics.mean(times), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_dict(wl, k),
+        "config": config_dict(wl, k, protect),
         "cpu_baseline": {"value": tokens_per_s, "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": tokens_per_s, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -231,7 +256,36 @@ def config_dict(wl: W.Workload, k: int, protect=(0, 0)):
          "l2": "flushed between steps (256 MiB write, outside the timed events)"}
     if protect != (0, 0):
         d["protected_bf16"] = {"sink": protect[0], "recent": protect[1]}
+    if wl.rotate_values:
+        d["value_rotation"] = {"clip": wl.v_clip}
+    if wl.refine:
+        d["diagonal_refinement"] = True
     return d
+
+
+def format_overrides(args) -> dict:
+    """Workload fields of the cache format the flags ask for."""
+    d = {"quant_group": args.group}
+    if args.rotate_values:
+        d.update(rotate_values=True, v_clip=0.92)
+    if args.refine:
+        d["refine"] = True
+    return d
+
+
+def protect_of(args):
+    return (64, 256) if args.protect else (0, 0)
+
+
+def format_tag(wl: W.Workload, protect=(0, 0)) -> str:
+    """Suffix naming a cache format other than the default (groups of 32,
+    no tier, no rotation, no refinement): the pages' whole recipe is
+    "_pages", anything else lists its parts."""
+    parts = [p for p, on in (("g128", wl.quant_group == 128), ("tier", protect != (0, 0)),
+                             ("rot", wl.rotate_values), ("ref", wl.refine)) if on]
+    if len(parts) == 4:
+        return "_pages"
+    return "_" + "-".join(parts) if parts else ""
 
 
 # ------------------------------------------------------------- ranks
@@ -280,7 +334,7 @@ def run_ours(args):
     n_pool = 8
     total_steps = args.warmup + args.steps
     n_appends = total_steps * (2 if args.e2e else 1) + 1
-    over = {"bits": args.bits, "n_steps": n_appends, "quant_group": args.group}
+    over = {"bits": args.bits, "n_steps": n_appends, **format_overrides(args)}
     if args.sparsity is not None:
         over["sparsity"] = args.sparsity
     wl = rank_workload(W.workload(args.workload, **over), rank)
@@ -301,9 +355,12 @@ def run_ours(args):
     Kd, Vd = dev_in(K_np), dev_in(V_np)
     stream = torch.cuda.current_stream(dev)
 
-    protect = (64, 256) if args.protect else (0, 0)
+    protect = protect_of(args)
+    Rv_np, delta_np = W.make_value_rotations(wl), W.make_deltas(wl)
+    Rv = None if Rv_np is None else torch.from_numpy(Rv_np).to(dev)
+    delta = None if delta_np is None else torch.from_numpy(delta_np).to(dev)
     cache = kvq.new_cache(B, Hkv, wl.capacity, wl.bits, device=dev, n_sink=protect[0], n_recent=protect[1],
-                          group=wl.quant_group)
+                          group=wl.quant_group, v_rot=Rv, v_clip=wl.v_clip)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record()
     kvq.append(cache, Kd, Vd, A)
@@ -316,7 +373,7 @@ def run_ours(args):
     kv_pool = [tuple(dev_in(t) for t in W.make_step_kv(wl, i)) for i in range(n_pool)]
     k = kvq.num_selected(wl.sparsity)
     tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
-    step = kvq.DecodeStep(cache, A, Ai, wl.sparsity, Hq, tdt, fused=args.fused)
+    step = kvq.DecodeStep(cache, A, Ai, wl.sparsity, Hq, tdt, fused=args.fused, delta=delta)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def stage(i):
@@ -374,7 +431,8 @@ def run_ours(args):
     hbm_peak, peak_src = measured_peaks()
     alg_bytes = [alg_fn(wl, k, tok // (B * Hkv), protect) for tok in tokens]
     achieved = statistics.mean(ab / (ms * 1e-3) for ab, ms in zip(alg_bytes, dec_ms)) / 1e9
-    traffic, traffic_note = committed_traffic("step_mma" if args.fused else "decode_mma", wl.name)
+    traffic, traffic_note = committed_traffic("step_mma" if args.fused else "decode_mma",
+                                              wl.name + format_tag(wl, protect))
 
     # end to end through the Python binding with host buffers
     e2e = None
@@ -431,7 +489,7 @@ def run_ours(args):
     # CPU baseline: the oracle on a bounded sample (rank 0, one GPU only)
     cpu = None
     if args.cpu_baseline and world == 1:
-        cv, ct, sample = oracle_sample(wl.with_(n_steps=8), 6, budget_s=25.0)
+        cv, ct, sample = oracle_sample(wl.with_(n_steps=8), 6, budget_s=25.0, protect=protect)
         cpu = {"value": cv, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample}
 
     csum = clocks.summary()
@@ -479,11 +537,19 @@ def main():
                     help="channels per quantization group (128: the pages' one grid per token)")
     ap.add_argument("--protect", action="store_true",
                     help="keep the first 64 and the last 256 tokens in BF16 (the pages' protected tier)")
+    ap.add_argument("--rotate-values", action="store_true",
+                    help="rotate the values before quantization, clip their grids at 0.92, rotate the output back")
+    ap.add_argument("--refine", action="store_true",
+                    help="fold a diagonal refinement into the transforms; select on the base queries")
+    ap.add_argument("--pages-recipe", action="store_true",
+                    help="the pages' whole format: --group 128 --protect --rotate-values --refine")
     ap.add_argument("--unfused", dest="fused", action="store_false",
                     help="run the step as three launches (append, select, decode) instead of one")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="launch the step's kernels eagerly instead of replaying a CUDA graph")
     args = ap.parse_args()
+    if args.pages_recipe:
+        args.group, args.protect, args.rotate_values, args.refine = 128, True, True, True
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
