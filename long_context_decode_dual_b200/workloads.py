@@ -30,6 +30,11 @@ Recipe (every array comes from its own numpy PCG64 stream keyed by
 * value rotation (optional): ``Rv = Q H / sqrt(128)``, ``Q`` a seeded Haar
   orthogonal matrix standing in for the calibrated rotation and ``H`` the
   Sylvester Hadamard matrix of order 128; ``Rv`` is orthogonal.
+* bucket-relative RoPE (optional): buckets of ``bucket`` tokens with anchors
+  ``a_b = b * bucket``; the rotary table holds ``cos`` and ``sin`` of
+  ``a_b * theta_i``, ``theta_i = base^(-2i/128)`` (base 500000, a
+  Llama-3-like model's).  Keys and queries are taken as already rotated by
+  the model's RoPE (the draws above).
 """
 from __future__ import annotations
 
@@ -72,6 +77,8 @@ class Workload:
     refine: bool = False    # diagonal refinement D folded into the transforms
     rotate_values: bool = False
     v_clip: float = 1.0     # value clipping ratio (the pages use 0.92 with rotated values)
+    bucket: int = 0         # tokens per RoPE bucket (the pages use 2048); 0: no buckets
+    rope_base: float = 500000.0
 
     @property
     def group_size(self) -> int:
@@ -209,6 +216,23 @@ def make_transforms(wl: Workload):
         As.append(A)
         Ais.append(Ai)
     return np.ascontiguousarray(np.stack(As)), np.ascontiguousarray(np.stack(Ais))
+
+
+def rope_table(n_buckets: int, w: int, base: float = 500000.0, d: int = HEAD_DIM) -> np.ndarray:
+    """cos and sin of a_b * theta_i for anchors a_b = b * w: float64 [n_buckets][d/2][2]."""
+    theta = base ** (-2.0 * np.arange(d // 2) / d)
+    ang = (np.arange(n_buckets, dtype=np.float64) * w)[:, None] * theta[None, :]
+    return np.ascontiguousarray(np.stack([np.cos(ang), np.sin(ang)], axis=-1))
+
+
+def n_buckets(wl: Workload) -> int:
+    """Buckets that cover the workload's cache capacity (0 without buckets)."""
+    return 0 if not wl.bucket else (wl.capacity + wl.bucket - 1) // wl.bucket
+
+
+def make_rope(wl: Workload) -> Optional[np.ndarray]:
+    """The rotary anchor table of the workload's buckets, or None."""
+    return None if not wl.bucket else rope_table(n_buckets(wl), wl.bucket, wl.rope_base)
 
 
 def make_deltas(wl: Workload) -> Optional[np.ndarray]:

@@ -38,6 +38,14 @@
  *   orc_select_scaled           §3.3 diagonal refinement and App. C.2: with
  *                               A = A0 D, selection uses the base queries
  *                               q A0 = (q A) D^{-1}, scores the final ones.
+ *   orc_rope_unanchor, orc_decode_buckets
+ *                               §3.4 and App. C.4 (bucket-relative RoPE):
+ *                               keys are stored in the frame of their bucket's
+ *                               anchor, z_n = k_n T_b B, the query of bucket b
+ *                               is q T_b A, each bucket has its own channel
+ *                               mask, one softmax over all buckets.  T_b
+ *                               removes the anchor's rotary rotation (rotate-
+ *                               half channel pairs).
  *   value rotation              §3.3 / App. B.2: values are multiplied by an
  *                               orthogonal rotation before quantization
  *                               (orc_transform) and the aggregated output by
@@ -436,6 +444,65 @@ void orc_attention(const double *q, const double *K, const double *V, long n,
     for (int j = 0; j < d; j++) all[j] = j;
     orc_decode_dense(K, V, n, q, g, d, all, d, out);
     free(all);
+}
+
+/* ------------------------------------------------------------------------ */
+/* bucket-relative RoPE                                                      */
+/* ------------------------------------------------------------------------ */
+/* Remove the anchor rotation of a bucket from rows of post-RoPE vectors:
+ * channel i (< d/2) is paired with channel i + d/2 (the rotate-half layout)
+ * and the pair is rotated by the angle -a*theta_i, given as cs[i] =
+ * {cos(a theta_i), sin(a theta_i)}:
+ *   y_i       = x_i cos + x_{i+d/2} sin
+ *   y_{i+d/2} = x_{i+d/2} cos - x_i sin
+ * each product rounded, then the sum or difference (no fused operations).   */
+void orc_rope_unanchor(const double *X, long n, int d, const double *cs, double *Y)
+{
+    const int hd = d / 2;
+    for (long t = 0; t < n; t++) {
+        const double *x = X + t * d;
+        double *y = Y + t * d;
+        for (int i = 0; i < hd; i++) {
+            double c = cs[2 * i], sn = cs[2 * i + 1];
+            double a = x[i], b = x[i + hd];
+            double p1 = a * c, p2 = b * sn, p3 = b * c, p4 = a * sn;
+            y[i] = p1 + p2;
+            y[i + hd] = p3 - p4;
+        }
+    }
+}
+
+/* Decode over buckets of w tokens: token t uses the queries and the channel
+ * list of its bucket t / w (qp: [nb][g][d], idx: [nb][k]); one softmax over
+ * all n tokens per query head, 1/sqrt(d) scaling.  out: [g][d].            */
+void orc_decode_buckets(const double *Khat, const double *Vhat, long n, const double *qp, int g, int d,
+                        const int32_t *idx, int k, long w, double *out)
+{
+    double *sc = (double *)malloc(sizeof(double) * (n > 0 ? n : 1));
+    double inv = 1.0 / sqrt((double)d);
+    for (int h = 0; h < g; h++) {
+        double mx = -INFINITY;
+        for (long t = 0; t < n; t++) {
+            long b = t / w;
+            const double *q = qp + (b * g + h) * (long)d;
+            const int32_t *ix = idx + b * k;
+            double s = 0.0;
+            for (int i = 0; i < k; i++)
+                s += q[ix[i]] * Khat[t * d + ix[i]];
+            sc[t] = s * inv;
+            if (sc[t] > mx) mx = sc[t];
+        }
+        double l = 0.0;
+        double *o = out + (long)h * d;
+        for (int c = 0; c < d; c++) o[c] = 0.0;
+        for (long t = 0; t < n; t++) {
+            double p = exp(sc[t] - mx);
+            l += p;
+            for (int c = 0; c < d; c++) o[c] += p * Vhat[t * d + c];
+        }
+        for (int c = 0; c < d; c++) o[c] = (n > 0) ? o[c] / l : 0.0;
+    }
+    free(sc);
 }
 
 /* ------------------------------------------------------------------------ */

@@ -81,6 +81,8 @@ def _load():
             lib.orc_is_protected.argtypes = [L, L, I, I]
             lib.orc_protect_store.argtypes = [P, I, I, L, L, L, P, P]
             lib.orc_protect_dequant.argtypes = [P, I, I, L, P, P]
+            lib.orc_rope_unanchor.argtypes = [P, L, I, P, P]
+            lib.orc_decode_buckets.argtypes = [P, P, L, P, I, I, P, I, L, P]
             _lib = lib
     return _lib
 
@@ -296,3 +298,66 @@ def decode_unit_protected(unit: np.ndarray, slots: np.ndarray, bits: int, n: int
     _load().orc_protect_dequant(_p(np.ascontiguousarray(slots)), n_sink, n_recent, n, _p(Kh), _p(Vh))
     out = decode_dense(Kh, Vh, qp, idx)
     return (out if Rv is None else value_unrotate(out, Rv)), idx
+
+
+# ------------------------------------------------------ bucket-relative RoPE
+def rope_unanchor(X, cs) -> np.ndarray:
+    """Rows of post-RoPE vectors moved into the frame of a bucket anchor
+    (Dual-QK §3.4, App. C.4): channel pairs (i, i + 64) rotated by -a*theta_i,
+    cs [64][2] = (cos, sin) of a*theta_i."""
+    X = _f64(X)
+    cs = _f64(cs)
+    d = X.shape[-1]
+    assert cs.shape == (d // 2, 2)
+    Y = np.empty_like(X)
+    _load().orc_rope_unanchor(_p(X), X.size // d, d, _p(cs), _p(Y))
+    return Y
+
+
+def bucket_queries(q, Ai, rope, n_buckets: int) -> np.ndarray:
+    """q'_b = (q T_b) A^{-T} for buckets 0..n_buckets-1: [nb][g][d]."""
+    return np.stack([transform(rope_unanchor(q, rope[b]), Ai) for b in range(n_buckets)])
+
+
+def bucket_keys(K, A, rope, w: int, pos0: int = 0) -> np.ndarray:
+    """K' of tokens pos0.. in their buckets' frames, z_n = (k_n T_b) A with
+    b = n // w (§3.4)."""
+    K = _f64(K).reshape(-1, D)
+    out = np.empty_like(K)
+    for i in range(K.shape[0]):
+        out[i] = transform(rope_unanchor(K[i:i + 1], rope[(pos0 + i) // w]), A)[0]
+    return out
+
+
+def decode_buckets(Khat, Vhat, qpb, idxb, w: int) -> np.ndarray:
+    """One softmax over all tokens; token t scored with bucket t // w's
+    queries qpb [nb][g][d] over its channel list idxb [nb][k]."""
+    Khat = _f64(Khat)
+    Vhat = _f64(Vhat)
+    qpb = _f64(qpb)
+    idxb = np.ascontiguousarray(idxb, dtype=np.int32)
+    nb, g, d = qpb.shape
+    n = Khat.shape[0]
+    assert (n + w - 1) // w <= nb and idxb.shape[0] == nb
+    out = np.zeros((g, d))
+    _load().orc_decode_buckets(_p(Khat), _p(Vhat), n, _p(qpb), g, d, _p(idxb), idxb.shape[1], w, _p(out))
+    return out
+
+
+def decode_unit_buckets(unit: np.ndarray, bits: int, n: int, qpb, sparsity: float, w: int, group: int = GROUP,
+                        delta=None, Rv=None, slots=None, n_sink: int = 0, n_recent: int = 0):
+    """Decode with bucket-relative RoPE (§3.4): per bucket b < ceil(n / w),
+    the channel choice on that bucket's queries qpb[b] (base queries with
+    delta), then one softmax over every token with its bucket's queries and
+    channels, the protected tier's BF16 rows in place of their codes, and
+    (with Rv) the inverse value rotation.  Returns (out [g][d], idx [nb][k])
+    for the buckets in use."""
+    k = num_selected(sparsity)
+    nb = max(1, (n + w - 1) // w)
+    qpb = _f64(qpb)[:nb]
+    idxb = np.stack([select(qpb[b], k, delta)[0] for b in range(nb)])
+    Kh, Vh = dequant_unit(unit, bits, n, group)
+    if slots is not None and n_sink + n_recent > 0:
+        _load().orc_protect_dequant(_p(np.ascontiguousarray(slots)), n_sink, n_recent, n, _p(Kh), _p(Vh))
+    out = decode_buckets(Kh, Vh, qpb, idxb, w)
+    return (out if Rv is None else value_unrotate(out, Rv)), idxb
