@@ -48,6 +48,13 @@
  *  (t mod (8/bits))*bits, least significant first.  Key group g is channels
  *  max(1, g group) .. (g+1) group - 1 (channel 0 is kept in bf16 and left out
  *  of the range); value group g is channels g group .. (g+1) group - 1.
+ *  With buckets (cache->bucket = w > 0) the key of position n is stored in
+ *  the frame of its bucket b = n / w (Dual-QK §3.4): its anchor's rotary
+ *  rotation removed, then the key transform, K' = (k T_b) A, where for
+ *  i < 64 (channel i paired with channel i + 64, the rotate-half layout)
+ *      (k T_b)[i]      = k[i] cos_bi + k[i+64] sin_bi
+ *      (k T_b)[i + 64] = k[i+64] cos_bi - k[i] sin_bi
+ *  in float64, each product rounded, then the sum or difference.
  *  Pages of one (sequence b, KV head h) are contiguous; unit (b, h) starts at
  *  byte ((b * n_kv_heads + h) * (capacity / 128)) * page_bytes.
  *  Dequantized value = scale * code + zero.
@@ -135,10 +142,25 @@ typedef struct {
     double v_clip;        /* clipping ratio of the value grids, in (0, 1]
                              (the pages use 0.92 with rotated values); 0 means
                              1, no clipping.  Keys are never clipped.        */
+    int32_t bucket;       /* bucket-relative RoPE (Dual-QK §3.4, App. C.4):
+                             tokens per bucket w, a positive multiple of 128,
+                             or 0 for none.  Bucket b holds positions
+                             [b w, (b+1) w) and has the anchor a_b = b w.   */
+    const double *rope;   /* with buckets: the anchors' rotary table,
+                             [kvq_num_buckets()][64][2] float64 {cos(a_b
+                             theta_i), sin(a_b theta_i)} with the model's
+                             rotary frequencies theta_i (any scaling such as
+                             YaRN included), 16-byte aligned, device memory */
 } kvq_cache;
 
 /* Largest n_sink + n_recent. */
 #define KVQ_MAX_PROTECTED 1024
+
+/* Buckets of a cache: ceil(capacity / bucket), or 1 without buckets (0 if
+ * the descriptor is invalid).  Every channel-selection array has one entry
+ * per bucket: idx [batch][n_kv_heads][nb][k], qsel [batch][n_q_heads][nb][k],
+ * qgsum [batch][n_q_heads][nb][4]. */
+int kvq_num_buckets(const kvq_cache *cache);
 
 /* Words of the cache's status array: 1 + batch + batch * n_kv_heads
  * (0 if an argument is below 1). */
@@ -163,7 +185,8 @@ int kvq_cache_init(const kvq_cache *cache, kvq_stream_t stream);
  * (channel 0 of K' kept as bf16 and excluded from the range; the other key
  * channels and all value channels quantized per token with an asymmetric
  * min/max grid, round to nearest; channel-major 128-token pages), App. B.2
- * (values rotated by cache->v_rot and their grids clipped by cache->v_clip).
+ * (values rotated by cache->v_rot and their grids clipped by cache->v_clip),
+ * §3.4 (with buckets, K' = (K T_b) A in the frame of the token's bucket).
  *
  *  K, V    [batch][n_kv_heads][n_new][128], dtype KVQ_DTYPE_F32 or _BF16
  *  A       [n_kv_heads][128][128] float64, row-major, 16-byte aligned:
@@ -201,7 +224,11 @@ int kvq_num_selected(float sparsity, int head_dim);
  * a positive diagonal D (and A the base key transform times D^{-1}), pass D
  * as delta; the energies are then those of the base queries,
  * u_{h,j} = q'_{h,j} / delta_j (one float64 division), e_j^2 = sum_h u_{h,j}^2,
- * while qsel / qgsum keep q'.
+ * while qsel / qgsum keep q'.  §3.4 (bucket-relative RoPE): with buckets the
+ * choice is made per bucket b that holds a token (b = 0, and b w < seq_len),
+ * on the query moved into the bucket's frame, q'_b = (q T_b) Ainvt (T_b as
+ * for keys), and written to entry b of idx / qsel / qgsum; entries of
+ * buckets beyond the length are not written.
  *
  *  q       [batch][n_q_heads][128], dtype F32 or BF16; query head h belongs
  *          to KV head h / g
@@ -210,10 +237,11 @@ int kvq_num_selected(float sparsity, int head_dim);
  *          (fma chain over c from 0.0), e^2 by an fma chain over h ascending
  *  delta   [n_kv_heads][128] float64 positive finite (NULL: no refinement);
  *          other values give an unspecified but valid channel list
- *  idx     out [batch][n_kv_heads][k] int32: channel 0 and the k-1 channels of
+ *  idx     out [batch][n_kv_heads][nb][k] int32 (nb = kvq_num_buckets(), 1
+ *          without buckets): channel 0 and the k-1 channels of
  *          1..127 with the largest e^2 (ties to the lower index), ascending
- *  qsel    out [batch][n_q_heads][k] float32: q'[h][idx[i]] rounded to fp32
- *  qgsum   out [batch][n_q_heads][4] float32: per key group, the float64 sum
+ *  qsel    out [batch][n_q_heads][nb][k] float32: q'[h][idx[i]] rounded to fp32
+ *  qgsum   out [batch][n_q_heads][nb][4] float32: per key group, the float64 sum
  *          of q'[h][c] over selected c != 0 of that group (ascending c),
  *          rounded to fp32 (the zero-point term of the dequantized dot); with
  *          one grid per token entry 0 holds the one sum and entries 1..3 are 0
@@ -247,7 +275,9 @@ size_t kvq_decode_workspace(const kvq_cache *cache, int n_q_heads, int k);
  *          (zeros for a sequence with no tokens); with cache->v_rot set the
  *          aggregate is rotated back (Dual-QK §3.3), out = o v_rot^T, in
  *          float64 over the 128 channels from the float32 merged sums
- *  idx, qsel, qgsum, k exactly as produced by kvq_select_channels
+ *  idx, qsel, qgsum, k exactly as produced by kvq_select_channels; with
+ *          buckets, token t is scored with the entries of its bucket t / w
+ *          (one softmax over all buckets and tiers, §3.4)
  *  ws      device workspace of at least kvq_decode_workspace() bytes,
  *          16-byte aligned; contents need no initialisation
  *  Arithmetic: float32 accumulation of tensor-core products of exact small
@@ -266,10 +296,11 @@ int kvq_decode_attn(const kvq_cache *cache, int n_q_heads, const int32_t *idx,
  * tokens, kvq_select_channels of the query, then kvq_decode_attn over every
  * token including the new ones.  Same arguments, results and errors as those
  * three calls made in that order on `stream` (idx / qsel / qgsum are written
- * too), and the same stored bits.  With INT2 codes, 4 query heads per KV head
- * and n_new <= 4 the step is one kernel launch: each CTA repeats the channel
- * choice of its (sequence, KV head) with the same float64 arithmetic, and the
- * CTA holding the last page appends the new tokens before reading it.
+ * too), and the same stored bits.  With INT2 codes, 4 query heads per KV head,
+ * n_new <= 4 and no buckets the step is one kernel launch: each CTA repeats
+ * the channel choice of its (sequence, KV head) with the same float64
+ * arithmetic, and the CTA holding the last page appends the new tokens before
+ * reading it.
  *
  *  q       [batch][n_q_heads][128]; k_new, v_new [batch][n_kv_heads][n_new][128];
  *          all of dtype KVQ_DTYPE_F32 or _BF16

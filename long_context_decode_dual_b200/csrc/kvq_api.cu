@@ -17,6 +17,9 @@ int check_cache(const kvq_cache *c) {
     if (c->capacity % kT) return KVQ_ERR_SHAPE;
     if (c->n_sink < 0 || c->n_recent < 0 || c->n_sink + c->n_recent > KVQ_MAX_PROTECTED) return KVQ_ERR_ARG;
     if (!(c->v_clip == 0.0 || (c->v_clip > 0.0 && c->v_clip <= 1.0))) return KVQ_ERR_ARG;
+    if (c->bucket < 0 || c->bucket % kT) return KVQ_ERR_SHAPE;
+    if (c->bucket > 0 && !c->rope) return KVQ_ERR_ARG;
+    if (!aligned(c->rope, 16)) return KVQ_ERR_ALIGN;
     if (!aligned(c->pages, 256) || !aligned(c->seq_len, 4) || !aligned(c->status, 4) || !aligned(c->v_rot, 16))
         return KVQ_ERR_ALIGN;
     return KVQ_OK;
@@ -47,7 +50,7 @@ int check_decode_args(const kvq_cache *c, int Hq, int k) {
 
 extern "C" {
 
-int kvq_version(void) { return 101; }
+int kvq_version(void) { return 102; }
 
 const char *kvq_status_string(int s) {
     switch (s) {
@@ -60,6 +63,11 @@ const char *kvq_status_string(int s) {
         case KVQ_ERR_ALIGN: return "misaligned pointer";
         default: return "unknown status";
     }
+}
+
+int kvq_num_buckets(const kvq_cache *c) {
+    if (!c || c->capacity < 1 || c->bucket < 0 || (c->bucket > 0 && c->bucket % kT)) return 0;
+    return buckets_of(*c);
 }
 
 size_t kvq_status_words(int batch, int n_kv_heads) {

@@ -8,6 +8,10 @@
 //        min/max grid per token; within each 128-token page the codes are
 //        stored channel-major, one channel of one page per 32-byte row.
 //
+// With bucket-relative RoPE (§3.4) each key is first moved into the frame of
+// its bucket's anchor (channel pairs (i, i + 64) rotated back by the anchor's
+// angle, from the caller's rotary table), then transformed.
+//
 // With a value rotation (§3.3, App. B.2: values are rotated before they are
 // quantized, with the grid clipped to [clip*min, clip*max]; keys are not
 // clipped) the values go through the same fixed-order transform as the keys,
@@ -57,7 +61,8 @@ __global__ void __launch_bounds__(128)
 append_kernel(uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len,
               uint32_t *__restrict__ status, const Tin *__restrict__ K,
               const Tin *__restrict__ V, const double *__restrict__ A, const double *__restrict__ Rv,
-              double vclip, int Hkv, int NB, int n_new, int capacity, int n_sink, int n_recent) {
+              double vclip, int Hkv, int NB, int n_new, int capacity, int n_sink, int n_recent,
+              const double *__restrict__ rope, int w) {
     constexpr int R = row_bytes(BITS);
     __shared__ double ks[kTile][kD];
     __shared__ double vs[kTile][kD];
@@ -87,6 +92,20 @@ append_kernel(uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len,
         vs[tt][c] = vv;
     }
     __syncthreads();
+    if (rope) {
+        // k T_b for the bucket of each position (thread j < 64: pair (j, j + 64))
+        if (threadIdx.x < kD / 2) {
+            const double2 *cs = reinterpret_cast<const double2 *>(rope);
+#pragma unroll 4
+            for (int tt = 0; tt < kTile; tt++) {
+                const int pos = first + tt;
+                if (pos < lo || pos >= hi) continue;
+                rope_unanchor_pair(ks[tt][threadIdx.x], ks[tt][threadIdx.x + kD / 2],
+                                   __ldg(cs + (size_t)(pos / w) * (kD / 2) + threadIdx.x));
+            }
+        }
+        __syncthreads();
+    }
 
     const int j = threadIdx.x;          // channel
     const int lane = j & 31;
@@ -214,7 +233,8 @@ __global__ void __launch_bounds__(128)
 append_small_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len,
                     uint32_t *__restrict__ status, const Tin *__restrict__ K,
                     const Tin *__restrict__ V, const double *__restrict__ A, const double *__restrict__ Rv,
-                    double vclip, int Hkv, int NB, int n_new, int capacity, int n_sink, int n_recent) {
+                    double vclip, int Hkv, int NB, int n_new, int capacity, int n_sink, int n_recent,
+                    const double *__restrict__ rope, int w_tok) {
     constexpr int R = row_bytes(BITS);
     constexpr int PER = 8 / BITS;
     static_assert(kSmallMax * 32 == 128, "one warp per new token");
@@ -245,6 +265,15 @@ append_small_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len,
     const int len = s_len;
     const bool ok = len >= 0 && len + n_new <= capacity;
     uint8_t *unit = pages + ((size_t)b * Hkv + h) * NB * (size_t)page_bytes(BITS);
+    if (rope && ok) {
+        // k T_b for the bucket of each new position
+        const double2 *cs = reinterpret_cast<const double2 *>(rope);
+        for (int e = t; e < n_new * (kD / 2); e += 128) {
+            const int i = e / (kD / 2), c = e % (kD / 2);
+            rope_unanchor_pair(ks[i][c], ks[i][c + kD / 2], __ldg(cs + (size_t)((len + i) / w_tok) * (kD / 2) + c));
+        }
+        __syncthreads();
+    }
 
     // K'[t][j] = sum_c K[t][c] A[c][j], fma chain c = 0..127 from 0.0
     double x = 0.0;
@@ -335,6 +364,7 @@ cudaError_t launch_append_t(const kvq_cache &c, const void *K, const void *V, in
                             const double *A, cudaStream_t st) {
     const double *Rv = c.v_rot;
     const double vclip = value_clip(c);
+    const double *rope = c.bucket > 0 ? c.rope : nullptr;
     const int NB = c.capacity / kT;
     // a few tokens with groups of 32: one CTA per group; otherwise (prefill,
     // or one grid per token) the tile kernel and the length advance
@@ -342,13 +372,15 @@ cudaError_t launch_append_t(const kvq_cache &c, const void *K, const void *V, in
         dim3 grid((unsigned)kNG, (unsigned)c.n_kv_heads, (unsigned)c.batch);
         append_small_kernel<Tin, BITS><<<grid, 128, 0, st>>>(
             static_cast<uint8_t *>(c.pages), c.seq_len, c.status, static_cast<const Tin *>(K),
-            static_cast<const Tin *>(V), A, Rv, vclip, c.n_kv_heads, NB, n_new, c.capacity, c.n_sink, c.n_recent);
+            static_cast<const Tin *>(V), A, Rv, vclip, c.n_kv_heads, NB, n_new, c.capacity, c.n_sink, c.n_recent,
+            rope, c.bucket);
         return cudaGetLastError();
     }
     dim3 grid((unsigned)((n_new + kTile - 1) / kTile + 1), (unsigned)c.n_kv_heads, (unsigned)c.batch);
     append_kernel<Tin, BITS, NG><<<grid, 128, 0, st>>>(
         static_cast<uint8_t *>(c.pages), c.seq_len, c.status, static_cast<const Tin *>(K),
-        static_cast<const Tin *>(V), A, Rv, vclip, c.n_kv_heads, NB, n_new, c.capacity, c.n_sink, c.n_recent);
+        static_cast<const Tin *>(V), A, Rv, vclip, c.n_kv_heads, NB, n_new, c.capacity, c.n_sink, c.n_recent,
+        rope, c.bucket);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     advance_kernel<<<(c.batch + 127) / 128, 128, 0, st>>>(c.seq_len, c.batch, n_new, c.capacity);

@@ -59,12 +59,13 @@ cudaError_t launch_decode(const kvq_cache &c, int Hq, const int32_t *idx, const 
 }
 
 // One decode step.  The tensor-core shape with at most step_mma_max_new() new
-// tokens runs as one fused launch; any other shape as the three calls.
+// tokens and no RoPE buckets runs as one fused launch; anything else as the
+// three calls.
 cudaError_t launch_decode_step(const kvq_cache &c, int Hq, const void *q, const void *k_new,
                                const void *v_new, int dtype, int n_new, const double *A,
                                const double *Ainvt, const double *delta, int k, int32_t *idx, float *qsel,
                                float *qgsum, float *out, void *ws, int S, cudaStream_t st) {
-    if (use_mma(c, Hq) && n_new <= step_mma_max_new()) {
+    if (use_mma(c, Hq) && n_new <= step_mma_max_new() && c.bucket == 0) {
         float *part_o = static_cast<float *>(ws);
         float2 *part_ml = reinterpret_cast<float2 *>(part_o + (size_t)c.batch * Hq * S * kD);
         return launch_step_mma(c, Hq, q, k_new, v_new, dtype, n_new, A, Ainvt, delta, k, idx, qsel, qgsum,

@@ -327,24 +327,32 @@ __device__ __forceinline__ void issue_keys(MmaShared &sh, int pair, int st, cons
 // `pair` taking every kPairs-th; tokens outside [lo, hi) (beyond the length,
 // or in the protected tier) are left out of the softmax.  `first_issued`: the pair's first page is
 // already in flight, whole, into stage 0 (one copy that arrives on the
-// barrier).
-template <int NG>
+// barrier).  With RoPE buckets of w_pages pages the split runs as segments,
+// one per bucket: before each, every warp is done with the previous one and
+// load_seg(bucket) puts that bucket's channel choice and page plan in place
+// (called by every thread; it ends with a barrier); the softmax state runs on
+// across segments.  w_pages = 0: one segment, the plan already in place.
+template <int NG, typename SegFn>
 __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restrict__ unit_pages, int lo, int hi,
                                           Split sp, int S, int s, size_t qrow0, float *__restrict__ part_o,
                                           float2 *__restrict__ part_ml, float *__restrict__ out,
                                           uint32_t *counter, uint32_t *status, bool first_issued,
-                                          const double *rot) {
+                                          const double *rot, int w_pages, SegFn &&load_seg) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int pair = warp >> 1, half = warp & 1;
     const int gid = lane >> 2, tig = lane & 3;
     const int hh = gid >> 1, part = gid & 1;
 
     // zero-point and channel-0 coefficients of head tig, pre-scaled to the
-    // base-2 score domain
+    // base-2 score domain (reloaded for each bucket's segment)
     float qg_t[NG];
+    float q0_t = 0.f;
+    auto load_coef = [&]() {
 #pragma unroll
-    for (int g = 0; g < NG; g++) qg_t[g] = sh.qg[tig][g] * kScoreScaleLog2;
-    const float q0_t = sh.q[tig][0] * kScoreScaleLog2;
+        for (int g = 0; g < NG; g++) qg_t[g] = sh.qg[tig][g] * kScoreScaleLog2;
+        q0_t = sh.q[tig][0] * kScoreScaleLog2;
+    };
+    load_coef();
 
     float m_run = -INFINITY;      // running max of head tig (base-2 domain)
     float l_thr = 0.f;            // this thread's share of the running sum of head tig
@@ -362,23 +370,30 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
     const float zmask = gid < NG ? 1.f : 0.f;                // z-term rows: one per group
     uint4 *pexw = &sh.pex[warp][0][0];
 
-    int it = 0;
+    int it = 0;                   // pages this pair has staged (the ring position, across segments)
     uint32_t late = 0;            // stages whose last wait gave up, with the parity waited for
     const bool issuer = (tid & 63) == 0;
-    const int first = sp.blk0 + pair;
-    if (issuer && first < sp.blk1 && !first_issued) {
-        const uint8_t *src = unit_pages + (size_t)first * page_bytes(2, NG);
-        issue_tail<NG>(sh, pair, 0, src);
-        issue_keys(sh, pair, 0, src);
+    for (int seg0 = sp.blk0; seg0 < sp.blk1;) {
+    const int seg1 = w_pages > 0 ? min(sp.blk1, (seg0 / w_pages + 1) * w_pages) : sp.blk1;
+    if (w_pages > 0) {
+        __syncthreads();                                     // every warp is done with the last plan
+        load_seg(seg0 / w_pages);
+        load_coef();
     }
-    for (int pg = first; pg < sp.blk1; pg += kPairs, it++) {
+    const int first = seg0 + pair;
+    if (issuer && first < seg1 && !(first_issued && seg0 == sp.blk0)) {
+        const uint8_t *src = unit_pages + (size_t)first * page_bytes(2, NG);
+        issue_tail<NG>(sh, pair, it & 1, src);
+        issue_keys(sh, pair, it & 1, src);
+    }
+    for (int pg = first; pg < seg1; pg += kPairs, it++) {
         const int st = it & 1;
         const uint8_t *cur = sh.stage[pair][st];
         const uint32_t par = (uint32_t)(it >> 1) & 1u;
         late = mbar_wait_bounded(smem_u32(&sh.mbar[pair][st]), par, status)
                    ? late & ~(3u << (2 * st)) : (late & ~(3u << (2 * st))) | ((2u | par) << (2 * st));
         pair_sync(pair);                                     // both warps left the other stage
-        if (issuer && pg + kPairs < sp.blk1) {
+        if (issuer && pg + kPairs < seg1) {
             const uint8_t *src = unit_pages + (size_t)(pg + kPairs) * page_bytes(2, NG);
             issue_tail<NG>(sh, pair, st ^ 1, src);
             issue_keys(sh, pair, st ^ 1, src);
@@ -590,6 +605,8 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
             }
         }
     }
+    seg0 = seg1;
+    }
     // a stage whose wait gave up may still receive bytes: wait once more
     // (bounded) before the staging memory is reused below
 #pragma unroll
@@ -645,29 +662,42 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
 }
 
 // A CTA that handles the protected tier instead of pages: half `half_idx` of
-// the unit's slots, then the split merge.  Needs the channel choice in
-// sh.chan_pos / sh.q (a barrier after their last write).
+// the unit's slots, then the split merge.  The query coefficients and channel
+// lists come from `qs` (a TierQShared or TierQBuckets).
+template <typename QS>
+__device__ __forceinline__ void tier_cta_q(MmaShared &sh, const uint8_t *slots, int len, int n_sink, int n_recent,
+                                           int half_idx, int k, const QS &qs, float *part_o, float2 *part_ml,
+                                           size_t qrow0, int S, int s, float *out, uint32_t *counter,
+                                           const double *rot) {
+    float *scratch = reinterpret_cast<float *>(sh.stage[0][0] + kD * sizeof(int));
+    static_assert(kD * sizeof(int) + tier_scratch_floats(4) * 4 <= 2 * (size_t)kStageBytes * 2,
+                  "tier scratch ends before the merge scratch in stages 2-3");
+    const int NP = n_sink + n_recent, per = (NP + 1) / 2;
+    const int slot0 = min(NP, half_idx * per), slot1 = min(NP, slot0 + per);
+    tier_partial<4, kThreads>(slots, len, n_sink, n_recent, slot0, slot1, qs, k, part_o, part_ml, qrow0, S, s,
+                              scratch);
+    merge_unit_if_last<4, kThreads>(part_o, part_ml, S, qrow0, out, counter, reinterpret_cast<float *>(sh.stage[2][0]),
+                                    rot);
+}
+// The same with the one channel choice in sh.chan_pos / sh.q (a barrier after
+// their last write).
 __device__ __forceinline__ void tier_cta(MmaShared &sh, const uint8_t *slots, int len, int n_sink, int n_recent,
                                          int half_idx, int k, float *part_o, float2 *part_ml, size_t qrow0, int S,
                                          int s, float *out, uint32_t *counter, const double *rot) {
     int *list = reinterpret_cast<int *>(sh.stage[0][0]);                    // position -> channel
-    float *scratch = reinterpret_cast<float *>(sh.stage[0][0] + kD * sizeof(int));
-    static_assert(kD * sizeof(int) + tier_scratch_floats(4) * 4 <= 2 * (size_t)kStageBytes * 2,
-                  "tier scratch ends before the merge scratch in stages 2-3");
     const int tid = threadIdx.x;
     if (tid < kD) list[tid] = 0;
     __syncthreads();
     if (tid < kD && sh.chan_pos[tid] >= 0) list[sh.chan_pos[tid]] = tid;
     __syncthreads();
-    const int NP = n_sink + n_recent, per = (NP + 1) / 2;
-    const int slot0 = min(NP, half_idx * per), slot1 = min(NP, slot0 + per);
-    tier_partial<4, kThreads>(slots, len, n_sink, n_recent, slot0, slot1, &sh.q[0][0], kD, 1, list, k, part_o,
-                              part_ml, qrow0, S, s, scratch);
-    merge_unit_if_last<4, kThreads>(part_o, part_ml, S, qrow0, out, counter, reinterpret_cast<float *>(sh.stage[2][0]),
-                                    rot);
+    tier_cta_q(sh, slots, len, n_sink, n_recent, half_idx, k, TierQShared{&sh.q[0][0], kD, 1, list}, part_o,
+               part_ml, qrow0, S, s, out, counter, rot);
 }
 
 // ---------------------------------------------------------------- decode
+// With RoPE buckets (w_pages > 0 pages each, nbk entries per selection
+// array) each split reads, per bucket its pages fall in, that bucket's
+// channel choice; the tier CTAs read each protected position's own bucket's.
 template <int NG>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len, int Hkv,
@@ -675,7 +705,7 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
                   const float *__restrict__ qgsum, int k, float *__restrict__ part_o,
                   float2 *__restrict__ part_ml, int S, float *__restrict__ out,
                   uint32_t *__restrict__ counters, uint32_t *__restrict__ status, int n_sink, int n_recent,
-                  const double *__restrict__ v_rot) {
+                  const double *__restrict__ v_rot, int nbk, int w_pages) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     MmaShared &sh = *reinterpret_cast<MmaShared *>(smem_raw);
 
@@ -685,39 +715,52 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
     const size_t unit = (size_t)b * Hkv + h;
     const size_t qrow0 = (size_t)b * Hq + (size_t)h * 4;
 
-    for (int e = tid; e < 4 * k; e += kThreads) {
-        const int hl = e / k, i = e % k;
-        sh.q[hl][i] = qsel[(qrow0 + hl) * k + i];
-    }
-    if (tid < 4 * kNG) sh.qg[tid / kNG][tid % kNG] = qgsum[qrow0 * kNG + tid];
-    if (tid < kD) sh.chan_pos[tid] = -1;
-    if (tid < 2 * kPairs) mbar_init(smem_u32(&sh.mbar[tid >> 1][tid & 1]), 1);
-    // the list must be channel 0 followed by ascending channels in 1..127;
-    // any other list reads no key rows and raises KVQ_DEV_INDEX
-    const int32_t *sel = idx + unit * k;
-    int my_c = -1;
-    bool bad = false;
-    if (tid < k) {
-        my_c = sel[tid];
-        bad = (tid == 0) ? my_c != 0 : (my_c <= sel[tid - 1] || my_c > kD - 1);
-    }
-    const bool any_bad = __syncthreads_or(bad);
-    if (any_bad && tid == 0) atomicOr(status, (uint32_t)KVQ_DEV_INDEX);
-    if (!any_bad && tid < k) sh.chan_pos[my_c] = tid;
-    __syncthreads();
-    build_plan<NG>(sh, tid, warp, lane);
+    // channel choice of bucket bk into shared memory, then the page plan.
+    // The list must be channel 0 followed by ascending channels in 1..127;
+    // any other list reads no key rows and raises KVQ_DEV_INDEX.
+    auto load_sel = [&](int bk) {
+        for (int e = tid; e < 4 * k; e += kThreads) {
+            const int hl = e / k, i = e % k;
+            sh.q[hl][i] = qsel[((qrow0 + hl) * nbk + bk) * k + i];
+        }
+        if (tid < 4 * kNG) sh.qg[tid / kNG][tid % kNG] = qgsum[((qrow0 + tid / kNG) * nbk + bk) * kNG + tid % kNG];
+        if (tid < kD) sh.chan_pos[tid] = -1;
+        const int32_t *sel = idx + (unit * nbk + bk) * k;
+        int my_c = -1;
+        bool bad = false;
+        if (tid < k) {
+            my_c = sel[tid];
+            bad = (tid == 0) ? my_c != 0 : (my_c <= sel[tid - 1] || my_c > kD - 1);
+        }
+        const bool any_bad = __syncthreads_or(bad);
+        if (any_bad && tid == 0) atomicOr(status, (uint32_t)KVQ_DEV_INDEX);
+        if (!any_bad && tid < k) sh.chan_pos[my_c] = tid;
+        __syncthreads();
+        build_plan<NG>(sh, tid, warp, lane);
+    };
 
+    if (tid < 2 * kPairs) mbar_init(smem_u32(&sh.mbar[tid >> 1][tid & 1]), 1);
     const int len = min(max(seq_len[b], 0), NB * kT);
     const int S_pages = S - ((n_sink + n_recent > 0) ? 2 : 0);   // the last two splits take the tier
+    uint8_t *slots = unit_slots(const_cast<uint8_t *>(pages), gridDim.z, Hkv, NB, 2, unit, n_sink + n_recent, NG);
     if (s >= S_pages) {
-        tier_cta(sh, unit_slots(const_cast<uint8_t *>(pages), gridDim.z, Hkv, NB, 2, unit, n_sink + n_recent, NG),
-                 len, n_sink, n_recent, s - S_pages, k, part_o, part_ml, qrow0, S, s, out, counters + unit, rot);
+        if (w_pages > 0) {
+            __syncthreads();
+            tier_cta_q(sh, slots, len, n_sink, n_recent, s - S_pages, k,
+                       TierQBuckets{qsel, idx + unit * nbk * k, k, nbk, w_pages * kT, qrow0}, part_o, part_ml,
+                       qrow0, S, s, out, counters + unit, rot);
+        } else {
+            load_sel(0);
+            tier_cta(sh, slots, len, n_sink, n_recent, s - S_pages, k, part_o, part_ml, qrow0, S, s, out,
+                     counters + unit, rot);
+        }
         return;
     }
+    if (w_pages == 0) load_sel(0);
     const Tier tr = tier_of(len, n_sink, n_recent);
     run_pages<NG>(sh, pages + unit * NB * (size_t)page_bytes(2, NG), tr.sink_end, tr.recent_start,
                   split_of(tr.recent_start, S_pages, s), S, s, qrow0, part_o, part_ml, out, counters + unit, status,
-                  false, rot);
+                  false, rot, w_pages, load_sel);
 }
 
 // ---------------------------------------------------------------- fused step
@@ -1044,7 +1087,7 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
                  part_ml, qrow0, S, s, out, status + 1 + B + unit, rot);
     else
         run_pages<NG>(sh, unit_pages, tr.sink_end, tr.recent_start, sp, S, s, qrow0, part_o, part_ml, out,
-                      status + 1 + B + unit, status, false, rot);
+                      status + 1 + B + unit, status, false, rot, 0, [](int) {});
     cluster_wait();            // the other CTA no longer reads this CTA's shared memory
 }
 
@@ -1077,7 +1120,8 @@ cudaError_t launch_decode_mma_t(const kvq_cache &c, int Hq, const int32_t *idx, 
     decode_mma_kernel<NG><<<grid, kThreads, smem, st>>>(static_cast<const uint8_t *>(c.pages), c.seq_len,
                                                         c.n_kv_heads, c.capacity / kT, Hq, idx, qsel, qgsum, k,
                                                         part_o, part_ml, S, out, unit_counter(c, 0, 0), c.status,
-                                                        c.n_sink, c.n_recent, c.v_rot);
+                                                        c.n_sink, c.n_recent, c.v_rot, buckets_of(c),
+                                                        c.bucket / kT);
     return cudaGetLastError();
 }
 

@@ -51,7 +51,7 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
                    const float *__restrict__ qgsum, int k, float *__restrict__ part_o,
                    float2 *__restrict__ part_ml, int S, float *__restrict__ out,
                    uint32_t *__restrict__ counters, uint32_t *__restrict__ status, int n_sink, int n_recent,
-                   int stage_area, const double *__restrict__ v_rot) {
+                   int stage_area, const double *__restrict__ v_rot, int nbk, int w_pages) {
     constexpr int R = row_bytes(BITS);
     constexpr int FIX = fixed_bytes(BITS, NG);
     constexpr int GS = kD / NG;                       // channels per quantization group
@@ -73,34 +73,39 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
     int *sgs = reinterpret_cast<int *>(sred + 4 * G);
 
     const size_t unit = (size_t)b * Hkv + h;
-    // the list must be channel 0 followed by ascending channels in 1..127;
-    // another list is clamped into the page and raises KVQ_DEV_INDEX
-    bool bad = false;
-    for (int i = tid; i < k; i += 128) {
-        const int c = idx[unit * k + i];
-        bad |= (i == 0) ? c != 0 : (c <= idx[unit * k + i - 1] || c > kD - 1);
-        sidx[i] = min(max(c, 0), kD - 1);
-    }
-    for (int e = tid; e < G * k; e += 128) {
-        const int hl = e / k, i = e % k;
-        sq[i * G + hl] = qsel[((size_t)b * Hq + (size_t)h * G + hl) * k + i];
-    }
-    if (tid < G * kNG) {
-        const int hl = tid / kNG, gr = tid % kNG;
-        sqg[gr * G + hl] = qgsum[((size_t)b * Hq + (size_t)h * G + hl) * kNG + gr];
-    }
-    if (__syncthreads_or(bad) && tid == 0) atomicOr(status, (uint32_t)KVQ_DEV_INDEX);
-    if (tid == 0) {
-        // selected list positions 1..k-1 hold channels >= 1 ascending; group
-        // gr spans positions [sgs[gr], sgs[gr+1])
-        int i = 1;
-        for (int gr = 0; gr < NG; gr++) {
-            sgs[gr] = i;
-            while (i < k && sidx[i] < (gr + 1) * GS) i++;
+    const size_t qrow0 = (size_t)b * Hq + (size_t)h * G;
+    // channel choice of bucket bk (0 without RoPE buckets) into shared memory.
+    // The list must be channel 0 followed by ascending channels in 1..127;
+    // another list is clamped into the page and raises KVQ_DEV_INDEX.
+    auto load_sel = [&](int bk) {
+        const int32_t *sel = idx + (unit * nbk + bk) * k;
+        bool bad = false;
+        for (int i = tid; i < k; i += 128) {
+            const int c = sel[i];
+            bad |= (i == 0) ? c != 0 : (c <= sel[i - 1] || c > kD - 1);
+            sidx[i] = min(max(c, 0), kD - 1);
         }
-        sgs[NG] = k;
-    }
-    __syncthreads();
+        for (int e = tid; e < G * k; e += 128) {
+            const int hl = e / k, i = e % k;
+            sq[i * G + hl] = qsel[((qrow0 + hl) * nbk + bk) * k + i];
+        }
+        if (tid < G * kNG) {
+            const int hl = tid / kNG, gr = tid % kNG;
+            sqg[gr * G + hl] = qgsum[((qrow0 + hl) * nbk + bk) * kNG + gr];
+        }
+        if (__syncthreads_or(bad) && tid == 0) atomicOr(status, (uint32_t)KVQ_DEV_INDEX);
+        if (tid == 0) {
+            // selected list positions 1..k-1 hold channels >= 1 ascending; group
+            // gr spans positions [sgs[gr], sgs[gr+1])
+            int i = 1;
+            for (int gr = 0; gr < NG; gr++) {
+                sgs[gr] = i;
+                while (i < k && sidx[i] < (gr + 1) * GS) i++;
+            }
+            sgs[NG] = k;
+        }
+        __syncthreads();
+    };
 
     // a caller-owned length outside [0, capacity] is clamped, never followed
     const int len = min(max(seq_len[b], 0), NB * kT);
@@ -108,13 +113,19 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
     // pages cover the coded tokens [lo, hi)
     const int NPt = n_sink + n_recent;
     const int S_pages = S - (NPt > 0 ? 2 : 0);
-    const size_t qrow0 = (size_t)b * Hq + (size_t)h * G;
     if (s >= S_pages) {
         const int per = (NPt + 1) / 2;
         const int slot0 = min(NPt, (s - S_pages) * per), slot1 = min(NPt, slot0 + per);
-        tier_partial<G, 128>(unit_slots(const_cast<uint8_t *>(pages), gridDim.z, Hkv, NB, BITS, unit, NPt, NG), len,
-                             n_sink, n_recent, slot0, slot1, sq, 1, G, sidx, k, part_o, part_ml, qrow0, S, s,
-                             reinterpret_cast<float *>(smem));
+        const uint8_t *slots = unit_slots(const_cast<uint8_t *>(pages), gridDim.z, Hkv, NB, BITS, unit, NPt, NG);
+        if (w_pages > 0) {
+            tier_partial<G, 128>(slots, len, n_sink, n_recent, slot0, slot1,
+                                 TierQBuckets{qsel, idx + unit * nbk * k, k, nbk, w_pages * kT, qrow0}, k, part_o,
+                                 part_ml, qrow0, S, s, reinterpret_cast<float *>(smem));
+        } else {
+            load_sel(0);
+            tier_partial<G, 128>(slots, len, n_sink, n_recent, slot0, slot1, TierQShared{sq, 1, G, sidx}, k, part_o,
+                                 part_ml, qrow0, S, s, reinterpret_cast<float *>(smem));
+        }
         merge_unit_if_last<G, 128>(part_o, part_ml, S, qrow0, out, counters + unit, reinterpret_cast<float *>(smem),
                                    v_rot ? v_rot + (size_t)h * kD * kD : nullptr);
         return;
@@ -146,11 +157,17 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
         o_acc[hl] = 0.f;
     }
 
-    if (blk0 < blk1) load(stage[0], blk0);
-    for (int blk = blk0; blk < blk1; blk++) {
-        uint8_t *cur = stage[(blk - blk0) & 1];
-        if (blk + 1 < blk1) {
-            load(stage[(blk - blk0 + 1) & 1], blk + 1);
+    // pages [blk0, blk1) as segments, one per RoPE bucket (one segment
+    // without buckets); the softmax state runs on across segments
+    if (w_pages == 0) load_sel(0);
+    for (int seg0 = blk0; seg0 < blk1;) {
+    const int seg1 = w_pages > 0 ? min(blk1, (seg0 / w_pages + 1) * w_pages) : blk1;
+    if (w_pages > 0) load_sel(seg0 / w_pages);      // the last page's barrier has passed
+    load(stage[0], seg0);
+    for (int blk = seg0; blk < seg1; blk++) {
+        uint8_t *cur = stage[(blk - seg0) & 1];
+        if (blk + 1 < seg1) {
+            load(stage[(blk - seg0 + 1) & 1], blk + 1);
             cp_async_wait<1>();
         } else {
             cp_async_wait<0>();
@@ -231,6 +248,8 @@ decode_simt_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict_
         }
         __syncthreads();
     }
+    seg0 = seg1;
+    }
 
     // partial result of this split (an empty split reports m = -inf, l = 0)
 #pragma unroll
@@ -266,7 +285,8 @@ cudaError_t launch_simt_t(const kvq_cache &c, int Hq, const int32_t *idx, const 
     dim3 grid((unsigned)S, (unsigned)c.n_kv_heads, (unsigned)c.batch);
     fn<<<grid, 128, smem, st>>>(static_cast<const uint8_t *>(c.pages), c.seq_len, c.n_kv_heads,
                                 c.capacity / kT, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out,
-                                unit_counter(c, 0, 0), c.status, c.n_sink, c.n_recent, stage_area, c.v_rot);
+                                unit_counter(c, 0, 0), c.status, c.n_sink, c.n_recent, stage_area, c.v_rot,
+                                buckets_of(c), c.bucket / kT);
     return cudaGetLastError();
 }
 

@@ -40,6 +40,19 @@ __host__ __device__ constexpr int fixed_bytes(int bits, int ng = kNG) { return p
 inline int groups_of(const kvq_cache &c) { return kD / c.group; }
 // clipping ratio of the value grids (0 in the descriptor: none)
 inline double value_clip(const kvq_cache &c) { return c.v_clip == 0.0 ? 1.0 : c.v_clip; }
+// RoPE buckets of a cache (1 without buckets): entries of every selection array
+inline int buckets_of(const kvq_cache &c) { return c.bucket > 0 ? (c.capacity + c.bucket - 1) / c.bucket : 1; }
+
+// Bucket-relative RoPE (Dual-QK §3.4): move channel pair (x_i, x_{i+64}) of a
+// post-RoPE vector into the frame of a bucket anchor, i.e. rotate it by
+// -a*theta_i given cs = {cos, sin} of a*theta_i; each product rounded, then
+// the sum or difference (no contraction), the definition both the library
+// and its tests use.
+__device__ __forceinline__ void rope_unanchor_pair(double &xi, double &xj, double2 cs) {
+    const double a = xi, b = xj;
+    xi = __dadd_rn(__dmul_rn(a, cs.x), __dmul_rn(b, cs.y));
+    xj = __dsub_rn(__dmul_rn(b, cs.x), __dmul_rn(a, cs.y));
+}
 
 // ------------------------------------------------------------ protected tier
 // slot of the protected BF16 tier: 128 bf16 of K' then 128 bf16 of V
@@ -335,9 +348,29 @@ constexpr int kTierChunk = 32;
 __host__ __device__ constexpr int tier_scratch_floats(int G) {
     return kD * (kTierChunk + 1) + kTierChunk * kD + G * kTierChunk + 4 * G;
 }
-template <int G, int NT>
+// Where the tier's scores take the query coefficients and the channel list
+// of a protected position p: one selection in shared memory (q'[head hl] of
+// list position i at q[hl * hs + i * ps]), or -- with RoPE buckets -- the
+// selection arrays of p's bucket in global memory (list entries clamped into
+// 0..127).
+struct TierQShared {
+    const float *q;
+    int hs, ps;
+    const int *chan;
+    __device__ float q_at(int hl, int i, int) const { return q[hl * hs + i * ps]; }
+    __device__ int ch(int i, int) const { return chan[i]; }
+};
+struct TierQBuckets {
+    const float *qsel;             // [..][nb][k] rows of this unit's heads from qrow0
+    const int32_t *idx;            // [nb][k] of this unit
+    int k, nb, w;
+    size_t qrow0;
+    __device__ float q_at(int hl, int i, int p) const { return __ldg(qsel + ((qrow0 + hl) * nb + p / w) * k + i); }
+    __device__ int ch(int i, int p) const { return min(max(__ldg(idx + (size_t)(p / w) * k + i), 0), kD - 1); }
+};
+template <int G, int NT, typename QS>
 __device__ void tier_partial(const uint8_t *__restrict__ slots, int len, int n_sink, int n_recent, int slot0,
-                             int slot1, const float *q, int hs, int ps, const int *chan, int k,
+                             int slot1, const QS &qs, int k,
                              float *__restrict__ part_o, float2 *__restrict__ part_ml, size_t qrow0, int S, int s,
                              float *scratch) {
     constexpr int C = kTierChunk;
@@ -380,20 +413,21 @@ __device__ void tier_partial(const uint8_t *__restrict__ slots, int len, int n_s
         for (int e = t; e < G * C; e += NT) {
             const int hl = e / C, tt = e % C, slot = c0 + tt;
             bool valid = false;
+            int p = slot;                              // the position this slot holds
             if (tt < n) {
                 if (slot < n_sink) {
                     valid = slot < tr.sink_end;
                 } else if (n_recent > 0) {
                     // the one position of the recent window that owns this ring slot
                     const int j = slot - n_sink;
-                    const int p = tr.recent_start + ((j - tr.recent_start % n_recent) % n_recent + n_recent) % n_recent;
+                    p = tr.recent_start + ((j - tr.recent_start % n_recent) % n_recent + n_recent) % n_recent;
                     valid = p < len;
                 }
             }
             float v = -INFINITY;
             if (valid) {
                 float a = 0.f;
-                for (int i = 0; i < k; i++) a = fmaf(q[hl * hs + i * ps], kT[chan[i] * (C + 1) + tt], a);
+                for (int i = 0; i < k; i++) a = fmaf(qs.q_at(hl, i, p), kT[qs.ch(i, p) * (C + 1) + tt], a);
                 v = a * kScoreScaleLog2;
             }
             sc[e] = v;

@@ -9,6 +9,11 @@
 //        the energies are those of the base queries, q'_{h,j} / delta_j.
 // Channel 0 is always kept; ties go to the lower channel index.
 //
+// With bucket-relative RoPE (§3.4) the grid has one cluster per bucket too:
+// the cluster of bucket b first moves the query into b's frame (its anchor's
+// rotary rotation removed) and writes entry b of the outputs; buckets past
+// the sequence's length (other than bucket 0) do nothing.
+//
 // One thread-block cluster of four CTAs = one (sequence, KV head); CTA r owns
 // channels 32r..32r+31 (key group r).  It stages its 32 columns of A^{-T}
 // (32 KB) with one cp.async burst and runs the fixed-order fp64 fma chains
@@ -34,7 +39,8 @@ template <typename Tin>
 __global__ void __cluster_dims__(kCtas, 1, 1) __launch_bounds__(kThreads)
 select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, const double *__restrict__ delta,
               int Hq, int Hkv, int g, int k, int32_t *__restrict__ idx, float *__restrict__ qsel,
-              float *__restrict__ qgsum, int ng) {
+              float *__restrict__ qgsum, int ng, const int32_t *__restrict__ seq_len,
+              const double *__restrict__ rope, int nbk, int w) {
     extern __shared__ __align__(16) double sm[];   // As[128][32], qin[g][128], qp[g][32]
     double *As = sm;
     double *qin = sm + kD * kGroup;
@@ -46,10 +52,12 @@ select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, const
     __shared__ int warp_cnt[4];
 
     cg::cluster_group cluster = cg::this_cluster();
-    const int r = (int)cluster.block_rank();       // = blockIdx.x
+    const int r = (int)cluster.block_rank();       // = blockIdx.x % 4
+    const int bk = blockIdx.x / kCtas;              // RoPE bucket (0 without buckets)
     const int h = blockIdx.y, b = blockIdx.z, t = threadIdx.x;
     const int lane = t & 31, warp = t >> 5;
     const size_t qrow0 = (size_t)b * Hq + (size_t)h * g;
+    if (bk > 0 && (size_t)bk * w >= (size_t)max(seq_len[b], 0)) return;   // the whole cluster
 
     // columns 32r..32r+31 of A^{-T} for this KV head: 128 rows of 256 bytes
     const double *Ai = Ainvt + (size_t)h * kD * kD + r * kGroup;
@@ -61,6 +69,15 @@ select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, const
     for (int e = t; e < g * kD; e += kThreads) qin[e] = in_to_double(q[qrow0 * kD + e]);
     cp_async_wait<0>();
     __syncthreads();
+    if (rope) {
+        // q T_b: channel pairs (i, i + 64) rotated back by the anchor's angle
+        const double2 *cs = reinterpret_cast<const double2 *>(rope) + (size_t)bk * (kD / 2);
+        for (int e = t; e < g * (kD / 2); e += kThreads) {
+            const int hl = e / (kD / 2), i = e % (kD / 2);
+            rope_unanchor_pair(qin[hl * kD + i], qin[hl * kD + i + kD / 2], __ldg(cs + i));
+        }
+        __syncthreads();
+    }
 
     // q'[hl][j] = sum_c q[hl][c] Ainvt[c][j], fma chain c = 0..127 from 0.0
     for (int hl = warp; hl < g; hl += kThreads / 32) {
@@ -114,8 +131,8 @@ select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, const
     // this CTA's channels are t = 32r..32r+31 (warp r)
     if (warp == r && pos >= 0) {
         for (int w = 0; w < r; w++) pos += warp_cnt[w];
-        idx[((size_t)b * Hkv + h) * k + pos] = t;
-        for (int hl = 0; hl < g; hl++) qsel[(qrow0 + hl) * k + pos] = (float)qp[hl * kGroup + lane];
+        idx[(((size_t)b * Hkv + h) * nbk + bk) * k + pos] = t;
+        for (int hl = 0; hl < g; hl++) qsel[((qrow0 + hl) * nbk + bk) * k + pos] = (float)qp[hl * kGroup + lane];
     }
     // zero-point sum of each key group (channel 0 is bf16, not in group 0),
     // kept channels ascending from 0.0: groups of 32 -- CTA r sums group r;
@@ -126,7 +143,7 @@ select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, const
             double s = 0.0;
             for (int c = (r == 0 ? 1 : 0); c < kGroup; c++)
                 if (sel_s[r * kGroup + c]) s += qp[hl * kGroup + c];
-            qgsum[(qrow0 + hl) * kNG + r] = (float)s;
+            qgsum[((qrow0 + hl) * nbk + bk) * kNG + r] = (float)s;
         }
     } else if (r == 0) {
         const double *pq[kCtas];
@@ -136,9 +153,9 @@ select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, const
             double s = 0.0;
             for (int c = 1; c < kD; c++)
                 if (sel_s[c]) s += pq[c / kGroup][hl * kGroup + c % kGroup];
-            qgsum[(qrow0 + hl) * kNG] = (float)s;
+            qgsum[((qrow0 + hl) * nbk + bk) * kNG] = (float)s;
 #pragma unroll
-            for (int gr = 1; gr < kNG; gr++) qgsum[(qrow0 + hl) * kNG + gr] = 0.f;
+            for (int gr = 1; gr < kNG; gr++) qgsum[((qrow0 + hl) * nbk + bk) * kNG + gr] = 0.f;
         }
     }
     cluster.sync();                                // keep e2own alive until all have read it
@@ -152,18 +169,22 @@ cudaError_t launch_select(const kvq_cache &c, const void *q, int dtype, int Hq, 
     const size_t smem = (size_t)(kD * kGroup + g * kD + g * kGroup) * sizeof(double);
     constexpr int kMaxSmem = (kD * kGroup + 32 * kD + 32 * kGroup) * (int)sizeof(double);   // g <= 32
     static std::atomic<uint64_t> done_f32{0}, done_bf16{0};
-    dim3 grid((unsigned)kCtas, (unsigned)c.n_kv_heads, (unsigned)c.batch);
+    const int nbk = buckets_of(c);
+    dim3 grid((unsigned)(kCtas * nbk), (unsigned)c.n_kv_heads, (unsigned)c.batch);
+    const double *rope = c.bucket > 0 ? c.rope : nullptr;
     cudaError_t e;
     if (dtype == KVQ_DTYPE_F32) {
         e = set_smem_once(select_kernel<float>, kMaxSmem, done_f32);
         if (e != cudaSuccess) return e;
         select_kernel<float><<<grid, kThreads, smem, st>>>(static_cast<const float *>(q), Ainvt, delta, Hq,
-                                                           c.n_kv_heads, g, k, idx, qsel, qgsum, groups_of(c));
+                                                           c.n_kv_heads, g, k, idx, qsel, qgsum, groups_of(c),
+                                                           c.seq_len, rope, nbk, c.bucket);
     } else {
         e = set_smem_once(select_kernel<uint16_t>, kMaxSmem, done_bf16);
         if (e != cudaSuccess) return e;
         select_kernel<uint16_t><<<grid, kThreads, smem, st>>>(static_cast<const uint16_t *>(q), Ainvt, delta, Hq,
-                                                              c.n_kv_heads, g, k, idx, qsel, qgsum, groups_of(c));
+                                                              c.n_kv_heads, g, k, idx, qsel, qgsum, groups_of(c),
+                                                              c.seq_len, rope, nbk, c.bucket);
     }
     return cudaGetLastError();
 }

@@ -47,6 +47,7 @@ class CacheDesc(ctypes.Structure):
         ("pages", ctypes.c_void_p), ("seq_len", ctypes.c_void_p), ("status", ctypes.c_void_p),
         ("n_sink", ctypes.c_int32), ("n_recent", ctypes.c_int32),
         ("v_rot", ctypes.c_void_p), ("v_clip", ctypes.c_double),
+        ("bucket", ctypes.c_int32), ("rope", ctypes.c_void_p),
     ]
 
 
@@ -57,7 +58,7 @@ EXPORTS = (
     "kvq_select_channels", "kvq_decode_workspace", "kvq_decode_attn",
     "kvq_bf16_decode_workspace", "kvq_bf16_decode_attn", "kvq_read_status",
     "kvq_status_string", "kvq_version", "kvq_decode_static_scratch_bytes",
-    "kvq_decode_attn_static", "kvq_decode_step",
+    "kvq_decode_attn_static", "kvq_decode_step", "kvq_num_buckets",
 )
 
 
@@ -89,6 +90,7 @@ def lib() -> ctypes.CDLL:
             "kvq_decode_static_scratch_bytes": (S, []),
             "kvq_decode_attn_static": (I, [C, I, P, P, P, I, P, P]),
             "kvq_decode_step": (I, [C, P, P, P, I, I, I, P, P, P, ctypes.c_float, P, P, P, P, P, S, P]),
+            "kvq_num_buckets": (I, [C]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -143,13 +145,20 @@ class KVCache:
     group: int = GROUP        # channels per quantization group: 32, or 128 (one grid per token)
     v_rot: Optional[torch.Tensor] = None   # value rotation [Hkv][128][128] f64 (orthogonal), or None
     v_clip: float = 1.0       # clipping ratio of the value grids
+    bucket: int = 0           # tokens per RoPE bucket (0: none)
+    rope: Optional[torch.Tensor] = None    # anchors' rotary table [n_buckets][64][2] f64
 
     @property
     def desc(self) -> CacheDesc:
         return CacheDesc(self.batch, self.n_kv_heads, HEAD_DIM, self.group, self.bits, self.capacity,
                          self.pages.data_ptr(), self.seq_len.data_ptr(), self.status.data_ptr(),
                          self.n_sink, self.n_recent, 0 if self.v_rot is None else self.v_rot.data_ptr(),
-                         float(self.v_clip))
+                         float(self.v_clip), self.bucket, 0 if self.rope is None else self.rope.data_ptr())
+
+    @property
+    def n_buckets(self) -> int:
+        """Entries per selection array: RoPE buckets of the capacity, 1 without."""
+        return (self.capacity + self.bucket - 1) // self.bucket if self.bucket else 1
 
     @property
     def n_blocks(self) -> int:
@@ -181,15 +190,22 @@ def page_bytes(bits: int, group: int = GROUP) -> int:
 
 def new_cache(batch: int, n_kv_heads: int, capacity: int, bits: int = 2,
               device="cuda", stream=None, n_sink: int = 0, n_recent: int = 0, group: int = GROUP,
-              v_rot: Optional[torch.Tensor] = None, v_clip: float = 1.0) -> KVCache:
+              v_rot: Optional[torch.Tensor] = None, v_clip: float = 1.0, bucket: int = 0,
+              rope: Optional[torch.Tensor] = None) -> KVCache:
     """A zeroed cache.  ``v_rot`` (device f64 [Hkv][128][128], orthogonal) makes
     appends store rotated values and decodes rotate their output back;
-    ``v_clip`` clips the value grids (Dual-QK App. B.2 uses 0.92)."""
+    ``v_clip`` clips the value grids (Dual-QK App. B.2 uses 0.92); ``bucket``
+    tokens per RoPE bucket with the anchors' rotary table ``rope`` (device f64
+    [n_buckets][64][2] of cos, sin) store keys in their bucket's frame and
+    choose channels per bucket (Dual-QK §3.4)."""
     if v_rot is not None:
         assert v_rot.dtype == torch.float64 and v_rot.is_contiguous()
         assert tuple(v_rot.shape) == (n_kv_heads, HEAD_DIM, HEAD_DIM)
+    if bucket:
+        assert rope is not None and rope.dtype == torch.float64 and rope.is_contiguous()
+        assert tuple(rope.shape) == ((capacity + bucket - 1) // bucket, HEAD_DIM // 2, 2)
     desc = CacheDesc(batch, n_kv_heads, HEAD_DIM, group, bits, capacity, 0, 0, 0, n_sink, n_recent,
-                     None, float(v_clip))
+                     None, float(v_clip), bucket, None)
     nbytes = int(lib().kvq_cache_bytes(ctypes.byref(desc)))
     if nbytes == 0:
         raise KvqError("kvq_cache_bytes", -2)
@@ -198,7 +214,7 @@ def new_cache(batch: int, n_kv_heads: int, capacity: int, bits: int = 2,
     status = torch.empty(int(lib().kvq_status_words(batch, n_kv_heads)), dtype=torch.int32,
                          device=device)
     c = KVCache(batch, n_kv_heads, capacity, bits, pages, seq_len, status, n_sink, n_recent, group, v_rot,
-                float(v_clip))
+                float(v_clip), bucket, rope)
     _check("kvq_cache_init", lib().kvq_cache_init(ctypes.byref(c.desc), _stream(stream)))
     return c
 
@@ -220,10 +236,13 @@ class Selection:
 
 
 def alloc_selection(cache: KVCache, n_q_heads: int, k: int, device="cuda") -> Selection:
+    """Selection arrays: idx [B][Hkv][k], qsel [B][Hq][k], qgsum [B][Hq][4];
+    with RoPE buckets one entry per bucket, [B][H][n_buckets][...]."""
+    nb = (cache.n_buckets,) if cache.bucket else ()
     return Selection(
-        torch.empty(cache.batch, cache.n_kv_heads, k, dtype=torch.int32, device=device),
-        torch.empty(cache.batch, n_q_heads, k, dtype=torch.float32, device=device),
-        torch.empty(cache.batch, n_q_heads, 4, dtype=torch.float32, device=device), k)
+        torch.empty(cache.batch, cache.n_kv_heads, *nb, k, dtype=torch.int32, device=device),
+        torch.empty(cache.batch, n_q_heads, *nb, k, dtype=torch.float32, device=device),
+        torch.empty(cache.batch, n_q_heads, *nb, 4, dtype=torch.float32, device=device), k)
 
 
 def select_channels(cache: KVCache, q: torch.Tensor, Ainvt: torch.Tensor, sparsity: float,

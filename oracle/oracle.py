@@ -324,8 +324,12 @@ def bucket_keys(K, A, rope, w: int, pos0: int = 0) -> np.ndarray:
     b = n // w (§3.4)."""
     K = _f64(K).reshape(-1, D)
     out = np.empty_like(K)
-    for i in range(K.shape[0]):
-        out[i] = transform(rope_unanchor(K[i:i + 1], rope[(pos0 + i) // w]), A)[0]
+    i = 0
+    while i < K.shape[0]:                       # the tokens of one bucket at a time
+        b = (pos0 + i) // w
+        j = min(K.shape[0], (b + 1) * w - pos0)
+        out[i:j] = transform(rope_unanchor(K[i:j], rope[b]), A)
+        i = j
     return out
 
 

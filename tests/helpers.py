@@ -30,13 +30,16 @@ class Case:
         self.A, self.Ai = W.make_transforms(self.wl)      # refinement folded in when the workload has one
         self.delta = W.make_deltas(self.wl)                # [Hkv][128] or None
         self.Rv = W.make_value_rotations(self.wl)          # [Hkv][128][128] or None
+        w = self.wl.bucket                                 # RoPE anchors of the cache's buckets, or None
+        self.rope = W.rope_table(-(-self.capacity // w), w, self.wl.rope_base) if w else None
         self.K, self.V = W.make_kv(self.wl)
         self._oracle_units = {}
 
     def cache_kw(self) -> dict:
         """new_cache keywords of the workload's format (group, value rotation, clip)."""
         return dict(group=self.wl.quant_group, v_rot=None if self.Rv is None else dev64(self.Rv),
-                    v_clip=self.wl.v_clip)
+                    v_clip=self.wl.v_clip, bucket=self.wl.bucket,
+                    rope=None if self.rope is None else dev64(self.rope))
 
     def dev_delta(self):
         return None if self.delta is None else dev64(self.delta)
@@ -50,6 +53,36 @@ class Case:
     def oracle_values(self, Vf: np.ndarray, h: int) -> np.ndarray:
         """Values as the cache stores them: rotated when the workload rotates them."""
         return Vf if self.Rv is None else orc.value_rotate(Vf, self.Rv[h])
+
+    def oracle_keys(self, Kf: np.ndarray, h: int, pos0: int = 0) -> np.ndarray:
+        """K' as the cache stores it: in the frame of each token's RoPE bucket
+        when the workload has buckets."""
+        if self.rope is None:
+            return orc.transform(Kf, self.A[h])
+        return orc.bucket_keys(Kf, self.A[h], self.rope, self.wl.bucket, pos0)
+
+    def n_buckets(self, n: int) -> int:
+        return max(1, -(-n // self.wl.bucket)) if self.wl.bucket else 1
+
+    def oracle_decode_any(self, q, b, h, sparsity, n, slots=None, n_sink=0, n_recent=0):
+        """The oracle's decode of one unit over n tokens in the workload's
+        format (buckets, tier, rotation, refinement).  Returns (out, idx) with
+        idx [n_buckets][k] when the workload has buckets, else [k]."""
+        wl = self.wl
+        unit = self.oracle_unit(b, h, n)
+        g = wl.group_size
+        qf = W.as_float(q[b, h * g:(h + 1) * g], wl.dtype)
+        if self.rope is not None:
+            qpb = orc.bucket_queries(qf, self.Ai[h], self.rope, self.n_buckets(n))
+            return orc.decode_unit_buckets(unit, wl.bits, n, qpb, sparsity, wl.bucket, wl.quant_group,
+                                           delta=self.delta_of(h), Rv=self.rv_of(h), slots=slots, n_sink=n_sink,
+                                           n_recent=n_recent)
+        qp = orc.transform(qf, self.Ai[h])
+        if slots is not None and n_sink + n_recent > 0:
+            return orc.decode_unit_protected(unit, slots, wl.bits, n, qp, sparsity, n_sink, n_recent,
+                                             wl.quant_group, delta=self.delta_of(h), Rv=self.rv_of(h))
+        return orc.decode_unit(unit, wl.bits, n, qp, sparsity, wl.quant_group, delta=self.delta_of(h),
+                               Rv=self.rv_of(h))
 
     # ---------------------------------------------------------------- GPU
     def gpu_cache(self, chunks=None) -> kvq.KVCache:
@@ -78,7 +111,7 @@ class Case:
             Kf = W.as_float(self.K[b, h, :n], wl.dtype)
             Vf = W.as_float(self.V[b, h, :n], wl.dtype)
             u = orc.new_unit(self.capacity, wl.bits, wl.quant_group)
-            orc.append_unit(u, wl.bits, 0, orc.transform(Kf, self.A[h]), self.oracle_values(Vf, h),
+            orc.append_unit(u, wl.bits, 0, self.oracle_keys(Kf, h), self.oracle_values(Vf, h),
                             group=wl.quant_group, vclip=wl.v_clip)
             self._oracle_units[key] = u
         return self._oracle_units[key]
@@ -91,8 +124,7 @@ class Case:
     def oracle_decode(self, q: np.ndarray, b: int, h: int, sparsity: float, n: int | None = None):
         n = self.K.shape[2] if n is None else n
         qp = self.oracle_qp(q, b, h)
-        out, idx = orc.decode_unit(self.oracle_unit(b, h), self.wl.bits, n, qp, sparsity, self.wl.quant_group,
-                                   delta=self.delta_of(h), Rv=self.rv_of(h))
+        out, idx = self.oracle_decode_any(q, b, h, sparsity, n)
         return out, idx, qp
 
 

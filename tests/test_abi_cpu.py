@@ -30,7 +30,7 @@ def test_every_declared_symbol_is_exported():
 
 def test_host_side_queries():
     L = kvq.lib()
-    assert L.kvq_version() == 101
+    assert L.kvq_version() == 102
     assert L.kvq_page_bytes(2, 32) == 12544 and L.kvq_page_bytes(4, 32) == 20736 and L.kvq_page_bytes(3, 32) == 0
     assert L.kvq_page_bytes(2, 128) == 9472 and L.kvq_page_bytes(4, 128) == 17664 and L.kvq_page_bytes(2, 64) == 0
     for s, k in ((0.0, 128), (0.2, 103), (0.4, 77), (0.6, 52), (0.25, 96)):
@@ -81,6 +81,18 @@ def test_validation_rejects_before_launch():
         assert L.kvq_append(ctypes.byref(bad_clip), 8, 8, 0, 1, 16, None) == -1
     ok_rot = kvq.CacheDesc(1, 1, 128, 32, 2, 128, 0x1000, 256, 256, 0, 0, 0x1000, 0.92)
     assert L.kvq_append(ctypes.byref(ok_rot), 8, 8, 0, 0, 16, None) == 0        # valid, no-op
+    # RoPE buckets: a multiple of 128 tokens, with the anchors' table
+    def bk(w, rope):
+        return kvq.CacheDesc(1, 1, 128, 32, 2, 1000 * 128, 0x1000, 256, 256, 0, 0, 0, 0.0, w, rope)
+    assert L.kvq_append(ctypes.byref(bk(200, 0x2000)), 8, 8, 0, 0, 16, None) == -2
+    assert L.kvq_append(ctypes.byref(bk(-128, 0x2000)), 8, 8, 0, 0, 16, None) == -2
+    assert L.kvq_append(ctypes.byref(bk(2048, 0)), 8, 8, 0, 0, 16, None) == -1
+    assert L.kvq_append(ctypes.byref(bk(2048, 0x2008)), 8, 8, 0, 0, 16, None) == -6
+    assert L.kvq_append(ctypes.byref(bk(2048, 0x2000)), 8, 8, 0, 0, 16, None) == 0
+    assert L.kvq_num_buckets(ctypes.byref(bk(2048, 0x2000))) == 63          # ceil(128000 / 2048)
+    assert L.kvq_num_buckets(ctypes.byref(bk(128, 0x2000))) == 1000
+    assert L.kvq_num_buckets(ctypes.byref(bk(0, 0))) == 1
+    assert L.kvq_num_buckets(ctypes.byref(bk(200, 0x2000))) == 0
     assert L.kvq_decode_attn(ctypes.byref(two), 6, 8, 8, 8, 77, 8, 8, 1 << 20, None) == -2  # g = 3
     assert L.kvq_decode_attn(ctypes.byref(two), 4, 8, 8, 8, 0, 8, 8, 1 << 20, None) == -1   # k = 0
     assert L.kvq_bf16_decode_attn(8, 8, 8, 1, 3, 2, 10, 8, 8, 1 << 20, None) == -2
