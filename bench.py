@@ -182,12 +182,17 @@ def oracle_sample(wl: W.Workload, n_steps: int, budget_s: float = 30.0, skip_fir
     Rv = W.make_value_rotations(wl.with_(n_kv_heads=1))
     Rv = None if Rv is None else Rv[0]
     vals = (lambda v: v) if Rv is None else (lambda v: orc.value_rotate(v, Rv))
+    rope = W.make_rope(wl)
+    if rope is None:
+        keys = lambda k, pos0: orc.transform(k, A)                          # noqa: E731
+    else:
+        keys = lambda k, pos0: orc.bucket_keys(k, A, rope, wl.bucket, pos0)  # noqa: E731
     n_sink, n_recent = protect
     K, V = W.make_kv_unit(wl, 0, 0)
     gq = wl.quant_group
     unit = orc.new_unit(wl.capacity, wl.bits, gq)
     slots = orc.new_slots(n_sink, n_recent)
-    Kp, Vr = orc.transform(W.as_float(K, wl.dtype), A), vals(W.as_float(V, wl.dtype))
+    Kp, Vr = keys(W.as_float(K, wl.dtype), 0), vals(W.as_float(V, wl.dtype))
     orc.append_unit(unit, wl.bits, 0, Kp, Vr, group=gq, vclip=wl.v_clip)
     length = wl.n_ctx
     if n_sink + n_recent:
@@ -199,9 +204,20 @@ def oracle_sample(wl: W.Workload, n_steps: int, budget_s: float = 30.0, skip_fir
         kn, vn = W.make_step_kv(wl, i)
         q = W.make_q(wl, i)
         t0 = time.perf_counter()
-        kp, vr = orc.transform(W.as_float(kn[0, 0], wl.dtype), A), vals(W.as_float(vn[0, 0], wl.dtype))
+        kp, vr = keys(W.as_float(kn[0, 0], wl.dtype), length), vals(W.as_float(vn[0, 0], wl.dtype))
         orc.append_unit(unit, wl.bits, length, kp, vr, group=gq, vclip=wl.v_clip)
         length += 1
+        if rope is not None:
+            if n_sink + n_recent:
+                orc.protect_store(slots, n_sink, n_recent, length - 1, kp, vr, length)
+            qpb = orc.bucket_queries(W.as_float(q[0, :g], wl.dtype), Ai, rope, -(-length // wl.bucket))
+            orc.decode_unit_buckets(unit, wl.bits, length, qpb, wl.sparsity, wl.bucket, gq, delta=delta, Rv=Rv,
+                                    slots=slots, n_sink=n_sink, n_recent=n_recent)
+            times.append(time.perf_counter() - t0)
+            tokens.append(length)
+            if time.perf_counter() - t_start > budget_s and i >= 1:
+                break
+            continue
         qp = orc.transform(W.as_float(q[0, :g], wl.dtype), Ai)
         if n_sink + n_recent:
             orc.protect_store(slots, n_sink, n_recent, length - 1, kp, vr, length)
@@ -260,12 +276,14 @@ def config_dict(wl: W.Workload, k: int, protect=(0, 0)):
         d["value_rotation"] = {"clip": wl.v_clip}
     if wl.refine:
         d["diagonal_refinement"] = True
+    if wl.bucket:
+        d["rope_bucket"] = wl.bucket
     return d
 
 
 def format_overrides(args) -> dict:
     """Workload fields of the cache format the flags ask for."""
-    d = {"quant_group": args.group}
+    d = {"quant_group": args.group, "bucket": args.bucket}
     if args.rotate_values:
         d.update(rotate_values=True, v_clip=0.92)
     if args.refine:
@@ -279,11 +297,11 @@ def protect_of(args):
 
 def format_tag(wl: W.Workload, protect=(0, 0)) -> str:
     """Suffix naming a cache format other than the default (groups of 32,
-    no tier, no rotation, no refinement): the pages' whole recipe is
-    "_pages", anything else lists its parts."""
+    no tier, no rotation, no refinement, no RoPE buckets): the pages' whole
+    recipe is "_pages", anything else lists its parts."""
     parts = [p for p, on in (("g128", wl.quant_group == 128), ("tier", protect != (0, 0)),
-                             ("rot", wl.rotate_values), ("ref", wl.refine)) if on]
-    if len(parts) == 4:
+                             ("rot", wl.rotate_values), ("ref", wl.refine), (f"bkt{wl.bucket}", wl.bucket > 0)) if on]
+    if len(parts) == 5 and wl.bucket == 2048:
         return "_pages"
     return "_" + "-".join(parts) if parts else ""
 
@@ -359,8 +377,10 @@ def run_ours(args):
     Rv_np, delta_np = W.make_value_rotations(wl), W.make_deltas(wl)
     Rv = None if Rv_np is None else torch.from_numpy(Rv_np).to(dev)
     delta = None if delta_np is None else torch.from_numpy(delta_np).to(dev)
+    rope_np = W.make_rope(wl)
+    rope = None if rope_np is None else torch.from_numpy(rope_np).to(dev)
     cache = kvq.new_cache(B, Hkv, wl.capacity, wl.bits, device=dev, n_sink=protect[0], n_recent=protect[1],
-                          group=wl.quant_group, v_rot=Rv, v_clip=wl.v_clip)
+                          group=wl.quant_group, v_rot=Rv, v_clip=wl.v_clip, bucket=wl.bucket, rope=rope)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record()
     kvq.append(cache, Kd, Vd, A)
@@ -541,8 +561,11 @@ def main():
                     help="rotate the values before quantization, clip their grids at 0.92, rotate the output back")
     ap.add_argument("--refine", action="store_true",
                     help="fold a diagonal refinement into the transforms; select on the base queries")
+    ap.add_argument("--bucket", type=int, default=0,
+                    help="tokens per bucket of bucket-relative RoPE (the pages use 2048; 0: none); "
+                         "a bucketed step runs as the three calls")
     ap.add_argument("--pages-recipe", action="store_true",
-                    help="the pages' whole format: --group 128 --protect --rotate-values --refine")
+                    help="the pages' whole format: --group 128 --protect --rotate-values --refine --bucket 2048")
     ap.add_argument("--unfused", dest="fused", action="store_false",
                     help="run the step as three launches (append, select, decode) instead of one")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
@@ -550,6 +573,9 @@ def main():
     args = ap.parse_args()
     if args.pages_recipe:
         args.group, args.protect, args.rotate_values, args.refine = 128, True, True, True
+        args.bucket = 2048
+    if args.bucket:
+        args.fused = False          # the bucketed step runs as append, select, decode
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":

@@ -25,6 +25,8 @@
 // the stored bytes reproducible bit for bit.
 #include "kvq_internal.cuh"
 
+#include <cooperative_groups.h>
+
 namespace kvq {
 namespace {
 
@@ -223,13 +225,15 @@ append_kernel(uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len,
 // memory to one thread per channel row, which merges the new tokens into the
 // packed bytes in order (neighbouring tokens share bytes).  With a value
 // rotation the same staging memory then takes the group's 32 columns of the
-// rotation for the values' chains.  The last CTA of a sequence to finish
-// advances its length, using the sequence's completion counter in the status
-// array.
+// rotation for the values' chains.  The four CTAs of a (sequence, KV head)
+// form a cluster: with one grid per token (NG = 1) each token's key and value
+// ranges are met over the four CTAs' warps through distributed shared memory.
+// The last CTA of a sequence to finish advances its length, using the
+// sequence's completion counter in the status array.
 constexpr int kSmallMax = 4;
 
-template <typename Tin, int BITS>
-__global__ void __launch_bounds__(128)
+template <typename Tin, int BITS, int NG>
+__global__ void __cluster_dims__(kNG, 1, 1) __launch_bounds__(128)
 append_small_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len,
                     uint32_t *__restrict__ status, const Tin *__restrict__ K,
                     const Tin *__restrict__ V, const double *__restrict__ A, const double *__restrict__ Rv,
@@ -243,7 +247,10 @@ append_small_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len,
     __shared__ double vsd[kSmallMax][kD];                  // full value rows (value rotation only)
     __shared__ uint8_t kcode[kSmallMax][kGroup];
     __shared__ uint8_t vcode[kSmallMax][kGroup];
+    __shared__ double trange[kSmallMax][4];                // NG = 1: this CTA's {key lo, hi, value lo, hi}
     __shared__ int s_len;
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
 
     const int grp = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int t = threadIdx.x, lane = t & 31, w = t >> 5;
@@ -264,7 +271,7 @@ append_small_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len,
     __syncthreads();
     const int len = s_len;
     const bool ok = len >= 0 && len + n_new <= capacity;
-    uint8_t *unit = pages + ((size_t)b * Hkv + h) * NB * (size_t)page_bytes(BITS);
+    uint8_t *unit = pages + ((size_t)b * Hkv + h) * NB * (size_t)page_bytes(BITS, NG);
     if (rope && ok) {
         // k T_b for the bucket of each new position
         const double2 *cs = reinterpret_cast<const double2 *>(rope);
@@ -301,21 +308,53 @@ append_small_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len,
         }
     }
 
+    // one grid per token: the token's ranges over all four CTAs of the cluster
+    double klo = 0.0, khi = 0.0, vlo = 0.0, vhi = 0.0;
+    if constexpr (NG == 1) {
+        if (ok && w < n_new) {
+            const double a = warp_min(j != 0 ? x : pos_inf()), bk = warp_max(j != 0 ? x : neg_inf());
+            const double c = warp_min(v), d = warp_max(v);
+            if (lane == 0) {
+                trange[w][0] = a;
+                trange[w][1] = bk;
+                trange[w][2] = c;
+                trange[w][3] = d;
+            }
+        }
+        cluster.sync();
+        if (ok && w < n_new) {
+            klo = pos_inf(), khi = neg_inf(), vlo = pos_inf(), vhi = neg_inf();
+#pragma unroll
+            for (int rr = 0; rr < kNG; rr++) {
+                const double *pr = cluster.map_shared_rank(&trange[w][0], rr);
+                klo = fmin(klo, pr[0]);
+                khi = fmax(khi, pr[1]);
+                vlo = fmin(vlo, pr[2]);
+                vhi = fmax(vhi, pr[3]);
+            }
+        }
+        cluster.sync();                                    // the peers are done reading trange
+    }
+
     if (ok && w < n_new) {                                 // uniform over the warp
         const int pos = len + w, tt = pos % kT;
-        uint8_t *page = unit + (size_t)(pos / kT) * page_bytes(BITS);
+        uint8_t *page = unit + (size_t)(pos / kT) * page_bytes(BITS, NG);
+        const int mg = NG == 1 ? 0 : grp;                  // metadata group
+        const bool meta_writer = lane == 0 && (NG != 1 || grp == 0);
         uint16_t sb, zb;
-        kcode[w][lane] = (uint8_t)quantize_lane<BITS>(x, j != 0, sb, zb);
-        if (lane == 0)
-            reinterpret_cast<uint32_t *>(page + off_kmeta(BITS))[meta_word(grp, tt)] = (uint32_t)sb | ((uint32_t)zb << 16);
+        kcode[w][lane] = (uint8_t)(NG == 1 ? code_in_range<BITS>(x, klo, khi, sb, zb)
+                                           : quantize_lane<BITS>(x, j != 0, sb, zb));
+        if (meta_writer)
+            reinterpret_cast<uint32_t *>(page + off_kmeta(BITS))[meta_word(mg, tt)] = (uint32_t)sb | ((uint32_t)zb << 16);
         if (j == 0) reinterpret_cast<uint16_t *>(page + off_ch0(BITS))[tt] = __bfloat16_as_ushort(__double2bfloat16(x));
-        vcode[w][lane] = (uint8_t)quantize_lane<BITS>(v, true, sb, zb, vclip);
-        if (lane == 0)
-            reinterpret_cast<uint32_t *>(page + off_vmeta(BITS))[meta_word(grp, tt)] = (uint32_t)sb | ((uint32_t)zb << 16);
+        vcode[w][lane] = (uint8_t)(NG == 1 ? code_in_range<BITS>(v, __dmul_rn(vclip, vlo), __dmul_rn(vclip, vhi), sb, zb)
+                                           : quantize_lane<BITS>(v, true, sb, zb, vclip));
+        if (meta_writer)
+            reinterpret_cast<uint32_t *>(page + off_vmeta(BITS, NG))[meta_word(mg, tt)] = (uint32_t)sb | ((uint32_t)zb << 16);
         // protected tier: BF16 copies (sink tokens, the last n_recent tokens)
         if (n_sink + n_recent > 0 && stores_slot(pos, len + n_new, n_sink, n_recent)) {
             uint16_t *dst = reinterpret_cast<uint16_t *>(
-                unit_slots(pages, gridDim.z, Hkv, NB, BITS, (size_t)b * Hkv + h, n_sink + n_recent) +
+                unit_slots(pages, gridDim.z, Hkv, NB, BITS, (size_t)b * Hkv + h, n_sink + n_recent, NG) +
                 (size_t)slot_of(pos, n_sink, n_recent) * kSlotBytes);
             dst[j] = __bfloat16_as_ushort(__double2bfloat16(x));
             dst[kD + j] = __bfloat16_as_ushort(__double2bfloat16(v));
@@ -329,7 +368,7 @@ append_small_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len,
             for (int i = 0; i < n_new; i++) {
                 const int pos = len + i, tt = pos % kT;
                 const int byte = tt / PER, sh = (tt % PER) * BITS;
-                uint8_t *p = unit + (size_t)(pos / kT) * page_bytes(BITS) + (val ? off_vcodes(BITS) : 0) +
+                uint8_t *p = unit + (size_t)(pos / kT) * page_bytes(BITS, NG) + (val ? off_vcodes(BITS) : 0) +
                              (size_t)j * R + byte;
                 const uint8_t clear = (uint8_t)~(((1u << BITS) - 1u) << sh);
                 const uint32_t code = val ? vcode[i][lane] : kcode[i][lane];
@@ -366,11 +405,11 @@ cudaError_t launch_append_t(const kvq_cache &c, const void *K, const void *V, in
     const double vclip = value_clip(c);
     const double *rope = c.bucket > 0 ? c.rope : nullptr;
     const int NB = c.capacity / kT;
-    // a few tokens with groups of 32: one CTA per group; otherwise (prefill,
-    // or one grid per token) the tile kernel and the length advance
-    if (NG == kNG && n_new <= kSmallMax) {
+    // a few tokens: one CTA per 32-channel group (a cluster of four per
+    // sequence and KV head); a prefill: the tile kernel and the length advance
+    if (n_new <= kSmallMax) {
         dim3 grid((unsigned)kNG, (unsigned)c.n_kv_heads, (unsigned)c.batch);
-        append_small_kernel<Tin, BITS><<<grid, 128, 0, st>>>(
+        append_small_kernel<Tin, BITS, NG><<<grid, 128, 0, st>>>(
             static_cast<uint8_t *>(c.pages), c.seq_len, c.status, static_cast<const Tin *>(K),
             static_cast<const Tin *>(V), A, Rv, vclip, c.n_kv_heads, NB, n_new, c.capacity, c.n_sink, c.n_recent,
             rope, c.bucket);

@@ -6,23 +6,25 @@
 //   §3.2 Eq. 4: channel energy pooled over the query heads sharing a KV head,
 //        e_j^2 = sum_h q'_{h,j}^2, one mask per KV head, chosen per query;
 //   §3.3, App. C.2: with a diagonal refinement D folded into the transforms
-//        the energies are those of the base queries, q'_{h,j} / delta_j.
+//        the energies are those of the base queries, q'_{h,j} / delta_j;
+//   §3.4: with bucket-relative RoPE each bucket that holds a token gets its
+//        own choice, made on the query moved into the bucket's frame (its
+//        anchor's rotary rotation removed).
 // Channel 0 is always kept; ties go to the lower channel index.
 //
-// With bucket-relative RoPE (§3.4) the grid has one cluster per bucket too:
-// the cluster of bucket b first moves the query into b's frame (its anchor's
-// rotary rotation removed) and writes entry b of the outputs; buckets past
-// the sequence's length (other than bucket 0) do nothing.
-//
-// One thread-block cluster of four CTAs = one (sequence, KV head); CTA r owns
+// One thread-block cluster of four CTAs = one (sequence, KV head) and a run
+// of up to nbb consecutive RoPE buckets (one bucket without RoPE); CTA r owns
 // channels 32r..32r+31 (key group r).  It stages its 32 columns of A^{-T}
-// (32 KB) with one cp.async burst and runs the fixed-order fp64 fma chains
-// q'[h][j] of its channels, then their pooled energies.  After a cluster
-// barrier every CTA reads the four energy blocks through distributed shared
-// memory and makes the same exact, order-free choice (each candidate counts
-// the channels that beat it), so no CTA waits for another's decision; each
-// writes the outputs of its own channels: their list positions (a ballot
-// prefix sum over the 128 flags), q' in fp32 and its group's zero-point sum.
+// (32 KB) once with one cp.async burst, moves the query into each bucket's
+// frame, and runs the fixed-order fp64 fma chains q'_b[h][j] of its channels
+// for every bucket (four independent chains per thread at a time), then their
+// pooled energies.  After a cluster barrier every CTA reads the four energy
+// blocks of every bucket through distributed shared memory and makes the same
+// exact, order-free choice (each candidate counts the channels that beat it),
+// so no CTA waits for another's decision; each writes the outputs of its own
+// channels: their list positions (prefix counts of per-bucket 128-bit
+// masks), q' in fp32 and its group's zero-point sum.  Buckets past the
+// sequence's length (other than bucket 0) are skipped.
 #include "kvq_internal.cuh"
 
 #include <cooperative_groups.h>
@@ -34,30 +36,53 @@ namespace cg = cooperative_groups;
 
 constexpr int kThreads = 256;
 constexpr int kCtas = kNG;                 // CTAs per cluster, one per key group
+constexpr int kMaxGNbb = 32;               // heads x buckets of one cluster
+
+// Dynamic shared memory of one CTA: doubles As[128][32], qin[g][128],
+// qr[nbb][g][128] (the query in each bucket's frame), qp[nbb][g][32],
+// e2own[nbb][32], e2s[nbb][128]; then ints sel[nbb][128] and words
+// mask[nbb][4].
+struct SelLayout {
+    int g, nbb;
+    __host__ __device__ int off_qin() const { return kD * kGroup; }
+    __host__ __device__ int off_qr() const { return off_qin() + g * kD; }
+    __host__ __device__ int off_qp() const { return off_qr() + nbb * g * kD; }
+    __host__ __device__ int off_e2own() const { return off_qp() + nbb * g * kGroup; }
+    __host__ __device__ int off_e2s() const { return off_e2own() + nbb * kGroup; }
+    __host__ __device__ int end_doubles() const { return off_e2s() + nbb * kD; }
+    __host__ __device__ size_t bytes() const {
+        return (size_t)end_doubles() * sizeof(double) + (size_t)nbb * (kD + 4) * sizeof(int);
+    }
+};
 
 template <typename Tin>
 __global__ void __cluster_dims__(kCtas, 1, 1) __launch_bounds__(kThreads)
 select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, const double *__restrict__ delta,
               int Hq, int Hkv, int g, int k, int32_t *__restrict__ idx, float *__restrict__ qsel,
               float *__restrict__ qgsum, int ng, const int32_t *__restrict__ seq_len,
-              const double *__restrict__ rope, int nbk, int w) {
-    extern __shared__ __align__(16) double sm[];   // As[128][32], qin[g][128], qp[g][32]
+              const double *__restrict__ rope, int nbk, int w, int nbb) {
+    extern __shared__ __align__(16) double sm[];
+    const SelLayout L{g, nbb};
     double *As = sm;
-    double *qin = sm + kD * kGroup;
-    double *qp = qin + (size_t)g * kD;
-    __shared__ double e2own[kGroup];
-    __shared__ double e2s[kD];
-    __shared__ int rank_part[2][kD];
-    __shared__ int sel_s[kD];
-    __shared__ int warp_cnt[4];
+    double *qin = sm + L.off_qin();
+    double *qr = rope ? sm + L.off_qr() : qin;       // without RoPE the one "bucket" is the query itself
+    double *qp = sm + L.off_qp();
+    double *e2own = sm + L.off_e2own();
+    double *e2s = sm + L.off_e2s();
+    int *sel = reinterpret_cast<int *>(sm + L.end_doubles());
+    uint32_t *mask = reinterpret_cast<uint32_t *>(sel + nbb * kD);
 
     cg::cluster_group cluster = cg::this_cluster();
-    const int r = (int)cluster.block_rank();       // = blockIdx.x % 4
-    const int bk = blockIdx.x / kCtas;              // RoPE bucket (0 without buckets)
+    const int r = (int)cluster.block_rank();        // = blockIdx.x % 4
+    const int b0 = (blockIdx.x / kCtas) * nbb;       // first bucket of the cluster
     const int h = blockIdx.y, b = blockIdx.z, t = threadIdx.x;
     const int lane = t & 31, warp = t >> 5;
     const size_t qrow0 = (size_t)b * Hq + (size_t)h * g;
-    if (bk > 0 && (size_t)bk * w >= (size_t)max(seq_len[b], 0)) return;   // the whole cluster
+    // buckets that hold a token (bucket 0 always): a prefix of the buckets
+    const int len = max(seq_len[b], 0);
+    const int used = rope ? max(1, (int)(((long long)len + w - 1) / w)) : 1;
+    const int nb = min(min(nbb, nbk - b0), used - b0);   // buckets of this cluster to do
+    if (nb <= 0) return;                                // the whole cluster
 
     // columns 32r..32r+31 of A^{-T} for this KV head: 128 rows of 256 bytes
     const double *Ai = Ainvt + (size_t)h * kD * kD + r * kGroup;
@@ -67,98 +92,159 @@ select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, const
     }
     cp_async_commit();
     for (int e = t; e < g * kD; e += kThreads) qin[e] = in_to_double(q[qrow0 * kD + e]);
-    cp_async_wait<0>();
     __syncthreads();
     if (rope) {
-        // q T_b: channel pairs (i, i + 64) rotated back by the anchor's angle
-        const double2 *cs = reinterpret_cast<const double2 *>(rope) + (size_t)bk * (kD / 2);
-        for (int e = t; e < g * (kD / 2); e += kThreads) {
-            const int hl = e / (kD / 2), i = e % (kD / 2);
-            rope_unanchor_pair(qin[hl * kD + i], qin[hl * kD + i + kD / 2], __ldg(cs + i));
+        // q T_b for each bucket: channel pairs (i, i + 64) rotated back by the anchor's angle
+        const double2 *cs = reinterpret_cast<const double2 *>(rope);
+        for (int e = t; e < nb * g * (kD / 2); e += kThreads) {
+            const int bi = e / (g * (kD / 2)), rem = e % (g * (kD / 2));
+            const int hl = rem / (kD / 2), i = rem % (kD / 2);
+            double x0 = qin[hl * kD + i], x1 = qin[hl * kD + i + kD / 2];
+            rope_unanchor_pair(x0, x1, __ldg(cs + (size_t)(b0 + bi) * (kD / 2) + i));
+            qr[(bi * g + hl) * kD + i] = x0;
+            qr[(bi * g + hl) * kD + i + kD / 2] = x1;
         }
-        __syncthreads();
     }
+    cp_async_wait<0>();
+    __syncthreads();
 
-    // q'[hl][j] = sum_c q[hl][c] Ainvt[c][j], fma chain c = 0..127 from 0.0
-    for (int hl = warp; hl < g; hl += kThreads / 32) {
-        double acc = 0.0;
-#pragma unroll 16
-        for (int c = 0; c < kD; c++) acc = fma(qin[hl * kD + c], As[c * kGroup + lane], acc);
-        qp[hl * kGroup + lane] = acc;
+    // q'_b[hl][j] = sum_c qr_b[hl][c] Ainvt[c][j], fma chain c = 0..127 from
+    // 0.0; task (bi, hl, lane), four independent chains per thread at a time
+    const int ntask = nb * g * kGroup;
+    for (int t0 = t; t0 < ntask; t0 += 4 * kThreads) {
+        double acc[4] = {0.0, 0.0, 0.0, 0.0};
+        const double *qrow[4];
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            const int task = min(t0 + u * kThreads, ntask - 1);
+            qrow[u] = qr + (task / kGroup) * kD;          // row (bi * g + hl)
+        }
+#pragma unroll 8
+        for (int c = 0; c < kD; c++) {
+            const double a = As[c * kGroup + lane];
+#pragma unroll
+            for (int u = 0; u < 4; u++) acc[u] = fma(qrow[u][c], a, acc[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            const int task = t0 + u * kThreads;
+            if (task < ntask) qp[task] = acc[u];          // [bi][hl][lane]
+        }
     }
     __syncthreads();
-    // e_j^2, fma chain over heads ascending from 0.0; with a diagonal
-    // refinement D, of the base queries q'_{h,j} / delta_j
-    if (t < kGroup) {
-        const double dj = delta ? delta[(size_t)h * kD + r * kGroup + t] : 1.0;
-        double e = 0.0;
+    // e_j^2 per bucket, fma chain over heads ascending from 0.0; with a
+    // diagonal refinement D, of the base queries q'_{h,j} / delta_j
+    for (int e = t; e < nb * kGroup; e += kThreads) {
+        const int bi = e / kGroup, l = e % kGroup;
+        const double dj = delta ? delta[(size_t)h * kD + r * kGroup + l] : 1.0;
+        double en = 0.0;
         for (int hl = 0; hl < g; hl++) {
-            const double u = delta ? qp[hl * kGroup + t] / dj : qp[hl * kGroup + t];
-            e = fma(u, u, e);
+            const double v = qp[(bi * g + hl) * kGroup + l];
+            const double u = delta ? v / dj : v;
+            en = fma(u, u, en);
         }
-        e2own[t] = e;
+        e2own[e] = en;
     }
     cluster.sync();                                // every CTA's energies are ready
-    if (t < kD) {
-        const double *src = cluster.map_shared_rank(e2own, t / kGroup);
-        e2s[t] = src[t % kGroup];
+    for (int e = t; e < nb * kD; e += kThreads) {
+        const int bi = e / kD, j = e % kD;
+        const double *src = cluster.map_shared_rank(e2own, j / kGroup);
+        e2s[e] = src[bi * kGroup + j % kGroup];
     }
     __syncthreads();
-    // rank of candidate j >= 1 among channels 1..127, counted in two halves
-    {
-        const int j = t & (kD - 1), part = t >> 7;
-        // energies are >= 0, so their bit patterns order like their values
-        const unsigned long long e = __double_as_longlong(e2s[j]);
-        int rk = 0;
-        const int i0 = part == 0 ? 1 : 64, i1 = part == 0 ? 64 : kD;
-#pragma unroll 4
-        for (int i = i0; i < i1; i++) {
-            const unsigned long long ei = __double_as_longlong(e2s[i]);
-            rk += (ei > e) || (ei == e && i < j);
+    // per bucket: sort the channels by (energy descending, index ascending)
+    // with a bitonic network -- channel 0 last (key 0; every other channel's
+    // key is its energy's bit pattern + 1, and energies are >= 0, so bit
+    // patterns order like values) -- then keep channel 0 and the first k-1.
+    // (sort keys in the rotated queries' place, free since the chains ended;
+    // e2own stays: the other CTAs of the cluster read it)
+    unsigned long long *skey = reinterpret_cast<unsigned long long *>(sm + L.off_qr());   // [nb][128]
+    static_assert(sizeof(double) == sizeof(unsigned long long), "a key per double");
+    int *sj = sel;                                                                          // [nb][128]
+    for (int e = t; e < nb * kD; e += kThreads) {
+        const int j = e % kD;
+        skey[e] = j == 0 ? 0ull : (unsigned long long)__double_as_longlong(e2s[e]) + 1ull;
+        sj[e] = j;
+    }
+    __syncthreads();
+    for (int size = 2; size <= kD; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int e = t; e < nb * (kD / 2); e += kThreads) {
+                const int bi = e / (kD / 2), p = e % (kD / 2);
+                const int i = 2 * stride * (p / stride) + (p % stride), l = i + stride;
+                unsigned long long *kb = skey + bi * kD;
+                int *jb = sj + bi * kD;
+                const unsigned long long ki = kb[i], kl = kb[l];
+                const int ji = jb[i], jl = jb[l];
+                const bool l_first = (kl > ki) || (kl == ki && jl < ji);      // l belongs before i
+                if (((i & size) == 0) == l_first) {
+                    kb[i] = kl; kb[l] = ki;
+                    jb[i] = jl; jb[l] = ji;
+                }
+            }
+            __syncthreads();
         }
-        rank_part[part][j] = rk;
+    }
+    // keep flags into e2s's place: [nb][128] ints
+    int *keep = reinterpret_cast<int *>(e2s);
+    for (int e = t; e < nb * kD; e += kThreads) keep[e] = (e % kD) == 0;
+    __syncthreads();
+    for (int e = t; e < nb * kD; e += kThreads)
+        if (e % kD < k - 1) keep[(e / kD) * kD + sj[e]] = 1;
+    __syncthreads();
+    for (int e = t; e < nb * kD; e += kThreads) sel[e] = keep[e];
+    __syncthreads();
+    // 128-bit keep masks per bucket, one 32-bit word per warp ballot
+    for (int wd = warp; wd < nb * 4; wd += kThreads / 32) {
+        const unsigned m = __ballot_sync(0xffffffffu, sel[wd * 32 + lane] != 0);
+        if (lane == 0) mask[wd] = m;
     }
     __syncthreads();
-    int pos = -1;
-    if (t < kD) {
-        const bool sel = (t == 0) || (rank_part[0][t] + rank_part[1][t] < k - 1);
-        sel_s[t] = sel;
-        const unsigned ballot = __ballot_sync(0xffffffffu, sel);
-        if (lane == 0) warp_cnt[warp] = __popc(ballot);
-        if (sel) pos = (int)__popc(ballot & ((1u << lane) - 1u));
-    }
-    __syncthreads();
-    // this CTA's channels are t = 32r..32r+31 (warp r)
-    if (warp == r && pos >= 0) {
-        for (int w = 0; w < r; w++) pos += warp_cnt[w];
-        idx[(((size_t)b * Hkv + h) * nbk + bk) * k + pos] = t;
-        for (int hl = 0; hl < g; hl++) qsel[((qrow0 + hl) * nbk + bk) * k + pos] = (float)qp[hl * kGroup + lane];
+    // this CTA's channels 32r..32r+31: list position = kept channels below
+    for (int e = t; e < nb * kGroup; e += kThreads) {
+        const int bi = e / kGroup, l = e % kGroup, c = r * kGroup + l;
+        if (!sel[bi * kD + c]) continue;
+        int pos = __popc(mask[bi * 4 + r] & ((1u << l) - 1u));
+        for (int m = 0; m < r; m++) pos += __popc(mask[bi * 4 + m]);
+        const int bk = b0 + bi;
+        idx[(((size_t)b * Hkv + h) * nbk + bk) * k + pos] = c;
+        for (int hl = 0; hl < g; hl++)
+            qsel[((qrow0 + hl) * nbk + bk) * k + pos] = (float)qp[(bi * g + hl) * kGroup + l];
     }
     // zero-point sum of each key group (channel 0 is bf16, not in group 0),
     // kept channels ascending from 0.0: groups of 32 -- CTA r sums group r;
     // one grid per token -- CTA 0 sums all channels (reading the others' q'
     // through distributed shared memory) into entry 0, the rest are 0
     if (ng == kNG) {
-        for (int hl = t; hl < g; hl += kThreads) {
+        for (int e = t; e < nb * g; e += kThreads) {
+            const int bi = e / g, hl = e % g;
             double s = 0.0;
-            for (int c = (r == 0 ? 1 : 0); c < kGroup; c++)
-                if (sel_s[r * kGroup + c]) s += qp[hl * kGroup + c];
-            qgsum[((qrow0 + hl) * nbk + bk) * kNG + r] = (float)s;
+            for (int l = (r == 0 ? 1 : 0); l < kGroup; l++)
+                if (sel[bi * kD + r * kGroup + l]) s += qp[(bi * g + hl) * kGroup + l];
+            qgsum[((qrow0 + hl) * nbk + b0 + bi) * kNG + r] = (float)s;
         }
     } else if (r == 0) {
-        const double *pq[kCtas];
-#pragma unroll
-        for (int rr = 0; rr < kCtas; rr++) pq[rr] = cluster.map_shared_rank(qp, rr);
-        for (int hl = t; hl < g; hl += kThreads) {
+        // all 128 channels of q' into local memory first (the rotated
+        // queries are no longer needed), one parallel pass over the peers
+        double *qall = sm + L.off_qr();                       // [nb][g][128]
+        for (int e = t; e < nb * g * kD; e += kThreads) {
+            const int row = e / kD, c = e % kD;
+            qall[e] = cluster.map_shared_rank(qp, c / kGroup)[row * kGroup + c % kGroup];
+        }
+        __syncthreads();
+        for (int e = t; e < nb * g; e += kThreads) {
+            const int bi = e / g, hl = e % g;
+            const double *qrow = qall + (bi * g + hl) * kD;
             double s = 0.0;
             for (int c = 1; c < kD; c++)
-                if (sel_s[c]) s += pq[c / kGroup][hl * kGroup + c % kGroup];
-            qgsum[((qrow0 + hl) * nbk + bk) * kNG] = (float)s;
+                if (sel[bi * kD + c]) s += qrow[c];
+            float *o = qgsum + ((qrow0 + hl) * nbk + b0 + bi) * kNG;
+            o[0] = (float)s;
 #pragma unroll
-            for (int gr = 1; gr < kNG; gr++) qgsum[((qrow0 + hl) * nbk + bk) * kNG + gr] = 0.f;
+            for (int gr = 1; gr < kNG; gr++) o[gr] = 0.f;
         }
     }
-    cluster.sync();                                // keep e2own alive until all have read it
+    cluster.sync();                                // keep e2own and qp alive until all have read them
 }
 
 }  // namespace
@@ -166,25 +252,28 @@ select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, const
 cudaError_t launch_select(const kvq_cache &c, const void *q, int dtype, int Hq, const double *Ainvt,
                           const double *delta, int k, int32_t *idx, float *qsel, float *qgsum, cudaStream_t st) {
     const int g = Hq / c.n_kv_heads;
-    const size_t smem = (size_t)(kD * kGroup + g * kD + g * kGroup) * sizeof(double);
-    constexpr int kMaxSmem = (kD * kGroup + 32 * kD + 32 * kGroup) * (int)sizeof(double);   // g <= 32
-    static std::atomic<uint64_t> done_f32{0}, done_bf16{0};
     const int nbk = buckets_of(c);
-    dim3 grid((unsigned)(kCtas * nbk), (unsigned)c.n_kv_heads, (unsigned)c.batch);
     const double *rope = c.bucket > 0 ? c.rope : nullptr;
+    const int nbb = rope ? std::min(nbk, std::max(1, kMaxGNbb / g)) : 1;     // buckets per cluster
+    const size_t smem = SelLayout{g, nbb}.bytes();
+    // the largest layout any call can ask for (g <= 32, g * nbb <= 32 or nbb = 1)
+    size_t max_smem = 0;
+    for (int gg = 1; gg <= 32; gg++) max_smem = std::max(max_smem, SelLayout{gg, std::max(1, kMaxGNbb / gg)}.bytes());
+    static std::atomic<uint64_t> done_f32{0}, done_bf16{0};
+    dim3 grid((unsigned)(kCtas * ((nbk + nbb - 1) / nbb)), (unsigned)c.n_kv_heads, (unsigned)c.batch);
     cudaError_t e;
     if (dtype == KVQ_DTYPE_F32) {
-        e = set_smem_once(select_kernel<float>, kMaxSmem, done_f32);
+        e = set_smem_once(select_kernel<float>, (int)max_smem, done_f32);
         if (e != cudaSuccess) return e;
         select_kernel<float><<<grid, kThreads, smem, st>>>(static_cast<const float *>(q), Ainvt, delta, Hq,
                                                            c.n_kv_heads, g, k, idx, qsel, qgsum, groups_of(c),
-                                                           c.seq_len, rope, nbk, c.bucket);
+                                                           c.seq_len, rope, nbk, c.bucket, nbb);
     } else {
-        e = set_smem_once(select_kernel<uint16_t>, kMaxSmem, done_bf16);
+        e = set_smem_once(select_kernel<uint16_t>, (int)max_smem, done_bf16);
         if (e != cudaSuccess) return e;
         select_kernel<uint16_t><<<grid, kThreads, smem, st>>>(static_cast<const uint16_t *>(q), Ainvt, delta, Hq,
                                                               c.n_kv_heads, g, k, idx, qsel, qgsum, groups_of(c),
-                                                              c.seq_len, rope, nbk, c.bucket);
+                                                              c.seq_len, rope, nbk, c.bucket, nbb);
     }
     return cudaGetLastError();
 }
