@@ -362,6 +362,17 @@ int kvq_decode_attn_static(const kvq_cache *cache, int n_q_heads, const int32_t 
                            const float *qsel, const float *qgsum, int k, float *out,
                            kvq_stream_t stream);
 
+/*
+ * kvq_copy_async -- stream-ordered copy of `bytes` bytes between caller
+ * buffers, device memory or pinned host memory, the direction taken from the
+ * pointers (unified addressing).  For moving a decode step's packed inputs in
+ * and its result out as one transfer each; with pinned host buffers the copy
+ * can be recorded into a CUDA graph together with the step.  The paper has no
+ * counterpart; this is a serving convenience.
+ * Errors: KVQ_ERR_ARG (null pointer with bytes > 0), KVQ_ERR_CUDA.
+ */
+int kvq_copy_async(void *dst, const void *src, size_t bytes, kvq_stream_t stream);
+
 /* Copy the device status flags (word 0) into *flags (synchronises the stream).
  * KVQ_ERR_ARG on null pointers, KVQ_ERR_CUDA on a failed copy. */
 int kvq_read_status(const kvq_cache *cache, uint32_t *flags, kvq_stream_t stream);

@@ -208,6 +208,12 @@ int kvq_bf16_decode_attn(const void *q, const void *K, const void *V, int B, int
     return cuda_status(launch_bf16_decode(q, K, V, B, Hq, Hkv, N, out, ws, S, (cudaStream_t)stream));
 }
 
+int kvq_copy_async(void *dst, const void *src, size_t bytes, kvq_stream_t stream) {
+    if (bytes == 0) return KVQ_OK;
+    if (!dst || !src) return KVQ_ERR_ARG;
+    return cuda_status(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDefault, (cudaStream_t)stream));
+}
+
 int kvq_read_status(const kvq_cache *c, uint32_t *flags, kvq_stream_t stream) {
     if (!c || !c->status || !flags) return KVQ_ERR_ARG;
     cudaStream_t s = (cudaStream_t)stream;

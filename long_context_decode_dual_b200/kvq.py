@@ -58,7 +58,7 @@ EXPORTS = (
     "kvq_select_channels", "kvq_decode_workspace", "kvq_decode_attn",
     "kvq_bf16_decode_workspace", "kvq_bf16_decode_attn", "kvq_read_status",
     "kvq_status_string", "kvq_version", "kvq_decode_static_scratch_bytes",
-    "kvq_decode_attn_static", "kvq_decode_step", "kvq_num_buckets",
+    "kvq_decode_attn_static", "kvq_decode_step", "kvq_num_buckets", "kvq_copy_async",
 )
 
 
@@ -91,6 +91,7 @@ def lib() -> ctypes.CDLL:
             "kvq_decode_attn_static": (I, [C, I, P, P, P, I, P, P]),
             "kvq_decode_step": (I, [C, P, P, P, I, I, I, P, P, P, ctypes.c_float, P, P, P, P, P, S, P]),
             "kvq_num_buckets": (I, [C]),
+            "kvq_copy_async": (I, [P, P, S, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -371,6 +372,29 @@ def read_status(cache: KVCache, stream=None) -> int:
     return int(flags.value)
 
 
+def copy_async(dst: torch.Tensor, src: torch.Tensor, stream=None) -> None:
+    """kvq_copy_async: stream-ordered copy of src's bytes into dst (device or
+    pinned host tensors, same byte size); capturable into a CUDA graph."""
+    nbytes = src.numel() * src.element_size()
+    assert dst.numel() * dst.element_size() == nbytes and dst.is_contiguous() and src.is_contiguous()
+    _check("kvq_copy_async", lib().kvq_copy_async(_ptr(dst), _ptr(src), nbytes, _stream(stream)))
+
+
+def _packed(n_elems, dtype: torch.dtype, device, pin: bool = False):
+    """One byte buffer holding tensors of the given element counts, each at a
+    256-byte aligned offset; returns (buffer, views)."""
+    esize = torch.tensor([], dtype=dtype).element_size()
+    offs, total = [], 0
+    for n in n_elems:
+        offs.append(total)
+        total += (n * esize + 255) // 256 * 256
+    buf = torch.zeros(total, dtype=torch.uint8, device=device)
+    if pin:
+        buf = buf.pin_memory()
+    views = [buf[o:o + n * esize].view(dtype) for o, n in zip(offs, n_elems)]
+    return buf, views
+
+
 class DecodeStep:
     """One decode step of the path -- append the new token, select channels,
     decode -- on static device buffers, replayable as a CUDA graph.
@@ -381,8 +405,12 @@ class DecodeStep:
     call; otherwise it is kvq_append, kvq_select_channels and kvq_decode_attn.
     :meth:`capture` records the step once (after at least one eager
     :meth:`run`, so every kernel is loaded); later runs replay the graph.
-    :meth:`run_host` copies the inputs from (pinned) host tensors and the
-    output back, around the same step.
+
+    The three inputs are views of one device buffer, and ``q_host``,
+    ``k_host``, ``v_host`` / ``out_host`` of pinned host buffers with the same
+    layout: :meth:`run_host` moves the inputs in with one copy, runs the step
+    and moves the result out with one copy -- all three in one graph replay
+    once :meth:`capture` has run.
     """
 
     def __init__(self, cache: KVCache, A: torch.Tensor, Ainvt: torch.Tensor, sparsity: float,
@@ -393,15 +421,28 @@ class DecodeStep:
         self.cache, self.A, self.Ainvt, self.sparsity = cache, A, Ainvt, float(sparsity)
         self.delta = delta
         self.fused = fused
-        self.q = torch.zeros(B, n_q_heads, HEAD_DIM, dtype=dtype, device=dev)
-        self.k_new = torch.zeros(B, Hkv, 1, HEAD_DIM, dtype=dtype, device=dev)
-        self.v_new = torch.zeros(B, Hkv, 1, HEAD_DIM, dtype=dtype, device=dev)
+        shapes = [(B, n_q_heads, HEAD_DIM), (B, Hkv, 1, HEAD_DIM), (B, Hkv, 1, HEAD_DIM)]
+        counts = [B * n_q_heads * HEAD_DIM, B * Hkv * HEAD_DIM, B * Hkv * HEAD_DIM]
+        self._in_dev, views = _packed(counts, dtype, dev)
+        self.q, self.k_new, self.v_new = (v.view(*sh) for v, sh in zip(views, shapes))
+        self._in_host, hviews = _packed(counts, dtype, "cpu", pin=True)
+        self.q_host, self.k_host, self.v_host = (v.view(*sh) for v, sh in zip(hviews, shapes))
         self.k = num_selected(sparsity)
         self.sel = alloc_selection(cache, n_q_heads, self.k, dev)
         self.out = torch.empty(B, n_q_heads, HEAD_DIM, dtype=torch.float32, device=dev)
+        self.out_host = torch.empty(B, n_q_heads, HEAD_DIM, dtype=torch.float32).pin_memory()
         self.ws = alloc_workspace(decode_workspace_bytes(cache, n_q_heads, self.k), dev)
         self.graph = None
+        self.host_graph = None         # inputs in, the step, result out
         self.decode_events = None      # optional (start, end) events around the decode call
+
+    @property
+    def h2d_bytes(self) -> int:
+        return self._in_host.numel()
+
+    @property
+    def d2h_bytes(self) -> int:
+        return self.out_host.numel() * 4
 
     def _pre(self):
         if not self.fused:
@@ -415,6 +456,12 @@ class DecodeStep:
         else:
             decode_attn(self.cache, self.sel, out=self.out, ws=self.ws)
 
+    def _host_step(self):
+        copy_async(self._in_dev, self._in_host)
+        self._pre()
+        self._decode()
+        copy_async(self.out_host, self.out)
+
     def time_decode(self) -> None:
         """Record timing events around the decode call (the whole fused step)
         of every later run."""
@@ -422,8 +469,9 @@ class DecodeStep:
 
     def capture(self) -> None:
         """Record the step as CUDA graphs: append + select (unfused only) and
-        the decode call; the decode timing events, if any, are recorded
-        between the replays."""
+        the decode call, the decode timing events, if any, recorded between
+        the replays; and the whole host step (inputs in, the step, result
+        out) as one more graph."""
         pre = None
         if not self.fused:
             pre = torch.cuda.CUDAGraph()
@@ -433,6 +481,10 @@ class DecodeStep:
         with torch.cuda.graph(dec):
             self._decode()
         self.graph = (pre, dec)
+        hg = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(hg):
+            self._host_step()
+        self.host_graph = hg
 
     def run(self) -> torch.Tensor:
         ev = self.decode_events
@@ -451,11 +503,18 @@ class DecodeStep:
             ev[1].record()
         return self.out
 
-    def run_host(self, q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tensor,
-                 out_host: torch.Tensor) -> torch.Tensor:
-        self.q.copy_(q_host, non_blocking=True)
-        self.k_new.copy_(k_host, non_blocking=True)
-        self.v_new.copy_(v_host, non_blocking=True)
-        self.run()
-        out_host.copy_(self.out, non_blocking=True)
-        return out_host
+    def run_host(self, q_host: Optional[torch.Tensor] = None, k_host: Optional[torch.Tensor] = None,
+                 v_host: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """One step from host inputs to a host result: the inputs (given as
+        host tensors, or already written into ``q_host`` / ``k_host`` /
+        ``v_host``) go in with one copy and the result comes back into
+        ``out_host`` (returned) with one copy, stream-ordered on the current
+        stream; synchronise before reading it."""
+        for src, dst in ((q_host, self.q_host), (k_host, self.k_host), (v_host, self.v_host)):
+            if src is not None and src.data_ptr() != dst.data_ptr():
+                dst.copy_(src)
+        if self.host_graph is not None:
+            self.host_graph.replay()
+        else:
+            self._host_step()
+        return self.out_host

@@ -47,6 +47,8 @@ def test_host_side_queries():
     assert L.kvq_cache_bytes(ctypes.byref(kvq.CacheDesc(2, 8, 128, 64, 2, 256, 0, 0, 0))) == 0
     assert L.kvq_cache_bytes(ctypes.byref(kvq.CacheDesc(2, 8, 128, 32, 2, 256, 0, 0, 0, 1000, 25))) == 0
     assert kvq.status_string(-3) == "capacity exceeded"
+    assert L.kvq_copy_async(None, None, 0, None) == 0                 # nothing to copy
+    assert L.kvq_copy_async(None, 8, 16, None) == -1
 
 
 def test_validation_rejects_before_launch():
