@@ -20,8 +20,8 @@
 // for every bucket (four independent chains per thread at a time), then their
 // pooled energies.  After a cluster barrier every CTA reads the four energy
 // blocks of every bucket through distributed shared memory and makes the same
-// exact, order-free choice (each candidate counts the channels that beat it),
-// so no CTA waits for another's decision; each writes the outputs of its own
+// exact choice (a bitonic sort per bucket, one warp each, in registers), so
+// no CTA waits for another's decision; each writes the outputs of its own
 // channels: their list positions (prefix counts of per-bucket 128-bit
 // masks), q' in fp32 and its group's zero-point sum.  Buckets past the
 // sequence's length (other than bucket 0) are skipped.
@@ -152,52 +152,69 @@ select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, const
         e2s[e] = src[bi * kGroup + j % kGroup];
     }
     __syncthreads();
-    // per bucket: sort the channels by (energy descending, index ascending)
-    // with a bitonic network -- channel 0 last (key 0; every other channel's
-    // key is its energy's bit pattern + 1, and energies are >= 0, so bit
-    // patterns order like values) -- then keep channel 0 and the first k-1.
-    // (sort keys in the rotated queries' place, free since the chains ended;
-    // e2own stays: the other CTAs of the cluster read it)
-    unsigned long long *skey = reinterpret_cast<unsigned long long *>(sm + L.off_qr());   // [nb][128]
-    static_assert(sizeof(double) == sizeof(unsigned long long), "a key per double");
-    int *sj = sel;                                                                          // [nb][128]
-    for (int e = t; e < nb * kD; e += kThreads) {
-        const int j = e % kD;
-        skey[e] = j == 0 ? 0ull : (unsigned long long)__double_as_longlong(e2s[e]) + 1ull;
-        sj[e] = j;
-    }
-    __syncthreads();
-    for (int size = 2; size <= kD; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int e = t; e < nb * (kD / 2); e += kThreads) {
-                const int bi = e / (kD / 2), p = e % (kD / 2);
-                const int i = 2 * stride * (p / stride) + (p % stride), l = i + stride;
-                unsigned long long *kb = skey + bi * kD;
-                int *jb = sj + bi * kD;
-                const unsigned long long ki = kb[i], kl = kb[l];
-                const int ji = jb[i], jl = jb[l];
-                const bool l_first = (kl > ki) || (kl == ki && jl < ji);      // l belongs before i
-                if (((i & size) == 0) == l_first) {
-                    kb[i] = kl; kb[l] = ki;
-                    jb[i] = jl; jb[l] = ji;
+    // per bucket, one warp: sort the channels by (energy descending, index
+    // ascending) with a bitonic network held in registers (element
+    // e = 32 r + lane in register r; partners closer than 32 through
+    // shuffles, the others inside the thread) -- channel 0 last (key 0; every
+    // other channel's key is its energy's bit pattern + 1, and energies are
+    // >= 0, so bit patterns order like values) -- then keep channel 0 and the
+    // first k-1, and the per-bucket 128-bit keep masks by ballots.
+    for (int bi = warp; bi < nb; bi += kThreads / 32) {
+        unsigned long long key[4];
+        int jj[4];
+#pragma unroll
+        for (int r4 = 0; r4 < 4; r4++) {
+            const int j = r4 * 32 + lane;
+            key[r4] = j == 0 ? 0ull : (unsigned long long)__double_as_longlong(e2s[bi * kD + j]) + 1ull;
+            jj[r4] = j;
+        }
+#pragma unroll
+        for (int size = 2; size <= kD; size <<= 1) {
+#pragma unroll
+            for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                if (stride >= 32) {
+                    const int rs = stride / 32;
+#pragma unroll
+                    for (int ra = 0; ra < 4; ra++) {
+                        if (ra & rs) continue;                   // each pair once, from its lower register
+                        const int rb = ra | rs;
+                        const bool up = ((ra * 32 + lane) & size) == 0;
+                        const bool b_first = (key[rb] > key[ra]) || (key[rb] == key[ra] && jj[rb] < jj[ra]);
+                        if (b_first == up) {
+                            const unsigned long long tk = key[ra];
+                            key[ra] = key[rb];
+                            key[rb] = tk;
+                            const int tj = jj[ra];
+                            jj[ra] = jj[rb];
+                            jj[rb] = tj;
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int r4 = 0; r4 < 4; r4++) {
+                        const int e = r4 * 32 + lane;
+                        const unsigned long long pk = __shfl_xor_sync(0xffffffffu, key[r4], stride);
+                        const int pj = __shfl_xor_sync(0xffffffffu, jj[r4], stride);
+                        const bool low = (e & stride) == 0, up = (e & size) == 0;
+                        const bool p_first = (pk > key[r4]) || (pk == key[r4] && pj < jj[r4]);
+                        // the lower element of a rising pair takes the first of the
+                        // two, the upper one the second; reversed in a falling pair
+                        if ((low == up) ? p_first : !p_first) {
+                            key[r4] = pk;
+                            jj[r4] = pj;
+                        }
+                    }
                 }
             }
-            __syncthreads();
         }
-    }
-    // keep flags into e2s's place: [nb][128] ints
-    int *keep = reinterpret_cast<int *>(e2s);
-    for (int e = t; e < nb * kD; e += kThreads) keep[e] = (e % kD) == 0;
-    __syncthreads();
-    for (int e = t; e < nb * kD; e += kThreads)
-        if (e % kD < k - 1) keep[(e / kD) * kD + sj[e]] = 1;
-    __syncthreads();
-    for (int e = t; e < nb * kD; e += kThreads) sel[e] = keep[e];
-    __syncthreads();
-    // 128-bit keep masks per bucket, one 32-bit word per warp ballot
-    for (int wd = warp; wd < nb * 4; wd += kThreads / 32) {
-        const unsigned m = __ballot_sync(0xffffffffu, sel[wd * 32 + lane] != 0);
-        if (lane == 0) mask[wd] = m;
+#pragma unroll
+        for (int r4 = 0; r4 < 4; r4++) sel[bi * kD + jj[r4]] = (jj[r4] == 0) || (r4 * 32 + lane < k - 1);
+        __syncwarp();
+#pragma unroll
+        for (int w4 = 0; w4 < 4; w4++) {
+            const unsigned m = __ballot_sync(0xffffffffu, sel[bi * kD + w4 * 32 + lane] != 0);
+            if (lane == 0) mask[bi * 4 + w4] = m;
+        }
     }
     __syncthreads();
     // this CTA's channels 32r..32r+31: list position = kept channels below
