@@ -257,7 +257,7 @@ def run_reference(args):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_dict(wl, k, protect),
         "cpu_baseline": {"value": tokens_per_s, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "host": host_cpu()},
         "e2e": {"value": tokens_per_s, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -279,6 +279,20 @@ def config_dict(wl: W.Workload, k: int, protect=(0, 0)):
     if wl.bucket:
         d["rope_bucket"] = wl.bucket
     return d
+
+
+def host_cpu() -> dict:
+    """The host the CPU baseline ran on: logical CPUs and model name."""
+    model = ""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "model": model}
 
 
 def format_overrides(args) -> dict:
@@ -509,7 +523,8 @@ def run_ours(args):
     cpu = None
     if args.cpu_baseline and world == 1:
         cv, ct, sample = oracle_sample(wl.with_(n_steps=8), 6, budget_s=25.0, protect=protect)
-        cpu = {"value": cv, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample}
+        cpu = {"value": cv, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample,
+               "host": host_cpu()}
 
     csum = clocks.summary()
     line = {
@@ -526,6 +541,9 @@ def run_ours(args):
         "step_launch": "cuda graph" if args.graph else "eager",
         "decode_alg_bytes": statistics.mean(alg_bytes),
         "prefill_ms": prefill_ms,
+        # the prefill reads K and V once and writes the pages (and slots)
+        "prefill_gbs": (Kd.numel() * Kd.element_size() * 2 + cache.pages.numel()) / (prefill_ms * 1e-3) / 1e9,
+        "seq_tokens_per_s": world * B * statistics.mean(tokens) / (B * Hkv) / (total_ms / args.steps * 1e-3),
         "gpu_launches": launches_per_step * args.steps,
         "clocks": csum,
         "e2e": e2e,
