@@ -695,10 +695,11 @@ __device__ __forceinline__ void tier_cta(MmaShared &sh, const uint8_t *slots, in
 }
 
 // ---------------------------------------------------------------- decode
-// With RoPE buckets (w_pages > 0 pages each, nbk entries per selection
+// With RoPE buckets (BK; w_pages > 0 pages each, nbk entries per selection
 // array) each split reads, per bucket its pages fall in, that bucket's
 // channel choice; the tier CTAs read each protected position's own bucket's.
-template <int NG>
+// Without buckets the segment machinery is compiled out.
+template <int NG, bool BK>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len, int Hkv,
                   int NB, int Hq, const int32_t *__restrict__ idx, const float *__restrict__ qsel,
@@ -743,8 +744,9 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
     const int len = min(max(seq_len[b], 0), NB * kT);
     const int S_pages = S - ((n_sink + n_recent > 0) ? 2 : 0);   // the last two splits take the tier
     uint8_t *slots = unit_slots(const_cast<uint8_t *>(pages), gridDim.z, Hkv, NB, 2, unit, n_sink + n_recent, NG);
+    const int wp = BK ? w_pages : 0;               // pages per bucket, 0 without buckets
     if (s >= S_pages) {
-        if (w_pages > 0) {
+        if (BK) {
             __syncthreads();
             tier_cta_q(sh, slots, len, n_sink, n_recent, s - S_pages, k,
                        TierQBuckets{qsel, idx + unit * nbk * k, k, nbk, w_pages * kT, qrow0}, part_o, part_ml,
@@ -756,11 +758,11 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
         }
         return;
     }
-    if (w_pages == 0) load_sel(0);
+    if (!BK) load_sel(0);
     const Tier tr = tier_of(len, n_sink, n_recent);
     run_pages<NG>(sh, pages + unit * NB * (size_t)page_bytes(2, NG), tr.sink_end, tr.recent_start,
                   split_of(tr.recent_start, S_pages, s), S, s, qrow0, part_o, part_ml, out, counters + unit, status,
-                  false, rot, w_pages, load_sel);
+                  false, rot, wp, load_sel);
 }
 
 // ---------------------------------------------------------------- fused step
@@ -1108,28 +1110,32 @@ int decode_mma_splits(int units, int nblk, int num_sms, int tier) {
 
 int step_mma_max_new() { return kStepMaxNew; }
 
-template <int NG>
+template <int NG, bool BK>
 cudaError_t launch_decode_mma_t(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
                                 const float *qgsum, int k, float *part_o, float2 *part_ml, int S,
                                 float *out, cudaStream_t st) {
     const size_t smem = sizeof(MmaShared);
     static std::atomic<uint64_t> done{0};
-    cudaError_t e = set_smem_once(decode_mma_kernel<NG>, (int)smem, done);
+    cudaError_t e = set_smem_once(decode_mma_kernel<NG, BK>, (int)smem, done);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)S, (unsigned)c.n_kv_heads, (unsigned)c.batch);
-    decode_mma_kernel<NG><<<grid, kThreads, smem, st>>>(static_cast<const uint8_t *>(c.pages), c.seq_len,
-                                                        c.n_kv_heads, c.capacity / kT, Hq, idx, qsel, qgsum, k,
-                                                        part_o, part_ml, S, out, unit_counter(c, 0, 0), c.status,
-                                                        c.n_sink, c.n_recent, c.v_rot, buckets_of(c),
-                                                        c.bucket / kT);
+    decode_mma_kernel<NG, BK><<<grid, kThreads, smem, st>>>(static_cast<const uint8_t *>(c.pages), c.seq_len,
+                                                            c.n_kv_heads, c.capacity / kT, Hq, idx, qsel, qgsum, k,
+                                                            part_o, part_ml, S, out, unit_counter(c, 0, 0), c.status,
+                                                            c.n_sink, c.n_recent, c.v_rot, buckets_of(c),
+                                                            c.bucket / kT);
     return cudaGetLastError();
 }
 
 cudaError_t launch_decode_mma(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
                               const float *qgsum, int k, float *part_o, float2 *part_ml, int S,
                               float *out, cudaStream_t st) {
-    return groups_of(c) == 1 ? launch_decode_mma_t<1>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, st)
-                             : launch_decode_mma_t<kNG>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, st);
+    const bool one = groups_of(c) == 1, bk = c.bucket > 0;
+    if (bk)
+        return one ? launch_decode_mma_t<1, true>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, st)
+                   : launch_decode_mma_t<kNG, true>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, st);
+    return one ? launch_decode_mma_t<1, false>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, st)
+               : launch_decode_mma_t<kNG, false>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, st);
 }
 
 template <typename Tin, int NG>
