@@ -537,6 +537,7 @@ def run_ours(args):
                      "kernel": ("fused step (kvq_decode_step: append + select + decode + merge)" if args.fused
                                 else "decode partial + merge (kvq_decode_attn)"),
                      "peak_source": f"{peak_src} hbm_gbs", "traffic_note": traffic_note},
+        "ms_per_step_median": statistics.median(step_ms),
         "decode_ms": statistics.mean(dec_ms),
         "step_launch": "cuda graph" if args.graph else "eager",
         "decode_alg_bytes": statistics.mean(alg_bytes),
