@@ -267,7 +267,8 @@ def run_reference(args):
 def config_dict(wl: W.Workload, k: int, protect=(0, 0)):
     d = {"workload": wl.name, "batch": wl.batch, "n_q_heads": wl.n_q_heads,
          "n_kv_heads": wl.n_kv_heads, "context": wl.n_ctx, "head_dim": 128, "bits": wl.bits,
-         "group": wl.quant_group, "sparsity": wl.sparsity, "k": k,
+         "group": wl.quant_group, "sparsity": wl.sparsity, "k": k, "input_dtype": wl.dtype,
+         "arithmetic": "f16 x f16 -> f32 tensor-core products of exact codes, f32 softmax, f64 transforms",
          "step": "append 1 token + query transform/select + decode + merge",
          "l2": "flushed between steps (256 MiB write, outside the timed events)"}
     if protect != (0, 0):
@@ -415,9 +416,11 @@ def run_ours(args):
         step.k_new.copy_(kv_pool[i % n_pool][0])
         step.v_new.copy_(kv_pool[i % n_pool][1])
 
-    # fused: one kvq_decode_step launch; unfused: one-token append (with its
-    # length advance), select, decode (with its merge)
-    launches_per_step = 1 if args.fused else 3
+    # fused: one kvq_decode_step launch (with RoPE buckets two: the
+    # preparation kernel and the decode as its programmatic dependent);
+    # unfused: one-token append (with its length advance), select, decode
+    # (with its merge)
+    launches_per_step = (2 if wl.bucket else 1) if args.fused else 3
     alg_fn = algorithmic_step_bytes if args.fused else algorithmic_decode_bytes
     step.time_decode()
     length = wl.n_ctx
@@ -464,7 +467,8 @@ def run_ours(args):
     # roofline of the dominant kernel (decode partial + merge, timed together)
     hbm_peak, peak_src = measured_peaks()
     alg_bytes = [alg_fn(wl, k, tok // (B * Hkv), protect) for tok in tokens]
-    achieved = statistics.mean(ab / (ms * 1e-3) for ab, ms in zip(alg_bytes, dec_ms)) / 1e9
+    # bytes over time of all timed launches (not a mean of per-step ratios)
+    achieved = sum(alg_bytes) / (sum(dec_ms) * 1e-3) / 1e9
     traffic, traffic_note = committed_traffic("step_mma" if args.fused else "decode_mma",
                                               wl.name + format_tag(wl, protect))
 
@@ -581,7 +585,7 @@ def main():
                     help="fold a diagonal refinement into the transforms; select on the base queries")
     ap.add_argument("--bucket", type=int, default=0,
                     help="tokens per bucket of bucket-relative RoPE (the pages use 2048; 0: none); "
-                         "a bucketed step runs as the three calls")
+                         "a bucketed step is two launches (preparation + decode)")
     ap.add_argument("--pages-recipe", action="store_true",
                     help="the pages' whole format: --group 128 --protect --rotate-values --refine --bucket 2048")
     ap.add_argument("--unfused", dest="fused", action="store_false",
@@ -592,8 +596,6 @@ def main():
     if args.pages_recipe:
         args.group, args.protect, args.rotate_values, args.refine = 128, True, True, True
         args.bucket = 2048
-    if args.bucket:
-        args.fused = False          # the bucketed step runs as append, select, decode
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":

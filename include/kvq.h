@@ -292,6 +292,23 @@ int kvq_decode_attn(const kvq_cache *cache, int n_q_heads, const int32_t *idx,
                     void *ws, size_t ws_bytes, kvq_stream_t stream);
 
 /*
+ * kvq_decode_attn_wait_bound -- kvq_decode_attn with an explicit bound on each
+ * wait of the tensor-core decode for a staged page (INT2, 4 query heads per
+ * KV head, the shapes that decode runs on; other shapes return
+ * KVQ_ERR_SHAPE).  A fault-handling hook, not part of the method: the pages
+ * describe no failure path.  kvq_decode_attn waits up to about a million
+ * polls per stage.  With wait_polls = 0 a wait gives up at once unless the
+ * page has already landed.  A wait that gives up sets KVQ_DEV_TIMEOUT; its
+ * pair of warps then issues no further copy, waits for the copies already in
+ * flight to land, and finishes, so the call leaves the cache, the counters
+ * and the GPU ready for the next call, but its `out` is not valid.
+ * Same arguments and errors as kvq_decode_attn otherwise.
+ */
+int kvq_decode_attn_wait_bound(const kvq_cache *cache, int n_q_heads, const int32_t *idx,
+                               const float *qsel, const float *qgsum, int k, float *out,
+                               void *ws, size_t ws_bytes, uint32_t wait_polls, kvq_stream_t stream);
+
+/*
  * kvq_decode_step -- one whole decode step: kvq_append of the n_new new
  * tokens, kvq_select_channels of the query, then kvq_decode_attn over every
  * token including the new ones.  Same arguments, results and errors as those
@@ -347,7 +364,10 @@ int kvq_bf16_decode_attn(const void *q, const void *K, const void *V, int batch,
  * library holds until the process exits.  The library allocates nothing.
  *  - The first call on a device, with that device current, looks up the
  *    array's device address (cudaGetSymbolAddress) and caches it; make that
- *    first call before any stream capture.
+ *    first call before any stream capture.  The cached address is never
+ *    refreshed: after cudaDeviceReset() on a device (which unloads the
+ *    library's device code there) do not call this entry point again on that
+ *    device in the same process.
  *  - All calls share the one array, and it keeps the last call's contents.
  *    Nothing in it needs to start at zero.  Calls whose kernels can overlap
  *    on the GPU (different streams, or different host threads) race on it:

@@ -159,6 +159,23 @@ int kvq_decode_attn(const kvq_cache *c, int n_q_heads, const int32_t *idx, const
     return cuda_status(launch_decode(*c, n_q_heads, idx, qsel, qgsum, k, out, ws, S, (cudaStream_t)stream));
 }
 
+int kvq_decode_attn_wait_bound(const kvq_cache *c, int n_q_heads, const int32_t *idx, const float *qsel,
+                               const float *qgsum, int k, float *out, void *ws, size_t ws_bytes,
+                               uint32_t wait_polls, kvq_stream_t stream) {
+    int st = check_decode_args(c, n_q_heads, k);
+    if (st) return st;
+    if (!decode_uses_mma(*c, n_q_heads)) return KVQ_ERR_SHAPE;
+    if (!idx || !qsel || !qgsum || !out) return KVQ_ERR_ARG;
+    if (!aligned(idx, 4) || !aligned(qsel, 4) || !aligned(qgsum, 4) || !aligned(out, 4)) return KVQ_ERR_ALIGN;
+    const int sms = num_sms();
+    if (sms <= 0) return KVQ_ERR_CUDA;
+    const int S = decode_splits(*c, n_q_heads, k, sms);
+    if (!ws || ws_bytes < decode_ws_bytes(*c, n_q_heads, S)) return KVQ_ERR_WORKSPACE;
+    if (!aligned(ws, 16)) return KVQ_ERR_ALIGN;
+    return cuda_status(launch_decode(*c, n_q_heads, idx, qsel, qgsum, k, out, ws, S, (cudaStream_t)stream,
+                                     (long long)wait_polls));
+}
+
 int kvq_decode_step(const kvq_cache *c, const void *q, const void *k_new, const void *v_new, int dtype,
                     int n_q_heads, int n_new, const double *A, const double *Ainvt, const double *delta,
                     float sparsity, int32_t *idx, float *qsel, float *qgsum, float *out, void *ws,

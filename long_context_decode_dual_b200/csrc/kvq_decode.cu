@@ -9,13 +9,21 @@ cudaError_t launch_decode_simt(const kvq_cache &c, int Hq, const int32_t *idx, c
                                float *out, cudaStream_t st);
 cudaError_t launch_decode_mma(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
                               const float *qgsum, int k, float *part_o, float2 *part_ml, int S,
-                              float *out, cudaStream_t st);
+                              float *out, uint32_t polls, cudaStream_t st);
+uint32_t default_wait_polls();
 int decode_mma_splits(int units, int nblk, int num_sms, int tier);
 int step_mma_max_new();
 cudaError_t launch_step_mma(const kvq_cache &c, int Hq, const void *q, const void *k_new, const void *v_new,
                             int dtype, int n_new, const double *A, const double *Ainvt, const double *delta,
                             int k, int32_t *idx, float *qsel, float *qgsum, float *part_o, float2 *part_ml,
                             int S, float *out, cudaStream_t st);
+cudaError_t launch_decode_mma_step(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
+                                   const float *qgsum, int k, float *part_o, float2 *part_ml, int S,
+                                   float *out, int n_new, cudaStream_t st);
+cudaError_t launch_step_prep(const kvq_cache &c, const void *q, int dtype, int Hq, const void *k_new,
+                             const void *v_new, int n_new, const double *A, const double *Ainvt,
+                             const double *delta, int k, int32_t *idx, float *qsel, float *qgsum, cudaStream_t st);
+int step_prep_max_new();
 
 // The tensor-core kernel covers INT2 codes with 4 query heads per KV head;
 // other shapes use the CUDA-core kernel.
@@ -49,27 +57,40 @@ size_t decode_ws_bytes(const kvq_cache &c, int Hq, int S) {
     return (size_t)c.batch * Hq * S * (kD * sizeof(float) + sizeof(float2));
 }
 
+// polls < 0: the tensor-core kernel's default bound on each wait for a
+// staged page; any other value replaces it (0: give up unless the page has
+// already landed -- the test path for the give-up).
 cudaError_t launch_decode(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
-                          const float *qgsum, int k, float *out, void *ws, int S, cudaStream_t st) {
+                          const float *qgsum, int k, float *out, void *ws, int S, cudaStream_t st,
+                          long long polls) {
     float *part_o = static_cast<float *>(ws);
     float2 *part_ml = reinterpret_cast<float2 *>(part_o + (size_t)c.batch * Hq * S * kD);
     // one launch: the last CTA of each (sequence, KV head) merges the splits
-    return use_mma(c, Hq) ? launch_decode_mma(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, st)
+    return use_mma(c, Hq) ? launch_decode_mma(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out,
+                                              polls < 0 ? default_wait_polls() : (uint32_t)polls, st)
                           : launch_decode_simt(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, st);
 }
+bool decode_uses_mma(const kvq_cache &c, int Hq) { return use_mma(c, Hq); }
 
-// One decode step.  The tensor-core shape with at most step_mma_max_new() new
-// tokens and no RoPE buckets runs as one fused launch; anything else as the
-// three calls.
+// One decode step.  The tensor-core shape with at most step_mma_max_new()
+// new tokens runs as one fused launch, or with RoPE buckets as two launches
+// (the preparation kernel -- per-bucket channel choice + append -- and the
+// decode as its programmatic dependent); anything else as the three calls.
 cudaError_t launch_decode_step(const kvq_cache &c, int Hq, const void *q, const void *k_new,
                                const void *v_new, int dtype, int n_new, const double *A,
                                const double *Ainvt, const double *delta, int k, int32_t *idx, float *qsel,
                                float *qgsum, float *out, void *ws, int S, cudaStream_t st) {
-    if (use_mma(c, Hq) && n_new <= step_mma_max_new() && c.bucket == 0) {
+    if (use_mma(c, Hq) && n_new <= step_mma_max_new() && n_new <= step_prep_max_new()) {
         float *part_o = static_cast<float *>(ws);
         float2 *part_ml = reinterpret_cast<float2 *>(part_o + (size_t)c.batch * Hq * S * kD);
-        return launch_step_mma(c, Hq, q, k_new, v_new, dtype, n_new, A, Ainvt, delta, k, idx, qsel, qgsum,
-                               part_o, part_ml, S, out, st);
+        if (c.bucket == 0)
+            return launch_step_mma(c, Hq, q, k_new, v_new, dtype, n_new, A, Ainvt, delta, k, idx, qsel, qgsum, part_o,
+                                   part_ml, S, out, st);
+        cudaError_t e = launch_step_prep(c, q, dtype, Hq, k_new, v_new, n_new, A, Ainvt, delta, k, idx, qsel,
+                                         qgsum, st);
+        if (e == cudaSuccess)
+            e = launch_decode_mma_step(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, n_new, st);
+        return e;
     }
     cudaError_t e = cudaSuccess;
     if (n_new > 0) e = launch_append(c, k_new, v_new, dtype, n_new, A, st);

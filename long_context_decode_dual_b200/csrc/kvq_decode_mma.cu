@@ -32,29 +32,43 @@
 // groups) so the per-token value scale is folded into the weights once per
 // group.  The value zero-point term sum_t p(t) z(t) is one more MMA.
 //
-// Work split: one CTA = one (sequence, KV head, split of the context), eight
-// warps in four pairs.  A pair processes one 128-token page at a time from a
-// two-stage ring filled by bulk asynchronous copies completing on an
-// mbarrier: key rows are copied in 64-byte chunks (two rows, the unit in which
-// the memory system fetches anyway) as a few runs of chunks that hold a
-// selected row, into their own place in the stage, and the tail of the page
-// (value codes, channel 0, metadata) in one copy.  Warp w of the pair takes
-// half w of every 16-token word of the page (64 tokens) and keeps its own
-// online softmax; its softmax weights pass from the score layout to the value
-// layout through a small buffer of its own.
+// Work split: one CTA = one (sequence, KV head, split), eight warps in four
+// pairs.  A pair processes one 128-token page at a time from a two-stage ring
+// filled by bulk asynchronous copies completing on an mbarrier: key rows are
+// copied in 64-byte chunks (two rows, the unit in which the memory system
+// fetches anyway) as a few runs of chunks that hold a selected row, into their
+// own place in the stage, and the tail of the page (value codes, channel 0,
+// metadata) in one copy.  Warp w of the pair takes half w of every 16-token
+// word of the page (64 tokens) and keeps its own online softmax; its softmax
+// weights pass from the score layout to the value layout through a small
+// buffer of its own.
 //
-// The fused step kernel runs as clusters of two CTAs, the two taking
-// consecutive splits of one (sequence, KV head).  CTA r of a cluster computes
-// q' for channels 64r..64r+63 (64 columns of A^{-T}, staged in shared memory;
-// the same fixed-order float64 arithmetic as kvq_select_channels) and their
-// pooled energies; after a cluster barrier both CTAs read the 128 energies and
-// all of q' through distributed shared memory and make the same channel
-// choice.  In the cluster whose splits receive the new tokens, CTA r also
+// Page schedule (without RoPE buckets): the pages a unit reads form a pool,
+// taken from the last page backwards and dealt round-robin to the unit's
+// pairs (the appending cluster of a fused step sits out the second round).
+// The schedule is fixed by the shapes alone, so results are reproducible bit
+// for bit.  The tail of a page (everything but the key rows) does not depend
+// on the channel choice, so a pair copies its first tail before the choice
+// is made or loaded.  With RoPE buckets each split reads a contiguous range
+// of pages, one segment per bucket.
+//
+// The fused step kernel (kvq_decode_step without RoPE buckets) runs as
+// clusters of two CTAs, the two taking consecutive splits of one (sequence,
+// KV head).  CTA r of a cluster computes q' for channels 64r..64r+63 (64
+// columns of A^{-T}, staged in shared memory around the first pages' tails;
+// the same fixed-order float64 arithmetic as kvq_select_channels, the four
+// heads' chains side by side in one thread) and their pooled energies; after a
+// cluster barrier both CTAs read the 128 energies and all of q' through
+// distributed shared memory and make the same channel choice.  The first
+// cluster holds the pages of the new tokens (the first pool pages): its CTA r
 // transforms, quantizes and writes key groups 2r and 2r+1 of them (the
 // arithmetic of kvq_append; code bits are OR-ed into positions that are still
-// zero) before the same barrier, so the page owner stages those pages after
-// it.  (Pairs of CTAs pack the SMs' two CTA slots exactly; clusters of four
-// leave slots of some GPCs unused.)
+// zero) before the same barrier, so those pages are staged after it.  (Pairs
+// of CTAs pack the SMs' two CTA slots exactly; clusters of four leave slots of
+// some GPCs unused.)  With RoPE buckets a step is two launches instead: the
+// preparation kernel (kvq_select.cu: the per-bucket channel choice and the
+// append) and this decode as its programmatic dependent, which waits for it
+// only before it reads what the preparation writes.
 #include "kvq_internal.cuh"
 
 #include <cooperative_groups.h>
@@ -76,6 +90,7 @@ constexpr uint32_t kWaitPolls = 1u << 20;         // bound on mbarrier polls per
 constexpr int kStepMaxNew = 4;                    // new tokens per fused step
 constexpr int kCluster = 2;                       // CTAs per cluster of the fused step
 constexpr int kCols = kD / kCluster;              // channels whose q' one CTA of a cluster computes
+constexpr int kAppendRounds = 1;                  // rounds the appending cluster's pairs sit out
 
 struct __align__(16) MmaShared {
     uint8_t stage[kPairs][2][kStageBytes];
@@ -96,11 +111,16 @@ struct __align__(16) MmaShared {
     double trange[kWarps][4];          // fused step, one grid per token: per-warp key / value ranges
 };
 
-// Prologue scratch of the fused step.  No page copy has been issued yet, so
-// the staging memory P is free: P[0, 64K) holds A^{-T}[:, 64r..64r+63] and
-// later rows 64..127 of A[:, 64r..64r+63]; P[64K, 96K) rows 0..63 of the latter;
-// then energies and ranks.  Smaller arrays use the softmax exchange buffers
-// and the B-fragment table, which the page loop fills later.
+// Prologue scratch of the fused step.  Before the page loop the staging
+// memory P holds the 64-column block of A^{-T} as 128 rows of 512 bytes.  A
+// CTA that appends nothing keeps the tails of its pairs' first pages in
+// flight into stage 0 meanwhile, so its rows go around them: rows 32p..32p+7
+// in the key area of pair p's stage 0, rows 32p+8..32p+31 in its stage 1.  A
+// CTA that appends (the first cluster, the tier cluster) holds the block in
+// P[0, 64K); A's column block then follows it through P[0, 96K) in two
+// halves (below), and no stage is in flight during the prologue.
+// Energies, ranks and the gathered q' come after the q' chains in the same
+// memory (outside the first tails).
 constexpr int kBlkRowBytes = kCols * (int)sizeof(double);        // 512
 constexpr int kOffAHi = 0;                                        // A rows 64..127
 constexpr int kOffALo = kD * kBlkRowBytes;                        // A rows 0..63
@@ -109,8 +129,12 @@ constexpr int kOffRank = kOffE2 + kD * (int)sizeof(double);       // int[2][128]
 constexpr int kOffQp = kStageBytes;                               // double[4][128] in stage[0][1], after the append
 static_assert(kOffRank + 2 * kD * (int)sizeof(int) <= kPairs * 2 * kStageBytes, "scratch fits the stages");
 static_assert(kOffQp + 4 * kD * (int)sizeof(double) <= 2 * kStageBytes, "q' copy inside stage[0][1]");
+static_assert(kOffE2 >= 3 * 2 * kStageBytes + kStageBytes && kOffQp >= kStageBytes,
+              "energies, ranks and q' lie outside the stage-0 tails of the first pages");
+static_assert(8 * kBlkRowBytes <= kKeyBytes && 24 * kBlkRowBytes <= kStageBytes,
+              "32 rows of the A^{-T} block per pair around its first tail");
 struct PexScratch {                    // in MmaShared::pex
-    double qin[4][kD];                 // query rows, float64 (exact for bf16 / f32 inputs)
+    double qin[kD][4];                 // query rows, float64 (exact for bf16 / f32 inputs), [channel][head]
 };
 // new key rows: float (exact) in MmaShared::q until the channel choice, then
 // float64 in the staging memory freed by the A^{-T} block; new value rows in
@@ -147,8 +171,13 @@ __device__ __forceinline__ void mma16816_z(float (&d)[4], uint32_t a0, uint32_t 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(z));
 }
 
-__device__ __forceinline__ void pair_sync(int pair) {
-    asm volatile("bar.sync %0, 64;\n" ::"r"(pair + 1) : "memory");
+// barrier of the two warps of a pair that also ANDs a flag over them
+__device__ __forceinline__ bool pair_sync_and(int pair, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, %2, 64, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+        : "=r"(r) : "r"((uint32_t)v), "r"(pair + 1) : "memory");
+    return r != 0;
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -167,6 +196,10 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
                  ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
 }
+// bring `bytes` (a multiple of 16, 16-byte aligned) of global memory into L2
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(src), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -174,15 +207,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
     return ok != 0;
 }
-// Wait for a stage's copies.  The wait is bounded: after kWaitPolls polls the
-// device status word gets KVQ_DEV_TIMEOUT and the caller goes on (that call's
-// output is then reported invalid) instead of waiting forever; both warps of
-// a pair keep the same control flow either way.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint32_t *status) {
-    for (uint32_t i = 0; i < kWaitPolls; i++)
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+// Wait for a stage's copies.  The wait is bounded: after `polls` polls the
+// device status word gets KVQ_DEV_TIMEOUT and the caller is told; it then
+// issues no further copy, drains what it issued (drain_stage) and reports
+// that call's output invalid.  polls = 0 gives up at once unless the stage
+// has already landed (the path a test takes to exercise the give-up).
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint32_t *status,
+                                                  uint32_t polls) {
+    if (mbar_test_wait(bar, parity)) return true;
+    for (uint32_t i = 0; i < polls; i++)
         if (mbar_try_wait(bar, parity)) return true;
     atomicOr(status, (uint32_t)KVQ_DEV_TIMEOUT);
     return false;
+}
+// After a give-up: wait (bounded by kWaitPolls) until the stage's copies
+// have landed, so that no copy still writes into shared memory when the CTA
+// goes on to reuse it or exits.
+__device__ __forceinline__ void drain_stage(uint32_t bar, uint32_t parity) {
+    for (uint32_t i = 0; i < kWaitPolls; i++)
+        if (mbar_try_wait(bar, parity)) return;
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -217,36 +267,50 @@ __device__ __forceinline__ Split split_of(int len, int S, int s) {
     return {blk0, min(nblk, blk0 + bps)};
 }
 
-// The fused step's split: the last cluster also appends the new tokens, which
-// costs about kAppendPages pages of work per CTA, so it takes that many fewer
-// pages; the other splits take equal shares of the rest.  owner_of() is the
-// inverse (the split holding page pg).
-constexpr int kAppendPages = 8;
-struct StepPlan {
-    int S, nblk, bps, head, tail_bps;   // head = pages of the first S - kCluster splits
+// The page schedule of a unit without RoPE buckets.  The pages that hold the
+// coded tokens [lo, hi) are [P0, P1); pool index q is page P1 - 1 - q (the
+// last page first: it holds the new tokens of a fused step).  The unit's NP =
+// kPairs * S_pages pairs take the pool round-robin, pair P = kPairs s + pair
+// taking q = P in round 0.  With `skip` > 0 the first `appenders` pairs (the
+// fused step's appending cluster) sit out rounds 1..skip, which the other
+// pairs take in turn, so the work of appending makes no straggler.  The
+// schedule is a pure function of the shapes: every run assigns the same pages
+// to the same pairs in the same order, so results are reproducible bit for
+// bit.
+struct Pool {
+    int P0, P1;
+    int P, NP;                 // this pair's index and the pairs of the unit
+    int appenders, skip;
+    bool tail_issued;          // the first page's tail is already in flight into stage 0
+    __device__ int size() const { return P1 - P0; }
+    __device__ int page(int q) const { return P1 - 1 - q; }
+    // pool index of this pair's j-th page, -1 past the end
+    __device__ int index(int j) const {
+        const int A = appenders, K = skip;
+        int q;
+        if (j == 0)
+            q = P;
+        else if (P < A)
+            q = NP + K * (NP - A) + (j - 1) * NP + P;
+        else if (j <= K)
+            q = NP + (j - 1) * (NP - A) + (P - A);
+        else
+            q = NP + K * (NP - A) + (j - K - 1) * NP + P;
+        return q < size() ? q : -1;
+    }
 };
-__device__ __forceinline__ StepPlan step_plan(int len, int S) {
-    StepPlan p;
-    p.S = S;
-    p.nblk = (len + kT - 1) / kT;
-    p.bps = (p.nblk + kCluster * kAppendPages + S - 1) / S;
-    p.head = min(p.nblk, (S - kCluster) * p.bps);
-    p.tail_bps = (p.nblk - p.head + kCluster - 1) / kCluster;
+__device__ __forceinline__ Pool unit_pool(int lo, int hi, int s, int pair, int S_pages, int appenders, int skip,
+                                          bool tail_issued) {
+    Pool p;
+    p.P0 = lo / kT;
+    p.P1 = hi > lo ? (hi + kT - 1) / kT : p.P0;
+    p.P = kPairs * s + pair;
+    p.NP = kPairs * S_pages;
+    p.appenders = min(appenders, p.NP);
+    p.skip = p.appenders < p.NP ? skip : 0;
+    p.tail_issued = tail_issued;
     return p;
 }
-__device__ __forceinline__ Split step_split(const StepPlan &p, int s) {
-    if (s < p.S - kCluster) {
-        const int blk0 = min(p.nblk, s * p.bps);
-        return {blk0, min(p.nblk, blk0 + p.bps)};
-    }
-    const int blk0 = min(p.nblk, p.head + (s - (p.S - kCluster)) * p.tail_bps);
-    return {blk0, min(p.nblk, blk0 + p.tail_bps)};
-}
-__device__ __forceinline__ int owner_of(const StepPlan &p, int pg) {
-    if (pg < p.head) return pg / p.bps;
-    return p.S - kCluster + (pg - p.head) / max(p.tail_bps, 1);
-}
-
 // The page plan from the channel choice (sh.chan_pos, sh.q): score-MMA B
 // fragments, and the copy list of a page.  Called by every thread after a
 // barrier that follows the last write of chan_pos / q; ends with a barrier.
@@ -323,21 +387,28 @@ __device__ __forceinline__ void issue_keys(MmaShared &sh, int pair, int st, cons
     }
 }
 
-// The page loop and the merges: pages [sp.blk0, sp.blk1) of the unit, pair
-// `pair` taking every kPairs-th; tokens outside [lo, hi) (beyond the length,
-// or in the protected tier) are left out of the softmax.  `first_issued`: the pair's first page is
-// already in flight, whole, into stage 0 (one copy that arrives on the
-// barrier).  With RoPE buckets of w_pages pages the split runs as segments,
-// one per bucket: before each, every warp is done with the previous one and
-// load_seg(bucket) puts that bucket's channel choice and page plan in place
-// (called by every thread; it ends with a barrier); the softmax state runs on
-// across segments.  w_pages = 0: one segment, the plan already in place.
-template <int NG, typename SegFn>
+// The page loop and the merges.  Tokens outside [lo, hi) (beyond the length,
+// or in the protected tier) are left out of the softmax.
+//  DYN (no RoPE buckets): this pair's pages of the unit's round-robin
+//    schedule `pool`, each staged while the one before it is computed.
+//    pool.tail_issued: the first page's tail is already in flight into
+//    stage 0.
+//  static: pages [sp.blk0, sp.blk1), pair `pair` taking every kPairs-th.
+//    With RoPE buckets of w_pages pages the split runs as segments, one per
+//    bucket: before each, every warp is done with the previous one and
+//    load_seg(bucket) puts that bucket's channel choice and page plan in place
+//    (called by every thread; it ends with a barrier); the softmax state runs
+//    on across segments.  w_pages = 0: one segment, the plan already in place.
+// A wait that gives up (mbar_wait_bounded) stops the pair on both of its warps
+// (the flag is ANDed over the pair at its barrier): no further copy is issued,
+// the stage still in flight is drained after the loop, and the call's result
+// is reported invalid through KVQ_DEV_TIMEOUT.
+template <int NG, bool DYN, typename SegFn>
 __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restrict__ unit_pages, int lo, int hi,
-                                          Split sp, int S, int s, size_t qrow0, float *__restrict__ part_o,
-                                          float2 *__restrict__ part_ml, float *__restrict__ out,
-                                          uint32_t *counter, uint32_t *status, bool first_issued,
-                                          const double *rot, int w_pages, SegFn &&load_seg) {
+                                          Split sp, const Pool &pool, int S, int s, size_t qrow0,
+                                          float *__restrict__ part_o, float2 *__restrict__ part_ml,
+                                          float *__restrict__ out, uint32_t *counter, uint32_t *status,
+                                          uint32_t polls, const double *rot, int w_pages, SegFn &&load_seg) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int pair = warp >> 1, half = warp & 1;
     const int gid = lane >> 2, tig = lane & 3;
@@ -370,35 +441,8 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
     const float zmask = gid < NG ? 1.f : 0.f;                // z-term rows: one per group
     uint4 *pexw = &sh.pex[warp][0][0];
 
-    int it = 0;                   // pages this pair has staged (the ring position, across segments)
-    uint32_t late = 0;            // stages whose last wait gave up, with the parity waited for
-    const bool issuer = (tid & 63) == 0;
-    for (int seg0 = sp.blk0; seg0 < sp.blk1;) {
-    const int seg1 = w_pages > 0 ? min(sp.blk1, (seg0 / w_pages + 1) * w_pages) : sp.blk1;
-    if (w_pages > 0) {
-        __syncthreads();                                     // every warp is done with the last plan
-        load_seg(seg0 / w_pages);
-        load_coef();
-    }
-    const int first = seg0 + pair;
-    if (issuer && first < seg1 && !(first_issued && seg0 == sp.blk0)) {
-        const uint8_t *src = unit_pages + (size_t)first * page_bytes(2, NG);
-        issue_tail<NG>(sh, pair, it & 1, src);
-        issue_keys(sh, pair, it & 1, src);
-    }
-    for (int pg = first; pg < seg1; pg += kPairs, it++) {
-        const int st = it & 1;
-        const uint8_t *cur = sh.stage[pair][st];
-        const uint32_t par = (uint32_t)(it >> 1) & 1u;
-        late = mbar_wait_bounded(smem_u32(&sh.mbar[pair][st]), par, status)
-                   ? late & ~(3u << (2 * st)) : (late & ~(3u << (2 * st))) | ((2u | par) << (2 * st));
-        pair_sync(pair);                                     // both warps left the other stage
-        if (issuer && pg + kPairs < seg1) {
-            const uint8_t *src = unit_pages + (size_t)(pg + kPairs) * page_bytes(2, NG);
-            issue_tail<NG>(sh, pair, st ^ 1, src);
-            issue_keys(sh, pair, st ^ 1, src);
-        }
-
+    // one page `pg` staged in `cur`: scores, online softmax, value aggregation
+    auto page = [&](const uint8_t *cur, int pg) {
         const uint8_t *vcodes = cur + kKeyBytes;
         const uint32_t *ch0w = reinterpret_cast<const uint32_t *>(vcodes + 128 * 32);
         const uint32_t *kmeta = reinterpret_cast<const uint32_t *>(vcodes + 128 * 32 + 256);
@@ -604,15 +648,79 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
                 mma16816(cz, a[0], 0u, a[1], 0u, ph[j][0], ph[j][1]);
             }
         }
+    };
+
+    const bool issuer = (tid & 63) == 0;
+    int pend_st = -1;             // a stage still in flight after a give-up, and its parity
+    uint32_t pend_par = 0;
+    if constexpr (DYN) {
+        // this pair's pages of the schedule, the next one staged while the
+        // current one is computed; the same sequence on both warps
+        int q_cur = pool.index(0);
+        if (issuer && q_cur >= 0) {
+            const uint8_t *src = unit_pages + (size_t)pool.page(q_cur) * page_bytes(2, NG);
+            if (!pool.tail_issued) issue_tail<NG>(sh, pair, 0, src);
+            issue_keys(sh, pair, 0, src);
+        }
+        for (int it = 0; q_cur >= 0; it++) {
+            const int st = it & 1;
+            const uint32_t par = (uint32_t)(it >> 1) & 1u;
+            bool ok = mbar_wait_bounded(smem_u32(&sh.mbar[pair][st]), par, status, polls);
+            ok = pair_sync_and(pair, ok);                        // both warps left the other stage
+            if (!ok) {
+                pend_st = st;
+                pend_par = par;
+                break;
+            }
+            const int q_next = pool.index(it + 1);
+            if (issuer && q_next >= 0) {
+                const uint8_t *src = unit_pages + (size_t)pool.page(q_next) * page_bytes(2, NG);
+                issue_tail<NG>(sh, pair, st ^ 1, src);
+                issue_keys(sh, pair, st ^ 1, src);
+            }
+            page(sh.stage[pair][st], pool.page(q_cur));
+            q_cur = q_next;
+        }
+    } else {
+        int it = 0;                   // pages this pair has staged (the ring position, across segments)
+        bool dead = false;            // a wait gave up: no more copies, no more pages
+        for (int seg0 = sp.blk0; seg0 < sp.blk1;) {
+            const int seg1 = w_pages > 0 ? min(sp.blk1, (seg0 / w_pages + 1) * w_pages) : sp.blk1;
+            if (w_pages > 0) {
+                __syncthreads();                                 // every warp is done with the last plan
+                load_seg(seg0 / w_pages);
+                load_coef();
+            }
+            const int first = seg0 + pair;
+            if (issuer && !dead && first < seg1) {
+                const uint8_t *src = unit_pages + (size_t)first * page_bytes(2, NG);
+                issue_tail<NG>(sh, pair, it & 1, src);
+                issue_keys(sh, pair, it & 1, src);
+            }
+            for (int pg = first; pg < seg1 && !dead; pg += kPairs, it++) {
+                const int st = it & 1;
+                const uint32_t par = (uint32_t)(it >> 1) & 1u;
+                bool ok = mbar_wait_bounded(smem_u32(&sh.mbar[pair][st]), par, status, polls);
+                ok = pair_sync_and(pair, ok);                    // both warps left the other stage
+                if (!ok) {
+                    dead = true;
+                    pend_st = st;
+                    pend_par = par;
+                    break;
+                }
+                if (issuer && pg + kPairs < seg1) {
+                    const uint8_t *src = unit_pages + (size_t)(pg + kPairs) * page_bytes(2, NG);
+                    issue_tail<NG>(sh, pair, st ^ 1, src);
+                    issue_keys(sh, pair, st ^ 1, src);
+                }
+                page(sh.stage[pair][st], pg);
+            }
+            seg0 = seg1;
+        }
     }
-    seg0 = seg1;
-    }
-    // a stage whose wait gave up may still receive bytes: wait once more
-    // (bounded) before the staging memory is reused below
-#pragma unroll
-    for (int st = 0; st < 2; st++)
-        if (late & (2u << (2 * st)))
-            mbar_wait_bounded(smem_u32(&sh.mbar[pair][st]), (late >> (2 * st)) & 1u, status);
+    // a stage whose wait gave up may still receive bytes: wait (bounded)
+    // until they have landed before the staging memory is reused below
+    if (pend_st >= 0) drain_stage(smem_u32(&sh.mbar[pair][pend_st]), pend_par);
 
     // ------------------------------------------------------------ merge
     // per warp: head tig's max, sum and output; then across the 8 warps
@@ -696,17 +804,27 @@ __device__ __forceinline__ void tier_cta(MmaShared &sh, const uint8_t *slots, in
 
 // ---------------------------------------------------------------- decode
 // With RoPE buckets (BK; w_pages > 0 pages each, nbk entries per selection
-// array) each split reads, per bucket its pages fall in, that bucket's
-// channel choice; the tier CTAs read each protected position's own bucket's.
-// Without buckets the segment machinery is compiled out.
-template <int NG, bool BK>
+// array) each split reads a contiguous range of pages and, per bucket its
+// pages fall in, that bucket's channel choice; the tier CTAs read each
+// protected position's own bucket's.  Without buckets the pages come from the
+// unit's round-robin schedule, and each pair's first tail is in flight, and
+// its next tails on their way to L2, while the channel choice is loaded.
+//
+// STEP: the second launch of a decode step, a programmatic dependent of the
+// preparation kernel (the channel choice and the append of the step's n_new
+// tokens, kvq_select.cu).  Until griddepcontrol.wait it reads only what that
+// kernel does not write -- the length before the step and the tails of pages
+// that hold no new token -- and it advances the length after the wait, once
+// every CTA of the sequence has read it.
+template <int NG, bool BK, bool STEP>
 __global__ void __launch_bounds__(kThreads, 2)
-decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__ seq_len, int Hkv,
+decode_mma_kernel(const uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, int Hkv,
                   int NB, int Hq, const int32_t *__restrict__ idx, const float *__restrict__ qsel,
                   const float *__restrict__ qgsum, int k, float *__restrict__ part_o,
                   float2 *__restrict__ part_ml, int S, float *__restrict__ out,
-                  uint32_t *__restrict__ counters, uint32_t *__restrict__ status, int n_sink, int n_recent,
-                  const double *__restrict__ v_rot, int nbk, int w_pages) {
+                  uint32_t *__restrict__ counters, uint32_t *__restrict__ status,
+                  int n_sink, int n_recent, const double *__restrict__ v_rot, int nbk, int w_pages,
+                  uint32_t polls, int n_new) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     MmaShared &sh = *reinterpret_cast<MmaShared *>(smem_raw);
 
@@ -741,11 +859,31 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
     };
 
     if (tid < 2 * kPairs) mbar_init(smem_u32(&sh.mbar[tid >> 1][tid & 1]), 1);
-    const int len = min(max(seq_len[b], 0), NB * kT);
+    // the length (with the step's new tokens once they are in; a step that
+    // would overflow the capacity appends nothing)
+    const int L0 = seq_len[b];
+    const bool fits = L0 >= 0 && L0 + n_new <= NB * kT;
+    const int len = min(max(STEP && fits ? L0 + n_new : L0, 0), NB * kT);
+    // after the preparation kernel: wait for it, make its page writes visible
+    // to the bulk copies, and advance the length once every CTA of sequence b
+    // has read it (its completion counter reaches S * Hkv)
+    auto after_prep = [&]() {
+        if constexpr (STEP) {
+            asm volatile("griddepcontrol.wait;\n" ::: "memory");
+            asm volatile("fence.proxy.async.global;\n" ::: "memory");
+            if (tid == 0) {
+                const unsigned prev = atomicAdd(status + 1 + b, 1u);
+                if (prev == (unsigned)(S * Hkv) - 1u) {
+                    if (fits) seq_len[b] = L0 + n_new;
+                    atomicExch(status + 1 + b, 0u);
+                }
+            }
+        }
+    };
     const int S_pages = S - ((n_sink + n_recent > 0) ? 2 : 0);   // the last two splits take the tier
     uint8_t *slots = unit_slots(const_cast<uint8_t *>(pages), gridDim.z, Hkv, NB, 2, unit, n_sink + n_recent, NG);
-    const int wp = BK ? w_pages : 0;               // pages per bucket, 0 without buckets
     if (s >= S_pages) {
+        after_prep();
         if (BK) {
             __syncthreads();
             tier_cta_q(sh, slots, len, n_sink, n_recent, s - S_pages, k,
@@ -758,11 +896,28 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, const int32_t *__restrict__
         }
         return;
     }
-    if (!BK) load_sel(0);
     const Tier tr = tier_of(len, n_sink, n_recent);
-    run_pages<NG>(sh, pages + unit * NB * (size_t)page_bytes(2, NG), tr.sink_end, tr.recent_start,
-                  split_of(tr.recent_start, S_pages, s), S, s, qrow0, part_o, part_ml, out, counters + unit, status,
-                  false, rot, wp, load_sel);
+    const uint8_t *unit_pages = pages + unit * NB * (size_t)page_bytes(2, NG);
+    if constexpr (BK) {
+        after_prep();
+        run_pages<NG, false>(sh, unit_pages, tr.sink_end, tr.recent_start, split_of(tr.recent_start, S_pages, s),
+                             Pool{}, S, s, qrow0, part_o, part_ml, out, counters + unit, status, polls, rot,
+                             w_pages, load_sel);
+    } else {
+        // a first page that may hold a new token is staged only after the wait
+        const Pool pool0 = unit_pool(tr.sink_end, tr.recent_start, s, warp >> 1, S_pages, 0, 0, false);
+        const bool early = pool0.index(0) >= 0 && !(STEP && pool0.page(pool0.index(0)) >= L0 / kT);
+        Pool pool = pool0;
+        pool.tail_issued = early;
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+        __syncthreads();                              // barriers initialised before copies complete on them
+        if ((tid & 63) == 0 && early)
+            issue_tail<NG>(sh, warp >> 1, 0, unit_pages + (size_t)pool.page(pool.index(0)) * page_bytes(2, NG));
+        after_prep();
+        load_sel(0);
+        run_pages<NG, true>(sh, unit_pages, tr.sink_end, tr.recent_start, Split{0, 0}, pool, S, s, qrow0, part_o,
+                            part_ml, out, counters + unit, status, polls, rot, 0, [](int) {});
+    }
 }
 
 // ---------------------------------------------------------------- fused step
@@ -786,7 +941,6 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
     extern __shared__ __align__(16) uint8_t smem_raw[];
     MmaShared &sh = *reinterpret_cast<MmaShared *>(smem_raw);
     uint8_t *P = &sh.stage[0][0][0];
-    double (*aiT)[kCols] = reinterpret_cast<double (*)[kCols]>(P);              // A^{-T}[:, 64r + .]
     double (*a_hi)[kCols] = reinterpret_cast<double (*)[kCols]>(P + kOffAHi);   // A[64 + ., 64r + .]
     double (*a_lo)[kCols] = reinterpret_cast<double (*)[kCols]>(P + kOffALo);   // A[., 64r + .]
     double *e2 = reinterpret_cast<double *>(P + kOffE2);
@@ -807,6 +961,12 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
     const size_t qrow0 = (size_t)b * Hq + (size_t)h * 4;
     uint8_t *unit_pages = pages + unit * NB * (size_t)page_bytes(2, NG);
     const int capacity = NB * kT;
+    const int NPt = n_sink + n_recent;
+    const int S_pages = S - (NPt > 0 ? kCluster : 0);
+    const bool is_tier = s >= S_pages;
+    // the first cluster holds the new tokens' pages and the tier cluster
+    // writes what no split reads: only these may append
+    const bool may_append = is_tier || s < kCluster;
     // 64-column block of a 128 x 128 float64 matrix: 128 rows of 512 bytes
     auto stage_block = [&](double (*dst)[kCols], const double *src, int row0, int rows) {
         for (int e = tid; e < rows * (kBlkRowBytes / 16); e += kThreads) {
@@ -814,65 +974,71 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
             cp_async16(&dst[c][2 * part], src + (size_t)(row0 + c) * kD + 2 * part);
         }
     };
+    // rows 32p..32p+7 and 32p+8..32p+31 of the staged A^{-T} block
+    auto ai_base = [&](int p, int upper) -> uint8_t * {
+        if (may_append) return P + (32 * p + 8 * upper) * kBlkRowBytes;
+        return upper ? sh.stage[p][1] : sh.stage[p][0];
+    };
 
-    if (tid == 0) sh.s_len = seq_len[b];
+    // every global read that does not depend on the length is issued first,
+    // so that the prologue waits for one round trip: the A^{-T} block, the
+    // query, and in the CTAs that may append, A's low rows and the new rows
     if (tid < kD) sh.chan_pos[tid] = -1;
     if (tid < 2 * kPairs) mbar_init(smem_u32(&sh.mbar[tid >> 1][tid & 1]), 1);
     const double *Ai_blk = Ainvt + (size_t)h * kD * kD + r * kCols;
     const double *A_blk = A + (size_t)h * kD * kD + r * kCols;
-    stage_block(aiT, Ai_blk, 0, kD);
-    for (int e = tid; e < 4 * kD; e += kThreads) px.qin[e / kD][e % kD] = in_to_double(q[qrow0 * kD + e]);
+    for (int e = tid; e < kD * (kBlkRowBytes / 16); e += kThreads) {
+        const int c = e >> 5, part = e & 31, rr = c & 31;
+        double *row = reinterpret_cast<double *>(ai_base(c >> 5, rr >= 8) +
+                                                 (rr < 8 ? rr : rr - 8) * kBlkRowBytes);
+        cp_async16(row + 2 * part, Ai_blk + (size_t)c * kD + 2 * part);
+    }
+    const int nload = may_append ? min(n_new, kStepMaxNew) : 0;   // new rows this CTA may need
+    float vpre[kVPre];
+    if (nload > 0) {
+        stage_block(a_lo, A_blk, 0, 64);
+        const size_t in0 = unit * (size_t)n_new;
+        for (int e = tid; e < nload * kD; e += kThreads) ks_f[e] = in_to_float(k_new[in0 * kD + e]);
+#pragma unroll
+        for (int i = 0; i < kVPre; i++) {
+            const int e = tid + i * kThreads;
+            vpre[i] = e < nload * kD ? in_to_float(v_new[in0 * kD + e]) : 0.f;
+        }
+    }
+    cp_async_commit();
+    if (tid == 0) sh.s_len = seq_len[b];
+    for (int e = tid; e < 4 * kD; e += kThreads) px.qin[e % kD][e / kD] = in_to_double(q[qrow0 * kD + e]);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     __syncthreads();
 
     // new length (a step that would overflow the capacity appends nothing and
-    // raises KVQ_DEV_CAPACITY, like kvq_append) and this CTA's pages
+    // raises KVQ_DEV_CAPACITY, like kvq_append) and this pair's page pool;
+    // with a protected tier the last cluster reads the BF16 slots instead of
+    // pages, and the pages cover the coded tokens [sink_end, recent_start)
     const int L0 = sh.s_len;
     const bool ok = L0 >= 0 && L0 + n_new <= capacity;
     const int len = min(max(ok ? L0 + n_new : L0, 0), capacity);
-    // with a protected tier the last cluster reads the BF16 slots instead of
-    // pages; the pages cover the coded tokens [sink_end, recent_start)
-    const int NPt = n_sink + n_recent;
-    const int S_pages = S - (NPt > 0 ? kCluster : 0);
-    const bool is_tier = s >= S_pages;
     const Tier tr = tier_of(len, n_sink, n_recent);
-    const StepPlan plan = step_plan(tr.recent_start, S_pages);
-    const Split sp = is_tier ? Split{0, 0} : step_split(plan, s);
-    // New tokens w in [w0, w1) are transformed here: in the cluster whose
-    // splits hold their pages (it writes their codes before it stages those
-    // pages), or -- all of them -- in the tier cluster, which writes their
+    const Pool pool = unit_pool(tr.sink_end, tr.recent_start, s, warp >> 1, S_pages, kPairs * kCluster,
+                                kAppendRounds, !may_append);
+    // the first page's tail (no new token in it) is copied while the channels
+    // are chosen
+    if (!is_tier && !may_append && (tid & 63) == 0 && pool.index(0) >= 0)
+        issue_tail<NG>(sh, warp >> 1, 0, unit_pages + (size_t)pool.page(pool.index(0)) * page_bytes(2, NG));
+    // New tokens w in [w0, w1) are transformed here: in the first cluster,
+    // those whose pages are in the pool (its pairs read them first, after the
+    // append), or -- all of them -- in the tier cluster, which writes their
     // BF16 slots and the codes of pages no split reads in this step.
     int w0 = 0, w1 = 0;
     if (ok && n_new > 0) {
         if (is_tier) {
             w1 = n_new;
-        } else {
-            const int s_first = s - r;
-            w0 = n_new;
-            for (int w = n_new - 1; w >= 0; w--) {
-                const int pg = (L0 + w) / kT;
-                const int owner = pg < plan.nblk ? owner_of(plan, pg) : -1;
-                if (owner >= s_first && owner < s_first + kCluster) {
-                    w1 = max(w1, w + 1);
-                    w0 = w;
-                }
-            }
-            if (w1 == 0) w0 = 0;
+        } else if (s < kCluster) {
+            for (int w = 0; w < n_new; w++)
+                if ((L0 + w) / kT < pool.P1) w1 = w + 1;
         }
     }
-    const int nw = w1 - w0;
-    const size_t in_base = unit * (size_t)n_new + w0;
-    float vpre[kVPre];
-    if (nw > 0) {
-        stage_block(a_lo, A_blk, 0, 64);
-        for (int e = tid; e < nw * kD; e += kThreads) ks_f[e] = in_to_float(k_new[in_base * kD + e]);
-#pragma unroll
-        for (int i = 0; i < kVPre; i++) {
-            const int e = tid + i * kThreads;
-            vpre[i] = e < nw * kD ? in_to_float(v_new[in_base * kD + e]) : 0.f;
-        }
-    }
-    cp_async_commit();
+    const int nw = w1 - w0;           // w0 = 0: the rows loaded above are tokens 0..nw-1
     // every CTA of sequence b has read its length once the counter reaches
     // S * Hkv; the last one stores the new length
     if (tid == 0) {
@@ -887,13 +1053,37 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
     __syncthreads();
 
     // q'[hl][64r + jj] = sum_c q[hl][c] Ainvt[c][64r + jj], fma chain c =
-    // 0..127 from 0.0; hl = warp / 2, jj = 32 (warp % 2) + lane
-    {
-        const int hl = warp >> 1, jj = (warp & 1) * 32 + lane;
-        double acc = 0.0;
-#pragma unroll 16
-        for (int c = 0; c < kD; c++) acc = fma(px.qin[hl][c], aiT[c][jj], acc);
-        sh.qp_own[hl][jj] = acc;
+    // 0..127 from 0.0, the four heads' chains side by side in thread jj (each
+    // A^{-T} element loaded once); then the pooled energy of channel 64r + jj,
+    // with a diagonal refinement of the base queries q'_{h,j} / delta_j (the
+    // arithmetic of kvq_select_channels)
+    if (tid < kCols) {
+        double acc[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 1
+        for (int p = 0; p < 4; p++) {
+            const double *lo8 = reinterpret_cast<const double *>(ai_base(p, 0));
+            const double *hi24 = reinterpret_cast<const double *>(ai_base(p, 1));
+#pragma unroll
+            for (int rr = 0; rr < 32; rr++) {
+                const int c = 32 * p + rr;
+                const double a = rr < 8 ? lo8[rr * kCols + tid] : hi24[(rr - 8) * kCols + tid];
+                const double2 q01 = *reinterpret_cast<const double2 *>(&px.qin[c][0]);
+                const double2 q23 = *reinterpret_cast<const double2 *>(&px.qin[c][2]);
+                acc[0] = fma(q01.x, a, acc[0]);
+                acc[1] = fma(q01.y, a, acc[1]);
+                acc[2] = fma(q23.x, a, acc[2]);
+                acc[3] = fma(q23.y, a, acc[3]);
+            }
+        }
+        const double dj = delta ? delta[(size_t)h * kD + r * kCols + tid] : 1.0;
+        double e = 0.0;
+#pragma unroll
+        for (int hl = 0; hl < 4; hl++) {
+            sh.qp_own[hl][tid] = acc[hl];
+            const double u = delta ? acc[hl] / dj : acc[hl];
+            e = fma(u, u, e);
+        }
+        sh.e2_own[tid] = e;
     }
     __syncthreads();                                // A^{-T} block no longer needed
     if (nw > 0) {
@@ -983,7 +1173,7 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
                 vhi = fmax(fmax(sh.trange[w2][3], sh.trange[w2 + 1][3]), fmax(peer->trange[w2][3], peer->trange[w2 + 1][3]));
             }
         }
-        if (w < nw && (!is_tier || (L0 + w0 + w) / kT >= plan.nblk)) {
+        if (w < nw && (!is_tier || (L0 + w0 + w) / kT >= pool.P1)) {
             const int g = NG == 1 ? 0 : 2 * r + (warp & 1);                  // metadata group
             const bool meta_writer = NG == 1 ? (r == 0 && (warp & 1) == 0 && lane == 0) : lane == 0;
             const int pos = L0 + w0 + w, tt = pos % kT;
@@ -1007,18 +1197,6 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
         }
     }
     __syncthreads();
-    if (tid < kCols) {
-        // pooled energy; with a diagonal refinement, of the base queries
-        // q'_{h,j} / delta_j (the arithmetic of kvq_select_channels)
-        const double dj = delta ? delta[(size_t)h * kD + r * kCols + tid] : 1.0;
-        double e = 0.0;
-#pragma unroll
-        for (int hl = 0; hl < 4; hl++) {
-            const double u = delta ? sh.qp_own[hl][tid] / dj : sh.qp_own[hl][tid];
-            e = fma(u, u, e);
-        }
-        sh.e2_own[tid] = e;
-    }
     cluster.sync();            // the cluster's q', energies and new tokens are in place
     if (tid < kD) {
         const MmaShared *peer = cluster.map_shared_rank(&sh, tid / kCols);
@@ -1088,8 +1266,8 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
         tier_cta(sh, unit_slots(pages, B, Hkv, NB, 2, unit, NPt, NG), len, n_sink, n_recent, s - S_pages, k, part_o,
                  part_ml, qrow0, S, s, out, status + 1 + B + unit, rot);
     else
-        run_pages<NG>(sh, unit_pages, tr.sink_end, tr.recent_start, sp, S, s, qrow0, part_o, part_ml, out,
-                      status + 1 + B + unit, status, false, rot, 0, [](int) {});
+        run_pages<NG, true>(sh, unit_pages, tr.sink_end, tr.recent_start, Split{0, 0}, pool, S, s, qrow0, part_o,
+                            part_ml, out, status + 1 + B + unit, status, kWaitPolls, rot, 0, [](int) {});
     cluster_wait();            // the other CTA no longer reads this CTA's shared memory
 }
 
@@ -1107,35 +1285,48 @@ int decode_mma_splits(int units, int nblk, int num_sms, int tier) {
     S -= S % kCluster;
     return (S < kCluster ? kCluster : S) + tier;
 }
-
 int step_mma_max_new() { return kStepMaxNew; }
 
-template <int NG, bool BK>
+uint32_t default_wait_polls() { return kWaitPolls; }
+
+template <int NG, bool BK, bool STEP>
 cudaError_t launch_decode_mma_t(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
                                 const float *qgsum, int k, float *part_o, float2 *part_ml, int S,
-                                float *out, cudaStream_t st) {
+                                float *out, uint32_t polls, int n_new, cudaStream_t st) {
     const size_t smem = sizeof(MmaShared);
     static std::atomic<uint64_t> done{0};
-    cudaError_t e = set_smem_once(decode_mma_kernel<NG, BK>, (int)smem, done);
+    cudaError_t e = set_smem_once(decode_mma_kernel<NG, BK, STEP>, (int)smem, done);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)S, (unsigned)c.n_kv_heads, (unsigned)c.batch);
-    decode_mma_kernel<NG, BK><<<grid, kThreads, smem, st>>>(static_cast<const uint8_t *>(c.pages), c.seq_len,
-                                                            c.n_kv_heads, c.capacity / kT, Hq, idx, qsel, qgsum, k,
-                                                            part_o, part_ml, S, out, unit_counter(c, 0, 0), c.status,
-                                                            c.n_sink, c.n_recent, c.v_rot, buckets_of(c),
-                                                            c.bucket / kT);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)S, (unsigned)c.n_kv_heads, (unsigned)c.batch);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    // a step's decode may start while the preparation kernel still runs
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = STEP ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, decode_mma_kernel<NG, BK, STEP>, static_cast<const uint8_t *>(c.pages),
+                              c.seq_len, (int)c.n_kv_heads, c.capacity / kT, Hq, idx, qsel, qgsum, k, part_o,
+                              part_ml, S, out, unit_counter(c, 0, 0), c.status, (int)c.n_sink, (int)c.n_recent,
+                              c.v_rot, buckets_of(c), c.bucket / kT, polls, n_new);
 }
 
 cudaError_t launch_decode_mma(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
                               const float *qgsum, int k, float *part_o, float2 *part_ml, int S,
-                              float *out, cudaStream_t st) {
+                              float *out, uint32_t polls, cudaStream_t st) {
     const bool one = groups_of(c) == 1, bk = c.bucket > 0;
     if (bk)
-        return one ? launch_decode_mma_t<1, true>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, st)
-                   : launch_decode_mma_t<kNG, true>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, st);
-    return one ? launch_decode_mma_t<1, false>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, st)
-               : launch_decode_mma_t<kNG, false>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, st);
+        return one ? launch_decode_mma_t<1, true, false>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, polls,
+                                                         0, st)
+                   : launch_decode_mma_t<kNG, true, false>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out,
+                                                           polls, 0, st);
+    return one ? launch_decode_mma_t<1, false, false>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, polls,
+                                                      0, st)
+               : launch_decode_mma_t<kNG, false, false>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, polls,
+                                                        0, st);
 }
 
 template <typename Tin, int NG>
@@ -1155,6 +1346,7 @@ cudaError_t launch_step_mma_t(const kvq_cache &c, int Hq, const void *q, const v
     return cudaGetLastError();
 }
 
+// The whole decode step in one launch (no RoPE buckets).
 cudaError_t launch_step_mma(const kvq_cache &c, int Hq, const void *q, const void *k_new, const void *v_new,
                             int dtype, int n_new, const double *A, const double *Ainvt, const double *delta,
                             int k, int32_t *idx, float *qsel, float *qgsum, float *part_o, float2 *part_ml,
@@ -1169,6 +1361,19 @@ cudaError_t launch_step_mma(const kvq_cache &c, int Hq, const void *q, const voi
                                                 qgsum, part_o, part_ml, S, out, st)
                : launch_step_mma_t<uint16_t, kNG>(c, Hq, q, k_new, v_new, n_new, A, Ainvt, delta, k, idx, qsel,
                                                   qgsum, part_o, part_ml, S, out, st);
+}
+
+// The decode of a step with RoPE buckets whose preparation kernel (the
+// per-bucket channel choice + the append of n_new tokens) was launched just
+// before it on `st`.
+cudaError_t launch_decode_mma_step(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
+                                   const float *qgsum, int k, float *part_o, float2 *part_ml, int S,
+                                   float *out, int n_new, cudaStream_t st) {
+    return groups_of(c) == 1
+               ? launch_decode_mma_t<1, true, true>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, kWaitPolls,
+                                                    n_new, st)
+               : launch_decode_mma_t<kNG, true, true>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out,
+                                                      kWaitPolls, n_new, st);
 }
 
 size_t decode_mma_smem_bytes() { return sizeof(MmaShared); }

@@ -196,11 +196,11 @@ cudaError_t set_smem_once(Kernel *fn, int bytes, std::atomic<uint64_t> &done) {
 // softmax over the whole context (Dual-QK §3.4).  Nothing waits: the other
 // CTAs simply exit.  Called by every thread of an NT-thread CTA; `scratch` is
 // 16-byte aligned shared memory for merge_scratch_floats(G, NT, S) floats.
-// The (m, l) pairs are read in one parallel pass and turned into per-split
-// weights; then the G * 128 outputs, as float4 columns, are summed over the
-// splits with R = NT / columns threads per column (each a strided subset of
-// the splits, many independent loads in flight), and the R partial sums are
-// added in a fixed order.
+// The G * 128 outputs, as float4 columns, are summed over the splits with
+// R = NT / columns threads per column (each a strided subset of the splits);
+// the first kMergeChunk partials of every thread are loaded together with
+// the (m, l) pairs, so the merge costs one round trip to L2 for S <= R *
+// kMergeChunk, and the R partial sums are added in a fixed order.
 // With a value rotation `rot` (the unit's KV head's 128 x 128 float64 matrix,
 // row-major, 16-byte aligned; values were stored as V rot) the merged output
 // is rotated back, out[c] = sum_j o[j] rot[c][j] (rot is orthogonal; §3.3
@@ -213,6 +213,7 @@ struct MergeShape {
     static constexpr int CPT = NT >= F ? 1 : F / NT;     // columns per thread
     static_assert(NT >= F ? NT % F == 0 : F % NT == 0, "merge: columns and threads must divide");
 };
+constexpr int kMergeChunk = 20;
 __host__ __device__ constexpr int merge_scratch_floats(int G, int NT, int S) {
     return ((2 * G * S + G + 3) & ~3) + (NT > G * kD / 4 ? NT / (G * kD / 4) * G * kD : 0) + G * kD;
 }
@@ -247,10 +248,26 @@ __device__ __forceinline__ void merge_unit_if_last(const float *part_o, const fl
         o[2] = a.z;
         o[3] = a.w;
     };
+    const int sub = t / (NT / MS::R >= 1 ? NT / MS::R : 1);   // split subset of this thread
+    const int col0 = (t % (NT / MS::R)) * MS::CPT;
+    auto column = [&](int col) {
+        const int hl = (4 * col) / kD, c0 = (4 * col) % kD;
+        return reinterpret_cast<const float4 *>(part_o + ((qrow0 + hl) * S) * kD + c0);
+    };
+    // the first chunk of the first column's partials, in flight with the (m, l) pass
+    float4 v[kMergeChunk];
+    {
+        const float4 *po = column(col0);
+#pragma unroll
+        for (int j = 0; j < kMergeChunk; j++) {
+            const int sj = sub + j * MS::R;
+            v[j] = sj < S ? __ldcg(po + (size_t)sj * (kD / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
     for (int e = t; e < G * S; e += NT) {
-        const float2 v = __ldcg(part_ml + qrow0 * S + e);     // rows qrow0.. are contiguous
-        wm[e] = v.x;
-        wl[e] = v.y;
+        const float2 ml = __ldcg(part_ml + qrow0 * S + e);     // rows qrow0.. are contiguous
+        wm[e] = ml.x;
+        wl[e] = ml.y;
     }
     __syncthreads();
     for (int hl = warp; hl < G; hl += NT / 32) {
@@ -269,21 +286,28 @@ __device__ __forceinline__ void merge_unit_if_last(const float *part_o, const fl
         if (lane == 0) inv[hl] = L > 0.f ? 1.f / L : 0.f;
     }
     __syncthreads();
-    const int sub = t / (NT / MS::R >= 1 ? NT / MS::R : 1);   // split subset of this thread
-    const int col0 = (t % (NT / MS::R)) * MS::CPT;
 #pragma unroll
     for (int cc = 0; cc < MS::CPT; cc++) {
         const int col = col0 + cc, hl = (4 * col) / kD, c0 = (4 * col) % kD;
-        const float4 *po = reinterpret_cast<const float4 *>(part_o + ((qrow0 + hl) * S) * kD + c0);
+        const float4 *po = column(col);
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-        for (int s = sub; s < S; s += MS::R) {
-            const float w = wm[hl * S + s];
-            const float4 v = __ldcg(po + (size_t)s * (kD / 4));
-            acc.x = fmaf(w, v.x, acc.x);
-            acc.y = fmaf(w, v.y, acc.y);
-            acc.z = fmaf(w, v.z, acc.z);
-            acc.w = fmaf(w, v.w, acc.w);
+        for (int j0 = 0; sub + j0 * MS::R < S; j0 += kMergeChunk) {
+            if (cc > 0 || j0 > 0) {
+#pragma unroll
+                for (int j = 0; j < kMergeChunk; j++) {
+                    const int sj = sub + (j0 + j) * MS::R;
+                    v[j] = sj < S ? __ldcg(po + (size_t)sj * (kD / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < kMergeChunk; j++) {
+                const int sj = sub + (j0 + j) * MS::R;
+                const float w = sj < S ? wm[hl * S + sj] : 0.f;
+                acc.x = fmaf(w, v[j].x, acc.x);
+                acc.y = fmaf(w, v[j].y, acc.y);
+                acc.z = fmaf(w, v[j].z, acc.z);
+                acc.w = fmaf(w, v[j].w, acc.w);
+            }
         }
         if constexpr (MS::R == 1) {
             const float r = inv[hl];
@@ -298,8 +322,8 @@ __device__ __forceinline__ void merge_unit_if_last(const float *part_o, const fl
             const int hl = (4 * col) / kD, c0 = (4 * col) % kD;
             float4 a = part[col];
             for (int q = 1; q < MS::R; q++) {
-                const float4 v = part[q * MS::F + col];
-                a.x += v.x; a.y += v.y; a.z += v.z; a.w += v.w;
+                const float4 v2 = part[q * MS::F + col];
+                a.x += v2.x; a.y += v2.y; a.z += v2.z; a.w += v2.w;
             }
             const float r = inv[hl];
             emit(hl, c0, make_float4(a.x * r, a.y * r, a.z * r, a.w * r));
@@ -477,7 +501,8 @@ int decode_splits(const kvq_cache &c, int Hq, int k, int num_sms);
 size_t decode_ws_bytes(const kvq_cache &c, int Hq, int n_splits);
 cudaError_t launch_decode(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
                           const float *qgsum, int k, float *out, void *ws, int n_splits,
-                          cudaStream_t st);
+                          cudaStream_t st, long long polls = -1);
+bool decode_uses_mma(const kvq_cache &c, int Hq);
 cudaError_t launch_decode_step(const kvq_cache &c, int Hq, const void *q, const void *k_new,
                                const void *v_new, int dtype, int n_new, const double *A,
                                const double *Ainvt, const double *delta, int k, int32_t *idx, float *qsel,

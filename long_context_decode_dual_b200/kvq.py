@@ -59,6 +59,7 @@ EXPORTS = (
     "kvq_bf16_decode_workspace", "kvq_bf16_decode_attn", "kvq_read_status",
     "kvq_status_string", "kvq_version", "kvq_decode_static_scratch_bytes",
     "kvq_decode_attn_static", "kvq_decode_step", "kvq_num_buckets", "kvq_copy_async",
+    "kvq_decode_attn_wait_bound",
 )
 
 
@@ -92,6 +93,7 @@ def lib() -> ctypes.CDLL:
             "kvq_decode_step": (I, [C, P, P, P, I, I, I, P, P, P, ctypes.c_float, P, P, P, P, P, S, P]),
             "kvq_num_buckets": (I, [C]),
             "kvq_copy_async": (I, [P, P, S, P]),
+            "kvq_decode_attn_wait_bound": (I, [C, I, P, P, P, I, P, P, S, ctypes.c_uint32, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -290,6 +292,22 @@ def decode_attn(cache: KVCache, sel: Selection, out: Optional[torch.Tensor] = No
     _check("kvq_decode_attn", lib().kvq_decode_attn(
         ctypes.byref(cache.desc), Hq, _ptr(sel.idx), _ptr(sel.qsel), _ptr(sel.qgsum), k, _ptr(out),
         _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def decode_attn_wait_bound(cache: KVCache, sel: Selection, wait_polls: int, out: Optional[torch.Tensor] = None,
+                           ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """kvq_decode_attn_wait_bound: kvq_decode_attn with an explicit bound on
+    each wait for a staged page (a fault-handling test hook; 0 gives up at
+    once unless the page has landed, which sets KVQ_DEV_TIMEOUT)."""
+    B, Hq, k = cache.batch, int(sel.qsel.shape[1]), sel.k
+    if out is None:
+        out = torch.empty(B, Hq, HEAD_DIM, dtype=torch.float32, device=sel.qsel.device)
+    if ws is None:
+        ws = alloc_workspace(decode_workspace_bytes(cache, Hq, k), sel.qsel.device)
+    _check("kvq_decode_attn_wait_bound", lib().kvq_decode_attn_wait_bound(
+        ctypes.byref(cache.desc), Hq, _ptr(sel.idx), _ptr(sel.qsel), _ptr(sel.qgsum), k, _ptr(out),
+        _ptr(ws), ws.numel(), int(wait_polls), _stream(stream)))
     return out
 
 

@@ -98,8 +98,12 @@ def test_decode_parity(bits, g, w, group):
 
 def test_one_bucket_equals_no_buckets():
     """Buckets as large as the capacity: anchor 0 (cos 1, sin 0) leaves keys
-    and queries as they are; pages, channels and outputs are those of the
-    cache without buckets, bit for bit."""
+    and queries as they are; pages and channels are those of the cache
+    without buckets, bit for bit, and so are the scores and weights of every
+    token.  The outputs agree to float32 summation order only: a bucketed
+    decode reads each split's pages as one contiguous range (one segment per
+    bucket), an unbucketed one deals the pages round-robin to the pairs, so
+    the splits' partial sums are formed in different orders."""
     base = W.workload("llama8b_b8_32k", batch=2)
     outs = []
     for w in (0, 2048):
@@ -112,7 +116,8 @@ def test_one_bucket_equals_no_buckets():
         outs.append((cache.all_pages().clone(), sel.idx.reshape(2, 8, -1).clone(), out.clone()))
     assert torch.equal(outs[0][0], outs[1][0])
     assert torch.equal(outs[0][1], outs[1][1])
-    assert torch.equal(outs[0][2], outs[1][2])
+    emax, _ = rel_errors(outs[0][2].cpu().numpy(), outs[1][2].cpu().numpy())
+    assert emax <= 1e-5, emax
 
 
 @pytest.mark.parametrize("sparsity", W.SWEEP_SPARSITIES)
