@@ -90,7 +90,7 @@ constexpr uint32_t kWaitPolls = 1u << 20;         // bound on mbarrier polls per
 constexpr int kStepMaxNew = 4;                    // new tokens per fused step
 constexpr int kCluster = 2;                       // CTAs per cluster of the fused step
 constexpr int kCols = kD / kCluster;              // channels whose q' one CTA of a cluster computes
-constexpr int kAppendRounds = 1;                  // rounds the appending cluster's pairs sit out
+constexpr int kAppendRounds = 2;                  // rounds the appending cluster's pairs sit out
 
 struct __align__(16) MmaShared {
     uint8_t stage[kPairs][2][kStageBytes];
@@ -104,7 +104,7 @@ struct __align__(16) MmaShared {
     uint32_t touched[2];               // chunk bitmask halves
     uint32_t tx_keys;                  // bytes of the key-chunk copies of one page
     int n_copies;
-    int warp_cnt[4];
+    uint32_t selmask[4];               // fused step: the channel choice, 128 bits
     int s_len;
     double qp_own[4][kCols];           // fused step: q' of this CTA's channels (read by the cluster)
     double e2_own[kCols];              // and their pooled energies
@@ -146,11 +146,7 @@ constexpr int kOffVs = kOffKs + kStepMaxNew * kD * (int)sizeof(double);
 static_assert(kOffVs + kStepMaxNew * kD * (int)sizeof(double) <= kOffALo, "new rows below the low rows of A");
 constexpr int kVPre = kStepMaxNew * kD / kThreads;                 // value elements per thread
 static_assert(kVPre * kThreads == kStepMaxNew * kD, "value rows split evenly over the threads");
-struct BqScratch {                     // in MmaShared::bq
-    int sel[kD];
-};
 static_assert(sizeof(PexScratch) <= sizeof(((MmaShared *)0)->pex), "query and key rows fit the exchange buffers");
-static_assert(sizeof(BqScratch) <= sizeof(((MmaShared *)0)->bq), "value rows and flags fit the fragment table");
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -414,14 +410,16 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
     const int gid = lane >> 2, tig = lane & 3;
     const int hh = gid >> 1, part = gid & 1;
 
-    // zero-point and channel-0 coefficients of head tig, pre-scaled to the
-    // base-2 score domain (reloaded for each bucket's segment)
-    float qg_t[NG];
+    // Channel-0 coefficient of head tig, and the B fragment of the score
+    // zero-point MMA: k-slot 2tig holds group tig's sum of kept q' of head
+    // gid >> 1 (hi or lo fp16 part by gid & 1), every other k-slot 0; both
+    // pre-scaled to the base-2 score domain (reloaded for each bucket's
+    // segment)
     float q0_t = 0.f;
+    uint32_t bz = 0;
     auto load_coef = [&]() {
-#pragma unroll
-        for (int g = 0; g < NG; g++) qg_t[g] = sh.qg[tig][g] * kScoreScaleLog2;
         q0_t = sh.q[tig][0] * kScoreScaleLog2;
+        bz = tig < NG ? (uint32_t)f16_part(sh.qg[hh][tig] * kScoreScaleLog2, part) : 0u;
     };
     load_coef();
 
@@ -449,12 +447,9 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
         const uint32_t *vmeta = kmeta + NG * kT;
 
         // ---------------- scores: tokens 16gid + 8half + 2i + r, head tig
-        float sc[4][2], zt[4][2];
+        float sc[4][2];
 #pragma unroll
-        for (int i = 0; i < 4; i++) {
-            sc[i][0] = sc[i][1] = 0.f;
-            zt[i][0] = zt[i][1] = 0.f;
-        }
+        for (int i = 0; i < 4; i++) sc[i][0] = sc[i][1] = 0.f;
         const uint8_t *kb = cur + tig * 32 + 4 * gid;
 #pragma unroll
         for (int g = 0; g < NG; g++) {
@@ -483,7 +478,7 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
                         mma16816(C[i], x1 & m0, x1 & m1, x2 & m0, x2 & m1, bb.x, bb.y);
                 }
             }
-            // scale and zero-point of group g for the thread's 8 tokens
+            // scale of group g for the thread's 8 tokens
 #pragma unroll
             for (int q4 = 0; q4 < 2; q4++) {
                 const uint4 w = *reinterpret_cast<const uint4 *>(
@@ -493,9 +488,26 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
                 for (int e = 0; e < 4; e++) {
                     const int tt = 4 * q4 + e, i = tt >> 1, r = tt & 1;
                     sc[i][r] = fmaf(lo_f16(ws[e]), C[i][2 * r] + C[i][2 * r + 1], sc[i][r]);
-                    zt[i][r] = fmaf(hi_f16(ws[e]), qg_t[g], zt[i][r]);
                 }
             }
+        }
+        // zero-point term sum_g zero_g(t) qgsum_g, one MMA per tile: thread
+        // tig puts its group's fp16 zero point (exact) of tokens T and T+1
+        // (rows gid and gid+8) into k-slot 2tig; the rest of A is 0
+        float Cz[4][4];
+        {
+            const int zg = tig < NG ? tig : 0;
+            uint32_t zw[8];
+#pragma unroll
+            for (int q4 = 0; q4 < 2; q4++) {
+                const uint4 w = *reinterpret_cast<const uint4 *>(
+                    kmeta + 128 * zg + 4 * meta_chunk(zg, 4 * gid + 2 * half + q4));
+                zw[4 * q4] = w.x; zw[4 * q4 + 1] = w.y; zw[4 * q4 + 2] = w.z; zw[4 * q4 + 3] = w.w;
+            }
+            const uint32_t zkeep = tig < NG ? 0xffffffffu : 0u;
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+                mma16816_z(Cz[i], (zw[2 * i] >> 16) & zkeep, (zw[2 * i + 1] >> 16) & zkeep, 0u, 0u, bz, 0u);
         }
         // full scores (base-2 domain), masked beyond the sequence on the last page
         float mx = -INFINITY;
@@ -509,7 +521,7 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
                     const float c0v = __uint_as_float(r ? (ws[i] & 0xffff0000u) : (ws[i] << 16));
                     // 2^(24 - field position) undoes the code scaling; times log2(e)/sqrt(d)
                     const float comp = __int_as_float((127 + 24 - 4 * (i & 1) - 2 * r) << 23) * kScoreScaleLog2;
-                    sc[i][r] = fmaf(sc[i][r], comp, fmaf(q0_t, c0v, zt[i][r]));
+                    sc[i][r] = fmaf(sc[i][r], comp, fmaf(q0_t, c0v, Cz[i][2 * r] + Cz[i][2 * r + 1]));
                 }
             }
             if (pg * kT < lo || (pg + 1) * kT > hi) {       // page with tokens outside [lo, hi)
@@ -911,8 +923,11 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, int32_t *__restrict__ seq_l
         pool.tail_issued = early;
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
         __syncthreads();                              // barriers initialised before copies complete on them
-        if ((tid & 63) == 0 && early)
-            issue_tail<NG>(sh, warp >> 1, 0, unit_pages + (size_t)pool.page(pool.index(0)) * page_bytes(2, NG));
+        if ((tid & 63) == 0 && early) {
+            const uint8_t *first = unit_pages + (size_t)pool.page(pool.index(0)) * page_bytes(2, NG);
+            issue_tail<NG>(sh, warp >> 1, 0, first);
+            prefetch_l2(first, kKeyBytes);      // the key rows: in L2 once the choice is loaded
+        }
         after_prep();
         load_sel(0);
         run_pages<NG, true>(sh, unit_pages, tr.sink_end, tr.recent_start, Split{0, 0}, pool, S, s, qrow0, part_o,
@@ -928,6 +943,7 @@ __device__ __forceinline__ void cluster_wait() {
     asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
 }
 
+static_assert(4 * kD == 2 * kThreads, "two query elements per thread");
 template <typename Tin, int NG>
 __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 2)
 step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint32_t *__restrict__ status,
@@ -950,7 +966,6 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
     float *ks_f = &sh.q[0][0];                                                   // [nw][128]
     double (*ks)[kD] = reinterpret_cast<double (*)[kD]>(P + kOffKs);             // [nw][128], later
     double (*vsd)[kD] = reinterpret_cast<double (*)[kD]>(P + kOffVs);            // [nw][128], later
-    BqScratch &bx = *reinterpret_cast<BqScratch *>(&sh.bq[0][0]);
 
     cg::cluster_group cluster = cg::this_cluster();
     const int r = (int)cluster.block_rank();        // channels 64r..64r+63
@@ -985,6 +1000,11 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
     // query, and in the CTAs that may append, A's low rows and the new rows
     if (tid < kD) sh.chan_pos[tid] = -1;
     if (tid < 2 * kPairs) mbar_init(smem_u32(&sh.mbar[tid >> 1][tid & 1]), 1);
+    // the length and the query first: small, and what the first barrier waits for
+    if (tid == 0) sh.s_len = seq_len[b];
+    double qv[2];
+#pragma unroll
+    for (int i = 0; i < 2; i++) qv[i] = in_to_double(q[qrow0 * kD + tid + i * kThreads]);
     const double *Ai_blk = Ainvt + (size_t)h * kD * kD + r * kCols;
     const double *A_blk = A + (size_t)h * kD * kD + r * kCols;
     for (int e = tid; e < kD * (kBlkRowBytes / 16); e += kThreads) {
@@ -1006,8 +1026,11 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
         }
     }
     cp_async_commit();
-    if (tid == 0) sh.s_len = seq_len[b];
-    for (int e = tid; e < 4 * kD; e += kThreads) px.qin[e % kD][e / kD] = in_to_double(q[qrow0 * kD + e]);
+#pragma unroll
+    for (int i = 0; i < 2; i++) {
+        const int e = tid + i * kThreads;
+        px.qin[e % kD][e / kD] = qv[i];
+    }
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     __syncthreads();
 
@@ -1023,8 +1046,11 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
                                 kAppendRounds, !may_append);
     // the first page's tail (no new token in it) is copied while the channels
     // are chosen
-    if (!is_tier && !may_append && (tid & 63) == 0 && pool.index(0) >= 0)
-        issue_tail<NG>(sh, warp >> 1, 0, unit_pages + (size_t)pool.page(pool.index(0)) * page_bytes(2, NG));
+    if (!is_tier && !may_append && (tid & 63) == 0 && pool.index(0) >= 0) {
+        const uint8_t *first = unit_pages + (size_t)pool.page(pool.index(0)) * page_bytes(2, NG);
+        issue_tail<NG>(sh, warp >> 1, 0, first);
+        prefetch_l2(first, kKeyBytes);          // the key rows: in L2 once the choice is made
+    }
     // New tokens w in [w0, w1) are transformed here: in the first cluster,
     // those whose pages are in the pool (its pairs read them first, after the
     // append), or -- all of them -- in the tier cluster, which writes their
@@ -1198,25 +1224,33 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
     }
     __syncthreads();
     cluster.sync();            // the cluster's q', energies and new tokens are in place
+    // the 128 energies and all of q', this CTA's half and the peer's (each
+    // thread's five values loaded before it stores any)
+    double my_q[4] = {0.0, 0.0, 0.0, 0.0};
     if (tid < kD) {
         const MmaShared *peer = cluster.map_shared_rank(&sh, tid / kCols);
         const int l = tid % kCols;
-        e2[tid] = peer->e2_own[l];
+        const double my_e = peer->e2_own[l];
 #pragma unroll
-        for (int hl = 0; hl < 4; hl++) qp[hl][tid] = peer->qp_own[hl][l];
+        for (int hl = 0; hl < 4; hl++) my_q[hl] = peer->qp_own[hl][l];
+        e2[tid] = my_e;
+#pragma unroll
+        for (int hl = 0; hl < 4; hl++) qp[hl][tid] = my_q[hl];
     }
     __syncthreads();
     cluster_arrive();          // done reading the other CTA's shared memory (waited for at exit)
 
     // ---- channel choice (the arithmetic of kvq_select_channels)
     {
-        // energies are >= 0, so their bit patterns order like their values
-        // (integer compares keep the float64 pipe free)
+        // rank of channel j among 1..127 by (energy descending, index
+        // ascending), in two halves; energies are >= 0, so their bit
+        // patterns order like their values (integer compares keep the
+        // float64 pipe free)
         const int j = tid & (kD - 1), part = tid >> 7;
         const unsigned long long e = __double_as_longlong(e2[j]);
         int rk = 0;
         const int i0 = part == 0 ? 1 : 64, i1 = part == 0 ? 64 : kD;
-#pragma unroll 4
+#pragma unroll 8
         for (int i = i0; i < i1; i++) {
             const unsigned long long ei = __double_as_longlong(e2[i]);
             rk += (ei > e) || (ei == e && i < j);
@@ -1224,42 +1258,98 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
         rank_part[part][j] = rk;
     }
     __syncthreads();
-    int pos = -1;
     if (tid < kD) {
         const bool sel = (tid == 0) || (rank_part[0][tid] + rank_part[1][tid] < k - 1);
-        bx.sel[tid] = sel;
-        const unsigned ballot = __ballot_sync(0xffffffffu, sel);
-        if (lane == 0) sh.warp_cnt[warp] = __popc(ballot);
-        if (sel) pos = (int)__popc(ballot & ((1u << lane) - 1u));
+        const unsigned m = __ballot_sync(0xffffffffu, sel);
+        if (lane == 0) sh.selmask[warp] = m;
     }
     __syncthreads();
-    if (pos >= 0) {
-        for (int w = 0; w < warp; w++) pos += sh.warp_cnt[w];
-        sh.chan_pos[tid] = pos;
+    // Everything else follows from the 128-bit choice mask, in parallel:
+    // warps 0..3 the list positions, fp32 q' and the outputs; warp 4 the
+    // zero-point sums; warp 5 the copy list; every warp one k-step's B
+    // fragments.
+    uint32_t msk[4];
 #pragma unroll
-        for (int hl = 0; hl < 4; hl++) {
-            const float qf = (float)qp[hl][tid];
-            sh.q[hl][pos] = qf;
-            if (s == 0) qsel[(qrow0 + hl) * k + pos] = qf;
+    for (int w = 0; w < 4; w++) msk[w] = sh.selmask[w];
+    auto selected = [&](int c) {
+        const uint32_t m = c < 64 ? (c < 32 ? msk[0] : msk[1]) : (c < 96 ? msk[2] : msk[3]);
+        return (m >> (c & 31)) & 1u;
+    };
+    if (tid < kD) {
+        const uint32_t mw = warp < 2 ? (warp == 0 ? msk[0] : msk[1]) : (warp == 2 ? msk[2] : msk[3]);
+        if ((mw >> lane) & 1u) {
+            int pos = __popc(mw & ((1u << lane) - 1u));
+#pragma unroll
+            for (int w = 0; w < 3; w++) pos += w < warp ? __popc(msk[w]) : 0;
+            sh.chan_pos[tid] = pos;
+#pragma unroll
+            for (int hl = 0; hl < 4; hl++) {
+                const float qf = (float)my_q[hl];
+                sh.q[hl][pos] = qf;
+                if (s == 0) qsel[(qrow0 + hl) * k + pos] = qf;
+            }
+            if (s == 0) idx[unit * k + pos] = tid;
         }
-        if (s == 0) idx[unit * k + pos] = tid;
-    }
-    if (tid < 4 * kNG) {
+    } else if (warp == 4 && lane < 4 * kNG) {
         // zero-point sum of key group gr (channel 0 is bf16, not in group 0),
-        // kept channels ascending from 0.0; one grid per token: entry 0 sums
-        // every channel, the others are 0
-        const int hl = tid / kNG, gr = tid % kNG;
+        // kept channels ascending from 0.0 (a kept channel adds fma(1, q', s)
+        // = s + q' exactly, a dropped one fma(0, q', s) = s); one grid per
+        // token: entry 0 sums every channel, the others are 0
+        const int hl = lane / kNG, gr = lane % kNG;
         constexpr int GS = kD / NG;                 // channels per key group
         double sm = 0.0;
         if (gr < NG)
             for (int c = (gr == 0 ? 1 : gr * GS); c < (gr + 1) * GS; c++)
-                if (bx.sel[c]) sm += qp[hl][c];
+                sm = fma(selected(c) ? 1.0 : 0.0, qp[hl][c], sm);
         const float gf = (float)sm;
         sh.qg[hl][gr] = gf;
         if (s == 0) qgsum[(qrow0 + hl) * kNG + gr] = gf;
+    } else if (warp == 5 && lane == 0) {
+        // 64-byte chunks of key rows that hold a selected row (channel 0's
+        // row is unused), as runs; single unselected chunks between two
+        // selected ones filled in (one copy instead of two); then the tail
+        uint64_t T = 0;
+#pragma unroll
+        for (int w = 0; w < 4; w++) {
+            uint32_t x = w == 0 ? (msk[0] & ~1u) : msk[w];
+            x = (x | (x >> 1)) & 0x55555555u;       // chunk bit at each even position
+            x = (x | (x >> 1)) & 0x33333333u;       // then compressed to 16 bits
+            x = (x | (x >> 2)) & 0x0f0f0f0fu;
+            x = (x | (x >> 4)) & 0x00ff00ffu;
+            x = (x | (x >> 8)) & 0x0000ffffu;
+            T |= (uint64_t)x << (16 * w);
+        }
+        uint64_t Mr = T | ((T << 1) & (T >> 1));
+        int n = 0;
+        uint32_t bytes = 0;
+        while (Mr) {
+            const int st = __ffsll((long long)Mr) - 1;
+            const uint64_t inv = ~(Mr >> st);
+            const int len = inv ? __ffsll((long long)inv) - 1 : kChunks - st;
+            sh.copy[n++] = make_uint2(64u * (uint32_t)st, 64u * (uint32_t)len);
+            bytes += 64u * (uint32_t)len;
+            Mr = (len == kChunks) ? 0ull : (Mr & ~(((1ull << len) - 1ull) << st));
+        }
+        sh.copy[n++] = make_uint2((uint32_t)kKeyBytes, (uint32_t)fixed_bytes(2, NG));
+        sh.n_copies = n;
+        sh.tx_keys = bytes;
     }
+    {
+        // score-MMA B fragments of k-step `warp` (the layout build_plan
+        // writes): channel 0 and unselected channels get q' = 0
+        const int gid = lane >> 2, tig = lane & 3, hh = gid >> 1, part = gid & 1;
+        uint32_t w2[2];
+#pragma unroll
+        for (int r2 = 0; r2 < 2; r2++) {
+            const int c0 = 16 * warp + tig + 8 * r2, c1 = c0 + 4;
+            const float q0 = (c0 >= 1 && selected(c0)) ? (float)qp[hh][c0] : 0.f;
+            const float q1 = (c1 >= 1 && selected(c1)) ? (float)qp[hh][c1] : 0.f;
+            w2[r2] = (uint32_t)f16_part(q0, part) | ((uint32_t)f16_part(q1, part) << 16);
+        }
+        sh.bq[warp][lane] = make_uint2(w2[0], w2[1]);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     __syncthreads();
-    build_plan<NG>(sh, tid, warp, lane);
 
     const double *rot = v_rot ? v_rot + (size_t)h * kD * kD : nullptr;
     if (is_tier)
