@@ -189,10 +189,14 @@ def test_decode_edge_lengths():
     np.testing.assert_allclose(out[1, 0], Vh[0], rtol=1e-6, atol=1e-6)
 
 
-def test_bf16_comparator_matches_plain_attention():
-    wl = W.workload("llama8b_b8_32k", batch=2)
-    case = Case(wl, n_ctx=1000)
-    q = case.q(0)
+@pytest.mark.parametrize("g,n_ctx,qscale", [(4, 1000, 1.0), (1, 777, 1.0), (2, 130, 1.0), (8, 64, 1.0),
+                                             (4, 1, 1.0), (4, 3000, 8.0)])
+def test_bf16_comparator_matches_plain_attention(g, n_ctx, qscale):
+    """The unpruned BF16 comparator against the oracle's plain attention:
+    GQA 1/2/4/8, ragged tile tails, a single token, sharp attention."""
+    wl = W.workload("llama8b_b8_32k", batch=2, n_q_heads=8 * g)
+    case = Case(wl, n_ctx=n_ctx)
+    q = W.bf16_bits_from_f32((W.f32_from_bf16_bits(case.q(0)) * qscale).astype(np.float32))
     out = kvq.bf16_decode_attn(to_dev(q, "bf16"), to_dev(case.K, "bf16"), to_dev(case.V, "bf16")).cpu().numpy()
     g = wl.group_size
     for b in range(2):
