@@ -377,6 +377,8 @@ def run_ours(args):
     over = {"bits": args.bits, "n_steps": n_appends, **format_overrides(args)}
     if args.sparsity is not None:
         over["sparsity"] = args.sparsity
+    if args.batch is not None:
+        over["batch"] = args.batch
     wl = rank_workload(W.workload(args.workload, **over), rank)
     B, Hq, Hkv = wl.batch, wl.n_q_heads, wl.n_kv_heads
 
@@ -620,6 +622,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(W.WORKLOADS))
     ap.add_argument("--sparsity", type=float, default=None)
+    ap.add_argument("--batch", type=int, default=None,
+                    help="sequences per step (default: the workload's); for smaller profiling captures")
     ap.add_argument("--bits", type=int, default=2, choices=[2, 4])
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
