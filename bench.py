@@ -63,11 +63,12 @@ def measured_peaks():
 
 
 def decode_source_hash() -> str:
-    """Hash of the sources of the timed kernel (the fused step and the decode
-    kernels share kvq_decode_mma.cu and the internal header)."""
+    """Hash of the sources of the timed kernels (the step's preparation kernel
+    in kvq_select.cu, the decode kernels in kvq_decode*.cu, the internal
+    header)."""
     h = hashlib.sha256()
     for name in sorted(os.listdir(CSRC)):
-        if name.startswith("kvq_decode") or name.endswith(".cuh"):
+        if name.startswith("kvq_decode") or name == "kvq_select.cu" or name.endswith(".cuh"):
             with open(os.path.join(CSRC, name), "rb") as f:
                 h.update(name.encode())
                 h.update(f.read())
@@ -443,10 +444,10 @@ def run_ours(args):
         st.k_new.copy_(kv_pool[i % n_pool][0])
         st.v_new.copy_(kv_pool[i % n_pool][1])
 
-    # fused: one kvq_decode_step launch (with RoPE buckets two: the
-    # preparation kernel and the decode as its programmatic dependent);
-    # unfused: one-token append (with its length advance), select, decode
-    # (with its merge)
+    # step: one kvq_decode_step call = one fused launch (with RoPE buckets
+    # two: the preparation kernel and the decode as its programmatic
+    # dependent); unfused: one-token append (with its length advance),
+    # select, decode (with its merge)
     launches_per_step = (2 if wl.bucket else 1) if args.fused else 3
     lengths = [wl.n_ctx] * n_copies
     for st in steps:
@@ -509,7 +510,9 @@ def run_ours(args):
     value = job_throughput(sum(tokens), total_ms, world)
     assert kvq.read_status(cache) == 0
 
-    # roofline of the dominant kernel (decode partial + merge, timed together)
+    # roofline of the dominant kernel (decode partial + merge, timed together;
+    # a bucketed step's preparation kernel runs under the decode's first
+    # pages, so there the events bracket both launches)
     hbm_peak, peak_src = measured_peaks()
     alg_bytes = [alg_fn(wl, k, tok // (B * Hkv), protect) for tok in tokens]
     # bytes over time of all timed launches (not a mean of per-step ratios)
@@ -637,8 +640,7 @@ def main():
     ap.add_argument("--refine", action="store_true",
                     help="fold a diagonal refinement into the transforms; select on the base queries")
     ap.add_argument("--bucket", type=int, default=0,
-                    help="tokens per bucket of bucket-relative RoPE (the pages use 2048; 0: none); "
-                         "a bucketed step is two launches (preparation + decode)")
+                    help="tokens per bucket of bucket-relative RoPE (the pages use 2048; 0: none)")
     ap.add_argument("--pages-recipe", action="store_true",
                     help="the pages' whole format: --group 128 --protect --rotate-values --refine --bucket 2048")
     ap.add_argument("--unfused", dest="fused", action="store_false",

@@ -141,7 +141,7 @@ int kvq_select_channels(const kvq_cache *c, const void *q, int dtype, int n_q_he
 size_t kvq_decode_workspace(const kvq_cache *c, int n_q_heads, int k) {
     if (check_decode_args(c, n_q_heads, k)) return 0;
     const int S = decode_splits(*c, n_q_heads, k, num_sms());
-    return decode_ws_bytes(*c, n_q_heads, S);
+    return decode_ws_bytes(*c, n_q_heads, S, true);
 }
 
 int kvq_decode_attn(const kvq_cache *c, int n_q_heads, const int32_t *idx, const float *qsel,
@@ -198,7 +198,7 @@ int kvq_decode_step(const kvq_cache *c, const void *q, const void *k_new, const 
     const int sms = num_sms();
     if (sms <= 0) return KVQ_ERR_CUDA;
     const int S = decode_splits(*c, n_q_heads, k, sms);
-    if (!ws || ws_bytes < decode_ws_bytes(*c, n_q_heads, S)) return KVQ_ERR_WORKSPACE;
+    if (!ws || ws_bytes < decode_ws_bytes(*c, n_q_heads, S, true)) return KVQ_ERR_WORKSPACE;
     if (!aligned(ws, 16)) return KVQ_ERR_ALIGN;
     return cuda_status(launch_decode_step(*c, n_q_heads, q, k_new, v_new, dtype, n_new, A, Ainvt, delta, k, idx,
                                           qsel, qgsum, out, ws, S, (cudaStream_t)stream));

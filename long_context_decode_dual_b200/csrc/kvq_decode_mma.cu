@@ -45,12 +45,12 @@
 //
 // Page schedule (without RoPE buckets): the pages a unit reads form a pool,
 // taken from the last page backwards and dealt round-robin to the unit's
-// pairs (the appending cluster of a fused step sits out the second round).
-// The schedule is fixed by the shapes alone, so results are reproducible bit
-// for bit.  The tail of a page (everything but the key rows) does not depend
-// on the channel choice, so a pair copies its first tail before the choice
-// is made or loaded.  With RoPE buckets each split reads a contiguous range
-// of pages, one segment per bucket.
+// pairs.  The schedule is fixed by the shapes alone, so results are
+// reproducible bit for bit.  The tail of a page (everything but the key rows)
+// does not depend on the channel choice, so a pair copies the tails of its
+// first two pages, and brings their key rows into L2, before the choice is
+// loaded.  With RoPE buckets each split reads a contiguous range of pages,
+// one segment per bucket.
 //
 // The fused step kernel (kvq_decode_step without RoPE buckets) runs as
 // clusters of two CTAs, the two taking consecutive splits of one (sequence,
@@ -65,10 +65,15 @@
 // arithmetic of kvq_append; code bits are OR-ed into positions that are still
 // zero) before the same barrier, so those pages are staged after it.  (Pairs
 // of CTAs pack the SMs' two CTA slots exactly; clusters of four leave slots of
-// some GPCs unused.)  With RoPE buckets a step is two launches instead: the
-// preparation kernel (kvq_select.cu: the per-bucket channel choice and the
-// append) and this decode as its programmatic dependent, which waits for it
-// only before it reads what the preparation writes.
+// some GPCs unused.)
+//
+// With RoPE buckets a step is two launches: the preparation kernel
+// (kvq_select.cu: the channel choice of every bucket, the page plans and the
+// append of the step's new tokens) and this decode as its programmatic
+// dependent.  The decode's CTAs start while the preparation runs and stream
+// the tails of pages that hold no new token; they wait for it only before
+// they read what it writes (the plans, the new tokens' pages and protected
+// slots), then copy their plan in with 16-byte loads.
 #include "kvq_internal.cuh"
 
 #include <cooperative_groups.h>
@@ -85,7 +90,7 @@ constexpr int kFixBytes = fixed_bytes(2);         // value codes, ch0, metadata 
 constexpr int kStageBytes = kKeyBytes + kFixBytes;
 static_assert(kStageBytes == page_bytes(2) && page_bytes(2, 1) <= kStageBytes, "a stage holds one page image");
 constexpr int kChunks = kKeyBytes / 64;           // 64-byte chunks of key rows
-constexpr int kMaxCopies = kChunks / 2 + 2;       // runs after gap filling, plus the tail
+static_assert(kChunks == kPlanChunks, "the plan's chunks are the page's");
 constexpr uint32_t kWaitPolls = 1u << 20;         // bound on mbarrier polls per stage
 constexpr int kStepMaxNew = 4;                    // new tokens per fused step
 constexpr int kCluster = 2;                       // CTAs per cluster of the fused step
@@ -96,21 +101,16 @@ struct __align__(16) MmaShared {
     uint8_t stage[kPairs][2][kStageBytes];
     uint64_t mbar[kPairs][2];
     uint4 pex[kWarps][4][8];           // per warp: fp16 softmax weights [head][8-token block]
-    uint2 copy[kMaxCopies];            // {byte offset in the page, bytes}; the last one is the tail
-    uint2 bq[8][32];                   // score-MMA B fragments per k-step and lane
+    PagePlan plan;                     // score-MMA operands and copy list of the channel choice
     float q[4][kD];                    // qsel of the 4 heads, by selected position
-    float qg[4][kNG];
     int chan_pos[kD];                  // channel -> position in the selected list, -1 = not selected
     uint32_t touched[2];               // chunk bitmask halves
-    uint32_t tx_keys;                  // bytes of the key-chunk copies of one page
-    int n_copies;
     uint32_t selmask[4];               // fused step: the channel choice, 128 bits
     int s_len;
     double qp_own[4][kCols];           // fused step: q' of this CTA's channels (read by the cluster)
     double e2_own[kCols];              // and their pooled energies
     double trange[kWarps][4];          // fused step, one grid per token: per-warp key / value ranges
 };
-
 // Prologue scratch of the fused step.  Before the page loop the staging
 // memory P holds the 64-column block of A^{-T} as 128 rows of 512 bytes.  A
 // CTA that appends nothing keeps the tails of its pairs' first pages in
@@ -148,6 +148,7 @@ constexpr int kVPre = kStepMaxNew * kD / kThreads;                 // value elem
 static_assert(kVPre * kThreads == kStepMaxNew * kD, "value rows split evenly over the threads");
 static_assert(sizeof(PexScratch) <= sizeof(((MmaShared *)0)->pex), "query and key rows fit the exchange buffers");
 
+
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -176,53 +177,6 @@ __device__ __forceinline__ bool pair_sync_and(int pair, bool v) {
     return r != 0;
 }
 
-__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
-}
-// expect bytes without arriving (the arrival comes with the key copies)
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
-                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
-}
-// bring `bytes` (a multiple of 16, 16-byte aligned) of global memory into L2
-__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(src), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-    return ok != 0;
-}
-// Wait for a stage's copies.  The wait is bounded: after `polls` polls the
-// device status word gets KVQ_DEV_TIMEOUT and the caller is told; it then
-// issues no further copy, drains what it issued (drain_stage) and reports
-// that call's output invalid.  polls = 0 gives up at once unless the stage
-// has already landed (the path a test takes to exercise the give-up).
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint32_t *status,
-                                                  uint32_t polls) {
-    if (mbar_test_wait(bar, parity)) return true;
-    for (uint32_t i = 0; i < polls; i++)
-        if (mbar_try_wait(bar, parity)) return true;
-    atomicOr(status, (uint32_t)KVQ_DEV_TIMEOUT);
-    return false;
-}
 // After a give-up: wait (bounded by kWaitPolls) until the stage's copies
 // have landed, so that no copy still writes into shared memory when the CTA
 // goes on to reuse it or exits.
@@ -242,13 +196,6 @@ __device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__
 __device__ __forceinline__ float lo_f16(uint32_t w) { return __half2float(__ushort_as_half((uint16_t)(w & 0xffffu))); }
 __device__ __forceinline__ float hi_f16(uint32_t w) { return __half2float(__ushort_as_half((uint16_t)(w >> 16))); }
 
-// fp16 hi/lo split of a float: hi = fp16(x), lo = fp16(x - hi)
-__device__ __forceinline__ uint16_t f16_part(float x, int part) {
-    const __half hi = __float2half_rn(x);
-    if (part == 0) return __half_as_ushort(hi);
-    return __half_as_ushort(__float2half_rn(x - __half2float(hi)));
-}
-
 // 4-token metadata chunk c of group g (the page format's XOR permutation)
 __device__ __forceinline__ int meta_chunk(int g, int c) { return c ^ (((c >> 3) & 3) ^ ((g & 1) << 2)); }
 
@@ -265,19 +212,18 @@ __device__ __forceinline__ Split split_of(int len, int S, int s) {
 
 // The page schedule of a unit without RoPE buckets.  The pages that hold the
 // coded tokens [lo, hi) are [P0, P1); pool index q is page P1 - 1 - q (the
-// last page first: it holds the new tokens of a fused step).  The unit's NP =
-// kPairs * S_pages pairs take the pool round-robin, pair P = kPairs s + pair
-// taking q = P in round 0.  With `skip` > 0 the first `appenders` pairs (the
-// fused step's appending cluster) sit out rounds 1..skip, which the other
-// pairs take in turn, so the work of appending makes no straggler.  The
-// schedule is a pure function of the shapes: every run assigns the same pages
-// to the same pairs in the same order, so results are reproducible bit for
-// bit.
+// last page first: it holds a step's new tokens).  The unit's NP = kPairs *
+// S_pages pairs take the pool round-robin, pair P = kPairs s + pair taking
+// q = P in round 0.  With `skip` > 0 the first `appenders` pairs (the fused
+// step's appending cluster) sit out rounds 1..skip, which the other pairs
+// take in turn, so the work of appending makes no straggler.  The schedule is
+// a pure function of the shapes: every run assigns the same pages to the
+// same pairs in the same order, so results are reproducible bit for bit.
 struct Pool {
     int P0, P1;
     int P, NP;                 // this pair's index and the pairs of the unit
     int appenders, skip;
-    bool tail_issued;          // the first page's tail is already in flight into stage 0
+    int pre;                   // the tails of this pair's first `pre` pages are already in flight
     __device__ int size() const { return P1 - P0; }
     __device__ int page(int q) const { return P1 - 1 - q; }
     // pool index of this pair's j-th page, -1 past the end
@@ -295,42 +241,30 @@ struct Pool {
         return q < size() ? q : -1;
     }
 };
-__device__ __forceinline__ Pool unit_pool(int lo, int hi, int s, int pair, int S_pages, int appenders, int skip,
-                                          bool tail_issued) {
+__device__ __forceinline__ Pool unit_pool(int lo, int hi, int s, int pair, int S_pages) {
     Pool p;
     p.P0 = lo / kT;
     p.P1 = hi > lo ? (hi + kT - 1) / kT : p.P0;
     p.P = kPairs * s + pair;
     p.NP = kPairs * S_pages;
-    p.appenders = min(appenders, p.NP);
-    p.skip = p.appenders < p.NP ? skip : 0;
-    p.tail_issued = tail_issued;
+    p.appenders = 0;
+    p.skip = 0;
+    p.pre = 0;
     return p;
 }
-// The page plan from the channel choice (sh.chan_pos, sh.q): score-MMA B
-// fragments, and the copy list of a page.  Called by every thread after a
-// barrier that follows the last write of chan_pos / q; ends with a barrier.
+// The page plan from the channel choice (sh.chan_pos, sh.q, and the
+// zero-point sums already in sh.plan.qg): score-MMA B fragments, channel 0's
+// q' and the copy list of a page.  Called by every thread after a barrier
+// that follows the last write of chan_pos / q; ends with a barrier.
 template <int NG>
 __device__ __forceinline__ void build_plan(MmaShared &sh, int tid, int warp, int lane) {
-    const int gid = lane >> 2, tig = lane & 3;
-    const int hh = gid >> 1, part = gid & 1;
-    // B fragments of k-step ks (channels 16ks..16ks+15): column gid = (head
-    // gid>>1, part gid&1); k-slots 2tig, 2tig+1, 2tig+8, 2tig+9 are channels
-    // +tig, +tig+4, +tig+8, +tig+12 (this order makes the code loads
-    // bank-conflict free).  Channel 0 and unselected channels get q' = 0.
-    {
-        const int ks = warp;
-        uint32_t w[2];
-#pragma unroll
-        for (int r = 0; r < 2; r++) {
-            const int c0 = 16 * ks + tig + 8 * r, c1 = c0 + 4;
-            const int p0 = sh.chan_pos[c0], p1 = sh.chan_pos[c1];
-            const float q0 = p0 >= 1 ? sh.q[hh][p0] : 0.f;
-            const float q1 = p1 >= 1 ? sh.q[hh][p1] : 0.f;
-            w[r] = (uint32_t)f16_part(q0, part) | ((uint32_t)f16_part(q1, part) << 16);
-        }
-        sh.bq[ks][lane] = make_uint2(w[0], w[1]);
-    }
+    // B fragments of k-step `warp`: channel 0 and unselected channels get q' = 0
+    auto qf = [&](int hh, int c) -> float {
+        const int p = sh.chan_pos[c];
+        return p >= 1 ? sh.q[hh][p] : 0.f;
+    };
+    sh.plan.bq[warp][lane] = make_uint2(plan_bq_word(warp, lane, 0, qf), plan_bq_word(warp, lane, 1, qf));
+    if (tid < 4) sh.plan.q0[tid] = sh.q[tid][0];
     // 64-byte chunks of key rows that hold a selected row
     if (tid < kChunks) {
         const bool t = sh.chan_pos[2 * tid] >= 1 || sh.chan_pos[2 * tid + 1] >= 1;
@@ -338,26 +272,7 @@ __device__ __forceinline__ void build_plan(MmaShared &sh, int tid, int warp, int
         if (lane == 0) sh.touched[warp] = m;
     }
     __syncthreads();
-    if (tid == 0) {
-        // runs of touched chunks, single untouched chunks between two touched
-        // ones filled in (one copy instead of two); then the page tail
-        const uint64_t T = (uint64_t)sh.touched[0] | ((uint64_t)sh.touched[1] << 32);
-        uint64_t M = T | ((T << 1) & (T >> 1));
-        int n = 0;
-        uint32_t bytes = 0;
-        while (M) {
-            const int st = __ffsll((long long)M) - 1;
-            const uint64_t inv = ~(M >> st);
-            const int len = inv ? __ffsll((long long)inv) - 1 : kChunks - st;
-            sh.copy[n++] = make_uint2(64u * (uint32_t)st, 64u * (uint32_t)len);
-            bytes += 64u * (uint32_t)len;
-            M = (len == kChunks) ? 0ull : (M & ~(((1ull << len) - 1ull) << st));
-        }
-        sh.copy[n++] = make_uint2((uint32_t)kKeyBytes, (uint32_t)fixed_bytes(2, NG));
-        sh.n_copies = n;
-        sh.tx_keys = bytes;
-    }
-    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    if (warp == 0) plan_copies_warp(sh.plan, (uint64_t)sh.touched[0] | ((uint64_t)sh.touched[1] << 32), NG, lane);
     __syncthreads();
 }
 
@@ -375,10 +290,10 @@ __device__ __forceinline__ void issue_tail(MmaShared &sh, int pair, int st, cons
 __device__ __forceinline__ void issue_keys(MmaShared &sh, int pair, int st, const uint8_t *src) {
     const uint32_t bar = smem_u32(&sh.mbar[pair][st]);
     const uint32_t dst = smem_u32(sh.stage[pair][st]);
-    mbar_arrive_expect_tx(bar, sh.tx_keys);
-    const int n = sh.n_copies - 1;
+    mbar_arrive_expect_tx(bar, sh.plan.tx_keys);
+    const int n = sh.plan.n_copies - 1;
     for (int r = 0; r < n; r++) {
-        const uint2 c = sh.copy[r];
+        const uint2 c = sh.plan.copy[r];
         bulk_g2s(dst + c.x, src + c.x, c.y, bar);
     }
 }
@@ -387,8 +302,8 @@ __device__ __forceinline__ void issue_keys(MmaShared &sh, int pair, int st, cons
 // or in the protected tier) are left out of the softmax.
 //  DYN (no RoPE buckets): this pair's pages of the unit's round-robin
 //    schedule `pool`, each staged while the one before it is computed.
-//    pool.tail_issued: the first page's tail is already in flight into
-//    stage 0.
+//    The tails of its first pool.pre (0..2) pages are already in flight
+//    into stages 0 and 1.
 //  static: pages [sp.blk0, sp.blk1), pair `pair` taking every kPairs-th.
 //    With RoPE buckets of w_pages pages the split runs as segments, one per
 //    bucket: before each, every warp is done with the previous one and
@@ -418,8 +333,8 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
     float q0_t = 0.f;
     uint32_t bz = 0;
     auto load_coef = [&]() {
-        q0_t = sh.q[tig][0] * kScoreScaleLog2;
-        bz = tig < NG ? (uint32_t)f16_part(sh.qg[hh][tig] * kScoreScaleLog2, part) : 0u;
+        q0_t = sh.plan.q0[tig] * kScoreScaleLog2;
+        bz = tig < NG ? (uint32_t)f16_part(sh.plan.qg[hh][tig] * kScoreScaleLog2, part) : 0u;
     };
     load_coef();
 
@@ -465,7 +380,7 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
                 const uint32_t Wd = *reinterpret_cast<const uint32_t *>(sb + 12 * 32);
                 const uint32_t Xab = __byte_perm(Wa, Wb, half_sel), Xcd = __byte_perm(Wc, Wd, half_sel);
                 const uint32_t Yab = Xab >> 8, Ycd = Xcd >> 8;
-                const uint2 bb = sh.bq[ks][lane];
+                const uint2 bb = sh.plan.bq[ks][lane];
 #pragma unroll
                 for (int i = 0; i < 4; i++) {
                     const uint32_t x1 = (i & 2) ? Yab : Xab;
@@ -663,15 +578,16 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
     };
 
     const bool issuer = (tid & 63) == 0;
-    int pend_st = -1;             // a stage still in flight after a give-up, and its parity
-    uint32_t pend_par = 0;
+    // after a give-up: the stage still in flight (bit 0) and its parity (bit
+    // 1), bit 2: stage 1's first phase too (a tail copied ahead); -1: none
+    int pend = -1;
     if constexpr (DYN) {
         // this pair's pages of the schedule, the next one staged while the
         // current one is computed; the same sequence on both warps
         int q_cur = pool.index(0);
         if (issuer && q_cur >= 0) {
             const uint8_t *src = unit_pages + (size_t)pool.page(q_cur) * page_bytes(2, NG);
-            if (!pool.tail_issued) issue_tail<NG>(sh, pair, 0, src);
+            if (pool.pre < 1) issue_tail<NG>(sh, pair, 0, src);
             issue_keys(sh, pair, 0, src);
         }
         for (int it = 0; q_cur >= 0; it++) {
@@ -680,14 +596,19 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
             bool ok = mbar_wait_bounded(smem_u32(&sh.mbar[pair][st]), par, status, polls);
             ok = pair_sync_and(pair, ok);                        // both warps left the other stage
             if (!ok) {
-                pend_st = st;
-                pend_par = par;
+                pend = st | (int)(par << 1);
+                if (it == 0 && pool.pre >= 2) {
+                    // the second page's tail is in flight without its key
+                    // copies: complete that phase's arrival so it can drain
+                    if (issuer) mbar_arrive(smem_u32(&sh.mbar[pair][1]));
+                    pend |= 4;
+                }
                 break;
             }
             const int q_next = pool.index(it + 1);
             if (issuer && q_next >= 0) {
                 const uint8_t *src = unit_pages + (size_t)pool.page(q_next) * page_bytes(2, NG);
-                issue_tail<NG>(sh, pair, st ^ 1, src);
+                if (it + 1 >= pool.pre) issue_tail<NG>(sh, pair, st ^ 1, src);
                 issue_keys(sh, pair, st ^ 1, src);
             }
             page(sh.stage[pair][st], pool.page(q_cur));
@@ -716,8 +637,7 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
                 ok = pair_sync_and(pair, ok);                    // both warps left the other stage
                 if (!ok) {
                     dead = true;
-                    pend_st = st;
-                    pend_par = par;
+                    pend = st | (int)(par << 1);
                     break;
                 }
                 if (issuer && pg + kPairs < seg1) {
@@ -732,7 +652,10 @@ __device__ __forceinline__ void run_pages(MmaShared &sh, const uint8_t *__restri
     }
     // a stage whose wait gave up may still receive bytes: wait (bounded)
     // until they have landed before the staging memory is reused below
-    if (pend_st >= 0) drain_stage(smem_u32(&sh.mbar[pair][pend_st]), pend_par);
+    if (pend >= 0) {
+        drain_stage(smem_u32(&sh.mbar[pair][pend & 1]), (uint32_t)(pend >> 1) & 1u);
+        if (pend & 4) drain_stage(smem_u32(&sh.mbar[pair][1]), 0u);
+    }
 
     // ------------------------------------------------------------ merge
     // per warp: head tig's max, sum and output; then across the 8 warps
@@ -819,15 +742,18 @@ __device__ __forceinline__ void tier_cta(MmaShared &sh, const uint8_t *slots, in
 // array) each split reads a contiguous range of pages and, per bucket its
 // pages fall in, that bucket's channel choice; the tier CTAs read each
 // protected position's own bucket's.  Without buckets the pages come from the
-// unit's round-robin schedule, and each pair's first tail is in flight, and
-// its next tails on their way to L2, while the channel choice is loaded.
+// unit's round-robin schedule, and the tails of each pair's first two pages
+// are in flight, and their key rows on their way to L2, while the channel
+// choice is loaded.
 //
 // STEP: the second launch of a decode step, a programmatic dependent of the
-// preparation kernel (the channel choice and the append of the step's n_new
-// tokens, kvq_select.cu).  Until griddepcontrol.wait it reads only what that
-// kernel does not write -- the length before the step and the tails of pages
-// that hold no new token -- and it advances the length after the wait, once
-// every CTA of the sequence has read it.
+// preparation kernel (the channel choices, page plans and the append of the
+// step's n_new tokens, kvq_select.cu).  Until griddepcontrol.wait it reads
+// only what that kernel does not write -- the length before the step and the
+// tails of pages that hold no new token -- and it advances the length after
+// the wait, once every CTA of the sequence has read it.  Its page plans come
+// from `plans` ([unit][bucket]); the three-call decode builds them from the
+// channel lists.
 template <int NG, bool BK, bool STEP>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_mma_kernel(const uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, int Hkv,
@@ -836,7 +762,7 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, int32_t *__restrict__ seq_l
                   float2 *__restrict__ part_ml, int S, float *__restrict__ out,
                   uint32_t *__restrict__ counters, uint32_t *__restrict__ status,
                   int n_sink, int n_recent, const double *__restrict__ v_rot, int nbk, int w_pages,
-                  uint32_t polls, int n_new) {
+                  uint32_t polls, int n_new, const PagePlan *__restrict__ plans) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     MmaShared &sh = *reinterpret_cast<MmaShared *>(smem_raw);
 
@@ -854,7 +780,8 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, int32_t *__restrict__ seq_l
             const int hl = e / k, i = e % k;
             sh.q[hl][i] = qsel[((qrow0 + hl) * nbk + bk) * k + i];
         }
-        if (tid < 4 * kNG) sh.qg[tid / kNG][tid % kNG] = qgsum[((qrow0 + tid / kNG) * nbk + bk) * kNG + tid % kNG];
+        if (tid < 4 * kNG)
+            sh.plan.qg[tid / kNG][tid % kNG] = qgsum[((qrow0 + tid / kNG) * nbk + bk) * kNG + tid % kNG];
         if (tid < kD) sh.chan_pos[tid] = -1;
         const int32_t *sel = idx + (unit * nbk + bk) * k;
         int my_c = -1;
@@ -869,13 +796,22 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, int32_t *__restrict__ seq_l
         __syncthreads();
         build_plan<NG>(sh, tid, warp, lane);
     };
+    // the preparation kernel's plan of bucket bk (after the wait)
+    auto load_plan = [&](int bk) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(plans + unit * nbk + bk);
+        uint4 *dst = reinterpret_cast<uint4 *>(&sh.plan);
+        for (int e = tid; e < (int)(sizeof(PagePlan) / 16); e += kThreads) dst[e] = __ldcg(src + e);
+        __syncthreads();
+    };
 
     if (tid < 2 * kPairs) mbar_init(smem_u32(&sh.mbar[tid >> 1][tid & 1]), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     // the length (with the step's new tokens once they are in; a step that
     // would overflow the capacity appends nothing)
     const int L0 = seq_len[b];
     const bool fits = L0 >= 0 && L0 + n_new <= NB * kT;
     const int len = min(max(STEP && fits ? L0 + n_new : L0, 0), NB * kT);
+    __syncthreads();                              // barriers initialised before copies complete on them
     // after the preparation kernel: wait for it, make its page writes visible
     // to the bulk copies, and advance the length once every CTA of sequence b
     // has read it (its completion counter reaches S * Hkv)
@@ -912,24 +848,36 @@ decode_mma_kernel(const uint8_t *__restrict__ pages, int32_t *__restrict__ seq_l
     const uint8_t *unit_pages = pages + unit * NB * (size_t)page_bytes(2, NG);
     if constexpr (BK) {
         after_prep();
-        run_pages<NG, false>(sh, unit_pages, tr.sink_end, tr.recent_start, split_of(tr.recent_start, S_pages, s),
-                             Pool{}, S, s, qrow0, part_o, part_ml, out, counters + unit, status, polls, rot,
-                             w_pages, load_sel);
+        if constexpr (STEP)
+            run_pages<NG, false>(sh, unit_pages, tr.sink_end, tr.recent_start,
+                                 split_of(tr.recent_start, S_pages, s), Pool{}, S, s, qrow0, part_o, part_ml, out,
+                                 counters + unit, status, polls, rot, w_pages, load_plan);
+        else
+            run_pages<NG, false>(sh, unit_pages, tr.sink_end, tr.recent_start,
+                                 split_of(tr.recent_start, S_pages, s), Pool{}, S, s, qrow0, part_o, part_ml, out,
+                                 counters + unit, status, polls, rot, w_pages, load_sel);
     } else {
-        // a first page that may hold a new token is staged only after the wait
-        const Pool pool0 = unit_pool(tr.sink_end, tr.recent_start, s, warp >> 1, S_pages, 0, 0, false);
-        const bool early = pool0.index(0) >= 0 && !(STEP && pool0.page(pool0.index(0)) >= L0 / kT);
-        Pool pool = pool0;
-        pool.tail_issued = early;
-        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-        __syncthreads();                              // barriers initialised before copies complete on them
-        if ((tid & 63) == 0 && early) {
-            const uint8_t *first = unit_pages + (size_t)pool.page(pool.index(0)) * page_bytes(2, NG);
-            issue_tail<NG>(sh, warp >> 1, 0, first);
-            prefetch_l2(first, kKeyBytes);      // the key rows: in L2 once the choice is loaded
+        // the tails of the pair's first two pages (while they hold no new
+        // token) are copied, and their key rows brought into L2, before the
+        // channel choice is in place
+        Pool pool = unit_pool(tr.sink_end, tr.recent_start, s, warp >> 1, S_pages);
+        for (int j = 0; j < 2; j++) {
+            const int qj = pool.index(j);
+            if (qj < 0 || (STEP && pool.page(qj) >= L0 / kT)) break;
+            pool.pre = j + 1;
+        }
+        if ((tid & 63) == 0) {
+            for (int j = 0; j < pool.pre; j++) {
+                const uint8_t *pg = unit_pages + (size_t)pool.page(pool.index(j)) * page_bytes(2, NG);
+                issue_tail<NG>(sh, warp >> 1, j, pg);
+                prefetch_l2(pg, kKeyBytes);
+            }
         }
         after_prep();
-        load_sel(0);
+        if constexpr (STEP)
+            load_plan(0);
+        else
+            load_sel(0);
         run_pages<NG, true>(sh, unit_pages, tr.sink_end, tr.recent_start, Split{0, 0}, pool, S, s, qrow0, part_o,
                             part_ml, out, counters + unit, status, polls, rot, 0, [](int) {});
     }
@@ -1042,8 +990,10 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
     const bool ok = L0 >= 0 && L0 + n_new <= capacity;
     const int len = min(max(ok ? L0 + n_new : L0, 0), capacity);
     const Tier tr = tier_of(len, n_sink, n_recent);
-    const Pool pool = unit_pool(tr.sink_end, tr.recent_start, s, warp >> 1, S_pages, kPairs * kCluster,
-                                kAppendRounds, !may_append);
+    Pool pool = unit_pool(tr.sink_end, tr.recent_start, s, warp >> 1, S_pages);
+    pool.appenders = min(kPairs * kCluster, pool.NP);
+    pool.skip = pool.appenders < pool.NP ? kAppendRounds : 0;
+    pool.pre = may_append ? 0 : 1;
     // the first page's tail (no new token in it) is copied while the channels
     // are chosen
     if (!is_tier && !may_append && (tid & 63) == 0 && pool.index(0) >= 0) {
@@ -1243,19 +1193,9 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
     // ---- channel choice (the arithmetic of kvq_select_channels)
     {
         // rank of channel j among 1..127 by (energy descending, index
-        // ascending), in two halves; energies are >= 0, so their bit
-        // patterns order like their values (integer compares keep the
-        // float64 pipe free)
+        // ascending), in two halves
         const int j = tid & (kD - 1), part = tid >> 7;
-        const unsigned long long e = __double_as_longlong(e2[j]);
-        int rk = 0;
-        const int i0 = part == 0 ? 1 : 64, i1 = part == 0 ? 64 : kD;
-#pragma unroll 8
-        for (int i = i0; i < i1; i++) {
-            const unsigned long long ei = __double_as_longlong(e2[i]);
-            rk += (ei > e) || (ei == e && i < j);
-        }
-        rank_part[part][j] = rk;
+        rank_part[part][j] = rank_half(reinterpret_cast<const unsigned long long *>(e2), j, part);
     }
     __syncthreads();
     if (tid < kD) {
@@ -1286,6 +1226,7 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
             for (int hl = 0; hl < 4; hl++) {
                 const float qf = (float)my_q[hl];
                 sh.q[hl][pos] = qf;
+                if (tid == 0) sh.plan.q0[hl] = qf;      // channel 0 is position 0
                 if (s == 0) qsel[(qrow0 + hl) * k + pos] = qf;
             }
             if (s == 0) idx[unit * k + pos] = tid;
@@ -1302,51 +1243,17 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
             for (int c = (gr == 0 ? 1 : gr * GS); c < (gr + 1) * GS; c++)
                 sm = fma(selected(c) ? 1.0 : 0.0, qp[hl][c], sm);
         const float gf = (float)sm;
-        sh.qg[hl][gr] = gf;
+        sh.plan.qg[hl][gr] = gf;
         if (s == 0) qgsum[(qrow0 + hl) * kNG + gr] = gf;
-    } else if (warp == 5 && lane == 0) {
-        // 64-byte chunks of key rows that hold a selected row (channel 0's
-        // row is unused), as runs; single unselected chunks between two
-        // selected ones filled in (one copy instead of two); then the tail
-        uint64_t T = 0;
-#pragma unroll
-        for (int w = 0; w < 4; w++) {
-            uint32_t x = w == 0 ? (msk[0] & ~1u) : msk[w];
-            x = (x | (x >> 1)) & 0x55555555u;       // chunk bit at each even position
-            x = (x | (x >> 1)) & 0x33333333u;       // then compressed to 16 bits
-            x = (x | (x >> 2)) & 0x0f0f0f0fu;
-            x = (x | (x >> 4)) & 0x00ff00ffu;
-            x = (x | (x >> 8)) & 0x0000ffffu;
-            T |= (uint64_t)x << (16 * w);
-        }
-        uint64_t Mr = T | ((T << 1) & (T >> 1));
-        int n = 0;
-        uint32_t bytes = 0;
-        while (Mr) {
-            const int st = __ffsll((long long)Mr) - 1;
-            const uint64_t inv = ~(Mr >> st);
-            const int len = inv ? __ffsll((long long)inv) - 1 : kChunks - st;
-            sh.copy[n++] = make_uint2(64u * (uint32_t)st, 64u * (uint32_t)len);
-            bytes += 64u * (uint32_t)len;
-            Mr = (len == kChunks) ? 0ull : (Mr & ~(((1ull << len) - 1ull) << st));
-        }
-        sh.copy[n++] = make_uint2((uint32_t)kKeyBytes, (uint32_t)fixed_bytes(2, NG));
-        sh.n_copies = n;
-        sh.tx_keys = bytes;
+    } else if (warp == 5) {
+        // the copy list of a page
+        plan_copies_warp(sh.plan, plan_chunks(msk), NG, lane);
     }
     {
-        // score-MMA B fragments of k-step `warp` (the layout build_plan
-        // writes): channel 0 and unselected channels get q' = 0
-        const int gid = lane >> 2, tig = lane & 3, hh = gid >> 1, part = gid & 1;
-        uint32_t w2[2];
-#pragma unroll
-        for (int r2 = 0; r2 < 2; r2++) {
-            const int c0 = 16 * warp + tig + 8 * r2, c1 = c0 + 4;
-            const float q0 = (c0 >= 1 && selected(c0)) ? (float)qp[hh][c0] : 0.f;
-            const float q1 = (c1 >= 1 && selected(c1)) ? (float)qp[hh][c1] : 0.f;
-            w2[r2] = (uint32_t)f16_part(q0, part) | ((uint32_t)f16_part(q1, part) << 16);
-        }
-        sh.bq[warp][lane] = make_uint2(w2[0], w2[1]);
+        // score-MMA B fragments of k-step `warp`: channel 0 and unselected
+        // channels get q' = 0
+        auto qf = [&](int hh, int c) -> float { return (c >= 1 && selected(c)) ? (float)qp[hh][c] : 0.f; };
+        sh.plan.bq[warp][lane] = make_uint2(plan_bq_word(warp, lane, 0, qf), plan_bq_word(warp, lane, 1, qf));
     }
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     __syncthreads();
@@ -1364,25 +1271,21 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
 }  // namespace
 
 // Splits per (sequence, KV head): about two CTAs per SM in all (counting the
-// `tier` CTAs that handle the protected tier), the page splits a multiple of
-// the fused step's cluster size (at least one cluster), at most one page
-// split per kPairs pages unless that is below one cluster.  Returns page
-// splits + tier.
+// `tier` CTAs that handle the protected tier), at most one page split per
+// kPairs pages, at least one.  Returns page splits + tier.
 int decode_mma_splits(int units, int nblk, int num_sms, int tier) {
     int S = (2 * num_sms) / units - tier;
     const int max_s = nblk / kPairs;
     if (S > max_s) S = max_s;
-    S -= S % kCluster;
-    return (S < kCluster ? kCluster : S) + tier;
+    return (S < 1 ? 1 : S) + tier;
 }
-int step_mma_max_new() { return kStepMaxNew; }
 
 uint32_t default_wait_polls() { return kWaitPolls; }
 
 template <int NG, bool BK, bool STEP>
 cudaError_t launch_decode_mma_t(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
                                 const float *qgsum, int k, float *part_o, float2 *part_ml, int S,
-                                float *out, uint32_t polls, int n_new, cudaStream_t st) {
+                                float *out, uint32_t polls, int n_new, const PagePlan *plans, cudaStream_t st) {
     const size_t smem = sizeof(MmaShared);
     static std::atomic<uint64_t> done{0};
     cudaError_t e = set_smem_once(decode_mma_kernel<NG, BK, STEP>, (int)smem, done);
@@ -1401,22 +1304,39 @@ cudaError_t launch_decode_mma_t(const kvq_cache &c, int Hq, const int32_t *idx, 
     return cudaLaunchKernelEx(&cfg, decode_mma_kernel<NG, BK, STEP>, static_cast<const uint8_t *>(c.pages),
                               c.seq_len, (int)c.n_kv_heads, c.capacity / kT, Hq, idx, qsel, qgsum, k, part_o,
                               part_ml, S, out, unit_counter(c, 0, 0), c.status, (int)c.n_sink, (int)c.n_recent,
-                              c.v_rot, buckets_of(c), c.bucket / kT, polls, n_new);
+                              c.v_rot, buckets_of(c), c.bucket / kT, polls, n_new, plans);
+}
+
+template <bool STEP>
+cudaError_t launch_decode_mma_any(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
+                                  const float *qgsum, int k, float *part_o, float2 *part_ml, int S, float *out,
+                                  uint32_t polls, int n_new, const PagePlan *plans, cudaStream_t st) {
+    const bool one = groups_of(c) == 1, bk = c.bucket > 0;
+    if (bk)
+        return one ? launch_decode_mma_t<1, true, STEP>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, polls,
+                                                        n_new, plans, st)
+                   : launch_decode_mma_t<kNG, true, STEP>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out,
+                                                          polls, n_new, plans, st);
+    return one ? launch_decode_mma_t<1, false, STEP>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, polls,
+                                                     n_new, plans, st)
+               : launch_decode_mma_t<kNG, false, STEP>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, polls,
+                                                       n_new, plans, st);
 }
 
 cudaError_t launch_decode_mma(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
                               const float *qgsum, int k, float *part_o, float2 *part_ml, int S,
                               float *out, uint32_t polls, cudaStream_t st) {
-    const bool one = groups_of(c) == 1, bk = c.bucket > 0;
-    if (bk)
-        return one ? launch_decode_mma_t<1, true, false>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, polls,
-                                                         0, st)
-                   : launch_decode_mma_t<kNG, true, false>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out,
-                                                           polls, 0, st);
-    return one ? launch_decode_mma_t<1, false, false>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, polls,
-                                                      0, st)
-               : launch_decode_mma_t<kNG, false, false>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, polls,
-                                                        0, st);
+    return launch_decode_mma_any<false>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, polls, 0, nullptr, st);
+}
+
+// The decode of a step whose preparation kernel (the channel choices, the
+// page plans `plans` and the append of n_new tokens) was launched just before
+// it on `st`.
+cudaError_t launch_decode_mma_step(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
+                                   const float *qgsum, int k, float *part_o, float2 *part_ml, int S,
+                                   float *out, int n_new, const PagePlan *plans, cudaStream_t st) {
+    return launch_decode_mma_any<true>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, kWaitPolls, n_new,
+                                       plans, st);
 }
 
 template <typename Tin, int NG>
@@ -1453,18 +1373,8 @@ cudaError_t launch_step_mma(const kvq_cache &c, int Hq, const void *q, const voi
                                                   qgsum, part_o, part_ml, S, out, st);
 }
 
-// The decode of a step with RoPE buckets whose preparation kernel (the
-// per-bucket channel choice + the append of n_new tokens) was launched just
-// before it on `st`.
-cudaError_t launch_decode_mma_step(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
-                                   const float *qgsum, int k, float *part_o, float2 *part_ml, int S,
-                                   float *out, int n_new, cudaStream_t st) {
-    return groups_of(c) == 1
-               ? launch_decode_mma_t<1, true, true>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, kWaitPolls,
-                                                    n_new, st)
-               : launch_decode_mma_t<kNG, true, true>(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out,
-                                                      kWaitPolls, n_new, st);
-}
+int step_mma_max_new() { return kStepMaxNew; }
+int step_mma_cluster() { return kCluster; }
 
 size_t decode_mma_smem_bytes() { return sizeof(MmaShared); }
 

@@ -87,6 +87,108 @@ inline int tier_ctas(const kvq_cache &c) { return c.n_sink + c.n_recent > 0 ? 2 
 // log2(e) / sqrt(128): scores are kept in the base-2 exponent domain
 constexpr float kScoreScaleLog2 = 0.12751743074460787f;
 
+// ------------------------------------------------------------ channel choice
+// How many of channels 64*half .. 64*half + 63 (channel 0 left out) come
+// before channel j in the order (energy descending, index ascending).
+// `key` holds the 128 energies' bit patterns: energies are >= 0, so the
+// patterns order like the values and integer compares decide exactly.  The
+// keys are read eight at a time, ahead of their compares.
+__device__ __forceinline__ int rank_half(const unsigned long long *key, int j, int half) {
+    const unsigned long long kj = key[j];
+    int rk = 0;
+#pragma unroll
+    for (int b = 0; b < 8; b++) {
+        unsigned long long v[8];
+#pragma unroll
+        for (int u = 0; u < 8; u++) v[u] = key[64 * half + 8 * b + u];
+#pragma unroll
+        for (int u = 0; u < 8; u++) {
+            const int i = 64 * half + 8 * b + u;
+            rk += (int)((i != 0) & ((v[u] > kj) | ((v[u] == kj) & (i < j))));
+        }
+    }
+    return rk;
+}
+
+// ------------------------------------------------------------ page plan
+// What the tensor-core decode (INT2, four query heads per KV head) needs of
+// one channel choice, in the order its shared memory holds it.  A decode
+// step's preparation kernel writes one per (sequence, KV head, RoPE bucket)
+// into the workspace; the decode copies it in after waiting for that kernel.
+// The three-call decode builds the same plan from the channel list.
+constexpr int kPlanChunks = 64;                   // 64-byte chunks of a page's key rows
+constexpr int kPlanCopies = kPlanChunks / 2 + 2;  // runs after gap filling, plus the tail
+struct __align__(16) PagePlan {
+    uint2 bq[8][32];          // score-MMA B fragments per k-step and lane
+    float q0[4];              // channel 0's q' per head (fp32, as in qsel)
+    float qg[4][kNG];         // zero-point sums per head and key group (as in qgsum)
+    uint2 copy[kPlanCopies];  // {byte offset in the page, bytes}; the last one is the page tail
+    uint32_t tx_keys;         // bytes of the key-chunk copies of one page
+    int n_copies;
+    uint32_t pad[2];
+};
+static_assert(sizeof(PagePlan) % 16 == 0, "plans are copied in 16-byte pieces");
+
+// fp16 hi/lo split of a float: hi = fp16(x), lo = fp16(x - hi)
+__device__ __forceinline__ uint16_t f16_part(float x, int part) {
+    const __half hi = __float2half_rn(x);
+    if (part == 0) return __half_as_ushort(hi);
+    return __half_as_ushort(__float2half_rn(x - __half2float(hi)));
+}
+// B fragment word of k-step ks, lane, register half rr of the score MMAs:
+// column gid = lane / 4 is (head gid / 2, fp16 part gid % 2); k-slots 2tig,
+// 2tig+1 (rr = 0) and 2tig+8, 2tig+9 (rr = 1) are channels 16ks + tig + 8rr
+// and that + 4 (this order makes the code loads bank-conflict free).
+// `qf(c)` is the fp32 q' of channel c for the column's head, 0 for channel 0
+// and for channels that are not selected.
+template <typename QF>
+__device__ __forceinline__ uint32_t plan_bq_word(int ks, int lane, int rr, QF &&qf) {
+    const int gid = lane >> 2, tig = lane & 3, part = gid & 1;
+    const int c0 = 16 * ks + tig + 8 * rr, c1 = c0 + 4;
+    return (uint32_t)f16_part(qf(gid >> 1, c0), part) | ((uint32_t)f16_part(qf(gid >> 1, c1), part) << 16);
+}
+// The copy list of a plan from T, the 64-byte chunks of key rows that hold a
+// selected row (channel 0's row is never read): runs of chunks in ascending
+// order, single unselected chunks between two selected ones filled in (one
+// copy instead of two); then the page tail (value codes, channel 0,
+// metadata).  Called by a whole warp: lane l looks at chunks 2l and 2l + 1
+// as run starts.
+__device__ __forceinline__ void plan_copies_warp(PagePlan &p, uint64_t T, int ng, int lane) {
+    const uint64_t M = T | ((T << 1) & (T >> 1));
+    const uint64_t starts = M & ~(M << 1);
+#pragma unroll
+    for (int h = 0; h < 2; h++) {
+        const int st = 2 * lane + h;
+        if ((starts >> st) & 1ull) {
+            const int n = __popcll(starts & ((1ull << st) - 1ull));
+            const uint64_t inv = ~(M >> st);
+            const int len = inv ? __ffsll((long long)inv) - 1 : kPlanChunks - st;
+            p.copy[n] = make_uint2(64u * (uint32_t)st, 64u * (uint32_t)len);
+        }
+    }
+    if (lane == 0) {
+        const int n = __popcll(starts);
+        p.copy[n] = make_uint2((uint32_t)off_vcodes(2), (uint32_t)fixed_bytes(2, ng));
+        p.n_copies = n + 1;
+        p.tx_keys = 64u * (uint32_t)__popcll(M);
+    }
+}
+// chunk mask from the 128-bit channel choice (word w = channels 32w..32w+31)
+__device__ __forceinline__ uint64_t plan_chunks(const uint32_t (&msk)[4]) {
+    uint64_t T = 0;
+#pragma unroll
+    for (int w = 0; w < 4; w++) {
+        uint32_t x = w == 0 ? (msk[0] & ~1u) : msk[w];
+        x = (x | (x >> 1)) & 0x55555555u;       // chunk bit at each even position
+        x = (x | (x >> 1)) & 0x33333333u;       // then compressed to 16 bits
+        x = (x | (x >> 2)) & 0x0f0f0f0fu;
+        x = (x | (x >> 4)) & 0x00ff00ffu;
+        x = (x | (x >> 8)) & 0x0000ffffu;
+        T |= (uint64_t)x << (16 * w);
+    }
+    return T;
+}
+
 // ------------------------------------------------------------ conversions
 __device__ __forceinline__ double in_to_double(float x) { return (double)x; }
 __device__ __forceinline__ double in_to_double(uint16_t bf) {
@@ -171,6 +273,59 @@ __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src)
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+
+// ------------------------------------------------------------ bulk copies, mbarriers
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+// expect bytes without arriving (the arrival comes with the key copies)
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+// bring `bytes` (a multiple of 16, 16-byte aligned) of global memory into L2
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(src), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+// Wait for a phase of a barrier with bulk copies on it.  The wait is bounded: after `polls` polls the
+// device status word gets KVQ_DEV_TIMEOUT and the caller is told; it then
+// issues no further copy, drains what it issued (drain_stage) and reports
+// that call's output invalid.  polls = 0 gives up at once unless the stage
+// has already landed (the path a test takes to exercise the give-up).
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint32_t *status,
+                                                  uint32_t polls) {
+    if (mbar_test_wait(bar, parity)) return true;
+    for (uint32_t i = 0; i < polls; i++)
+        if (mbar_try_wait(bar, parity)) return true;
+    atomicOr(status, (uint32_t)KVQ_DEV_TIMEOUT);
+    return false;
+}
 
 // ------------------------------------------------------------ launch set-up
 // Raise a kernel's dynamic shared memory limit to `bytes` once per device and
@@ -498,7 +653,7 @@ cudaError_t launch_append(const kvq_cache &c, const void *K, const void *V, int 
 cudaError_t launch_select(const kvq_cache &c, const void *q, int dtype, int Hq, const double *Ainvt,
                           const double *delta, int k, int32_t *idx, float *qsel, float *qgsum, cudaStream_t st);
 int decode_splits(const kvq_cache &c, int Hq, int k, int num_sms);
-size_t decode_ws_bytes(const kvq_cache &c, int Hq, int n_splits);
+size_t decode_ws_bytes(const kvq_cache &c, int Hq, int n_splits, bool step = false);
 cudaError_t launch_decode(const kvq_cache &c, int Hq, const int32_t *idx, const float *qsel,
                           const float *qgsum, int k, float *out, void *ws, int n_splits,
                           cudaStream_t st, long long polls = -1);
