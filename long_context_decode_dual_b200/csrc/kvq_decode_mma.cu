@@ -955,16 +955,20 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
     for (int i = 0; i < 2; i++) qv[i] = in_to_double(q[qrow0 * kD + tid + i * kThreads]);
     const double *Ai_blk = Ainvt + (size_t)h * kD * kD + r * kCols;
     const double *A_blk = A + (size_t)h * kD * kD + r * kCols;
-    for (int e = tid; e < kD * (kBlkRowBytes / 16); e += kThreads) {
-        const int c = e >> 5, part = e & 31, rr = c & 31;
-        double *row = reinterpret_cast<double *>(ai_base(c >> 5, rr >= 8) +
-                                                 (rr < 8 ? rr : rr - 8) * kBlkRowBytes);
-        cp_async16(row + 2 * part, Ai_blk + (size_t)c * kD + 2 * part);
+    // one commit group per 32 rows, so the chains start on the first rows
+#pragma unroll 1
+    for (int p = 0; p < 4; p++) {
+        for (int e = tid; e < 32 * (kBlkRowBytes / 16); e += kThreads) {
+            const int rr = e >> 5, part = e & 31, c = 32 * p + rr;
+            double *row = reinterpret_cast<double *>(ai_base(p, rr >= 8) + (rr < 8 ? rr : rr - 8) * kBlkRowBytes);
+            cp_async16(row + 2 * part, Ai_blk + (size_t)c * kD + 2 * part);
+        }
+        cp_async_commit();
     }
     const int nload = may_append ? min(n_new, kStepMaxNew) : 0;   // new rows this CTA may need
     float vpre[kVPre];
     if (nload > 0) {
-        stage_block(a_lo, A_blk, 0, 64);
+        stage_block(a_lo, A_blk, 0, 64);            // a fifth commit group
         const size_t in0 = unit * (size_t)n_new;
         for (int e = tid; e < nload * kD; e += kThreads) ks_f[e] = in_to_float(k_new[in0 * kD + e]);
 #pragma unroll
@@ -1025,32 +1029,46 @@ step_mma_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len, uint
             atomicExch(status + 1 + b, 0u);
         }
     }
-    cp_async_wait<0>();
-    __syncthreads();
-
     // q'[hl][64r + jj] = sum_c q[hl][c] Ainvt[c][64r + jj], fma chain c =
     // 0..127 from 0.0, the four heads' chains side by side in thread jj (each
-    // A^{-T} element loaded once); then the pooled energy of channel 64r + jj,
-    // with a diagonal refinement of the base queries q'_{h,j} / delta_j (the
-    // arithmetic of kvq_select_channels)
-    if (tid < kCols) {
-        double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    // A^{-T} element loaded once), each 32-row group as soon as it has landed,
+    // the operands loaded four steps ahead; then the pooled energy of channel
+    // 64r + jj, with a diagonal refinement of the base queries q'_{h,j} /
+    // delta_j (the arithmetic of kvq_select_channels)
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll 1
-        for (int p = 0; p < 4; p++) {
+    for (int p = 0; p < 4; p++) {
+        cp_async_wait_upto(3 - p + (nload > 0 ? 1 : 0));
+        __syncthreads();
+        if (tid < kCols) {
             const double *lo8 = reinterpret_cast<const double *>(ai_base(p, 0));
             const double *hi24 = reinterpret_cast<const double *>(ai_base(p, 1));
+            auto arow = [&](int rr) { return rr < 8 ? lo8[rr * kCols + tid] : hi24[(rr - 8) * kCols + tid]; };
+            double a[4];
+            double2 qa[4], qb[4];
+#pragma unroll
+            for (int u = 0; u < 4; u++) {
+                a[u] = arow(u);
+                qa[u] = *reinterpret_cast<const double2 *>(&px.qin[32 * p + u][0]);
+                qb[u] = *reinterpret_cast<const double2 *>(&px.qin[32 * p + u][2]);
+            }
 #pragma unroll
             for (int rr = 0; rr < 32; rr++) {
-                const int c = 32 * p + rr;
-                const double a = rr < 8 ? lo8[rr * kCols + tid] : hi24[(rr - 8) * kCols + tid];
-                const double2 q01 = *reinterpret_cast<const double2 *>(&px.qin[c][0]);
-                const double2 q23 = *reinterpret_cast<const double2 *>(&px.qin[c][2]);
-                acc[0] = fma(q01.x, a, acc[0]);
-                acc[1] = fma(q01.y, a, acc[1]);
-                acc[2] = fma(q23.x, a, acc[2]);
-                acc[3] = fma(q23.y, a, acc[3]);
+                const int u = rr & 3;
+                acc[0] = fma(qa[u].x, a[u], acc[0]);
+                acc[1] = fma(qa[u].y, a[u], acc[1]);
+                acc[2] = fma(qb[u].x, a[u], acc[2]);
+                acc[3] = fma(qb[u].y, a[u], acc[3]);
+                if (rr + 4 < 32) {
+                    a[u] = arow(rr + 4);
+                    qa[u] = *reinterpret_cast<const double2 *>(&px.qin[32 * p + rr + 4][0]);
+                    qb[u] = *reinterpret_cast<const double2 *>(&px.qin[32 * p + rr + 4][2]);
+                }
             }
         }
+    }
+    if (nload > 0) cp_async_wait<0>();              // A's low rows (read after the barrier below)
+    if (tid < kCols) {
         const double dj = delta ? delta[(size_t)h * kD + r * kCols + tid] : 1.0;
         double e = 0.0;
 #pragma unroll

@@ -273,6 +273,14 @@ __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src)
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+// wait until at most `pending` (0..4) of this thread's commit groups are in flight
+__device__ __forceinline__ void cp_async_wait_upto(int pending) {
+    if (pending >= 4) cp_async_wait<4>();
+    else if (pending == 3) cp_async_wait<3>();
+    else if (pending == 2) cp_async_wait<2>();
+    else if (pending == 1) cp_async_wait<1>();
+    else cp_async_wait<0>();
+}
 
 // ------------------------------------------------------------ bulk copies, mbarriers
 __device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
