@@ -238,9 +238,12 @@ append_small_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len,
                     uint32_t *__restrict__ status, const Tin *__restrict__ K,
                     const Tin *__restrict__ V, const double *__restrict__ A, const double *__restrict__ Rv,
                     double vclip, int Hkv, int NB, int n_new, int capacity, int n_sink, int n_recent,
-                    const double *__restrict__ rope, int w_tok) {
+                    const double *__restrict__ rope, int w_tok, int advance) {
     constexpr int R = row_bytes(BITS);
     constexpr int PER = 8 / BITS;
+    // a decode step's channel choice may start meanwhile (it reads nothing
+    // this kernel writes, and waits for it before it exits)
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
     static_assert(kSmallMax * 32 == 128, "one warp per new token");
     __shared__ __align__(16) double As[kD][kGroup];        // A[:, 32 grp .. 32 grp + 31], then Rv[...]
     __shared__ double ks[kSmallMax][kD];
@@ -380,7 +383,7 @@ append_small_kernel(uint8_t *__restrict__ pages, int32_t *__restrict__ seq_len,
     }
 
     __syncthreads();
-    if (t == 0) {
+    if (advance && t == 0) {
         __threadfence();
         const unsigned prev = atomicAdd(status + 1 + b, 1u);
         if (prev == (unsigned)(Hkv * kNG) - 1u) {   // every CTA of sequence b has read its length
@@ -400,7 +403,7 @@ __global__ void advance_kernel(int32_t *seq_len, int B, int n_new, int capacity)
 
 template <typename Tin, int BITS, int NG>
 cudaError_t launch_append_t(const kvq_cache &c, const void *K, const void *V, int n_new,
-                            const double *A, cudaStream_t st) {
+                            const double *A, cudaStream_t st, bool advance = true) {
     const double *Rv = c.v_rot;
     const double vclip = value_clip(c);
     const double *rope = c.bucket > 0 ? c.rope : nullptr;
@@ -412,7 +415,7 @@ cudaError_t launch_append_t(const kvq_cache &c, const void *K, const void *V, in
         append_small_kernel<Tin, BITS, NG><<<grid, 128, 0, st>>>(
             static_cast<uint8_t *>(c.pages), c.seq_len, c.status, static_cast<const Tin *>(K),
             static_cast<const Tin *>(V), A, Rv, vclip, c.n_kv_heads, NB, n_new, c.capacity, c.n_sink, c.n_recent,
-            rope, c.bucket);
+            rope, c.bucket, advance ? 1 : 0);
         return cudaGetLastError();
     }
     dim3 grid((unsigned)((n_new + kTile - 1) / kTile + 1), (unsigned)c.n_kv_heads, (unsigned)c.batch);
@@ -428,13 +431,13 @@ cudaError_t launch_append_t(const kvq_cache &c, const void *K, const void *V, in
 
 }  // namespace
 
-cudaError_t launch_append(const kvq_cache &c, const void *K, const void *V, int dtype, int n_new,
-                          const double *A, cudaStream_t st) {
+cudaError_t launch_append_adv(const kvq_cache &c, const void *K, const void *V, int dtype, int n_new,
+                              const double *A, cudaStream_t st, bool advance) {
     const bool one = groups_of(c) == 1;
 #define KVQ_APPEND_CASE(TIN, BITS)                                                              \
     if (c.bits == BITS)                                                                        \
-        return one ? launch_append_t<TIN, BITS, 1>(c, K, V, n_new, A, st)                      \
-                   : launch_append_t<TIN, BITS, kNG>(c, K, V, n_new, A, st);
+        return one ? launch_append_t<TIN, BITS, 1>(c, K, V, n_new, A, st, advance)             \
+                   : launch_append_t<TIN, BITS, kNG>(c, K, V, n_new, A, st, advance);
     if (dtype == KVQ_DTYPE_F32) {
         KVQ_APPEND_CASE(float, 2)
         KVQ_APPEND_CASE(float, 4)
@@ -444,6 +447,21 @@ cudaError_t launch_append(const kvq_cache &c, const void *K, const void *V, int 
     }
 #undef KVQ_APPEND_CASE
     return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_append(const kvq_cache &c, const void *K, const void *V, int dtype, int n_new,
+                          const double *A, cudaStream_t st) {
+    return launch_append_adv(c, K, V, dtype, n_new, A, st, true);
+}
+
+// The append of a decode step whose length the step's decode advances: at
+// most kSmallMax tokens, the small-append kernel without its length advance;
+// the step's channel choice is launched after it as its programmatic
+// dependent.
+cudaError_t launch_step_append(const kvq_cache &c, const void *K, const void *V, int dtype, int n_new,
+                               const double *A, cudaStream_t st) {
+    if (n_new < 1 || n_new > kSmallMax) return cudaErrorInvalidValue;
+    return launch_append_adv(c, K, V, dtype, n_new, A, st, false);
 }
 
 }  // namespace kvq

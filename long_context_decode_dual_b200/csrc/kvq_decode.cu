@@ -26,7 +26,9 @@ cudaError_t launch_decode_mma_step(const kvq_cache &c, int Hq, const int32_t *id
 cudaError_t launch_step_prep(const kvq_cache &c, const void *q, int dtype, int Hq, const void *k_new,
                              const void *v_new, int n_new, const double *A, const double *Ainvt,
                              const double *delta, int k, int32_t *idx, float *qsel, float *qgsum, PagePlan *plans,
-                             cudaStream_t st);
+                             bool append_here, cudaStream_t st);
+cudaError_t launch_step_append(const kvq_cache &c, const void *K, const void *V, int dtype, int n_new,
+                               const double *A, cudaStream_t st);
 int step_prep_max_new();
 
 // The tensor-core kernel covers INT2 codes with 4 query heads per KV head;
@@ -100,10 +102,12 @@ cudaError_t launch_decode(const kvq_cache &c, int Hq, const int32_t *idx, const 
 bool decode_uses_mma(const kvq_cache &c, int Hq) { return use_mma(c, Hq); }
 
 // One decode step.  The tensor-core shape with at most 4 new tokens runs as
-// one fused launch without RoPE buckets, and with buckets as two launches:
-// the preparation kernel (the channel choice of every bucket, the page plans,
-// the append) and the decode as its programmatic dependent; anything else as
-// the three calls.
+// one fused launch without RoPE buckets.  With buckets it is a chain of
+// programmatic dependent launches: the append of the new tokens (without the
+// length advance), the channel choice of every bucket with the page plans
+// (which starts while the append runs and waits for it before it exits), and
+// the decode, which waits for the choice and advances the length.  Anything
+// else runs as the three calls.
 cudaError_t launch_decode_step(const kvq_cache &c, int Hq, const void *q, const void *k_new,
                                const void *v_new, int dtype, int n_new, const double *A,
                                const double *Ainvt, const double *delta, int k, int32_t *idx, float *qsel,
@@ -119,8 +123,11 @@ cudaError_t launch_decode_step(const kvq_cache &c, int Hq, const void *q, const 
         float *part_o = static_cast<float *>(ws);
         float2 *part_ml = reinterpret_cast<float2 *>(part_o + (size_t)c.batch * Hq * S * kD);
         PagePlan *plans = reinterpret_cast<PagePlan *>(static_cast<uint8_t *>(ws) + partials_bytes(c, Hq, S));
-        cudaError_t e = launch_step_prep(c, q, dtype, Hq, k_new, v_new, n_new, A, Ainvt, delta, k, idx, qsel,
-                                         qgsum, plans, st);
+        cudaError_t e = cudaSuccess;
+        if (n_new > 0) e = launch_step_append(c, k_new, v_new, dtype, n_new, A, st);
+        if (e == cudaSuccess)
+            e = launch_step_prep(c, q, dtype, Hq, k_new, v_new, n_new, A, Ainvt, delta, k, idx, qsel, qgsum, plans,
+                                 n_new == 0, st);
         if (e == cudaSuccess)
             e = launch_decode_mma_step(c, Hq, idx, qsel, qgsum, k, part_o, part_ml, S, out, n_new, plans, st);
         return e;

@@ -100,6 +100,8 @@ struct StepAppend {
     const double *A, *Rv;         // [Hkv][128][128]; Rv may be null
     double vclip;
     int n_new, NB, capacity, n_sink, n_recent;
+    int here;                     // 1: this kernel appends; 0: the kernel before it does (this one is
+                                  // its programmatic dependent and waits for it before exiting)
 };
 
 constexpr uint32_t kPrepPolls = 1u << 20;         // bound on the polls of one wait for a row group
@@ -118,7 +120,8 @@ select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, const
               const double *__restrict__ rope, int nbk, int w, int nbb, StepAppend ap,
               PagePlan *__restrict__ plans) {
     extern __shared__ __align__(16) double sm[];
-    const SelLayout L{g, nbb, APPEND, APPEND && ap.Rv != nullptr, rope != nullptr};
+    const bool app_here = APPEND && ap.here;        // this kernel writes the new tokens
+    const SelLayout L{g, nbb, app_here, app_here && ap.Rv != nullptr, rope != nullptr};
     const int Rp = L.Rp();
     double *As = sm;
     double *Ab = sm + L.off_Ab();
@@ -153,8 +156,8 @@ select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, const
     // of 32 rows; the query and the new rows; then the length.
     __shared__ uint64_t grp_bar[4];
     const double *Ai = Ainvt + (size_t)h * kD * kD;
-    const double *Ah = APPEND ? ap.A + (size_t)h * kD * kD : nullptr;
-    const bool stage_a = APPEND && first;
+    const double *Ah = app_here ? ap.A + (size_t)h * kD * kD : nullptr;
+    const bool stage_a = app_here && first;
     const double *Rh = (stage_a && ap.Rv) ? ap.Rv + (size_t)h * kD * kD : nullptr;
     constexpr uint32_t kRowBytes = kGroup * sizeof(double);
     if (t < 4) {
@@ -175,7 +178,7 @@ select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, const
     const int aw = warp - kThreads / 64;             // new token of this warp (warps 4..7 append)
     double vnew = 0.0;                               // the value of (token aw, channel j)
     if constexpr (APPEND) {
-        if (first && ap.n_new > 0) {
+        if (stage_a && ap.n_new > 0) {
             const Tin *Kn = static_cast<const Tin *>(ap.K), *Vn = static_cast<const Tin *>(ap.V);
             const size_t in_base = unit * (size_t)ap.n_new;
             for (int e = t; e < ap.n_new * kD; e += kThreads) {
@@ -197,7 +200,7 @@ select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, const
     // overflow the capacity appends nothing)
     const int L0 = seq_len[b];
     const bool ok = !APPEND || (L0 >= 0 && L0 + ap.n_new <= ap.capacity);
-    const bool appends = APPEND && first && ok;
+    const bool appends = stage_a && ok;
     // buckets that hold a token (bucket 0 always): a prefix of the buckets
     const int len = max(APPEND && ok ? L0 + ap.n_new : L0, 0);
     const int used = rope ? max(1, (int)(((long long)len + w - 1) / w)) : 1;
@@ -522,6 +525,10 @@ select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, const
     }
     // after a give-up, no copy may land once the CTA has exited
     if (__syncthreads_or(gave_up) && t < 4) drain_bar(smem_u32(&grp_bar[t]));
+    // the step's append ran in the kernel before this one: this grid
+    // completes only after it, so the decode that waits for this grid sees
+    // the new tokens
+    if (APPEND && !ap.here) asm volatile("griddepcontrol.wait;\n" ::: "memory");
     cluster_wait_acquire();                          // no other CTA still reads this one's shared memory
 }
 
@@ -533,7 +540,8 @@ cudaError_t launch_select_t(const kvq_cache &c, const void *q, int Hq, const dou
     const int nbk = buckets_of(c);
     const double *rope = c.bucket > 0 ? c.rope : nullptr;
     const int nbb = rope ? std::min(nbk, std::max(1, kMaxGNbb / g)) : 1;     // buckets per cluster
-    const SelLayout L{g, nbb, APPEND, APPEND && ap.Rv != nullptr, rope != nullptr};
+    const bool here = APPEND && ap.here;
+    const SelLayout L{g, nbb, here, here && ap.Rv != nullptr, rope != nullptr};
     // the largest layout any call can ask for (g <= 32, g * nbb <= 32 or nbb =
     // 1; the step's preparation only for four query heads per KV head)
     size_t max_smem = 0;
@@ -545,12 +553,21 @@ cudaError_t launch_select_t(const kvq_cache &c, const void *q, int Hq, const dou
     static std::atomic<uint64_t> done{0};
     cudaError_t e = set_smem_once(select_kernel<Tin, APPEND, NG>, (int)max_smem, done);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)(kCtas * ((nbk + nbb - 1) / nbb)), (unsigned)c.n_kv_heads, (unsigned)c.batch);
-    select_kernel<Tin, APPEND, NG><<<grid, kThreads, L.bytes(), st>>>(static_cast<const Tin *>(q), Ainvt, delta, Hq,
-                                                                      c.n_kv_heads, g, k, idx, qsel, qgsum,
-                                                                      groups_of(c), c.seq_len, rope, nbk, c.bucket,
-                                                                      nbb, ap, plans);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(kCtas * ((nbk + nbb - 1) / nbb)), (unsigned)c.n_kv_heads, (unsigned)c.batch);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = L.bytes();
+    cfg.stream = st;
+    // after the step's append kernel: start while it runs (programmatic
+    // dependent launch); the kernel waits for it before it exits
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = (APPEND && !ap.here) ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, select_kernel<Tin, APPEND, NG>, static_cast<const Tin *>(q), Ainvt, delta, Hq,
+                              (int)c.n_kv_heads, g, k, idx, qsel, qgsum, groups_of(c),
+                              static_cast<const int32_t *>(c.seq_len), rope, nbk, (int)c.bucket, nbb, ap, plans);
 }
 
 }  // namespace
@@ -559,6 +576,7 @@ cudaError_t launch_select(const kvq_cache &c, const void *q, int dtype, int Hq, 
                           const double *delta, int k, int32_t *idx, float *qsel, float *qgsum, cudaStream_t st) {
     StepAppend none{};
     none.status = c.status;                          // for the bounded waits' KVQ_DEV_TIMEOUT
+    none.here = 1;
     return dtype == KVQ_DTYPE_F32
                ? launch_select_t<float, false, kNG>(c, q, Hq, Ainvt, delta, k, idx, qsel, qgsum, none, nullptr, st)
                : launch_select_t<uint16_t, false, kNG>(c, q, Hq, Ainvt, delta, k, idx, qsel, qgsum, none, nullptr,
@@ -573,9 +591,9 @@ cudaError_t launch_select(const kvq_cache &c, const void *q, int dtype, int Hq, 
 cudaError_t launch_step_prep(const kvq_cache &c, const void *q, int dtype, int Hq, const void *k_new,
                              const void *v_new, int n_new, const double *A, const double *Ainvt,
                              const double *delta, int k, int32_t *idx, float *qsel, float *qgsum, PagePlan *plans,
-                             cudaStream_t st) {
+                             bool append_here, cudaStream_t st) {
     const StepAppend ap{static_cast<uint8_t *>(c.pages), c.status, k_new, v_new, A, c.v_rot, value_clip(c), n_new,
-                        c.capacity / kT, c.capacity, c.n_sink, c.n_recent};
+                        c.capacity / kT, c.capacity, c.n_sink, c.n_recent, append_here ? 1 : 0};
     const bool one = groups_of(c) == 1;
     if (dtype == KVQ_DTYPE_F32)
         return one ? launch_select_t<float, true, 1>(c, q, Hq, Ainvt, delta, k, idx, qsel, qgsum, ap, plans, st)
