@@ -63,12 +63,12 @@ def measured_peaks():
 
 
 def decode_source_hash() -> str:
-    """Hash of the sources of the timed kernels (the step's preparation kernel
-    in kvq_select.cu, the decode kernels in kvq_decode*.cu, the internal
-    header)."""
+    """Hash of the sources of the decode kernels whose DRAM traffic profiles/
+    records (the fused step and the three-call decode in kvq_decode_mma.cu,
+    the CUDA-core decode in kvq_decode_simt.cu, the internal header)."""
     h = hashlib.sha256()
     for name in sorted(os.listdir(CSRC)):
-        if name.startswith("kvq_decode") or name == "kvq_select.cu" or name.endswith(".cuh"):
+        if name in ("kvq_decode_mma.cu", "kvq_decode_simt.cu") or name.endswith(".cuh"):
             with open(os.path.join(CSRC, name), "rb") as f:
                 h.update(name.encode())
                 h.update(f.read())
@@ -463,10 +463,10 @@ def run_ours(args):
         st.v_new.copy_(kv_pool[i % n_pool][1])
 
     # step: one kvq_decode_step call = one fused launch (with RoPE buckets
-    # two: the preparation kernel and the decode as its programmatic
-    # dependent); unfused: one-token append (with its length advance),
-    # select, decode (with its merge)
-    launches_per_step = (2 if wl.bucket else 1) if args.fused else 3
+    # three: the append, the per-bucket choice as its programmatic dependent,
+    # the decode as the choice's); unfused: one-token append (with its length
+    # advance), select, decode (with its merge)
+    launches_per_step = (3 if wl.bucket else 1) if args.fused else 3
     lengths = [wl.n_ctx] * n_copies
     for st in steps:
         st.time_decode()

@@ -317,7 +317,10 @@ int kvq_decode_attn_wait_bound(const kvq_cache *cache, int n_q_heads, const int3
  * n_new <= 4 and no buckets the step is one kernel launch: each CTA repeats
  * the channel choice of its (sequence, KV head) with the same float64
  * arithmetic, and the CTA holding the last page appends the new tokens before
- * reading it.
+ * reading it.  With buckets it is three launches, each a programmatic
+ * dependent of the one before: the append (the length not yet advanced), the
+ * channel choice of every bucket with the decode's page plans (written into
+ * `ws`), and the decode, which advances the length.
  *
  *  q       [batch][n_q_heads][128]; k_new, v_new [batch][n_kv_heads][n_new][128];
  *          all of dtype KVQ_DTYPE_F32 or _BF16
