@@ -88,26 +88,32 @@ inline int tier_ctas(const kvq_cache &c) { return c.n_sink + c.n_recent > 0 ? 2 
 constexpr float kScoreScaleLog2 = 0.12751743074460787f;
 
 // ------------------------------------------------------------ channel choice
-// How many of channels 64*half .. 64*half + 63 (channel 0 left out) come
-// before channel j in the order (energy descending, index ascending).
-// `key` holds the 128 energies' bit patterns: energies are >= 0, so the
-// patterns order like the values and integer compares decide exactly.  The
-// keys are read eight at a time, ahead of their compares.
-__device__ __forceinline__ int rank_half(const unsigned long long *key, int j, int half) {
+// How many of channels i0 .. i0 + N - 1 (channel 0 left out) come before
+// channel j in the order (energy descending, index ascending).  `key` holds
+// the 128 energies' bit patterns: energies are >= 0, so the patterns order
+// like the values and integer compares decide exactly.  The keys are read
+// eight at a time, ahead of their compares.
+template <int N>
+__device__ __forceinline__ int rank_count(const unsigned long long *key, int j, int i0) {
+    static_assert(N % 8 == 0, "keys are read eight at a time");
     const unsigned long long kj = key[j];
     int rk = 0;
 #pragma unroll
-    for (int b = 0; b < 8; b++) {
+    for (int b = 0; b < N / 8; b++) {
         unsigned long long v[8];
 #pragma unroll
-        for (int u = 0; u < 8; u++) v[u] = key[64 * half + 8 * b + u];
+        for (int u = 0; u < 8; u++) v[u] = key[i0 + 8 * b + u];
 #pragma unroll
         for (int u = 0; u < 8; u++) {
-            const int i = 64 * half + 8 * b + u;
+            const int i = i0 + 8 * b + u;
             rk += (int)((i != 0) & ((v[u] > kj) | ((v[u] == kj) & (i < j))));
         }
     }
     return rk;
+}
+// the same over channels 64*half .. 64*half + 63
+__device__ __forceinline__ int rank_half(const unsigned long long *key, int j, int half) {
+    return rank_count<64>(key, j, 64 * half);
 }
 
 // ------------------------------------------------------------ page plan

@@ -22,10 +22,11 @@
 // of four query rows side by side in one thread (one A^{-T} load for the
 // four), then their pooled energies.  After a cluster barrier every CTA reads
 // the four energy blocks of every bucket through distributed shared memory
-// and makes the same exact choice (each channel's rank by energy, counted in
-// parallel), so no CTA waits for another's decision; each writes the outputs
-// of its own channels: their list positions (prefix counts of per-bucket
-// 128-bit masks), q' in fp32 and its group's zero-point sum.  Buckets past
+// and ranks its own 32 channels by energy among all 128 (eight threads per
+// channel, exact integer compares); after a second barrier each CTA reads
+// the others' 32-bit keep masks, so all four hold the same 128-bit choice.
+// Each writes the outputs of its own channels: their list positions (prefix
+// counts of the per-bucket masks), q' in fp32 and its group's zero-point sum.  Buckets past
 // the sequence's length (other than bucket 0) are skipped.  Before a
 // tensor-core decode the kernel also writes each bucket's page plan (the
 // decode's score-MMA operands and copy list).
@@ -68,7 +69,8 @@ __device__ __forceinline__ void cluster_wait_acquire() {
 // channels qp[R][32]; energies e2own[nbb][32] and e2s[nbb][128]; the new
 // rows ks[4][128], vs[4][128] and the ranges trange[4][4][4] (CTA, token,
 // {key lo, hi, value lo, hi}); words mask[nbb][4]; bytes sel[nbb][128],
-// rank[2][nbb][128] and the new tokens' codes codes[4][64] (key, value).
+// rank[nbb][32][8] (this CTA's channels' partial ranks) and the new tokens'
+// codes codes[4][64] (key, value).
 constexpr int kPrepMaxNew = 4;
 struct SelLayout {
     int g, nbb;
@@ -136,7 +138,7 @@ select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, const
     double *trange = sm + L.off_tr();
     uint32_t *mask = reinterpret_cast<uint32_t *>(sm + L.end_doubles());   // [nbb][4]
     uint8_t *sel = reinterpret_cast<uint8_t *>(mask + nbb * 4);           // [nbb][128]
-    uint8_t *rank = sel + nbb * kD;                                       // [2][nbb][128], ranks <= 126
+    uint8_t *rank = sel + nbb * kD;                                       // [nbb][32][8], each <= 16
     uint8_t *codes = rank + 2 * nbb * kD;                                 // [token][key 32, value 32]
 
     if constexpr (APPEND) asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
@@ -380,24 +382,36 @@ select_kernel(const Tin *__restrict__ q, const double *__restrict__ Ainvt, const
         }
     }
     __syncthreads();
-    cluster_arrive_release();                        // done reading the other CTAs (waited for at exit)
-    // per bucket: the rank of channel j among 1..127 by (energy descending,
-    // index ascending), each in two halves of the comparison range; energies
-    // are >= 0, so their bit patterns order like their values.  Channel 0 and
-    // the k - 1 channels of rank below k - 1 are kept; per-bucket 128-bit
-    // keep masks by ballots.
-    for (int e = t; e < nb * 2 * kD; e += kThreads) {
-        const int bi = e / (2 * kD), part = (e / kD) & 1, jj = e % kD;
-        const int rk = rank_half(reinterpret_cast<const unsigned long long *>(e2s + bi * kD), jj, part);
-        rank[(part * nbb + bi) * kD + jj] = (uint8_t)rk;
+    // Per bucket, the rank of each of this CTA's 32 channels among 1..127 by
+    // (energy descending, index ascending), counted in eight parts of 16
+    // channels by eight threads; channel 0 and the k - 1 channels of rank
+    // below k - 1 are kept.  The CTA's 32 keep bits go to its slot of the
+    // buckets' 128-bit masks, which the CTAs then read from one another.
+    for (int e = t; e < nb * kGroup * 8; e += kThreads) {
+        const int bi = e / (kGroup * 8), l = (e / 8) % kGroup, part = e % 8;
+        rank[e] = (uint8_t)rank_count<16>(reinterpret_cast<const unsigned long long *>(e2s + bi * kD),
+                                          r * kGroup + l, 16 * part);
     }
     __syncthreads();
-    for (int e = t; e < nb * kD; e += kThreads) {      // whole warps: nb * kD is a multiple of 128
+    for (int e = t; e < nb * kGroup; e += kThreads) {  // whole warps: one warp per bucket
+        const int bi = e / kGroup, l = e % kGroup, c = r * kGroup + l;
+        int rk = 0;
+#pragma unroll
+        for (int part = 0; part < 8; part++) rk += rank[e * 8 + part];
+        const unsigned m = __ballot_sync(0xffffffffu, c == 0 || rk < k - 1);
+        if (l == 0) mask[bi * 4 + r] = m;
+    }
+    cluster.sync();                                // every CTA's keep bits are in place
+    for (int e = t; e < nb * 4; e += kThreads) {
+        // CTA rr's bits sit in its own slot rr, the only slot the others read
+        const int rr = e % 4;
+        if (rr != r) mask[e] = cluster.map_shared_rank(mask, rr)[e];
+    }
+    __syncthreads();
+    cluster_arrive_release();                        // done reading the other CTAs (waited for at exit)
+    for (int e = t; e < nb * kD; e += kThreads) {
         const int bi = e / kD, jj = e % kD;
-        const bool kept = jj == 0 || rank[bi * kD + jj] + rank[(nbb + bi) * kD + jj] < k - 1;
-        sel[bi * kD + jj] = (uint8_t)kept;
-        const unsigned m = __ballot_sync(0xffffffffu, kept);
-        if (lane == 0) mask[bi * 4 + jj / 32] = m;
+        sel[e] = (uint8_t)((mask[bi * 4 + jj / 32] >> (jj % 32)) & 1u);
     }
     __syncthreads();
     // Outputs, by warp role (a role's loop wraps onto the next threads when it
