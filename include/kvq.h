@@ -254,9 +254,11 @@ int kvq_select_channels(const kvq_cache *cache, const void *q, int dtype,
                         int32_t *idx, float *qsel, float *qgsum, int *k_out,
                         kvq_stream_t stream);
 
-/* Workspace bytes kvq_decode_attn needs for this cache on the CURRENT device
- * (it sizes the split over the context by the device's SM count).
- * 0 if the arguments are invalid. */
+/* Workspace bytes kvq_decode_attn and kvq_decode_step need for this cache on
+ * the CURRENT device (the split over the context is sized by the device's SM
+ * count): the split partials, and for INT2 with 4 query heads per KV head
+ * also the decode step's page plans, one per (sequence, KV head, RoPE
+ * bucket).  0 if the arguments are invalid. */
 size_t kvq_decode_workspace(const kvq_cache *cache, int n_q_heads, int k);
 
 /*
