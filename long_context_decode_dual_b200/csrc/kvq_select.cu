@@ -40,7 +40,11 @@
 // metadata, channel 0 and protected slots.  The sequence length is not
 // advanced here: the decode kernel that follows (launched as a programmatic
 // dependent, so that it starts streaming its first pages while this kernel
-// runs) advances it once it has waited for this grid.
+// runs) advances it once it has waited for this grid.  A decode step with RoPE
+// buckets runs the append in the small-append kernel before this one instead
+// (StepAppend::here = 0): this kernel then makes the choice for the length
+// with the new tokens, starts as that kernel's programmatic dependent, and
+// waits for it before exiting, so its own completion implies the append's.
 #include "kvq_internal.cuh"
 
 #include <cooperative_groups.h>
