@@ -69,3 +69,39 @@ def test_selection_minimises_dropped_variance():
     for _ in range(50):
         other = rng.choice(np.arange(1, 128), size=128 - k, replace=False)
         assert np.sum(q[0, other] ** 2) >= var_formula - 1e-12
+
+
+def _by_ranks(e2, k):
+    """The choice as rank counts (channel 0 always; channel j of 1..d-1 when
+    fewer than k - 1 channels of 1..d-1 come before it by (energy descending,
+    index ascending)), with energies compared as their float64 bit patterns,
+    each rank summed from eight partial counts over 16-channel ranges."""
+    d = e2.shape[0]
+    key = e2.view(np.uint64)
+    kept = [0]
+    for j in range(1, d):
+        parts = []
+        for p in range(8):
+            lo, hi = p * d // 8, (p + 1) * d // 8
+            parts.append(sum(1 for i in range(lo, hi)
+                             if i != 0 and (key[i] > key[j] or (key[i] == key[j] and i < j))))
+        if sum(parts) < k - 1:
+            kept.append(j)
+    return kept
+
+
+def test_rank_counts_equal_the_sort():
+    """Reading of the channel choice used by the tensor-core path: counting
+    each channel's rank gives the oracle's sorted choice, ties and zero
+    energies included (energies are >= 0, so bit patterns order like values)."""
+    rng = np.random.default_rng(3)
+    for trial in range(60):
+        g = int(rng.choice([1, 4, 8]))
+        if trial % 3 == 0:
+            qp = rng.integers(-2, 3, size=(g, 128)).astype(np.float64)     # many exact ties and zeros
+        else:
+            qp = rng.standard_normal((g, 128))
+        k = int(rng.choice([1, 2, 52, 77, 103, 128]))
+        idx, e2 = orc.select(qp, k)
+        assert (e2 >= 0).all()
+        assert list(idx) == _by_ranks(np.ascontiguousarray(e2, dtype=np.float64), k)
